@@ -1,0 +1,356 @@
+#!/usr/bin/env python
+"""Benchmark of the DeepSeekMoE layer forward on B200.
+
+One step = one full layer forward (router + top-K, permutation, routed
+gate/up + SwiGLU, routed down + gate scale, shared experts, final sum) over
+one batch of T synthetic tokens already resident in HBM.  The default
+workload is the DeepSeekMoE-16B-shaped prefill layer (T=16384, d=2048,
+64 routed experts of 1408, top-6, 2 shared experts of 1408).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  ``--impl reference`` times the CPU oracle
+(the plain float64 restatement of the layer) on a bounded sample of the same
+workload.  Under torchrun every rank runs an independent replica (the layer
+has no data-path exchange on one GPU; replicas only), timed on the device and
+reduced as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "MoE layer fwd tokens/s; activated-expert TFLOP/s as % of B200 bf16 peak"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 2**20
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DOMINANT = "routed_gate_up"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "routed_gate_up_16b_prefill.txt")
+KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/ffn_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", default="16b_prefill", choices=sorted(W.CONFIGS))
+    p.add_argument("--cpu-sample", type=int, default=256, help="tokens of the CPU-baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def workload_config(shape: W.LayerShape, parallelism: str) -> dict:
+    return {"workload": f"deepseekmoe_layer_{shape.name}", "T": shape.T, "d_model": shape.d,
+            "n_routed": shape.N, "d_ff": shape.I, "top_k": shape.K, "n_shared": shape.Ks,
+            "d_ff_shared": shape.Is, "gate": shape.gate, "bias": shape.bias,
+            "global_batch": shape.T, "parallelism": parallelism,
+            "l2": "no flush: every step streams its >1 GB working set (1.14 GB of expert weights) "
+                  "through the 126 MB L2"}
+
+
+def layer_flop(shape: W.LayerShape) -> float:
+    return shape.routed_flop + shape.shared_flop + shape.router_flop
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return PEAK_FALLBACK, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(shape: W.LayerShape):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    vals = {}
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        per_token = float(vals["traffic_bytes_per_token"])
+    except (KeyError, ValueError):
+        return None
+    return per_token * shape.T
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled with nvidia-smi during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            gpu = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            return None
+        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 8]
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows]
+        mx = float(rows[0][1])
+        busy = [s for s in sm if s > 0.5 * mx] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[4 + i].strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows), "power_w_max": max(float(r[2]) for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------
+
+def host_inputs(shape: W.LayerShape):
+    return W.layer_inputs(shape, with_experts=True)
+
+
+def to_device(host: dict, dev) -> dict:
+    return {k: (v.to(dev) if v is not None else None) for k, v in host.items()}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the baseline arm)
+# ---------------------------------------------------------------------------
+
+def oracle_tokens_per_s(shape: W.LayerShape, host: dict, n_tokens: int, repeats: int = 1):
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    rows = W.sample_tokens(shape, n_tokens)
+    ex = (host["w_gate"], host["w_up"], host["w_down"])
+    sh = (host["ws_gate"], host["ws_up"], host["ws_down"]) if shape.Ks else None
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        O.moe_forward(host["x"], host["router"], shape.K, ex, sh, gate_kind=shape.gate,
+                      logit_bias=host["logit_bias"], select_bias=host["select_bias"], rows=rows)
+        times.append(time.perf_counter() - t0)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return rows.size, times, threads
+
+
+def run_reference(args):
+    shape = W.CONFIGS[args.config]
+    host = host_inputs(shape)
+    # size each step's sample so that warmup + steps finish in about three minutes
+    n_cal, t_cal, threads = oracle_tokens_per_s(shape, host, 4)
+    per_token = t_cal[0] / n_cal
+    budget = 180.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(shape.T, budget / per_token)))
+    for _ in range(args.warmup):
+        oracle_tokens_per_s(shape, host, n)
+    t0 = time.perf_counter()
+    total = 0
+    for _ in range(args.steps):
+        m, _, threads = oracle_tokens_per_s(shape, host, n)
+        total += m
+    dt = time.perf_counter() - t0
+    value = total / dt
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": workload_config(shape, "cpu"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{n} seeded tokens of the T={shape.T} batch per step (routing, "
+                                       f"routed and shared experts, final sum, float64 numpy)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    from fine_grained_shared_b200 import moe as B
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    shape = W.CONFIGS[args.config]
+    host = host_inputs(shape)
+    d_in = to_device(host, dev)
+    layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks,
+                       d_ff_shared=shape.Is, max_tokens=shape.T, max_k=shape.K, gate=shape.gate,
+                       device=local)
+    shared = (d_in["ws_gate"], d_in["ws_up"], d_in["ws_down"]) if shape.Ks else None
+    layer.set_weights(d_in["router"], (d_in["w_gate"], d_in["w_up"], d_in["w_down"]), shared,
+                      logit_bias=d_in["logit_bias"], select_bias=d_in["select_bias"])
+    x = d_in["x"]
+    out = torch.empty_like(x)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(max(3, args.warmup)):
+        layer.forward(x, shape.K, out)
+    st = layer.status()
+    if st != B.MOE_OK:
+        raise B.MoEError(st, "warm-up")
+
+    # ---- device-resident timing ----
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    layer.set_timing(True)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(args.steps):
+        layer.forward(x, shape.K, out)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clk = clocks.stop()
+    ktimes = layer.kernel_times()
+    layer.set_timing(False)
+    st = layer.status()
+    if st != B.MOE_OK:
+        raise B.MoEError(st, "timed region")
+    ms_total = max_over_ranks(start.elapsed_time(end))
+    ms_step = ms_total / args.steps
+    value = world * shape.T / (ms_step * 1e-3)
+
+    # ---- end to end through the host-buffer entry point ----
+    x_h = host["x"].pin_memory()
+    out_h = torch.empty_like(x_h).pin_memory()
+    e2e_steps = max(1, min(args.steps, 100))
+    for _ in range(3):
+        layer.forward_host(x_h, shape.K, out_h)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward_host(x_h, shape.K, out_h)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    e2e_value = world * shape.T / (e2e_ms * 1e-3)
+
+    # ---- roofline of the dominant kernel (routed gate/up GEMM + SwiGLU) ----
+    peaks, peak_src = measured_peaks()
+    k_ms, k_n = ktimes[DOMINANT]
+    k_avg_ms = max_over_ranks(k_ms / max(1, k_n))
+    k_flop = 4.0 * shape.T * shape.K * shape.d * shape.I
+    achieved = k_flop / (k_avg_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops_sustained"])
+    layer_tflops = world * layer_flop(shape) / (ms_step * 1e-3) / 1e12
+    launches = sum(n for _, n in ktimes.values())
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(shape, f"replicas{world}" if world > 1 else "single"),
+        "tflops": layer_tflops,
+        "tflops_frac_of_peak": layer_tflops / (world * peak),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(shape),
+                     "kernel": "ffn_gemm_kernel<EPI_SWIGLU> (routed gate/up + SwiGLU)",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained",
+                     "flop_per_launch": k_flop, "avg_launch_ms": k_avg_ms},
+        "kernel_ms_per_step": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in ktimes.items()},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_h.numel() * 2),
+                "d2h_bytes_per_step": int(out_h.numel() * 2), "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, times, threads = oracle_tokens_per_s(shape, host, args.cpu_sample)
+        line["cpu_baseline"] = {"value": n / times[0], "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{n} seeded tokens of the T={shape.T} batch (routing, routed and "
+                                          f"shared experts, final sum; float64 numpy)"}
+    layer.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,661 @@
+// moe_api.cu -- the C ABI declared in include/fgs_moe.h: argument checks,
+// workspace, TMA descriptors and the launch sequence of one layer forward.
+//
+// Launch sequence on the caller's stream S0 (and the handle's stream S1):
+//   S1: shared experts' gate/up GEMM + SwiGLU          Hs = SwiGLU(x)
+//   S0: router_topk (logits, top-K, histogram, scan)   idx, gate, offsets
+//   S0: permute_gather                                 X_perm, slot_of, g
+//   S0: routed gate/up grouped GEMM + SwiGLU           H
+//   S0: routed down grouped GEMM + gate scale          Y = g * (H W_down^T)
+//   S0 waits S1; shared down GEMM + combine            out = x + Hs Wsd^T + sum_k Y
+// With no shared experts (or MOE_FLAG_NO_SHARED) the last step is the plain
+// combine kernel.  Nothing is copied back to the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/fgs_moe.h"
+#include "ffn_gemm.cuh"
+#include "permute.cuh"
+#include "router_topk.cuh"
+
+using namespace fgs;
+
+namespace {
+
+constexpr int kMaxRouted = 256;
+constexpr int kMaxK = 8;
+constexpr int64_t kMaxTokens = int64_t(1) << 20;
+constexpr uint64_t kTimeoutNs = 2000ull * 1000 * 1000;  // 2 s: no legitimate wait comes close
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool load_encode() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// bf16 tensor [d2][rows][cols] (d2 = 1 for a matrix), box [1][box_rows][64],
+// 128-byte swizzle, zero fill outside the tensor.
+bool encode_bf16(CUtensorMap* m, const void* base, uint64_t d2, uint64_t rows, uint64_t cols, uint32_t box_rows,
+                 int rank) {
+  cuuint64_t dims[3] = {cols, rows, d2};
+  cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct MapCache {
+  const void* ptr = nullptr;
+  int64_t rows = -1;
+  CUtensorMap map;
+};
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+struct Layout {
+  // byte offsets into the workspace
+  size_t err, done, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, gate_perm, x_perm, h, y, hs, xdev,
+      outdev, total;
+  int64_t P, Tpad, nblk;
+};
+
+Layout make_layout(const moe_config& c) {
+  Layout L{};
+  const int64_t Tm = c.max_tokens, Km = c.max_k, N = c.n_routed;
+  L.nblk = ceil_div(Tm, 128);
+  L.P = Tm * Km + N * 127;  // sum over experts of ceil(count / 128) * 128
+  L.Tpad = L.nblk * 128;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.err = take(16);
+  L.done = take(16);
+  L.idx = take(Tm * Km * 4);
+  L.gate = take(Tm * Km * 4);
+  L.slot = take(Tm * Km * 4);
+  L.src = take(Tm * Km * 4);
+  L.bc = take(L.nblk * N * 4);
+  L.counts = take(N * 4);
+  L.offsets = take((N + 1) * 4);
+  L.row_start = take((N + 1) * 4);
+  L.mtile = take((N + 1) * 4);
+  L.gate_perm = take(L.P * 4);
+  L.x_perm = take(L.P * c.d_model * 2);
+  L.h = take(L.P * c.d_ff * 2);
+  L.y = take(L.P * c.d_model * 2);
+  L.hs = take(c.n_shared > 0 ? L.Tpad * int64_t(c.n_shared) * c.d_ff_shared * 2 : 0);
+  L.xdev = take(Tm * c.d_model * 2);
+  L.outdev = take(Tm * c.d_model * 2);
+  L.total = o;
+  return L;
+}
+
+moe_status check_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->gate != MOE_GATE_SOFTMAX && c->gate != MOE_GATE_SIGMOID_BIASED) return MOE_ERR_INVALID_ARG;
+  if (c->n_routed < 1 || c->max_k < 1 || c->max_tokens < 1 || c->n_shared < 0) return MOE_ERR_SHAPE;
+  if (c->d_model < 16 || c->d_ff < 16 || (c->n_shared > 0 && c->d_ff_shared < 16)) return MOE_ERR_SHAPE;
+  if (c->max_tokens > kMaxTokens || c->d_model > 65536 || c->d_ff > 65536 || c->d_ff_shared > 65536 ||
+      c->n_shared > 64)
+    return MOE_ERR_SHAPE;
+  if (c->n_routed > kMaxRouted || c->max_k > kMaxK) return MOE_ERR_UNSUPPORTED;
+  if (c->max_k > c->n_routed) return MOE_ERR_INVALID_ARG;
+  if (c->d_model % 16 || c->d_ff % 16 || (c->n_shared > 0 && c->d_ff_shared % 16)) return MOE_ERR_ALIGNMENT;
+  const uint32_t known = MOE_FLAG_NO_RESIDUAL | MOE_FLAG_NO_SHARED | MOE_FLAG_NO_ROUTED | MOE_FLAG_DEBUG_WAIT_TIMEOUT;
+  if (c->flags & ~known) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || !na || !nb) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+class DeviceGuard {
+ public:
+  explicit DeviceGuard(int dev) {
+    cudaGetDevice(&prev_);
+    if (prev_ != dev) cudaSetDevice(dev);
+  }
+  ~DeviceGuard() { cudaSetDevice(prev_); }
+
+ private:
+  int prev_ = 0;
+};
+
+}  // namespace
+
+struct moe_ctx {
+  moe_config cfg;
+  int device = 0;
+  int num_sms = 148;
+  Layout L;
+  uint8_t* ws = nullptr;
+  cudaStream_t s1 = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_shared = nullptr;
+  cudaStream_t last_stream = nullptr;
+  int64_t last_T = 0;
+  int last_K = 0;
+  // TMA descriptors: workspace ones are fixed, the others follow the caller's pointers
+  CUtensorMap tm_xperm, tm_h, tm_hs;
+  MapCache tm_x, tm_router, tm_wg, tm_wu, tm_wd, tm_swg, tm_swu, tm_swd;
+  // per-kernel timing: event pairs recorded around each launch while enabled
+  bool timing = false;
+  std::vector<cudaEvent_t> ev_pool[MOE_KERNEL_COUNT];
+  size_t ev_used[MOE_KERNEL_COUNT] = {};
+
+  template <typename T>
+  T* at(size_t off) const {
+    return reinterpret_cast<T*>(ws + off);
+  }
+};
+
+namespace {
+
+template <int K>
+void launch_router_k(bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, const CUtensorMap& tx,
+                     const CUtensorMap& te, const RouterArgs& ra) {
+  if (sigmoid)
+    router_topk_kernel<K, true><<<grid, kRouterThreads, smem, s>>>(tx, te, ra);
+  else
+    router_topk_kernel<K, false><<<grid, kRouterThreads, smem, s>>>(tx, te, ra);
+}
+
+void launch_router(int K, bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, const CUtensorMap& tx,
+                   const CUtensorMap& te, const RouterArgs& ra) {
+  switch (K) {
+    case 1: launch_router_k<1>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 2: launch_router_k<2>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 3: launch_router_k<3>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 4: launch_router_k<4>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 5: launch_router_k<5>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 6: launch_router_k<6>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 7: launch_router_k<7>(sigmoid, grid, smem, s, tx, te, ra); break;
+    default: launch_router_k<8>(sigmoid, grid, smem, s, tx, te, ra); break;
+  }
+}
+
+template <int K>
+cudaError_t set_router_attrs_k(size_t smem) {
+  cudaError_t e = cudaFuncSetAttribute(router_topk_kernel<K, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(router_topk_kernel<K, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(smem));
+}
+
+cudaError_t set_kernel_attrs() {
+  const size_t rs = router_smem_bytes(256);
+  cudaError_t e = cudaSuccess;
+  if ((e = set_router_attrs_k<1>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<2>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<3>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<4>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<5>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<6>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<7>(rs)) != cudaSuccess) return e;
+  if ((e = set_router_attrs_k<8>(rs)) != cudaSuccess) return e;
+  const int gs = static_cast<int>(gemm_smem_bytes());
+  if ((e = cudaFuncSetAttribute(ffn_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs)))
+    return e;
+  if ((e = cudaFuncSetAttribute(ffn_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs)))
+    return e;
+  return cudaFuncSetAttribute(ffn_gemm_kernel<EPI_COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs);
+}
+
+// Re-encode a cached descriptor when the caller's pointer (or row count) changes.
+bool refresh(MapCache& c, const void* p, int64_t rows_key, uint64_t d2, uint64_t rows, uint64_t cols,
+             uint32_t box_rows, int rank) {
+  if (c.ptr == p && c.rows == rows_key) return true;
+  if (!encode_bf16(&c.map, p, d2, rows, cols, box_rows, rank)) {
+    c.ptr = nullptr;
+    return false;
+  }
+  c.ptr = p;
+  c.rows = rows_key;
+  return true;
+}
+
+void launch_gemm(int epi, int grid, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& B0,
+                 const CUtensorMap& B1, const GemmArgs& ga) {
+  const size_t smem = gemm_smem_bytes();
+  if (epi == EPI_SWIGLU)
+    ffn_gemm_kernel<EPI_SWIGLU><<<grid, kGemmThreads, smem, s>>>(A, B0, B1, ga);
+  else if (epi == EPI_SCALE)
+    ffn_gemm_kernel<EPI_SCALE><<<grid, kGemmThreads, smem, s>>>(A, B0, B1, ga);
+  else
+    ffn_gemm_kernel<EPI_COMBINE><<<grid, kGemmThreads, smem, s>>>(A, B0, B1, ga);
+}
+
+// Records a start/stop event pair around one launch when timing is enabled.
+class KernelTimer {
+ public:
+  KernelTimer(moe_ctx* h, int id, cudaStream_t s) : h_(h), id_(id), s_(s) {
+    if (!h_->timing) return;
+    auto& pool = h_->ev_pool[id_];
+    size_t& used = h_->ev_used[id_];
+    while (pool.size() < used + 2) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return;
+      pool.push_back(e);
+    }
+    stop_ = pool[used + 1];
+    cudaEventRecord(pool[used], s_);
+    used += 2;
+  }
+  ~KernelTimer() {
+    if (stop_) cudaEventRecord(stop_, s_);
+  }
+
+ private:
+  moe_ctx* h_;
+  int id_;
+  cudaStream_t s_;
+  cudaEvent_t stop_ = nullptr;
+};
+
+GemmArgs base_args(moe_ctx* h) {
+  GemmArgs g{};
+  g.err = h->at<uint32_t>(h->L.err);
+  g.timeout_ns = kTimeoutNs;
+  g.J = 1;
+  return g;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_SHAPE: return "MOE_ERR_SHAPE";
+    case MOE_ERR_ALIGNMENT: return "MOE_ERR_ALIGNMENT";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_NOMEM: return "MOE_ERR_NOMEM";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+moe_status moe_workspace_bytes(const moe_config* cfg, uint64_t* bytes) {
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  const moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  *bytes = make_layout(*cfg).total;
+  return MOE_OK;
+}
+
+moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  moe_status st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return MOE_ERR_CUDA;
+  if (prop.major != 10) return MOE_ERR_UNSUPPORTED;
+  if (!load_encode()) return MOE_ERR_CUDA;
+  DeviceGuard guard(device);
+  if (set_kernel_attrs() != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe_ctx* h = new moe_ctx();
+  h->cfg = *cfg;
+  h->device = device;
+  h->num_sms = prop.multiProcessorCount;
+  h->L = make_layout(*cfg);
+  if (cudaMalloc(&h->ws, h->L.total) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return MOE_ERR_NOMEM;
+  }
+  bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
+  ok = ok && cudaStreamCreateWithFlags(&h->s1, cudaStreamNonBlocking) == cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+  ok = ok && cudaEventCreateWithFlags(&h->ev_shared, cudaEventDisableTiming) == cudaSuccess;
+  const moe_config& c = *cfg;
+  ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, 128, 2);
+  ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, 128, 2);
+  if (c.n_shared > 0)
+    ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, 128, 2);
+  ok = ok && cudaDeviceSynchronize() == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    moe_destroy(h);
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router* router,
+                       const moe_experts* experts, const moe_shared* shared, int32_t K, void* out,
+                       void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_SHAPE;
+  if (K < 1 || K > c.max_k || K > c.n_routed) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;  // nothing to enqueue (an empty tensor may carry a null pointer)
+  if (!router || !experts) return MOE_ERR_INVALID_ARG;
+  if ((c.n_shared > 0) != (shared != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!x || !out || !router->weight || !experts->w_gate || !experts->w_up || !experts->w_down)
+    return MOE_ERR_INVALID_ARG;
+  if (shared && (!shared->w_gate || !shared->w_up || !shared->w_down)) return MOE_ERR_INVALID_ARG;
+  const bool sigmoid = c.gate == MOE_GATE_SIGMOID_BIASED;
+  if (sigmoid ? router->logit_bias != nullptr : router->select_bias != nullptr) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, out, router->weight, router->logit_bias, router->select_bias, experts->w_gate,
+                        experts->w_up, experts->w_down, shared ? shared->w_gate : nullptr,
+                        shared ? shared->w_up : nullptr, shared ? shared->w_down : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  const int64_t d = c.d_model, N = c.n_routed, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const size_t out_bytes = size_t(T) * d * 2;
+  const size_t wsz = size_t(N) * I * d * 2, swsz = size_t(Ks) * Is * d * 2;
+  if (overlaps(out, out_bytes, x, out_bytes) || overlaps(out, out_bytes, router->weight, size_t(N) * d * 2) ||
+      overlaps(out, out_bytes, experts->w_gate, wsz) || overlaps(out, out_bytes, experts->w_up, wsz) ||
+      overlaps(out, out_bytes, experts->w_down, wsz) ||
+      (shared && (overlaps(out, out_bytes, shared->w_gate, swsz) || overlaps(out, out_bytes, shared->w_up, swsz) ||
+                  overlaps(out, out_bytes, shared->w_down, swsz))))
+    return MOE_ERR_INVALID_ARG;
+
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const Layout& L = h->L;
+  const bool do_shared = Ks > 0 && !(c.flags & MOE_FLAG_NO_SHARED);
+  const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
+  const int Npad = ((int)N + 15) / 16 * 16;
+
+  // descriptors that follow the caller's pointers
+  bool ok = refresh(h->tm_x, x, T, 1, T, d, 128, 2);
+  ok = ok && refresh(h->tm_router, router->weight, 0, 1, N, d, (uint32_t)Npad, 2);
+  ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, 128, 3);
+  ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, 128, 3);
+  ok = ok && refresh(h->tm_wd, experts->w_down, 0, N, d, I, 256, 3);
+  if (shared) {
+    ok = ok && refresh(h->tm_swg, shared->w_gate, 0, 1, Ks * Is, d, 128, 3);
+    ok = ok && refresh(h->tm_swu, shared->w_up, 0, 1, Ks * Is, d, 128, 3);
+    ok = ok && refresh(h->tm_swd, shared->w_down, 0, Ks, d, Is, 256, 3);
+  }
+  if (!ok) return MOE_ERR_CUDA;
+
+  h->last_stream = s0;
+  h->last_T = T;
+  h->last_K = K;
+  const int nblk = ceil_div(T, 128);
+
+  // ---- S1: shared experts' gate/up projection (needs only x) ----
+  if (do_shared) {
+    if (cudaEventRecord(h->ev_fork, s0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamWaitEvent(h->s1, h->ev_fork, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    GemmArgs g = base_args(h);
+    g.grouped = 0;
+    g.dense_rows = (int)T;
+    g.n_tiles = ceil_div(Ks * Is, kGemmBN / 2);
+    g.num_kb = ceil_div(d, kGemmBK);
+    g.k_per_j = (int)d;
+    g.n_limit = (int)(Ks * Is);
+    g.out = h->at<__nv_bfloat16>(L.hs);
+    g.ld_out = (int)(Ks * Is);
+    const int tiles = nblk * g.n_tiles;
+    KernelTimer kt(h, MOE_KERNEL_SHARED_GATE_UP, h->s1);
+    launch_gemm(EPI_SWIGLU, tiles < h->num_sms ? tiles : h->num_sms, h->s1, h->tm_x.map, h->tm_swg.map,
+                h->tm_swu.map, g);
+    if (cudaEventRecord(h->ev_shared, h->s1) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
+  // ---- S0: router, permutation, routed experts ----
+  RouterArgs ra{};
+  ra.T = (int)T;
+  ra.N = (int)N;
+  ra.Npad = Npad;
+  ra.num_kb = ceil_div(d, kBK);
+  ra.nblk = nblk;
+  ra.tmem_cols = Npad <= 32 ? 32u : Npad <= 64 ? 64u : Npad <= 128 ? 128u : 256u;
+  ra.logit_bias = router->logit_bias;
+  ra.select_bias = router->select_bias;
+  ra.idx = h->at<int32_t>(L.idx);
+  ra.gate = h->at<float>(L.gate);
+  ra.block_counts = h->at<int32_t>(L.bc);
+  ra.counts = h->at<int32_t>(L.counts);
+  ra.offsets = h->at<int32_t>(L.offsets);
+  ra.row_start = h->at<int32_t>(L.row_start);
+  ra.mtile_start = h->at<int32_t>(L.mtile);
+  ra.done_counter = h->at<uint32_t>(L.done);
+  ra.err = h->at<uint32_t>(L.err);
+  ra.timeout_ns = kTimeoutNs;
+  {
+    KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
+    launch_router(K, sigmoid, dim3(nblk), router_smem_bytes(Npad), s0, h->tm_x.map, h->tm_router.map, ra);
+  }
+
+  PermuteArgs pa{};
+  pa.T = (int)T;
+  pa.K = K;
+  pa.N = (int)N;
+  pa.d = (int)d;
+  int split = (2 * h->num_sms + nblk - 1) / nblk;
+  pa.split = split < 1 ? 1 : split > 8 ? 8 : split;
+  pa.idx = ra.idx;
+  pa.gate = ra.gate;
+  pa.block_base = ra.block_counts;
+  pa.offsets = ra.offsets;
+  pa.row_start = ra.row_start;
+  pa.src = h->at<int32_t>(L.src);
+  pa.slot_of = h->at<int32_t>(L.slot);
+  pa.gate_perm = h->at<float>(L.gate_perm);
+  pa.x = static_cast<const __nv_bfloat16*>(x);
+  pa.x_perm = h->at<__nv_bfloat16>(L.x_perm);
+  pa.gather = do_routed ? 1 : 0;
+  {
+    KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
+    permute_gather_kernel<<<dim3(nblk, do_routed ? pa.split : 1), kPermThreads, 0, s0>>>(pa);
+  }
+
+  if (do_routed) {
+    GemmArgs g = base_args(h);
+    g.grouped = 1;
+    g.num_groups = (int)N;
+    g.mtile_start = ra.mtile_start;
+    g.row_start = ra.row_start;
+    g.n_tiles = ceil_div(I, kGemmBN / 2);
+    g.num_kb = ceil_div(d, kGemmBK);
+    g.k_per_j = (int)d;
+    g.n_limit = (int)I;
+    g.out = h->at<__nv_bfloat16>(L.h);
+    g.ld_out = (int)I;
+    g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
+    {
+      KernelTimer kt(h, MOE_KERNEL_ROUTED_GATE_UP, s0);
+      launch_gemm(EPI_SWIGLU, h->num_sms, s0, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, g);
+    }
+
+    GemmArgs g2 = base_args(h);
+    g2.grouped = 1;
+    g2.num_groups = (int)N;
+    g2.mtile_start = ra.mtile_start;
+    g2.row_start = ra.row_start;
+    g2.n_tiles = ceil_div(d, kGemmBN);
+    g2.num_kb = ceil_div(I, kGemmBK);
+    g2.k_per_j = (int)I;
+    g2.n_limit = (int)d;
+    g2.out = h->at<__nv_bfloat16>(L.y);
+    g2.ld_out = (int)d;
+    g2.row_scale = pa.gate_perm;
+    KernelTimer kt(h, MOE_KERNEL_ROUTED_DOWN, s0);
+    launch_gemm(EPI_SCALE, h->num_sms, s0, h->tm_h, h->tm_wd.map, h->tm_wd.map, g2);
+  }
+
+  // ---- the final sum ----
+  const int add_residual = (c.flags & MOE_FLAG_NO_RESIDUAL) ? 0 : 1;
+  if (do_shared) {
+    if (cudaStreamWaitEvent(s0, h->ev_shared, 0) != cudaSuccess) return MOE_ERR_CUDA;
+    GemmArgs g = base_args(h);
+    g.grouped = 0;
+    g.dense_rows = (int)T;
+    g.n_tiles = ceil_div(d, kGemmBN);
+    g.num_kb = ceil_div(Is, kGemmBK);
+    g.J = (int)Ks;
+    g.k_per_j = (int)Is;
+    g.n_limit = (int)d;
+    g.out = static_cast<__nv_bfloat16*>(out);
+    g.ld_out = (int)d;
+    g.x = static_cast<const __nv_bfloat16*>(x);
+    g.y = h->at<__nv_bfloat16>(L.y);
+    g.slot_of = pa.slot_of;
+    g.K = K;
+    g.T = (int)T;
+    g.d = (int)d;
+    g.add_residual = add_residual;
+    g.add_routed = do_routed ? 1 : 0;
+    const int tiles = nblk * g.n_tiles;
+    KernelTimer kt(h, MOE_KERNEL_SHARED_DOWN_COMBINE, s0);
+    launch_gemm(EPI_COMBINE, tiles < h->num_sms ? tiles : h->num_sms, s0, h->tm_hs, h->tm_swd.map,
+                h->tm_swd.map, g);
+  } else {
+    CombineArgs ca{};
+    ca.T = (int)T;
+    ca.K = K;
+    ca.d = (int)d;
+    ca.x = static_cast<const __nv_bfloat16*>(x);
+    ca.y = h->at<__nv_bfloat16>(L.y);
+    ca.slot_of = pa.slot_of;
+    ca.out = static_cast<__nv_bfloat16*>(out);
+    ca.add_residual = add_residual;
+    ca.add_routed = do_routed ? 1 : 0;
+    KernelTimer kt(h, MOE_KERNEL_COMBINE, s0);
+    combine_kernel<<<ceil_div(T * 32, 256), 256, 0, s0>>>(ca);
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
+                            const moe_experts* experts, const moe_shared* shared, int32_t K, void* out_host,
+                            void* stream) {
+  if (!h || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_SHAPE;
+  if (T == 0) return MOE_OK;
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const size_t bytes = size_t(T) * h->cfg.d_model * 2;
+  void* xd = h->ws + h->L.xdev;
+  void* od = h->ws + h->L.outdev;
+  if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s0) != cudaSuccess) return MOE_ERR_CUDA;
+  const moe_status st = moe_forward(h, xd, T, router, experts, shared, K, od, stream);
+  if (st != MOE_OK) return st;
+  if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s0) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(s0) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts, int32_t* offsets,
+                           int32_t* src, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t tk = size_t(h->last_T) * h->last_K;
+  const int64_t N = h->cfg.n_routed;
+  const Layout& L = h->L;
+  bool ok = true;
+  auto cp = [&](void* dst, size_t off, size_t bytes) {
+    if (dst && bytes) ok = ok && cudaMemcpyAsync(dst, h->ws + off, bytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  };
+  cp(idx, L.idx, tk * 4);
+  cp(gate, L.gate, tk * 4);
+  cp(counts, L.counts, N * 4);
+  cp(offsets, L.offsets, (N + 1) * 4);
+  cp(src, L.src, tk * 4);
+  return ok ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_status_query(moe_handle h) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (cudaStreamSynchronize(h->s1) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t err = 0;
+  if (cudaMemcpy(&err, h->ws + h->L.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (err) {
+    if (cudaMemset(h->ws + h->L.err, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_TIMEOUT;
+  }
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_set_timing(moe_handle h, int enable) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  h->timing = enable != 0;
+  return MOE_OK;
+}
+
+moe_status moe_kernel_times(moe_handle h, float* total_ms, int32_t* launches) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  moe_status st = MOE_OK;
+  for (int k = 0; k < MOE_KERNEL_COUNT; ++k) {
+    double sum = 0.0;
+    const size_t used = h->ev_used[k];
+    for (size_t i = 0; i + 1 < used; i += 2) {
+      float ms = 0.f;
+      if (cudaEventSynchronize(h->ev_pool[k][i + 1]) != cudaSuccess ||
+          cudaEventElapsedTime(&ms, h->ev_pool[k][i], h->ev_pool[k][i + 1]) != cudaSuccess) {
+        st = MOE_ERR_CUDA;
+        break;
+      }
+      sum += ms;
+    }
+    if (total_ms) total_ms[k] = static_cast<float>(sum);
+    if (launches) launches[k] = static_cast<int32_t>(used / 2);
+    h->ev_used[k] = 0;
+  }
+  return st;
+}
+
+moe_status moe_destroy(moe_handle h) {
+  if (!h) return MOE_OK;
+  {
+    DeviceGuard guard(h->device);
+    cudaDeviceSynchronize();
+    for (auto& pool : h->ev_pool)
+      for (cudaEvent_t e : pool) cudaEventDestroy(e);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_shared) cudaEventDestroy(h->ev_shared);
+    if (h->s1) cudaStreamDestroy(h->s1);
+    if (h->ws) cudaFree(h->ws);
+  }
+  delete h;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// permute.cuh -- step 3 of the layer: group the (token, slot) pairs by expert
+// and gather the token rows into expert-contiguous order; plus the plain
+// combine used when no shared-expert GEMM carries the final sum.
+//
+// The expert-parallel dispatch of the DeepSeek-V3 technical report (section
+// 3.2.1, all-to-all dispatch and combine) sends each token to the experts
+// chosen for it.  On one GPU the same step is a stable counting sort: expert
+// e's tokens land in rows [row_start[e], row_start[e] + counts[e]) in
+// ascending token order; row_start pads every expert's segment to a multiple
+// of 128 rows so that no 128-row GEMM tile straddles two experts.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fgs {
+
+constexpr int kPermThreads = 256;
+constexpr int kPermBlockTokens = 128;  // same token blocks as the router
+
+struct PermuteArgs {
+  int T, K, N, d, split;
+  const int32_t* idx;         // [T, K]
+  const float* gate;          // [T, K]
+  const int32_t* block_base;  // [nblk, N] first rank of this block's tokens within each expert
+  const int32_t* offsets;     // [N + 1] unpadded
+  const int32_t* row_start;   // [N + 1] padded
+  int32_t* src;               // [T * K] token ids, expert-contiguous (unpadded)
+  int32_t* slot_of;           // [T, K] padded row of (t, k)
+  float* gate_perm;           // [padded rows] gate of the pair in each row
+  const __nv_bfloat16* x;     // [T, d]
+  __nv_bfloat16* x_perm;      // [padded rows, d]
+  int gather;
+};
+
+// grid (nblk, split): CTA (b, s) ranks block b's pairs (cheap, repeated by
+// every s) and copies the rows of the tokens tl with tl % split == s.
+__global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(PermuteArgs a) {
+  __shared__ uint32_t masks[256 * 4];
+  __shared__ int32_t base[256], roff[256], rstart[256];
+  __shared__ int32_t dst[kPermBlockTokens * 8];
+  const int tid = threadIdx.x;
+  const int b = blockIdx.x, sp = blockIdx.y;
+  const int t0 = b * kPermBlockTokens;
+  const int ntok = min(kPermBlockTokens, a.T - t0);
+  const int K = a.K;
+
+  for (int i = tid; i < a.N * 4; i += kPermThreads) masks[i] = 0u;
+  for (int e = tid; e < a.N; e += kPermThreads) {
+    base[e] = a.block_base[static_cast<size_t>(b) * a.N + e];
+    roff[e] = a.offsets[e];
+    rstart[e] = a.row_start[e];
+  }
+  __syncthreads();
+  if (tid < ntok) {
+    for (int k = 0; k < K; ++k) {
+      const int e = a.idx[static_cast<size_t>(t0 + tid) * K + k];
+      atomicOr(&masks[e * 4 + (tid >> 5)], 1u << (tid & 31));
+    }
+  }
+  __syncthreads();
+  if (tid < ntok) {
+    const int t = t0 + tid;
+    const int w = tid >> 5;
+    const uint32_t below = (1u << (tid & 31)) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int e = a.idx[static_cast<size_t>(t) * K + k];
+      int rank = __popc(masks[e * 4 + w] & below);
+      for (int ww = 0; ww < w; ++ww) rank += __popc(masks[e * 4 + ww]);
+      const int pos = base[e] + rank;
+      const int prow = rstart[e] + pos;
+      dst[tid * K + k] = prow;
+      if (sp == 0) {
+        a.src[roff[e] + pos] = t;
+        a.slot_of[static_cast<size_t>(t) * K + k] = prow;
+        a.gate_perm[prow] = a.gate[static_cast<size_t>(t) * K + k];
+      }
+    }
+  }
+  if (!a.gather) return;
+  __syncthreads();
+  // gather: one warp per token row, read once, written K times (16-byte vectors)
+  const int warp = tid >> 5, lane = tid & 31, nwarps = kPermThreads / 32;
+  const int nvec = a.d >> 3;
+  for (int tl = sp + a.split * warp; tl < ntok; tl += a.split * nwarps) {
+    const uint4* srow = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + tl) * a.d);
+    for (int c = lane; c < nvec; c += 32 * 4) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (c + 32 * u < nvec) v[u] = __ldg(srow + c + 32 * u);
+      for (int k = 0; k < K; ++k) {
+        uint4* drow = reinterpret_cast<uint4*>(a.x_perm + static_cast<size_t>(dst[tl * K + k]) * a.d);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (c + 32 * u < nvec) drow[c + 32 * u] = v[u];
+      }
+    }
+  }
+}
+
+struct CombineArgs {
+  int T, K, d;
+  const __nv_bfloat16* x;   // [T, d]
+  const __nv_bfloat16* y;   // [padded rows, d]: g-scaled routed rows
+  const int32_t* slot_of;   // [T, K]
+  __nv_bfloat16* out;       // [T, d]
+  int add_residual, add_routed;
+};
+
+// out[t] = x[t] + sum_k y[slot_of[t, k]] (k ascending, fp32), one warp per token.
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= a.T) return;
+  const int t = warp;
+  int slots[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) slots[k] = (k < a.K && a.add_routed) ? a.slot_of[static_cast<size_t>(t) * a.K + k] : -1;
+  const int nvec = a.d >> 3;
+  for (int c = lane; c < nvec; c += 32) {
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    if (a.add_residual) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d) + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[2 * j] += bf16lo(w[j]);
+        acc[2 * j + 1] += bf16hi(w[j]);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (slots[k] >= 0) {
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(slots[k]) * a.d) + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[2 * j] += bf16lo(w[j]);
+          acc[2 * j + 1] += bf16hi(w[j]);
+        }
+      }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.d)[c] = o;
+  }
+}
+
+}  // namespace fgs

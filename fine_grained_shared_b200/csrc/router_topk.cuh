@@ -1,0 +1,295 @@
+// router_topk.cuh -- step 1 and 2 of the layer: affinity logits on the
+// tensor cores, softmax or sigmoid, top-K in registers, per-block expert
+// histogram and (in the last CTA to finish) the expert-offset scan.
+//
+// DeepSeekMoE (arXiv 2401.06066), Abstract: each token activates mK of the mN
+// fine-grained routed experts.  DeepSeek-V3 technical report, section 2
+// ("Auxiliary-Loss-Free Load Balancing"): per-expert biases steer which
+// experts are chosen; every token keeps its K experts (no dropping).
+//
+// One CTA owns 128 tokens.  Warp 0 streams x[128 tokens, 64-column k-block]
+// and e[mN (padded to 16), 64] into shared memory with TMA (128-byte
+// swizzle); warp 1 issues tcgen05.mma (M = 128, N = mN padded) accumulating
+// the logits z in TMEM; warps 2-5 (one TMEM lane = one token each) read the
+// row of logits back and keep the K best keys in registers.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fgs {
+
+constexpr int kRouterThreads = 192;
+constexpr int kRouterStages = 4;
+constexpr int kRouterBM = 128;
+constexpr int kBK = 64;  // bf16 elements per 128-byte swizzle row
+
+struct RouterArgs {
+  int T, N, Npad, num_kb, nblk;
+  uint32_t tmem_cols;
+  const float* logit_bias;   // [N] or null (softmax)
+  const float* select_bias;  // [N] or null (sigmoid)
+  int32_t* idx;              // [T, K]
+  float* gate;               // [T, K]
+  int32_t* block_counts;     // [nblk, N]; rewritten as per-block exclusive bases by the last CTA
+  int32_t* counts;           // [N]
+  int32_t* offsets;          // [N + 1] unpadded
+  int32_t* row_start;        // [N + 1] start row of each expert, segments padded to 128 rows
+  int32_t* mtile_start;      // [N + 1] prefix sum of ceil(count / 128)
+  uint32_t* done_counter;    // CTAs finished; reset to 0 by the last CTA
+  uint32_t* err;
+  uint64_t timeout_ns;
+};
+
+__host__ __device__ constexpr size_t router_smem_bytes(int Npad) {
+  return 1024 + static_cast<size_t>(kRouterStages) * (16384 + static_cast<size_t>(Npad) * 128) +
+         8 * (2 * kRouterStages + 2) + 16 + 4 * (256 + 256 + 256) + 64;
+}
+
+__device__ __forceinline__ void record_error(uint32_t* err, volatile int* abort, uint32_t site) {
+  *abort = 1;
+  atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
+}
+
+template <int K, bool SIGMOID>
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    router_topk_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
+                       RouterArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int Bbytes = a.Npad * 128;
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kRouterStages * 16384;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kRouterStages * Bbytes);
+  uint64_t* empty = full + kRouterStages;
+  uint64_t* acc_full = empty + kRouterStages;
+  uint64_t* teardown = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* is_last = reinterpret_cast<int*>(tmem_slot + 2);
+  int* hist = reinterpret_cast<int*>(tmem_slot + 4);
+  float* bias = reinterpret_cast<float*>(hist + 256);
+  int* scan_tmp = reinterpret_cast<int*>(bias + 256);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m0 = blockIdx.x * kRouterBM;
+
+  if (tid == 0) {
+    for (int s = 0; s < kRouterStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(teardown, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  for (int i = tid; i < 256; i += kRouterThreads) {
+    hist[i] = 0;
+    float b = 0.f;
+    if (i < a.N) {
+      if (SIGMOID) {
+        if (a.select_bias) b = a.select_bias[i];
+      } else {
+        if (a.logit_bias) b = a.logit_bias[i];
+      }
+    }
+    bias[i] = b;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_e);
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    for (int kb = 0; kb < a.num_kb; ++kb) {
+      if (!mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag)) {
+        record_error(a.err, abort_flag, 0);
+        break;
+      }
+      mbar_arrive_expect_tx(&full[s], 16384u + static_cast<uint32_t>(Bbytes));
+      tma_load_2d(sA + s * 16384, &tm_x, &full[s], kb * kBK, m0);
+      tma_load_2d(sB + s * Bbytes, &tm_e, &full[s], kb * kBK, 0);
+      ++issued;
+      if (++s == kRouterStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    // make sure no copy is still landing in shared memory when the CTA exits
+    for (int st = 0; st < kRouterStages; ++st) {
+      if (issued > st) {
+        const int n = (issued - 1 - st) / kRouterStages + 1;
+        mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idesc = idesc_bf16_f32(128, a.Npad);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (int kb = 0; kb < a.num_kb; ++kb) {
+      if (!mbar_wait(&full[s], ph, a.timeout_ns, abort_flag)) {
+        record_error(a.err, abort_flag, 1);
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * 16384));
+      const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * Bbytes));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        umma_bf16_ss(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+      umma_commit(&empty[s]);
+      if (++s == kRouterStages) {
+        s = 0;
+        ph ^= 1u;
+      }
+    }
+    if (ok) umma_commit(acc_full);
+    umma_commit(teardown);
+    mbar_wait(teardown, 0, a.timeout_ns, nullptr);
+  } else if (warp >= 2) {
+    // ---------------- epilogue: one token per thread ----------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int t = m0 + r;
+    bool ok = mbar_wait(acc_full, 0, a.timeout_ns, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) {
+      if (lane == 0) record_error(a.err, abort_flag, 2);
+    } else {
+      tc_fence_after_sync();
+      float tk[K], ts[K];
+      int ti[K];
+#pragma unroll
+      for (int k = 0; k < K; ++k) {
+        tk[k] = -INFINITY;
+        ts[k] = 0.f;
+        ti[k] = 0x7fffffff;
+      }
+      float mx = -INFINITY, sum = 0.f;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      for (int c0 = 0; c0 < a.Npad; c0 += 16) {
+        uint32_t rr[16];
+        tmem_ld16(tbase + c0, rr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int col = c0 + j;
+          if (col < a.N) {
+            float z = __uint_as_float(rr[j]);
+            float key, sv;
+            if (SIGMOID) {
+              sv = 1.f / (1.f + __expf(-z));
+              key = sv + bias[col];
+            } else {
+              z += bias[col];
+              if (z > mx) {
+                sum = sum * __expf(mx - z) + 1.f;
+                mx = z;
+              } else {
+                sum += __expf(z - mx);
+              }
+              key = z;  // softmax is monotone in z: rank on the logits
+              sv = 0.f;
+            }
+            // insert (key, col) into the list ordered by (key descending,
+            // index ascending); an element pushed down keeps competing by the
+            // same order, so ties always go to the lower expert index
+            float v = key, vs = sv;
+            int vi = col;
+#pragma unroll
+            for (int k = 0; k < K; ++k) {
+              const bool sw = (v > tk[k]) || (v == tk[k] && vi < ti[k]);
+              const float t0 = tk[k], t1 = ts[k];
+              const int t2 = ti[k];
+              tk[k] = sw ? v : t0;
+              ts[k] = sw ? vs : t1;
+              ti[k] = sw ? vi : t2;
+              v = sw ? t0 : v;
+              vs = sw ? t1 : vs;
+              vi = sw ? t2 : vi;
+            }
+          }
+        }
+      }
+      if (t < a.T) {
+        float g[K];
+        if (SIGMOID) {
+          float tot = 0.f;
+#pragma unroll
+          for (int k = 0; k < K; ++k) tot += ts[k];
+#pragma unroll
+          for (int k = 0; k < K; ++k) g[k] = ts[k] / tot;
+        } else {
+          const float inv = 1.f / sum;
+#pragma unroll
+          for (int k = 0; k < K; ++k) g[k] = __expf(tk[k] - mx) * inv;
+        }
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          a.idx[static_cast<size_t>(t) * K + k] = ti[k];
+          a.gate[static_cast<size_t>(t) * K + k] = g[k];
+          atomicAdd(&hist[ti[k]], 1);
+        }
+      }
+    }
+    tc_fence_before_sync();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+
+  // ---------------- per-block histogram and the last-CTA scan ----------------
+  for (int e = tid; e < a.N; e += kRouterThreads)
+    a.block_counts[static_cast<size_t>(blockIdx.x) * a.N + e] = hist[e];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) *is_last = (atomicAdd(a.done_counter, 1u) == static_cast<uint32_t>(a.nblk - 1));
+  __syncthreads();
+  if (!*is_last) return;
+  __threadfence();
+  for (int e = tid; e < a.N; e += kRouterThreads) {
+    int run = 0;
+    for (int b = 0; b < a.nblk; ++b) {
+      int32_t* p = a.block_counts + static_cast<size_t>(b) * a.N + e;
+      const int v = __ldcg(p);
+      *p = run;
+      run += v;
+    }
+    a.counts[e] = run;
+    scan_tmp[e] = run;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int o = 0, ro = 0, mo = 0;
+    for (int e = 0; e < a.N; ++e) {
+      a.offsets[e] = o;
+      a.row_start[e] = ro;
+      a.mtile_start[e] = mo;
+      const int c = scan_tmp[e];
+      const int mt = (c + 127) / 128;
+      o += c;
+      mo += mt;
+      ro += mt * 128;
+    }
+    a.offsets[a.N] = o;
+    a.row_start[a.N] = ro;
+    a.mtile_start[a.N] = mo;
+    *a.done_counter = 0u;
+  }
+}
+
+}  // namespace fgs

@@ -1,0 +1,238 @@
+"""ctypes binding of the C ABI in ``include/fgs_moe.h`` (argument marshalling only).
+
+Every step of the layer runs in ``libfgs_moe.so``; this module only turns
+torch tensors into pointers and sizes.  There is no fallback: if the library
+is missing the import of :func:`lib` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_char_p, c_int, c_int32, c_int64, c_uint32, c_uint64, c_void_p
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfgs_moe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_SHAPE = 2
+MOE_ERR_ALIGNMENT = 3
+MOE_ERR_UNSUPPORTED = 4
+MOE_ERR_NOMEM = 5
+MOE_ERR_CUDA = 6
+MOE_ERR_TIMEOUT = 7
+
+MOE_GATE_SOFTMAX = 0
+MOE_GATE_SIGMOID_BIASED = 1
+
+MOE_FLAG_NO_RESIDUAL = 0x1
+MOE_FLAG_NO_SHARED = 0x2
+MOE_FLAG_NO_ROUTED = 0x4
+MOE_FLAG_DEBUG_WAIT_TIMEOUT = 0x100
+
+KERNEL_NAMES = ("router", "permute", "shared_gate_up", "routed_gate_up", "routed_down",
+                "shared_down_combine", "combine")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("d_model", c_int32), ("n_routed", c_int32), ("d_ff", c_int32),
+                ("n_shared", c_int32), ("d_ff_shared", c_int32), ("max_tokens", c_int32),
+                ("max_k", c_int32), ("gate", c_int32), ("flags", c_uint32)]
+
+
+class moe_router(ctypes.Structure):
+    _fields_ = [("weight", c_void_p), ("logit_bias", c_void_p), ("select_bias", c_void_p)]
+
+
+class moe_experts(ctypes.Structure):
+    _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p)]
+
+
+class moe_shared(ctypes.Structure):
+    _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p)]
+
+
+moe_handle = c_void_p
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libfgs_moe.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with fine_grained_shared_b200.csrc.build.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    L.moe_workspace_bytes.argtypes = [POINTER(moe_config), POINTER(c_uint64)]
+    L.moe_create.argtypes = [POINTER(moe_config), c_int, POINTER(moe_handle)]
+    L.moe_forward.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), POINTER(moe_experts),
+                              POINTER(moe_shared), c_int32, c_void_p, c_void_p]
+    L.moe_forward_host.argtypes = L.moe_forward.argtypes
+    L.moe_get_routing.argtypes = [moe_handle, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.moe_status_query.argtypes = [moe_handle]
+    L.moe_destroy.argtypes = [moe_handle]
+    L.moe_set_timing.argtypes = [moe_handle, c_int]
+    L.moe_kernel_times.argtypes = [moe_handle, c_void_p, c_void_p]
+    L.moe_status_string.argtypes = [c_int]
+    L.moe_status_string.restype = c_char_p
+    for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_get_routing",
+                 "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times"):
+        getattr(L, name).restype = c_int
+    _lib = L
+    return L
+
+
+def status_string(s: int) -> str:
+    return lib().moe_status_string(int(s)).decode()
+
+
+# --- the C entry points under their own names ------------------------------
+
+def moe_workspace_bytes(cfg: moe_config):
+    n = c_uint64(0)
+    st = lib().moe_workspace_bytes(ctypes.byref(cfg), ctypes.byref(n))
+    return st, n.value
+
+
+def moe_create(cfg: moe_config, device: int = 0):
+    h = moe_handle()
+    st = lib().moe_create(ctypes.byref(cfg), int(device), ctypes.byref(h))
+    return st, h
+
+
+def moe_forward(h, x, T, router, experts, shared, K, out, stream):
+    return lib().moe_forward(h, x, int(T), ctypes.byref(router), ctypes.byref(experts),
+                             ctypes.byref(shared) if shared is not None else None, int(K), out, stream)
+
+
+def moe_forward_host(h, x_host, T, router, experts, shared, K, out_host, stream):
+    return lib().moe_forward_host(h, x_host, int(T), ctypes.byref(router), ctypes.byref(experts),
+                                  ctypes.byref(shared) if shared is not None else None, int(K),
+                                  out_host, stream)
+
+
+def moe_get_routing(h, idx, gate, counts, offsets, src, stream):
+    return lib().moe_get_routing(h, idx, gate, counts, offsets, src, stream)
+
+
+def moe_status_query(h):
+    return lib().moe_status_query(h)
+
+
+def moe_destroy(h):
+    return lib().moe_destroy(h)
+
+
+def moe_set_timing(h, enable):
+    return lib().moe_set_timing(h, int(bool(enable)))
+
+
+def moe_kernel_times(h):
+    total = (ctypes.c_float * len(KERNEL_NAMES))()
+    count = (c_int32 * len(KERNEL_NAMES))()
+    st = lib().moe_kernel_times(h, total, count)
+    return st, {n: (float(total[i]), int(count[i])) for i, n in enumerate(KERNEL_NAMES)}
+
+
+# --- torch convenience wrapper (pointers and sizes only) --------------------
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+class MoELayer:
+    """A handle plus the layer's weights as torch CUDA tensors.
+
+    ``router`` bf16 [mN, d]; ``logit_bias`` / ``select_bias`` float32 [mN] or
+    None; ``experts`` = (W_gate [mN,I,d], W_up [mN,I,d], W_down [mN,d,I]);
+    ``shared`` = (W_gate [Ks,Is,d], W_up [Ks,Is,d], W_down [Ks,d,Is]) or None.
+    """
+
+    def __init__(self, *, d_model, n_routed, d_ff, n_shared, d_ff_shared, max_tokens, max_k,
+                 gate="softmax", flags=0, device=0):
+        self.cfg = moe_config(d_model, n_routed, d_ff, n_shared, d_ff_shared if n_shared else 0,
+                              max_tokens, max_k,
+                              MOE_GATE_SIGMOID_BIASED if gate == "sigmoid" else MOE_GATE_SOFTMAX, flags)
+        st, self.h = moe_create(self.cfg, device)
+        if st != MOE_OK:
+            raise MoEError(st, "moe_create")
+        self.device = device
+
+    def close(self):
+        if self.h:
+            moe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_weights(self, router, experts, shared=None, logit_bias=None, select_bias=None):
+        self._keep = (router, experts, shared, logit_bias, select_bias)
+        self.router = moe_router(router.data_ptr(), _ptr(logit_bias), _ptr(select_bias))
+        self.experts = moe_experts(*(w.data_ptr() for w in experts))
+        self.shared = moe_shared(*(w.data_ptr() for w in shared)) if shared is not None else None
+
+    def forward(self, x, K, out=None, stream=None, check=True):
+        import torch
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        st = moe_forward(self.h, _ptr(x), T, self.router, self.experts, self.shared, K, _ptr(out),
+                         _stream_ptr(stream))
+        if check and st != MOE_OK:
+            raise MoEError(st, "moe_forward")
+        return out if check else (st, out)
+
+    def forward_host(self, x_host, K, out_host, stream=None):
+        st = moe_forward_host(self.h, c_void_p(x_host.data_ptr()), x_host.shape[0], self.router,
+                              self.experts, self.shared, K, c_void_p(out_host.data_ptr()),
+                              _stream_ptr(stream))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_forward_host")
+        return out_host
+
+    def routing(self, T, K, stream=None):
+        import torch
+        dev = torch.device("cuda", self.device)
+        N = self.cfg.n_routed
+        idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+        gate = torch.empty((T, K), dtype=torch.float32, device=dev)
+        counts = torch.empty(N, dtype=torch.int32, device=dev)
+        offsets = torch.empty(N + 1, dtype=torch.int32, device=dev)
+        src = torch.empty(T * K, dtype=torch.int32, device=dev)
+        st = moe_get_routing(self.h, _ptr(idx), _ptr(gate), _ptr(counts), _ptr(offsets), _ptr(src),
+                             _stream_ptr(stream))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_get_routing")
+        return idx, gate, counts, offsets, src
+
+    def status(self):
+        return moe_status_query(self.h)
+
+    def set_timing(self, enable):
+        st = moe_set_timing(self.h, enable)
+        if st != MOE_OK:
+            raise MoEError(st, "moe_set_timing")
+
+    def kernel_times(self):
+        st, t = moe_kernel_times(self.h)
+        if st != MOE_OK:
+            raise MoEError(st, "moe_kernel_times")
+        return t

@@ -1,0 +1,179 @@
+/*
+ * fgs_moe.h -- C ABI of the B200 (sm_100a) DeepSeekMoE layer forward.
+ *
+ * The layer (DeepSeekMoE, arXiv 2401.06066, Abstract; blog summary sections
+ * "Fine-Grained Expert Segmentation (Section 3.1)" and "Shared Expert
+ * Isolation (Section 3.2)"): mN fine-grained routed experts of which mK are
+ * active per token, plus K_s shared experts that every token uses.  For a
+ * token u_t (a row of x):
+ *
+ *   z_{t,i} = u_t . e_i (+ c_i)                       affinity logits
+ *   s_{t,i} = softmax_i(z_t)  or  sigmoid(z_{t,i})    affinities
+ *   Sel_t   = the mK experts with the largest s (softmax) or s + b (sigmoid),
+ *             ordered by that key descending, ties to the lower expert index
+ *   g_{t,k} = s of the k-th selected expert (softmax), or that s divided by
+ *             the sum of the selected s (sigmoid)
+ *   FFN(u)  = W_down (SiLU(W_gate u) * (W_up u))
+ *   h_t     = u_t + sum_j FFN^shared_j(u_t) + sum_k g_{t,k} FFN_{Sel_t,k}(u_t)
+ *
+ * The sigmoid variant with a per-expert selection bias b is the
+ * auxiliary-loss-free routing of the DeepSeek-V3 technical report (section 2,
+ * "Auxiliary-Loss-Free Load Balancing"); no token is ever dropped (same
+ * section).  The pages state the layer in prose; the formulas above are the
+ * standard reading of it.
+ *
+ * Conventions for every call:
+ *   - bf16 means IEEE bfloat16 stored as 2-byte little-endian values; all
+ *     matrices are row-major.
+ *   - Device pointers are borrowed for the duration of the enqueued work; the
+ *     caller owns them and must keep them alive until the stream reaches the
+ *     end of the call.  Every device pointer must be 16-byte aligned.
+ *   - Calls are asynchronous on the given stream unless stated otherwise.
+ *   - Host-detectable errors return before anything is enqueued.  Errors the
+ *     kernels detect (a bounded wait that ran out) are recorded on the device
+ *     and returned by moe_status_query().
+ *   - One handle serves one stream at a time; calls on one handle that overlap
+ *     on the GPU race on its workspace.
+ */
+#ifndef FGS_MOE_H
+#define FGS_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, K outside [1, min(max_k, mN)], bad enum, aliasing */
+  MOE_ERR_SHAPE = 2,       /* T < 0, T > max_tokens, or a size outside the supported range */
+  MOE_ERR_ALIGNMENT = 3,   /* d, I or I_s not a multiple of 16, or a pointer not 16-byte aligned */
+  MOE_ERR_UNSUPPORTED = 4, /* mN > 256, max_k > 8, or a device that is not sm_100 */
+  MOE_ERR_NOMEM = 5,       /* workspace allocation failed */
+  MOE_ERR_CUDA = 6,        /* a CUDA runtime or driver call failed */
+  MOE_ERR_TIMEOUT = 7      /* a device-side wait ran out; the kernel stopped early */
+} moe_status;
+
+typedef enum moe_gate_kind {
+  MOE_GATE_SOFTMAX = 0,        /* s = softmax over all mN experts; gates not renormalised */
+  MOE_GATE_SIGMOID_BIASED = 1  /* s = sigmoid; select on s + b; gates renormalised over Sel */
+} moe_gate_kind;
+
+/* moe_config.flags: leave terms out of h_t so each can be checked alone. */
+#define MOE_FLAG_NO_RESIDUAL 0x1u /* drop u_t */
+#define MOE_FLAG_NO_SHARED 0x2u   /* drop the shared experts */
+#define MOE_FLAG_NO_ROUTED 0x4u   /* drop the routed experts (routing still runs) */
+/* Test only: the first grouped-GEMM CTA waits on a barrier that nothing
+ * arrives on, with a 20 ms limit; the call then reports MOE_ERR_TIMEOUT. */
+#define MOE_FLAG_DEBUG_WAIT_TIMEOUT 0x100u
+
+/* Sizes fixed for the life of a handle.  Limits: 16 <= d_model, d_ff,
+ * d_ff_shared (each a multiple of 16); 1 <= n_routed <= 256;
+ * 1 <= max_k <= min(8, n_routed); 0 <= n_shared; 1 <= max_tokens <= 2^20. */
+typedef struct moe_config {
+  int32_t d_model;     /* d: hidden size */
+  int32_t n_routed;    /* mN: routed experts */
+  int32_t d_ff;        /* I: intermediate size of one routed expert */
+  int32_t n_shared;    /* K_s: shared experts (0 allowed) */
+  int32_t d_ff_shared; /* I_s: intermediate size of one shared expert */
+  int32_t max_tokens;  /* largest T passed to moe_forward */
+  int32_t max_k;       /* largest mK passed to moe_forward */
+  int32_t gate;        /* moe_gate_kind */
+  uint32_t flags;      /* MOE_FLAG_* */
+} moe_config;
+
+/* Router.  weight: bf16 [mN, d], row i is e_i.
+ * logit_bias: float32 [mN] or NULL; softmax only: c_i added to z before
+ *   the softmax (moves both selection and gate values).
+ * select_bias: float32 [mN] or NULL; sigmoid only: b_i added to s for the
+ *   selection alone (the gate values use s). */
+typedef struct moe_router {
+  const void* weight;
+  const float* logit_bias;
+  const float* select_bias;
+} moe_router;
+
+/* Routed experts, stacked: w_gate, w_up bf16 [mN, I, d]; w_down bf16 [mN, d, I]
+ * (each expert's matrices in the [out, in] layout of a linear layer). */
+typedef struct moe_experts {
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+} moe_experts;
+
+/* Shared experts, stacked: w_gate, w_up bf16 [K_s, I_s, d]; w_down bf16 [K_s, d, I_s]. */
+typedef struct moe_shared {
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down;
+} moe_shared;
+
+typedef struct moe_ctx* moe_handle;
+
+/* Device bytes the handle allocates for cfg (host only; no CUDA call). */
+moe_status moe_workspace_bytes(const moe_config* cfg, uint64_t* bytes);
+
+/* Validate cfg, allocate the workspace on `device` and create the handle's
+ * second stream.  The caller's current device is restored before returning.
+ * Returns MOE_ERR_UNSUPPORTED if the device is not sm_100. */
+moe_status moe_create(const moe_config* cfg, int device, moe_handle* out);
+
+/* Enqueue one layer forward on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream).  x: bf16 [T, d] device; out: bf16 [T, d] device, must not
+ * overlap x or any weight.  shared must be NULL iff cfg.n_shared == 0.
+ * T == 0 enqueues nothing and returns MOE_OK.  Asynchronous. */
+moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router* router,
+                       const moe_experts* experts, const moe_shared* shared, int32_t K,
+                       void* out, void* stream);
+
+/* The same forward for callers whose activations live in host memory:
+ * x_host: bf16 [T, d] host; out_host: bf16 [T, d] host (pinned memory makes
+ * the copies asynchronous to other host work).  Copies x to the device,
+ * runs moe_forward on `stream`, copies the result back and synchronizes the
+ * stream before returning.  The weights stay device pointers. */
+moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
+                            const moe_experts* experts, const moe_shared* shared, int32_t K,
+                            void* out_host, void* stream);
+
+/* Stream-ordered copies of the last forward's routing into device buffers
+ * (any may be NULL): idx int32 [T, K] and gate float32 [T, K] (Sel_t and
+ * g_t in selection order); counts int32 [mN] tokens per expert; offsets
+ * int32 [mN + 1] exclusive prefix sum of counts; src int32 [T*K] token ids
+ * grouped by expert, ascending within an expert. */
+moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts,
+                           int32_t* offsets, int32_t* src, void* stream);
+
+/* Synchronize the handle's streams and report (then clear) any error the
+ * kernels recorded: MOE_ERR_TIMEOUT if a device-side wait ran out. */
+moe_status moe_status_query(moe_handle h);
+
+/* Free the workspace and the handle (synchronizes first).  NULL is a no-op. */
+moe_status moe_destroy(moe_handle h);
+
+/* Per-kernel timing.  While enabled, moe_forward records a CUDA event pair
+ * around each kernel it launches, on the stream that kernel runs on.
+ * moe_kernel_times synchronizes those events, writes each kernel's summed
+ * duration in milliseconds (total_ms[MOE_KERNEL_COUNT]) and launch count
+ * (launches[MOE_KERNEL_COUNT]; either array may be NULL) and clears them. */
+typedef enum moe_kernel_id {
+  MOE_KERNEL_ROUTER = 0,              /* affinities, top-K, histogram, scan */
+  MOE_KERNEL_PERMUTE = 1,             /* expert-contiguous rows of x */
+  MOE_KERNEL_SHARED_GATE_UP = 2,      /* shared experts: SwiGLU(x W_gate^T, x W_up^T) */
+  MOE_KERNEL_ROUTED_GATE_UP = 3,      /* routed experts: the same, grouped by expert */
+  MOE_KERNEL_ROUTED_DOWN = 4,         /* routed experts: g * (H W_down^T) */
+  MOE_KERNEL_SHARED_DOWN_COMBINE = 5, /* shared down projection + the final sum */
+  MOE_KERNEL_COMBINE = 6,             /* the final sum when no shared GEMM carries it */
+  MOE_KERNEL_COUNT = 7
+} moe_kernel_id;
+moe_status moe_set_timing(moe_handle h, int enable);
+moe_status moe_kernel_times(moe_handle h, float* total_ms, int32_t* launches);
+
+/* A static string naming the status. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FGS_MOE_H */

@@ -1,0 +1,91 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad configurations before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from fine_grained_shared_b200 import moe as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"^\s*(?:moe_status|const char\*)\s+(moe_\w+)\s*\(", text, re.M)
+    return names
+
+
+def test_library_exports_every_declared_entry_point():
+    lib = B.lib()
+    names = _declared()
+    assert "moe_forward" in names and "moe_create" in names and len(names) >= 8
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def _cfg(**kw):
+    base = dict(d_model=256, n_routed=16, d_ff=128, n_shared=1, d_ff_shared=128, max_tokens=512, max_k=4,
+                gate=B.MOE_GATE_SOFTMAX, flags=0)
+    base.update(kw)
+    return B.moe_config(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    ({}, B.MOE_OK),
+    ({"d_model": 200}, B.MOE_ERR_ALIGNMENT),
+    ({"d_ff": 72}, B.MOE_ERR_ALIGNMENT),
+    ({"d_ff_shared": 24}, B.MOE_ERR_ALIGNMENT),
+    ({"n_routed": 257, "max_k": 4}, B.MOE_ERR_UNSUPPORTED),
+    ({"max_k": 9, "n_routed": 64}, B.MOE_ERR_UNSUPPORTED),
+    ({"max_k": 17}, B.MOE_ERR_UNSUPPORTED),
+    ({"max_k": 8, "n_routed": 4}, B.MOE_ERR_INVALID_ARG),
+    ({"max_tokens": 0}, B.MOE_ERR_SHAPE),
+    ({"max_tokens": (1 << 20) + 1}, B.MOE_ERR_SHAPE),
+    ({"n_shared": -1}, B.MOE_ERR_SHAPE),
+    ({"d_model": 0}, B.MOE_ERR_SHAPE),
+    ({"gate": 7}, B.MOE_ERR_INVALID_ARG),
+    ({"flags": 0x40}, B.MOE_ERR_INVALID_ARG),
+    ({"n_shared": 0, "d_ff_shared": 0}, B.MOE_OK),
+])
+def test_config_validation(kw, status):
+    st, nbytes = B.moe_workspace_bytes(_cfg(**kw))
+    assert st == status, B.status_string(st)
+    if status == B.MOE_OK:
+        assert nbytes > 0
+    else:
+        st2, h = B.moe_create(_cfg(**kw), 0)
+        assert st2 == status and not h.value
+
+
+def test_workspace_grows_with_the_layer():
+    _, small = B.moe_workspace_bytes(_cfg())
+    _, big = B.moe_workspace_bytes(_cfg(max_tokens=4096))
+    _, wider = B.moe_workspace_bytes(_cfg(d_model=512))
+    assert big > small and wider > small
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_create_without_a_gpu_fails_cleanly():
+    st, h = B.moe_create(_cfg(), 0)
+    assert st == B.MOE_ERR_CUDA and not h.value
+
+
+def test_null_handles():
+    lib = B.lib()
+    assert lib.moe_destroy(None) == B.MOE_OK
+    assert lib.moe_status_query(None) == B.MOE_ERR_INVALID_ARG
+    r, e = B.moe_router(), B.moe_experts()
+    assert lib.moe_forward(None, None, 1, ctypes.byref(r), ctypes.byref(e), None, 1, None, None) == \
+        B.MOE_ERR_INVALID_ARG
+    assert lib.moe_get_routing(None, None, None, None, None, None, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_status_strings():
+    for v, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (7, "MOE_ERR_TIMEOUT"), (99, "MOE_ERR_UNKNOWN")]:
+        assert B.status_string(v) == name

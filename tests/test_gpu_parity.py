@@ -1,0 +1,246 @@
+"""Parity of the sm_100a path (through the C ABI) with the CPU oracle.
+
+Small shapes are compared on every token; the five layer shapes at full size
+are compared on their whole routing and on a seeded sample of tokens (tokens
+are independent, so a sampled row of the oracle equals that row of the full
+layer).  Rules in ``tests/harness.py``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+from fine_grained_shared_b200 import moe as B
+
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+LS = W.LayerShape
+SMALL = {
+    "tiny": W.CONFIGS["tiny"],
+    "ragged": LS("ragged", T=300, d=208, N=13, I=48, K=3, Ks=2, Is=80, sigma=0.05, bias="normal", seed=11),
+    "k1": LS("k1", T=257, d=128, N=8, I=64, K=1, Ks=1, Is=64, sigma=0.05, seed=12),
+    "k_equals_n": LS("k_equals_n", T=130, d=64, N=8, I=32, K=8, Ks=1, Is=32, sigma=0.05, seed=13),
+    "no_shared": LS("no_shared", T=200, d=256, N=16, I=128, K=4, Ks=0, Is=0, seed=14),
+    "one_token": LS("one_token", T=1, d=256, N=16, I=128, K=4, Ks=1, Is=128, seed=15),
+    "sigmoid": LS("sigmoid", T=333, d=192, N=40, I=96, K=8, Ks=1, Is=64, gate="sigmoid", sigma=0.03,
+                  bias="uniform", seed=16),
+    "n256": LS("n256", T=512, d=128, N=256, I=64, K=8, Ks=3, Is=64, sigma=0.05, seed=17),
+    "wide_k_dim": LS("wide_k_dim", T=160, d=1104, N=12, I=272, K=2, Ks=1, Is=176, sigma=0.02, seed=18),
+}
+
+FLAGS_ROUTED = B.MOE_FLAG_NO_RESIDUAL | B.MOE_FLAG_NO_SHARED
+FLAGS_SHARED = B.MOE_FLAG_NO_RESIDUAL | B.MOE_FLAG_NO_ROUTED
+
+
+def _gpu_rows(out, rows):
+    return out.float().cpu().numpy()[rows].astype(np.float64)
+
+
+def _check_layer(shape, host, dev, rows, routing=None):
+    """Whole output and the routed / shared terms alone, on ``rows``."""
+    experts = H.oracle_experts(shape, host)
+    shared = H.oracle_shared(shape, host)
+    ref_routing = routing if routing is not None else H.oracle_routing(shape, host)
+    cases = [(0, "output")]
+    cases.append((FLAGS_ROUTED, "routed term"))
+    if shape.Ks:
+        cases.append((FLAGS_SHARED, "shared term"))
+    results = {}
+    for flags, what in cases:
+        layer = H.make_layer(shape, dev, flags=flags)
+        out = H.run(layer, dev["x"], shape.K)
+        if flags == 0:
+            exempt, gpu_idx = H.check_routing(shape, layer, ref_routing)
+            results["exempt"] = exempt
+        layer.close()
+        ref, _ = O.moe_forward(host["x"], host["router"], shape.K, experts, shared, gate_kind=shape.gate,
+                               logit_bias=host["logit_bias"], select_bias=host["select_bias"], flags=flags,
+                               rows=rows, routing=ref_routing)
+        results[what] = H.compare_output(_gpu_rows(out, rows), ref, f"{shape.name} {what}", term=flags != 0)
+    return results
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_shapes_every_token(name):
+    shape = SMALL[name]
+    host, dev = H.device_inputs(shape)
+    ref = H.oracle_routing(shape, host)
+    rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]   # near-tied tokens compared by routing rules only
+    _check_layer(shape, host, dev, rows, ref)
+
+
+@pytest.mark.parametrize("name,sample", [("2b", 192), ("16b_prefill", 96), ("16b_decode", 32), ("v3", 12)])
+def test_full_size_layers(name, sample):
+    shape = W.CONFIGS[name]
+    host, dev = H.device_inputs(shape)
+    ref = H.oracle_routing(shape, host)
+    rows = W.sample_tokens(shape, sample)
+    rows = rows[ref.gap[rows] >= H.GAP_EXEMPT]
+    res = _check_layer(shape, host, dev, rows, ref)
+    print(f"{name}: exempt tokens {res['exempt']}, compared rows {rows.size}, "
+          + ", ".join(f"{k}: max err {v[0]:.2e} rms err {v[2]:.2e} rms {v[1]:.2e}"
+                      for k, v in res.items() if k != "exempt"))
+
+
+def _custom_layer(shape, router=None, logit_bias=None):
+    host = W.layer_inputs(shape)
+    if router is not None:
+        host["router"] = router
+    if logit_bias is not None:
+        host["logit_bias"] = logit_bias
+    return H.device_inputs(shape, host)
+
+
+def test_exact_ties_go_to_the_lower_expert_index():
+    """Integer-valued tokens and affinity vectors: every logit is an integer
+    of magnitude <= 256, exact in float32 whatever the summation order, so
+    ties are exact on both sides and must go to the lower expert index on
+    every token (no near-tie exemption)."""
+    shape = LS("ties", T=384, d=128, N=12, I=64, K=3, Ks=1, Is=64, sigma=0.05, seed=21)
+    g = torch.Generator().manual_seed(21)
+    x = torch.randint(-2, 3, (shape.T, shape.d), generator=g).to(torch.bfloat16)
+    r = torch.randint(-1, 2, (shape.N, shape.d), generator=g).to(torch.bfloat16)
+    r[1] = r[0]
+    r[2] = r[0]          # experts 0, 1, 2 always tie
+    r[7] = r[5]
+    r[9] = r[5]          # experts 5, 7, 9 always tie
+    host = W.layer_inputs(shape)
+    host["x"], host["router"] = x, r
+    host, dev = H.device_inputs(shape, host)
+    ref = H.oracle_routing(shape, host)
+    assert (ref.gap == 0).sum() > 50            # many tokens tie at the selection boundary
+    layer = H.make_layer(shape, dev)
+    out = H.run(layer, dev["x"], shape.K)
+    idx = layer.routing(shape.T, shape.K)[0].cpu().numpy()
+    np.testing.assert_array_equal(idx, ref.idx)
+    has = lambda e: (idx == e).any(axis=1)
+    assert (~has(1) | has(0)).all() and (~has(2) | (has(0) & has(1))).all()
+    assert (~has(7) | has(5)).all() and (~has(9) | (has(5) & has(7))).all()
+    h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), routing=ref)
+    H.compare_output(_gpu_rows(out, slice(None)), h, "ties output")
+
+
+def test_zero_router_sends_every_token_to_the_first_experts():
+    shape = LS("zero_router", T=700, d=128, N=16, I=64, K=4, Ks=1, Is=64, sigma=0.05, seed=22)
+    host, dev = _custom_layer(shape, router=torch.zeros((16, 128), dtype=torch.bfloat16))
+    layer = H.make_layer(shape, dev)
+    out = H.run(layer, dev["x"], shape.K)
+    idx, gate, counts, offsets, src = (t.cpu().numpy() for t in layer.routing(shape.T, shape.K))
+    assert (idx == np.arange(4)[None, :]).all()
+    np.testing.assert_allclose(gate, 1.0 / 16, rtol=1e-6)
+    assert counts.tolist() == [700] * 4 + [0] * 12
+    ref = H.oracle_routing(shape, host)
+    h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), routing=ref)
+    H.compare_output(_gpu_rows(out, slice(None)), h, "zero router output")
+
+
+def test_one_expert_takes_every_token():
+    shape = LS("skew", T=1000, d=256, N=32, I=128, K=2, Ks=1, Is=128, sigma=0.02, bias="normal", seed=23)
+    lb = torch.zeros(32)
+    lb[5] = 4.0          # expert 5 leads every token; the others keep real score gaps
+    host, dev = _custom_layer(shape, logit_bias=lb)
+    ref = H.oracle_routing(shape, host)
+    layer = H.make_layer(shape, dev)
+    out = H.run(layer, dev["x"], shape.K)
+    H.check_routing(shape, layer, ref)
+    counts = layer.routing(shape.T, shape.K)[2].cpu().numpy()
+    assert counts[5] == 1000
+    h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), routing=ref, logit_bias=host["logit_bias"])
+    rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
+    H.compare_output(_gpu_rows(out, rows), h[rows], "skewed output")
+
+
+def test_runs_are_bitwise_deterministic():
+    shape = W.CONFIGS["tiny"].with_(T=512)
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    a = H.run(layer, dev["x"], shape.K).clone()
+    b = H.run(layer, dev["x"], shape.K).clone()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_smaller_batches_reuse_one_handle():
+    shape = SMALL["ragged"]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    full = H.run(layer, dev["x"], shape.K).float().cpu()
+    for T in (1, 77, 128, 129, 300):
+        x = dev["x"][:T].contiguous()
+        part = H.run(layer, x, shape.K).float().cpu()
+        # tokens are independent: a prefix batch gives the prefix rows (up to summation order)
+        assert torch.allclose(part, full[:T], atol=1e-2, rtol=0)
+    # K below max_k
+    out = H.run(layer, dev["x"], 2)
+    ref = O.route(host["x"], host["router"], 2, "softmax", host["logit_bias"])
+    h, _ = O.moe_forward(host["x"], host["router"], 2, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), routing=ref)
+    rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
+    H.compare_output(_gpu_rows(out, rows), h[rows], "K=2 on a K=3 handle")
+
+
+def test_host_buffer_entry_point_matches_device_entry_point():
+    shape = W.CONFIGS["tiny"]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    dev_out = H.run(layer, dev["x"], shape.K).cpu()
+    x_pinned = host["x"].pin_memory()
+    out_pinned = torch.empty_like(x_pinned).pin_memory()
+    layer.forward_host(x_pinned, shape.K, out_pinned)
+    assert torch.equal(out_pinned.view(torch.int16), dev_out.view(torch.int16))
+
+
+def test_empty_batch_is_a_no_op():
+    shape = W.CONFIGS["tiny"]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    x = torch.empty((0, shape.d), dtype=torch.bfloat16, device="cuda")
+    st, _ = layer.forward(x, shape.K, out=torch.empty_like(x), check=False)
+    assert st == B.MOE_OK
+
+
+def test_bad_arguments_are_rejected_before_launch():
+    shape = W.CONFIGS["tiny"]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    x = dev["x"]
+    out = torch.empty_like(x)
+    assert layer.forward(x, 0, out, check=False)[0] == B.MOE_ERR_INVALID_ARG
+    assert layer.forward(x, shape.K + 1, out, check=False)[0] == B.MOE_ERR_INVALID_ARG
+    big = torch.zeros((shape.T + 1, shape.d), dtype=torch.bfloat16, device="cuda")
+    assert layer.forward(big, shape.K, torch.empty_like(big), check=False)[0] == B.MOE_ERR_SHAPE
+    assert layer.forward(x, shape.K, x, check=False)[0] == B.MOE_ERR_INVALID_ARG       # out aliases x
+    buf = torch.zeros(shape.T * shape.d + 8, dtype=torch.bfloat16, device="cuda")
+    mis = buf[1:1 + shape.T * shape.d].view(shape.T, shape.d)                           # 2-byte offset
+    assert layer.forward(mis, shape.K, out, check=False)[0] == B.MOE_ERR_ALIGNMENT
+    saved = layer.shared
+    layer.shared = None
+    assert layer.forward(x, shape.K, out, check=False)[0] == B.MOE_ERR_INVALID_ARG     # Ks > 0 needs shared
+    layer.shared = saved
+    layer.router.select_bias = dev["x"].data_ptr()                                      # sigmoid-only input
+    assert layer.forward(x, shape.K, out, check=False)[0] == B.MOE_ERR_INVALID_ARG
+    layer.router.select_bias = None
+    assert layer.status() == B.MOE_OK
+    H.run(layer, x, shape.K)
+
+
+def test_device_wait_timeout_is_reported_and_the_context_stays_usable():
+    shape = W.CONFIGS["tiny"]
+    host, dev = H.device_inputs(shape)
+    bad = H.make_layer(shape, dev, flags=B.MOE_FLAG_DEBUG_WAIT_TIMEOUT)
+    bad.forward(dev["x"], shape.K)
+    assert bad.status() == B.MOE_ERR_TIMEOUT
+    assert bad.status() == B.MOE_OK          # the error word is cleared once reported
+    bad.close()
+    good = H.make_layer(shape, dev)
+    out = H.run(good, dev["x"], shape.K)
+    ref = H.oracle_routing(shape, host)
+    h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), routing=ref)
+    rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
+    H.compare_output(_gpu_rows(out, rows), h[rows], "after a timeout")
