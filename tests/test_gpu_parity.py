@@ -124,6 +124,27 @@ def test_exact_ties_go_to_the_lower_expert_index():
     H.compare_output(_gpu_rows(out, slice(None)), h, "ties output")
 
 
+def test_duplicated_expert_rows_tie_exactly():
+    """Random-valued affinity vectors with duplicated rows: the tensor cores
+    give the copies bit-identical logits, so the copies tie exactly and the
+    lower index must win on every token (no near-tie exemption)."""
+    shape = LS("ties_rand", T=2048, d=512, N=12, I=64, K=3, Ks=1, Is=64, sigma=0.05, seed=21)
+    host = W.layer_inputs(shape)
+    r = host["router"].clone()
+    r[1] = r[0]
+    r[2] = r[0]
+    r[7] = r[5]
+    r[9] = r[5]
+    host["router"] = r
+    host, dev = H.device_inputs(shape, host)
+    ref = H.oracle_routing(shape, host)
+    assert (ref.gap == 0).sum() > 200
+    layer = H.make_layer(shape, dev)
+    H.run(layer, dev["x"], shape.K)
+    idx = layer.routing(shape.T, shape.K)[0].cpu().numpy()
+    np.testing.assert_array_equal(idx, ref.idx)
+
+
 def test_zero_router_sends_every_token_to_the_first_experts():
     shape = LS("zero_router", T=700, d=128, N=16, I=64, K=4, Ks=1, Is=64, sigma=0.05, seed=22)
     host, dev = _custom_layer(shape, router=torch.zeros((16, 128), dtype=torch.bfloat16))
