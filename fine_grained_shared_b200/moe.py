@@ -81,10 +81,12 @@ def lib() -> ctypes.CDLL:
     L.moe_destroy.argtypes = [moe_handle]
     L.moe_set_timing.argtypes = [moe_handle, c_int]
     L.moe_kernel_times.argtypes = [moe_handle, c_void_p, c_void_p]
+    L.moe_route_noalloc.argtypes = [c_void_p, c_int64, c_int32, POINTER(moe_router), c_int32, c_int32, c_int32,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.moe_status_string.argtypes = [c_int]
     L.moe_status_string.restype = c_char_p
     for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_get_routing",
-                 "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times"):
+                 "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc"):
         getattr(L, name).restype = c_int
     _lib = L
     return L
@@ -129,6 +131,12 @@ def moe_status_query(h):
 
 def moe_destroy(h):
     return lib().moe_destroy(h)
+
+
+def moe_route_noalloc(x, T, d_model, router, n_routed, gate, K, idx, gate_out, counts, offsets, err, stream):
+    """Routing with the library's fixed device scratch (no allocation); see the header."""
+    return lib().moe_route_noalloc(x, int(T), int(d_model), ctypes.byref(router), int(n_routed), int(gate),
+                                   int(K), idx, gate_out, counts, offsets, err, stream)
 
 
 def moe_set_timing(h, enable):

@@ -169,6 +169,34 @@ typedef enum moe_kernel_id {
 moe_status moe_set_timing(moe_handle h, int enable);
 moe_status moe_kernel_times(moe_handle h, float* total_ms, int32_t* launches);
 
+/* Routing without any device allocation (the pages have no counterpart: this
+ * serves callers, not the method).  For callers that cannot call cudaMalloc --
+ * a serving runtime that plans all device memory before it starts, a framework
+ * whose allocator must own every allocation, or a latency-critical loop that
+ * cannot take cudaMalloc's implicit device synchronisation -- this runs the
+ * router kernel of moe_forward (affinities, top-K, per-expert histogram and
+ * offsets) with its scratch in a fixed 528 KB device array that the library
+ * holds on every GPU that loads it, until the process exits.
+ *
+ * Runs on the calling thread's current device, on `stream`.  x: bf16 [T, d]
+ * device; router as for moe_forward; gate: moe_gate_kind; outputs (device,
+ * caller-allocated): idx int32 [T, K], gate_out float32 [T, K], counts int32
+ * [mN], offsets int32 [mN + 1] -- the same values moe_get_routing returns after
+ * moe_forward.  err: optional device word that receives error bits (OR-ed) if
+ * a device-side wait runs out; NULL keeps them in the scratch array.
+ * Limits: T <= 65536 (else MOE_ERR_SHAPE: the static scratch is full),
+ * mN <= 256, K <= 8, d a multiple of 16, 16-byte aligned pointers.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * The first call on a device looks up the scratch array's device address and
+ * sets the kernels' shared-memory limits; make that first call before any
+ * stream capture.  Every call shares the one array and finds the previous
+ * call's contents there (the call clears what must start at zero itself), so
+ * calls that overlap on the GPU -- on different streams or different threads
+ * of one device -- race and must be serialised by the caller. */
+moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_model, const moe_router* router,
+                             int32_t n_routed, int32_t gate, int32_t K, int32_t* idx, float* gate_out,
+                             int32_t* counts, int32_t* offsets, uint32_t* err, void* stream);
+
 /* A static string naming the status. */
 const char* moe_status_string(moe_status s);
 
