@@ -42,7 +42,7 @@ L2_BYTES = 126 * 2**20
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT = "routed_gate_up"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "routed_gate_up_16b_prefill.txt")
-KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/ffn_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
+KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/gateup_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
 
 
 def parse_args():
@@ -319,7 +319,7 @@ def run_ours(args):
         "tflops_frac_of_peak": layer_tflops / (world * peak),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(shape),
-                     "kernel": "ffn_gemm_kernel<EPI_SWIGLU> (routed gate/up + SwiGLU)",
+                     "kernel": "gateup_gemm_kernel (routed experts: gate/up GEMM + SwiGLU)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
                      "flop_per_launch": k_flop, "avg_launch_ms": k_avg_ms},
         "kernel_ms_per_step": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in ktimes.items()},

@@ -1,0 +1,290 @@
+// gateup_gemm.cuh -- step 4 of the layer: the expert FFNs' first half,
+// H = SiLU(u W_gate^T) * (u W_up^T), as a grouped GEMM on the 5th-generation
+// tensor cores with the SwiGLU fused into the epilogue.
+//
+// FFN_i(u) = W_down,i (SiLU(W_gate,i u) * (W_up,i u)) for every routed expert
+// i (the fine-grained experts of DeepSeekMoE, arXiv 2401.06066, Abstract and
+// blog section "Fine-Grained Expert Segmentation (Section 3.1)") and for the
+// always-active shared experts (blog section "Shared Expert Isolation
+// (Section 3.2)").
+//
+// One persistent kernel, one CTA per SM, 192 threads:
+//   warp 0      TMA producer.  Per 64-column k-block it stages the A tile
+//               [128 rows, 64] (routed experts: rows of the expert-ordered
+//               copy of x; shared experts: rows of x) and B = [W_gate rows
+//               n0..n0+127 ; W_up rows n0..n0+127] in a 4-stage ring
+//               (128-byte swizzle).
+//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.mma
+//               (M = 128, N = 256: gate and up side by side, K = 16) into one
+//               of two 256-column fp32 accumulators, so the epilogue of tile
+//               i overlaps the MMAs of tile i + 1
+//   warps 2-5   epilogue; warp w reads TMEM lanes 32*(w%4) .. +31 (one H row
+//               per thread) and stores bf16 SiLU(gate) * up
+// Tiles are (group, 128-row m-tile, 128-column n-tile); for routed experts
+// the groups' m-tile starts come from the router on the device, so the host
+// never synchronises.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fgs {
+
+constexpr int kGuThreads = 192;
+constexpr int kGuStages = 4;
+constexpr int kGuBM = 128;
+constexpr int kGuBN = 256;  // MMA N: 128 gate + 128 up columns
+constexpr int kGuBK = 64;
+constexpr uint32_t kGuStageA = kGuBM * kGuBK * 2;  // 16 KB
+constexpr uint32_t kGuStageB = kGuBN * kGuBK * 2;  // 32 KB
+constexpr uint32_t kGuTmemCols = 512;
+// TMA box heights the host must encode
+constexpr uint32_t kGuBoxRowsA = kGuBM;      // tiled x (shared experts)
+constexpr uint32_t kGuBoxRowsB = kGuBN / 2;  // W_gate and W_up
+
+struct GateUpArgs {
+  int grouped;                 // 1: routed experts (groups from the router); 0: dense rows of x
+  int num_groups;              // experts (grouped)
+  const int32_t* mtile_start;  // [G + 1] prefix sum of ceil(count / 128) (grouped)
+  const int32_t* row_start;    // [G + 1] first row of each expert in X_perm and H (grouped)
+  int T;                       // tokens (dense row count)
+  int n_tiles;                 // 128-column H tiles per group
+  int num_kb;                  // 64-wide k-blocks over d
+  int n_limit;                 // valid H columns
+  __nv_bfloat16* out;          // H
+  int ld_out;
+  uint32_t* err;
+  uint64_t timeout_ns;
+  int debug_wait;              // CTA 0 waits on a barrier nothing arrives on
+};
+
+__host__ __device__ constexpr size_t gateup_smem_bytes() {
+  return 1024 + static_cast<size_t>(kGuStages) * (kGuStageA + kGuStageB) + 8 * (2 * kGuStages + 4 + 2) + 16 +
+         4 * 2 * 264;
+}
+
+__device__ __forceinline__ void gu_record_error(uint32_t* err, volatile int* abort, uint32_t site) {
+  *abort = 1;
+  atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
+}
+
+struct GuTile {
+  int g, m_tile, n_tile;
+};
+
+__device__ __forceinline__ GuTile gu_decode(int tile, const int32_t* s_mts, int G, int n_tiles) {
+  int lo = 0, hi = G;  // largest g with s_mts[g] * n_tiles <= tile
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_mts[mid] * n_tiles <= tile) lo = mid;
+    else hi = mid;
+  }
+  GuTile c;
+  c.g = lo;
+  const int local = tile - s_mts[lo] * n_tiles;
+  c.m_tile = local / n_tiles;
+  c.n_tile = local - c.m_tile * n_tiles;
+  return c;
+}
+
+// tmA: X_perm (grouped) or x (dense) with a 128-row box.
+// tmG, tmU: W_gate, W_up as [groups][rows][d] with a 128-row box.
+__global__ void __launch_bounds__(kGuThreads, 1)
+    gateup_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
+                       const __grid_constant__ CUtensorMap tmU, GateUpArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kGuStages * kGuStageA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kGuStages * kGuStageB);
+  uint64_t* empty = full + kGuStages;
+  uint64_t* acc_full = empty + kGuStages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* never = acc_empty + 2;
+  uint64_t* teardown = never + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_mts = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [264]
+  int32_t* s_rows = s_mts + 264;                                // [264]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  int G;
+  if (a.grouped) {
+    G = a.num_groups;
+    for (int i = tid; i <= G; i += kGuThreads) {
+      s_mts[i] = a.mtile_start[i];
+      s_rows[i] = a.row_start[i];
+    }
+  } else {
+    G = 1;
+    if (tid == 0) {
+      s_mts[0] = 0;
+      s_mts[1] = (a.T + kGuBM - 1) / kGuBM;
+      s_rows[0] = 0;
+      s_rows[1] = s_mts[1] * kGuBM;
+    }
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kGuStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 4 * 32);
+    }
+    mbar_init(never, 1);
+    mbar_init(teardown, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kGuTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const int total_tiles = s_mts[G] * a.n_tiles;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmG);
+    tma_prefetch_desc(&tmU);
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
+      const GuTile c = gu_decode(tile, s_mts, G, a.n_tiles);
+      const int n0 = c.n_tile * (kGuBN / 2);
+      const int row0 = s_rows[c.g] + c.m_tile * kGuBM;
+      for (int kb = 0; kb < a.num_kb; ++kb) {
+        if (!mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag)) {
+          gu_record_error(a.err, abort_flag, 3);
+          stop = true;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], kGuStageA + kGuStageB);
+        const int kc = kb * kGuBK;
+        tma_load_2d(sA + s * kGuStageA, &tmA, &full[s], kc, row0);
+        tma_load_3d(sB + s * kGuStageB, &tmG, &full[s], kc, n0, c.g);
+        tma_load_3d(sB + s * kGuStageB + kGuStageB / 2, &tmU, &full[s], kc, n0, c.g);
+        ++issued;
+        if (++s == kGuStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    for (int st = 0; st < kGuStages; ++st) {
+      if (issued > st) {
+        const int n = (issued - 1 - st) / kGuStages + 1;
+        mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------ MMA issuer --------------------------------
+    const uint32_t idesc = idesc_bf16_f32(kGuBM, kGuBN);
+    int s = 0, acc = 0;
+    uint32_t ph = 0, acc_ph = 0;
+    bool stop = false;
+    if (a.debug_wait && blockIdx.x == 0) {
+      if (!mbar_wait(never, 0, 20ull * 1000 * 1000, abort_flag)) {
+        gu_record_error(a.err, abort_flag, 4);
+        stop = true;
+      }
+    }
+    for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
+      if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, a.timeout_ns, abort_flag)) {
+        gu_record_error(a.err, abort_flag, 5);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGuBN);
+      for (int kb = 0; kb < a.num_kb; ++kb) {
+        if (!mbar_wait(&full[s], ph, a.timeout_ns, abort_flag)) {
+          gu_record_error(a.err, abort_flag, 6);
+          stop = true;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * kGuStageA));
+        const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * kGuStageB));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16_ss(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        umma_commit(&empty[s]);
+        if (++s == kGuStages) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (stop) break;
+      umma_commit(&acc_full[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_ph ^= 1u;
+      }
+    }
+    umma_commit(teardown);
+    mbar_wait(teardown, 0, a.timeout_ns, nullptr);
+  } else if (warp >= 2) {
+    // ------------------------------ epilogue ----------------------------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      const GuTile c = gu_decode(tile, s_mts, G, a.n_tiles);
+      bool ok = mbar_wait(&acc_full[acc], acc_ph, a.timeout_ns, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) gu_record_error(a.err, abort_flag, 7);
+        break;
+      }
+      tc_fence_after_sync();
+      const uint32_t tb = tmem + static_cast<uint32_t>(acc * kGuBN) + (static_cast<uint32_t>(q * 32) << 16);
+      const size_t row = static_cast<size_t>(s_rows[c.g]) + c.m_tile * kGuBM + r;
+      const int n0 = c.n_tile * (kGuBN / 2);
+      __nv_bfloat16* orow = a.out + row * a.ld_out;
+#pragma unroll 1
+      for (int cc = 0; cc < kGuBN / 2; cc += 16) {
+        uint32_t gr[16], ur[16];
+        tmem_ld16(tb + cc, gr);
+        tmem_ld16(tb + kGuBN / 2 + cc, ur);
+        tmem_ld_wait();
+        const int col = n0 + cc;
+        if (col < a.n_limit) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float g0 = __uint_as_float(gr[2 * j]), g1 = __uint_as_float(gr[2 * j + 1]);
+            const float u0 = __uint_as_float(ur[2 * j]), u1 = __uint_as_float(ur[2 * j + 1]);
+            const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+            const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+            pk[j] = pack_bf16x2(h0, h1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + col);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&acc_empty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_ph ^= 1u;
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kGuTmemCols);
+  }
+}
+
+}  // namespace fgs

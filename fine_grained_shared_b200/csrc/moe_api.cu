@@ -1,15 +1,18 @@
 // moe_api.cu -- the C ABI declared in include/fgs_moe.h: argument checks,
 // workspace, TMA descriptors and the launch sequence of one layer forward.
 //
-// Launch sequence on the caller's stream S0 (and the handle's stream S1):
-//   S1: shared experts' gate/up GEMM + SwiGLU          Hs = SwiGLU(x)
-//   S0: router_topk (logits, top-K, histogram, scan)   idx, gate, offsets
-//   S0: permute_gather                                 X_perm, slot_of, g
-//   S0: routed gate/up grouped GEMM + SwiGLU           H
-//   S0: routed down grouped GEMM + gate scale          Y = g * (H W_down^T)
-//   S0 waits S1; shared down GEMM + combine            out = x + Hs Wsd^T + sum_k Y
-// With no shared experts (or MOE_FLAG_NO_SHARED) the last step is the plain
-// combine kernel.  Nothing is copied back to the host.
+// Launch sequence, all on the caller's stream:
+//   shared experts' gate/up GEMM + SwiGLU         Hs = SwiGLU(x)
+//   shared experts' down GEMM                     Ys = Hs W_down,s^T
+//   router_topk (logits, top-K, histogram, scan)  idx, gate, offsets
+//   permute_gather                                X_perm, slot_of, g
+//   routed gate/up grouped GEMM + SwiGLU          H
+//   routed down grouped GEMM + gate scale         Y = g * (H W_down^T)
+//   combine                                       out = x + Ys + sum_k Y (k ascending)
+// Every GEMM is a persistent kernel that fills all SMs, so running the
+// shared experts on a second stream gave no overlap (measured: 2.62 ms per
+// 16B-prefill forward with two streams, 2.60 ms with one); one stream keeps
+// each kernel's timing clean.  Nothing is copied back to the host.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -21,11 +24,14 @@
 #include <vector>
 
 #include "../../include/fgs_moe.h"
-#include "ffn_gemm.cuh"
+#include "down_gemm.cuh"
+#include "gateup_gemm.cuh"
 #include "permute.cuh"
 #include "router_topk.cuh"
 
 using namespace fgs;
+
+static_assert(kGemmBM == kExpertRowAlign, "GEMM pair tiles must not straddle two experts");
 
 namespace {
 
@@ -73,7 +79,8 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 
 struct Layout {
   // byte offsets into the workspace
-  size_t err, done, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, gate_perm, x_perm, h, y, hs, xdev,
+  size_t err, done, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, mtile128, gate_perm, x_perm, h, y, hs, ys,
+      xdev,
       outdev, total;
   int64_t P, Tpad, nblk;
 };
@@ -82,8 +89,9 @@ Layout make_layout(const moe_config& c) {
   Layout L{};
   const int64_t Tm = c.max_tokens, Km = c.max_k, N = c.n_routed;
   L.nblk = ceil_div(Tm, 128);
-  L.P = Tm * Km + N * 127;  // sum over experts of ceil(count / 128) * 128
-  L.Tpad = L.nblk * 128;
+  // sum over experts of ceil(count / 256) * 256 <= T*K + 255*N
+  L.P = Tm * Km + N * (kExpertRowAlign - 1);
+  L.Tpad = int64_t(ceil_div(Tm, kGemmBM)) * kGemmBM;
   size_t o = 0;
   auto take = [&](size_t bytes) {
     size_t at = o;
@@ -101,11 +109,13 @@ Layout make_layout(const moe_config& c) {
   L.offsets = take((N + 1) * 4);
   L.row_start = take((N + 1) * 4);
   L.mtile = take((N + 1) * 4);
+  L.mtile128 = take((N + 1) * 4);
   L.gate_perm = take(L.P * 4);
   L.x_perm = take(L.P * c.d_model * 2);
   L.h = take(L.P * c.d_ff * 2);
   L.y = take(L.P * c.d_model * 2);
   L.hs = take(c.n_shared > 0 ? L.Tpad * int64_t(c.n_shared) * c.d_ff_shared * 2 : 0);
+  L.ys = take(c.n_shared > 0 ? L.Tpad * int64_t(c.d_model) * 2 : 0);
   L.xdev = take(Tm * c.d_model * 2);
   L.outdev = take(Tm * c.d_model * 2);
   L.total = o;
@@ -154,10 +164,9 @@ struct moe_ctx {
   moe_config cfg;
   int device = 0;
   int num_sms = 148;
+  int max_pairs = 74;  // co-resident CTA pairs of the GEMM kernel (clusters live within one GPC)
   Layout L;
   uint8_t* ws = nullptr;
-  cudaStream_t s1 = nullptr;
-  cudaEvent_t ev_fork = nullptr, ev_shared = nullptr;
   cudaStream_t last_stream = nullptr;
   int64_t last_T = 0;
   int last_K = 0;
@@ -220,12 +229,10 @@ cudaError_t set_kernel_attrs() {
   if ((e = set_router_attrs_k<6>(rs)) != cudaSuccess) return e;
   if ((e = set_router_attrs_k<7>(rs)) != cudaSuccess) return e;
   if ((e = set_router_attrs_k<8>(rs)) != cudaSuccess) return e;
+  const int us = static_cast<int>(gateup_smem_bytes());
+  if ((e = cudaFuncSetAttribute(gateup_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
   const int gs = static_cast<int>(gemm_smem_bytes());
-  if ((e = cudaFuncSetAttribute(ffn_gemm_kernel<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs)))
-    return e;
-  if ((e = cudaFuncSetAttribute(ffn_gemm_kernel<EPI_SCALE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs)))
-    return e;
-  return cudaFuncSetAttribute(ffn_gemm_kernel<EPI_COMBINE>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs);
+  return cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs);
 }
 
 // Re-encode a cached descriptor when the caller's pointer (or row count) changes.
@@ -241,15 +248,27 @@ bool refresh(MapCache& c, const void* p, int64_t rows_key, uint64_t d2, uint64_t
   return true;
 }
 
-void launch_gemm(int epi, int grid, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& B0,
-                 const CUtensorMap& B1, const GemmArgs& ga) {
-  const size_t smem = gemm_smem_bytes();
-  if (epi == EPI_SWIGLU)
-    ffn_gemm_kernel<EPI_SWIGLU><<<grid, kGemmThreads, smem, s>>>(A, B0, B1, ga);
-  else if (epi == EPI_SCALE)
-    ffn_gemm_kernel<EPI_SCALE><<<grid, kGemmThreads, smem, s>>>(A, B0, B1, ga);
-  else
-    ffn_gemm_kernel<EPI_COMBINE><<<grid, kGemmThreads, smem, s>>>(A, B0, B1, ga);
+// Launch `pairs` CTA pairs (clusters of 2) of the GEMM kernel.
+cudaError_t launch_down(int pairs, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& B, const GemmArgs& ga) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = gemm_smem_bytes();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, down_gemm_kernel, A, B, ga);
+}
+
+cudaError_t launch_gateup(int ctas, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& G, const CUtensorMap& U,
+                          const GateUpArgs& ga) {
+  gateup_gemm_kernel<<<ctas, kGuThreads, gateup_smem_bytes(), s>>>(A, G, U, ga);
+  return cudaGetLastError();
 }
 
 // Records a start/stop event pair around one launch when timing is enabled.
@@ -335,20 +354,37 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
   h->device = device;
   h->num_sms = prop.multiProcessorCount;
   h->L = make_layout(*cfg);
+  {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(2 * (prop.multiProcessorCount / 2));
+    lc.blockDim = dim3(kGemmThreads);
+    lc.dynamicSmemBytes = gemm_smem_bytes();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, down_gemm_kernel, &lc) != cudaSuccess || clusters < 1) {
+      cudaGetLastError();
+      delete h;
+      return MOE_ERR_CUDA;
+    }
+    h->max_pairs = clusters < prop.multiProcessorCount / 2 ? clusters : prop.multiProcessorCount / 2;
+  }
   if (cudaMalloc(&h->ws, h->L.total) != cudaSuccess) {
     cudaGetLastError();
     delete h;
     return MOE_ERR_NOMEM;
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
-  ok = ok && cudaStreamCreateWithFlags(&h->s1, cudaStreamNonBlocking) == cudaSuccess;
-  ok = ok && cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess;
-  ok = ok && cudaEventCreateWithFlags(&h->ev_shared, cudaEventDisableTiming) == cudaSuccess;
   const moe_config& c = *cfg;
-  ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, 128, 2);
-  ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, 128, 2);
+  ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);  // A of the routed down GEMM
   if (c.n_shared > 0)
-    ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, 128, 2);
+    ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kBoxRowsA, 2);
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -397,15 +433,16 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   const int Npad = ((int)N + 15) / 16 * 16;
 
   // descriptors that follow the caller's pointers
-  bool ok = refresh(h->tm_x, x, T, 1, T, d, 128, 2);
+  static_assert(kGuBoxRowsA == kRouterBM, "x serves as A of the router and of the shared gate/up GEMM");
+  bool ok = refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2);
   ok = ok && refresh(h->tm_router, router->weight, 0, 1, N, d, (uint32_t)Npad, 2);
-  ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, 128, 3);
-  ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, 128, 3);
-  ok = ok && refresh(h->tm_wd, experts->w_down, 0, N, d, I, 256, 3);
+  ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, kGuBoxRowsB, 3);
+  ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, kGuBoxRowsB, 3);
+  ok = ok && refresh(h->tm_wd, experts->w_down, 0, N, d, I, kBoxRowsB, 3);
   if (shared) {
-    ok = ok && refresh(h->tm_swg, shared->w_gate, 0, 1, Ks * Is, d, 128, 3);
-    ok = ok && refresh(h->tm_swu, shared->w_up, 0, 1, Ks * Is, d, 128, 3);
-    ok = ok && refresh(h->tm_swd, shared->w_down, 0, Ks, d, Is, 256, 3);
+    ok = ok && refresh(h->tm_swg, shared->w_gate, 0, 1, Ks * Is, d, kGuBoxRowsB, 3);
+    ok = ok && refresh(h->tm_swu, shared->w_up, 0, 1, Ks * Is, d, kGuBoxRowsB, 3);
+    ok = ok && refresh(h->tm_swd, shared->w_down, 0, Ks, d, Is, kBoxRowsB, 3);
   }
   if (!ok) return MOE_ERR_CUDA;
 
@@ -414,27 +451,45 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   h->last_K = K;
   const int nblk = ceil_div(T, 128);
 
-  // ---- S1: shared experts' gate/up projection (needs only x) ----
+  // ---- shared experts (need only x) ----
   if (do_shared) {
-    if (cudaEventRecord(h->ev_fork, s0) != cudaSuccess) return MOE_ERR_CUDA;
-    if (cudaStreamWaitEvent(h->s1, h->ev_fork, 0) != cudaSuccess) return MOE_ERR_CUDA;
-    GemmArgs g = base_args(h);
+    GateUpArgs g{};
     g.grouped = 0;
-    g.dense_rows = (int)T;
-    g.n_tiles = ceil_div(Ks * Is, kGemmBN / 2);
-    g.num_kb = ceil_div(d, kGemmBK);
-    g.k_per_j = (int)d;
+    g.T = (int)T;
+    g.n_tiles = ceil_div(Ks * Is, kGuBN / 2);
+    g.num_kb = ceil_div(d, kGuBK);
     g.n_limit = (int)(Ks * Is);
     g.out = h->at<__nv_bfloat16>(L.hs);
     g.ld_out = (int)(Ks * Is);
-    const int tiles = nblk * g.n_tiles;
-    KernelTimer kt(h, MOE_KERNEL_SHARED_GATE_UP, h->s1);
-    launch_gemm(EPI_SWIGLU, tiles < h->num_sms ? tiles : h->num_sms, h->s1, h->tm_x.map, h->tm_swg.map,
-                h->tm_swu.map, g);
-    if (cudaEventRecord(h->ev_shared, h->s1) != cudaSuccess) return MOE_ERR_CUDA;
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
+    const int tiles = ceil_div(T, kGuBM) * g.n_tiles;
+    {
+      KernelTimer kt(h, MOE_KERNEL_SHARED_GATE_UP, s0);
+      if (launch_gateup(tiles < h->num_sms ? tiles : h->num_sms, s0, h->tm_x.map, h->tm_swg.map,
+                        h->tm_swu.map, g) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    GemmArgs g2 = base_args(h);
+    g2.grouped = 0;
+    g2.dense_rows = (int)T;
+    g2.n_tiles = ceil_div(d, kGemmBN);
+    g2.num_kb = ceil_div(Is, kGemmBK);
+    g2.J = (int)Ks;
+    g2.k_per_j = (int)Is;
+    g2.n_limit = (int)d;
+    g2.out = h->at<__nv_bfloat16>(L.ys);
+    g2.ld_out = (int)d;
+    const int tiles2 = ceil_div(T, kGemmBM) * g2.n_tiles;
+    {
+      KernelTimer kt(h, MOE_KERNEL_SHARED_DOWN, s0);
+      if (launch_down(tiles2 < h->max_pairs ? tiles2 : h->max_pairs, s0, h->tm_hs, h->tm_swd.map, g2) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
   }
 
-  // ---- S0: router, permutation, routed experts ----
+  // ---- router, permutation, routed experts ----
   RouterArgs ra{};
   ra.T = (int)T;
   ra.N = (int)N;
@@ -451,6 +506,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   ra.offsets = h->at<int32_t>(L.offsets);
   ra.row_start = h->at<int32_t>(L.row_start);
   ra.mtile_start = h->at<int32_t>(L.mtile);
+  ra.mtile128_start = h->at<int32_t>(L.mtile128);
   ra.done_counter = h->at<uint32_t>(L.done);
   ra.err = h->at<uint32_t>(L.err);
   ra.timeout_ns = kTimeoutNs;
@@ -464,7 +520,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   pa.K = K;
   pa.N = (int)N;
   pa.d = (int)d;
-  int split = (2 * h->num_sms + nblk - 1) / nblk;
+  const int split = (2 * h->num_sms + nblk - 1) / nblk;
   pa.split = split < 1 ? 1 : split > 8 ? 8 : split;
   pa.idx = ra.idx;
   pa.gate = ra.gate;
@@ -483,21 +539,24 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   }
 
   if (do_routed) {
-    GemmArgs g = base_args(h);
+    GateUpArgs g{};
     g.grouped = 1;
     g.num_groups = (int)N;
-    g.mtile_start = ra.mtile_start;
+    g.mtile_start = ra.mtile128_start;
     g.row_start = ra.row_start;
-    g.n_tiles = ceil_div(I, kGemmBN / 2);
-    g.num_kb = ceil_div(d, kGemmBK);
-    g.k_per_j = (int)d;
+    g.T = (int)T;
+    g.n_tiles = ceil_div(I, kGuBN / 2);
+    g.num_kb = ceil_div(d, kGuBK);
     g.n_limit = (int)I;
     g.out = h->at<__nv_bfloat16>(L.h);
     g.ld_out = (int)I;
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
     g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
     {
       KernelTimer kt(h, MOE_KERNEL_ROUTED_GATE_UP, s0);
-      launch_gemm(EPI_SWIGLU, h->num_sms, s0, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, g);
+      if (launch_gateup(h->num_sms, s0, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, g) != cudaSuccess)
+        return MOE_ERR_CUDA;
     }
 
     GemmArgs g2 = base_args(h);
@@ -513,46 +572,22 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     g2.ld_out = (int)d;
     g2.row_scale = pa.gate_perm;
     KernelTimer kt(h, MOE_KERNEL_ROUTED_DOWN, s0);
-    launch_gemm(EPI_SCALE, h->num_sms, s0, h->tm_h, h->tm_wd.map, h->tm_wd.map, g2);
+    if (launch_down(h->max_pairs, s0, h->tm_h, h->tm_wd.map, g2) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // ---- the final sum ----
-  const int add_residual = (c.flags & MOE_FLAG_NO_RESIDUAL) ? 0 : 1;
-  if (do_shared) {
-    if (cudaStreamWaitEvent(s0, h->ev_shared, 0) != cudaSuccess) return MOE_ERR_CUDA;
-    GemmArgs g = base_args(h);
-    g.grouped = 0;
-    g.dense_rows = (int)T;
-    g.n_tiles = ceil_div(d, kGemmBN);
-    g.num_kb = ceil_div(Is, kGemmBK);
-    g.J = (int)Ks;
-    g.k_per_j = (int)Is;
-    g.n_limit = (int)d;
-    g.out = static_cast<__nv_bfloat16*>(out);
-    g.ld_out = (int)d;
-    g.x = static_cast<const __nv_bfloat16*>(x);
-    g.y = h->at<__nv_bfloat16>(L.y);
-    g.slot_of = pa.slot_of;
-    g.K = K;
-    g.T = (int)T;
-    g.d = (int)d;
-    g.add_residual = add_residual;
-    g.add_routed = do_routed ? 1 : 0;
-    const int tiles = nblk * g.n_tiles;
-    KernelTimer kt(h, MOE_KERNEL_SHARED_DOWN_COMBINE, s0);
-    launch_gemm(EPI_COMBINE, tiles < h->num_sms ? tiles : h->num_sms, s0, h->tm_hs, h->tm_swd.map,
-                h->tm_swd.map, g);
-  } else {
-    CombineArgs ca{};
-    ca.T = (int)T;
-    ca.K = K;
-    ca.d = (int)d;
-    ca.x = static_cast<const __nv_bfloat16*>(x);
-    ca.y = h->at<__nv_bfloat16>(L.y);
-    ca.slot_of = pa.slot_of;
-    ca.out = static_cast<__nv_bfloat16*>(out);
-    ca.add_residual = add_residual;
-    ca.add_routed = do_routed ? 1 : 0;
+  CombineArgs ca{};
+  ca.T = (int)T;
+  ca.K = K;
+  ca.d = (int)d;
+  ca.x = static_cast<const __nv_bfloat16*>(x);
+  ca.ys = do_shared ? h->at<__nv_bfloat16>(L.ys) : nullptr;
+  ca.y = h->at<__nv_bfloat16>(L.y);
+  ca.slot_of = pa.slot_of;
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.add_residual = (c.flags & MOE_FLAG_NO_RESIDUAL) ? 0 : 1;
+  ca.add_routed = do_routed ? 1 : 0;
+  {
     KernelTimer kt(h, MOE_KERNEL_COMBINE, s0);
     combine_kernel<<<ceil_div(T * 32, 256), 256, 0, s0>>>(ca);
   }
@@ -601,7 +636,6 @@ moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* cou
 moe_status moe_status_query(moe_handle h) {
   if (!h) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
-  if (cudaStreamSynchronize(h->s1) != cudaSuccess) return MOE_ERR_CUDA;
   if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return MOE_ERR_CUDA;
   uint32_t err = 0;
   if (cudaMemcpy(&err, h->ws + h->L.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
@@ -649,9 +683,6 @@ moe_status moe_destroy(moe_handle h) {
     cudaDeviceSynchronize();
     for (auto& pool : h->ev_pool)
       for (cudaEvent_t e : pool) cudaEventDestroy(e);
-    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
-    if (h->ev_shared) cudaEventDestroy(h->ev_shared);
-    if (h->s1) cudaStreamDestroy(h->s1);
     if (h->ws) cudaFree(h->ws);
   }
   delete h;

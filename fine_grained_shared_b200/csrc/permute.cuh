@@ -7,7 +7,7 @@
 // chosen for it.  On one GPU the same step is a stable counting sort: expert
 // e's tokens land in rows [row_start[e], row_start[e] + counts[e]) in
 // ascending token order; row_start pads every expert's segment to a multiple
-// of 128 rows so that no 128-row GEMM tile straddles two experts.
+// of 256 rows so that no GEMM tile straddles two experts.
 #pragma once
 
 #include "sm100.cuh"
@@ -101,13 +101,17 @@ __global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(PermuteArg
 struct CombineArgs {
   int T, K, d;
   const __nv_bfloat16* x;   // [T, d]
+  const __nv_bfloat16* ys;  // [T, d] the shared experts' output, or nullptr
   const __nv_bfloat16* y;   // [padded rows, d]: g-scaled routed rows
   const int32_t* slot_of;   // [T, K]
   __nv_bfloat16* out;       // [T, d]
   int add_residual, add_routed;
 };
 
-// out[t] = x[t] + sum_k y[slot_of[t, k]] (k ascending, fp32), one warp per token.
+// Step 5, the layer's output: out[t] = x[t] + ys[t] + sum_k y[slot_of[t, k]]
+// with the routed rows in ascending k (a fixed order, so the result is
+// deterministic), summed in fp32 and rounded once to bf16.  One warp per
+// token streams whole rows (512 contiguous bytes per warp load).
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -123,6 +127,15 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
     if (a.add_residual) {
       const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d) + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[2 * j] += bf16lo(w[j]);
+        acc[2 * j + 1] += bf16hi(w[j]);
+      }
+    }
+    if (a.ys) {
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ys + static_cast<size_t>(t) * a.d) + c);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {

@@ -135,7 +135,8 @@ extern "C" moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_mode
     return MOE_ERR_CUDA;
 
   // scratch layout: [0] CTA completion counter, [4] error word,
-  // [256, +1028) row starts, [1536, +1028) m-tile starts, [4096, ...) block histograms
+  // [256, +1028) row starts, [1536, +1028) and [2816, +1028) m-tile starts,
+  // [4096, ...) block histograms
   uint32_t* done = reinterpret_cast<uint32_t*>(scratch);
   fgs::RouterArgs ra{};
   ra.T = static_cast<int>(T);
@@ -153,6 +154,7 @@ extern "C" moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_mode
   ra.offsets = offsets;
   ra.row_start = reinterpret_cast<int32_t*>(scratch + 256);
   ra.mtile_start = reinterpret_cast<int32_t*>(scratch + 1536);
+  ra.mtile128_start = reinterpret_cast<int32_t*>(scratch + 2816);
   ra.done_counter = done;
   ra.err = err ? err : reinterpret_cast<uint32_t*>(scratch + 4);
   ra.timeout_ns = kTimeoutNs;

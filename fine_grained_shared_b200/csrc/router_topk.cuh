@@ -22,6 +22,9 @@ constexpr int kRouterThreads = 192;
 constexpr int kRouterStages = 4;
 constexpr int kRouterBM = 128;
 constexpr int kBK = 64;  // bf16 elements per 128-byte swizzle row
+// Every expert's rows start on a multiple of this in the permuted row space,
+// so that no 256-row GEMM tile (a CTA pair's tile) straddles two experts.
+constexpr int kExpertRowAlign = 256;
 
 struct RouterArgs {
   int T, N, Npad, num_kb, nblk;
@@ -33,8 +36,9 @@ struct RouterArgs {
   int32_t* block_counts;     // [nblk, N]; rewritten as per-block exclusive bases by the last CTA
   int32_t* counts;           // [N]
   int32_t* offsets;          // [N + 1] unpadded
-  int32_t* row_start;        // [N + 1] start row of each expert, segments padded to 128 rows
-  int32_t* mtile_start;      // [N + 1] prefix sum of ceil(count / 128)
+  int32_t* row_start;        // [N + 1] start row of each expert, segments padded to kExpertRowAlign rows
+  int32_t* mtile_start;      // [N + 1] prefix sum of ceil(count / kExpertRowAlign)
+  int32_t* mtile128_start;   // [N + 1] prefix sum of ceil(count / 128)
   uint32_t* done_counter;    // CTAs finished; reset to 0 by the last CTA
   uint32_t* err;
   uint64_t timeout_ns;
@@ -274,20 +278,23 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   }
   __syncthreads();
   if (tid == 0) {
-    int o = 0, ro = 0, mo = 0;
+    int o = 0, ro = 0, mo = 0, m128 = 0;
     for (int e = 0; e < a.N; ++e) {
       a.offsets[e] = o;
       a.row_start[e] = ro;
       a.mtile_start[e] = mo;
+      a.mtile128_start[e] = m128;
       const int c = scan_tmp[e];
-      const int mt = (c + 127) / 128;
+      const int mt = (c + kExpertRowAlign - 1) / kExpertRowAlign;
       o += c;
       mo += mt;
-      ro += mt * 128;
+      m128 += (c + 127) / 128;
+      ro += mt * kExpertRowAlign;
     }
     a.offsets[a.N] = o;
     a.row_start[a.N] = ro;
     a.mtile_start[a.N] = mo;
+    a.mtile128_start[a.N] = m128;
     *a.done_counter = 0u;
   }
 }

@@ -31,7 +31,7 @@ MOE_FLAG_NO_ROUTED = 0x4
 MOE_FLAG_DEBUG_WAIT_TIMEOUT = 0x100
 
 KERNEL_NAMES = ("router", "permute", "shared_gate_up", "routed_gate_up", "routed_down",
-                "shared_down_combine", "combine")
+                "shared_down", "combine")
 
 
 class moe_config(ctypes.Structure):

@@ -114,8 +114,8 @@ typedef struct moe_ctx* moe_handle;
 /* Device bytes the handle allocates for cfg (host only; no CUDA call). */
 moe_status moe_workspace_bytes(const moe_config* cfg, uint64_t* bytes);
 
-/* Validate cfg, allocate the workspace on `device` and create the handle's
- * second stream.  The caller's current device is restored before returning.
+/* Validate cfg and allocate the workspace on `device`.  The caller's current
+ * device is restored before returning.
  * Returns MOE_ERR_UNSUPPORTED if the device is not sm_100. */
 moe_status moe_create(const moe_config* cfg, int device, moe_handle* out);
 
@@ -144,8 +144,8 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
 moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts,
                            int32_t* offsets, int32_t* src, void* stream);
 
-/* Synchronize the handle's streams and report (then clear) any error the
- * kernels recorded: MOE_ERR_TIMEOUT if a device-side wait ran out. */
+/* Synchronize the stream of the last forward and report (then clear) any
+ * error the kernels recorded: MOE_ERR_TIMEOUT if a device-side wait ran out. */
 moe_status moe_status_query(moe_handle h);
 
 /* Free the workspace and the handle (synchronizes first).  NULL is a no-op. */
@@ -162,8 +162,8 @@ typedef enum moe_kernel_id {
   MOE_KERNEL_SHARED_GATE_UP = 2,      /* shared experts: SwiGLU(x W_gate^T, x W_up^T) */
   MOE_KERNEL_ROUTED_GATE_UP = 3,      /* routed experts: the same, grouped by expert */
   MOE_KERNEL_ROUTED_DOWN = 4,         /* routed experts: g * (H W_down^T) */
-  MOE_KERNEL_SHARED_DOWN_COMBINE = 5, /* shared down projection + the final sum */
-  MOE_KERNEL_COMBINE = 6,             /* the final sum when no shared GEMM carries it */
+  MOE_KERNEL_SHARED_DOWN = 5,         /* shared experts: Hs W_down^T */
+  MOE_KERNEL_COMBINE = 6,             /* h = x + shared + sum_k g * routed, k ascending */
   MOE_KERNEL_COUNT = 7
 } moe_kernel_id;
 moe_status moe_set_timing(moe_handle h, int enable);
