@@ -22,7 +22,12 @@
 //               per thread) and stores bf16 SiLU(gate) * up
 // Tiles are (group, 128-row m-tile, 128-column n-tile); for routed experts
 // the groups' m-tile starts come from the router on the device, so the host
-// never synchronises.
+// never synchronises.  Routed tiles are handed out dynamically: the SMs of
+// each of the B200's two dies take tiles from their own half of the tile
+// range (so the two dies' L2 halves do not both fetch every expert's
+// weights) and steal from the other half when theirs runs out.  The
+// producer fetches each tile id and passes it to the MMA and epilogue warps
+// through a 4-entry shared-memory queue.
 #pragma once
 
 #include "sm100.cuh"
@@ -52,14 +57,18 @@ struct GateUpArgs {
   int n_limit;                 // valid H columns
   __nv_bfloat16* out;          // H
   int ld_out;
+  int* tile_ctr;               // [2] per-die tile counters, zero at launch (grouped); null: static order
+  int die_split;               // SMs with smid below this are on the first die
   uint32_t* err;
   uint64_t timeout_ns;
   int debug_wait;              // CTA 0 waits on a barrier nothing arrives on
 };
 
+constexpr int kGuQueue = 4;  // tile-id queue entries
+
 __host__ __device__ constexpr size_t gateup_smem_bytes() {
-  return 1024 + static_cast<size_t>(kGuStages) * (kGuStageA + kGuStageB) + 8 * (2 * kGuStages + 4 + 2) + 16 +
-         4 * 2 * 264;
+  return 1024 + static_cast<size_t>(kGuStages) * (kGuStageA + kGuStageB) +
+         8 * (2 * kGuStages + 4 + 2 + 2 * kGuQueue) + 16 + 4 * (2 * 264 + kGuQueue);
 }
 
 __device__ __forceinline__ void gu_record_error(uint32_t* err, volatile int* abort, uint32_t site) {
@@ -101,10 +110,13 @@ __global__ void __launch_bounds__(kGuThreads, 1)
   uint64_t* acc_empty = acc_full + 2;      // [2]
   uint64_t* never = acc_empty + 2;
   uint64_t* teardown = never + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* tq_full = teardown + 1;        // [kGuQueue] a tile id is in the slot
+  uint64_t* tq_empty = tq_full + kGuQueue;  // [kGuQueue] MMA + 4 epilogue warps have read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_empty + kGuQueue);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_mts = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [264]
   int32_t* s_rows = s_mts + 264;                                // [264]
+  volatile int32_t* s_tq = s_rows + 264;                        // [kGuQueue]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -135,6 +147,10 @@ __global__ void __launch_bounds__(kGuThreads, 1)
     }
     mbar_init(never, 1);
     mbar_init(teardown, 1);
+    for (int i = 0; i < kGuQueue; ++i) {
+      mbar_init(&tq_full[i], 1);
+      mbar_init(&tq_empty[i], 1 + 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -156,7 +172,38 @@ __global__ void __launch_bounds__(kGuThreads, 1)
     int s = 0, issued = 0;
     uint32_t ph = 0;
     bool stop = false;
-    for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
+    // dynamic schedule: each die owns half of the tiles; static: blockIdx.x + i * gridDim.x
+    const int half = total_tiles / 2;
+    const int die = static_cast<int>(sm_id()) >= a.die_split ? 1 : 0;
+    const int own_lo = die ? half : 0, own_hi = die ? total_tiles : half;
+    const int oth_lo = die ? 0 : half, oth_hi = die ? half : total_tiles;
+    int q = 0, next_static = blockIdx.x;
+    uint32_t qph = 0;
+    while (!stop) {
+      int tile = -1;
+      if (a.tile_ctr) {
+        const int t = own_lo + atomicAdd(&a.tile_ctr[die], 1);
+        if (t < own_hi) {
+          tile = t;
+        } else {  // this die's half is done: help the other die
+          const int u = oth_lo + atomicAdd(&a.tile_ctr[die ^ 1], 1);
+          if (u < oth_hi) tile = u;
+        }
+      } else {
+        tile = next_static < total_tiles ? next_static : -1;
+        next_static += gridDim.x;
+      }
+      if (!mbar_wait(&tq_empty[q], qph ^ 1u, a.timeout_ns, abort_flag)) {
+        gu_record_error(a.err, abort_flag, 8);
+        break;
+      }
+      s_tq[q] = tile;
+      mbar_arrive(&tq_full[q]);
+      if (++q == kGuQueue) {
+        q = 0;
+        qph ^= 1u;
+      }
+      if (tile < 0) break;
       const GuTile c = gu_decode(tile, s_mts, G, a.n_tiles);
       const int n0 = c.n_tile * (kGuBN / 2);
       const int row0 = s_rows[c.g] + c.m_tile * kGuBM;
@@ -196,7 +243,20 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         stop = true;
       }
     }
-    for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
+    int q = 0;
+    uint32_t qph = 0;
+    while (!stop) {
+      if (!mbar_wait(&tq_full[q], qph, a.timeout_ns, abort_flag)) {
+        gu_record_error(a.err, abort_flag, 9);
+        break;
+      }
+      const int tile = s_tq[q];
+      mbar_arrive(&tq_empty[q]);
+      if (++q == kGuQueue) {
+        q = 0;
+        qph ^= 1u;
+      }
+      if (tile < 0) break;
       if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, a.timeout_ns, abort_flag)) {
         gu_record_error(a.err, abort_flag, 5);
         break;
@@ -232,11 +292,27 @@ __global__ void __launch_bounds__(kGuThreads, 1)
     mbar_wait(teardown, 0, a.timeout_ns, nullptr);
   } else if (warp >= 2) {
     // ------------------------------ epilogue ----------------------------------
-    const int q = warp & 3;
-    const int r = q * 32 + lane;
+    const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    int q = 0;
+    uint32_t qph = 0;
+    while (true) {
+      bool okq = mbar_wait(&tq_full[q], qph, a.timeout_ns, abort_flag);
+      okq = __all_sync(0xffffffffu, okq);
+      if (!okq) {
+        if (lane == 0) gu_record_error(a.err, abort_flag, 10);
+        break;
+      }
+      const int tile = s_tq[q];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tq_empty[q]);
+      if (++q == kGuQueue) {
+        q = 0;
+        qph ^= 1u;
+      }
+      if (tile < 0) break;
       const GuTile c = gu_decode(tile, s_mts, G, a.n_tiles);
       bool ok = mbar_wait(&acc_full[acc], acc_ph, a.timeout_ns, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
@@ -245,7 +321,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      const uint32_t tb = tmem + static_cast<uint32_t>(acc * kGuBN) + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tb = tmem + static_cast<uint32_t>(acc * kGuBN) + (static_cast<uint32_t>(quarter * 32) << 16);
       const size_t row = static_cast<size_t>(s_rows[c.g]) + c.m_tile * kGuBM + r;
       const int n0 = c.n_tile * (kGuBN / 2);
       __nv_bfloat16* orow = a.out + row * a.ld_out;

@@ -79,7 +79,7 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 
 struct Layout {
   // byte offsets into the workspace
-  size_t err, done, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, mtile128, gate_perm, x_perm, h, y, hs, ys,
+  size_t err, done, tile_ctr, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, mtile128, gate_perm, x_perm, h, y, hs, ys,
       xdev,
       outdev, total;
   int64_t P, Tpad, nblk;
@@ -100,6 +100,7 @@ Layout make_layout(const moe_config& c) {
   };
   L.err = take(16);
   L.done = take(16);
+  L.tile_ctr = take(16);
   L.idx = take(Tm * Km * 4);
   L.gate = take(Tm * Km * 4);
   L.slot = take(Tm * Km * 4);
@@ -533,6 +534,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   pa.x = static_cast<const __nv_bfloat16*>(x);
   pa.x_perm = h->at<__nv_bfloat16>(L.x_perm);
   pa.gather = do_routed ? 1 : 0;
+  pa.tile_ctr = h->at<int>(L.tile_ctr);
   {
     KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
     permute_gather_kernel<<<dim3(nblk, do_routed ? pa.split : 1), kPermThreads, 0, s0>>>(pa);
@@ -542,6 +544,8 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     GateUpArgs g{};
     g.grouped = 1;
     g.num_groups = (int)N;
+    g.tile_ctr = pa.tile_ctr;
+    g.die_split = h->num_sms / 2;
     g.mtile_start = ra.mtile128_start;
     g.row_start = ra.row_start;
     g.T = (int)T;

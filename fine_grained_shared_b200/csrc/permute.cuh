@@ -30,6 +30,7 @@ struct PermuteArgs {
   const __nv_bfloat16* x;     // [T, d]
   __nv_bfloat16* x_perm;      // [padded rows, d]
   int gather;
+  int* tile_ctr;              // [2] zeroed here for the routed gate/up GEMM that follows
 };
 
 // grid (nblk, split): CTA (b, s) ranks block b's pairs (cheap, repeated by
@@ -44,6 +45,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(PermuteArg
   const int ntok = min(kPermBlockTokens, a.T - t0);
   const int K = a.K;
 
+  if (b == 0 && blockIdx.y == 0 && tid < 2) a.tile_ctr[tid] = 0;
   for (int i = tid; i < a.N * 4; i += kPermThreads) masks[i] = 0u;
   for (int e = tid; e < a.N; e += kPermThreads) {
     base[e] = a.block_base[static_cast<size_t>(b) * a.N + e];
