@@ -383,7 +383,7 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
-  ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);  // A of the routed down GEMM
+  ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
   if (c.n_shared > 0)
     ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kBoxRowsA, 2);
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
@@ -436,6 +436,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   // descriptors that follow the caller's pointers
   static_assert(kGuBoxRowsA == kRouterBM, "x serves as A of the router and of the shared gate/up GEMM");
   bool ok = refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2);
+
   ok = ok && refresh(h->tm_router, router->weight, 0, 1, N, d, (uint32_t)Npad, 2);
   ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, kGuBoxRowsB, 3);
   ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, kGuBoxRowsB, 3);
@@ -513,7 +514,18 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   ra.timeout_ns = kTimeoutNs;
   {
     KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
-    launch_router(K, sigmoid, dim3(nblk), router_smem_bytes(Npad), s0, h->tm_x.map, h->tm_router.map, ra);
+    if (T <= kSmallRouterMaxT) {
+      // a few tokens: one CTA per token on the CUDA cores (counts by atomics, from zero)
+      if (cudaMemsetAsync(ra.block_counts, 0, size_t(nblk) * N * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
+      const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+      const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
+      if (sigmoid)
+        router_small_kernel<true><<<(int)T, kSmallRouterThreads, 0, s0>>>(xb, eb, (int)d, K, ra);
+      else
+        router_small_kernel<false><<<(int)T, kSmallRouterThreads, 0, s0>>>(xb, eb, (int)d, K, ra);
+    } else {
+      launch_router(K, sigmoid, dim3(nblk), router_smem_bytes(Npad), s0, h->tm_x.map, h->tm_router.map, ra);
+    }
   }
 
   PermuteArgs pa{};
@@ -593,7 +605,10 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   ca.add_routed = do_routed ? 1 : 0;
   {
     KernelTimer kt(h, MOE_KERNEL_COMBINE, s0);
-    combine_kernel<<<ceil_div(T * 32, 256), 256, 0, s0>>>(ca);
+    // small batches: one warp per 256 columns of a row; large: one warp per row
+    const int cols = T <= 4 * h->num_sms ? 256 : (int)d;
+    const int64_t warps = T * ceil_div(d, cols);
+    combine_kernel<<<ceil_div(warps * 32, 256), 256, 0, s0>>>(ca, cols);
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

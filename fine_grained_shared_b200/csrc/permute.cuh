@@ -85,15 +85,15 @@ __global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(PermuteArg
   const int nvec = a.d >> 3;
   for (int tl = sp + a.split * warp; tl < ntok; tl += a.split * nwarps) {
     const uint4* srow = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + tl) * a.d);
-    for (int c = lane; c < nvec; c += 32 * 4) {
-      uint4 v[4];
+    for (int c = lane; c < nvec; c += 32 * 8) {  // 8 vectors per lane: a 4 KB row per pass
+      uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+      for (int u = 0; u < 8; ++u)
         if (c + 32 * u < nvec) v[u] = __ldg(srow + c + 32 * u);
       for (int k = 0; k < K; ++k) {
         uint4* drow = reinterpret_cast<uint4*>(a.x_perm + static_cast<size_t>(dst[tl * K + k]) * a.d);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 8; ++u)
           if (c + 32 * u < nvec) drow[c + 32 * u] = v[u];
       }
     }
@@ -113,43 +113,40 @@ struct CombineArgs {
 // Step 5, the layer's output: out[t] = x[t] + ys[t] + sum_k y[slot_of[t, k]]
 // with the routed rows in ascending k (a fixed order, so the result is
 // deterministic), summed in fp32 and rounded once to bf16.  One warp per
-// token streams whole rows (512 contiguous bytes per warp load).
-__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// (token, chunk of cols_per_warp columns): every lane issues all of its
+// 16-byte loads (x, ys and the K routed rows) for 8 columns before it sums,
+// so each warp load reads 512 contiguous bytes of one row.  Large batches
+// give a warp a whole row (it loops over the row); small batches split the
+// row over warps so that enough loads are in flight.
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a, int cols_per_warp) {
+  const int chunks = (a.d + cols_per_warp - 1) / cols_per_warp;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= a.T) return;
-  const int t = warp;
+  if (gw >= a.T * chunks) return;
+  const int t = gw / chunks;
+  const int c0 = (gw - t * chunks) * cols_per_warp;
+  const int c1 = min(a.d, c0 + cols_per_warp);
+  const int K = a.add_routed ? a.K : 0;
   int slots[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) slots[k] = (k < a.K && a.add_routed) ? a.slot_of[static_cast<size_t>(t) * a.K + k] : -1;
-  const int nvec = a.d >> 3;
-  for (int c = lane; c < nvec; c += 32) {
+  for (int k = 0; k < 8; ++k) slots[k] = k < K ? a.slot_of[static_cast<size_t>(t) * a.K + k] : 0;
+  for (int col = c0 + lane * 8; col < c1; col += 256) {
+    uint4 v[10];
+    int nv = 0;
+    if (a.add_residual) v[nv++] = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + col));
+    if (a.ys) v[nv++] = __ldcg(reinterpret_cast<const uint4*>(a.ys + static_cast<size_t>(t) * a.d + col));
+    const int base = nv;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < K) v[base + k] = __ldcg(reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(slots[k]) * a.d + col));
+    nv = base + K;
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    if (a.add_residual) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d) + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[2 * j] += bf16lo(w[j]);
-        acc[2 * j + 1] += bf16hi(w[j]);
-      }
-    }
-    if (a.ys) {
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.ys + static_cast<size_t>(t) * a.d) + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[2 * j] += bf16lo(w[j]);
-        acc[2 * j + 1] += bf16hi(w[j]);
-      }
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (slots[k] >= 0) {
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(slots[k]) * a.d) + c);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < 10; ++i) {
+      if (i < nv) {
+        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           acc[2 * j] += bf16lo(w[j]);
@@ -162,7 +159,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     o.y = pack_bf16x2(acc[2], acc[3]);
     o.z = pack_bf16x2(acc[4], acc[5]);
     o.w = pack_bf16x2(acc[6], acc[7]);
-    reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.d)[c] = o;
+    *reinterpret_cast<uint4*>(a.out + static_cast<size_t>(t) * a.d + col) = o;
   }
 }
 

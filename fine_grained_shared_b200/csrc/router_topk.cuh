@@ -266,12 +266,19 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   if (!*is_last) return;
   __threadfence();
   for (int e = tid; e < a.N; e += kRouterThreads) {
+    // exclusive scan of expert e's column over the blocks, 16 independent
+    // loads in flight at a time (the column is strided by N in memory)
     int run = 0;
-    for (int b = 0; b < a.nblk; ++b) {
-      int32_t* p = a.block_counts + static_cast<size_t>(b) * a.N + e;
-      const int v = __ldcg(p);
-      *p = run;
-      run += v;
+    for (int b0 = 0; b0 < a.nblk; b0 += 16) {
+      int v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        v[i] = (b0 + i < a.nblk) ? __ldcg(a.block_counts + static_cast<size_t>(b0 + i) * a.N + e) : 0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (b0 + i < a.nblk) a.block_counts[static_cast<size_t>(b0 + i) * a.N + e] = run;
+        run += v[i];
+      }
     }
     a.counts[e] = run;
     scan_tmp[e] = run;
@@ -285,6 +292,147 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       a.mtile_start[e] = mo;
       a.mtile128_start[e] = m128;
       const int c = scan_tmp[e];
+      const int mt = (c + kExpertRowAlign - 1) / kExpertRowAlign;
+      o += c;
+      mo += mt;
+      m128 += (c + 127) / 128;
+      ro += mt * kExpertRowAlign;
+    }
+    a.offsets[a.N] = o;
+    a.row_start[a.N] = ro;
+    a.mtile_start[a.N] = mo;
+    a.mtile128_start[a.N] = m128;
+    *a.done_counter = 0u;
+  }
+}
+
+}  // namespace fgs
+
+namespace fgs {
+
+// ---------------------------------------------------------------------------
+// Small batches (T <= kSmallRouterMaxT): one CTA per token on the CUDA cores.
+// The tensor-core router gives a 128-token block to one CTA, so a decode
+// batch of a few dozen tokens would run on a single SM walking d serially.
+// Here each warp computes the logits of experts w, w + 8, ... as dot
+// products (16-byte loads, warp reduction), then warp 0 picks the top K by K
+// rounds of a warp argmax ordered by (key descending, index ascending).
+// Per-block counts are accumulated with integer atomics (exact) and the
+// last CTA runs the same scan as the tensor-core router.
+// ---------------------------------------------------------------------------
+constexpr int kSmallRouterMaxT = 256;
+constexpr int kSmallRouterThreads = 256;
+
+template <bool SIGMOID>
+__global__ void __launch_bounds__(kSmallRouterThreads)
+    router_small_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ e, int d, int K,
+                        RouterArgs a) {
+  __shared__ float key[256], sval[256];
+  __shared__ int is_last;
+  __shared__ int scan_tmp[256];
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+  const int nvec = d >> 3;
+  for (int i = warp; i < a.N; i += kSmallRouterThreads / 32) {
+    const uint4* er = reinterpret_cast<const uint4*>(e + static_cast<size_t>(i) * d);
+    float acc = 0.f;
+    for (int c = lane; c < nvec; c += 32) {
+      const uint4 xv = __ldg(xr + c), ev = __ldg(er + c);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, ew[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc = fmaf(bf16lo(xw[j]), bf16lo(ew[j]), acc);
+        acc = fmaf(bf16hi(xw[j]), bf16hi(ew[j]), acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      if (SIGMOID) {
+        const float sv = 1.f / (1.f + __expf(-acc));
+        sval[i] = sv;
+        key[i] = sv + (a.select_bias ? a.select_bias[i] : 0.f);
+      } else {
+        key[i] = acc + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // softmax statistics over all N logits (softmax mode)
+    float mx = -INFINITY, sum = 0.f;
+    if (!SIGMOID) {
+      for (int i = lane; i < a.N; i += 32) mx = fmaxf(mx, key[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      for (int i = lane; i < a.N; i += 32) sum += __expf(key[i] - mx);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    uint32_t taken = 0;  // bit j: this lane's expert lane + 32 * j is already selected
+    int sel[8];
+    float sel_s[8];
+    float tot = 0.f;
+    for (int k = 0; k < K; ++k) {
+      float bk = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int j = 0, i = lane; i < a.N; ++j, i += 32) {
+        if (taken & (1u << j)) continue;
+        const float v = key[i];
+        if (v > bk || (v == bk && i < bi)) {
+          bk = v;
+          bi = i;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bk, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bk || (ov == bk && oi < bi)) {
+          bk = ov;
+          bi = oi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      sel[k] = bi;
+      sel_s[k] = SIGMOID ? sval[bi] : __expf(bk - mx) / sum;
+      tot += sel_s[k];
+    }
+    if (lane == 0) {
+      for (int k = 0; k < K; ++k) {
+        a.idx[static_cast<size_t>(t) * K + k] = sel[k];
+        a.gate[static_cast<size_t>(t) * K + k] = SIGMOID ? sel_s[k] / tot : sel_s[k];
+        atomicAdd(&a.block_counts[static_cast<size_t>(t / 128) * a.N + sel[k]], 1);
+      }
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = (atomicAdd(a.done_counter, 1u) == static_cast<uint32_t>(gridDim.x - 1));
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  for (int ex = tid; ex < a.N; ex += kSmallRouterThreads) {
+    int run = 0;
+    for (int b = 0; b < a.nblk; ++b) {
+      int32_t* p = a.block_counts + static_cast<size_t>(b) * a.N + ex;
+      const int v = __ldcg(p);
+      *p = run;
+      run += v;
+    }
+    a.counts[ex] = run;
+    scan_tmp[ex] = run;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int o = 0, ro = 0, mo = 0, m128 = 0;
+    for (int ex = 0; ex < a.N; ++ex) {
+      a.offsets[ex] = o;
+      a.row_start[ex] = ro;
+      a.mtile_start[ex] = mo;
+      a.mtile128_start[ex] = m128;
+      const int c = scan_tmp[ex];
       const int mt = (c + kExpertRowAlign - 1) / kExpertRowAlign;
       o += c;
       mo += mt;
