@@ -40,8 +40,8 @@ METRIC = "MoE layer fwd tokens/s; activated-expert TFLOP/s as % of B200 bf16 pea
 UNIT = "tokens/s"
 L2_BYTES = 126 * 2**20
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-DOMINANT = "routed_gate_up"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "routed_gate_up_16b_prefill.txt")
+DOMINANT = "gate_up"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt")
 KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/gateup_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
 
 
@@ -300,11 +300,11 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
     e2e_value = world * shape.T / (e2e_ms * 1e-3)
 
-    # ---- roofline of the dominant kernel (routed gate/up GEMM + SwiGLU) ----
+    # ---- roofline of the dominant kernel (shared + routed gate/up GEMM + SwiGLU) ----
     peaks, peak_src = measured_peaks()
     k_ms, k_n = ktimes[DOMINANT]
     k_avg_ms = max_over_ranks(k_ms / max(1, k_n))
-    k_flop = 4.0 * shape.T * shape.K * shape.d * shape.I
+    k_flop = 4.0 * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is)
     achieved = k_flop / (k_avg_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops_sustained"])
     layer_tflops = world * layer_flop(shape) / (ms_step * 1e-3) / 1e12
@@ -319,7 +319,7 @@ def run_ours(args):
         "tflops_frac_of_peak": layer_tflops / (world * peak),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(shape),
-                     "kernel": "gateup_gemm_kernel (routed experts: gate/up GEMM + SwiGLU)",
+                     "kernel": "gateup_gemm_kernel (shared and routed experts: gate/up GEMM + SwiGLU)",
                      "peak_source": f"{peak_src} bf16_tflops_sustained",
                      "flop_per_launch": k_flop, "avg_launch_ms": k_avg_ms},
         "kernel_ms_per_step": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in ktimes.items()},

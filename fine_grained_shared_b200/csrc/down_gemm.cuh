@@ -23,15 +23,18 @@
 //   warps 2-5   epilogue (both CTAs); warp w reads TMEM lanes 32*(w%4) .. +31
 //               (one output row per thread) and releases the accumulator on
 //               the even CTA's barrier
-// Tiles are (group, 256-row m-tile, 256-column n-tile).  A "group" is one
-// routed expert (its rows are read from device-side offsets written by the
-// router, so the host never synchronises; every expert's rows start on a
-// 256-row boundary) or the single dense group of the shared experts, whose
-// K loop runs over (shared expert j, 64-column block) with a 3-D map of
-// W_down,s [K_s][d][I_s].
+// One launch covers both kinds of expert.  Its tiles are (part, group,
+// 256-row m-tile, 256-column n-tile): first the shared experts' tiles over
+// the rows of Hs, whose K loop runs over (shared expert j, 64-column block)
+// with a 3-D map of W_down,s [K_s][d][I_s] so that one accumulator sums the
+// shared experts, then one group per routed expert (its rows are read from
+// device-side offsets written by the router, so the host never synchronises;
+// every expert's rows start on a 256-row boundary).  The longer shared tiles
+// go first so that they do not make the tail.  Pairs take tiles in a static
+// round-robin order.
 //
-// Epilogue: Y[row, n0 + c] = g[row] * acc[c] (bf16); g = 1 for the shared
-// experts (row_scale == nullptr).  The layer's final k-ordered sum runs in
+// Epilogue: Y[row, n0 + c] = g[row] * acc[c] (bf16) for routed tiles and
+// Ys[row, n0 + c] = acc[c] for shared ones.  The layer's final k-ordered sum runs in
 // combine_kernel, which streams whole rows (permute.cuh).
 #pragma once
 
@@ -55,22 +58,23 @@ static_assert(kStageA == kBoxRowsA * kGemmBK * 2 && kStageB == kBoxRowsB * kGemm
 
 
 struct GemmArgs {
-  // schedule
-  int grouped;                 // 1: groups from mtile_start/row_start; 0: one dense group
-  int num_groups;              // groups when grouped
-  const int32_t* mtile_start;  // [num_groups + 1]
+  // routed experts (grouped rows of H; tiles after the shared ones)
+  int num_groups;              // experts; 0: no routed tiles
+  const int32_t* mtile_start;  // [num_groups + 1] prefix sum of ceil(count / 256)
   const int32_t* row_start;    // [num_groups + 1]
-  int dense_rows;              // rows of the dense group
-  int n_tiles;                 // output tiles along N per group
-  int num_kb;                  // 64-wide k-blocks per sub-expert
-  int J;                       // sub-experts summed into one accumulator
-  int k_per_j;                 // A columns per sub-expert
-  // epilogue
-  int n_limit;                 // valid output columns
-  __nv_bfloat16* out;
+  int num_kb;                  // 64-wide k-blocks over I
+  const float* row_scale;      // g of each row of Y
+  __nv_bfloat16* out;          // Y
+  // shared experts (dense rows of Hs; their tiles come first)
+  int sh_rows;                 // tokens; 0: no shared tiles
+  int sh_num_kb;               // 64-wide k-blocks over I_s
+  int sh_J;                    // shared experts summed into one accumulator
+  int sh_k_per_j;              // Hs columns per shared expert (I_s)
+  __nv_bfloat16* sh_out;       // Ys
+  // both parts
+  int n_tiles;                 // 256-column output tiles (over d)
+  int n_limit;                 // valid output columns (d)
   int ld_out;
-  const float* row_scale;      // g of each row, or nullptr for 1
-  // errors
   uint32_t* err;
   uint64_t timeout_ns;
   int debug_wait;              // CTA 0 waits on a barrier nothing arrives on
@@ -82,11 +86,24 @@ __host__ __device__ constexpr size_t gemm_smem_bytes() {
 }
 
 struct TileCoord {
+  int shared;  // 1: a shared-expert tile over the rows of Hs
   int g, m_tile, n_tile, row0;
 };
 
-__device__ __forceinline__ TileCoord decode_tile(int tile, const int32_t* s_mts, const int32_t* s_rows, int G,
-                                                 int n_tiles) {
+// tiles [0, sh_tiles) are the shared experts' (m-tile major); the rest are
+// the routed experts', expert by expert
+__device__ __forceinline__ TileCoord decode_tile(int tile, int sh_tiles, const int32_t* s_mts,
+                                                 const int32_t* s_rows, int G, int n_tiles) {
+  TileCoord c;
+  if (tile < sh_tiles) {
+    c.shared = 1;
+    c.g = 0;
+    c.m_tile = tile / n_tiles;
+    c.n_tile = tile - c.m_tile * n_tiles;
+    c.row0 = c.m_tile * kGemmBM;
+    return c;
+  }
+  tile -= sh_tiles;
   // largest g with s_mts[g] * n_tiles <= tile (empty groups share a start)
   int lo = 0, hi = G;
   while (hi - lo > 1) {
@@ -94,7 +111,7 @@ __device__ __forceinline__ TileCoord decode_tile(int tile, const int32_t* s_mts,
     if (s_mts[mid] * n_tiles <= tile) lo = mid;
     else hi = mid;
   }
-  TileCoord c;
+  c.shared = 0;
   c.g = lo;
   const int local = tile - s_mts[lo] * n_tiles;
   c.m_tile = local / n_tiles;
@@ -112,9 +129,12 @@ __device__ __forceinline__ void pair_record_error(uint32_t* err, volatile int* a
   atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
 }
 
-// tmA: H (routed) or Hs (shared) rows; tmB: W_down as [groups * J][d][I].
+// tmA: H rows; tmB: W_down as [experts][d][I].  tmAs: Hs rows; tmBs: the
+// shared experts' W_down as [K_s][d][I_s].  Maps of an absent part are never
+// read.
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    down_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs a) {
+    down_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmAs, const __grid_constant__ CUtensorMap tmBs, GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -135,22 +155,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
-  int G;
-  if (a.grouped) {
-    G = a.num_groups;
-    for (int i = tid; i <= G; i += kGemmThreads) {
-      s_mts[i] = a.mtile_start[i];
-      s_rows[i] = a.row_start[i];
-    }
-  } else {
-    G = 1;
-    if (tid == 0) {
-      s_mts[0] = 0;
-      s_mts[1] = (a.dense_rows + kGemmBM - 1) / kGemmBM;
-      s_rows[0] = 0;
-      s_rows[1] = s_mts[1] * kGemmBM;
-    }
+  const int G = a.num_groups;
+  for (int i = tid; i <= G; i += kGemmThreads) {
+    s_mts[i] = G ? a.mtile_start[i] : 0;
+    s_rows[i] = G ? a.row_start[i] : 0;
   }
+  const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGemmBM - 1) / kGemmBM * a.n_tiles : 0;
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
       mbar_init(&full[s], 1);
@@ -173,25 +183,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   cluster_sync();  // both CTAs' barriers exist before any copy or arrive targets them
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int total_tiles = s_mts[G] * a.n_tiles;
+  const int total_tiles = sh_tiles + s_mts[G] * a.n_tiles;
   const uint32_t full_lead = mapa_shared(smem_u32(full), 0);         // the even CTA's full[0]
   const uint32_t acc_empty_lead = mapa_shared(smem_u32(acc_empty), 0);
   bool aborted = false;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------ TMA producer ------------------------------
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    if (G) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+    }
+    if (sh_tiles) {
+      tma_prefetch_desc(&tmAs);
+      tma_prefetch_desc(&tmBs);
+    }
     int s = 0, issued = 0;
     uint32_t ph = 0;
     for (int tile = pair; tile < total_tiles && !aborted; tile += num_pairs) {
-      const TileCoord c = decode_tile(tile, s_mts, s_rows, G, a.n_tiles);
+      const TileCoord c = decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
       const int row0 = c.row0 + static_cast<int>(rank) * kCtaRows;
       // each CTA stages its half of the tile's 256 output columns of W_down
       const int brow = c.n_tile * kGemmBN + static_cast<int>(rank) * (kGemmBN / 2);
-      for (int j = 0; j < a.J && !aborted; ++j) {
-        const int bz = c.g * a.J + j;
-        for (int kb = 0; kb < a.num_kb; ++kb) {
+      const CUtensorMap* mA = c.shared ? &tmAs : &tmA;
+      const CUtensorMap* mB = c.shared ? &tmBs : &tmB;
+      const int J = c.shared ? a.sh_J : 1;
+      const int num_kb = c.shared ? a.sh_num_kb : a.num_kb;
+      for (int j = 0; j < J && !aborted; ++j) {
+        // shared: sub-expert j of the one dense group; routed: expert g
+        const int bz = c.shared ? j : c.g;
+        const int k0 = c.shared ? j * a.sh_k_per_j : 0;
+        for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag)) {
             pair_record_error(a.err, abort_flag, rank, 3);
             aborted = true;
@@ -200,8 +222,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kStageA + kStageB));
           const int kc = kb * kGemmBK;
           const uint32_t fb = full_lead + 8u * static_cast<uint32_t>(s);
-          tma_load_2d_pair(sA + s * kStageA, &tmA, fb, j * a.k_per_j + kc, row0);
-          tma_load_3d_pair(sB + s * kStageB, &tmB, fb, kc, brow, bz);
+          tma_load_2d_pair(sA + s * kStageA, mA, fb, k0 + kc, row0);
+          tma_load_3d_pair(sB + s * kStageB, mB, fb, kc, brow, bz);
           ++issued;
           if (++s == kGemmStages) {
             s = 0;
@@ -232,6 +254,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     for (int tile = pair; tile < total_tiles && !aborted; tile += num_pairs) {
+      const int kblocks = tile < sh_tiles ? a.sh_J * a.sh_num_kb : a.num_kb;
       if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, a.timeout_ns, abort_flag)) {
         pair_record_error(a.err, abort_flag, rank, 5);
         aborted = true;
@@ -239,27 +262,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       tc_fence_after_sync();
       const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * kGemmBN);
-      bool first = true;
-      for (int j = 0; j < a.J && !aborted; ++j) {
-        for (int kb = 0; kb < a.num_kb; ++kb) {
-          if (!mbar_wait(&full[s], ph, a.timeout_ns, abort_flag)) {
-            pair_record_error(a.err, abort_flag, rank, 6);
-            aborted = true;
-            break;
-          }
-          tc_fence_after_sync();
-          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * kStageA));
-          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * kStageB));
+      for (int kb = 0; kb < kblocks; ++kb) {
+        if (!mbar_wait(&full[s], ph, a.timeout_ns, abort_flag)) {
+          pair_record_error(a.err, abort_flag, rank, 6);
+          aborted = true;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * kStageA));
+        const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * kStageB));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, first ? 0u : 1u);
-            first = false;
-          }
-          umma_commit_pair_multicast(&empty[s], 0x3);
-          if (++s == kGemmStages) {
-            s = 0;
-            ph ^= 1u;
-          }
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+        umma_commit_pair_multicast(&empty[s], 0x3);
+        if (++s == kGemmStages) {
+          s = 0;
+          ph ^= 1u;
         }
       }
       if (aborted) break;
@@ -278,7 +296,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = pair; tile < total_tiles; tile += num_pairs) {
-      const TileCoord c = decode_tile(tile, s_mts, s_rows, G, a.n_tiles);
+      const TileCoord c = decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
       bool ok = mbar_wait(&acc_full[acc], acc_ph, a.timeout_ns, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -292,8 +310,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
       {
         const int n0 = c.n_tile * kGemmBN;
-        const float sc = a.row_scale ? a.row_scale[row] : 1.f;
-        __nv_bfloat16* orow = a.out + row * a.ld_out;
+        const float sc = c.shared ? 1.f : a.row_scale[row];
+        __nv_bfloat16* orow = (c.shared ? a.sh_out : a.out) + row * a.ld_out;
 #pragma unroll 1
         for (int cc = 0; cc < kGemmBN; cc += 16) {
           uint32_t vr[16];

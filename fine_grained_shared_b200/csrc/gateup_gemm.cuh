@@ -20,14 +20,17 @@
 //               i overlaps the MMAs of tile i + 1
 //   warps 2-5   epilogue; warp w reads TMEM lanes 32*(w%4) .. +31 (one H row
 //               per thread) and stores bf16 SiLU(gate) * up
-// Tiles are (group, 128-row m-tile, 128-column n-tile); for routed experts
-// the groups' m-tile starts come from the router on the device, so the host
-// never synchronises.  Routed tiles are handed out dynamically: the SMs of
-// each of the B200's two dies take tiles from their own half of the tile
-// range (so the two dies' L2 halves do not both fetch every expert's
-// weights) and steal from the other half when theirs runs out.  The
-// producer fetches each tile id and passes it to the MMA and epilogue warps
-// through a 4-entry shared-memory queue.
+// One launch covers both kinds of expert.  Its tiles are (part, group,
+// 128-row m-tile, 128-column n-tile): first the shared experts' tiles over
+// the rows of x (one dense group whose H columns are the shared experts'
+// intermediate columns side by side), then the routed experts' tiles, whose
+// groups' m-tile starts come from the router on the device, so the host never
+// synchronises.  Tiles are handed out dynamically: the SMs of each of the
+// B200's two dies take tiles from their own half of the tile range (so the
+// two dies' L2 halves do not both fetch every expert's weights) and steal
+// from the other half when theirs runs out.  The producer fetches each tile
+// id and passes it to the MMA and epilogue warps through a 4-entry
+// shared-memory queue.
 #pragma once
 
 #include "sm100.cuh"
@@ -47,17 +50,23 @@ constexpr uint32_t kGuBoxRowsA = kGuBM;      // tiled x (shared experts)
 constexpr uint32_t kGuBoxRowsB = kGuBN / 2;  // W_gate and W_up
 
 struct GateUpArgs {
-  int grouped;                 // 1: routed experts (groups from the router); 0: dense rows of x
-  int num_groups;              // experts (grouped)
-  const int32_t* mtile_start;  // [G + 1] prefix sum of ceil(count / 128) (grouped)
-  const int32_t* row_start;    // [G + 1] first row of each expert in X_perm and H (grouped)
-  int T;                       // tokens (dense row count)
-  int n_tiles;                 // 128-column H tiles per group
-  int num_kb;                  // 64-wide k-blocks over d
+  // routed experts (grouped rows of X_perm; their tiles follow the shared ones)
+  int num_groups;              // experts; 0: no routed tiles
+  const int32_t* mtile_start;  // [G + 1] prefix sum of ceil(count / 128)
+  const int32_t* row_start;    // [G + 1] first row of each expert in X_perm and H
+  int n_tiles;                 // 128-column H tiles per expert
   int n_limit;                 // valid H columns
   __nv_bfloat16* out;          // H
   int ld_out;
-  int* tile_ctr;               // [2] per-die tile counters, zero at launch (grouped); null: static order
+  // shared experts (the dense rows of x; their tiles come first)
+  int sh_rows;                 // tokens; 0: no shared tiles
+  int sh_n_tiles;              // 128-column Hs tiles
+  int sh_n_limit;              // valid Hs columns (shared experts x their intermediate size)
+  __nv_bfloat16* sh_out;       // Hs
+  int sh_ld_out;
+  // both parts
+  int num_kb;                  // 64-wide k-blocks over d
+  int* tile_ctr;               // [2] per-die tile counters, zero at launch; null: static order
   int die_split;               // SMs with smid below this are on the first die
   uint32_t* err;
   uint64_t timeout_ns;
@@ -77,29 +86,48 @@ __device__ __forceinline__ void gu_record_error(uint32_t* err, volatile int* abo
 }
 
 struct GuTile {
-  int g, m_tile, n_tile;
+  int shared;  // 1: a shared-expert tile over the rows of x
+  int g, m_tile, n_tile, row0;
 };
 
-__device__ __forceinline__ GuTile gu_decode(int tile, const int32_t* s_mts, int G, int n_tiles) {
+// tiles [0, sh_tiles) are the shared experts' (m-tile major); the rest are
+// the routed experts', expert by expert
+__device__ __forceinline__ GuTile gu_decode(int tile, int sh_tiles, int sh_n_tiles, const int32_t* s_mts,
+                                           const int32_t* s_rows, int G, int n_tiles) {
+  GuTile c;
+  if (tile < sh_tiles) {
+    c.shared = 1;
+    c.g = 0;
+    c.m_tile = tile / sh_n_tiles;
+    c.n_tile = tile - c.m_tile * sh_n_tiles;
+    c.row0 = c.m_tile * kGuBM;
+    return c;
+  }
+  tile -= sh_tiles;
   int lo = 0, hi = G;  // largest g with s_mts[g] * n_tiles <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
     if (s_mts[mid] * n_tiles <= tile) lo = mid;
     else hi = mid;
   }
-  GuTile c;
+  c.shared = 0;
   c.g = lo;
   const int local = tile - s_mts[lo] * n_tiles;
   c.m_tile = local / n_tiles;
   c.n_tile = local - c.m_tile * n_tiles;
+  c.row0 = s_rows[lo] + c.m_tile * kGuBM;
   return c;
 }
 
-// tmA: X_perm (grouped) or x (dense) with a 128-row box.
-// tmG, tmU: W_gate, W_up as [groups][rows][d] with a 128-row box.
+// tmA: X_perm with a 128-row box; tmG, tmU: W_gate, W_up as [experts][I][d]
+// with a 128-row box.  tmAs: x with a 128-row box; tmGs, tmUs: the shared
+// experts' W_gate, W_up as [1][K_s * I_s][d].  Maps of an absent part are
+// never read.
 __global__ void __launch_bounds__(kGuThreads, 1)
     gateup_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
-                       const __grid_constant__ CUtensorMap tmU, GateUpArgs a) {
+                       const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmAs,
+                       const __grid_constant__ CUtensorMap tmGs, const __grid_constant__ CUtensorMap tmUs,
+                       GateUpArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -120,22 +148,12 @@ __global__ void __launch_bounds__(kGuThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  int G;
-  if (a.grouped) {
-    G = a.num_groups;
-    for (int i = tid; i <= G; i += kGuThreads) {
-      s_mts[i] = a.mtile_start[i];
-      s_rows[i] = a.row_start[i];
-    }
-  } else {
-    G = 1;
-    if (tid == 0) {
-      s_mts[0] = 0;
-      s_mts[1] = (a.T + kGuBM - 1) / kGuBM;
-      s_rows[0] = 0;
-      s_rows[1] = s_mts[1] * kGuBM;
-    }
+  const int G = a.num_groups;
+  for (int i = tid; i <= G; i += kGuThreads) {
+    s_mts[i] = G ? a.mtile_start[i] : 0;
+    s_rows[i] = G ? a.row_start[i] : 0;
   }
+  const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGuBM - 1) / kGuBM * a.sh_n_tiles : 0;
   if (tid == 0) {
     for (int s = 0; s < kGuStages; ++s) {
       mbar_init(&full[s], 1);
@@ -162,13 +180,20 @@ __global__ void __launch_bounds__(kGuThreads, 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int total_tiles = s_mts[G] * a.n_tiles;
+  const int total_tiles = sh_tiles + s_mts[G] * a.n_tiles;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------ TMA producer ------------------------------
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmG);
-    tma_prefetch_desc(&tmU);
+    if (G) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmG);
+      tma_prefetch_desc(&tmU);
+    }
+    if (sh_tiles) {
+      tma_prefetch_desc(&tmAs);
+      tma_prefetch_desc(&tmGs);
+      tma_prefetch_desc(&tmUs);
+    }
     int s = 0, issued = 0;
     uint32_t ph = 0;
     bool stop = false;
@@ -204,9 +229,11 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         qph ^= 1u;
       }
       if (tile < 0) break;
-      const GuTile c = gu_decode(tile, s_mts, G, a.n_tiles);
+      const GuTile c = gu_decode(tile, sh_tiles, a.sh_n_tiles, s_mts, s_rows, G, a.n_tiles);
       const int n0 = c.n_tile * (kGuBN / 2);
-      const int row0 = s_rows[c.g] + c.m_tile * kGuBM;
+      const CUtensorMap* mA = c.shared ? &tmAs : &tmA;
+      const CUtensorMap* mG = c.shared ? &tmGs : &tmG;
+      const CUtensorMap* mU = c.shared ? &tmUs : &tmU;
       for (int kb = 0; kb < a.num_kb; ++kb) {
         if (!mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag)) {
           gu_record_error(a.err, abort_flag, 3);
@@ -215,9 +242,9 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         }
         mbar_arrive_expect_tx(&full[s], kGuStageA + kGuStageB);
         const int kc = kb * kGuBK;
-        tma_load_2d(sA + s * kGuStageA, &tmA, &full[s], kc, row0);
-        tma_load_3d(sB + s * kGuStageB, &tmG, &full[s], kc, n0, c.g);
-        tma_load_3d(sB + s * kGuStageB + kGuStageB / 2, &tmU, &full[s], kc, n0, c.g);
+        tma_load_2d(sA + s * kGuStageA, mA, &full[s], kc, c.row0);
+        tma_load_3d(sB + s * kGuStageB, mG, &full[s], kc, n0, c.g);
+        tma_load_3d(sB + s * kGuStageB + kGuStageB / 2, mU, &full[s], kc, n0, c.g);
         ++issued;
         if (++s == kGuStages) {
           s = 0;
@@ -313,7 +340,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         qph ^= 1u;
       }
       if (tile < 0) break;
-      const GuTile c = gu_decode(tile, s_mts, G, a.n_tiles);
+      const GuTile c = gu_decode(tile, sh_tiles, a.sh_n_tiles, s_mts, s_rows, G, a.n_tiles);
       bool ok = mbar_wait(&acc_full[acc], acc_ph, a.timeout_ns, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -322,9 +349,10 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       }
       tc_fence_after_sync();
       const uint32_t tb = tmem + static_cast<uint32_t>(acc * kGuBN) + (static_cast<uint32_t>(quarter * 32) << 16);
-      const size_t row = static_cast<size_t>(s_rows[c.g]) + c.m_tile * kGuBM + r;
+      const size_t row = static_cast<size_t>(c.row0) + r;
       const int n0 = c.n_tile * (kGuBN / 2);
-      __nv_bfloat16* orow = a.out + row * a.ld_out;
+      const int n_limit = c.shared ? a.sh_n_limit : a.n_limit;
+      __nv_bfloat16* orow = c.shared ? a.sh_out + row * a.sh_ld_out : a.out + row * a.ld_out;
 #pragma unroll 1
       for (int cc = 0; cc < kGuBN / 2; cc += 16) {
         uint32_t gr[16], ur[16];
@@ -332,7 +360,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         tmem_ld16(tb + kGuBN / 2 + cc, ur);
         tmem_ld_wait();
         const int col = n0 + cc;
-        if (col < a.n_limit) {
+        if (col < n_limit) {
           uint32_t pk[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {

@@ -2,17 +2,15 @@
 // workspace, TMA descriptors and the launch sequence of one layer forward.
 //
 // Launch sequence, all on the caller's stream:
-//   shared experts' gate/up GEMM + SwiGLU         Hs = SwiGLU(x)
-//   shared experts' down GEMM                     Ys = Hs W_down,s^T
 //   router_topk (logits, top-K, histogram, scan)  idx, gate, offsets
 //   permute_gather                                X_perm, slot_of, g
-//   routed gate/up grouped GEMM + SwiGLU          H
-//   routed down grouped GEMM + gate scale         Y = g * (H W_down^T)
+//   gate/up GEMM + SwiGLU, shared and routed      Hs = SwiGLU(x), H = SwiGLU(X_perm)
+//   down GEMM, shared and routed (+ gate scale)   Ys = Hs W_down,s^T, Y = g * (H W_down^T)
 //   combine                                       out = x + Ys + sum_k Y (k ascending)
-// Every GEMM is a persistent kernel that fills all SMs, so running the
-// shared experts on a second stream gave no overlap (measured: 2.62 ms per
-// 16B-prefill forward with two streams, 2.60 ms with one); one stream keeps
-// each kernel's timing clean.  Nothing is copied back to the host.
+// Each GEMM launch covers the shared experts' tiles and the routed experts'
+// tiles in one persistent kernel, so the shared experts fill the SMs that a
+// small batch's routed tiles leave idle and the two never wait on each
+// other's tail.  Nothing is copied back to the host.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -249,8 +247,9 @@ bool refresh(MapCache& c, const void* p, int64_t rows_key, uint64_t d2, uint64_t
   return true;
 }
 
-// Launch `pairs` CTA pairs (clusters of 2) of the GEMM kernel.
-cudaError_t launch_down(int pairs, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& B, const GemmArgs& ga) {
+// Launch `pairs` CTA pairs (clusters of 2) of the down GEMM kernel.
+cudaError_t launch_down(int pairs, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& As,
+                        const CUtensorMap& Bs, const GemmArgs& ga) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(kGemmThreads);
@@ -263,12 +262,12 @@ cudaError_t launch_down(int pairs, cudaStream_t s, const CUtensorMap& A, const C
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, down_gemm_kernel, A, B, ga);
+  return cudaLaunchKernelEx(&cfg, down_gemm_kernel, A, B, As, Bs, ga);
 }
 
 cudaError_t launch_gateup(int ctas, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& G, const CUtensorMap& U,
-                          const GateUpArgs& ga) {
-  gateup_gemm_kernel<<<ctas, kGuThreads, gateup_smem_bytes(), s>>>(A, G, U, ga);
+                          const CUtensorMap& As, const CUtensorMap& Gs, const CUtensorMap& Us, const GateUpArgs& ga) {
+  gateup_gemm_kernel<<<ctas, kGuThreads, gateup_smem_bytes(), s>>>(A, G, U, As, Gs, Us, ga);
   return cudaGetLastError();
 }
 
@@ -298,14 +297,6 @@ class KernelTimer {
   cudaStream_t s_;
   cudaEvent_t stop_ = nullptr;
 };
-
-GemmArgs base_args(moe_ctx* h) {
-  GemmArgs g{};
-  g.err = h->at<uint32_t>(h->L.err);
-  g.timeout_ns = kTimeoutNs;
-  g.J = 1;
-  return g;
-}
 
 }  // namespace
 
@@ -453,45 +444,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   h->last_K = K;
   const int nblk = ceil_div(T, 128);
 
-  // ---- shared experts (need only x) ----
-  if (do_shared) {
-    GateUpArgs g{};
-    g.grouped = 0;
-    g.T = (int)T;
-    g.n_tiles = ceil_div(Ks * Is, kGuBN / 2);
-    g.num_kb = ceil_div(d, kGuBK);
-    g.n_limit = (int)(Ks * Is);
-    g.out = h->at<__nv_bfloat16>(L.hs);
-    g.ld_out = (int)(Ks * Is);
-    g.err = h->at<uint32_t>(L.err);
-    g.timeout_ns = kTimeoutNs;
-    const int tiles = ceil_div(T, kGuBM) * g.n_tiles;
-    {
-      KernelTimer kt(h, MOE_KERNEL_SHARED_GATE_UP, s0);
-      if (launch_gateup(tiles < h->num_sms ? tiles : h->num_sms, s0, h->tm_x.map, h->tm_swg.map,
-                        h->tm_swu.map, g) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    GemmArgs g2 = base_args(h);
-    g2.grouped = 0;
-    g2.dense_rows = (int)T;
-    g2.n_tiles = ceil_div(d, kGemmBN);
-    g2.num_kb = ceil_div(Is, kGemmBK);
-    g2.J = (int)Ks;
-    g2.k_per_j = (int)Is;
-    g2.n_limit = (int)d;
-    g2.out = h->at<__nv_bfloat16>(L.ys);
-    g2.ld_out = (int)d;
-    const int tiles2 = ceil_div(T, kGemmBM) * g2.n_tiles;
-    {
-      KernelTimer kt(h, MOE_KERNEL_SHARED_DOWN, s0);
-      if (launch_down(tiles2 < h->max_pairs ? tiles2 : h->max_pairs, s0, h->tm_hs, h->tm_swd.map, g2) !=
-          cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-  }
-
-  // ---- router, permutation, routed experts ----
+  // ---- router and permutation ----
   RouterArgs ra{};
   ra.T = (int)T;
   ra.N = (int)N;
@@ -515,8 +468,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   {
     KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
     if (T <= kSmallRouterMaxT) {
-      // a few tokens: one CTA per token on the CUDA cores (counts by atomics, from zero)
-      if (cudaMemsetAsync(ra.block_counts, 0, size_t(nblk) * N * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
+      // a few tokens: one CTA per token on the CUDA cores
       const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
       const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
       if (sigmoid)
@@ -552,43 +504,72 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     permute_gather_kernel<<<dim3(nblk, do_routed ? pa.split : 1), kPermThreads, 0, s0>>>(pa);
   }
 
-  if (do_routed) {
+  // ---- the expert GEMMs: shared experts' tiles first, then the routed experts' ----
+  if (do_routed || do_shared) {
+    const int num_kb = ceil_div(d, kGuBK);
     GateUpArgs g{};
-    g.grouped = 1;
-    g.num_groups = (int)N;
+    if (do_routed) {
+      g.num_groups = (int)N;
+      g.mtile_start = ra.mtile128_start;
+      g.row_start = ra.row_start;
+      g.n_tiles = ceil_div(I, kGuBN / 2);
+      g.n_limit = (int)I;
+      g.out = h->at<__nv_bfloat16>(L.h);
+      g.ld_out = (int)I;
+    }
+    if (do_shared) {
+      g.sh_rows = (int)T;
+      g.sh_n_tiles = ceil_div(Ks * Is, kGuBN / 2);
+      g.sh_n_limit = (int)(Ks * Is);
+      g.sh_out = h->at<__nv_bfloat16>(L.hs);
+      g.sh_ld_out = (int)(Ks * Is);
+    }
+    g.num_kb = num_kb;
     g.tile_ctr = pa.tile_ctr;
     g.die_split = h->num_sms / 2;
-    g.mtile_start = ra.mtile128_start;
-    g.row_start = ra.row_start;
-    g.T = (int)T;
-    g.n_tiles = ceil_div(I, kGuBN / 2);
-    g.num_kb = ceil_div(d, kGuBK);
-    g.n_limit = (int)I;
-    g.out = h->at<__nv_bfloat16>(L.h);
-    g.ld_out = (int)I;
     g.err = h->at<uint32_t>(L.err);
     g.timeout_ns = kTimeoutNs;
     g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
+    // with routed tiles the count is known only on the device: one CTA per SM
+    const int sh_tiles = do_shared ? ceil_div(T, kGuBM) * g.sh_n_tiles : 0;
+    const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
+    // an absent part's maps are never read; the present part's stand in
+    const CUtensorMap& sA = do_shared ? h->tm_x.map : h->tm_xperm;
+    const CUtensorMap& sG = do_shared ? h->tm_swg.map : h->tm_wg.map;
+    const CUtensorMap& sU = do_shared ? h->tm_swu.map : h->tm_wu.map;
     {
-      KernelTimer kt(h, MOE_KERNEL_ROUTED_GATE_UP, s0);
-      if (launch_gateup(h->num_sms, s0, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, g) != cudaSuccess)
+      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+      if (launch_gateup(ctas, s0, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
 
-    GemmArgs g2 = base_args(h);
-    g2.grouped = 1;
-    g2.num_groups = (int)N;
-    g2.mtile_start = ra.mtile_start;
-    g2.row_start = ra.row_start;
+    GemmArgs g2{};
+    if (do_routed) {
+      g2.num_groups = (int)N;
+      g2.mtile_start = ra.mtile_start;
+      g2.row_start = ra.row_start;
+      g2.num_kb = ceil_div(I, kGemmBK);
+      g2.row_scale = pa.gate_perm;
+      g2.out = h->at<__nv_bfloat16>(L.y);
+    }
+    if (do_shared) {
+      g2.sh_rows = (int)T;
+      g2.sh_num_kb = ceil_div(Is, kGemmBK);
+      g2.sh_J = (int)Ks;
+      g2.sh_k_per_j = (int)Is;
+      g2.sh_out = h->at<__nv_bfloat16>(L.ys);
+    }
     g2.n_tiles = ceil_div(d, kGemmBN);
-    g2.num_kb = ceil_div(I, kGemmBK);
-    g2.k_per_j = (int)I;
     g2.n_limit = (int)d;
-    g2.out = h->at<__nv_bfloat16>(L.y);
     g2.ld_out = (int)d;
-    g2.row_scale = pa.gate_perm;
-    KernelTimer kt(h, MOE_KERNEL_ROUTED_DOWN, s0);
-    if (launch_down(h->max_pairs, s0, h->tm_h, h->tm_wd.map, g2) != cudaSuccess) return MOE_ERR_CUDA;
+    g2.err = h->at<uint32_t>(L.err);
+    g2.timeout_ns = kTimeoutNs;
+    const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
+    const int pairs = do_routed || sh_tiles2 > h->max_pairs ? h->max_pairs : sh_tiles2;
+    const CUtensorMap& sA2 = do_shared ? h->tm_hs : h->tm_h;
+    const CUtensorMap& sB2 = do_shared ? h->tm_swd.map : h->tm_wd.map;
+    KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
+    if (launch_down(pairs, s0, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // ---- the final sum ----

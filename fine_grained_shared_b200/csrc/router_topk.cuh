@@ -314,47 +314,77 @@ namespace fgs {
 // Small batches (T <= kSmallRouterMaxT): one CTA per token on the CUDA cores.
 // The tensor-core router gives a 128-token block to one CTA, so a decode
 // batch of a few dozen tokens would run on a single SM walking d serially.
-// Here each warp computes the logits of experts w, w + 8, ... as dot
-// products (16-byte loads, warp reduction), then warp 0 picks the top K by K
-// rounds of a warp argmax ordered by (key descending, index ascending).
-// Per-block counts are accumulated with integer atomics (exact) and the
-// last CTA runs the same scan as the tensor-core router.
+// Here each warp computes the logits of kSmallRouterBatch experts at once as
+// dot products (16-byte loads of x and of the experts' rows in flight
+// together, warp reduction), then warp 0 picks the top K by K rounds of a
+// warp argmax ordered by (key descending, index ascending).  The last CTA to
+// finish counts the selected experts of every 128-token block from the
+// written indices (shared-memory integer atomics: exact, and no buffer needs
+// clearing between calls) and runs the same scan as the tensor-core router.
 // ---------------------------------------------------------------------------
 constexpr int kSmallRouterMaxT = 256;
 constexpr int kSmallRouterThreads = 256;
+constexpr int kSmallRouterBatch = 8;  // experts one warp reduces together
 
 template <bool SIGMOID>
 __global__ void __launch_bounds__(kSmallRouterThreads)
     router_small_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ e, int d, int K,
                         RouterArgs a) {
+  static_assert(kSmallRouterMaxT <= 2 * 128, "the last CTA's histogram holds two 128-token blocks");
   __shared__ float key[256], sval[256];
   __shared__ int is_last;
   __shared__ int scan_tmp[256];
+  __shared__ int hist[2][256];
   const int t = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
   const int nvec = d >> 3;
-  for (int i = warp; i < a.N; i += kSmallRouterThreads / 32) {
-    const uint4* er = reinterpret_cast<const uint4*>(e + static_cast<size_t>(i) * d);
-    float acc = 0.f;
-    for (int c = lane; c < nvec; c += 32) {
-      const uint4 xv = __ldg(xr + c), ev = __ldg(er + c);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, ew[4] = {ev.x, ev.y, ev.z, ev.w};
+  constexpr int kWarps = kSmallRouterThreads / 32;
+  for (int i0 = warp * kSmallRouterBatch; i0 < a.N; i0 += kWarps * kSmallRouterBatch) {
+    const uint4* er[kSmallRouterBatch];
+    float acc[kSmallRouterBatch];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc = fmaf(bf16lo(xw[j]), bf16lo(ew[j]), acc);
-        acc = fmaf(bf16hi(xw[j]), bf16hi(ew[j]), acc);
+    for (int q = 0; q < kSmallRouterBatch; ++q) {
+      const int i = i0 + q < a.N ? i0 + q : a.N - 1;  // past the end: re-read the last row, result unused
+      er[q] = reinterpret_cast<const uint4*>(e + static_cast<size_t>(i) * d);
+      acc[q] = 0.f;
+    }
+#pragma unroll 2
+    for (int c = lane; c < nvec; c += 32) {
+      const uint4 xv = __ldg(xr + c);
+      uint4 ev[kSmallRouterBatch];
+#pragma unroll
+      for (int q = 0; q < kSmallRouterBatch; ++q) ev[q] = __ldg(er[q] + c);
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float xl[4] = {bf16lo(xw[0]), bf16lo(xw[1]), bf16lo(xw[2]), bf16lo(xw[3])};
+      const float xh[4] = {bf16hi(xw[0]), bf16hi(xw[1]), bf16hi(xw[2]), bf16hi(xw[3])};
+#pragma unroll
+      for (int q = 0; q < kSmallRouterBatch; ++q) {
+        const uint32_t ew[4] = {ev[q].x, ev[q].y, ev[q].z, ev[q].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[q] = fmaf(xl[j], bf16lo(ew[j]), acc[q]);
+          acc[q] = fmaf(xh[j], bf16hi(ew[j]), acc[q]);
+        }
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    for (int q = 0; q < kSmallRouterBatch; ++q) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
+    }
     if (lane == 0) {
-      if (SIGMOID) {
-        const float sv = 1.f / (1.f + __expf(-acc));
-        sval[i] = sv;
-        key[i] = sv + (a.select_bias ? a.select_bias[i] : 0.f);
-      } else {
-        key[i] = acc + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
+#pragma unroll
+      for (int q = 0; q < kSmallRouterBatch; ++q) {
+        const int i = i0 + q;
+        if (i >= a.N) break;
+        if (SIGMOID) {
+          const float sv = 1.f / (1.f + __expf(-acc[q]));
+          sval[i] = sv;
+          key[i] = sv + (a.select_bias ? a.select_bias[i] : 0.f);
+        } else {
+          key[i] = acc[q] + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
+        }
       }
     }
   }
@@ -403,7 +433,6 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
       for (int k = 0; k < K; ++k) {
         a.idx[static_cast<size_t>(t) * K + k] = sel[k];
         a.gate[static_cast<size_t>(t) * K + k] = SIGMOID ? sel_s[k] / tot : sel_s[k];
-        atomicAdd(&a.block_counts[static_cast<size_t>(t / 128) * a.N + sel[k]], 1);
       }
     }
   }
@@ -413,13 +442,17 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
   __syncthreads();
   if (!is_last) return;
   __threadfence();
+  // every token's selection is written: count them per 128-token block
+  for (int i = tid; i < 2 * 256; i += kSmallRouterThreads) (&hist[0][0])[i] = 0;
+  __syncthreads();
+  const int TK = a.T * K;
+  for (int i = tid; i < TK; i += kSmallRouterThreads) atomicAdd(&hist[(i / K) >> 7][__ldcg(a.idx + i)], 1);
+  __syncthreads();
   for (int ex = tid; ex < a.N; ex += kSmallRouterThreads) {
     int run = 0;
     for (int b = 0; b < a.nblk; ++b) {
-      int32_t* p = a.block_counts + static_cast<size_t>(b) * a.N + ex;
-      const int v = __ldcg(p);
-      *p = run;
-      run += v;
+      a.block_counts[static_cast<size_t>(b) * a.N + ex] = run;  // exclusive base of block b
+      run += hist[b][ex];
     }
     a.counts[ex] = run;
     scan_tmp[ex] = run;

@@ -30,8 +30,7 @@ MOE_FLAG_NO_SHARED = 0x2
 MOE_FLAG_NO_ROUTED = 0x4
 MOE_FLAG_DEBUG_WAIT_TIMEOUT = 0x100
 
-KERNEL_NAMES = ("router", "permute", "shared_gate_up", "routed_gate_up", "routed_down",
-                "shared_down", "combine")
+KERNEL_NAMES = ("router", "permute", "gate_up", "down", "combine")
 
 
 class moe_config(ctypes.Structure):

@@ -157,14 +157,12 @@ moe_status moe_destroy(moe_handle h);
  * duration in milliseconds (total_ms[MOE_KERNEL_COUNT]) and launch count
  * (launches[MOE_KERNEL_COUNT]; either array may be NULL) and clears them. */
 typedef enum moe_kernel_id {
-  MOE_KERNEL_ROUTER = 0,              /* affinities, top-K, histogram, scan */
-  MOE_KERNEL_PERMUTE = 1,             /* expert-contiguous rows of x */
-  MOE_KERNEL_SHARED_GATE_UP = 2,      /* shared experts: SwiGLU(x W_gate^T, x W_up^T) */
-  MOE_KERNEL_ROUTED_GATE_UP = 3,      /* routed experts: the same, grouped by expert */
-  MOE_KERNEL_ROUTED_DOWN = 4,         /* routed experts: g * (H W_down^T) */
-  MOE_KERNEL_SHARED_DOWN = 5,         /* shared experts: Hs W_down^T */
-  MOE_KERNEL_COMBINE = 6,             /* h = x + shared + sum_k g * routed, k ascending */
-  MOE_KERNEL_COUNT = 7
+  MOE_KERNEL_ROUTER = 0,   /* affinities, top-K, histogram, scan */
+  MOE_KERNEL_PERMUTE = 1,  /* expert-contiguous rows of x */
+  MOE_KERNEL_GATE_UP = 2,  /* SwiGLU(x W_gate^T, x W_up^T): shared experts on x, routed ones grouped */
+  MOE_KERNEL_DOWN = 3,     /* shared experts: Hs W_down^T; routed experts: g * (H W_down^T) */
+  MOE_KERNEL_COMBINE = 4,  /* h = x + shared + sum_k g * routed, k ascending */
+  MOE_KERNEL_COUNT = 5
 } moe_kernel_id;
 moe_status moe_set_timing(moe_handle h, int enable);
 moe_status moe_kernel_times(moe_handle h, float* total_ms, int32_t* launches);
