@@ -34,6 +34,14 @@ SMALL = {
                         bias="uniform", seed=19),
     "small_softmax_n256": LS("small_softmax_n256", T=48, d=512, N=256, I=64, K=6, Ks=2, Is=64, sigma=0.03,
                              bias="normal", seed=20),
+    # T <= 32: 32-row gate/up and down tiles; T <= 64: 32-row down tiles (the
+    # zipf bias piles most tokens onto the first experts, so whole tiles fill)
+    "decode_t32": LS("decode_t32", T=32, d=208, N=24, I=160, K=4, Ks=2, Is=96, sigma=0.03, bias="zipf",
+                     seed=24),
+    "decode_t64": LS("decode_t64", T=64, d=320, N=16, I=144, K=6, Ks=1, Is=80, sigma=0.03, bias="zipf",
+                     seed=25),
+    "decode_t7_sigmoid": LS("decode_t7_sigmoid", T=7, d=256, N=20, I=96, K=3, Ks=1, Is=64, gate="sigmoid",
+                            sigma=0.03, bias="uniform", seed=26),
 }
 
 FLAGS_ROUTED = B.MOE_FLAG_NO_RESIDUAL | B.MOE_FLAG_NO_SHARED
