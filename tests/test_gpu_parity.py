@@ -200,6 +200,20 @@ def test_runs_are_bitwise_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("name", ["decode_t32", "16b_decode"])
+def test_small_batch_forwards_back_to_back(name):
+    """Twenty forwards queued without a synchronize in between give the same bits as one."""
+    shape = SMALL[name] if name in SMALL else W.CONFIGS[name]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    ref = H.run(layer, dev["x"], shape.K).clone()
+    out = torch.empty_like(ref)
+    for _ in range(20):
+        layer.forward(dev["x"], shape.K, out)
+    assert layer.status() == B.MOE_OK
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+
+
 def test_smaller_batches_reuse_one_handle():
     shape = SMALL["ragged"]
     host, dev = H.device_inputs(shape)
