@@ -156,10 +156,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
   const int G = a.num_groups;
-  for (int i = tid; i <= G; i += kGemmThreads) {
-    s_mts[i] = G ? a.mtile_start[i] : 0;
-    s_rows[i] = G ? a.row_start[i] : 0;
-  }
   const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGemmBM - 1) / kGemmBM * a.n_tiles : 0;
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
@@ -178,6 +174,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
     tmem_relinquish_pair();
+  }
+  pdl_wait();  // H, Hs and the router's tables are complete from here
+  pdl_launch_dependents();
+  for (int i = tid; i <= G; i += kGemmThreads) {
+    s_mts[i] = G ? a.mtile_start[i] : 0;
+    s_rows[i] = G ? a.row_start[i] : 0;
   }
   tc_fence_before_sync();
   cluster_sync();  // both CTAs' barriers exist before any copy or arrive targets them

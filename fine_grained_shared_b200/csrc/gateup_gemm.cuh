@@ -149,10 +149,6 @@ __global__ void __launch_bounds__(kGuThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int G = a.num_groups;
-  for (int i = tid; i <= G; i += kGuThreads) {
-    s_mts[i] = G ? a.mtile_start[i] : 0;
-    s_rows[i] = G ? a.row_start[i] : 0;
-  }
   const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGuBM - 1) / kGuBM * a.sh_n_tiles : 0;
   if (tid == 0) {
     for (int s = 0; s < kGuStages; ++s) {
@@ -175,6 +171,12 @@ __global__ void __launch_bounds__(kGuThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, kGuTmemCols);
     tmem_relinquish();
+  }
+  pdl_wait();  // the router's m-tile starts and the permuted rows are complete from here
+  pdl_launch_dependents();
+  for (int i = tid; i <= G; i += kGuThreads) {
+    s_mts[i] = G ? a.mtile_start[i] : 0;
+    s_rows[i] = G ? a.row_start[i] : 0;
   }
   tc_fence_before_sync();
   __syncthreads();

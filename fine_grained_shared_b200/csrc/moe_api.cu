@@ -10,7 +10,9 @@
 // Each GEMM launch covers the shared experts' tiles and the routed experts'
 // tiles in one persistent kernel, so the shared experts fill the SMs that a
 // small batch's routed tiles leave idle and the two never wait on each
-// other's tail.  Nothing is copied back to the host.
+// other's tail.  Batches of up to 512 tokens launch every kernel with
+// programmatic dependent launch, so each kernel's prologue overlaps the tail
+// of the one before.  Nothing is copied back to the host.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -19,6 +21,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "../../include/fgs_moe.h"
@@ -77,9 +80,8 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 
 struct Layout {
   // byte offsets into the workspace
-  size_t err, done, tile_ctr, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, mtile128, gate_perm, x_perm, h, y, hs, ys,
-      xdev,
-      outdev, total;
+  size_t err, done, tile_ctr, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, mtile128, gate_perm,
+      x_perm, h, y, hs, ys, xdev, outdev, total;
   int64_t P, Tpad, nblk;
 };
 
@@ -185,26 +187,61 @@ struct moe_ctx {
 
 namespace {
 
-template <int K>
-void launch_router_k(bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, const CUtensorMap& tx,
-                     const CUtensorMap& te, const RouterArgs& ra) {
-  if (sigmoid)
-    router_topk_kernel<K, true><<<grid, kRouterThreads, smem, s>>>(tx, te, ra);
-  else
-    router_topk_kernel<K, false><<<grid, kRouterThreads, smem, s>>>(tx, te, ra);
+// Batches up to this size launch every kernel of the forward with
+// programmatic stream serialization: a kernel may be scheduled while the one
+// before it drains, runs its prologue, and waits (griddepcontrol.wait) before
+// touching memory that another kernel writes.  Small forwards are bound by
+// launch and ramp latency and gain from the overlap (16B decode, T = 32:
+// 0.194 -> 0.185 ms); large ones run at the power cap, where it gained nothing
+// (16B prefill: 2.234 -> 2.264 ms), so they launch plainly.
+constexpr int64_t kPdlMaxT = 512;
+
+// cluster > 1 launches clusters of that many CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster,
+                       bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-void launch_router(int K, bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, const CUtensorMap& tx,
-                   const CUtensorMap& te, const RouterArgs& ra) {
+template <int K>
+cudaError_t launch_router_k(bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, bool pdl, const CUtensorMap& tx,
+                            const CUtensorMap& te, const RouterArgs& ra) {
+  return sigmoid ? launch_pdl(router_topk_kernel<K, true>, grid, dim3(kRouterThreads), smem, s, 1, pdl, tx, te, ra)
+                 : launch_pdl(router_topk_kernel<K, false>, grid, dim3(kRouterThreads), smem, s, 1, pdl, tx, te, ra);
+}
+
+cudaError_t launch_router(int K, bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, bool pdl,
+                          const CUtensorMap& tx, const CUtensorMap& te, const RouterArgs& ra) {
   switch (K) {
-    case 1: launch_router_k<1>(sigmoid, grid, smem, s, tx, te, ra); break;
-    case 2: launch_router_k<2>(sigmoid, grid, smem, s, tx, te, ra); break;
-    case 3: launch_router_k<3>(sigmoid, grid, smem, s, tx, te, ra); break;
-    case 4: launch_router_k<4>(sigmoid, grid, smem, s, tx, te, ra); break;
-    case 5: launch_router_k<5>(sigmoid, grid, smem, s, tx, te, ra); break;
-    case 6: launch_router_k<6>(sigmoid, grid, smem, s, tx, te, ra); break;
-    case 7: launch_router_k<7>(sigmoid, grid, smem, s, tx, te, ra); break;
-    default: launch_router_k<8>(sigmoid, grid, smem, s, tx, te, ra); break;
+    case 1: return launch_router_k<1>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    case 2: return launch_router_k<2>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    case 3: return launch_router_k<3>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    case 4: return launch_router_k<4>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    case 5: return launch_router_k<5>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    case 6: return launch_router_k<6>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    case 7: return launch_router_k<7>(sigmoid, grid, smem, s, pdl, tx, te, ra);
+    default: return launch_router_k<8>(sigmoid, grid, smem, s, pdl, tx, te, ra);
   }
 }
 
@@ -248,27 +285,17 @@ bool refresh(MapCache& c, const void* p, int64_t rows_key, uint64_t d2, uint64_t
 }
 
 // Launch `pairs` CTA pairs (clusters of 2) of the down GEMM kernel.
-cudaError_t launch_down(int pairs, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& B, const CUtensorMap& As,
-                        const CUtensorMap& Bs, const GemmArgs& ga) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs);
-  cfg.blockDim = dim3(kGemmThreads);
-  cfg.dynamicSmemBytes = gemm_smem_bytes();
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, down_gemm_kernel, A, B, As, Bs, ga);
+cudaError_t launch_down(int pairs, cudaStream_t s, bool pdl, const CUtensorMap& A, const CUtensorMap& B,
+                        const CUtensorMap& As, const CUtensorMap& Bs, const GemmArgs& ga) {
+  return launch_pdl(down_gemm_kernel, dim3(2 * pairs), dim3(kGemmThreads), gemm_smem_bytes(), s, 2, pdl, A, B, As, Bs,
+                    ga);
 }
 
-cudaError_t launch_gateup(int ctas, cudaStream_t s, const CUtensorMap& A, const CUtensorMap& G, const CUtensorMap& U,
-                          const CUtensorMap& As, const CUtensorMap& Gs, const CUtensorMap& Us, const GateUpArgs& ga) {
-  gateup_gemm_kernel<<<ctas, kGuThreads, gateup_smem_bytes(), s>>>(A, G, U, As, Gs, Us, ga);
-  return cudaGetLastError();
+cudaError_t launch_gateup(int ctas, cudaStream_t s, bool pdl, const CUtensorMap& A, const CUtensorMap& G,
+                          const CUtensorMap& U, const CUtensorMap& As, const CUtensorMap& Gs, const CUtensorMap& Us,
+                          const GateUpArgs& ga) {
+  return launch_pdl(gateup_gemm_kernel, dim3(ctas), dim3(kGuThreads), gateup_smem_bytes(), s, 1, pdl, A, G, U, As, Gs,
+                    Us, ga);
 }
 
 // Records a start/stop event pair around one launch when timing is enabled.
@@ -439,6 +466,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   }
   if (!ok) return MOE_ERR_CUDA;
 
+  const bool pdl = T <= kPdlMaxT;
   h->last_stream = s0;
   h->last_T = T;
   h->last_K = K;
@@ -471,12 +499,15 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
       // a few tokens: one CTA per token on the CUDA cores
       const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
       const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
-      if (sigmoid)
-        router_small_kernel<true><<<(int)T, kSmallRouterThreads, 0, s0>>>(xb, eb, (int)d, K, ra);
-      else
-        router_small_kernel<false><<<(int)T, kSmallRouterThreads, 0, s0>>>(xb, eb, (int)d, K, ra);
+      const dim3 grid((unsigned)T), block(kSmallRouterThreads);
+      const cudaError_t e =
+          sigmoid ? launch_pdl(router_small_kernel<true>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra)
+                  : launch_pdl(router_small_kernel<false>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra);
+      if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
-      launch_router(K, sigmoid, dim3(nblk), router_smem_bytes(Npad), s0, h->tm_x.map, h->tm_router.map, ra);
+      const size_t smem = router_smem_bytes(Npad);
+      if (launch_router(K, sigmoid, dim3(nblk), smem, s0, pdl, h->tm_x.map, h->tm_router.map, ra) != cudaSuccess)
+        return MOE_ERR_CUDA;
     }
   }
 
@@ -501,7 +532,9 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   pa.tile_ctr = h->at<int>(L.tile_ctr);
   {
     KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
-    permute_gather_kernel<<<dim3(nblk, do_routed ? pa.split : 1), kPermThreads, 0, s0>>>(pa);
+    const dim3 grid(nblk, do_routed ? pa.split : 1);
+    if (launch_pdl(permute_gather_kernel, grid, dim3(kPermThreads), 0, s0, 1, pdl, pa) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
 
   // ---- the expert GEMMs: shared experts' tiles first, then the routed experts' ----
@@ -539,7 +572,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     const CUtensorMap& sU = do_shared ? h->tm_swu.map : h->tm_wu.map;
     {
       KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
-      if (launch_gateup(ctas, s0, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g) != cudaSuccess)
+      if (launch_gateup(ctas, s0, pdl, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g) != cudaSuccess)
         return MOE_ERR_CUDA;
     }
 
@@ -569,7 +602,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     const CUtensorMap& sA2 = do_shared ? h->tm_hs : h->tm_h;
     const CUtensorMap& sB2 = do_shared ? h->tm_swd.map : h->tm_wd.map;
     KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
-    if (launch_down(pairs, s0, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
+    if (launch_down(pairs, s0, pdl, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
   // ---- the final sum ----
@@ -589,7 +622,8 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     // small batches: one warp per 256 columns of a row; large: one warp per row
     const int cols = T <= 4 * h->num_sms ? 256 : (int)d;
     const int64_t warps = T * ceil_div(d, cols);
-    combine_kernel<<<ceil_div(warps * 32, 256), 256, 0, s0>>>(ca, cols);
+    if (launch_pdl(combine_kernel, dim3(ceil_div(warps * 32, 256)), dim3(256), 0, s0, 1, pdl, ca, cols) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

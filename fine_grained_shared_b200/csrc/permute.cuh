@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(PermuteArg
   const int ntok = min(kPermBlockTokens, a.T - t0);
   const int K = a.K;
 
+  pdl_wait();  // the router's outputs are complete and visible from here
+  pdl_launch_dependents();
   if (b == 0 && blockIdx.y == 0 && tid < 2) a.tile_ctr[tid] = 0;
   for (int i = tid; i < a.N * 4; i += kPermThreads) masks[i] = 0u;
   for (int e = tid; e < a.N; e += kPermThreads) {
@@ -119,6 +121,9 @@ struct CombineArgs {
 // give a warp a whole row (it loops over the row); small batches split the
 // row over warps so that enough loads are in flight.
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a, int cols_per_warp) {
+  // no early launch of the next kernel: the next forward's router may start
+  // only when this forward has finished with every buffer it shares
+  pdl_wait();
   const int chunks = (a.d + cols_per_warp - 1) / cols_per_warp;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;

@@ -87,6 +87,12 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, a.tmem_cols);
+    tmem_relinquish();
+  }
+  pdl_wait();  // x, the biases and every output buffer belong to earlier kernels until here
+  pdl_launch_dependents();
   for (int i = tid; i < 256; i += kRouterThreads) {
     hist[i] = 0;
     float b = 0.f;
@@ -98,10 +104,6 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       }
     }
     bias[i] = b;
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, a.tmem_cols);
-    tmem_relinquish();
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -337,6 +339,8 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
   __shared__ int hist[2][256];
   const int t = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_launch_dependents();
   const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
   const int nvec = d >> 3;
   constexpr int kWarps = kSmallRouterThreads / 32;

@@ -285,4 +285,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream serialization attribute may start while the kernel before it in the
+// stream is still running; griddepcontrol.wait blocks until that kernel (and,
+// through its own wait, every kernel before it) has completed and its memory
+// is visible.  Each kernel of the layer runs only its prologue (barrier
+// initialisation, TMEM allocation, descriptor prefetch) before the wait and
+// touches no global memory there.  launch_dependents lets the next kernel be
+// scheduled early.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace fgs
