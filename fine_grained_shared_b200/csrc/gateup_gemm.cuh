@@ -25,12 +25,14 @@
 // the rows of x (one dense group whose H columns are the shared experts'
 // intermediate columns side by side), then the routed experts' tiles, whose
 // groups' m-tile starts come from the router on the device, so the host never
-// synchronises.  Tiles are handed out dynamically: the SMs of each of the
-// B200's two dies take tiles from their own half of the tile range (so the
+// synchronises.  The shared experts' tiles go round-robin over the CTAs and
+// need neither the router nor the permutation, so under programmatic
+// dependent launch they run while those kernels finish; the producer then
+// waits for them and takes routed tiles dynamically: the SMs of each of the
+// B200's two dies take tiles from their own half of the routed range (so the
 // two dies' L2 halves do not both fetch every expert's weights) and steal
-// from the other half when theirs runs out.  The producer fetches each tile
-// id and passes it to the MMA and epilogue warps through a 4-entry
-// shared-memory queue.
+// from the other half when theirs runs out.  The producer passes each tile id
+// to the MMA and epilogue warps through a 4-entry shared-memory queue.
 #pragma once
 
 #include "sm100.cuh"
@@ -66,7 +68,7 @@ struct GateUpArgs {
   int sh_ld_out;
   // both parts
   int num_kb;                  // 64-wide k-blocks over d
-  int* tile_ctr;               // [2] per-die tile counters, zero at launch; null: static order
+  int* tile_ctr;               // [2] per-die counters of the routed tiles, zeroed by the permutation
   int die_split;               // SMs with smid below this are on the first die
   uint32_t* err;
   uint64_t timeout_ns;
@@ -172,57 +174,24 @@ __global__ void __launch_bounds__(kGuThreads, 1)
     tmem_alloc(tmem_slot, kGuTmemCols);
     tmem_relinquish();
   }
-  pdl_wait();  // the router's m-tile starts and the permuted rows are complete from here
   pdl_launch_dependents();
-  for (int i = tid; i <= G; i += kGuThreads) {
-    s_mts[i] = G ? a.mtile_start[i] : 0;
-    s_rows[i] = G ? a.row_start[i] : 0;
-  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int total_tiles = sh_tiles + s_mts[G] * a.n_tiles;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
-    if (G) {
-      tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(&tmG);
-      tma_prefetch_desc(&tmU);
-    }
-    if (sh_tiles) {
-      tma_prefetch_desc(&tmAs);
-      tma_prefetch_desc(&tmGs);
-      tma_prefetch_desc(&tmUs);
-    }
-    int s = 0, issued = 0;
-    uint32_t ph = 0;
+    // lane 0 issues every copy and hands each tile id to the MMA and epilogue
+    // warps; the whole warp loads the routed experts' tables
+    int s = 0, issued = 0, q = 0;
+    uint32_t ph = 0, qph = 0;
     bool stop = false;
-    // dynamic schedule: each die owns half of the tiles; static: blockIdx.x + i * gridDim.x
-    const int half = total_tiles / 2;
-    const int die = static_cast<int>(sm_id()) >= a.die_split ? 1 : 0;
-    const int own_lo = die ? half : 0, own_hi = die ? total_tiles : half;
-    const int oth_lo = die ? 0 : half, oth_hi = die ? half : total_tiles;
-    int q = 0, next_static = blockIdx.x;
-    uint32_t qph = 0;
-    while (!stop) {
-      int tile = -1;
-      if (a.tile_ctr) {
-        const int t = own_lo + atomicAdd(&a.tile_ctr[die], 1);
-        if (t < own_hi) {
-          tile = t;
-        } else {  // this die's half is done: help the other die
-          const int u = oth_lo + atomicAdd(&a.tile_ctr[die ^ 1], 1);
-          if (u < oth_hi) tile = u;
-        }
-      } else {
-        tile = next_static < total_tiles ? next_static : -1;
-        next_static += gridDim.x;
-      }
+    auto publish = [&](int tile) {  // tile -1: no more tiles
       if (!mbar_wait(&tq_empty[q], qph ^ 1u, a.timeout_ns, abort_flag)) {
         gu_record_error(a.err, abort_flag, 8);
-        break;
+        stop = true;
+        return;
       }
       s_tq[q] = tile;
       mbar_arrive(&tq_full[q]);
@@ -230,7 +199,8 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         q = 0;
         qph ^= 1u;
       }
-      if (tile < 0) break;
+    };
+    auto load_tile = [&](int tile) {
       const GuTile c = gu_decode(tile, sh_tiles, a.sh_n_tiles, s_mts, s_rows, G, a.n_tiles);
       const int n0 = c.n_tile * (kGuBN / 2);
       const CUtensorMap* mA = c.shared ? &tmAs : &tmA;
@@ -240,7 +210,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         if (!mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag)) {
           gu_record_error(a.err, abort_flag, 3);
           stop = true;
-          break;
+          return;
         }
         mbar_arrive_expect_tx(&full[s], kGuStageA + kGuStageB);
         const int kc = kb * kGuBK;
@@ -253,11 +223,58 @@ __global__ void __launch_bounds__(kGuThreads, 1)
           ph ^= 1u;
         }
       }
+    };
+    if (lane == 0) {
+      if (G) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmG);
+        tma_prefetch_desc(&tmU);
+      }
+      if (sh_tiles) {
+        tma_prefetch_desc(&tmAs);
+        tma_prefetch_desc(&tmGs);
+        tma_prefetch_desc(&tmUs);
+      }
+      // the shared experts' tiles read only x and the shared weights, so they
+      // run while the router and the permutation may still be running
+      for (int tile = blockIdx.x; tile < sh_tiles && !stop; tile += gridDim.x) {
+        publish(tile);
+        if (!stop) load_tile(tile);
+      }
     }
-    for (int st = 0; st < kGuStages; ++st) {
-      if (issued > st) {
-        const int n = (issued - 1 - st) / kGuStages + 1;
-        mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+    // the routed experts' tiles need the router's tables, the permuted rows and
+    // the tile counters the permutation zeroed
+    pdl_wait();
+    for (int i = lane; i <= G; i += 32) {
+      s_mts[i] = G ? a.mtile_start[i] : 0;
+      s_rows[i] = G ? a.row_start[i] : 0;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      // each die owns half of the routed tiles and helps the other at the end
+      const int routed = s_mts[G] * a.n_tiles;
+      const int half = routed / 2;
+      const int die = static_cast<int>(sm_id()) >= a.die_split ? 1 : 0;
+      const int own_lo = sh_tiles + (die ? half : 0), own_hi = sh_tiles + (die ? routed : half);
+      const int oth_lo = sh_tiles + (die ? 0 : half), oth_hi = sh_tiles + (die ? half : routed);
+      while (!stop) {
+        int tile = -1;
+        const int t = own_lo + atomicAdd(&a.tile_ctr[die], 1);
+        if (t < own_hi) {
+          tile = t;
+        } else {  // this die's half is done: help the other die
+          const int u = oth_lo + atomicAdd(&a.tile_ctr[die ^ 1], 1);
+          if (u < oth_hi) tile = u;
+        }
+        publish(tile);
+        if (stop || tile < 0) break;
+        load_tile(tile);
+      }
+      for (int st = 0; st < kGuStages; ++st) {
+        if (issued > st) {
+          const int n = (issued - 1 - st) / kGuStages + 1;
+          mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+        }
       }
     }
   } else if (warp == 1 && lane == 0) {

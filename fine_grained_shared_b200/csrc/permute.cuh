@@ -45,8 +45,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_gather_kernel(PermuteArg
   const int ntok = min(kPermBlockTokens, a.T - t0);
   const int K = a.K;
 
-  pdl_wait();  // the router's outputs are complete and visible from here
-  pdl_launch_dependents();
+  pdl_launch_dependents();  // the gate/up kernel may start its shared experts' tiles
+  pdl_wait();               // the router's outputs are complete and visible from here
   if (b == 0 && blockIdx.y == 0 && tid < 2) a.tile_ctr[tid] = 0;
   for (int i = tid; i < a.N * 4; i += kPermThreads) masks[i] = 0u;
   for (int e = tid; e < a.N; e += kPermThreads) {
