@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -40,6 +41,9 @@ constexpr int kMaxRouted = 256;
 constexpr int kMaxK = 8;
 constexpr int64_t kMaxTokens = int64_t(1) << 20;
 constexpr uint64_t kTimeoutNs = 2000ull * 1000 * 1000;  // 2 s: no legitimate wait comes close
+// the host-buffer forward pipelines batches of at least 2 x kHostChunkRows tokens in up to kHostChunks chunks
+constexpr int kHostChunks = 4;
+constexpr int64_t kHostChunkRows = 2048;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -174,6 +178,9 @@ struct moe_ctx {
   // TMA descriptors: workspace ones are fixed, the others follow the caller's pointers
   CUtensorMap tm_xperm, tm_h, tm_hs;
   MapCache tm_x, tm_router, tm_wg, tm_wu, tm_wd, tm_swg, tm_swu, tm_swd;
+  // host-buffer forward: copy streams and per-chunk events, created on first use
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t host_start = nullptr, in_done[kHostChunks] = {}, fwd_done[kHostChunks] = {};
   // per-kernel timing: event pairs recorded around each launch while enabled
   bool timing = false;
   std::vector<cudaEvent_t> ev_pool[MOE_KERNEL_COUNT];
@@ -643,15 +650,63 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
   if (T == 0) return MOE_OK;
   DeviceGuard guard(h->device);
   cudaStream_t s0 = static_cast<cudaStream_t>(stream);
-  const size_t bytes = size_t(T) * h->cfg.d_model * 2;
-  void* xd = h->ws + h->L.xdev;
-  void* od = h->ws + h->L.outdev;
-  if (cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s0) != cudaSuccess) return MOE_ERR_CUDA;
-  const moe_status st = moe_forward(h, xd, T, router, experts, shared, K, od, stream);
-  if (st != MOE_OK) return st;
-  if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, s0) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaStreamSynchronize(s0) != cudaSuccess) return MOE_ERR_CUDA;
-  return MOE_OK;
+  const size_t row_bytes = size_t(h->cfg.d_model) * 2;
+  uint8_t* xd = h->ws + h->L.xdev;
+  uint8_t* od = h->ws + h->L.outdev;
+  const uint8_t* xh = static_cast<const uint8_t*>(x_host);
+  uint8_t* oh = static_cast<uint8_t*>(out_host);
+  // Tokens are independent, so a large batch runs as up to 4 chunks: chunk
+  // c + 1 is copied in and chunk c - 1 copied out on two copy streams while
+  // chunk c computes on `stream` (16B prefill, T = 16384: the 67 MB copies
+  // each way otherwise add their full time to the forward's).
+  const int chunks = static_cast<int>(std::min<int64_t>(kHostChunks, T / kHostChunkRows));
+  if (chunks <= 1) {
+    if (cudaMemcpyAsync(xd, xh, size_t(T) * row_bytes, cudaMemcpyHostToDevice, s0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    const moe_status st = moe_forward(h, xd, T, router, experts, shared, K, od, stream);
+    if (st != MOE_OK) return st;
+    if (cudaMemcpyAsync(oh, od, size_t(T) * row_bytes, cudaMemcpyDeviceToHost, s0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return cudaStreamSynchronize(s0) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  if (!h->copy_in) {
+    bool ok = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->host_start, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; c < kHostChunks && ok; ++c)
+      ok = cudaEventCreateWithFlags(&h->in_done[c], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->fwd_done[c], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return MOE_ERR_CUDA;
+  }
+  // finish everything in flight on all three streams before returning, also on an error
+  auto finish = [&](moe_status st) {
+    const bool ok = cudaStreamSynchronize(h->copy_in) == cudaSuccess &&
+                    cudaStreamSynchronize(s0) == cudaSuccess && cudaStreamSynchronize(h->copy_out) == cudaSuccess;
+    return st != MOE_OK ? st : ok ? MOE_OK : MOE_ERR_CUDA;
+  };
+  // the copies in start after the work already queued on `stream`
+  if (cudaEventRecord(h->host_start, s0) != cudaSuccess ||
+      cudaStreamWaitEvent(h->copy_in, h->host_start, 0) != cudaSuccess)
+    return finish(MOE_ERR_CUDA);
+  auto rows_of = [&](int c) { return T * c / chunks; };
+  for (int c = 0; c < chunks; ++c) {
+    const size_t off = size_t(rows_of(c)) * row_bytes, n = size_t(rows_of(c + 1) - rows_of(c)) * row_bytes;
+    if (cudaMemcpyAsync(xd + off, xh + off, n, cudaMemcpyHostToDevice, h->copy_in) != cudaSuccess ||
+        cudaEventRecord(h->in_done[c], h->copy_in) != cudaSuccess)
+      return finish(MOE_ERR_CUDA);
+  }
+  for (int c = 0; c < chunks; ++c) {
+    const size_t off = size_t(rows_of(c)) * row_bytes, n = size_t(rows_of(c + 1) - rows_of(c)) * row_bytes;
+    if (cudaStreamWaitEvent(s0, h->in_done[c], 0) != cudaSuccess) return finish(MOE_ERR_CUDA);
+    const moe_status st =
+        moe_forward(h, xd + off, rows_of(c + 1) - rows_of(c), router, experts, shared, K, od + off, stream);
+    if (st != MOE_OK) return finish(st);
+    if (cudaEventRecord(h->fwd_done[c], s0) != cudaSuccess ||
+        cudaStreamWaitEvent(h->copy_out, h->fwd_done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(oh + off, od + off, n, cudaMemcpyDeviceToHost, h->copy_out) != cudaSuccess)
+      return finish(MOE_ERR_CUDA);
+  }
+  return finish(MOE_OK);
 }
 
 moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts, int32_t* offsets,
@@ -724,6 +779,13 @@ moe_status moe_destroy(moe_handle h) {
     cudaDeviceSynchronize();
     for (auto& pool : h->ev_pool)
       for (cudaEvent_t e : pool) cudaEventDestroy(e);
+    if (h->copy_in) cudaStreamDestroy(h->copy_in);
+    if (h->copy_out) cudaStreamDestroy(h->copy_out);
+    if (h->host_start) cudaEventDestroy(h->host_start);
+    for (int c = 0; c < kHostChunks; ++c) {
+      if (h->in_done[c]) cudaEventDestroy(h->in_done[c]);
+      if (h->fwd_done[c]) cudaEventDestroy(h->fwd_done[c]);
+    }
     if (h->ws) cudaFree(h->ws);
   }
   delete h;

@@ -129,9 +129,14 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
 
 /* The same forward for callers whose activations live in host memory:
  * x_host: bf16 [T, d] host; out_host: bf16 [T, d] host (pinned memory makes
- * the copies asynchronous to other host work).  Copies x to the device,
- * runs moe_forward on `stream`, copies the result back and synchronizes the
- * stream before returning.  The weights stay device pointers. */
+ * the copies asynchronous to other host work and lets them overlap the
+ * compute).  Copies x to the device, runs moe_forward on `stream`, copies the
+ * result back and returns when out_host holds it.  Batches of 4096 tokens or
+ * more run as up to 4 chunks of whole tokens whose copies in and out overlap
+ * the other chunks' compute (on two copy streams the handle owns); the
+ * output is bit-identical to one moe_forward over the whole batch, and
+ * moe_get_routing afterwards returns the last chunk's routing.  The weights
+ * stay device pointers. */
 moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
                             const moe_experts* experts, const moe_shared* shared, int32_t K,
                             void* out_host, void* stream);

@@ -233,8 +233,11 @@ def test_smaller_batches_reuse_one_handle():
     H.compare_output(_gpu_rows(out, rows), h[rows], "K=2 on a K=3 handle")
 
 
-def test_host_buffer_entry_point_matches_device_entry_point():
-    shape = W.CONFIGS["tiny"]
+@pytest.mark.parametrize("T", [512, 4096, 9000])  # one chunk; 2 chunks; 4 uneven chunks
+def test_host_buffer_entry_point_matches_device_entry_point(T):
+    """The host-buffer forward (copies pipelined with token chunks for large T)
+    gives the device forward's bits: tokens are independent."""
+    shape = W.CONFIGS["tiny"].with_(T=T)
     host, dev = H.device_inputs(shape)
     layer = H.make_layer(shape, dev)
     dev_out = H.run(layer, dev["x"], shape.K).cpu()
