@@ -42,7 +42,7 @@ constexpr int kMaxK = 8;
 constexpr int64_t kMaxTokens = int64_t(1) << 20;
 constexpr uint64_t kTimeoutNs = 2000ull * 1000 * 1000;  // 2 s: no legitimate wait comes close
 // the host-buffer forward pipelines batches of at least 2 x kHostChunkRows tokens in up to kHostChunks chunks
-constexpr int kHostChunks = 4;
+constexpr int kHostChunks = 5;
 constexpr int64_t kHostChunkRows = 2048;
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -655,12 +655,14 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
   uint8_t* od = h->ws + h->L.outdev;
   const uint8_t* xh = static_cast<const uint8_t*>(x_host);
   uint8_t* oh = static_cast<uint8_t*>(out_host);
-  // Tokens are independent, so a large batch runs as up to 4 chunks: chunk
-  // c + 1 is copied in and chunk c - 1 copied out on two copy streams while
-  // chunk c computes on `stream` (16B prefill, T = 16384: the 67 MB copies
-  // each way otherwise add their full time to the forward's).
-  const int chunks = static_cast<int>(std::min<int64_t>(kHostChunks, T / kHostChunkRows));
-  if (chunks <= 1) {
+  // Tokens are independent, so a large batch runs in chunks: chunk c + 1 is
+  // copied in and chunk c - 1 copied out on two copy streams while chunk c
+  // computes on `stream` (16B prefill, T = 16384: the 67 MB copies each way
+  // otherwise add their full time to the forward's).  The first and last
+  // chunks are small (T/16) so that little copying is left exposed before the
+  // first kernel and after the last; the middle chunks share the rest.
+  const int middle = static_cast<int>(std::min<int64_t>(kHostChunks - 2, T / kHostChunkRows));
+  if (middle <= 1) {
     if (cudaMemcpyAsync(xd, xh, size_t(T) * row_bytes, cudaMemcpyHostToDevice, s0) != cudaSuccess)
       return MOE_ERR_CUDA;
     const moe_status st = moe_forward(h, xd, T, router, experts, shared, K, od, stream);
@@ -688,7 +690,14 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
   if (cudaEventRecord(h->host_start, s0) != cudaSuccess ||
       cudaStreamWaitEvent(h->copy_in, h->host_start, 0) != cudaSuccess)
     return finish(MOE_ERR_CUDA);
-  auto rows_of = [&](int c) { return T * c / chunks; };
+  const int chunks = middle + 2;
+  const int64_t edge = T / 16;
+  auto rows_of = [&](int c) -> int64_t {  // first row of chunk c (c == chunks: T)
+    if (c <= 0) return 0;
+    if (c >= chunks) return T;
+    if (c == chunks - 1) return T - edge;
+    return edge + (T - 2 * edge) * (c - 1) / middle;
+  };
   for (int c = 0; c < chunks; ++c) {
     const size_t off = size_t(rows_of(c)) * row_bytes, n = size_t(rows_of(c + 1) - rows_of(c)) * row_bytes;
     if (cudaMemcpyAsync(xd + off, xh + off, n, cudaMemcpyHostToDevice, h->copy_in) != cudaSuccess ||

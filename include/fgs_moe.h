@@ -132,8 +132,9 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
  * the copies asynchronous to other host work and lets them overlap the
  * compute).  Copies x to the device, runs moe_forward on `stream`, copies the
  * result back and returns when out_host holds it.  Batches of 4096 tokens or
- * more run as up to 4 chunks of whole tokens whose copies in and out overlap
- * the other chunks' compute (on two copy streams the handle owns); the
+ * more run as up to 5 chunks of whole tokens (the first and last T/16) whose
+ * copies in and out overlap the other chunks' compute (on two copy streams
+ * the handle owns); the
  * output is bit-identical to one moe_forward over the whole batch, and
  * moe_get_routing afterwards returns the last chunk's routing.  The weights
  * stay device pointers. */
