@@ -215,30 +215,60 @@ def run_reference(args):
 # the GPU arm
 # ---------------------------------------------------------------------------
 
+class Ranks:
+    """One process per GPU, launched by torchrun: rank and world size from its
+    environment, and a process group for the barrier and the max-over-ranks
+    time only (the layer has no exchange step; every rank runs a full replica).
+    NCCL on GPUs; the tests run the same code over gloo on CPU."""
+
+    def __init__(self, backend: str = "nccl", device=None, timeout_s: float = 120.0):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.device = device if device is not None else torch.device("cpu")
+        self.dist = None
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"timeout": datetime.timedelta(seconds=timeout_s)}
+            if backend == "nccl":
+                kw["device_id"] = self.device
+            dist.init_process_group(backend, **kw)
+            self.dist = dist
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        """The largest of the ranks' values (every rank gets it)."""
+        if self.dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def aggregate_rate(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest rank's time."""
+    return world * units_per_rank / (max_ms * 1e-3)
+
+
 def run_ours(args):
     from fine_grained_shared_b200 import moe as B
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     shape = W.CONFIGS[args.config]
     host = host_inputs(shape)
@@ -280,7 +310,7 @@ def run_ours(args):
         raise B.MoEError(st, "timed region")
     ms_total = max_over_ranks(start.elapsed_time(end))
     ms_step = ms_total / args.steps
-    value = world * shape.T / (ms_step * 1e-3)
+    value = aggregate_rate(shape.T, world, ms_step)
 
     # ---- end to end through the host-buffer entry point ----
     x_h = host["x"].pin_memory()
@@ -298,7 +328,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
-    e2e_value = world * shape.T / (e2e_ms * 1e-3)
+    e2e_value = aggregate_rate(shape.T, world, e2e_ms)
 
     # ---- roofline of the dominant kernel (shared + routed gate/up GEMM + SwiGLU) ----
     peaks, peak_src = measured_peaks()
@@ -337,9 +367,7 @@ def run_ours(args):
     layer.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def main():

@@ -1,0 +1,63 @@
+"""The benchmark's multi-rank plumbing on CPU: two gloo ranks, as torchrun
+would launch them, agree on the slowest rank's time, pass the barrier and
+report whole-job throughput; under the reference arm only rank 0 works."""
+import contextlib
+import io
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, results):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world)})
+    ranks = bench.Ranks("gloo", timeout_s=60)
+    assert (ranks.rank, ranks.world) == (rank, world)
+    ranks.barrier()
+    slowest = ranks.max(10.0 + rank)  # rank r took 10 + r ms
+    results[rank] = (slowest, bench.aggregate_rate(1000, ranks.world, slowest))
+    ranks.close()
+
+
+def test_two_gloo_ranks_agree_on_the_slowest_time():
+    world, port = 2, _free_port()
+    results = mp.Manager().dict()
+    mp.start_processes(_rank_main, args=(world, port, results), nprocs=world, start_method="spawn", join=True)
+    assert sorted(results.keys()) == [0, 1]
+    for r in range(world):
+        slowest, rate = results[r]
+        assert slowest == pytest.approx(11.0)
+        # 2 replicas x 1000 tokens in the slowest rank's 11 ms
+        assert rate == pytest.approx(2000 / 11e-3)
+
+
+def test_single_process_needs_no_process_group():
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        os.environ.pop(k, None)
+    ranks = bench.Ranks("gloo")
+    assert ranks.world == 1 and ranks.dist is None
+    assert ranks.max(3.5) == 3.5
+    ranks.barrier()
+    ranks.close()
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+                                      "--warmup", "1"])
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.main()
+    assert out.getvalue() == ""
