@@ -7,7 +7,7 @@ input generators in ``workloads`` serve both.
 """
 from .moe_oracle import (  # noqa: F401
     GATE_SIGMOID, GATE_SOFTMAX, FLAG_NO_RESIDUAL, FLAG_NO_ROUTED, FLAG_NO_SHARED,
-    Permutation, Routing, affinity_logits, expert_permutation, f64, gate_values,
+    Permutation, Routing, affinity_logits, bias_update, expert_permutation, f64, gate_values,
     moe_forward, route, select_top_k, sigmoid_affinity, silu, softmax_affinity,
     swiglu_ffn,
 )

@@ -259,3 +259,26 @@ def moe_forward(u, router_w, K: int, experts, shared=None, *,
         for k in range(K):                     # gate-weighted sum, k ascending
             h += y[:, k]
     return h, routing
+
+
+def bias_update(bias, counts, gamma: float) -> np.ndarray:
+    """One auxiliary-loss-free balancing step of the per-expert selection biases.
+
+    DeepSeek-V3 technical report summary, section 2 "Auxiliary-Loss-Free Load
+    Balancing": after each training step every expert's bias moves according
+    to whether the expert was overloaded or underloaded.  The pages give no
+    formula; the reading taken is the plainest one: with load_i the number of
+    (token, slot) pairs routed to expert i in the step and mean = sum(load)/mN,
+    b_i <- b_i + gamma * sign(mean - load_i) -- an overloaded expert's bias
+    drops by gamma, an underloaded one's rises by gamma, an expert exactly at
+    the mean keeps its bias.  The comparison is made on integers
+    (load_i * mN against sum(load)), so no rounding decides a sign.  The
+    biases are float32 (they are a float32 input of the layer); the float64
+    sum of two float32 values rounded once to float32 is the float32 sum.
+    """
+    counts = np.asarray(counts, dtype=np.int64)
+    N = counts.size
+    total = int(counts.sum())
+    sign = np.sign(total - counts * N).astype(np.float64)  # sign(mean - load) with mean = total / N
+    b = np.asarray(bias, dtype=np.float32).astype(np.float64)
+    return (b + np.float64(np.float32(gamma)) * sign).astype(np.float32)

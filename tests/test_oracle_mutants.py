@@ -12,7 +12,7 @@ import tests.test_oracle_pins as P
 
 _orig = {name: getattr(M, name) for name in
          ("silu", "softmax_affinity", "sigmoid_affinity", "select_top_k", "gate_values",
-          "swiglu_ffn", "affinity_logits", "expert_permutation", "moe_forward")}
+          "swiglu_ffn", "affinity_logits", "expert_permutation", "moe_forward", "bias_update")}
 
 
 def _silu_wrong_sign(a):
@@ -77,6 +77,10 @@ def _forward_drops_shared(u, router_w, K, experts, shared=None, **kw):
     return _orig["moe_forward"](u, router_w, K, experts, None, **kw)
 
 
+def _bias_update_wrong_sign(bias, counts, gamma):
+    return _orig["bias_update"](bias, counts, -gamma)
+
+
 MUTANTS = {
     "silu_wrong_sign": ("silu", _silu_wrong_sign),
     "softmax_wrong_normaliser": ("softmax_affinity", _softmax_no_shift_renorm_topk),
@@ -90,6 +94,7 @@ MUTANTS = {
     "permutation_not_stable": ("expert_permutation", _permutation_descending),
     "residual_dropped": ("moe_forward", _forward_drops_residual),
     "shared_dropped": ("moe_forward", _forward_drops_shared),
+    "bias_update_wrong_sign": ("bias_update", _bias_update_wrong_sign),
 }
 
 PINS = [
@@ -106,6 +111,8 @@ PINS = [
     P.test_dense_counterpart_when_all_experts_active,
     lambda: P.test_gshard_reduction_matches_brute_force(0),
     lambda: P.test_permutation_matches_sorted_pairs(7, 3),
+    P.test_bias_update_hand_example,
+    P.test_bias_update_balances_a_skewed_router,
 ]
 
 

@@ -395,3 +395,48 @@ def test_workload_shapes_match_the_pages():
     assert 0.85 * s2b["total_params"] <= p2b <= 1.0 * s2b["total_params"]
     p16 = s16["moe_layers"] * (c3.N + c3.Ks) * 3 * c3.d * c3.I
     assert 0.85 * s16["total_params"] <= p16 <= 1.0 * s16["total_params"]
+
+
+# ---------------------------------------------------------------------------
+# auxiliary-loss-free bias update (DeepSeek-V3 summary, section 2)
+# ---------------------------------------------------------------------------
+
+def test_bias_update_hand_example():
+    # loads 5, 1, 3, 3 (mean 3): the overloaded expert drops, the underloaded rises, the rest stay
+    b = np.array([0.25, -0.5, 0.125, 0.0], dtype=np.float32)
+    got = O.bias_update(b, [5, 1, 3, 3], 0.0625)
+    assert got.dtype == np.float32
+    np.testing.assert_array_equal(got, np.array([0.1875, -0.4375, 0.125, 0.0], dtype=np.float32))
+
+
+def test_bias_update_compares_against_a_fractional_mean_exactly():
+    # loads 2 and 1: mean 1.5 lies between them; equal loads leave every bias alone
+    np.testing.assert_array_equal(O.bias_update(np.zeros(2, np.float32), [2, 1], 1.0), [-1.0, 1.0])
+    np.testing.assert_array_equal(O.bias_update(np.full(6, 0.3, np.float32), [7] * 6, 0.5),
+                                  np.full(6, 0.3, np.float32))
+
+
+def test_bias_update_balances_a_skewed_router():
+    """Routing with the updated biases spreads the load: the property the update exists for."""
+    rng = np.random.default_rng(31)
+    T, d, N, K = 512, 32, 8, 2
+    u = rng.standard_normal((T, d))
+    e = rng.standard_normal((N, d)) * 0.05
+    e[0] += 0.8 * u.mean(axis=0) / np.linalg.norm(u.mean(axis=0))  # experts 0 and 1 favoured
+    e[1] += 0.6 * u.mean(axis=0) / np.linalg.norm(u.mean(axis=0))
+    u += u.mean(axis=0)
+
+    def max_violation(b):
+        r = O.route(u, e, K, "sigmoid", select_bias=b)
+        load = np.bincount(r.idx.ravel(), minlength=N)
+        return (load.max() - load.mean()) / load.mean(), load
+
+    b = np.zeros(N, np.float32)
+    v0, load0 = max_violation(b)
+    for _ in range(300):
+        _, load = max_violation(b)
+        b = O.bias_update(b, load, 0.002)
+    v1, _ = max_violation(b)
+    assert v0 > 1.0, v0            # the skew is real
+    assert v1 < 0.2 * v0, (v0, v1)
+    assert b[0] < 0 and b[1] < 0   # the favoured experts were pushed down
