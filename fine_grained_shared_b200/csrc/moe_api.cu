@@ -18,6 +18,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -736,6 +737,15 @@ moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* cou
   cp(offsets, L.offsets, (N + 1) * 4);
   cp(src, L.src, tk * 4);
   return ok ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_update_bias(moe_handle h, float* bias, float gamma, void* stream) {
+  if (!h || !bias || (reinterpret_cast<uintptr_t>(bias) & 3u) || !std::isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+  if (h->last_T <= 0) return MOE_ERR_INVALID_ARG;  // no loads to balance yet
+  DeviceGuard guard(h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bias_update_kernel<<<1, kBiasThreads, 0, s>>>(bias, h->at<int32_t>(h->L.counts), h->cfg.n_routed, gamma);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe_status moe_status_query(moe_handle h) {

@@ -484,4 +484,34 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Auxiliary-loss-free load balancing (DeepSeek-V3 technical report summary,
+// section 2): after a step, every expert's selection bias moves by gamma
+// according to whether the expert was overloaded or underloaded.  With the
+// step's per-expert loads (the router's counts): b_i += gamma * sign(mean -
+// load_i), the comparison made on integers (load_i * N against the total).
+// One thread per expert; the total comes from a block reduction.
+// ---------------------------------------------------------------------------
+constexpr int kBiasThreads = 256;
+
+static __global__ void __launch_bounds__(kBiasThreads)
+    bias_update_kernel(float* __restrict__ bias, const int32_t* __restrict__ counts, int N, float gamma) {
+  __shared__ long long part[kBiasThreads / 32];
+  const int tid = threadIdx.x;
+  long long sum = 0;
+  for (int i = tid; i < N; i += kBiasThreads) sum += counts[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if ((tid & 31) == 0) part[tid >> 5] = sum;
+  __syncthreads();
+  long long total = 0;
+#pragma unroll
+  for (int w = 0; w < kBiasThreads / 32; ++w) total += part[w];
+  for (int i = tid; i < N; i += kBiasThreads) {
+    const long long scaled = static_cast<long long>(counts[i]) * N;  // load_i * N vs total = mean * N
+    const float step = scaled < total ? gamma : scaled > total ? -gamma : 0.f;
+    bias[i] = bias[i] + step;
+  }
+}
+
 }  // namespace fgs

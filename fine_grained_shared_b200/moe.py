@@ -82,10 +82,12 @@ def lib() -> ctypes.CDLL:
     L.moe_kernel_times.argtypes = [moe_handle, c_void_p, c_void_p]
     L.moe_route_noalloc.argtypes = [c_void_p, c_int64, c_int32, POINTER(moe_router), c_int32, c_int32, c_int32,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
+    L.moe_update_bias.argtypes = [moe_handle, c_void_p, ctypes.c_float, c_void_p]
     L.moe_status_string.argtypes = [c_int]
     L.moe_status_string.restype = c_char_p
     for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_get_routing",
-                 "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc"):
+                 "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc",
+                 "moe_update_bias"):
         getattr(L, name).restype = c_int
     _lib = L
     return L
@@ -136,6 +138,11 @@ def moe_route_noalloc(x, T, d_model, router, n_routed, gate, K, idx, gate_out, c
     """Routing with the library's fixed device scratch (no allocation); see the header."""
     return lib().moe_route_noalloc(x, int(T), int(d_model), ctypes.byref(router), int(n_routed), int(gate),
                                    int(K), idx, gate_out, counts, offsets, err, stream)
+
+
+def moe_update_bias(h, bias, gamma, stream):
+    """One auxiliary-loss-free update of float32 [mN] device biases from the last forward's loads."""
+    return lib().moe_update_bias(h, bias, float(gamma), stream)
 
 
 def moe_set_timing(h, enable):
@@ -214,6 +221,14 @@ class MoELayer:
         if st != MOE_OK:
             raise MoEError(st, "moe_forward_host")
         return out_host
+
+    def update_bias(self, bias, gamma, stream=None):
+        """bias: float32 [mN] CUDA tensor (normally the router's select_bias), updated in place
+        from the last forward's per-expert loads."""
+        st = moe_update_bias(self.h, _ptr(bias), gamma, _stream_ptr(stream))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_update_bias")
+        return bias
 
     def routing(self, T, K, stream=None):
         import torch

@@ -150,6 +150,22 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
 moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts,
                            int32_t* offsets, int32_t* src, void* stream);
 
+/* Auxiliary-loss-free load balancing: one update of the per-expert selection
+ * biases from the last forward's per-expert loads (DeepSeek-V3 technical
+ * report summary, section 2 "Auxiliary-Loss-Free Load Balancing": after each
+ * step a bias moves according to whether its expert was overloaded or
+ * underloaded).  With load_i the (token, slot) pairs routed to expert i by the
+ * last moe_forward on this handle and mean = sum(load) / mN:
+ *   bias[i] += gamma * sign(mean - load_i)
+ * (an overloaded expert's bias drops, an underloaded one's rises, an expert at
+ * exactly the mean keeps its bias; the comparison is exact, on integers).
+ * bias: float32 [mN] device, 4-byte aligned, updated in place -- normally the
+ * moe_router select_bias of a MOE_GATE_SIGMOID_BIASED layer; gamma: the
+ * update speed, finite.  Stream-ordered on `stream` after the forward whose
+ * loads it reads; asynchronous.  MOE_ERR_INVALID_ARG for a NULL handle or
+ * bias, a misaligned bias, a non-finite gamma, or no forward yet. */
+moe_status moe_update_bias(moe_handle h, float* bias, float gamma, void* stream);
+
 /* Synchronize the stream of the last forward and report (then clear) any
  * error the kernels recorded: MOE_ERR_TIMEOUT if a device-side wait ran out. */
 moe_status moe_status_query(moe_handle h);

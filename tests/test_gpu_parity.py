@@ -5,6 +5,7 @@ are compared on their whole routing and on a seeded sample of tokens (tokens
 are independent, so a sampled row of the oracle equals that row of the full
 layer).  Rules in ``tests/harness.py``.
 """
+import ctypes
 import numpy as np
 import pytest
 import torch
@@ -296,3 +297,61 @@ def test_device_wait_timeout_is_reported_and_the_context_stays_usable():
                          H.oracle_shared(shape, host), routing=ref)
     rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
     H.compare_output(_gpu_rows(out, rows), h[rows], "after a timeout")
+
+
+# ---------------------------------------------------------------------------
+# auxiliary-loss-free bias update
+# ---------------------------------------------------------------------------
+
+def test_bias_update_matches_the_oracle_bit_for_bit():
+    shape = SMALL["sigmoid"]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    bias = dev["select_bias"].clone()
+    with pytest.raises(B.MoEError):
+        layer.update_bias(bias, 0.01)          # no forward yet: no loads to balance
+    H.run(layer, dev["x"], shape.K)
+    _, _, counts, _, _ = layer.routing(shape.T, shape.K)
+    counts = counts.cpu().numpy()
+    for gamma in (0.01, 1e-3):
+        before = bias.cpu().numpy()
+        layer.update_bias(bias, gamma)
+        torch.cuda.synchronize()
+        want = O.bias_update(before, counts, gamma)
+        np.testing.assert_array_equal(bias.cpu().numpy(), want)
+    with pytest.raises(B.MoEError):
+        layer.update_bias(bias, float("nan"))
+    raw = torch.zeros(4 * shape.N + 4, dtype=torch.uint8, device="cuda")
+    assert B.moe_update_bias(layer.h, ctypes.c_void_p(raw.data_ptr() + 2), 0.1, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_bias_update_balances_a_skewed_layer_on_the_gpu():
+    """Forward, update, repeat: the routed load evens out (the reason for the update)."""
+    shape = LS("skewed", T=2048, d=256, N=16, I=64, K=2, Ks=1, Is=64, gate="sigmoid", sigma=0.05,
+               bias="uniform", seed=41)
+    host = W.layer_inputs(shape)
+    mean_dir = host["x"].float().mean(dim=0)
+    mean_dir = mean_dir / mean_dir.norm()
+    router = host["router"].float()
+    router[0] += 0.6 * mean_dir
+    router[1] += 0.4 * mean_dir
+    host["router"] = router.to(torch.bfloat16)
+    host["x"] = (host["x"].float() + 3.0 * mean_dir).to(torch.bfloat16)
+    _, dev = H.device_inputs(shape, host)
+    layer = H.make_layer(shape, dev)
+    bias = torch.zeros(shape.N, dtype=torch.float32, device="cuda")
+    layer.set_weights(dev["router"], (dev["w_gate"], dev["w_up"], dev["w_down"]),
+                      (dev["ws_gate"], dev["ws_up"], dev["ws_down"]), select_bias=bias)
+
+    def max_violation():
+        H.run(layer, dev["x"], shape.K)
+        c = layer.routing(shape.T, shape.K)[2].cpu().numpy()
+        return (c.max() - c.mean()) / c.mean()
+
+    v0 = max_violation()
+    for _ in range(150):
+        max_violation()
+        layer.update_bias(bias, 0.002)
+    v1 = max_violation()
+    assert v0 > 1.0, v0
+    assert v1 < 0.3 * v0, (v0, v1)
