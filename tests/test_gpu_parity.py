@@ -43,6 +43,8 @@ SMALL = {
                      seed=25),
     "decode_t7_sigmoid": LS("decode_t7_sigmoid", T=7, d=256, N=20, I=96, K=3, Ks=1, Is=64, gate="sigmoid",
                             sigma=0.03, bias="uniform", seed=26),
+    # the smallest sizes the ABI accepts: one 16-column k-block, K = N, a single m- and n-tile
+    "minimal": LS("minimal", T=5, d=16, N=4, I=16, K=4, Ks=1, Is=16, sigma=0.3, seed=27),
 }
 
 FLAGS_ROUTED = B.MOE_FLAG_NO_RESIDUAL | B.MOE_FLAG_NO_SHARED
@@ -355,3 +357,29 @@ def test_bias_update_balances_a_skewed_layer_on_the_gpu():
     v1 = max_violation()
     assert v0 > 1.0, v0
     assert v1 < 0.3 * v0, (v0, v1)
+
+
+# ---------------------------------------------------------------------------
+# seeded random shapes: every size the ABI accepts at small scale
+# ---------------------------------------------------------------------------
+
+def _random_shape(seed: int) -> W.LayerShape:
+    rng = np.random.default_rng(1000 + seed)
+    N = int(rng.choice([1, 2, 3, 5, 8, 13, 24, 40, 64, 100]))
+    K = int(rng.integers(1, min(8, N) + 1))
+    Ks = int(rng.integers(0, 3))
+    gate = "sigmoid" if rng.random() < 0.4 else "softmax"
+    bias = ("uniform" if rng.random() < 0.7 else "none") if gate == "sigmoid" else \
+        str(rng.choice(["none", "normal", "zipf"]))
+    return LS(f"random{seed}", T=int(rng.integers(1, 700)), d=16 * int(rng.integers(1, 33)),
+              N=N, I=16 * int(rng.integers(1, 21)), K=K, Ks=Ks, Is=16 * int(rng.integers(1, 17)) if Ks else 0,
+              gate=gate, sigma=0.02, bias=bias, seed=5000 + seed)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_shapes_every_token(seed):
+    shape = _random_shape(seed)
+    host, dev = H.device_inputs(shape)
+    ref = H.oracle_routing(shape, host)
+    rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
+    _check_layer(shape, host, dev, rows, ref)
