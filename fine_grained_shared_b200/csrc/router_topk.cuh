@@ -19,7 +19,15 @@
 namespace fgs {
 
 constexpr int kRouterThreads = 192;
-constexpr int kRouterStages = 4;
+// Pipeline depth: the ring holds kRouterMaxStages stages when they fit in
+// about 200 KB of shared memory (mN <= 128), else 4.  The router is bound by
+// the latency of its copies (measured: 16B prefill, 4 stages, DRAM 18% busy),
+// so depth is what speeds it up; 6 stages x 2 copies stay within the 12 bulk
+// copies in flight per CTA that every kernel here keeps to.
+constexpr int kRouterMaxStages = 6;
+__host__ __device__ constexpr int router_stages(int Npad) {
+  return (16384 + Npad * 128) * kRouterMaxStages <= 200 * 1024 ? kRouterMaxStages : 4;
+}
 constexpr int kRouterBM = 128;
 constexpr int kBK = 64;  // bf16 elements per 128-byte swizzle row
 // Every expert's rows start on a multiple of this in the permuted row space,
@@ -45,8 +53,8 @@ struct RouterArgs {
 };
 
 __host__ __device__ constexpr size_t router_smem_bytes(int Npad) {
-  return 1024 + static_cast<size_t>(kRouterStages) * (16384 + static_cast<size_t>(Npad) * 128) +
-         8 * (2 * kRouterStages + 2) + 16 + 4 * (256 + 256 + 256) + 64;
+  return 1024 + static_cast<size_t>(router_stages(Npad)) * (16384 + static_cast<size_t>(Npad) * 128) +
+         8 * (2 * kRouterMaxStages + 2) + 16 + 4 * (256 + 256 + 256) + 64;
 }
 
 __device__ __forceinline__ void record_error(uint32_t* err, volatile int* abort, uint32_t site) {
@@ -62,10 +70,11 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int Bbytes = a.Npad * 128;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + kRouterStages * 16384;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kRouterStages * Bbytes);
-  uint64_t* empty = full + kRouterStages;
-  uint64_t* acc_full = empty + kRouterStages;
+  const int S = router_stages(a.Npad);
+  uint8_t* sB = smem + S * 16384;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * Bbytes);
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;
   uint64_t* teardown = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -78,7 +87,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   const int m0 = blockIdx.x * kRouterBM;
 
   if (tid == 0) {
-    for (int s = 0; s < kRouterStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -125,15 +134,15 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       tma_load_2d(sA + s * 16384, &tm_x, &full[s], kb * kBK, m0);
       tma_load_2d(sB + s * Bbytes, &tm_e, &full[s], kb * kBK, 0);
       ++issued;
-      if (++s == kRouterStages) {
+      if (++s == S) {
         s = 0;
         ph ^= 1u;
       }
     }
     // make sure no copy is still landing in shared memory when the CTA exits
-    for (int st = 0; st < kRouterStages; ++st) {
+    for (int st = 0; st < S; ++st) {
       if (issued > st) {
-        const int n = (issued - 1 - st) / kRouterStages + 1;
+        const int n = (issued - 1 - st) / S + 1;
         mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
       }
     }
@@ -156,7 +165,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       for (int kk = 0; kk < 4; ++kk)
         umma_bf16_ss(tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
       umma_commit(&empty[s]);
-      if (++s == kRouterStages) {
+      if (++s == S) {
         s = 0;
         ph ^= 1u;
       }
