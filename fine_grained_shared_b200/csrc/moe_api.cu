@@ -85,8 +85,8 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 
 struct Layout {
   // byte offsets into the workspace
-  size_t err, done, tile_ctr, idx, gate, slot, src, bc, counts, offsets, row_start, mtile, mtile128, gate_perm,
-      x_perm, h, y, hs, ys, xdev, outdev, total;
+  size_t err, done, tile_ctr, tok_done, small_logits, idx, gate, slot, src, bc, counts, offsets, row_start, mtile,
+      mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, total;
   int64_t P, Tpad, nblk;
 };
 
@@ -106,6 +106,8 @@ Layout make_layout(const moe_config& c) {
   L.err = take(16);
   L.done = take(16);
   L.tile_ctr = take(16);
+  L.tok_done = take(kSmallRouterMaxT * 4);  // zeroed with the header block at creation
+  L.small_logits = take(size_t(kSmallRouterMaxT) * N * 4);
   L.idx = take(Tm * Km * 4);
   L.gate = take(Tm * Km * 4);
   L.slot = take(Tm * Km * 4);
@@ -507,10 +509,11 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
       // a few tokens: one CTA per token on the CUDA cores
       const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
       const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
-      const dim3 grid((unsigned)T), block(kSmallRouterThreads);
+      SmallRouterArgs sa{h->at<float>(L.small_logits), h->at<uint32_t>(L.tok_done)};
+      const dim3 grid((unsigned)T, (unsigned)ceil_div(N, kSmallRouterGroup)), block(kSmallRouterThreads);
       const cudaError_t e =
-          sigmoid ? launch_pdl(router_small_kernel<true>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra)
-                  : launch_pdl(router_small_kernel<false>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra);
+          sigmoid ? launch_pdl(router_small_kernel<true>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra, sa)
+                  : launch_pdl(router_small_kernel<false>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra, sa);
       if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
       const size_t smem = router_smem_bytes(Npad);

@@ -322,87 +322,102 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 namespace fgs {
 
 // ---------------------------------------------------------------------------
-// Small batches (T <= kSmallRouterMaxT): one CTA per token on the CUDA cores.
-// The tensor-core router gives a 128-token block to one CTA, so a decode
-// batch of a few dozen tokens would run on a single SM walking d serially.
-// Here each warp computes the logits of kSmallRouterBatch experts at once as
-// dot products (16-byte loads of x and of the experts' rows in flight
-// together, warp reduction), then warp 0 picks the top K by K rounds of a
-// warp argmax ordered by (key descending, index ascending).  The last CTA to
-// finish counts the selected experts of every 128-token block from the
-// written indices (shared-memory integer atomics: exact, and no buffer needs
-// clearing between calls) and runs the same scan as the tensor-core router.
+// Small batches (T <= kSmallRouterMaxT) on the CUDA cores.  The tensor-core
+// router gives a 128-token block to one CTA, so a decode batch of a few dozen
+// tokens would run on a single SM walking d serially.  Here the grid is
+// (token, group of kSmallRouterGroup experts): each warp computes one
+// expert's logit as a dot product, every lane issuing its loads for a whole
+// 2048-column pass at once (instead of one CTA pulling all mN experts' rows
+// through its lanes: 16B decode, T = 32, 25 -> 17 us), and writes it to a
+// per-token row of logits.  The last of a token's CTAs to finish (a
+// per-token counter) picks that token's top K by K rounds of a warp argmax
+// ordered by (key descending, index ascending); the last token to be
+// finished counts the selected experts of every 128-token block from the
+// written indices (shared-memory integer atomics: exact) and runs the same
+// scan as the tensor-core router.  Both counters are reset by their last
+// arriver, so no buffer needs clearing between calls.
 // ---------------------------------------------------------------------------
 constexpr int kSmallRouterMaxT = 256;
 constexpr int kSmallRouterThreads = 256;
-constexpr int kSmallRouterBatch = 8;  // experts one warp reduces together
+constexpr int kSmallRouterGroup = 8;   // experts per CTA: one per warp
+static_assert(kSmallRouterThreads / 32 == kSmallRouterGroup, "one warp per expert of the group");
+constexpr int kSmallRouterPass = 8;    // 16-byte vectors per lane per pass (2048 columns)
+
+struct SmallRouterArgs {
+  float* logits;          // [T, N] fp32 scratch
+  uint32_t* token_done;   // [T] CTAs finished per token, zero between calls
+};
 
 template <bool SIGMOID>
 __global__ void __launch_bounds__(kSmallRouterThreads)
     router_small_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ e, int d, int K,
-                        RouterArgs a) {
+                        RouterArgs a, SmallRouterArgs sa) {
   static_assert(kSmallRouterMaxT <= 2 * 128, "the last CTA's histogram holds two 128-token blocks");
   __shared__ float key[256], sval[256];
   __shared__ int is_last;
   __shared__ int scan_tmp[256];
   __shared__ int hist[2][256];
-  const int t = blockIdx.x;
+  const int t = blockIdx.x, grp = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_wait();
   pdl_launch_dependents();
-  const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
-  const int nvec = d >> 3;
-  constexpr int kWarps = kSmallRouterThreads / 32;
-  for (int i0 = warp * kSmallRouterBatch; i0 < a.N; i0 += kWarps * kSmallRouterBatch) {
-    const uint4* er[kSmallRouterBatch];
-    float acc[kSmallRouterBatch];
+  // ---- the logit of this warp's expert ----
+  {
+    const uint4* xr = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * d);
+    const int nvec = d >> 3;
+    const int i = grp * kSmallRouterGroup + warp;
+    if (i < a.N) {
+      const uint4* er = reinterpret_cast<const uint4*>(e + static_cast<size_t>(i) * d);
+      float acc = 0.f;
+      for (int c0 = 0; c0 < nvec; c0 += 32 * kSmallRouterPass) {
+        uint4 xv[kSmallRouterPass], ev[kSmallRouterPass];
+        // all 2 x kSmallRouterPass loads issue before any arithmetic; a column
+        // past the row reads column 0 of the same rows and is zeroed in x
 #pragma unroll
-    for (int q = 0; q < kSmallRouterBatch; ++q) {
-      const int i = i0 + q < a.N ? i0 + q : a.N - 1;  // past the end: re-read the last row, result unused
-      er[q] = reinterpret_cast<const uint4*>(e + static_cast<size_t>(i) * d);
-      acc[q] = 0.f;
-    }
-#pragma unroll 2
-    for (int c = lane; c < nvec; c += 32) {
-      const uint4 xv = __ldg(xr + c);
-      uint4 ev[kSmallRouterBatch];
+        for (int j = 0; j < kSmallRouterPass; ++j) {
+          const int c = c0 + lane + 32 * j;
+          const int cc = c < nvec ? c : 0;
+          xv[j] = ldg_v4_ordered(xr + cc);
+          ev[j] = ldg_v4_ordered(er + cc);
+        }
 #pragma unroll
-      for (int q = 0; q < kSmallRouterBatch; ++q) ev[q] = __ldg(er[q] + c);
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float xl[4] = {bf16lo(xw[0]), bf16lo(xw[1]), bf16lo(xw[2]), bf16lo(xw[3])};
-      const float xh[4] = {bf16hi(xw[0]), bf16hi(xw[1]), bf16hi(xw[2]), bf16hi(xw[3])};
+        for (int j = 0; j < kSmallRouterPass; ++j) {
+          if (c0 + lane + 32 * j >= nvec) xv[j] = make_uint4(0, 0, 0, 0);
+          const uint32_t xw[4] = {xv[j].x, xv[j].y, xv[j].z, xv[j].w};
+          const uint32_t w[4] = {ev[j].x, ev[j].y, ev[j].z, ev[j].w};
 #pragma unroll
-      for (int q = 0; q < kSmallRouterBatch; ++q) {
-        const uint32_t ew[4] = {ev[q].x, ev[q].y, ev[q].z, ev[q].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[q] = fmaf(xl[j], bf16lo(ew[j]), acc[q]);
-          acc[q] = fmaf(xh[j], bf16hi(ew[j]), acc[q]);
+          for (int q = 0; q < 4; ++q) {
+            acc = fmaf(bf16lo(xw[q]), bf16lo(w[q]), acc);
+            acc = fmaf(bf16hi(xw[q]), bf16hi(w[q]), acc);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int q = 0; q < kSmallRouterBatch; ++q) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xffffffffu, acc[q], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int q = 0; q < kSmallRouterBatch; ++q) {
-        const int i = i0 + q;
-        if (i >= a.N) break;
-        if (SIGMOID) {
-          const float sv = 1.f / (1.f + __expf(-acc[q]));
-          sval[i] = sv;
-          key[i] = sv + (a.select_bias ? a.select_bias[i] : 0.f);
-        } else {
-          key[i] = acc[q] + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
-        }
-      }
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (lane == 0) sa.logits[static_cast<size_t>(t) * a.N + i] = acc;
     }
   }
+  // ---- the last of the token's CTAs picks its top K ----
+  __threadfence();
   __syncthreads();
+  if (tid == 0) is_last = (atomicAdd(sa.token_done + t, 1u) == gridDim.y - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  if (tid == 0) sa.token_done[t] = 0u;  // every CTA of this token has counted itself
   if (warp == 0) {
+    const float* lrow = sa.logits + static_cast<size_t>(t) * a.N;
+    for (int i = lane; i < a.N; i += 32) {
+      const float z = __ldcg(lrow + i);
+      if (SIGMOID) {
+        const float sv = 1.f / (1.f + __expf(-z));
+        sval[i] = sv;
+        key[i] = sv + (a.select_bias ? a.select_bias[i] : 0.f);
+      } else {
+        key[i] = z + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
+      }
+    }
+    __syncwarp();
     // softmax statistics over all N logits (softmax mode)
     float mx = -INFINITY, sum = 0.f;
     if (!SIGMOID) {
