@@ -298,14 +298,4 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// A 16-byte read-only global load that the compiler keeps in program order
-// with the other such loads, so a batch of them is in flight together.
-__device__ __forceinline__ uint4 ldg_v4_ordered(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 }  // namespace fgs
