@@ -41,7 +41,9 @@ UNIT = "tokens/s"
 L2_BYTES = 126 * 2**20
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT = "gate_up"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt")
+# committed ncu summaries of the dominant kernel, per workload: DRAM bytes per token (prefill) or per launch
+PROFILE_SUMMARIES = {"16b_prefill": os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt"),
+                     "16b_decode": os.path.join(ROOT, "profiles", "gemms_16b_decode.txt")}
 KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/gateup_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
 
 
@@ -88,22 +90,31 @@ def kernel_source_hash() -> str:
 
 def profiled_traffic(shape: W.LayerShape):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
-    if not os.path.exists(PROFILE_SUMMARY):
+    summary of this workload, if it was taken on the current kernel source; else None."""
+    path = PROFILE_SUMMARIES.get(shape.name)
+    if path is None or not os.path.exists(path):
         return None
     vals = {}
-    with open(PROFILE_SUMMARY) as f:
+    with open(path) as f:
         for line in f:
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
-                vals[k.strip()] = v.strip()
+                vals.setdefault(k.strip(), v.strip())  # the first kernel listed is the dominant one
     if vals.get("source_sha256_16") != kernel_source_hash():
         return None
     try:
-        per_token = float(vals["traffic_bytes_per_token"])
+        if "traffic_bytes_per_token" in vals:
+            return float(vals["traffic_bytes_per_token"]) * shape.T
+        return float(vals["traffic_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
-    return per_token * shape.T
+
+
+def gate_up_weight_bytes(shape: W.LayerShape, counts) -> float:
+    """Weights one gate/up launch must stream: W_gate and W_up of every routed
+    expert that received a token, and of the shared experts."""
+    touched = int(sum(1 for c in counts if c > 0))
+    return 2.0 * 2 * shape.d * (touched * shape.I + shape.Ks * shape.Is)
 
 
 # ---------------------------------------------------------------------------
@@ -292,7 +303,9 @@ def run_ours(args):
     # ---- device-resident timing ----
     clocks = ClockSampler(local)
     time.sleep(0.3)
-    layer.set_timing(True)
+    # CUDA events around the dominant kernel only: events around every launch would add their own
+    # cost to the step time (a separate pass below times every kernel)
+    layer.set_timing(True, kernels=[DOMINANT])
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
@@ -308,9 +321,20 @@ def run_ours(args):
     st = layer.status()
     if st != B.MOE_OK:
         raise B.MoEError(st, "timed region")
+    # every kernel's time, and the launches of one forward, from a short pass outside the timed region
+    pass_steps = max(1, min(args.steps, 50))
+    layer.set_timing(True)
+    for _ in range(pass_steps):
+        layer.forward(x, shape.K, out)
+    all_ktimes = layer.kernel_times()
+    layer.set_timing(False)
+    launches_per_forward = sum(n for _, n in all_ktimes.values()) / pass_steps
     ms_total = max_over_ranks(start.elapsed_time(end))
     ms_step = ms_total / args.steps
     value = aggregate_rate(shape.T, world, ms_step)
+
+    # per-expert loads of the timed forwards (before the chunked host-buffer forwards overwrite them)
+    counts = layer.routing(shape.T, shape.K)[2].cpu().tolist()
 
     # ---- end to end through the host-buffer entry point ----
     x_h = host["x"].pin_memory()
@@ -331,14 +355,27 @@ def run_ours(args):
     e2e_value = aggregate_rate(shape.T, world, e2e_ms)
 
     # ---- roofline of the dominant kernel (shared + routed gate/up GEMM + SwiGLU) ----
+    # bound: tensor when the routed experts' FLOPs per weight byte exceed the measured ridge
+    # (sustained bf16 FLOP/s over copy bandwidth), else HBM (the weight-streaming regime)
     peaks, peak_src = measured_peaks()
     k_ms, k_n = ktimes[DOMINANT]
     k_avg_ms = max_over_ranks(k_ms / max(1, k_n))
     k_flop = 4.0 * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is)
-    achieved = k_flop / (k_avg_ms * 1e-3) / 1e12
-    peak = float(peaks["bf16_tflops_sustained"])
+    peak_flops = float(peaks["bf16_tflops_sustained"])
+    k_bytes = gate_up_weight_bytes(shape, counts)
+    if k_flop / k_bytes > peak_flops * 1e12 / (float(peaks["hbm_gbs"]) * 1e9):
+        roofline = {"bound": "tensor", "achieved": k_flop / (k_avg_ms * 1e-3) / 1e12, "peak": peak_flops,
+                    "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    else:
+        roofline = {"bound": "hbm", "achieved": k_bytes / (k_avg_ms * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
+                    "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
+    roofline["frac"] = roofline["achieved"] / roofline["peak"]
+    roofline.update({"traffic": profiled_traffic(shape),
+                     "kernel": "gateup_gemm_kernel (shared and routed experts: gate/up GEMM + SwiGLU)",
+                     "flop_per_launch": k_flop, "weight_bytes_per_launch": k_bytes, "avg_launch_ms": k_avg_ms})
+    peak = peak_flops
     layer_tflops = world * layer_flop(shape) / (ms_step * 1e-3) / 1e12
-    launches = sum(n for _, n in ktimes.values())
+    launches = int(round(launches_per_forward * args.steps))
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -347,12 +384,8 @@ def run_ours(args):
         "config": workload_config(shape, f"replicas{world}" if world > 1 else "single"),
         "tflops": layer_tflops,
         "tflops_frac_of_peak": layer_tflops / (world * peak),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": profiled_traffic(shape),
-                     "kernel": "gateup_gemm_kernel (shared and routed experts: gate/up GEMM + SwiGLU)",
-                     "peak_source": f"{peak_src} bf16_tflops_sustained",
-                     "flop_per_launch": k_flop, "avg_launch_ms": k_avg_ms},
-        "kernel_ms_per_step": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in ktimes.items()},
+        "roofline": roofline,
+        "kernel_ms_per_step": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in all_ktimes.items()},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_h.numel() * 2),
                 "d2h_bytes_per_step": int(out_h.numel() * 2), "ms_per_step": e2e_ms},
         "gpu_launches": launches,

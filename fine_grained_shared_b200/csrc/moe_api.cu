@@ -185,7 +185,7 @@ struct moe_ctx {
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
   cudaEvent_t host_start = nullptr, in_done[kHostChunks] = {}, fwd_done[kHostChunks] = {};
   // per-kernel timing: event pairs recorded around each launch while enabled
-  bool timing = false;
+  uint32_t timing_mask = 0;  // bit k: time kernel k
   std::vector<cudaEvent_t> ev_pool[MOE_KERNEL_COUNT];
   size_t ev_used[MOE_KERNEL_COUNT] = {};
 
@@ -312,7 +312,7 @@ cudaError_t launch_gateup(int ctas, cudaStream_t s, bool pdl, const CUtensorMap&
 class KernelTimer {
  public:
   KernelTimer(moe_ctx* h, int id, cudaStream_t s) : h_(h), id_(id), s_(s) {
-    if (!h_->timing) return;
+    if (!((h_->timing_mask >> id_) & 1u)) return;
     auto& pool = h_->ev_pool[id_];
     size_t& used = h_->ev_used[id_];
     while (pool.size() < used + 2) {
@@ -769,9 +769,9 @@ moe_status moe_status_query(moe_handle h) {
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-moe_status moe_set_timing(moe_handle h, int enable) {
-  if (!h) return MOE_ERR_INVALID_ARG;
-  h->timing = enable != 0;
+moe_status moe_set_timing(moe_handle h, uint32_t kernel_mask) {
+  if (!h || (kernel_mask & ~MOE_TIMING_ALL)) return MOE_ERR_INVALID_ARG;
+  h->timing_mask = kernel_mask;
   return MOE_OK;
 }
 

@@ -78,7 +78,7 @@ def lib() -> ctypes.CDLL:
     L.moe_get_routing.argtypes = [moe_handle, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.moe_status_query.argtypes = [moe_handle]
     L.moe_destroy.argtypes = [moe_handle]
-    L.moe_set_timing.argtypes = [moe_handle, c_int]
+    L.moe_set_timing.argtypes = [moe_handle, ctypes.c_uint32]
     L.moe_kernel_times.argtypes = [moe_handle, c_void_p, c_void_p]
     L.moe_route_noalloc.argtypes = [c_void_p, c_int64, c_int32, POINTER(moe_router), c_int32, c_int32, c_int32,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
@@ -145,8 +145,9 @@ def moe_update_bias(h, bias, gamma, stream):
     return lib().moe_update_bias(h, bias, float(gamma), stream)
 
 
-def moe_set_timing(h, enable):
-    return lib().moe_set_timing(h, int(bool(enable)))
+def moe_set_timing(h, kernel_mask):
+    """kernel_mask: bit k times kernel KERNEL_NAMES[k]; 0 turns timing off."""
+    return lib().moe_set_timing(h, int(kernel_mask))
 
 
 def moe_kernel_times(h):
@@ -248,8 +249,15 @@ class MoELayer:
     def status(self):
         return moe_status_query(self.h)
 
-    def set_timing(self, enable):
-        st = moe_set_timing(self.h, enable)
+    def set_timing(self, enable=True, kernels=None):
+        """Per-kernel CUDA-event timing: of every kernel, or of the named ones (KERNEL_NAMES)."""
+        if not enable:
+            mask = 0
+        elif kernels is None:
+            mask = (1 << len(KERNEL_NAMES)) - 1
+        else:
+            mask = sum(1 << KERNEL_NAMES.index(k) for k in kernels)
+        st = moe_set_timing(self.h, mask)
         if st != MOE_OK:
             raise MoEError(st, "moe_set_timing")
 

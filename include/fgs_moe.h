@@ -173,11 +173,14 @@ moe_status moe_status_query(moe_handle h);
 /* Free the workspace and the handle (synchronizes first).  NULL is a no-op. */
 moe_status moe_destroy(moe_handle h);
 
-/* Per-kernel timing.  While enabled, moe_forward records a CUDA event pair
- * around each kernel it launches, on the stream that kernel runs on.
- * moe_kernel_times synchronizes those events, writes each kernel's summed
- * duration in milliseconds (total_ms[MOE_KERNEL_COUNT]) and launch count
- * (launches[MOE_KERNEL_COUNT]; either array may be NULL) and clears them. */
+/* Per-kernel timing.  moe_set_timing(h, kernel_mask): bit k of kernel_mask
+ * (k a moe_kernel_id) makes moe_forward record a CUDA event pair around each
+ * launch of kernel k, on its stream; 0 turns timing off; MOE_TIMING_ALL times
+ * every kernel.  Event records add a few microseconds per launch, so time only
+ * the kernels you need in a timed loop.  moe_kernel_times synchronizes those
+ * events, writes each kernel's summed duration in milliseconds
+ * (total_ms[MOE_KERNEL_COUNT]) and launch count (launches[MOE_KERNEL_COUNT];
+ * either array may be NULL) and clears them. */
 typedef enum moe_kernel_id {
   MOE_KERNEL_ROUTER = 0,   /* affinities, top-K, histogram, scan */
   MOE_KERNEL_PERMUTE = 1,  /* expert-contiguous rows of x */
@@ -186,7 +189,8 @@ typedef enum moe_kernel_id {
   MOE_KERNEL_COMBINE = 4,  /* h = x + shared + sum_k g * routed, k ascending */
   MOE_KERNEL_COUNT = 5
 } moe_kernel_id;
-moe_status moe_set_timing(moe_handle h, int enable);
+#define MOE_TIMING_ALL ((1u << MOE_KERNEL_COUNT) - 1u)
+moe_status moe_set_timing(moe_handle h, uint32_t kernel_mask);
 moe_status moe_kernel_times(moe_handle h, float* total_ms, int32_t* launches);
 
 /* Routing without any device allocation (the pages have no counterpart: this

@@ -85,6 +85,7 @@ def test_null_handles():
         B.MOE_ERR_INVALID_ARG
     assert lib.moe_get_routing(None, None, None, None, None, None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_update_bias(None, None, 0.001, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_timing(None, 1) == B.MOE_ERR_INVALID_ARG
 
 
 def test_status_strings():

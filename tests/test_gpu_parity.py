@@ -383,3 +383,23 @@ def test_random_shapes_every_token(seed):
     ref = H.oracle_routing(shape, host)
     rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
     _check_layer(shape, host, dev, rows, ref)
+
+
+def test_timing_records_only_the_kernels_asked_for():
+    shape = SMALL["tiny"]
+    host, dev = H.device_inputs(shape)
+    layer = H.make_layer(shape, dev)
+    layer.set_timing(True, kernels=["gate_up"])
+    for _ in range(3):
+        H.run(layer, dev["x"], shape.K)
+    t = layer.kernel_times()
+    assert t["gate_up"][1] == 3 and t["gate_up"][0] > 0
+    assert all(n == 0 for k, (_, n) in t.items() if k != "gate_up")
+    layer.set_timing(True)
+    H.run(layer, dev["x"], shape.K)
+    assert all(n == 1 for _, n in layer.kernel_times().values())
+    layer.set_timing(False)
+    H.run(layer, dev["x"], shape.K)
+    assert all(n == 0 for _, n in layer.kernel_times().values())
+    assert B.moe_set_timing(layer.h, 1 << len(B.KERNEL_NAMES)) == B.MOE_ERR_INVALID_ARG
+
