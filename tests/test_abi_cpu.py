@@ -91,3 +91,43 @@ def test_null_handles():
 def test_status_strings():
     for v, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (7, "MOE_ERR_TIMEOUT"), (99, "MOE_ERR_UNKNOWN")]:
         assert B.status_string(v) == name
+
+
+def test_header_compiles_as_plain_c_and_links(tmp_path):
+    """A C99 program includes the header, links the library and calls the two
+    entry points that need no GPU."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "fgs_moe.h"
+int main(void) {
+  moe_config c;
+  uint64_t bytes = 0;
+  memset(&c, 0, sizeof c);
+  c.d_model = 2048; c.n_routed = 64; c.d_ff = 1408; c.n_shared = 2; c.d_ff_shared = 1408;
+  c.max_tokens = 16384; c.max_k = 6; c.gate = MOE_GATE_SOFTMAX; c.flags = 0;
+  if (moe_workspace_bytes(&c, &bytes) != MOE_OK || bytes == 0) return 1;
+  if (strcmp(moe_status_string(MOE_ERR_SHAPE), "MOE_ERR_SHAPE") != 0) return 2;
+  printf("%llu\n", (unsigned long long)bytes);
+  return 0;
+}
+''')
+    lib_dir = os.path.dirname(B.LIB_PATH)
+    exe = tmp_path / "abi"
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", str(src), "-I", os.path.join(ROOT, "include"),
+                        "-L", lib_dir, "-lfgs_moe", "-Wl,-rpath," + lib_dir, "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stderr)
+    cfg = B.moe_config(d_model=2048, n_routed=64, d_ff=1408, n_shared=2, d_ff_shared=1408, max_tokens=16384,
+                       max_k=6, gate=B.MOE_GATE_SOFTMAX, flags=0)
+    want = ctypes.c_uint64()
+    assert B.lib().moe_workspace_bytes(ctypes.byref(cfg), ctypes.byref(want)) == B.MOE_OK
+    assert int(r.stdout.strip()) == want.value
