@@ -86,6 +86,9 @@ def test_null_handles():
     assert lib.moe_get_routing(None, None, None, None, None, None, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_update_bias(None, None, 0.001, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_set_timing(None, 1) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host(None, None, 1, ctypes.byref(r), ctypes.byref(e), None, 1, None, None) == \
+        B.MOE_ERR_INVALID_ARG
+    assert lib.moe_kernel_times(None, None, None) == B.MOE_ERR_INVALID_ARG
 
 
 def test_status_strings():
