@@ -1,6 +1,6 @@
 // permute.cuh -- step 3 of the layer: group the (token, slot) pairs by expert
-// and gather the token rows into expert-contiguous order; plus the plain
-// combine used when no shared-expert GEMM carries the final sum.
+// and gather the token rows into expert-contiguous order; and the combine
+// that forms the layer's output from the expert GEMMs' rows.
 //
 // The expert-parallel dispatch of the DeepSeek-V3 technical report (section
 // 3.2.1, all-to-all dispatch and combine) sends each token to the experts

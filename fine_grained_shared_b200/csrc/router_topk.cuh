@@ -1,6 +1,8 @@
 // router_topk.cuh -- step 1 and 2 of the layer: affinity logits on the
 // tensor cores, softmax or sigmoid, top-K in registers, per-block expert
-// histogram and (in the last CTA to finish) the expert-offset scan.
+// histogram and (in the last CTA to finish) the expert-offset scan; the same
+// steps on the CUDA cores for small batches; and the auxiliary-loss-free
+// update of the selection biases from the per-expert counts.
 //
 // DeepSeekMoE (arXiv 2401.06066), Abstract: each token activates mK of the mN
 // fine-grained routed experts.  DeepSeek-V3 technical report, section 2
@@ -20,10 +22,9 @@ namespace fgs {
 
 constexpr int kRouterThreads = 192;
 // Pipeline depth: the ring holds kRouterMaxStages stages when they fit in
-// about 200 KB of shared memory (mN <= 128), else 4.  The router is bound by
-// the latency of its copies (measured: 16B prefill, 4 stages, DRAM 18% busy),
-// so depth is what speeds it up; 6 stages x 2 copies stay within the 12 bulk
-// copies in flight per CTA that every kernel here keeps to.
+// about 200 KB of shared memory (mN <= 128), else 4.  6 stages x 2 copies stay
+// within the 12 bulk copies in flight per CTA that every kernel here keeps
+// to (measured on the 16B prefill layer: 0.064 ms against 0.065 with 4).
 constexpr int kRouterMaxStages = 6;
 __host__ __device__ constexpr int router_stages(int Npad) {
   return (16384 + Npad * 128) * kRouterMaxStages <= 200 * 1024 ? kRouterMaxStages : 4;
