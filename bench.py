@@ -64,8 +64,19 @@ def workload_config(shape: W.LayerShape, parallelism: str) -> dict:
             "n_routed": shape.N, "d_ff": shape.I, "top_k": shape.K, "n_shared": shape.Ks,
             "d_ff_shared": shape.Is, "gate": shape.gate, "bias": shape.bias,
             "global_batch": shape.T, "parallelism": parallelism,
-            "l2": "no flush: every step streams its >1 GB working set (1.14 GB of expert weights) "
-                  "through the 126 MB L2"}
+            "l2": l2_note(shape)}
+
+
+def l2_note(shape: W.LayerShape) -> str:
+    gb = expert_weight_gb(shape)
+    if gb * 1e9 > L2_BYTES:
+        return (f"no flush: the expert weights a step reads (up to {gb:.2f} GB, the touched experts') "
+                f"exceed the 126 MB L2")
+    return f"no flush: the layer's {gb * 1e3:.1f} MB of weights fit in the 126 MB L2, so steps run L2-warm"
+
+
+def expert_weight_gb(shape: W.LayerShape) -> float:
+    return 3.0 * 2 * shape.d * (shape.N * shape.I + shape.Ks * shape.Is) / 1e9
 
 
 def layer_flop(shape: W.LayerShape) -> float:
