@@ -220,7 +220,7 @@ def _as_expert_fn(w_gate, w_up, w_down) -> ExpertFn:
 def moe_forward(u, router_w, K: int, experts, shared=None, *,
                 gate_kind: str = GATE_SOFTMAX, logit_bias=None, select_bias=None,
                 flags: int = 0, rows: Optional[np.ndarray] = None,
-                routing: Optional[Routing] = None):
+                routing: Optional[Routing] = None, ffn: Optional[Callable] = None):
     """h_t for the tokens ``rows`` (all tokens when None) -> (h [n, d], Routing).
 
     ``experts`` is either a tuple (W_gate [N,I,d], W_up [N,I,d], W_down [N,d,I])
@@ -229,6 +229,7 @@ def moe_forward(u, router_w, K: int, experts, shared=None, *,
     ``flags`` leaves out terms of the sum (residual, shared, routed) so that
     each term can be checked on its own.  Tokens are independent, so the
     output of a subset of rows equals those rows of the full output.
+    ``ffn`` replaces ``swiglu_ffn`` for every expert (the FP8 variant).
     """
     u_all = f64(u)
     if rows is None:
@@ -241,6 +242,8 @@ def moe_forward(u, router_w, K: int, experts, shared=None, *,
     else:
         idx, gate = routing.idx[rows], routing.gate[rows]
     expert_fn = experts if callable(experts) else _as_expert_fn(*experts)
+    if ffn is None:
+        ffn = swiglu_ffn
 
     n, d = ur.shape
     h = np.zeros((n, d), dtype=np.float64)
@@ -249,13 +252,13 @@ def moe_forward(u, router_w, K: int, experts, shared=None, *,
     if shared is not None and not flags & FLAG_NO_SHARED:
         ws_gate, ws_up, ws_down = shared
         for j in range(len(ws_gate)):          # every shared expert, gate 1
-            h += swiglu_ffn(ur, ws_gate[j], ws_up[j], ws_down[j])
+            h += ffn(ur, ws_gate[j], ws_up[j], ws_down[j])
     if not flags & FLAG_NO_ROUTED:
         y = np.zeros((n, K, d), dtype=np.float64)
         for e in np.unique(idx):               # FFN_e on the tokens that chose e
             r, k = np.nonzero(idx == e)
             wg, wu, wd = expert_fn(int(e))
-            y[r, k] = gate[r, k][:, None] * swiglu_ffn(ur[r], wg, wu, wd)
+            y[r, k] = gate[r, k][:, None] * ffn(ur[r], wg, wu, wd)
         for k in range(K):                     # gate-weighted sum, k ascending
             h += y[:, k]
     return h, routing

@@ -136,3 +136,98 @@ def test_pins_catch_mutant(name, monkeypatch):
 def test_pins_pass_without_mutant():
     for pin in PINS:
         pin()
+
+
+# --- the FP8 quantization oracle ------------------------------------------
+
+import oracle.fp8 as F8  # noqa: E402
+import tests.test_oracle_fp8 as P8  # noqa: E402
+
+_orig8 = {name: getattr(F8, name) for name in
+          ("e4m3_decode", "e4m3_encode", "scale_exponent", "quantize_rows", "qdq_rows", "qdq_blocks",
+           "swiglu_ffn_fp8")}
+
+
+def _encode_truncating(v):
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    code = np.searchsorted(F8._POS_VALUES, a, side="right") - 1   # largest value <= a
+    return np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+
+
+def _encode_ties_away(v):
+    v = np.asarray(v, dtype=np.float64)
+    nudged = np.nextafter(np.abs(v), np.inf)                       # a tie now rounds up
+    return _orig8["e4m3_encode"](np.where(np.signbit(v), -nudged, nudged).clip(-448, 448))
+
+
+def _decode_wrong_bias(codes):
+    return _orig8["e4m3_decode"](codes) / 2.0
+
+
+def _scale_exponent_off_at_powers(amax):
+    a = np.asarray(amax, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.int64)
+    for i, x in np.ndenumerate(a):
+        out[i] = -127 if x == 0 else min(max(int(np.frexp(x / 448.0)[1]), -127), 127)
+    return out
+
+
+def _rows_in_column_groups(x):
+    return F8.quantize_groups(x, F8.GROUP, 1)
+
+
+def _qdq_rows_in_column_groups(x):
+    return F8.dequantize_groups(*F8.quantize_groups(x, F8.GROUP, 1), F8.GROUP, 1)
+
+
+def _qdq_weights_row_wise(w):
+    w = M.f64(w)
+    if w.ndim == 3:
+        return np.stack([_qdq_weights_row_wise(m) for m in w])
+    return F8.dequantize_groups(*F8.quantize_groups(w, 1, F8.GROUP), 1, F8.GROUP)
+
+
+def _ffn_h_not_quantized(u, w_gate, w_up, w_down):
+    uq = F8.qdq_rows(u)
+    h = M.silu(uq @ F8.qdq_blocks(w_gate).T) * (uq @ F8.qdq_blocks(w_up).T)
+    return h @ F8.qdq_blocks(w_down).T
+
+
+def _ffn_u_not_quantized(u, w_gate, w_up, w_down):
+    u = M.f64(u)
+    h = F8.qdq_rows(M.silu(u @ F8.qdq_blocks(w_gate).T) * (u @ F8.qdq_blocks(w_up).T))
+    return h @ F8.qdq_blocks(w_down).T
+
+
+MUTANTS_FP8 = {
+    "e4m3_truncating": ("e4m3_encode", _encode_truncating),
+    "e4m3_ties_away_from_zero": ("e4m3_encode", _encode_ties_away),
+    "e4m3_wrong_exponent_bias": ("e4m3_decode", _decode_wrong_bias),
+    "scale_exponent_off_by_one_at_powers": ("scale_exponent", _scale_exponent_off_at_powers),
+    "activation_groups_128x1": ("quantize_rows", _rows_in_column_groups),
+    "activation_qdq_128x1": ("qdq_rows", _qdq_rows_in_column_groups),
+    "weights_grouped_row_wise": ("qdq_blocks", _qdq_weights_row_wise),
+    "h_not_quantized": ("swiglu_ffn_fp8", _ffn_h_not_quantized),
+    "input_rows_not_quantized": ("swiglu_ffn_fp8", _ffn_u_not_quantized),
+}
+
+PINS_FP8 = [getattr(P8, n) for n in dir(P8) if n.startswith("test_")]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_FP8))
+def test_fp8_pins_catch_mutant(name, monkeypatch):
+    fn_name, mutant = MUTANTS_FP8[name]
+    monkeypatch.setattr(F8, fn_name, mutant)
+    caught = 0
+    for pin in PINS_FP8:
+        try:
+            pin()
+        except Exception:
+            caught += 1
+    assert caught > 0, f"no FP8 pin caught the mutant {name}"
+
+
+def test_fp8_pins_pass_without_mutant():
+    for pin in PINS_FP8:
+        pin()
