@@ -56,6 +56,8 @@ def parse_args():
     p.add_argument("--config", default="16b_prefill", choices=sorted(W.CONFIGS))
     p.add_argument("--cpu-sample", type=int, default=256, help="tokens of the CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--fp8-quant", action="store_true",
+                   help="time the FP8 1x128 quantization of one forward's permuted activations instead")
     return p.parse_args()
 
 
@@ -414,8 +416,138 @@ def run_ours(args):
     ranks.close()
 
 
+def run_fp8_quant(args):
+    """One step = the FP8 1 x 128 quantization of the permuted activations of one forward of the
+    workload ([T * K, d] bf16, larger than L2: 403 MB for the 16B prefill layer) through the C ABI.
+    The 128 x 128 block quantization of the routed experts' W_gate is timed beside it.  Both kernels
+    stream (2 B read, 1 B + 1/128 B written per element): the roofline is HBM bandwidth."""
+    from ctypes import c_void_p
+    from fine_grained_shared_b200 import moe as B
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    shape = W.CONFIGS[args.config]
+    rows, cols = shape.T * shape.K, shape.d
+    groups = -(-cols // 128)
+    x_h = W.normal_bf16(shape.seed, 40, 0, (rows, cols), 1.0)
+    x = x_h.to(dev)
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    sc = torch.empty((rows, groups), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = c_void_p(stream.cuda_stream)
+
+    def step(src):
+        st = B.moe_quantize_fp8_rows(c_void_p(src.data_ptr()), rows, cols, c_void_p(q.data_ptr()),
+                                     c_void_p(sc.data_ptr()), sp)
+        if st != B.MOE_OK:
+            raise B.MoEError(st, "moe_quantize_fp8_rows")
+
+    for _ in range(max(3, args.warmup)):
+        step(x)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(args.steps):
+        step(x)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    clk = clocks.stop()
+    ms_step = ranks.max(start.elapsed_time(end)) / args.steps
+    step_bytes = rows * cols * 3 + rows * groups
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+
+    # end to end: pinned host activations in, codes and scales back to pinned host memory
+    xp = x_h.pin_memory()
+    qh = torch.empty((rows, cols), dtype=torch.uint8).pin_memory()
+    sh = torch.empty((rows, groups), dtype=torch.uint8).pin_memory()
+    xd = torch.empty_like(x)
+    e2e_steps = max(1, min(args.steps, 20))
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        xd.copy_(xp, non_blocking=True)
+        step(xd)
+        qh.copy_(q, non_blocking=True)
+        sh.copy_(sc, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    e2e_ms = ranks.max(e0.elapsed_time(e1)) / e2e_steps
+
+    # the routed experts' W_gate in 128 x 128 blocks, beside it
+    w = W.normal_bf16(shape.seed, 3, 0, (shape.N, shape.I, shape.d), shape.sigma).to(dev)
+    wq = torch.empty(w.shape, dtype=torch.uint8, device=dev)
+    ws = torch.empty((shape.N, -(-shape.I // 128), groups), dtype=torch.uint8, device=dev)
+
+    def wstep():
+        st = B.moe_quantize_fp8_blocks(c_void_p(w.data_ptr()), shape.N, shape.I, shape.d,
+                                       c_void_p(wq.data_ptr()), c_void_p(ws.data_ptr()), sp)
+        if st != B.MOE_OK:
+            raise B.MoEError(st, "moe_quantize_fp8_blocks")
+
+    for _ in range(3):
+        wstep()
+    torch.cuda.synchronize(dev)
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
+    for _ in range(10):
+        wstep()
+    w1.record(stream)
+    torch.cuda.synchronize(dev)
+    w_ms = w0.elapsed_time(w1) / 10
+    w_bytes = w.numel() * 3 + ws.numel()
+
+    peaks, peak_src = measured_peaks()
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": "FP8 1x128 activation quantization bandwidth", "value": value, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3",
+        "data": "synthetic",
+        "config": {"workload": f"{shape.name}: permuted activations [T*K={rows}, d={cols}] bf16, "
+                               f"1x128 groups", "l2": "input larger than L2 (no flush)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs", "kernel": "quantize_rows_kernel",
+                     "bytes_per_launch": step_bytes},
+        "weights_128x128": {"matrices": f"W_gate [{shape.N}, {shape.I}, {shape.d}]", "ms": w_ms,
+                            "gbs": w_bytes / (w_ms * 1e-3) / 1e9,
+                            "frac": w_bytes / (w_ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"])},
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": rows * cols * 2, "d2h_bytes_per_step": rows * cols + rows * groups,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle.fp8 as F8
+        n = 512
+        xs = x_h[:n].float().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        F8.quantize_rows(xs)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n * (cols * 3 + groups) / dt / 1e9, "unit": "GB/s", "cores": 1,
+                                "kind": "oracle", "sample": f"{n} rows of the [{rows}, {cols}] activations "
+                                                            "(float64 numpy, per-group loop)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.close()
+
+
 def main():
     args = parse_args()
+    if args.fp8_quant and args.impl == "ours":
+        run_fp8_quant(args)
+        return
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return

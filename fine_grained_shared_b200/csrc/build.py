@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libfgs_moe.so")
-SOURCES = ["moe_api.cu", "route_noalloc.cu"]
+SOURCES = ["moe_api.cu", "route_noalloc.cu", "fp8_quant.cu"]
 HEADERS = ["sm100.cuh", "router_topk.cuh", "permute.cuh", "gateup_gemm.cuh", "down_gemm.cuh"]
 
 

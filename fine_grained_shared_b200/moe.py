@@ -83,11 +83,13 @@ def lib() -> ctypes.CDLL:
     L.moe_route_noalloc.argtypes = [c_void_p, c_int64, c_int32, POINTER(moe_router), c_int32, c_int32, c_int32,
                                     c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.moe_update_bias.argtypes = [moe_handle, c_void_p, ctypes.c_float, c_void_p]
+    L.moe_quantize_fp8_rows.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
+    L.moe_quantize_fp8_blocks.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
     L.moe_status_string.argtypes = [c_int]
     L.moe_status_string.restype = c_char_p
     for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_get_routing",
                  "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc",
-                 "moe_update_bias"):
+                 "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks"):
         getattr(L, name).restype = c_int
     _lib = L
     return L
@@ -155,6 +157,16 @@ def moe_kernel_times(h):
     count = (c_int32 * len(KERNEL_NAMES))()
     st = lib().moe_kernel_times(h, total, count)
     return st, {n: (float(total[i]), int(count[i])) for i, n in enumerate(KERNEL_NAMES)}
+
+
+def moe_quantize_fp8_rows(x, rows, cols, q, scale, stream):
+    """E4M3 codes and UE8M0 scales of 1 x 128 row groups; see the header."""
+    return lib().moe_quantize_fp8_rows(x, int(rows), int(cols), q, scale, stream)
+
+
+def moe_quantize_fp8_blocks(w, batch, rows, cols, q, scale, stream):
+    """E4M3 codes and UE8M0 scales of 128 x 128 blocks of `batch` matrices; see the header."""
+    return lib().moe_quantize_fp8_blocks(w, int(batch), int(rows), int(cols), q, scale, stream)
 
 
 # --- torch convenience wrapper (pointers and sizes only) --------------------
@@ -266,3 +278,29 @@ class MoELayer:
         if st != MOE_OK:
             raise MoEError(st, "moe_kernel_times")
         return t
+
+
+def quantize_fp8_rows(x, stream=None):
+    """bf16 CUDA tensor [rows, cols] -> (codes uint8 [rows, cols], scales uint8 [rows, ceil(cols/128)])."""
+    import torch
+    rows, cols = x.shape
+    q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    sc = torch.empty((rows, -(-cols // 128)), dtype=torch.uint8, device=x.device)
+    st = moe_quantize_fp8_rows(_ptr(x), rows, cols, _ptr(q), _ptr(sc), _stream_ptr(stream))
+    if st != MOE_OK:
+        raise MoEError(st, "moe_quantize_fp8_rows")
+    return q, sc
+
+
+def quantize_fp8_blocks(w, stream=None):
+    """bf16 CUDA tensor [batch, rows, cols] (or [rows, cols]) -> (codes uint8, scales uint8
+    [batch, ceil(rows/128), ceil(cols/128)])."""
+    import torch
+    w3 = w if w.dim() == 3 else w.unsqueeze(0)
+    b, rows, cols = w3.shape
+    q = torch.empty((b, rows, cols), dtype=torch.uint8, device=w.device)
+    sc = torch.empty((b, -(-rows // 128), -(-cols // 128)), dtype=torch.uint8, device=w.device)
+    st = moe_quantize_fp8_blocks(_ptr(w3), b, rows, cols, _ptr(q), _ptr(sc), _stream_ptr(stream))
+    if st != MOE_OK:
+        raise MoEError(st, "moe_quantize_fp8_blocks")
+    return (q, sc) if w.dim() == 3 else (q[0], sc[0])

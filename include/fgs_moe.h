@@ -221,6 +221,38 @@ moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_model, const mo
                              int32_t n_routed, int32_t gate, int32_t K, int32_t* idx, float* gate_out,
                              int32_t* counts, int32_t* offsets, uint32_t* err, void* stream);
 
+/* Fine-grained FP8 quantization of GEMM operands (the first step of an FP8
+ * expert path).  DeepSeek-V3 technical report, section 3.3 "FP8 Training":
+ * GEMM inputs in FP8 with one scale per small group of values (fine-grained
+ * scaling), activation scales powers of two; Appendix B.2 "Discussion About
+ * Block-Wise Quantization": activations grouped 1 x 128 along the channels in
+ * the forward pass, weights in 128 x 128 blocks.
+ *
+ * Per group, e is the smallest integer with max|x| <= 448 * 2^e, clamped to
+ * [-127, 127] (an all-zero group takes -127); each element becomes the E4M3
+ * code ("fn" variant: largest finite 448, no infinities) of x * 2^-e, rounded
+ * to nearest with ties to the even code, keeping the sign (a negative value
+ * that rounds to zero is 0x80).  The scale is stored as the byte e + 127
+ * (UE8M0: the value it stands for is 2^(byte - 127)).  Inputs must be finite.
+ *
+ * Both run on the calling thread's current device, on `stream`, asynchronously;
+ * all pointers are caller-owned device memory.  Errors, returned before any
+ * launch: a null pointer -> MOE_ERR_INVALID_ARG; a negative size, cols <= 0, or
+ * a grid dimension past CUDA's limits -> MOE_ERR_SHAPE; cols not a multiple of
+ * 16, or x / w / q not 16-byte aligned -> MOE_ERR_ALIGNMENT; a failed launch ->
+ * MOE_ERR_CUDA.  An empty input launches nothing and returns MOE_OK.
+ *
+ * moe_quantize_fp8_rows: x bf16 [rows, cols] row-major (activations, one token
+ *   per row) -> q uint8 [rows, cols], scale uint8 [rows, ceil(cols / 128)];
+ *   group g of a row is columns [128 g, 128 g + 128) (the last may be shorter).
+ * moe_quantize_fp8_blocks: w bf16 [batch, rows, cols] (batch weight matrices,
+ *   [out, in] each) -> q uint8 [batch, rows, cols], scale uint8
+ *   [batch, ceil(rows / 128), ceil(cols / 128)]; batch <= 65535. */
+moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, uint8_t* q, uint8_t* scale,
+                                 void* stream);
+moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, int32_t cols, uint8_t* q,
+                                   uint8_t* scale, void* stream);
+
 /* A static string naming the status. */
 const char* moe_status_string(moe_status s);
 

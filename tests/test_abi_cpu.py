@@ -91,6 +91,28 @@ def test_null_handles():
     assert lib.moe_kernel_times(None, None, None) == B.MOE_ERR_INVALID_ARG
 
 
+def test_fp8_quantize_arguments_are_checked_before_any_cuda_call():
+    """Fake, never dereferenced device addresses: every case returns before a launch."""
+    lib = B.lib()
+    a, b, c = 0x10000, 0x20000, 0x30000
+    rows = lib.moe_quantize_fp8_rows
+    assert rows(None, 4, 128, b, c, None) == B.MOE_ERR_INVALID_ARG
+    assert rows(a, 4, 128, b, None, None) == B.MOE_ERR_INVALID_ARG
+    assert rows(a, -1, 128, b, c, None) == B.MOE_ERR_SHAPE
+    assert rows(a, 4, 0, b, c, None) == B.MOE_ERR_SHAPE
+    assert rows(a, 4, 120, b, c, None) == B.MOE_ERR_ALIGNMENT
+    assert rows(a + 8, 4, 128, b, c, None) == B.MOE_ERR_ALIGNMENT
+    assert rows(a, 4, 128, b + 4, c, None) == B.MOE_ERR_ALIGNMENT
+    assert rows(a, 0, 128, b, c, None) == B.MOE_OK
+    blocks = lib.moe_quantize_fp8_blocks
+    assert blocks(a, 2, 128, 128, None, c, None) == B.MOE_ERR_INVALID_ARG
+    assert blocks(a, 70000, 128, 128, b, c, None) == B.MOE_ERR_SHAPE
+    assert blocks(a, 2, -5, 128, b, c, None) == B.MOE_ERR_SHAPE
+    assert blocks(a, 2, 128, 136, b, c, None) == B.MOE_ERR_ALIGNMENT
+    assert blocks(a, 0, 128, 128, b, c, None) == B.MOE_OK
+    assert blocks(a, 3, 0, 128, b, c, None) == B.MOE_OK
+
+
 def test_status_strings():
     for v, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (7, "MOE_ERR_TIMEOUT"), (99, "MOE_ERR_UNKNOWN")]:
         assert B.status_string(v) == name
