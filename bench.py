@@ -45,6 +45,8 @@ DOMINANT = "gate_up"
 PROFILE_SUMMARIES = {"16b_prefill": os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt"),
                      "16b_decode": os.path.join(ROOT, "profiles", "gemms_16b_decode.txt")}
 KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/gateup_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
+FP8_PROFILES = {"16b_prefill": os.path.join(ROOT, "profiles", "fp8_quant_rows_16b_prefill.txt")}
+FP8_SOURCES = ["fine_grained_shared_b200/csrc/fp8_quant.cu"]
 
 
 def parse_args():
@@ -93,18 +95,18 @@ def measured_peaks():
     return PEAK_FALLBACK, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in sources:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(shape: W.LayerShape):
+def profiled_traffic(shape: W.LayerShape, path=None, sources=KERNEL_SOURCES):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary of this workload, if it was taken on the current kernel source; else None."""
-    path = PROFILE_SUMMARIES.get(shape.name)
+    path = path or PROFILE_SUMMARIES.get(shape.name)
     if path is None or not os.path.exists(path):
         return None
     vals = {}
@@ -113,7 +115,7 @@ def profiled_traffic(shape: W.LayerShape):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals.setdefault(k.strip(), v.strip())  # the first kernel listed is the dominant one
-    if vals.get("source_sha256_16") != kernel_source_hash():
+    if vals.get("source_sha256_16") != kernel_source_hash(sources):
         return None
     try:
         if "traffic_bytes_per_token" in vals:
@@ -516,7 +518,9 @@ def run_fp8_quant(args):
         "config": {"workload": f"{shape.name}: permuted activations [T*K={rows}, d={cols}] bf16, "
                                f"1x128 groups", "l2": "input larger than L2 (no flush)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
-                     "frac": achieved / float(peaks["hbm_gbs"]), "traffic": None,
+                     "frac": achieved / float(peaks["hbm_gbs"]),
+                     "traffic": profiled_traffic(shape, FP8_PROFILES.get(shape.name, ""), FP8_SOURCES)
+                     if shape.name in FP8_PROFILES else None,
                      "peak_source": f"{peak_src} hbm_gbs", "kernel": "quantize_rows_kernel",
                      "bytes_per_launch": step_bytes},
         "weights_128x128": {"matrices": f"W_gate [{shape.N}, {shape.I}, {shape.d}]", "ms": w_ms,
