@@ -231,3 +231,85 @@ def test_fp8_pins_catch_mutant(name, monkeypatch):
 def test_fp8_pins_pass_without_mutant():
     for pin in PINS_FP8:
         pin()
+
+
+# --- the backward oracle ----------------------------------------------------
+
+import oracle.moe_backward as MBW  # noqa: E402
+import tests.test_oracle_backward as PB  # noqa: E402
+
+_origb = {name: getattr(MBW, name) for name in ("silu_grad", "swiglu_ffn_backward", "gate_logit_backward")}
+
+
+def _silu_grad_sigma_only(a):
+    return 1.0 / (1.0 + np.exp(-a))
+
+
+def _ffn_backward_drops_up_path(u, w_gate, w_up, w_down, dy):
+    du, dwg, dwu, dwd = _origb["swiglu_ffn_backward"](u, w_gate, w_up, w_down, dy)
+    wg, wu, wd = M.f64(w_gate), M.f64(w_up), M.f64(w_down)
+    a = u @ wg.T
+    db = (dy @ wd) * M.silu(a)
+    return du - db @ wu, dwg, dwu, dwd
+
+
+def _ffn_backward_gate_up_weight_grads_swapped(u, w_gate, w_up, w_down, dy):
+    du, dwg, dwu, dwd = _origb["swiglu_ffn_backward"](u, w_gate, w_up, w_down, dy)
+    return du, dwu, dwg, dwd
+
+
+def _softmax_backward_not_centred(s, idx, gate, dg, gate_kind):
+    if gate_kind != M.GATE_SOFTMAX:
+        return _origb["gate_logit_backward"](s, idx, gate, dg, gate_kind)
+    T, N = s.shape
+    ds = np.zeros((T, N))
+    np.add.at(ds, (np.repeat(np.arange(T), idx.shape[1]), idx.ravel()), dg.ravel())
+    return s * ds
+
+
+def _sigmoid_backward_not_normalised(s, idx, gate, dg, gate_kind):
+    if gate_kind != M.GATE_SIGMOID:
+        return _origb["gate_logit_backward"](s, idx, gate, dg, gate_kind)
+    s_sel = np.take_along_axis(s, idx, axis=1)
+    dz = np.zeros_like(s)
+    np.put_along_axis(dz, idx, dg * s_sel * (1.0 - s_sel), axis=1)
+    return dz
+
+
+def _logit_backward_wrong_sign(s, idx, gate, dg, gate_kind):
+    return -_origb["gate_logit_backward"](s, idx, gate, dg, gate_kind)
+
+
+MUTANTS_BWD = {
+    "silu_grad_sigma_only": ("silu_grad", _silu_grad_sigma_only),
+    "ffn_backward_drops_up_path": ("swiglu_ffn_backward", _ffn_backward_drops_up_path),
+    "gate_up_weight_grads_swapped": ("swiglu_ffn_backward", _ffn_backward_gate_up_weight_grads_swapped),
+    "softmax_backward_not_centred": ("gate_logit_backward", _softmax_backward_not_centred),
+    "sigmoid_backward_not_normalised": ("gate_logit_backward", _sigmoid_backward_not_normalised),
+    "logit_backward_wrong_sign": ("gate_logit_backward", _logit_backward_wrong_sign),
+}
+
+PINS_BWD = [
+    lambda: [PB.test_gradients_match_central_differences(k, s) for k, s in
+             ((M.GATE_SOFTMAX, 1), (M.GATE_SIGMOID, 2))],
+    lambda: [PB.test_single_elements_match_central_differences(k) for k in (M.GATE_SOFTMAX, M.GATE_SIGMOID)],
+    PB.test_softmax_logit_gradients_sum_to_zero,
+]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS_BWD))
+def test_backward_pins_catch_mutant(name, monkeypatch):
+    fn_name, mutant = MUTANTS_BWD[name]
+    monkeypatch.setattr(MBW, fn_name, mutant)
+    caught = 0
+    for pin in PINS_BWD:
+        try:
+            pin()
+        except Exception:
+            caught += 1
+    assert caught > 0, f"no backward pin caught the mutant {name}"
+
+
+def test_backward_pins_pass_without_mutant():
+    for pin in PINS_BWD:
+        pin()
