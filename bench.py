@@ -237,6 +237,40 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+FP8_METRIC = "FP8 1x128 activation quantization bandwidth"
+
+
+def fp8_workload_config(shape: W.LayerShape) -> dict:
+    return {"workload": f"{shape.name}: permuted activations [T*K={shape.T * shape.K}, d={shape.d}] bf16, "
+                        f"1x128 groups", "l2": "input larger than L2 (no flush)"}
+
+
+def run_reference_fp8(args):
+    """The FP8 oracle (float64 numpy) quantizing a bounded sample of the rows each step."""
+    import oracle.fp8 as F8
+    shape = W.CONFIGS[args.config]
+    cols = shape.d
+    groups = -(-cols // 128)
+    n = max(1, min(shape.T * shape.K, args.cpu_sample))
+    x = W.normal_bf16(shape.seed, 40, 0, (n, cols), 1.0).float().numpy().astype(np.float64)
+    for _ in range(args.warmup):
+        F8.quantize_rows(x)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        F8.quantize_rows(x)
+    dt = time.perf_counter() - t0
+    value = args.steps * n * (3 * cols + groups) / dt / 1e9
+    line = {"metric": FP8_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": fp8_workload_config(shape),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n} rows of the [{shape.T * shape.K}, {cols}] activations per step "
+                                       f"(float64 numpy, per-group loop)"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
@@ -511,12 +545,11 @@ def run_fp8_quant(args):
     peaks, peak_src = measured_peaks()
     achieved = step_bytes / (ms_step * 1e-3) / 1e9
     line = {
-        "metric": "FP8 1x128 activation quantization bandwidth", "value": value, "unit": "GB/s",
+        "metric": FP8_METRIC, "value": value, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3",
         "data": "synthetic",
-        "config": {"workload": f"{shape.name}: permuted activations [T*K={rows}, d={cols}] bf16, "
-                               f"1x128 groups", "l2": "input larger than L2 (no flush)"},
+        "config": fp8_workload_config(shape),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                      "frac": achieved / float(peaks["hbm_gbs"]),
                      "traffic": profiled_traffic(shape, FP8_PROFILES.get(shape.name, ""), FP8_SOURCES)
@@ -549,13 +582,12 @@ def run_fp8_quant(args):
 
 def main():
     args = parse_args()
-    if args.fp8_quant and args.impl == "ours":
-        run_fp8_quant(args)
-        return
     if args.impl == "reference":
         if int(os.environ.get("RANK", "0")) != 0:
             return
-        run_reference(args)
+        run_reference_fp8(args) if args.fp8_quant else run_reference(args)
+    elif args.fp8_quant:
+        run_fp8_quant(args)
     else:
         run_ours(args)
 

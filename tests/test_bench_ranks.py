@@ -61,3 +61,18 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     with contextlib.redirect_stdout(out):
         bench.main()
     assert out.getvalue() == ""
+
+
+def test_fp8_reference_arm_times_the_fp8_oracle(monkeypatch):
+    import json
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--fp8-quant", "--steps", "2",
+                                      "--warmup", "1", "--cpu-sample", "16"])
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.main()
+    line = json.loads(out.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.FP8_METRIC and line["unit"] == "GB/s"
+    assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["config"]["workload"].startswith("16b_prefill")
