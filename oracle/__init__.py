@@ -10,6 +10,6 @@ the layer's backward pass.
 from .moe_oracle import (  # noqa: F401
     GATE_SIGMOID, GATE_SOFTMAX, FLAG_NO_RESIDUAL, FLAG_NO_ROUTED, FLAG_NO_SHARED,
     Permutation, Routing, affinity_logits, bias_update, expert_permutation, f64, gate_values,
-    moe_forward, route, select_top_k, sigmoid_affinity, silu, softmax_affinity,
+    moe_forward, route, select_top_k, select_top_k_node_limited, sigmoid_affinity, silu, softmax_affinity,
     swiglu_ffn,
 )

@@ -109,6 +109,31 @@ def select_top_k(key: np.ndarray, K: int) -> np.ndarray:
     return order[:, :K].astype(np.int64)
 
 
+def select_top_k_node_limited(key: np.ndarray, K: int, n_nodes: int, M: int) -> np.ndarray:
+    """Top-K restricted to at most M of the n_nodes nodes -> idx [T, K].
+
+    DeepSeek-V3 technical report summary, section 2 ("DeepSeekMoE"): routing
+    is node-limited, each token going to at most M nodes, chosen among the
+    nodes that hold its highest-affinity routed experts.  The pages give no
+    formula; the reading taken: the mN experts sit on the nodes in equal
+    contiguous ranges (expert i on node i // (mN / n_nodes)); a node ranks by
+    the largest key among its experts (equivalently: walk the experts by key,
+    descending, collecting their nodes until M are found), ties to the lower
+    node index; the token's K experts are then the top K of the chosen nodes'
+    experts, ordered and tie-broken as in ``select_top_k``.
+    """
+    T, N = key.shape
+    if N % n_nodes or not 1 <= M <= n_nodes or K > M * (N // n_nodes):
+        raise ValueError("node-limited routing needs mN % nodes == 0, 1 <= M <= nodes, K <= M * mN / nodes")
+    per = N // n_nodes
+    node_score = key.reshape(T, n_nodes, per).max(axis=2)
+    nodes = np.argsort(-node_score, axis=1, kind="stable")[:, :M]          # ties -> lower node
+    allowed = np.zeros((T, n_nodes), dtype=bool)
+    np.put_along_axis(allowed, nodes, True, axis=1)
+    masked = np.where(np.repeat(allowed, per, axis=1), key, -np.inf)
+    return select_top_k(masked, K)
+
+
 def gate_values(s: np.ndarray, idx: np.ndarray, gate_kind: str) -> np.ndarray:
     """g[t, k]: the affinity of the k-th selected expert (softmax), or that
     affinity divided by the sum over the selected experts (sigmoid)."""
@@ -129,8 +154,10 @@ class Routing:
 
 
 def route(u, router_w, K: int, gate_kind: str = GATE_SOFTMAX,
-          logit_bias=None, select_bias=None) -> Routing:
-    """Steps 1-5 for every token of u."""
+          logit_bias=None, select_bias=None, node_limit=None) -> Routing:
+    """Steps 1-5 for every token of u.  ``node_limit`` = (nodes, M) restricts
+    each token's experts to at most M nodes (``select_top_k_node_limited``);
+    ``gap`` is then left at +inf."""
     u, e = f64(u), f64(router_w)
     z = affinity_logits(u, e, logit_bias)
     if gate_kind == GATE_SOFTMAX:
@@ -141,10 +168,10 @@ def route(u, router_w, K: int, gate_kind: str = GATE_SOFTMAX,
         key = s if select_bias is None else s + f64(select_bias)[None, :]
     else:
         raise ValueError(gate_kind)
-    idx = select_top_k(key, K)
+    idx = select_top_k(key, K) if node_limit is None else select_top_k_node_limited(key, K, *node_limit)
     gate = gate_values(s, idx, gate_kind)
     N = key.shape[1]
-    if K < N:
+    if K < N and node_limit is None:
         srt = -np.sort(-key, axis=1)
         gap = srt[:, K - 1] - srt[:, K]
     else:
@@ -220,7 +247,8 @@ def _as_expert_fn(w_gate, w_up, w_down) -> ExpertFn:
 def moe_forward(u, router_w, K: int, experts, shared=None, *,
                 gate_kind: str = GATE_SOFTMAX, logit_bias=None, select_bias=None,
                 flags: int = 0, rows: Optional[np.ndarray] = None,
-                routing: Optional[Routing] = None, ffn: Optional[Callable] = None):
+                routing: Optional[Routing] = None, ffn: Optional[Callable] = None,
+                node_limit=None):
     """h_t for the tokens ``rows`` (all tokens when None) -> (h [n, d], Routing).
 
     ``experts`` is either a tuple (W_gate [N,I,d], W_up [N,I,d], W_down [N,d,I])
@@ -229,7 +257,8 @@ def moe_forward(u, router_w, K: int, experts, shared=None, *,
     ``flags`` leaves out terms of the sum (residual, shared, routed) so that
     each term can be checked on its own.  Tokens are independent, so the
     output of a subset of rows equals those rows of the full output.
-    ``ffn`` replaces ``swiglu_ffn`` for every expert (the FP8 variant).
+    ``ffn`` replaces ``swiglu_ffn`` for every expert (the FP8 variant);
+    ``node_limit`` = (nodes, M) is passed to ``route``.
     """
     u_all = f64(u)
     if rows is None:
@@ -237,7 +266,7 @@ def moe_forward(u, router_w, K: int, experts, shared=None, *,
     rows = np.asarray(rows, dtype=np.int64)
     ur = u_all[rows]
     if routing is None:
-        routing = route(ur, router_w, K, gate_kind, logit_bias, select_bias)
+        routing = route(ur, router_w, K, gate_kind, logit_bias, select_bias, node_limit)
         idx, gate = routing.idx, routing.gate
     else:
         idx, gate = routing.idx[rows], routing.gate[rows]

@@ -8,11 +8,13 @@ import numpy as np
 import pytest
 
 import oracle.moe_oracle as M
+import tests.test_oracle_node_limited as PN
 import tests.test_oracle_pins as P
 
 _orig = {name: getattr(M, name) for name in
          ("silu", "softmax_affinity", "sigmoid_affinity", "select_top_k", "gate_values",
-          "swiglu_ffn", "affinity_logits", "expert_permutation", "moe_forward", "bias_update")}
+          "swiglu_ffn", "affinity_logits", "expert_permutation", "moe_forward", "bias_update",
+          "select_top_k_node_limited")}
 
 
 def _silu_wrong_sign(a):
@@ -81,6 +83,20 @@ def _bias_update_wrong_sign(bias, counts, gamma):
     return _orig["bias_update"](bias, counts, -gamma)
 
 
+def _node_limited(score_fn=None, interleaved=False, ascending=False, extra=0):
+    def f(key, K, n_nodes, lim):
+        T, N = key.shape
+        per = N // n_nodes
+        node_of = np.arange(N) % n_nodes if interleaved else np.arange(N) // per
+        score = np.stack([(score_fn or np.max)(key[:, node_of == g], axis=1) for g in range(n_nodes)], axis=1)
+        nodes = np.argsort(score if ascending else -score, axis=1, kind="stable")[:, :min(n_nodes, lim + extra)]
+        allowed = np.zeros((T, N), dtype=bool)
+        for t in range(T):
+            allowed[t] = np.isin(node_of, nodes[t])
+        return M.select_top_k(np.where(allowed, key, -np.inf), K)
+    return f
+
+
 MUTANTS = {
     "silu_wrong_sign": ("silu", _silu_wrong_sign),
     "softmax_wrong_normaliser": ("softmax_affinity", _softmax_no_shift_renorm_topk),
@@ -95,6 +111,10 @@ MUTANTS = {
     "residual_dropped": ("moe_forward", _forward_drops_residual),
     "shared_dropped": ("moe_forward", _forward_drops_shared),
     "bias_update_wrong_sign": ("bias_update", _bias_update_wrong_sign),
+    "node_score_is_sum_of_keys": ("select_top_k_node_limited", _node_limited(score_fn=np.sum)),
+    "experts_interleaved_over_nodes": ("select_top_k_node_limited", _node_limited(interleaved=True)),
+    "worst_nodes_chosen": ("select_top_k_node_limited", _node_limited(ascending=True)),
+    "one_node_too_many": ("select_top_k_node_limited", _node_limited(extra=1)),
 }
 
 PINS = [
@@ -113,6 +133,9 @@ PINS = [
     lambda: P.test_permutation_matches_sorted_pairs(7, 3),
     P.test_bias_update_hand_example,
     P.test_bias_update_balances_a_skewed_router,
+    PN.test_hand_example,
+    lambda: PN.test_matches_the_walk_down_the_experts(2),
+    PN.test_properties,
 ]
 
 
