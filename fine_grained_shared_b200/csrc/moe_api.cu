@@ -184,6 +184,7 @@ struct moe_ctx {
   // host-buffer forward: copy streams and per-chunk events, created on first use
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
   cudaEvent_t host_start = nullptr, in_done[kHostChunks] = {}, fwd_done[kHostChunks] = {};
+  bool host_ready = false;  // all of the above created
   // per-kernel timing: event pairs recorded around each launch while enabled
   uint32_t timing_mask = 0;  // bit k: time kernel k
   std::vector<cudaEvent_t> ev_pool[MOE_KERNEL_COUNT];
@@ -306,6 +307,21 @@ cudaError_t launch_gateup(int ctas, cudaStream_t s, bool pdl, const CUtensorMap&
                           const GateUpArgs& ga) {
   return launch_pdl(gateup_gemm_kernel, dim3(ctas), dim3(kGuThreads), gateup_smem_bytes(), s, 1, pdl, A, G, U, As, Gs,
                     Us, ga);
+}
+
+// Destroys the host-buffer forward's copy streams and events (those that exist).
+void release_host_pipeline(moe_ctx* h) {
+  if (h->copy_in) cudaStreamDestroy(h->copy_in);
+  if (h->copy_out) cudaStreamDestroy(h->copy_out);
+  if (h->host_start) cudaEventDestroy(h->host_start);
+  h->copy_in = h->copy_out = nullptr;
+  h->host_start = nullptr;
+  for (int c = 0; c < kHostChunks; ++c) {
+    if (h->in_done[c]) cudaEventDestroy(h->in_done[c]);
+    if (h->fwd_done[c]) cudaEventDestroy(h->fwd_done[c]);
+    h->in_done[c] = h->fwd_done[c] = nullptr;
+  }
+  h->host_ready = false;
 }
 
 // Records a start/stop event pair around one launch when timing is enabled.
@@ -679,14 +695,19 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
       return MOE_ERR_CUDA;
     return cudaStreamSynchronize(s0) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
-  if (!h->copy_in) {
+  if (!h->host_ready) {
     bool ok = cudaStreamCreateWithFlags(&h->copy_in, cudaStreamNonBlocking) == cudaSuccess &&
               cudaStreamCreateWithFlags(&h->copy_out, cudaStreamNonBlocking) == cudaSuccess &&
               cudaEventCreateWithFlags(&h->host_start, cudaEventDisableTiming) == cudaSuccess;
     for (int c = 0; c < kHostChunks && ok; ++c)
       ok = cudaEventCreateWithFlags(&h->in_done[c], cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&h->fwd_done[c], cudaEventDisableTiming) == cudaSuccess;
-    if (!ok) return MOE_ERR_CUDA;
+    if (!ok) {  // release what was made, so that a later call starts over
+      release_host_pipeline(h);
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    h->host_ready = true;
   }
   // finish everything in flight on all three streams before returning, also on an error
   auto finish = [&](moe_status st) {
@@ -805,13 +826,7 @@ moe_status moe_destroy(moe_handle h) {
     cudaDeviceSynchronize();
     for (auto& pool : h->ev_pool)
       for (cudaEvent_t e : pool) cudaEventDestroy(e);
-    if (h->copy_in) cudaStreamDestroy(h->copy_in);
-    if (h->copy_out) cudaStreamDestroy(h->copy_out);
-    if (h->host_start) cudaEventDestroy(h->host_start);
-    for (int c = 0; c < kHostChunks; ++c) {
-      if (h->in_done[c]) cudaEventDestroy(h->in_done[c]);
-      if (h->fwd_done[c]) cudaEventDestroy(h->fwd_done[c]);
-    }
+    release_host_pipeline(h);
     if (h->ws) cudaFree(h->ws);
   }
   delete h;

@@ -155,7 +155,10 @@ moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* cou
  * report summary, section 2 "Auxiliary-Loss-Free Load Balancing": after each
  * step a bias moves according to whether its expert was overloaded or
  * underloaded).  With load_i the (token, slot) pairs routed to expert i by the
- * last moe_forward on this handle and mean = sum(load) / mN:
+ * last moe_forward on this handle and mean = sum(load) / mN (after a
+ * moe_forward_host that ran in chunks, the loads are its last chunk's, as for
+ * moe_get_routing; to balance on a whole batch, forward it from device
+ * buffers with moe_forward):
  *   bias[i] += gamma * sign(mean - load_i)
  * (an overloaded expert's bias drops, an underloaded one's rises, an expert at
  * exactly the mean keeps its bias; the comparison is exact, on integers).
