@@ -27,7 +27,9 @@ Q3 rounding  code = E4M3(x / s), round to nearest, ties to the even code, on
              of x, so a negative value that rounds to zero is -0 (0x80).
 Q4 groups    activations (the rows entering a GEMM): 1 x 128 along the
              reduction dimension; weights: 128 x 128 blocks of each [out, in]
-             matrix.  A ragged last group is a shorter group.
+             matrix; in the backward pass, activations that a weight-gradient
+             GEMM contracts over tokens: 128 x 1.  A ragged last group is a
+             shorter group.
 Q5 value     dequantized = decode(code) * s; the GEMMs accumulate in float64
              here (high-precision accumulation).
 Q6 layer     the router stays in high precision (section 3.3 keeps selected
@@ -132,6 +134,12 @@ def dequantize_groups(codes, exps, group_rows: int, group_cols: int) -> np.ndarr
 def quantize_rows(x):
     """Activations: 1 x 128 groups along the last dimension (reading Q4)."""
     return quantize_groups(x, 1, GROUP)
+
+
+def quantize_cols(x):
+    """Activations in the backward pass, where the weight-gradient GEMM contracts over tokens:
+    128 x 1 groups (128 consecutive rows of one column; Appendix B.2)."""
+    return quantize_groups(x, GROUP, 1)
 
 
 def quantize_blocks(w):

@@ -129,6 +129,20 @@ def test_weight_blocks_are_128_by_128():
     assert np.array_equal(F.qdq_blocks(w2), F.dequantize_groups(q1, e1, 128, 128))
 
 
+def test_backward_groups_are_128_tokens_of_one_channel():
+    rng = np.random.default_rng(15)
+    x = _bf16(rng.standard_normal((300, 40)) * np.exp2(rng.integers(-5, 5, size=(1, 40)))).astype(np.float64)
+    q, e = F.quantize_cols(x)
+    assert e.shape == (3, 40)                       # 128 + 128 + 44 rows
+    qt, et = F.quantize_rows(x.T)                   # the same groups, seen transposed
+    assert np.array_equal(q, qt.T) and np.array_equal(e, et.T)
+    x2 = x.copy()
+    x2[200, 7] = 1e4
+    q2, e2 = F.quantize_cols(x2)
+    assert np.argwhere(e != e2).tolist() == [[1, 7]]
+    assert all(c == 7 and 128 <= r < 256 for r, c in np.argwhere(q != q2))
+
+
 def test_ragged_last_group_has_its_own_scale():
     x = np.zeros((1, 144))
     x[0, :128] = 448.0

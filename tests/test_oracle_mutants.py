@@ -168,7 +168,7 @@ import tests.test_oracle_fp8 as P8  # noqa: E402
 
 _orig8 = {name: getattr(F8, name) for name in
           ("e4m3_decode", "e4m3_encode", "scale_exponent", "quantize_rows", "qdq_rows", "qdq_blocks",
-           "swiglu_ffn_fp8")}
+           "swiglu_ffn_fp8", "quantize_cols")}
 
 
 def _encode_truncating(v):
@@ -233,6 +233,7 @@ MUTANTS_FP8 = {
     "weights_grouped_row_wise": ("qdq_blocks", _qdq_weights_row_wise),
     "h_not_quantized": ("swiglu_ffn_fp8", _ffn_h_not_quantized),
     "input_rows_not_quantized": ("swiglu_ffn_fp8", _ffn_u_not_quantized),
+    "backward_groups_1x128": ("quantize_cols", lambda x: F8.quantize_groups(x, 1, F8.GROUP)),
 }
 
 PINS_FP8 = [getattr(P8, n) for n in dir(P8) if n.startswith("test_")]
