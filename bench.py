@@ -56,8 +56,10 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--config", default="16b_prefill", choices=sorted(W.CONFIGS))
-    p.add_argument("--cpu-sample", type=int, default=256, help="tokens of the CPU-baseline sample")
+    p.add_argument("--cpu-sample", type=int, default=256, help="rows of the FP8 oracle's CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-config", action="store_true",
+                   help="measure only the --config workload (by default the 2B, 16B decode and V3 layers follow)")
     p.add_argument("--fp8-quant", action="store_true",
                    help="time the FP8 1x128 quantization of one forward's permuted activations instead")
     return p.parse_args()
@@ -125,13 +127,6 @@ def profiled_traffic(shape: W.LayerShape, path=None, sources=KERNEL_SOURCES):
         return None
 
 
-def gate_up_weight_bytes(shape: W.LayerShape, counts) -> float:
-    """Weights one gate/up launch must stream: W_gate and W_up of every routed
-    expert that received a token, and of the shared experts."""
-    touched = int(sum(1 for c in counts if c > 0))
-    return 2.0 * 2 * shape.d * (touched * shape.I + shape.Ks * shape.Is)
-
-
 # ---------------------------------------------------------------------------
 # clocks sampled with nvidia-smi during the timed region
 # ---------------------------------------------------------------------------
@@ -193,20 +188,48 @@ def to_device(host: dict, dev) -> dict:
 # CPU oracle timing (the baseline arm)
 # ---------------------------------------------------------------------------
 
+def host_cpu():
+    """(logical cores, CPU model) of the host."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count() or 1, model
+
+
 def oracle_tokens_per_s(shape: W.LayerShape, host: dict, n_tokens: int, repeats: int = 1):
+    """The CPU oracle, as it stands, on ``n_tokens`` seeded tokens of the batch, on ONE thread (numpy's
+    BLAS limited to one thread for the call): the plain single-threaded baseline."""
     import oracle as O
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_limits
     rows = W.sample_tokens(shape, n_tokens)
     ex = (host["w_gate"], host["w_up"], host["w_down"])
     sh = (host["ws_gate"], host["ws_up"], host["ws_down"]) if shape.Ks else None
     times = []
-    for _ in range(repeats):
-        t0 = time.perf_counter()
-        O.moe_forward(host["x"], host["router"], shape.K, ex, sh, gate_kind=shape.gate,
-                      logit_bias=host["logit_bias"], select_bias=host["select_bias"], rows=rows)
-        times.append(time.perf_counter() - t0)
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return rows.size, times, threads
+    with threadpool_limits(limits=1):
+        for _ in range(repeats):
+            t0 = time.perf_counter()
+            O.moe_forward(host["x"], host["router"], shape.K, ex, sh, gate_kind=shape.gate,
+                          logit_bias=host["logit_bias"], select_bias=host["select_bias"], rows=rows)
+            times.append(time.perf_counter() - t0)
+    return rows.size, times, 1
+
+
+def cpu_baseline(shape: W.LayerShape, host: dict, seconds: float = 15.0, max_tokens: int = 4096):
+    """The oracle on a bounded sample sized to about ``seconds`` of one core's work."""
+    n_cal, t_cal, _ = oracle_tokens_per_s(shape, host, 8)
+    n = int(max(8, min(shape.T, max_tokens, seconds * n_cal / max(t_cal[0], 1e-6))))
+    n, times, threads = oracle_tokens_per_s(shape, host, n)
+    cores, model = host_cpu()
+    return {"value": n / times[0], "unit": UNIT, "cores": threads, "kind": "oracle",
+            "host_cores": cores, "cpu_model": model,
+            "sample": f"{n} seeded tokens of the T={shape.T} batch (routing, routed and shared experts, final "
+                      f"sum; float64 numpy on one thread), {times[0]:.1f} s"}
 
 
 def run_reference(args):
@@ -214,6 +237,7 @@ def run_reference(args):
     host = host_inputs(shape)
     # size each step's sample so that warmup + steps finish in about three minutes
     n_cal, t_cal, threads = oracle_tokens_per_s(shape, host, 4)
+    cores, model = host_cpu()
     per_token = t_cal[0] / n_cal
     budget = 180.0 / max(1, args.steps + args.warmup)
     n = int(max(1, min(shape.T, budget / per_token)))
@@ -231,8 +255,9 @@ def run_reference(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": workload_config(shape, "cpu"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "host_cores": cores, "cpu_model": model,
                              "sample": f"{n} seeded tokens of the T={shape.T} batch per step (routing, "
-                                       f"routed and shared experts, final sum, float64 numpy)"},
+                                       f"routed and shared experts, final sum, float64 numpy on one thread)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -320,19 +345,50 @@ def aggregate_rate(units_per_rank: float, world: int, max_ms: float) -> float:
     return world * units_per_rank / (max_ms * 1e-3)
 
 
-def run_ours(args):
-    from fine_grained_shared_b200 import moe as B
-
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    ranks = Ranks("nccl", dev)
-    world, rank = ranks.world, ranks.rank
-    barrier, max_over_ranks = ranks.barrier, ranks.max
-
-    shape = W.CONFIGS[args.config]
-    host = host_inputs(shape)
+def device_layer_inputs(shape: W.LayerShape, dev):
+    """(host inputs, device inputs) of a layer.  Routed experts are generated one at a time on the
+    host's cores and copied straight into stacked device tensors, so a large layer (V3: 22.5 GB of
+    expert weights) is never held whole in host memory."""
+    from concurrent.futures import ThreadPoolExecutor
+    host = W.layer_inputs(shape, with_experts=False)
     d_in = to_device(host, dev)
+    N, I, d = shape.N, shape.I, shape.d
+    wg = torch.empty((N, I, d), dtype=torch.bfloat16, device=dev)
+    wu = torch.empty((N, I, d), dtype=torch.bfloat16, device=dev)
+    wd = torch.empty((N, d, I), dtype=torch.bfloat16, device=dev)
+    with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        for e, (g, u, dn) in enumerate(ex.map(lambda e: W.expert_weights(shape, e), range(N))):
+            wg[e].copy_(g)
+            wu[e].copy_(u)
+            wd[e].copy_(dn)
+    d_in["w_gate"], d_in["w_up"], d_in["w_down"] = wg, wu, wd
+    return host, d_in
+
+
+def choose_peak(peaks: dict, timed_s: float, clk) -> tuple:
+    """(bf16 TFLOP/s, its name): the burst figure for a short timed region that held the maximum SM
+    clock, the sustained (power-capped) one for a long region or a clock below its maximum."""
+    at_max = clk is not None and clk.get("sm_mhz", 0) >= 0.97 * clk.get("sm_max_mhz", 1) \
+        and "sw_power_cap" not in clk.get("reasons", [])
+    if timed_s < 1.0 and (clk is None or at_max):
+        return float(peaks["bf16_tflops"]), "bf16_tflops"
+    return float(peaks["bf16_tflops_sustained"]), "bf16_tflops_sustained"
+
+
+def touched_weight_bytes(shape: W.LayerShape, counts) -> dict:
+    """Expert weights each GEMM launch must stream: every routed expert that received a token, and
+    the shared experts (gate/up: W_gate and W_up; down: W_down)."""
+    touched = int(sum(1 for c in counts if c > 0))
+    per_proj = 2.0 * shape.d * (touched * shape.I + shape.Ks * shape.Is)
+    return {"touched_experts": touched, "gate_up": 2 * per_proj, "down": per_proj, "layer": 3 * per_proj}
+
+
+def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: int, ranks, steps: int,
+                  warmup: int, with_e2e: bool):
+    """Time `steps` forwards of one layer on its resident inputs (CUDA events on the launching stream,
+    barrier + synchronize on both sides, max over ranks) with events around the dominant kernel, then
+    every kernel in a separate pass, then (optionally) the host-buffer entry point."""
+    world = ranks.world
     layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks,
                        d_ff_shared=shape.Is, max_tokens=shape.T, max_k=shape.K, gate=shape.gate,
                        device=local)
@@ -342,111 +398,183 @@ def run_ours(args):
     x = d_in["x"]
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream(dev)
-
-    for _ in range(max(3, args.warmup)):
+    for _ in range(warmup):
         layer.forward(x, shape.K, out)
     st = layer.status()
     if st != B.MOE_OK:
-        raise B.MoEError(st, "warm-up")
+        raise B.MoEError(st, f"{shape.name} warm-up")
 
-    # ---- device-resident timing ----
     clocks = ClockSampler(local)
     time.sleep(0.3)
     # CUDA events around the dominant kernel only: events around every launch would add their own
     # cost to the step time (a separate pass below times every kernel)
     layer.set_timing(True, kernels=[DOMINANT])
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
+    ranks.barrier()
     torch.cuda.synchronize(dev)
     start.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         layer.forward(x, shape.K, out)
     end.record(stream)
     torch.cuda.synchronize(dev)
-    barrier()
+    ranks.barrier()
     clk = clocks.stop()
     ktimes = layer.kernel_times()
     layer.set_timing(False)
     st = layer.status()
     if st != B.MOE_OK:
-        raise B.MoEError(st, "timed region")
+        raise B.MoEError(st, f"{shape.name} timed region")
+    ms_total = ranks.max(start.elapsed_time(end))
     # every kernel's time, and the launches of one forward, from a short pass outside the timed region
-    pass_steps = max(1, min(args.steps, 50))
+    pass_steps = max(1, min(steps, 50))
     layer.set_timing(True)
     for _ in range(pass_steps):
         layer.forward(x, shape.K, out)
     all_ktimes = layer.kernel_times()
     layer.set_timing(False)
-    launches_per_forward = sum(n for _, n in all_ktimes.values()) / pass_steps
-    ms_total = max_over_ranks(start.elapsed_time(end))
-    ms_step = ms_total / args.steps
-    value = aggregate_rate(shape.T, world, ms_step)
+    r = {"ms_total": ms_total, "ms_step": ms_total / steps, "clocks": clk,
+         "dominant_ms": ranks.max(ktimes[DOMINANT][0] / max(1, ktimes[DOMINANT][1])),
+         "kernel_ms": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in all_ktimes.items()},
+         "launches_per_forward": sum(n for _, n in all_ktimes.values()) / pass_steps,
+         # per-expert loads of the timed forwards (before any chunked host-buffer forward overwrites them)
+         "counts": layer.routing(shape.T, shape.K)[2].cpu().tolist()}
+    r["value"] = aggregate_rate(shape.T, world, r["ms_step"])
 
-    # per-expert loads of the timed forwards (before the chunked host-buffer forwards overwrite them)
-    counts = layer.routing(shape.T, shape.K)[2].cpu().tolist()
+    if with_e2e:
+        x_h = host["x"].pin_memory()
+        out_h = torch.empty_like(x_h).pin_memory()
+        e2e_steps = max(1, min(steps, 100))
+        for _ in range(3):
+            layer.forward_host(x_h, shape.K, out_h)
+        ranks.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            layer.forward_host(x_h, shape.K, out_h)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ranks.barrier()
+        e2e_ms = ranks.max(e0.elapsed_time(e1)) / e2e_steps
+        r["e2e"] = {"value": aggregate_rate(shape.T, world, e2e_ms), "unit": UNIT,
+                    "h2d_bytes_per_step": int(x_h.numel() * 2), "d2h_bytes_per_step": int(out_h.numel() * 2),
+                    "ms_per_step": e2e_ms}
+    layer.close()
+    return r
 
-    # ---- end to end through the host-buffer entry point ----
-    x_h = host["x"].pin_memory()
-    out_h = torch.empty_like(x_h).pin_memory()
-    e2e_steps = max(1, min(args.steps, 100))
-    for _ in range(3):
-        layer.forward_host(x_h, shape.K, out_h)
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        layer.forward_host(x_h, shape.K, out_h)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
-    e2e_value = aggregate_rate(shape.T, world, e2e_ms)
 
-    # ---- roofline of the dominant kernel (shared + routed gate/up GEMM + SwiGLU) ----
-    # bound: tensor when the routed experts' FLOPs per weight byte exceed the measured ridge
-    # (sustained bf16 FLOP/s over copy bandwidth), else HBM (the weight-streaming regime)
-    peaks, peak_src = measured_peaks()
-    k_ms, k_n = ktimes[DOMINANT]
-    k_avg_ms = max_over_ranks(k_ms / max(1, k_n))
+def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffic=None):
+    """Roofline of the dominant kernel (the shared + routed gate/up GEMM with SwiGLU): tensor-bound
+    when the routed experts' FLOPs per weight byte exceed the ridge (sustained bf16 FLOP/s over copy
+    bandwidth), else HBM-bound over the weights of the touched experts (the weight-streaming regime)."""
+    peak_flops, peak_name = choose_peak(peaks, r["ms_total"] * 1e-3, r["clocks"])
     k_flop = 4.0 * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is)
-    peak_flops = float(peaks["bf16_tflops_sustained"])
-    k_bytes = gate_up_weight_bytes(shape, counts)
-    if k_flop / k_bytes > peak_flops * 1e12 / (float(peaks["hbm_gbs"]) * 1e9):
-        roofline = {"bound": "tensor", "achieved": k_flop / (k_avg_ms * 1e-3) / 1e12, "peak": peak_flops,
-                    "unit": "TFLOP/s", "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    wb = touched_weight_bytes(shape, r["counts"])
+    k_avg_ms = r["dominant_ms"]
+    hbm = float(peaks["hbm_gbs"])
+    if k_flop / wb["gate_up"] > float(peaks["bf16_tflops_sustained"]) * 1e12 / (hbm * 1e9):
+        achieved = k_flop / (k_avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak_flops, "unit": "TFLOP/s",
+                "peak_source": f"{peak_src} {peak_name}",
+                "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
+                "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"])}
     else:
-        roofline = {"bound": "hbm", "achieved": k_bytes / (k_avg_ms * 1e-3) / 1e9, "peak": float(peaks["hbm_gbs"]),
-                    "unit": "GB/s", "peak_source": f"{peak_src} hbm_gbs"}
-    roofline["frac"] = roofline["achieved"] / roofline["peak"]
-    roofline.update({"traffic": profiled_traffic(shape),
-                     "kernel": "gateup_gemm_kernel (shared and routed experts: gate/up GEMM + SwiGLU)",
-                     "flop_per_launch": k_flop, "weight_bytes_per_launch": k_bytes, "avg_launch_ms": k_avg_ms})
-    peak = peak_flops
-    layer_tflops = world * layer_flop(shape) / (ms_step * 1e-3) / 1e12
-    launches = int(round(launches_per_forward * args.steps))
+        achieved = wb["gate_up"] / (k_avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "peak_source": f"{peak_src} hbm_gbs"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof.update({"traffic": traffic, "kernel": "gateup_gemm_kernel (shared and routed experts: gate/up GEMM + "
+                                               "SwiGLU)",
+                 "flop_per_launch": k_flop, "weight_bytes_per_launch": wb["gate_up"], "avg_launch_ms": k_avg_ms})
+    return roof, peak_flops, peak_name
 
+
+def hbm_fractions(shape: W.LayerShape, r: dict, peaks: dict) -> dict:
+    """Each expert GEMM's and the whole layer's rate over the touched experts' weight bytes, as a
+    fraction of the measured copy bandwidth (the roofline of the weight-streaming shapes)."""
+    wb = touched_weight_bytes(shape, r["counts"])
+    hbm = float(peaks["hbm_gbs"])
+    out = {"touched_experts": wb["touched_experts"], "weight_bytes": wb["layer"]}
+    for k in ("gate_up", "down"):
+        ms = r["kernel_ms"].get(k, 0.0)
+        out[f"{k}_gbs"] = wb[k] / (ms * 1e-3) / 1e9 if ms > 0 else None
+        out[f"{k}_frac"] = out[f"{k}_gbs"] / hbm if ms > 0 else None
+    out["layer_gbs"] = wb["layer"] / (r["ms_step"] * 1e-3) / 1e9
+    out["layer_frac"] = out["layer_gbs"] / hbm
+    return out
+
+
+PER_CONFIG = ("2b", "16b_decode", "v3")
+
+
+def run_ours(args):
+    from fine_grained_shared_b200 import moe as B
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    warmup = max(3, args.warmup)
+
+    shape = W.CONFIGS[args.config]
+    host = host_inputs(shape)
+    d_in = to_device(host, dev)
+    r = measure_layer(B, shape, host, d_in, dev, local, ranks, args.steps, warmup, with_e2e=True)
+    del d_in
+    torch.cuda.empty_cache()
+
+    peaks, peak_src = measured_peaks()
+    roofline, peak_flops, peak_name = roofline_of(shape, r, peaks, peak_src, profiled_traffic(shape))
+    layer_tflops = world * layer_flop(shape) / (r["ms_step"] * 1e-3) / 1e12
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+        "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": warmup, "ms_per_step": r["ms_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(shape, f"replicas{world}" if world > 1 else "single"),
         "tflops": layer_tflops,
-        "tflops_frac_of_peak": layer_tflops / (world * peak),
+        "tflops_frac_of_peak": layer_tflops / (world * peak_flops),
+        "tflops_peak": f"{peak_src} {peak_name}",
         "roofline": roofline,
-        "kernel_ms_per_step": {k: (v[0] / v[1] if v[1] else 0.0) for k, v in all_ktimes.items()},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_h.numel() * 2),
-                "d2h_bytes_per_step": int(out_h.numel() * 2), "ms_per_step": e2e_ms},
-        "gpu_launches": launches,
-        "clocks": clk,
+        "kernel_ms_per_step": r["kernel_ms"],
+        "e2e": r["e2e"],
+        "gpu_launches": int(round(r["launches_per_forward"] * args.steps)),
+        "clocks": r["clocks"],
     }
+    if roofline["bound"] == "hbm":
+        line["hbm"] = hbm_fractions(shape, r, peaks)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, times, threads = oracle_tokens_per_s(shape, host, args.cpu_sample)
-        line["cpu_baseline"] = {"value": n / times[0], "unit": UNIT, "cores": threads, "kind": "oracle",
-                                "sample": f"{n} seeded tokens of the T={shape.T} batch (routing, routed and "
-                                          f"shared experts, final sum; float64 numpy)"}
-    layer.close()
+        line["cpu_baseline"] = cpu_baseline(shape, host)
+
+    # the other single-GPU workloads, measured after the headline one: ms per step, tokens/s and the
+    # roofline that bounds each (tensor for the 2B layer, HBM over the touched experts' weights for
+    # the 16B decode and V3 layers)
+    if not args.no_per_config:
+        per = {}
+        for name in PER_CONFIG:
+            if name == args.config:
+                continue
+            cs = W.CONFIGS[name]
+            t0 = time.perf_counter()
+            chost, cdev = device_layer_inputs(cs, dev)
+            gen_s = time.perf_counter() - t0
+            # small steps are timed over at least ~0.1 s of forwards
+            steps = args.steps if cs.T >= 1024 else max(args.steps, 500)
+            cr = measure_layer(B, cs, chost, cdev, dev, local, ranks, steps, warmup, with_e2e=False)
+            del cdev
+            torch.cuda.empty_cache()
+            croof, cpeak, cpeak_name = roofline_of(cs, cr, peaks, peak_src, profiled_traffic(cs))
+            ctf = world * layer_flop(cs) / (cr["ms_step"] * 1e-3) / 1e12
+            per[name] = {"workload": workload_config(cs, f"replicas{world}" if world > 1 else "single")["workload"],
+                         "steps": steps, "ms_per_step": cr["ms_step"], "tokens_per_s": cr["value"],
+                         "tflops": ctf, "tflops_frac_of_peak": ctf / (world * cpeak),
+                         "tflops_peak": f"{peak_src} {cpeak_name}", "roofline": croof,
+                         "hbm": hbm_fractions(cs, cr, peaks), "kernel_ms_per_step": cr["kernel_ms"],
+                         "clocks": cr["clocks"], "l2": l2_note(cs), "input_generation_s": gen_s}
+            line["gpu_launches_per_config"] = line.get("gpu_launches_per_config", 0) + \
+                int(round(cr["launches_per_forward"] * steps))
+        line["per_config"] = per
     if rank == 0:
         print(json.dumps(line), flush=True)
     ranks.close()

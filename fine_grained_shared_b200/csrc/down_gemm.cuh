@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int st = 0; st < kGemmStages; ++st) {
         if (issued > st) {
           const int n = (issued - 1 - st) / kGemmStages + 1;
-          mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+          mbar_wait_drain(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns);
         }
       }
     }
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     umma_commit_pair_multicast(teardown, 0x1);
-    mbar_wait(teardown, 0, a.timeout_ns, nullptr);
+    mbar_wait_drain(teardown, 0, a.timeout_ns);
   } else if (warp >= 2) {
     // ------------------------------ epilogue ----------------------------------
     const int q = warp & 3;

@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       for (int st = 0; st < kGuStages; ++st) {
         if (issued > st) {
           const int n = (issued - 1 - st) / kGuStages + 1;
-          mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+          mbar_wait_drain(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns);
         }
       }
     }
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       }
     }
     umma_commit(teardown);
-    mbar_wait(teardown, 0, a.timeout_ns, nullptr);
+    mbar_wait_drain(teardown, 0, a.timeout_ns);
   } else if (warp >= 2) {
     // ------------------------------ epilogue ----------------------------------
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31

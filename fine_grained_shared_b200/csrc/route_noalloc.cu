@@ -113,7 +113,9 @@ extern "C" moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_mode
   if (gate != MOE_GATE_SOFTMAX && gate != MOE_GATE_SIGMOID_BIASED) return MOE_ERR_INVALID_ARG;
   if (d_model % 16) return MOE_ERR_ALIGNMENT;
   if (T == 0) return MOE_OK;
-  if (!x || !router || !router->weight || !idx || !gate_out || !counts || !offsets) return MOE_ERR_INVALID_ARG;
+  if (!x || !router || !router->weight || !idx || !gate_out || !counts || !offsets || !err)
+    return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(err) & 3u) return MOE_ERR_ALIGNMENT;
   const bool sigmoid = gate == MOE_GATE_SIGMOID_BIASED;
   if (sigmoid ? router->logit_bias != nullptr : router->select_bias != nullptr) return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {x, router->weight, router->logit_bias, router->select_bias, idx, gate_out, counts, offsets};
@@ -134,7 +136,7 @@ extern "C" moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_mode
       !encode_2d(&te, router->weight, N, d_model, static_cast<uint32_t>(Npad)))
     return MOE_ERR_CUDA;
 
-  // scratch layout: [0] CTA completion counter, [4] error word,
+  // scratch layout: [0] CTA completion counter,
   // [256, +1028) row starts, [1536, +1028) and [2816, +1028) m-tile starts,
   // [4096, ...) block histograms
   uint32_t* done = reinterpret_cast<uint32_t*>(scratch);
@@ -156,7 +158,7 @@ extern "C" moe_status moe_route_noalloc(const void* x, int64_t T, int32_t d_mode
   ra.mtile_start = reinterpret_cast<int32_t*>(scratch + 1536);
   ra.mtile128_start = reinterpret_cast<int32_t*>(scratch + 2816);
   ra.done_counter = done;
-  ra.err = err ? err : reinterpret_cast<uint32_t*>(scratch + 4);
+  ra.err = err;
   ra.timeout_ns = kTimeoutNs;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     for (int st = 0; st < S; ++st) {
       if (issued > st) {
         const int n = (issued - 1 - st) / S + 1;
-        mbar_wait(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns, nullptr);
+        mbar_wait_drain(&full[st], static_cast<uint32_t>((n - 1) & 1), a.timeout_ns);
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
     }
     if (ok) umma_commit(acc_full);
     umma_commit(teardown);
-    mbar_wait(teardown, 0, a.timeout_ns, nullptr);
+    mbar_wait_drain(teardown, 0, a.timeout_ns);
   } else if (warp >= 2) {
     // ---------------- epilogue: one token per thread ----------------
     const int q = warp & 3;
@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
               key = z;  // softmax is monotone in z: rank on the logits
               sv = 0.f;
             }
+            // a NaN key (a non-finite token or router row) ranks below every
+            // number; the index order then still fills the K slots with
+            // distinct experts in [0, N)
+            if (isnan(key)) key = -INFINITY;
             // insert (key, col) into the list ordered by (key descending,
             // index ascending); an element pushed down keeps competing by the
             // same order, so ties always go to the lower expert index
@@ -256,7 +260,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
         for (int k = 0; k < K; ++k) {
           a.idx[static_cast<size_t>(t) * K + k] = ti[k];
           a.gate[static_cast<size_t>(t) * K + k] = g[k];
-          atomicAdd(&hist[ti[k]], 1);
+          if (ti[k] < a.N) atomicAdd(&hist[ti[k]], 1);
         }
       }
     }
@@ -423,9 +427,11 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
       if (SIGMOID) {
         const float sv = 1.f / (1.f + __expf(-z));
         sval[i] = sv;
-        key[i] = sv + (a.select_bias ? a.select_bias[i] : 0.f);
+        const float k = sv + (a.select_bias ? a.select_bias[i] : 0.f);
+        key[i] = isnan(k) ? -INFINITY : k;  // NaN ranks below every number
       } else {
-        key[i] = z + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
+        const float k = z + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
+        key[i] = isnan(k) ? -INFINITY : k;
       }
     }
     __syncwarp();

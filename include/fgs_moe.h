@@ -208,11 +208,20 @@ moe_status moe_kernel_times(moe_handle h, float* total_ms, int32_t* launches);
  * Runs on the calling thread's current device, on `stream`.  x: bf16 [T, d]
  * device; router as for moe_forward; gate: moe_gate_kind; outputs (device,
  * caller-allocated): idx int32 [T, K], gate_out float32 [T, K], counts int32
- * [mN], offsets int32 [mN + 1] -- the same values moe_get_routing returns after
- * moe_forward.  err: optional device word that receives error bits (OR-ed) if
- * a device-side wait runs out; NULL keeps them in the scratch array.
+ * [mN], offsets int32 [mN + 1].  These are the values moe_get_routing returns
+ * after moe_forward on the same inputs: idx, counts and offsets bit for bit
+ * (batches of more than 256 tokens run the very same kernel; for smaller ones
+ * moe_forward computes the logits on the CUDA cores in another summation
+ * order, so a token whose K-th and (K+1)-th keys are closer than float32
+ * rounding may pick differently), gates within 1e-5.
+ * err: required device word (4-byte aligned) into which the kernel ORs its
+ * error bits if a device-side wait runs out (the outputs are then not valid);
+ * the caller clears it and reads it after the stream has finished.
  * Limits: T <= 65536 (else MOE_ERR_SHAPE: the static scratch is full),
- * mN <= 256, K <= 8, d a multiple of 16, 16-byte aligned pointers.
+ * mN <= 256, K <= 8, d a multiple of 16, 16-byte aligned pointers (x, router
+ * and its biases, idx, gate_out, counts, offsets).  A null input or output
+ * pointer, err included, -> MOE_ERR_INVALID_ARG; err not 4-byte aligned ->
+ * MOE_ERR_ALIGNMENT.
  * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  * The first call on a device looks up the scratch array's device address and
  * sets the kernels' shared-memory limits; make that first call before any

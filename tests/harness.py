@@ -83,16 +83,72 @@ def run(layer, x, K):
     return out
 
 
-def oracle_experts(shape: W.LayerShape, host: dict):
+def oracle_experts(shape: W.LayerShape, host: dict, prefetch=None):
+    """The routed experts' weights for the oracle, from the seeded generator:
+    the stacked host tensors when the layer is small, else a callable that
+    generates (and keeps) each expert on first use.  ``prefetch`` lists experts
+    to generate up front, in parallel on the host's cores."""
     if "w_gate" in host:
         return (host["w_gate"], host["w_up"], host["w_down"])
     cache = {}
+    if prefetch is not None:
+        ids = sorted({int(e) for e in prefetch})
+        workers = min(32, os.cpu_count() or 1)
+        with ThreadPoolExecutor(max_workers=workers) as ex:
+            for e, w in zip(ids, ex.map(lambda e: W.expert_weights(shape, e), ids)):
+                cache[e] = w
 
     def fn(e):
         if e not in cache:
             cache[e] = W.expert_weights(shape, e)
         return cache[e]
     return fn
+
+
+def stratified_rows(shape: W.LayerShape, ref: O.Routing, tile_rows: int = 128, seed: int = 0):
+    """Tokens that put at least one compared row in every GEMM tile of the layer.
+
+    The expert GEMMs run over 128-row m-tiles of each expert's segment of the
+    expert-ordered rows (the routed tiles) and over 128-token blocks of x (the
+    shared experts' tiles).  For every (expert, m-tile) this picks one token
+    whose row lands in that tile -- a seeded random one, its last row for the
+    expert's ragged tail -- and one token of every 128-token block of x, plus
+    the first and the last token.  Tokens with a near-tie at the selection
+    boundary are passed over (another token of the tile stands in).  The tiles
+    come from the oracle's own counting sort of its selection, which the GPU's
+    permutation must equal bit for bit on every other token.
+
+    Returns (sorted token ids, tiles covered, tiles in all)."""
+    rng = np.random.default_rng(seed)
+    ok = ref.gap >= GAP_EXEMPT
+    perm = O.expert_permutation(ref.idx, shape.N)
+    chosen = set()
+    covered = total = 0
+
+    def pick(cands):
+        cands = [int(t) for t in cands if ok[t]]
+        if not cands:
+            return False
+        chosen.add(cands[int(rng.integers(len(cands)))])
+        return True
+
+    for e in range(shape.N):
+        lo, hi = int(perm.offsets[e]), int(perm.offsets[e + 1])
+        for m0 in range(0, hi - lo, tile_rows):
+            total += 1
+            rows = perm.src[lo + m0: min(hi, lo + m0 + tile_rows)]
+            if ok[rows[-1]] and m0 + tile_rows >= hi - lo:   # the ragged tail's last row
+                chosen.add(int(rows[-1]))
+                covered += 1
+            elif pick(rows):
+                covered += 1
+    for b0 in range(0, shape.T, tile_rows):
+        total += 1
+        covered += pick(range(b0, min(shape.T, b0 + tile_rows)))
+    for t in (0, shape.T - 1):
+        if ok[t]:
+            chosen.add(t)
+    return np.array(sorted(chosen), dtype=np.int64), covered, total
 
 
 def oracle_shared(shape, host):

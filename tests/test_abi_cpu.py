@@ -113,6 +113,31 @@ def test_fp8_quantize_arguments_are_checked_before_any_cuda_call():
     assert blocks(a, 3, 0, 128, b, c, None) == B.MOE_OK
 
 
+def test_noalloc_routing_arguments_are_checked_before_any_cuda_call():
+    """Fake, never dereferenced device addresses: every case returns before a CUDA call."""
+    lib = B.lib()
+    x, w, o, e = 0x10000, 0x20000, 0x30000, 0x40000
+    r = B.moe_router(w, None, None)
+    rs = B.moe_router(w, None, 0x50000)            # a selection bias, which only the sigmoid gate takes
+    f = lib.moe_route_noalloc
+    soft, sig = B.MOE_GATE_SOFTMAX, B.MOE_GATE_SIGMOID_BIASED
+    call = lambda T=8, d=256, rt=r, N=16, g=soft, K=4, err=e, xp=x: f(xp, T, d, ctypes.byref(rt), N, g, K,
+                                                                      o, o, o, o, err, None)
+    assert call(T=65537) == B.MOE_ERR_SHAPE           # beyond the static scratch
+    assert call(T=-1) == B.MOE_ERR_SHAPE
+    assert call(N=257, K=4) == B.MOE_ERR_UNSUPPORTED
+    assert call(K=9, N=64) == B.MOE_ERR_UNSUPPORTED
+    assert call(K=0) == B.MOE_ERR_INVALID_ARG
+    assert call(g=5) == B.MOE_ERR_INVALID_ARG
+    assert call(d=200) == B.MOE_ERR_ALIGNMENT
+    assert call(err=None) == B.MOE_ERR_INVALID_ARG     # a timeout must have somewhere to be reported
+    assert call(err=e + 2) == B.MOE_ERR_ALIGNMENT
+    assert call(xp=None) == B.MOE_ERR_INVALID_ARG
+    assert call(xp=x + 8) == B.MOE_ERR_ALIGNMENT
+    assert call(rt=rs, g=soft) == B.MOE_ERR_INVALID_ARG
+    assert call(T=0) == B.MOE_OK                       # nothing to route
+
+
 def test_status_strings():
     for v, name in [(0, "MOE_OK"), (1, "MOE_ERR_INVALID_ARG"), (7, "MOE_ERR_TIMEOUT"), (99, "MOE_ERR_UNKNOWN")]:
         assert B.status_string(v) == name

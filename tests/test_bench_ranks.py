@@ -76,3 +76,53 @@ def test_fp8_reference_arm_times_the_fp8_oracle(monkeypatch):
     assert line["impl"] == "reference" and line["metric"] == bench.FP8_METRIC and line["unit"] == "GB/s"
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["config"]["workload"].startswith("16b_prefill")
+
+
+def test_reference_arm_times_the_oracle_on_one_thread(monkeypatch):
+    import json
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--config", "tiny", "--steps", "2",
+                                      "--warmup", "1"])
+    out = io.StringIO()
+    with contextlib.redirect_stdout(out):
+        bench.main()
+    line = json.loads(out.getvalue().strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["cores"] == 1 and line["cpu_baseline"]["host_cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_peak_follows_the_length_and_clock_of_the_timed_region():
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1667.0, "bf16_tflops_sustained": 1397.0}
+    at_max = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1400.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.choose_peak(peaks, 0.04, at_max) == (1667.0, "bf16_tflops")
+    assert bench.choose_peak(peaks, 0.04, None) == (1667.0, "bf16_tflops")
+    assert bench.choose_peak(peaks, 2.5, at_max) == (1397.0, "bf16_tflops_sustained")
+    assert bench.choose_peak(peaks, 0.04, capped) == (1397.0, "bf16_tflops_sustained")
+
+
+def test_roofline_of_the_dominant_kernel_from_its_own_numbers():
+    import workloads as W
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1667.0, "bf16_tflops_sustained": 1397.0}
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    shape = W.CONFIGS["16b_prefill"]
+    r = {"ms_total": 41.0, "ms_step": 2.05, "clocks": clk, "dominant_ms": 1.2252, "counts": [1536] * 64,
+         "kernel_ms": {"gate_up": 1.2252, "down": 0.56}}
+    roof, peak, _ = bench.roofline_of(shape, r, peaks, "measured")
+    flop = 4.0 * 16384 * 2048 * (6 * 1408 + 2 * 1408)
+    assert roof["bound"] == "tensor" and roof["flop_per_launch"] == flop
+    assert roof["achieved"] == pytest.approx(flop / 1.2252e-3 / 1e12)
+    assert roof["frac"] == pytest.approx(roof["achieved"] / 1667.0) and peak == 1667.0
+    decode = W.CONFIGS["16b_decode"]
+    counts = [6] * 30 + [0] * 34                  # 30 of the 64 experts touched
+    r = dict(r, ms_total=20.0, ms_step=0.18, dominant_ms=0.11, counts=counts,
+             kernel_ms={"gate_up": 0.11, "down": 0.055})
+    roof, _, _ = bench.roofline_of(decode, r, peaks, "measured")
+    wbytes = 2 * 2 * 2048 * (30 * 1408 + 2 * 1408)
+    assert roof["bound"] == "hbm" and roof["weight_bytes_per_launch"] == wbytes
+    assert roof["achieved"] == pytest.approx(wbytes / 0.11e-3 / 1e9)
+    f = bench.hbm_fractions(decode, r, peaks)
+    assert f["down_gbs"] == pytest.approx(wbytes / 2 / 0.055e-3 / 1e9)
+    assert f["layer_frac"] == pytest.approx(1.5 * wbytes / 0.18e-3 / 1e9 / 6500.0)

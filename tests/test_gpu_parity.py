@@ -57,7 +57,9 @@ def _gpu_rows(out, rows):
 
 def _check_layer(shape, host, dev, rows, routing=None):
     """Whole output and the routed / shared terms alone, on ``rows``."""
-    experts = H.oracle_experts(shape, host)
+    ref_routing_rows = routing.idx[rows] if routing is not None else None
+    experts = H.oracle_experts(shape, host, prefetch=None if ref_routing_rows is None
+                               else np.unique(ref_routing_rows))
     shared = H.oracle_shared(shape, host)
     ref_routing = routing if routing is not None else H.oracle_routing(shape, host)
     cases = [(0, "output")]
@@ -88,15 +90,20 @@ def test_small_shapes_every_token(name):
     _check_layer(shape, host, dev, rows, ref)
 
 
-@pytest.mark.parametrize("name,sample", [("2b", 192), ("16b_prefill", 96), ("16b_decode", 32), ("v3", 12)])
-def test_full_size_layers(name, sample):
+@pytest.mark.parametrize("name", ["2b", "16b_prefill", "16b_decode", "v3"])
+def test_full_size_layers(name):
+    """The whole routing on every token, and the output on a token set that
+    puts a compared row in every (expert, 128-row m-tile) GEMM tile and in
+    every 128-token tile of the shared experts."""
     shape = W.CONFIGS[name]
     host, dev = H.device_inputs(shape)
     ref = H.oracle_routing(shape, host)
-    rows = W.sample_tokens(shape, sample)
-    rows = rows[ref.gap[rows] >= H.GAP_EXEMPT]
+    rows, covered, total = H.stratified_rows(shape, ref)
+    assert covered == total, f"{total - covered} of {total} GEMM tiles have no comparable token"
+    if shape.T <= 512:          # a decode batch: every token
+        rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
     res = _check_layer(shape, host, dev, rows, ref)
-    print(f"{name}: exempt tokens {res['exempt']}, compared rows {rows.size}, "
+    print(f"{name}: exempt tokens {res['exempt']}, compared rows {rows.size}, tiles covered {covered}/{total}, "
           + ", ".join(f"{k}: max err {v[0]:.2e} rms err {v[2]:.2e} rms {v[1]:.2e}"
                       for k, v in res.items() if k != "exempt"))
 
@@ -160,6 +167,39 @@ def test_duplicated_expert_rows_tie_exactly():
     H.run(layer, dev["x"], shape.K)
     idx = layer.routing(shape.T, shape.K)[0].cpu().numpy()
     np.testing.assert_array_equal(idx, ref.idx)
+
+
+@pytest.mark.parametrize("T", [300, 100])  # tensor-core router, CUDA-core router
+def test_non_finite_tokens_still_route_to_valid_experts(T):
+    """A token whose row holds a NaN (or an infinity) has NaN affinities.  Its
+    K slots must still name K distinct experts in [0, mN) (a NaN key ranks
+    below every number, ties to the lower index), the counts must add up to
+    T*K, and every other token must be unaffected."""
+    shape = LS("nan_rows", T=T, d=256, N=24, I=64, K=4, Ks=1, Is=64, sigma=0.05, seed=28)
+    host = W.layer_inputs(shape)
+    bad = [0, 5, T // 2, T - 1]
+    x = host["x"].clone()
+    x[bad[0], 3] = float("nan")
+    x[bad[1], :] = float("nan")
+    x[bad[2], 7] = float("inf")
+    x[bad[3], 0] = float("-inf")
+    host_bad = dict(host, x=x)
+    _, dev = H.device_inputs(shape, host_bad)
+    layer = H.make_layer(shape, dev)
+    out = H.run(layer, dev["x"], shape.K)
+    idx, gate, counts, offsets, src = (t.cpu().numpy() for t in layer.routing(shape.T, shape.K))
+    assert ((idx >= 0) & (idx < shape.N)).all()
+    assert all(len(set(r)) == shape.K for r in idx.tolist())
+    assert counts.sum() == T * shape.K
+    np.testing.assert_array_equal(counts, np.bincount(idx.ravel(), minlength=shape.N))
+    good = np.setdiff1d(np.arange(T), bad)
+    ref = H.oracle_routing(shape, host)           # the finite tokens' routing does not depend on the others
+    ok = good[ref.gap[good] >= H.GAP_EXEMPT]
+    np.testing.assert_array_equal(idx[ok], ref.idx[ok])
+    np.testing.assert_allclose(gate[ok], ref.gate[ok], rtol=0, atol=H.GATE_TOL)
+    h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), routing=ref, rows=ok)
+    H.compare_output(_gpu_rows(out, ok), h, "finite tokens beside non-finite ones")
 
 
 def test_zero_router_sends_every_token_to_the_first_experts():
