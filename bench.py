@@ -221,8 +221,9 @@ def oracle_tokens_per_s(shape: W.LayerShape, host: dict, n_tokens: int, repeats:
 
 
 def cpu_baseline(shape: W.LayerShape, host: dict, seconds: float = 15.0, max_tokens: int = 4096):
-    """The oracle on a bounded sample sized to about ``seconds`` of one core's work."""
-    n_cal, t_cal, _ = oracle_tokens_per_s(shape, host, 8)
+    """The oracle on a bounded sample sized to about ``seconds`` of one core's work (calibrated on 64
+    tokens, which already pay the per-expert weight conversions)."""
+    n_cal, t_cal, _ = oracle_tokens_per_s(shape, host, 64)
     n = int(max(8, min(shape.T, max_tokens, seconds * n_cal / max(t_cal[0], 1e-6))))
     n, times, threads = oracle_tokens_per_s(shape, host, n)
     cores, model = host_cpu()
@@ -507,6 +508,25 @@ def hbm_fractions(shape: W.LayerShape, r: dict, peaks: dict) -> dict:
 PER_CONFIG = ("2b", "16b_decode", "v3")
 
 
+def estimate_step_s(B, shape: W.LayerShape, d_in: dict, dev, local: int) -> float:
+    """Seconds per forward of a layer, from 3 warm forwards (outside any timed region)."""
+    layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks,
+                       d_ff_shared=shape.Is, max_tokens=shape.T, max_k=shape.K, gate=shape.gate, device=local)
+    shared = (d_in["ws_gate"], d_in["ws_up"], d_in["ws_down"]) if shape.Ks else None
+    layer.set_weights(d_in["router"], (d_in["w_gate"], d_in["w_up"], d_in["w_down"]), shared,
+                      logit_bias=d_in["logit_bias"], select_bias=d_in["select_bias"])
+    out = torch.empty_like(d_in["x"])
+    layer.forward(d_in["x"], shape.K, out)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(3):
+        layer.forward(d_in["x"], shape.K, out)
+    torch.cuda.synchronize(dev)
+    dt = (time.perf_counter() - t0) / 3
+    layer.close()
+    return dt
+
+
 def run_ours(args):
     from fine_grained_shared_b200 import moe as B
 
@@ -559,8 +579,9 @@ def run_ours(args):
             t0 = time.perf_counter()
             chost, cdev = device_layer_inputs(cs, dev)
             gen_s = time.perf_counter() - t0
-            # small steps are timed over at least ~0.1 s of forwards
-            steps = args.steps if cs.T >= 1024 else max(args.steps, 500)
+            # each workload is timed over at least ~0.5 s of forwards, so that the clock sampler
+            # (one sample per 100 ms) sees the timed region; the warm-up gives the step time
+            steps = max(args.steps, int(0.5 / max(estimate_step_s(B, cs, cdev, dev, local), 1e-6)))
             cr = measure_layer(B, cs, chost, cdev, dev, local, ranks, steps, warmup, with_e2e=False)
             del cdev
             torch.cuda.empty_cache()

@@ -27,6 +27,7 @@
 #include <vector>
 
 #include "../../include/fgs_moe.h"
+#include "decode_gemm.cuh"
 #include "down_gemm.cuh"
 #include "gateup_gemm.cuh"
 #include "permute.cuh"
@@ -35,6 +36,15 @@
 using namespace fgs;
 
 static_assert(kGemmBM == kExpertRowAlign, "GEMM pair tiles must not straddle two experts");
+static_assert(kDecBoxRowsW == kGuBoxRowsB && kDecBoxRowsW == kBoxRowsB,
+              "the decode GEMMs share the weight maps of the prefill GEMMs");
+
+// Batches of at most this many tokens run the expert FFNs on the
+// weight-streaming decode GEMMs (decode_gemm.cuh); larger ones on the
+// 128-row-tile GEMMs.
+#ifndef FGS_DECODE_MAX_T
+#define FGS_DECODE_MAX_T 64
+#endif
 
 namespace {
 
@@ -42,6 +52,8 @@ constexpr int kMaxRouted = 256;
 constexpr int kMaxK = 8;
 constexpr int64_t kMaxTokens = int64_t(1) << 20;
 constexpr uint64_t kTimeoutNs = 2000ull * 1000 * 1000;  // 2 s: no legitimate wait comes close
+constexpr int64_t kDecodeMaxT = FGS_DECODE_MAX_T;
+constexpr int kDecMaxCtas = 148;  // the decode GEMMs' grid: one CTA per SM, at most this many
 // the host-buffer forward pipelines batches of at least 2 x kHostChunkRows tokens in up to kHostChunks chunks
 constexpr int kHostChunks = 5;
 constexpr int64_t kHostChunkRows = 2048;
@@ -86,9 +98,19 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 struct Layout {
   // byte offsets into the workspace
   size_t err, done, tile_ctr, tok_done, small_logits, idx, gate, slot, src, bc, counts, offsets, row_start, mtile,
-      mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, total;
+      mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, dec_part_gu, dec_part_dn, dec_ctr_gu, dec_ctr_dn,
+      dec_ctr_bytes, total;
   int64_t P, Tpad, nblk;
 };
+
+// Tiles a decode GEMM launch can have: 32-token blocks of the shared experts'
+// rows, and of each routed expert's rows (at most one partial block per
+// expert that received a token), times the weight blocks.
+int64_t decode_max_tiles(int64_t T, int64_t K, int64_t N, int64_t routed_wb, int64_t shared_wb) {
+  const int64_t tb = (T + kDecTB - 1) / kDecTB;
+  const int64_t routed_tb = std::min<int64_t>(N, T * K) + (T * K + kDecTB - 1) / kDecTB;
+  return tb * shared_wb + routed_tb * routed_wb;
+}
 
 Layout make_layout(const moe_config& c) {
   Layout L{};
@@ -126,6 +148,17 @@ Layout make_layout(const moe_config& c) {
   L.ys = take(c.n_shared > 0 ? L.Tpad * int64_t(c.d_model) * 2 : 0);
   L.xdev = take(Tm * c.d_model * 2);
   L.outdev = take(Tm * c.d_model * 2);
+  // the decode GEMMs' stream-K partial sums and per-quarter tile counters
+  const int64_t Td = std::min<int64_t>(Tm, kDecodeMaxT);
+  const int64_t sh_cols = int64_t(c.n_shared) * c.d_ff_shared;
+  const int64_t gu_tiles = decode_max_tiles(Td, Km, N, (c.d_ff + kDecWB - 1) / kDecWB, (sh_cols + kDecWB - 1) / kDecWB);
+  const int64_t dn_tiles =
+      decode_max_tiles(Td, Km, N, (c.d_model + kDecWB - 1) / kDecWB, (c.d_model + kDecWB - 1) / kDecWB);
+  L.dec_part_gu = take(dec_partials_bytes<true>(kDecMaxCtas));
+  L.dec_part_dn = take(dec_partials_bytes<false>(kDecMaxCtas));
+  L.dec_ctr_gu = take(size_t(gu_tiles) * 4 * 4 + size_t(dn_tiles) * 4 * 4);
+  L.dec_ctr_dn = L.dec_ctr_gu + size_t(gu_tiles) * 4 * 4;
+  L.dec_ctr_bytes = size_t(gu_tiles + dn_tiles) * 4 * 4;
   L.total = o;
   return L;
 }
@@ -180,7 +213,8 @@ struct moe_ctx {
   int last_K = 0;
   // TMA descriptors: workspace ones are fixed, the others follow the caller's pointers
   CUtensorMap tm_xperm, tm_h, tm_hs;
-  MapCache tm_x, tm_router, tm_wg, tm_wu, tm_wd, tm_swg, tm_swu, tm_swd;
+  CUtensorMap tm_xperm32, tm_h32, tm_hs32;  // 32-row token boxes of the decode GEMMs
+  MapCache tm_x, tm_x32, tm_router, tm_wg, tm_wu, tm_wd, tm_swg, tm_swu, tm_swd;
   // host-buffer forward: copy streams and per-chunk events, created on first use
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
   cudaEvent_t host_start = nullptr, in_done[kHostChunks] = {}, fwd_done[kHostChunks] = {};
@@ -279,7 +313,12 @@ cudaError_t set_kernel_attrs() {
   const int us = static_cast<int>(gateup_smem_bytes());
   if ((e = cudaFuncSetAttribute(gateup_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
   const int gs = static_cast<int>(gemm_smem_bytes());
-  return cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs);
+  if ((e = cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
+  if ((e = cudaFuncSetAttribute(decode_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(dec_smem_bytes<true>()))))
+    return e;
+  return cudaFuncSetAttribute(decode_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(dec_smem_bytes<false>()));
 }
 
 // Re-encode a cached descriptor when the caller's pointer (or row count) changes.
@@ -300,6 +339,14 @@ cudaError_t launch_down(int pairs, cudaStream_t s, bool pdl, const CUtensorMap& 
                         const CUtensorMap& As, const CUtensorMap& Bs, const GemmArgs& ga) {
   return launch_pdl(down_gemm_kernel, dim3(2 * pairs), dim3(kGemmThreads), gemm_smem_bytes(), s, 2, pdl, A, B, As, Bs,
                     ga);
+}
+
+template <bool GU>
+cudaError_t launch_decode(int ctas, cudaStream_t s, bool pdl, const CUtensorMap& W0, const CUtensorMap& W1,
+                          const CUtensorMap& X, const CUtensorMap& Ws0, const CUtensorMap& Ws1, const CUtensorMap& Xs,
+                          const DecodeArgs& da) {
+  return launch_pdl(decode_gemm_kernel<GU>, dim3(ctas), dim3(kDecThreads), dec_smem_bytes<GU>(), s, 1, pdl, W0, W1, X,
+                    Ws0, Ws1, Xs, da);
 }
 
 cudaError_t launch_gateup(int ctas, cudaStream_t s, bool pdl, const CUtensorMap& A, const CUtensorMap& G,
@@ -425,11 +472,17 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
     return MOE_ERR_NOMEM;
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
+  ok = ok && cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
-  if (c.n_shared > 0)
+  ok = ok && encode_bf16(&h->tm_xperm32, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kDecBoxRowsX, 2);
+  ok = ok && encode_bf16(&h->tm_h32, h->ws + h->L.h, 1, h->L.P, c.d_ff, kDecBoxRowsX, 2);
+  if (c.n_shared > 0) {
     ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kBoxRowsA, 2);
+    ok = ok &&
+         encode_bf16(&h->tm_hs32, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kDecBoxRowsX, 2);
+  }
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
@@ -479,7 +532,9 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
 
   // descriptors that follow the caller's pointers
   static_assert(kGuBoxRowsA == kRouterBM, "x serves as A of the router and of the shared gate/up GEMM");
+  const bool decode = T <= kDecodeMaxT;
   bool ok = refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2);
+  if (decode) ok = ok && refresh(h->tm_x32, x, T, 1, T, d, kDecBoxRowsX, 2);
 
   ok = ok && refresh(h->tm_router, router->weight, 0, 1, N, d, (uint32_t)Npad, 2);
   ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, kGuBoxRowsB, 3);
@@ -568,8 +623,79 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
       return MOE_ERR_CUDA;
   }
 
+  // ---- the expert GEMMs of a small batch: weight-streaming, stream-K ----
+  if (decode && (do_routed || do_shared)) {
+    const int ctas = std::min(h->num_sms, kDecMaxCtas);
+    DecodeArgs g{};
+    if (do_routed) {
+      g.num_groups = (int)N;
+      g.counts = ra.counts;
+      g.row_start = ra.row_start;
+      g.n_wb = ceil_div(I, kDecWB);
+      g.num_kb = ceil_div(d, kDecBK);
+      g.out = h->at<__nv_bfloat16>(L.h);
+      g.ld_out = (int)I;
+      g.n_limit = (int)I;
+    }
+    if (do_shared) {
+      g.sh_rows = (int)T;
+      g.sh_n_wb = ceil_div(Ks * Is, kDecWB);
+      g.sh_J = 1;
+      g.sh_kb_per_j = ceil_div(d, kDecBK);
+      g.sh_out = h->at<__nv_bfloat16>(L.hs);
+      g.sh_ld_out = (int)(Ks * Is);
+      g.sh_n_limit = (int)(Ks * Is);
+    }
+    g.partials = h->at<float>(L.dec_part_gu);
+    g.tile_ctr = h->at<uint32_t>(L.dec_ctr_gu);
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
+    // an absent part's maps are never read; the present part's stand in
+    const CUtensorMap& W0 = do_routed ? h->tm_wg.map : h->tm_swg.map;
+    const CUtensorMap& W1 = do_routed ? h->tm_wu.map : h->tm_swu.map;
+    const CUtensorMap& Ws0 = do_shared ? h->tm_swg.map : h->tm_wg.map;
+    const CUtensorMap& Ws1 = do_shared ? h->tm_swu.map : h->tm_wu.map;
+    {
+      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+      if (launch_decode<true>(ctas, s0, pdl, W0, W1, h->tm_xperm32, Ws0, Ws1, h->tm_x32.map, g) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    DecodeArgs g2{};
+    if (do_routed) {
+      g2.num_groups = (int)N;
+      g2.counts = ra.counts;
+      g2.row_start = ra.row_start;
+      g2.n_wb = ceil_div(d, kDecWB);
+      g2.num_kb = ceil_div(I, kDecBK);
+      g2.row_scale = pa.gate_perm;
+      g2.out = h->at<__nv_bfloat16>(L.y);
+      g2.ld_out = (int)d;
+      g2.n_limit = (int)d;
+    }
+    if (do_shared) {
+      g2.sh_rows = (int)T;
+      g2.sh_n_wb = ceil_div(d, kDecWB);
+      g2.sh_J = (int)Ks;
+      g2.sh_kb_per_j = ceil_div(Is, kDecBK);
+      g2.sh_k_per_j = (int)Is;
+      g2.sh_out = h->at<__nv_bfloat16>(L.ys);
+      g2.sh_ld_out = (int)d;
+      g2.sh_n_limit = (int)d;
+    }
+    g2.partials = h->at<float>(L.dec_part_dn);
+    g2.tile_ctr = h->at<uint32_t>(L.dec_ctr_dn);
+    g2.err = h->at<uint32_t>(L.err);
+    g2.timeout_ns = kTimeoutNs;
+    const CUtensorMap& D0 = do_routed ? h->tm_wd.map : h->tm_swd.map;
+    const CUtensorMap& Ds0 = do_shared ? h->tm_swd.map : h->tm_wd.map;
+    const CUtensorMap& HX = do_routed ? h->tm_h32 : h->tm_hs32;
+    const CUtensorMap& HXs = do_shared ? h->tm_hs32 : h->tm_h32;
+    KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
+    if (launch_decode<false>(ctas, s0, pdl, D0, D0, HX, Ds0, Ds0, HXs, g2) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+
   // ---- the expert GEMMs: shared experts' tiles first, then the routed experts' ----
-  if (do_routed || do_shared) {
+  if (!decode && (do_routed || do_shared)) {
     const int num_kb = ceil_div(d, kGuBK);
     GateUpArgs g{};
     if (do_routed) {
@@ -783,7 +909,10 @@ moe_status moe_status_query(moe_handle h) {
   uint32_t err = 0;
   if (cudaMemcpy(&err, h->ws + h->L.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (err) {
-    if (cudaMemset(h->ws + h->L.err, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+    // a kernel that gave up may have left stream-K tile counters part-counted
+    if (cudaMemset(h->ws + h->L.err, 0, 4) != cudaSuccess ||
+        cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) != cudaSuccess)
+      return MOE_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_ERR_TIMEOUT;
   }

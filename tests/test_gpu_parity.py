@@ -45,6 +45,12 @@ SMALL = {
                             sigma=0.03, bias="uniform", seed=26),
     # the smallest sizes the ABI accepts: one 16-column k-block, K = N, a single m- and n-tile
     "minimal": LS("minimal", T=5, d=16, N=4, I=16, K=4, Ks=1, Is=16, sigma=0.3, seed=27),
+    # batches of at most 64 tokens run the weight-streaming decode GEMMs; these cut tiles between
+    # CTAs (stream-K): 18 k-blocks of d against ~5 per CTA, two 32-token blocks (the second ragged),
+    # ragged weight blocks (I = 272, d = 1104) and a shared intermediate of 2.75 k-blocks
+    "decode_split": LS("decode_split", T=40, d=1104, N=12, I=272, K=2, Ks=1, Is=176, sigma=0.02, seed=29),
+    "decode_n256_sigmoid": LS("decode_n256_sigmoid", T=64, d=512, N=256, I=192, K=8, Ks=2, Is=128,
+                              gate="sigmoid", sigma=0.02, bias="uniform", seed=30),
 }
 
 FLAGS_ROUTED = B.MOE_FLAG_NO_RESIDUAL | B.MOE_FLAG_NO_SHARED
