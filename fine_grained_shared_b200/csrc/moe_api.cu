@@ -99,7 +99,7 @@ struct Layout {
   // byte offsets into the workspace
   size_t err, done, tile_ctr, tok_done, small_logits, idx, gate, slot, src, bc, counts, offsets, row_start, mtile,
       mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, dec_part_gu, dec_part_dn, dec_ctr_gu, dec_ctr_dn,
-      dec_ctr_bytes, total;
+      dec_ctr_bytes, arrive, arrive_bytes, total;
   int64_t P, Tpad, nblk;
 };
 
@@ -159,6 +159,9 @@ Layout make_layout(const moe_config& c) {
   L.dec_ctr_gu = take(size_t(gu_tiles) * 4 * 4 + size_t(dn_tiles) * 4 * 4);
   L.dec_ctr_dn = L.dec_ctr_gu + size_t(gu_tiles) * 4 * 4;
   L.dec_ctr_bytes = size_t(gu_tiles + dn_tiles) * 4 * 4;
+  // the fused final sum's arrival counters: one per token and 256-column output chunk
+  L.arrive_bytes = size_t(Tm) * ((c.d_model + kGemmBN - 1) / kGemmBN) * 4;
+  L.arrive = take(L.arrive_bytes);
   L.total = o;
   return L;
 }
@@ -473,6 +476,7 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
   ok = ok && cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) == cudaSuccess;
+  ok = ok && cudaMemset(h->ws + h->L.arrive, 0, h->L.arrive_bytes) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
@@ -754,6 +758,18 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     g2.ld_out = (int)d;
     g2.err = h->at<uint32_t>(L.err);
     g2.timeout_ns = kTimeoutNs;
+    // the final sum in the epilogue: each 256-column output chunk of a token is completed by the
+    // last of its K routed chunks and its shared chunk to be stored
+    g2.complete = 1;
+    g2.T = (int)T;
+    g2.K = K;
+    g2.arrivals = (do_routed ? K : 0) + (do_shared ? 1 : 0);
+    g2.offsets = ra.offsets;
+    g2.src = pa.src;
+    g2.slot_of = pa.slot_of;
+    g2.x = (c.flags & MOE_FLAG_NO_RESIDUAL) ? nullptr : static_cast<const __nv_bfloat16*>(x);
+    g2.final_out = static_cast<__nv_bfloat16*>(out);
+    g2.arrive_ctr = h->at<uint32_t>(L.arrive);
     const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
     const int pairs = do_routed || sh_tiles2 > h->max_pairs ? h->max_pairs : sh_tiles2;
     const CUtensorMap& sA2 = do_shared ? h->tm_hs : h->tm_h;
@@ -762,7 +778,8 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     if (launch_down(pairs, s0, pdl, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
-  // ---- the final sum ----
+  // ---- the final sum (the 128-row-tile path sums in the down GEMM's epilogue) ----
+  if (!decode && (do_routed || do_shared)) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   CombineArgs ca{};
   ca.T = (int)T;
   ca.K = K;
@@ -911,7 +928,8 @@ moe_status moe_status_query(moe_handle h) {
   if (err) {
     // a kernel that gave up may have left stream-K tile counters part-counted
     if (cudaMemset(h->ws + h->L.err, 0, 4) != cudaSuccess ||
-        cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) != cudaSuccess)
+        cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) != cudaSuccess ||
+        cudaMemset(h->ws + h->L.arrive, 0, h->L.arrive_bytes) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_ERR_TIMEOUT;

@@ -188,8 +188,10 @@ typedef enum moe_kernel_id {
   MOE_KERNEL_ROUTER = 0,   /* affinities, top-K, histogram, scan */
   MOE_KERNEL_PERMUTE = 1,  /* expert-contiguous rows of x */
   MOE_KERNEL_GATE_UP = 2,  /* SwiGLU(x W_gate^T, x W_up^T): shared experts on x, routed ones grouped */
-  MOE_KERNEL_DOWN = 3,     /* shared experts: Hs W_down^T; routed experts: g * (H W_down^T) */
-  MOE_KERNEL_COMBINE = 4,  /* h = x + shared + sum_k g * routed, k ascending */
+  MOE_KERNEL_DOWN = 3,     /* shared experts: Hs W_down^T; routed experts: g * (H W_down^T); for batches
+                              of more than 64 tokens also h = x + shared + sum_k g * routed, k ascending */
+  MOE_KERNEL_COMBINE = 4,  /* h = x + shared + sum_k g * routed, k ascending, as a kernel of its own:
+                              batches of at most 64 tokens only (no launch for larger ones) */
   MOE_KERNEL_COUNT = 5
 } moe_kernel_id;
 #define MOE_TIMING_ALL ((1u << MOE_KERNEL_COUNT) - 1u)
