@@ -34,9 +34,11 @@
 // round-robin order.
 //
 // Epilogue: Y[row, n0 + c] = g[row] * acc[c] (bf16) for routed tiles and
-// Ys[row, n0 + c] = acc[c] for shared ones; then the layer's final k-ordered
-// sum of every output chunk whose last operand this tile produced
-// (complete_chunks, below), so no separate pass re-reads Y.
+// Ys[row, n0 + c] = acc[c] for shared ones.  The layer's final k-ordered sum
+// runs in combine_kernel, which streams whole rows (permute.cuh): summing in
+// this epilogue, each chunk by the last of its K + 1 producers, left the
+// epilogue warps waiting on scattered row reads longer than the next tile's
+// MMAs (16B prefill: down 0.92 ms against 0.56 + 0.145 ms for down + combine).
 #pragma once
 
 #include "sm100.cuh"
@@ -72,16 +74,6 @@ struct GemmArgs {
   int sh_J;                    // shared experts summed into one accumulator
   int sh_k_per_j;              // Hs columns per shared expert (I_s)
   __nv_bfloat16* sh_out;       // Ys
-  // the layer's final sum, fused (complete != 0): out[t] = x[t] + Ys[t] + sum_k Y[slot_of[t, k]]
-  int complete;
-  int T, K;                    // tokens, routed slots per token
-  int arrivals;                // chunks a token's 256-column output chunk waits for: K (routed) + 1 (shared)
-  const int32_t* offsets;      // [num_groups + 1] unpadded: rows of expert g = offsets[g + 1] - offsets[g]
-  const int32_t* src;          // [T * K] token of each unpadded expert-ordered row
-  const int32_t* slot_of;      // [T, K] padded row of (t, k)
-  const __nv_bfloat16* x;      // [T, d] the residual, or null
-  __nv_bfloat16* final_out;    // [T, d] the layer's output
-  uint32_t* arrive_ctr;        // [T, n_tiles], zero between launches (the last arrival resets it)
   // both parts
   int n_tiles;                 // routed n-tiles (down: 256 output columns over d; gate/up: 128 H columns)
   int n_limit;                 // valid output columns of out (down: d; gate/up: I)
@@ -94,7 +86,7 @@ struct GemmArgs {
 
 __host__ __device__ constexpr size_t gemm_smem_bytes() {
   return 1024 + static_cast<size_t>(kGemmStages) * (kStageA + kStageB) + 8 * (2 * kGemmStages + 4 + 2) + 16 +
-         4 * 3 * 264;
+         4 * 2 * 264;
 }
 
 struct TileCoord {
@@ -141,82 +133,6 @@ __device__ __forceinline__ void pair_record_error(uint32_t* err, volatile int* a
   atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
 }
 
-// The layer's final sum, fused into the epilogue.  Every output chunk
-// out[t, n0 .. n0 + 255] waits for K + 1 chunks: g * FFN of each of the
-// token's K routed rows and the shared experts' Ys.  Each row, once its chunk
-// is stored, counts it on the token's counter for that chunk; the row whose
-// count completes it (the last to arrive) has its warp sum the chunk, with
-// each lane covering 8 columns: x + Ys + Y[slot_of[t, 0]] + ... + Y[slot_of[t,
-// K - 1]] in that order, in fp32, from the stored bf16 values, and rounds once
-// to bf16.  The order and the operands are the same whichever row arrives
-// last, so the output is deterministic; the rows written by other CTAs are
-// read through L2 after the fence that the counter orders.
-__device__ __forceinline__ void complete_chunks(const GemmArgs& a, const TileCoord& c, size_t row,
-                                                const int32_t* s_rows, const int32_t* s_offs, int lane) {
-  int tok = -1;
-  if (c.shared) {
-    if (row < static_cast<size_t>(a.T)) tok = static_cast<int>(row);
-  } else {
-    const int pos = static_cast<int>(row) - s_rows[c.g];
-    if (pos < s_offs[c.g + 1] - s_offs[c.g]) tok = a.src[s_offs[c.g] + pos];
-  }
-  __threadfence();  // this row's chunk is visible before it is counted
-  bool last = false;
-  if (tok >= 0) {
-    uint32_t* ctr = a.arrive_ctr + static_cast<size_t>(tok) * a.n_tiles + c.n_tile;
-    last = atomicAdd(ctr, 1u) == static_cast<uint32_t>(a.arrivals - 1);
-    if (last) *ctr = 0u;  // every chunk of this output chunk has arrived: ready for the next launch
-  }
-  uint32_t todo = __ballot_sync(0xffffffffu, last);
-  if (!todo) return;
-  __threadfence();  // the other rows' chunks, counted before this one, are visible from here
-  const int col = c.n_tile * kGemmBN + 8 * lane;
-  while (todo) {
-    const int l = __ffs(todo) - 1;
-    todo &= todo - 1;
-    const int t = __shfl_sync(0xffffffffu, tok, l);
-    if (col < a.n_limit) {
-      // every load first, then the sum in its fixed order
-      const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
-      const uint4 xv = a.x ? __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.ld_out + col)) : zero;
-      const uint4 sv =
-          a.sh_out ? __ldcg(reinterpret_cast<const uint4*>(a.sh_out + static_cast<size_t>(t) * a.ld_out + col)) : zero;
-      const int K = a.out ? a.K : 0;
-      uint4 yv[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        yv[k] = zero;
-        if (k < K) {
-          const int srow = __ldg(a.slot_of + static_cast<size_t>(t) * a.K + k);
-          yv[k] = __ldcg(reinterpret_cast<const uint4*>(a.out + static_cast<size_t>(srow) * a.ld_out + col));
-        }
-      }
-      float acc[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-      auto add = [&](const uint4& q) {
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[2 * j] += bf16lo(w[j]);
-          acc[2 * j + 1] += bf16hi(w[j]);
-        }
-      };
-      if (a.x) add(xv);
-      if (a.sh_out) add(sv);
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (k < K) add(yv[k]);
-      uint4 o;
-      o.x = pack_bf16x2(acc[0], acc[1]);
-      o.y = pack_bf16x2(acc[2], acc[3]);
-      o.z = pack_bf16x2(acc[4], acc[5]);
-      o.w = pack_bf16x2(acc[6], acc[7]);
-      *reinterpret_cast<uint4*>(a.final_out + static_cast<size_t>(t) * a.ld_out + col) = o;
-    }
-  }
-}
-
 // GU = false (the down projection): tmA: H rows; tmB: W_down as [experts][d][I]
 // (each CTA stages its 128 of the tile's 256 output columns); tmAs: Hs rows;
 // tmBs: the shared experts' W_down as [K_s][d][I_s].  tmB2 / tmBs2 unused.
@@ -245,7 +161,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_mts = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [264]
   int32_t* s_rows = s_mts + 264;                                // [264]
-  int32_t* s_offs = s_rows + 264;                               // [264]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
@@ -277,7 +192,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   for (int i = tid; i <= G; i += kGemmThreads) {
     s_mts[i] = G ? a.mtile_start[i] : 0;
     s_rows[i] = G ? a.row_start[i] : 0;
-    s_offs[i] = G && a.complete ? a.offsets[i] : 0;
   }
   tc_fence_before_sync();
   cluster_sync();  // both CTAs' barriers exist before any copy or arrive targets them
@@ -461,7 +375,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         acc = 0;
         acc_ph ^= 1u;
       }
-      if (!GU && a.complete) complete_chunks(a, c, row, s_rows, s_offs, lane);
     }
   }
   if (aborted || *abort_flag) {

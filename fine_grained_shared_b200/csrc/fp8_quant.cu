@@ -20,52 +20,19 @@
 #include <stdint.h>
 
 #include "fgs_moe.h"
+#include "fp8_util.cuh"
 
 namespace {
+
+using fgs::amax8;
+using fgs::encode8;
+using fgs::pow2_neg;
+using fgs::scale_exponent;
 
 constexpr int kGroup = 128;
 constexpr int kRowThreads = 256;          // 8 warps, one row at a time each
 constexpr int kRowBatch = 8;              // 256-column chunks of a row a lane loads before it converts
 constexpr int kBlockThreads = 256;        // one CTA per 128 x 128 block, 8 rows of 8 columns per thread
-
-// Smallest e with amax <= 448 * 2^e, from the bits of amax (>= 0, finite).
-// amax = (1 + m / 2^23) * 2^(E - 127) for a normal float; 448 = 1.75 * 2^8, so
-// e = E - 127 - 8 when the significand is <= 1.75 and one more above it.
-// Zero and subnormal maxima need e below -127 and take the clamp.
-__device__ __forceinline__ int scale_exponent(float amax) {
-  const uint32_t b = __float_as_uint(amax);
-  const int E = int(b >> 23);
-  const uint32_t m = b & 0x7FFFFFu;
-  const int e = E == 0 ? -127 : E - 135 + (m > 0x600000u ? 1 : 0);
-  return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
-__device__ __forceinline__ float pow2_neg(int e) {  // 2^-e for e in [-127, 127) as a normal float
-  return __uint_as_float(uint32_t(127 - e) << 23);
-}
-
-// max |x| of 8 bf16 values (exact: abs and max do not round)
-__device__ __forceinline__ float amax8(const uint4& v) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-  __nv_bfloat162 m = __hmax2(__habs2(h[0]), __habs2(h[1]));
-  m = __hmax2(m, __hmax2(__habs2(h[2]), __habs2(h[3])));
-  return fmaxf(__low2float(m), __high2float(m));
-}
-
-// E4M3 codes of 8 bf16 values times 2^-e, in memory order.  The product is
-// exact in fp32, so the paired conversion rounds once.
-__device__ __forceinline__ uint2 encode8(const uint4& v, float inv) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-  uint32_t c[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 p = __bfloat1622float2(h[i]);
-    p.x *= inv;
-    p.y *= inv;
-    c[i] = uint32_t(__nv_cvt_float2_to_fp8x2(p, __NV_SATFINITE, __NV_E4M3)) & 0xFFFFu;  // .x in the low byte
-  }
-  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-}
 
 // x bf16 [rows, cols] -> q [rows, cols], scale [rows, groups].  A warp takes
 // whole rows (grid-stride); within a row, 256-column chunks in batches of

@@ -29,6 +29,7 @@
 #include "../../include/fgs_moe.h"
 #include "decode_gemm.cuh"
 #include "down_gemm.cuh"
+#include "fp8_gemm.cuh"
 #include "gateup_gemm.cuh"
 #include "permute.cuh"
 #include "router_topk.cuh"
@@ -91,6 +92,19 @@ bool encode_bf16(CUtensorMap* m, const void* base, uint64_t d2, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
+// uint8 tensor [d2][rows][cols] (E4M3 codes), box [1][box_rows][128], 128-byte swizzle.
+bool encode_u8(CUtensorMap* m, const void* base, uint64_t d2, uint64_t rows, uint64_t cols, uint32_t box_rows,
+               int rank) {
+  cuuint64_t dims[3] = {cols, rows, d2};
+  cuuint64_t strides[2] = {cols, rows * cols};
+  cuuint32_t box[3] = {128, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 struct MapCache {
   const void* ptr = nullptr;
   int64_t rows = -1;
@@ -104,8 +118,8 @@ struct Layout {
   // byte offsets into the workspace
   size_t err, done, tile_ctr, tok_done, small_logits, idx, gate, slot, src, bc, counts, offsets, row_start, mtile,
       mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, dec_part_gu, dec_part_dn, dec_ctr_gu, dec_ctr_dn,
-      dec_ctr_bytes, arrive, arrive_bytes, total;
-  int64_t P, Tpad, nblk;
+      dec_ctr_bytes, xq_perm, xs_perm, xq, xs, hq, hs_perm, hsq, hss, total;
+  int64_t P, Pa, Tpad, nblk;
 };
 
 // Tiles a decode GEMM launch can have: 32-token blocks of the shared experts'
@@ -164,9 +178,20 @@ Layout make_layout(const moe_config& c) {
   L.dec_ctr_gu = take(size_t(gu_tiles) * 4 * 4 + size_t(dn_tiles) * 4 * 4);
   L.dec_ctr_dn = L.dec_ctr_gu + size_t(gu_tiles) * 4 * 4;
   L.dec_ctr_bytes = size_t(gu_tiles + dn_tiles) * 4 * 4;
-  // the fused final sum's arrival counters: one per token and 256-column output chunk
-  L.arrive_bytes = size_t(Tm) * ((c.d_model + kGemmBN - 1) / kGemmBN) * 4;
-  L.arrive = take(L.arrive_bytes);
+  // the FP8 path: E4M3 codes of the permuted rows, of x, of H and Hs, each with its scale atoms
+  // (512 bytes per 128 rows and 128 columns)
+  L.Pa = (L.P + 127) / 128 * 128;
+  if (c.flags & MOE_FLAG_FP8) {
+    const int64_t d = c.d_model, I = c.d_ff, SI = int64_t(c.n_shared) * c.d_ff_shared;
+    L.xq_perm = take(size_t(L.Pa) * d);
+    L.xs_perm = take(size_t(L.Pa / 128) * (d / 128) * kSfAtomBytes);
+    L.xq = take(size_t(L.Tpad) * d);
+    L.xs = take(size_t(L.Tpad / 128) * (d / 128) * kSfAtomBytes);
+    L.hq = take(size_t(L.Pa) * I);
+    L.hs_perm = take(size_t(L.Pa / 128) * (I / 128) * kSfAtomBytes);
+    L.hsq = take(size_t(L.Tpad) * SI);
+    L.hss = take(size_t(L.Tpad / 128) * (SI / 128) * kSfAtomBytes);
+  }
   L.total = o;
   return L;
 }
@@ -182,8 +207,11 @@ moe_status check_config(const moe_config* c) {
   if (c->n_routed > kMaxRouted || c->max_k > kMaxK) return MOE_ERR_UNSUPPORTED;
   if (c->max_k > c->n_routed) return MOE_ERR_INVALID_ARG;
   if (c->d_model % 16 || c->d_ff % 16 || (c->n_shared > 0 && c->d_ff_shared % 16)) return MOE_ERR_ALIGNMENT;
-  const uint32_t known = MOE_FLAG_NO_RESIDUAL | MOE_FLAG_NO_SHARED | MOE_FLAG_NO_ROUTED | MOE_FLAG_DEBUG_WAIT_TIMEOUT;
+  const uint32_t known =
+      MOE_FLAG_NO_RESIDUAL | MOE_FLAG_NO_SHARED | MOE_FLAG_NO_ROUTED | MOE_FLAG_FP8 | MOE_FLAG_DEBUG_WAIT_TIMEOUT;
   if (c->flags & ~known) return MOE_ERR_INVALID_ARG;
+  if ((c->flags & MOE_FLAG_FP8) && (c->d_model % 128 || c->d_ff % 128 || (c->n_shared > 0 && c->d_ff_shared % 128)))
+    return MOE_ERR_ALIGNMENT;
   return MOE_OK;
 }
 
@@ -222,6 +250,8 @@ struct moe_ctx {
   // TMA descriptors: workspace ones are fixed, the others follow the caller's pointers
   CUtensorMap tm_xperm, tm_h, tm_hs;
   CUtensorMap tm_xperm32, tm_h32, tm_hs32;  // 32-row token boxes of the decode GEMMs
+  CUtensorMap tm_xq_perm, tm_xq, tm_hq, tm_hsq;  // FP8 codes of the activations (128-row boxes)
+  MapCache tm8_wg, tm8_wu, tm8_wd, tm8_swg, tm8_swu, tm8_swd;  // FP8 weight codes
   MapCache tm_x, tm_x32, tm_router, tm_wg, tm_wu, tm_wd, tm_swg, tm_swu, tm_swd;
   // host-buffer forward: copy streams and per-chunk events, created on first use
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
@@ -326,8 +356,23 @@ cudaError_t set_kernel_attrs() {
   if ((e = cudaFuncSetAttribute(decode_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(dec_smem_bytes<true>()))))
     return e;
-  return cudaFuncSetAttribute(decode_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(dec_smem_bytes<false>()));
+  if ((e = cudaFuncSetAttribute(decode_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(dec_smem_bytes<false>()))))
+    return e;
+  const int fs = static_cast<int>(fp8_gemm_smem_bytes());
+  if ((e = cudaFuncSetAttribute(fp8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, fs))) return e;
+  return cudaFuncSetAttribute(fp8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, fs);
+}
+
+bool refresh_u8(MapCache& c, const void* p, uint64_t d2, uint64_t rows, uint64_t cols, uint32_t box_rows, int rank) {
+  if (c.ptr == p) return true;
+  if (!encode_u8(&c.map, p, d2, rows, cols, box_rows, rank)) {
+    c.ptr = nullptr;
+    return false;
+  }
+  c.ptr = p;
+  c.rows = 0;
+  return true;
 }
 
 // Re-encode a cached descriptor when the caller's pointer (or row count) changes.
@@ -407,6 +452,110 @@ class KernelTimer {
   cudaEvent_t stop_ = nullptr;
 };
 
+// The router step shared by the bf16 and FP8 forwards: affinities, top-K, the
+// per-block expert histogram and the scan (router_topk.cuh).  Records the
+// call's stream, T and K for moe_get_routing / moe_status_query.
+moe_status enqueue_router(moe_ctx* h, const void* x, int64_t T, const moe_router* router, int32_t K,
+                          cudaStream_t s0, bool pdl, RouterArgs& ra) {
+  const moe_config& c = h->cfg;
+  const Layout& L = h->L;
+  const int64_t d = c.d_model, N = c.n_routed;
+  const bool sigmoid = c.gate == MOE_GATE_SIGMOID_BIASED;
+  const int Npad = ((int)N + 15) / 16 * 16;
+  static_assert(kGuBoxRowsA == kRouterBM, "x serves as A of the router and of the shared gate/up GEMM");
+  if (!refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2) ||
+      !refresh(h->tm_router, router->weight, 0, 1, N, d, (uint32_t)Npad, 2))
+    return MOE_ERR_CUDA;
+  h->last_stream = s0;
+  h->last_T = T;
+  h->last_K = K;
+  const int nblk = ceil_div(T, 128);
+  ra = RouterArgs{};
+  ra.T = (int)T;
+  ra.N = (int)N;
+  ra.Npad = Npad;
+  ra.num_kb = ceil_div(d, kBK);
+  ra.nblk = nblk;
+  ra.tmem_cols = Npad <= 32 ? 32u : Npad <= 64 ? 64u : Npad <= 128 ? 128u : 256u;
+  ra.logit_bias = router->logit_bias;
+  ra.select_bias = router->select_bias;
+  ra.idx = h->at<int32_t>(L.idx);
+  ra.gate = h->at<float>(L.gate);
+  ra.block_counts = h->at<int32_t>(L.bc);
+  ra.counts = h->at<int32_t>(L.counts);
+  ra.offsets = h->at<int32_t>(L.offsets);
+  ra.row_start = h->at<int32_t>(L.row_start);
+  ra.mtile_start = h->at<int32_t>(L.mtile);
+  ra.mtile128_start = h->at<int32_t>(L.mtile128);
+  ra.done_counter = h->at<uint32_t>(L.done);
+  ra.err = h->at<uint32_t>(L.err);
+  ra.timeout_ns = kTimeoutNs;
+  KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
+  if (T <= kSmallRouterMaxT) {
+    // a few tokens: one CTA per token on the CUDA cores
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
+    SmallRouterArgs sa{h->at<float>(L.small_logits), h->at<uint32_t>(L.tok_done)};
+    const dim3 grid((unsigned)T, (unsigned)ceil_div(N, kSmallRouterGroup)), block(kSmallRouterThreads);
+    const cudaError_t e =
+        sigmoid ? launch_pdl(router_small_kernel<true>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra, sa)
+                : launch_pdl(router_small_kernel<false>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra, sa);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  const size_t smem = router_smem_bytes(Npad);
+  return launch_router(K, sigmoid, dim3(nblk), smem, s0, pdl, h->tm_x.map, h->tm_router.map, ra) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
+}
+
+// The permutation's arguments (permute.cuh), shared by both forwards.
+PermuteArgs permute_args(moe_ctx* h, const void* x, int64_t T, int32_t K, const RouterArgs& ra, bool gather) {
+  const Layout& L = h->L;
+  const int nblk = ceil_div(T, 128);
+  PermuteArgs pa{};
+  pa.T = (int)T;
+  pa.K = K;
+  pa.N = h->cfg.n_routed;
+  pa.d = h->cfg.d_model;
+  const int split = (2 * h->num_sms + nblk - 1) / nblk;
+  // CTAs per 128-token block for the row copies: about two per SM in all, at most 8, or 32 for
+  // batches of up to 4 blocks (a 32-token decode batch copies one token row per CTA: 16B decode
+  // permutation 10.2 -> 8.6 us; more than 8 measured slower on the V3 layer, T = 4096)
+  const int max_split = nblk <= 4 ? 32 : 8;
+  pa.split = split < 1 ? 1 : split > max_split ? max_split : split;
+  pa.idx = ra.idx;
+  pa.gate = ra.gate;
+  pa.block_base = ra.block_counts;
+  pa.offsets = ra.offsets;
+  pa.row_start = ra.row_start;
+  pa.src = h->at<int32_t>(L.src);
+  pa.slot_of = h->at<int32_t>(L.slot);
+  pa.gate_perm = h->at<float>(L.gate_perm);
+  pa.x = static_cast<const __nv_bfloat16*>(x);
+  pa.x_perm = h->at<__nv_bfloat16>(L.x_perm);
+  pa.gather = gather ? 1 : 0;
+  pa.tile_ctr = h->at<int>(L.tile_ctr);
+  return pa;
+}
+
+// The final sum (combine_kernel): one warp per (token, chunk of a row): whole
+// rows once the batch alone gives every SM a full load of warps, shorter
+// chunks (>= 256 columns) below that (V3 layer, T = 4096, d = 7168: 0.272 ->
+// 0.223 ms).
+moe_status launch_combine(moe_ctx* h, const CombineArgs& ca, int64_t T, int64_t d, cudaStream_t s0, bool pdl) {
+  KernelTimer kt(h, MOE_KERNEL_COMBINE, s0);
+  const int64_t resident = int64_t(h->num_sms) * 64;  // warps the SMs hold at once
+  int cols = (int)d;
+  if (T < resident) {
+    const int chunks = ceil_div(2 * resident, T);
+    cols = ceil_div(ceil_div(d, chunks), 256) * 256;
+  }
+  const int64_t warps = T * ceil_div(d, cols);
+  if (launch_pdl(combine_kernel, dim3(ceil_div(warps * 32, 256)), dim3(256), 0, s0, 1, pdl, ca, cols) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -482,7 +631,6 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
   ok = ok && cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) == cudaSuccess;
-  ok = ok && cudaMemset(h->ws + h->L.arrive, 0, h->L.arrive_bytes) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
@@ -492,6 +640,13 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
     ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kBoxRowsA, 2);
     ok = ok &&
          encode_bf16(&h->tm_hs32, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kDecBoxRowsX, 2);
+  }
+  if (c.flags & MOE_FLAG_FP8) {
+    const int64_t SI = int64_t(c.n_shared) * c.d_ff_shared;
+    ok = ok && encode_u8(&h->tm_xq_perm, h->ws + h->L.xq_perm, 1, h->L.Pa, c.d_model, 128, 2);
+    ok = ok && encode_u8(&h->tm_xq, h->ws + h->L.xq, 1, h->L.Tpad, c.d_model, 128, 2);
+    ok = ok && encode_u8(&h->tm_hq, h->ws + h->L.hq, 1, h->L.Pa, c.d_ff, 128, 2);
+    if (SI > 0) ok = ok && encode_u8(&h->tm_hsq, h->ws + h->L.hsq, 1, h->L.Tpad, SI, 128, 2);
   }
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
@@ -538,15 +693,11 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   const Layout& L = h->L;
   const bool do_shared = Ks > 0 && !(c.flags & MOE_FLAG_NO_SHARED);
   const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
-  const int Npad = ((int)N + 15) / 16 * 16;
 
   // descriptors that follow the caller's pointers
-  static_assert(kGuBoxRowsA == kRouterBM, "x serves as A of the router and of the shared gate/up GEMM");
   const bool decode = T <= kDecodeMaxT;
-  bool ok = refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2);
+  bool ok = true;
   if (decode) ok = ok && refresh(h->tm_x32, x, T, 1, T, d, kDecBoxRowsX, 2);
-
-  ok = ok && refresh(h->tm_router, router->weight, 0, 1, N, d, (uint32_t)Npad, 2);
   ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, kGuBoxRowsB, 3);
   ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, kGuBoxRowsB, 3);
   ok = ok && refresh(h->tm_wd, experts->w_down, 0, N, d, I, kBoxRowsB, 3);
@@ -558,74 +709,15 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   if (!ok) return MOE_ERR_CUDA;
 
   const bool pdl = T <= kPdlMaxT;
-  h->last_stream = s0;
-  h->last_T = T;
-  h->last_K = K;
   const int nblk = ceil_div(T, 128);
 
   // ---- router and permutation ----
-  RouterArgs ra{};
-  ra.T = (int)T;
-  ra.N = (int)N;
-  ra.Npad = Npad;
-  ra.num_kb = ceil_div(d, kBK);
-  ra.nblk = nblk;
-  ra.tmem_cols = Npad <= 32 ? 32u : Npad <= 64 ? 64u : Npad <= 128 ? 128u : 256u;
-  ra.logit_bias = router->logit_bias;
-  ra.select_bias = router->select_bias;
-  ra.idx = h->at<int32_t>(L.idx);
-  ra.gate = h->at<float>(L.gate);
-  ra.block_counts = h->at<int32_t>(L.bc);
-  ra.counts = h->at<int32_t>(L.counts);
-  ra.offsets = h->at<int32_t>(L.offsets);
-  ra.row_start = h->at<int32_t>(L.row_start);
-  ra.mtile_start = h->at<int32_t>(L.mtile);
-  ra.mtile128_start = h->at<int32_t>(L.mtile128);
-  ra.done_counter = h->at<uint32_t>(L.done);
-  ra.err = h->at<uint32_t>(L.err);
-  ra.timeout_ns = kTimeoutNs;
+  RouterArgs ra;
   {
-    KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
-    if (T <= kSmallRouterMaxT) {
-      // a few tokens: one CTA per token on the CUDA cores
-      const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-      const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
-      SmallRouterArgs sa{h->at<float>(L.small_logits), h->at<uint32_t>(L.tok_done)};
-      const dim3 grid((unsigned)T, (unsigned)ceil_div(N, kSmallRouterGroup)), block(kSmallRouterThreads);
-      const cudaError_t e =
-          sigmoid ? launch_pdl(router_small_kernel<true>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra, sa)
-                  : launch_pdl(router_small_kernel<false>, grid, block, 0, s0, 1, pdl, xb, eb, (int)d, K, ra, sa);
-      if (e != cudaSuccess) return MOE_ERR_CUDA;
-    } else {
-      const size_t smem = router_smem_bytes(Npad);
-      if (launch_router(K, sigmoid, dim3(nblk), smem, s0, pdl, h->tm_x.map, h->tm_router.map, ra) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
+    const moe_status st = enqueue_router(h, x, T, router, K, s0, pdl, ra);
+    if (st != MOE_OK) return st;
   }
-
-  PermuteArgs pa{};
-  pa.T = (int)T;
-  pa.K = K;
-  pa.N = (int)N;
-  pa.d = (int)d;
-  const int split = (2 * h->num_sms + nblk - 1) / nblk;
-  // CTAs per 128-token block for the row copies: about two per SM in all, at most 8, or 32 for
-  // batches of up to 4 blocks (a 32-token decode batch copies one token row per CTA: 16B decode
-  // permutation 10.2 -> 8.6 us; more than 8 measured slower on the V3 layer, T = 4096)
-  const int max_split = nblk <= 4 ? 32 : 8;
-  pa.split = split < 1 ? 1 : split > max_split ? max_split : split;
-  pa.idx = ra.idx;
-  pa.gate = ra.gate;
-  pa.block_base = ra.block_counts;
-  pa.offsets = ra.offsets;
-  pa.row_start = ra.row_start;
-  pa.src = h->at<int32_t>(L.src);
-  pa.slot_of = h->at<int32_t>(L.slot);
-  pa.gate_perm = h->at<float>(L.gate_perm);
-  pa.x = static_cast<const __nv_bfloat16*>(x);
-  pa.x_perm = h->at<__nv_bfloat16>(L.x_perm);
-  pa.gather = do_routed ? 1 : 0;
-  pa.tile_ctr = h->at<int>(L.tile_ctr);
+  PermuteArgs pa = permute_args(h, x, T, K, ra, do_routed);
   {
     KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
     const dim3 grid(nblk, do_routed ? pa.split : 1);
@@ -796,18 +888,6 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     g2.sh_ld_out = (int)d;
     g2.err = h->at<uint32_t>(L.err);
     g2.timeout_ns = kTimeoutNs;
-    // the final sum in the epilogue: each 256-column output chunk of a token is completed by the
-    // last of its K routed chunks and its shared chunk to be stored
-    g2.complete = 1;
-    g2.T = (int)T;
-    g2.K = K;
-    g2.arrivals = (do_routed ? K : 0) + (do_shared ? 1 : 0);
-    g2.offsets = ra.offsets;
-    g2.src = pa.src;
-    g2.slot_of = pa.slot_of;
-    g2.x = (c.flags & MOE_FLAG_NO_RESIDUAL) ? nullptr : static_cast<const __nv_bfloat16*>(x);
-    g2.final_out = static_cast<__nv_bfloat16*>(out);
-    g2.arrive_ctr = h->at<uint32_t>(L.arrive);
     const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
     const int pairs = do_routed || sh_tiles2 > h->max_pairs ? h->max_pairs : sh_tiles2;
     const CUtensorMap& sA2 = do_shared ? h->tm_hs : h->tm_h;
@@ -816,8 +896,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     if (launch_down(pairs, s0, pdl, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
   }
 
-  // ---- the final sum (the 128-row-tile path sums in the down GEMM's epilogue) ----
-  if (!decode && (do_routed || do_shared)) return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  // ---- the final sum ----
   CombineArgs ca{};
   ca.T = (int)T;
   ca.K = K;
@@ -829,22 +908,186 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   ca.out = static_cast<__nv_bfloat16*>(out);
   ca.add_residual = (c.flags & MOE_FLAG_NO_RESIDUAL) ? 0 : 1;
   ca.add_routed = do_routed ? 1 : 0;
+  return launch_combine(h, ca, T, d, s0, pdl);
+}
+
+moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_router* router,
+                           const moe_experts_fp8* experts, const moe_experts_fp8* shared, int32_t K, void* out,
+                           void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (!(c.flags & MOE_FLAG_FP8)) return MOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_SHAPE;
+  if (K < 1 || K > c.max_k || K > c.n_routed) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!router || !experts) return MOE_ERR_INVALID_ARG;
+  if ((c.n_shared > 0) != (shared != nullptr)) return MOE_ERR_INVALID_ARG;
+  auto complete = [](const moe_experts_fp8* e) {
+    return e->w_gate && e->w_up && e->w_down && e->s_gate && e->s_up && e->s_down;
+  };
+  if (!x || !out || !router->weight || !complete(experts) || (shared && !complete(shared))) return MOE_ERR_INVALID_ARG;
+  const bool sigmoid = c.gate == MOE_GATE_SIGMOID_BIASED;
+  if (sigmoid ? router->logit_bias != nullptr : router->select_bias != nullptr) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, out, router->weight, router->logit_bias, router->select_bias, experts->w_gate,
+                        experts->w_up, experts->w_down, shared ? shared->w_gate : nullptr,
+                        shared ? shared->w_up : nullptr, shared ? shared->w_down : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  const int64_t d = c.d_model, N = c.n_routed, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const size_t out_bytes = size_t(T) * d * 2;
+  const size_t wsz = size_t(N) * I * d, swsz = size_t(Ks) * Is * d;
+  if (overlaps(out, out_bytes, x, out_bytes) || overlaps(out, out_bytes, router->weight, size_t(N) * d * 2) ||
+      overlaps(out, out_bytes, experts->w_gate, wsz) || overlaps(out, out_bytes, experts->w_up, wsz) ||
+      overlaps(out, out_bytes, experts->w_down, wsz) ||
+      (shared && (overlaps(out, out_bytes, shared->w_gate, swsz) || overlaps(out, out_bytes, shared->w_up, swsz) ||
+                  overlaps(out, out_bytes, shared->w_down, swsz))))
+    return MOE_ERR_INVALID_ARG;
+
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const Layout& L = h->L;
+  const bool do_shared = Ks > 0 && !(c.flags & MOE_FLAG_NO_SHARED);
+  const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
+  // FP8 weight codes: W_gate / W_up [n][I][d] and W_down [n][d][I], 128-byte rows of K, 128-row boxes
+  // (W_down 256: one box holds a tile's 256 output rows)
+  bool ok = refresh_u8(h->tm8_wg, experts->w_gate, N, I, d, kF8BoxRowsW, 3) &&
+            refresh_u8(h->tm8_wu, experts->w_up, N, I, d, kF8BoxRowsW, 3) &&
+            refresh_u8(h->tm8_wd, experts->w_down, N, d, I, kF8BoxRowsWd, 3);
+  if (shared)
+    ok = ok && refresh_u8(h->tm8_swg, shared->w_gate, 1, Ks * Is, d, kF8BoxRowsW, 3) &&
+         refresh_u8(h->tm8_swu, shared->w_up, 1, Ks * Is, d, kF8BoxRowsW, 3) &&
+         refresh_u8(h->tm8_swd, shared->w_down, Ks, d, Is, kF8BoxRowsWd, 3);
+  if (!ok) return MOE_ERR_CUDA;
+  const bool pdl = T <= kPdlMaxT;
+  const int nblk = ceil_div(T, 128);
+
+  RouterArgs ra;
   {
-    KernelTimer kt(h, MOE_KERNEL_COMBINE, s0);
-    // one warp per (token, chunk of a row): whole rows once the batch alone
-    // gives every SM a full load of warps, shorter chunks (>= 256 columns)
-    // below that (V3 layer, T = 4096, d = 7168: 0.272 -> 0.223 ms)
-    const int64_t resident = int64_t(h->num_sms) * 64;  // warps the SMs hold at once
-    int cols = (int)d;
-    if (T < resident) {
-      const int chunks = ceil_div(2 * resident, T);
-      cols = ceil_div(ceil_div(d, chunks), 256) * 256;
-    }
-    const int64_t warps = T * ceil_div(d, cols);
-    if (launch_pdl(combine_kernel, dim3(ceil_div(warps * 32, 256)), dim3(256), 0, s0, 1, pdl, ca, cols) != cudaSuccess)
+    const moe_status st = enqueue_router(h, x, T, router, K, s0, pdl, ra);
+    if (st != MOE_OK) return st;
+  }
+  PermuteQuantArgs pq{};
+  pq.p = permute_args(h, x, T, K, ra, do_routed);
+  pq.xq_perm = h->at<uint8_t>(L.xq_perm);
+  pq.xs_perm = h->at<uint8_t>(L.xs_perm);
+  pq.xq = do_shared ? h->at<uint8_t>(L.xq) : nullptr;
+  pq.xs = do_shared ? h->at<uint8_t>(L.xs) : nullptr;
+  {
+    KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
+    if (launch_pdl(permute_quant_kernel, dim3(nblk, pq.p.split), dim3(kPermThreads), 0, s0, 1, pdl, pq) !=
+        cudaSuccess)
       return MOE_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+
+  if (do_routed || do_shared) {
+    const int64_t SI = Ks * Is;
+    // an absent part's maps are never read; the present part's stand in
+    const CUtensorMap& A = do_routed ? h->tm_xq_perm : h->tm_xq;
+    const CUtensorMap& As = do_shared ? h->tm_xq : h->tm_xq_perm;
+    const CUtensorMap& Wg = do_routed ? h->tm8_wg.map : h->tm8_swg.map;
+    const CUtensorMap& Wu = do_routed ? h->tm8_wu.map : h->tm8_swu.map;
+    const CUtensorMap& Wgs = do_shared ? h->tm8_swg.map : h->tm8_wg.map;
+    const CUtensorMap& Wus = do_shared ? h->tm8_swu.map : h->tm8_wu.map;
+    Fp8GemmArgs g{};
+    if (do_routed) {
+      g.num_groups = (int)N;
+      g.mtile_start = ra.mtile128_start;
+      g.row_start = ra.row_start;
+      g.n_tiles = ceil_div(I, kF8BN / 2);
+      g.num_kg = (int)(d / kF8BK);
+      g.a_atoms = h->at<uint8_t>(L.xs_perm);
+      g.a_groups = (int)(d / kF8BK);
+      g.w_scale0 = experts->s_gate;
+      g.w_scale1 = experts->s_up;
+      g.w_rows128 = (int)(I / 128);
+      g.hq = h->at<uint8_t>(L.hq);
+      g.hs_atoms = h->at<uint8_t>(L.hs_perm);
+      g.h_groups = (int)(I / kF8BK);
+      g.ld_out = (int)I;
+      g.n_limit = (int)I;
+    }
+    if (do_shared) {
+      g.sh_rows = (int)T;
+      g.sh_n_tiles = ceil_div(SI, kF8BN / 2);
+      g.sh_J = 1;
+      g.sh_kg_per_j = (int)(d / kF8BK);
+      g.sh_a_atoms = h->at<uint8_t>(L.xs);
+      g.sh_a_groups = (int)(d / kF8BK);
+      g.sh_w_scale0 = shared->s_gate;
+      g.sh_w_scale1 = shared->s_up;
+      g.sh_w_rows128 = (int)(Is / 128);
+      g.sh_hq = h->at<uint8_t>(L.hsq);
+      g.sh_hs_atoms = h->at<uint8_t>(L.hss);
+      g.sh_h_groups = (int)(SI / kF8BK);
+      g.sh_ld_out = (int)SI;
+      g.sh_n_limit = (int)SI;
+    }
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
+    const int sh_tiles = do_shared ? ceil_div(T, kF8BM) * g.sh_n_tiles : 0;
+    const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
+    {
+      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+      if (launch_pdl(fp8_gemm_kernel<true>, dim3(ctas), dim3(kF8Threads), fp8_gemm_smem_bytes(), s0, 1, pdl, A, Wg,
+                     Wu, As, Wgs, Wus, g) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    const CUtensorMap& HA = do_routed ? h->tm_hq : h->tm_hsq;
+    const CUtensorMap& HAs = do_shared ? h->tm_hsq : h->tm_hq;
+    const CUtensorMap& Wd = do_routed ? h->tm8_wd.map : h->tm8_swd.map;
+    const CUtensorMap& Wds = do_shared ? h->tm8_swd.map : h->tm8_wd.map;
+    Fp8GemmArgs g2{};
+    if (do_routed) {
+      g2.num_groups = (int)N;
+      g2.mtile_start = ra.mtile128_start;
+      g2.row_start = ra.row_start;
+      g2.n_tiles = ceil_div(d, kF8BN);
+      g2.num_kg = (int)(I / kF8BK);
+      g2.a_atoms = h->at<uint8_t>(L.hs_perm);
+      g2.a_groups = (int)(I / kF8BK);
+      g2.w_scale0 = experts->s_down;
+      g2.w_rows128 = (int)(d / 128);
+      g2.row_scale = h->at<float>(L.gate_perm);
+      g2.y = h->at<__nv_bfloat16>(L.y);
+      g2.ld_out = (int)d;
+      g2.n_limit = (int)d;
+    }
+    if (do_shared) {
+      g2.sh_rows = (int)T;
+      g2.sh_n_tiles = ceil_div(d, kF8BN);
+      g2.sh_J = (int)Ks;
+      g2.sh_kg_per_j = (int)(Is / kF8BK);
+      g2.sh_k_per_j = (int)Is;
+      g2.sh_a_atoms = h->at<uint8_t>(L.hss);
+      g2.sh_a_groups = (int)(SI / kF8BK);
+      g2.sh_w_scale0 = shared->s_down;
+      g2.sh_w_rows128 = (int)(d / 128);
+      g2.sh_y = h->at<__nv_bfloat16>(L.ys);
+      g2.sh_ld_out = (int)d;
+      g2.sh_n_limit = (int)d;
+    }
+    g2.err = h->at<uint32_t>(L.err);
+    g2.timeout_ns = kTimeoutNs;
+    const int sh_tiles2 = do_shared ? ceil_div(T, kF8BM) * g2.sh_n_tiles : 0;
+    const int ctas2 = do_routed || sh_tiles2 > h->num_sms ? h->num_sms : sh_tiles2;
+    KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
+    if (launch_pdl(fp8_gemm_kernel<false>, dim3(ctas2), dim3(kF8Threads), fp8_gemm_smem_bytes(), s0, 1, pdl, HA, Wd,
+                   Wd, HAs, Wds, Wds, g2) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+
+  CombineArgs ca{};
+  ca.T = (int)T;
+  ca.K = K;
+  ca.d = (int)d;
+  ca.x = static_cast<const __nv_bfloat16*>(x);
+  ca.ys = do_shared ? h->at<__nv_bfloat16>(L.ys) : nullptr;
+  ca.y = h->at<__nv_bfloat16>(L.y);
+  ca.slot_of = h->at<int32_t>(L.slot);
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.add_residual = (c.flags & MOE_FLAG_NO_RESIDUAL) ? 0 : 1;
+  ca.add_routed = do_routed ? 1 : 0;
+  return launch_combine(h, ca, T, d, s0, pdl);
 }
 
 moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
@@ -966,8 +1209,7 @@ moe_status moe_status_query(moe_handle h) {
   if (err) {
     // a kernel that gave up may have left stream-K tile counters part-counted
     if (cudaMemset(h->ws + h->L.err, 0, 4) != cudaSuccess ||
-        cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) != cudaSuccess ||
-        cudaMemset(h->ws + h->L.arrive, 0, h->L.arrive_bytes) != cudaSuccess)
+        cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_ERR_TIMEOUT;

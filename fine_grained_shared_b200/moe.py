@@ -28,6 +28,7 @@ MOE_GATE_SIGMOID_BIASED = 1
 MOE_FLAG_NO_RESIDUAL = 0x1
 MOE_FLAG_NO_SHARED = 0x2
 MOE_FLAG_NO_ROUTED = 0x4
+MOE_FLAG_FP8 = 0x8
 MOE_FLAG_DEBUG_WAIT_TIMEOUT = 0x100
 
 KERNEL_NAMES = ("router", "permute", "gate_up", "down", "combine")
@@ -49,6 +50,11 @@ class moe_experts(ctypes.Structure):
 
 class moe_shared(ctypes.Structure):
     _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p)]
+
+
+class moe_experts_fp8(ctypes.Structure):
+    _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p),
+                ("s_gate", c_void_p), ("s_up", c_void_p), ("s_down", c_void_p)]
 
 
 moe_handle = c_void_p
@@ -75,6 +81,8 @@ def lib() -> ctypes.CDLL:
     L.moe_forward.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), POINTER(moe_experts),
                               POINTER(moe_shared), c_int32, c_void_p, c_void_p]
     L.moe_forward_host.argtypes = L.moe_forward.argtypes
+    L.moe_forward_fp8.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), POINTER(moe_experts_fp8),
+                                  POINTER(moe_experts_fp8), c_int32, c_void_p, c_void_p]
     L.moe_get_routing.argtypes = [moe_handle, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.moe_status_query.argtypes = [moe_handle]
     L.moe_destroy.argtypes = [moe_handle]
@@ -87,7 +95,8 @@ def lib() -> ctypes.CDLL:
     L.moe_quantize_fp8_blocks.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
     L.moe_status_string.argtypes = [c_int]
     L.moe_status_string.restype = c_char_p
-    for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_get_routing",
+    for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_forward_fp8",
+                 "moe_get_routing",
                  "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc",
                  "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks"):
         getattr(L, name).restype = c_int
@@ -122,6 +131,12 @@ def moe_forward_host(h, x_host, T, router, experts, shared, K, out_host, stream)
     return lib().moe_forward_host(h, x_host, int(T), ctypes.byref(router), ctypes.byref(experts),
                                   ctypes.byref(shared) if shared is not None else None, int(K),
                                   out_host, stream)
+
+
+def moe_forward_fp8(h, x, T, router, experts, shared, K, out, stream):
+    """The layer forward with FP8 expert GEMMs (handle created with MOE_FLAG_FP8); see the header."""
+    return lib().moe_forward_fp8(h, x, int(T), ctypes.byref(router), ctypes.byref(experts),
+                                 ctypes.byref(shared) if shared is not None else None, int(K), out, stream)
 
 
 def moe_get_routing(h, idx, gate, counts, offsets, src, stream):
@@ -225,6 +240,28 @@ class MoELayer:
                          _stream_ptr(stream))
         if check and st != MOE_OK:
             raise MoEError(st, "moe_forward")
+        return out if check else (st, out)
+
+    def set_weights_fp8(self, experts_fp8, shared_fp8=None):
+        """FP8 expert weights for forward_fp8: (codes, scales) pairs as quantize_fp8_blocks returns
+        them, for (W_gate, W_up, W_down) of the routed experts and (when K_s > 0) of the shared ones."""
+        def pack(ws):
+            (g, sg), (u, su), (dn, sd) = ws
+            return moe_experts_fp8(g.data_ptr(), u.data_ptr(), dn.data_ptr(), sg.data_ptr(), su.data_ptr(),
+                                   sd.data_ptr())
+        self._keep_fp8 = (experts_fp8, shared_fp8)
+        self.experts_fp8 = pack(experts_fp8)
+        self.shared_fp8 = pack(shared_fp8) if shared_fp8 is not None else None
+
+    def forward_fp8(self, x, K, out=None, stream=None, check=True):
+        import torch
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty_like(x)
+        st = moe_forward_fp8(self.h, _ptr(x), T, self.router, self.experts_fp8, self.shared_fp8, K, _ptr(out),
+                             _stream_ptr(stream))
+        if check and st != MOE_OK:
+            raise MoEError(st, "moe_forward_fp8")
         return out if check else (st, out)
 
     def forward_host(self, x_host, K, out_host, stream=None):

@@ -64,6 +64,10 @@ typedef enum moe_gate_kind {
 #define MOE_FLAG_NO_RESIDUAL 0x1u /* drop u_t */
 #define MOE_FLAG_NO_SHARED 0x2u   /* drop the shared experts */
 #define MOE_FLAG_NO_ROUTED 0x4u   /* drop the routed experts (routing still runs) */
+/* The handle also holds the workspace of moe_forward_fp8 (FP8 copies of the
+ * permuted activations and of H, with their scales).  Requires d_model, d_ff
+ * and d_ff_shared to be multiples of 128 (else MOE_ERR_ALIGNMENT). */
+#define MOE_FLAG_FP8 0x8u
 /* Test only: the first grouped-GEMM CTA waits on a barrier that nothing
  * arrives on, with a 20 ms limit; the call then reports MOE_ERR_TIMEOUT. */
 #define MOE_FLAG_DEBUG_WAIT_TIMEOUT 0x100u
@@ -109,6 +113,21 @@ typedef struct moe_shared {
   const void* w_down;
 } moe_shared;
 
+/* Expert weights in fine-grained FP8, as moe_quantize_fp8_blocks writes them:
+ * E4M3 codes in the layout of the bf16 matrices (w_gate, w_up uint8 [n, I, d];
+ * w_down uint8 [n, d, I]) and one UE8M0 scale byte per 128 x 128 block
+ * (s_gate, s_up uint8 [n, I/128, d/128]; s_down uint8 [n, d/128, I/128]).
+ * n = mN and I = d_ff for the routed experts; n = K_s and I = d_ff_shared for
+ * the shared ones. */
+typedef struct moe_experts_fp8 {
+  const uint8_t* w_gate;
+  const uint8_t* w_up;
+  const uint8_t* w_down;
+  const uint8_t* s_gate;
+  const uint8_t* s_up;
+  const uint8_t* s_down;
+} moe_experts_fp8;
+
 typedef struct moe_ctx* moe_handle;
 
 /* Device bytes the handle allocates for cfg (host only; no CUDA call). */
@@ -141,6 +160,26 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
 moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
                             const moe_experts* experts, const moe_shared* shared, int32_t K,
                             void* out_host, void* stream);
+
+/* The layer forward with FP8 expert GEMMs (DeepSeek-V3 technical report,
+ * section 3.3 "FP8 Training" and Appendix B.2 "Discussion About Block-Wise
+ * Quantization"): routing as moe_forward (bf16 affinities, fp32 softmax or
+ * sigmoid and top-K); each token row x_t is quantized once to E4M3 with one
+ * power-of-two scale per 1 x 128 group (e = the smallest integer with
+ * max|x| <= 448 * 2^e, codes rounded to nearest even); the gate/up GEMM runs
+ * on those codes and the 128 x 128 block-quantized W_gate and W_up with
+ * block-scaled tensor-core MMAs and fp32 accumulation; H = SiLU(gate) * up is
+ * quantized 1 x 128 the same way in the GEMM's epilogue; the down GEMM runs on
+ * H's codes and W_down's, scales by g and forms h_t = u_t + shared + sum_k
+ * g FFN in k order (fp32, rounded once to bf16).  The residual u_t is the
+ * unquantized input.  x, out: bf16 [T, d] device; experts and shared (NULL iff
+ * K_s == 0): device FP8 weights as above.  The handle must have been created
+ * with MOE_FLAG_FP8 (else MOE_ERR_UNSUPPORTED); the other arguments and errors
+ * as moe_forward.  Asynchronous; moe_get_routing, moe_update_bias and
+ * moe_status_query see it as they see moe_forward. */
+moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_router* router,
+                           const moe_experts_fp8* experts, const moe_experts_fp8* shared, int32_t K,
+                           void* out, void* stream);
 
 /* Stream-ordered copies of the last forward's routing into device buffers
  * (any may be NULL): idx int32 [T, K] and gate float32 [T, K] (Sel_t and
@@ -188,10 +227,8 @@ typedef enum moe_kernel_id {
   MOE_KERNEL_ROUTER = 0,   /* affinities, top-K, histogram, scan */
   MOE_KERNEL_PERMUTE = 1,  /* expert-contiguous rows of x */
   MOE_KERNEL_GATE_UP = 2,  /* SwiGLU(x W_gate^T, x W_up^T): shared experts on x, routed ones grouped */
-  MOE_KERNEL_DOWN = 3,     /* shared experts: Hs W_down^T; routed experts: g * (H W_down^T); for batches
-                              of more than 64 tokens also h = x + shared + sum_k g * routed, k ascending */
-  MOE_KERNEL_COMBINE = 4,  /* h = x + shared + sum_k g * routed, k ascending, as a kernel of its own:
-                              batches of at most 64 tokens only (no launch for larger ones) */
+  MOE_KERNEL_DOWN = 3,     /* shared experts: Hs W_down^T; routed experts: g * (H W_down^T) */
+  MOE_KERNEL_COMBINE = 4,  /* h = x + shared + sum_k g * routed, k ascending */
   MOE_KERNEL_COUNT = 5
 } moe_kernel_id;
 #define MOE_TIMING_ALL ((1u << MOE_KERNEL_COUNT) - 1u)

@@ -52,6 +52,11 @@ def _cfg(**kw):
     ({"gate": 7}, B.MOE_ERR_INVALID_ARG),
     ({"flags": 0x40}, B.MOE_ERR_INVALID_ARG),
     ({"n_shared": 0, "d_ff_shared": 0}, B.MOE_OK),
+    # the FP8 workspace wants 128-column groups
+    ({"flags": 0x8}, B.MOE_OK),
+    ({"flags": 0x8, "d_ff": 208}, B.MOE_ERR_ALIGNMENT),
+    ({"flags": 0x8, "d_ff_shared": 144}, B.MOE_ERR_ALIGNMENT),
+    ({"flags": 0x8, "d_model": 272}, B.MOE_ERR_ALIGNMENT),
 ])
 def test_config_validation(kw, status):
     st, nbytes = B.moe_workspace_bytes(_cfg(**kw))
@@ -64,6 +69,9 @@ def test_config_validation(kw, status):
 
 
 def test_workspace_grows_with_the_layer():
+    _, plain = B.moe_workspace_bytes(_cfg())
+    _, fp8 = B.moe_workspace_bytes(_cfg(flags=0x8))
+    assert fp8 > plain
     _, small = B.moe_workspace_bytes(_cfg())
     _, big = B.moe_workspace_bytes(_cfg(max_tokens=4096))
     _, wider = B.moe_workspace_bytes(_cfg(d_model=512))

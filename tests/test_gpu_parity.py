@@ -443,10 +443,8 @@ def test_timing_records_only_the_kernels_asked_for():
     assert all(n == 0 for k, (_, n) in t.items() if k != "gate_up")
     layer.set_timing(True)
     H.run(layer, dev["x"], shape.K)
-    # a 512-token batch sums the output in the down kernel's epilogue: no combine launch
-    assert {k: n for k, (_, n) in layer.kernel_times().items()} == \
-        {"router": 1, "permute": 1, "gate_up": 1, "down": 1, "combine": 0}
-    small = dev["x"][:40].contiguous()          # a decode-sized batch launches all five
+    assert all(n == 1 for _, n in layer.kernel_times().values())
+    small = dev["x"][:40].contiguous()          # a decode-sized batch (the decode GEMMs) launches the same five
     H.run(layer, small, shape.K)
     assert all(n == 1 for _, n in layer.kernel_times().values())
     layer.set_timing(False)
