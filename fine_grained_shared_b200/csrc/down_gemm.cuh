@@ -36,9 +36,10 @@
 // Epilogue: Y[row, n0 + c] = g[row] * acc[c] (bf16) for routed tiles and
 // Ys[row, n0 + c] = acc[c] for shared ones.  The layer's final k-ordered sum
 // runs in combine_kernel, which streams whole rows (permute.cuh): summing in
-// this epilogue, each chunk by the last of its K + 1 producers, left the
-// epilogue warps waiting on scattered row reads longer than the next tile's
-// MMAs (16B prefill: down 0.92 ms against 0.56 + 0.145 ms for down + combine).
+// this epilogue, each output chunk by the last of its K + 1 producers to
+// arrive, left the epilogue warps waiting on scattered row reads longer than
+// the next tile's MMAs (16B prefill: down 0.92 ms against 0.56 + 0.145 ms for
+// down and combine).
 #pragma once
 
 #include "sm100.cuh"
@@ -75,10 +76,9 @@ struct GemmArgs {
   int sh_k_per_j;              // Hs columns per shared expert (I_s)
   __nv_bfloat16* sh_out;       // Ys
   // both parts
-  int n_tiles;                 // routed n-tiles (down: 256 output columns over d; gate/up: 128 H columns)
-  int n_limit;                 // valid output columns of out (down: d; gate/up: I)
+  int n_tiles;                 // 256-column output tiles (over d)
+  int n_limit;                 // valid output columns (d)
   int ld_out;
-  int sh_n_tiles, sh_n_limit, sh_ld_out;  // the same for the shared experts' output
   uint32_t* err;
   uint64_t timeout_ns;
   int debug_wait;              // CTA 0 waits on a barrier nothing arrives on
@@ -96,14 +96,14 @@ struct TileCoord {
 
 // tiles [0, sh_tiles) are the shared experts' (m-tile major); the rest are
 // the routed experts', expert by expert
-__device__ __forceinline__ TileCoord decode_tile(int tile, int sh_tiles, int sh_n_tiles, const int32_t* s_mts,
+__device__ __forceinline__ TileCoord decode_tile(int tile, int sh_tiles, const int32_t* s_mts,
                                                  const int32_t* s_rows, int G, int n_tiles) {
   TileCoord c;
   if (tile < sh_tiles) {
     c.shared = 1;
     c.g = 0;
-    c.m_tile = tile / sh_n_tiles;
-    c.n_tile = tile - c.m_tile * sh_n_tiles;
+    c.m_tile = tile / n_tiles;
+    c.n_tile = tile - c.m_tile * n_tiles;
     c.row0 = c.m_tile * kGemmBM;
     return c;
   }
@@ -133,20 +133,12 @@ __device__ __forceinline__ void pair_record_error(uint32_t* err, volatile int* a
   atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
 }
 
-// GU = false (the down projection): tmA: H rows; tmB: W_down as [experts][d][I]
-// (each CTA stages its 128 of the tile's 256 output columns); tmAs: Hs rows;
-// tmBs: the shared experts' W_down as [K_s][d][I_s].  tmB2 / tmBs2 unused.
-// GU = true (the gate/up projection on CTA pairs): tmA: X_perm rows, tmAs: x
-// rows; the even CTA stages 128 rows of W_gate (tmB, tmBs) and the odd CTA the
-// same 128 rows of W_up (tmB2, tmBs2), so the pair's N = 256 accumulator holds
-// gate and up side by side in each CTA's TMEM lanes, and the epilogue stores
-// SiLU(gate) * up.  Maps of an absent part are never read.
-template <bool GU>
+// tmA: H rows; tmB: W_down as [experts][d][I].  tmAs: Hs rows; tmBs: the
+// shared experts' W_down as [K_s][d][I_s].  Maps of an absent part are never
+// read.
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmAs,
-                     const __grid_constant__ CUtensorMap tmBs, const __grid_constant__ CUtensorMap tmBs2,
-                     GemmArgs a) {
+    down_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmAs, const __grid_constant__ CUtensorMap tmBs, GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -168,7 +160,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
   const int G = a.num_groups;
-  const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGemmBM - 1) / kGemmBM * a.sh_n_tiles : 0;
+  const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGemmBM - 1) / kGemmBM * a.n_tiles : 0;
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
       mbar_init(&full[s], 1);
@@ -206,22 +198,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------ TMA producer ------------------------------
     if (G) {
       tma_prefetch_desc(&tmA);
-      tma_prefetch_desc(GU && rank ? &tmB2 : &tmB);
+      tma_prefetch_desc(&tmB);
     }
     if (sh_tiles) {
       tma_prefetch_desc(&tmAs);
-      tma_prefetch_desc(GU && rank ? &tmBs2 : &tmBs);
+      tma_prefetch_desc(&tmBs);
     }
     int s = 0, issued = 0;
     uint32_t ph = 0;
     for (int tile = pair; tile < total_tiles && !aborted; tile += num_pairs) {
-      const TileCoord c = decode_tile(tile, sh_tiles, a.sh_n_tiles, s_mts, s_rows, G, a.n_tiles);
+      const TileCoord c = decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
       const int row0 = c.row0 + static_cast<int>(rank) * kCtaRows;
-      // down: each CTA stages its half of the tile's 256 output columns of W_down;
-      // gate/up: the even CTA the tile's 128 rows of W_gate, the odd CTA those of W_up
-      const int brow = GU ? c.n_tile * (kGemmBN / 2) : c.n_tile * kGemmBN + static_cast<int>(rank) * (kGemmBN / 2);
+      // each CTA stages its half of the tile's 256 output columns of W_down
+      const int brow = c.n_tile * kGemmBN + static_cast<int>(rank) * (kGemmBN / 2);
       const CUtensorMap* mA = c.shared ? &tmAs : &tmA;
-      const CUtensorMap* mB = c.shared ? (GU && rank ? &tmBs2 : &tmBs) : (GU && rank ? &tmB2 : &tmB);
+      const CUtensorMap* mB = c.shared ? &tmBs : &tmB;
       const int J = c.shared ? a.sh_J : 1;
       const int num_kb = c.shared ? a.sh_num_kb : a.num_kb;
       for (int j = 0; j < J && !aborted; ++j) {
@@ -311,7 +302,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = pair; tile < total_tiles; tile += num_pairs) {
-      const TileCoord c = decode_tile(tile, sh_tiles, a.sh_n_tiles, s_mts, s_rows, G, a.n_tiles);
+      const TileCoord c = decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
       bool ok = mbar_wait(&acc_full[acc], acc_ph, a.timeout_ns, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -323,41 +314,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tb = tmem + static_cast<uint32_t>(acc * kGemmBN) + (static_cast<uint32_t>(q * 32) << 16);
       const size_t row = static_cast<size_t>(c.row0) + rank * kCtaRows + r;
 
-      const int n_limit = c.shared ? a.sh_n_limit : a.n_limit;
-      __nv_bfloat16* orow = (c.shared ? a.sh_out : a.out) + row * (c.shared ? a.sh_ld_out : a.ld_out);
-      if (GU) {
-        // H[row, n0 + cc] = SiLU(gate) * up: TMEM columns [0, 128) gate, [128, 256) up
-        const int n0 = c.n_tile * (kGemmBN / 2);
-#pragma unroll 1
-        for (int cc = 0; cc < kGemmBN / 2; cc += 16) {
-          uint32_t gr[16], ur[16];
-          tmem_ld16(tb + cc, gr);
-          tmem_ld16(tb + kGemmBN / 2 + cc, ur);
-          tmem_ld_wait();
-          const int col = n0 + cc;
-          if (col < n_limit) {
-            uint32_t pk[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float g0 = __uint_as_float(gr[2 * j]), g1 = __uint_as_float(gr[2 * j + 1]);
-              const float u0 = __uint_as_float(ur[2 * j]), u1 = __uint_as_float(ur[2 * j + 1]);
-              pk[j] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(orow + col);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-          }
-        }
-      } else {
+      {
         const int n0 = c.n_tile * kGemmBN;
         const float sc = c.shared ? 1.f : a.row_scale[row];
+        __nv_bfloat16* orow = (c.shared ? a.sh_out : a.out) + row * a.ld_out;
 #pragma unroll 1
         for (int cc = 0; cc < kGemmBN; cc += 16) {
           uint32_t vr[16];
           tmem_ld16(tb + cc, vr);
           tmem_ld_wait();
           const int col = n0 + cc;
-          if (col < n_limit) {
+          if (col < a.n_limit) {
             uint32_t pk[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j)

@@ -46,11 +46,7 @@ static_assert(kDecBoxRowsW == kGuBoxRowsB && kDecBoxRowsW == kBoxRowsB,
 #ifndef FGS_DECODE_MAX_T
 #define FGS_DECODE_MAX_T 64
 #endif
-// 1: the gate/up projection of larger batches runs on CTA pairs (pair_gemm_kernel<true>,
-// 256 x 256 tiles with the 2-SM MMA); 0: on single SMs (gateup_gemm_kernel, 128 x 256 tiles).
-#ifndef FGS_GATEUP_PAIR
-#define FGS_GATEUP_PAIR 0
-#endif
+
 
 namespace {
 
@@ -351,8 +347,7 @@ cudaError_t set_kernel_attrs() {
   const int us = static_cast<int>(gateup_smem_bytes());
   if ((e = cudaFuncSetAttribute(gateup_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
   const int gs = static_cast<int>(gemm_smem_bytes());
-  if ((e = cudaFuncSetAttribute(pair_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
-  if ((e = cudaFuncSetAttribute(pair_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
+  if ((e = cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
   if ((e = cudaFuncSetAttribute(decode_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(dec_smem_bytes<true>()))))
     return e;
@@ -391,8 +386,8 @@ bool refresh(MapCache& c, const void* p, int64_t rows_key, uint64_t d2, uint64_t
 // Launch `pairs` CTA pairs (clusters of 2) of the down GEMM kernel.
 cudaError_t launch_down(int pairs, cudaStream_t s, bool pdl, const CUtensorMap& A, const CUtensorMap& B,
                         const CUtensorMap& As, const CUtensorMap& Bs, const GemmArgs& ga) {
-  return launch_pdl(pair_gemm_kernel<false>, dim3(2 * pairs), dim3(kGemmThreads), gemm_smem_bytes(), s, 2, pdl, A, B, B,
-                    As, Bs, Bs, ga);
+  return launch_pdl(down_gemm_kernel, dim3(2 * pairs), dim3(kGemmThreads), gemm_smem_bytes(), s, 2, pdl, A, B, As, Bs,
+                    ga);
 }
 
 template <bool GU>
@@ -617,7 +612,7 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
     lc.attrs = attr;
     lc.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, pair_gemm_kernel<false>, &lc) != cudaSuccess || clusters < 1) {
+    if (cudaOccupancyMaxActiveClusters(&clusters, down_gemm_kernel, &lc) != cudaSuccess || clusters < 1) {
       cudaGetLastError();
       delete h;
       return MOE_ERR_CUDA;
@@ -829,36 +824,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     const CUtensorMap& sA = do_shared ? h->tm_x.map : h->tm_xperm;
     const CUtensorMap& sG = do_shared ? h->tm_swg.map : h->tm_wg.map;
     const CUtensorMap& sU = do_shared ? h->tm_swu.map : h->tm_wu.map;
-    if (FGS_GATEUP_PAIR) {
-      GemmArgs gp{};
-      if (do_routed) {
-        gp.num_groups = (int)N;
-        gp.mtile_start = ra.mtile_start;
-        gp.row_start = ra.row_start;
-        gp.num_kb = num_kb;
-        gp.out = h->at<__nv_bfloat16>(L.h);
-        gp.ld_out = (int)I;
-        gp.n_tiles = ceil_div(I, kGemmBN / 2);
-        gp.n_limit = (int)I;
-      }
-      if (do_shared) {
-        gp.sh_rows = (int)T;
-        gp.sh_num_kb = num_kb;
-        gp.sh_J = 1;
-        gp.sh_out = h->at<__nv_bfloat16>(L.hs);
-        gp.sh_ld_out = (int)(Ks * Is);
-        gp.sh_n_tiles = ceil_div(Ks * Is, kGemmBN / 2);
-        gp.sh_n_limit = (int)(Ks * Is);
-      }
-      gp.err = h->at<uint32_t>(L.err);
-      gp.timeout_ns = kTimeoutNs;
-      const int sh_pt = do_shared ? ceil_div(T, kGemmBM) * gp.sh_n_tiles : 0;
-      const int pairs = do_routed || sh_pt > h->max_pairs ? h->max_pairs : sh_pt;
-      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
-      if (launch_pdl(pair_gemm_kernel<true>, dim3(2 * pairs), dim3(kGemmThreads), gemm_smem_bytes(), s0, 2, pdl,
-                     h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, gp) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    } else {
+    {
       KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
       if (launch_gateup(ctas, s0, pdl, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g) != cudaSuccess)
         return MOE_ERR_CUDA;
@@ -883,9 +849,6 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     g2.n_tiles = ceil_div(d, kGemmBN);
     g2.n_limit = (int)d;
     g2.ld_out = (int)d;
-    g2.sh_n_tiles = g2.n_tiles;
-    g2.sh_n_limit = (int)d;
-    g2.sh_ld_out = (int)d;
     g2.err = h->at<uint32_t>(L.err);
     g2.timeout_ns = kTimeoutNs;
     const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
