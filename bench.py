@@ -60,6 +60,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-per-config", action="store_true",
                    help="measure only the --config workload (by default the 2B, 16B decode and V3 layers follow)")
+    p.add_argument("--fp8", action="store_true",
+                   help="the layer with FP8 expert GEMMs (moe_forward_fp8) on the --config workload alone")
     p.add_argument("--fp8-quant", action="store_true",
                    help="time the FP8 1x128 quantization of one forward's permuted activations instead")
     return p.parse_args()
@@ -202,35 +204,39 @@ def host_cpu():
     return os.cpu_count() or 1, model
 
 
-def oracle_tokens_per_s(shape: W.LayerShape, host: dict, n_tokens: int, repeats: int = 1):
+def oracle_tokens_per_s(shape: W.LayerShape, host: dict, n_tokens: int, repeats: int = 1, fp8: bool = False):
     """The CPU oracle, as it stands, on ``n_tokens`` seeded tokens of the batch, on ONE thread (numpy's
-    BLAS limited to one thread for the call): the plain single-threaded baseline."""
+    BLAS limited to one thread for the call): the plain single-threaded baseline.  fp8: the FP8 layer's
+    oracle (expert operands quantized as the FP8 path quantizes them)."""
     import oracle as O
+    import oracle.fp8 as F8
     from threadpoolctl import threadpool_limits
     rows = W.sample_tokens(shape, n_tokens)
     ex = (host["w_gate"], host["w_up"], host["w_down"])
     sh = (host["ws_gate"], host["ws_up"], host["ws_down"]) if shape.Ks else None
+    fwd = F8.moe_forward_fp8 if fp8 else O.moe_forward
     times = []
     with threadpool_limits(limits=1):
         for _ in range(repeats):
             t0 = time.perf_counter()
-            O.moe_forward(host["x"], host["router"], shape.K, ex, sh, gate_kind=shape.gate,
-                          logit_bias=host["logit_bias"], select_bias=host["select_bias"], rows=rows)
+            fwd(host["x"], host["router"], shape.K, ex, sh, gate_kind=shape.gate,
+                logit_bias=host["logit_bias"], select_bias=host["select_bias"], rows=rows)
             times.append(time.perf_counter() - t0)
     return rows.size, times, 1
 
 
-def cpu_baseline(shape: W.LayerShape, host: dict, seconds: float = 15.0, max_tokens: int = 4096):
+def cpu_baseline(shape: W.LayerShape, host: dict, seconds: float = 15.0, max_tokens: int = 4096,
+                 fp8: bool = False):
     """The oracle on a bounded sample sized to about ``seconds`` of one core's work (calibrated on 64
     tokens, which already pay the per-expert weight conversions)."""
-    n_cal, t_cal, _ = oracle_tokens_per_s(shape, host, 64)
+    n_cal, t_cal, _ = oracle_tokens_per_s(shape, host, 64, fp8=fp8)
     n = int(max(8, min(shape.T, max_tokens, seconds * n_cal / max(t_cal[0], 1e-6))))
-    n, times, threads = oracle_tokens_per_s(shape, host, n)
+    n, times, threads = oracle_tokens_per_s(shape, host, n, fp8=fp8)
     cores, model = host_cpu()
     return {"value": n / times[0], "unit": UNIT, "cores": threads, "kind": "oracle",
             "host_cores": cores, "cpu_model": model,
             "sample": f"{n} seeded tokens of the T={shape.T} batch (routing, routed and shared experts, final "
-                      f"sum; float64 numpy on one thread), {times[0]:.1f} s"}
+                      f"sum; {'the FP8 layer, ' if fp8 else ''}float64 numpy on one thread), {times[0]:.1f} s"}
 
 
 def run_reference(args):
@@ -376,31 +382,39 @@ def choose_peak(peaks: dict, timed_s: float, clk) -> tuple:
     return float(peaks["bf16_tflops_sustained"]), "bf16_tflops_sustained"
 
 
-def touched_weight_bytes(shape: W.LayerShape, counts) -> dict:
+def touched_weight_bytes(shape: W.LayerShape, counts, fp8: bool = False) -> dict:
     """Expert weights each GEMM launch must stream: every routed expert that received a token, and
-    the shared experts (gate/up: W_gate and W_up; down: W_down)."""
+    the shared experts (gate/up: W_gate and W_up; down: W_down); bf16, or FP8 codes with one scale
+    byte per 128 x 128 block."""
     touched = int(sum(1 for c in counts if c > 0))
-    per_proj = 2.0 * shape.d * (touched * shape.I + shape.Ks * shape.Is)
+    per_elem = (1.0 + 1.0 / (128 * 128)) if fp8 else 2.0
+    per_proj = per_elem * shape.d * (touched * shape.I + shape.Ks * shape.Is)
     return {"touched_experts": touched, "gate_up": 2 * per_proj, "down": per_proj, "layer": 3 * per_proj}
 
 
 def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: int, ranks, steps: int,
-                  warmup: int, with_e2e: bool):
+                  warmup: int, with_e2e: bool, fp8: bool = False):
     """Time `steps` forwards of one layer on its resident inputs (CUDA events on the launching stream,
     barrier + synchronize on both sides, max over ranks) with events around the dominant kernel, then
-    every kernel in a separate pass, then (optionally) the host-buffer entry point."""
+    every kernel in a separate pass, then (optionally) the host-buffer entry point.  fp8: the FP8 layer
+    (moe_forward_fp8) on weights block-quantized by the library beforehand (not timed)."""
     world = ranks.world
     layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks,
                        d_ff_shared=shape.Is, max_tokens=shape.T, max_k=shape.K, gate=shape.gate,
-                       device=local)
+                       device=local, flags=B.MOE_FLAG_FP8 if fp8 else 0)
     shared = (d_in["ws_gate"], d_in["ws_up"], d_in["ws_down"]) if shape.Ks else None
     layer.set_weights(d_in["router"], (d_in["w_gate"], d_in["w_up"], d_in["w_down"]), shared,
                       logit_bias=d_in["logit_bias"], select_bias=d_in["select_bias"])
+    if fp8:
+        layer.set_weights_fp8(tuple(B.quantize_fp8_blocks(d_in[k]) for k in ("w_gate", "w_up", "w_down")),
+                              tuple(B.quantize_fp8_blocks(d_in[k]) for k in ("ws_gate", "ws_up", "ws_down"))
+                              if shape.Ks else None)
+    fwd = layer.forward_fp8 if fp8 else layer.forward
     x = d_in["x"]
     out = torch.empty_like(x)
     stream = torch.cuda.current_stream(dev)
     for _ in range(warmup):
-        layer.forward(x, shape.K, out)
+        fwd(x, shape.K, out)
     st = layer.status()
     if st != B.MOE_OK:
         raise B.MoEError(st, f"{shape.name} warm-up")
@@ -415,7 +429,7 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
     torch.cuda.synchronize(dev)
     start.record(stream)
     for _ in range(steps):
-        layer.forward(x, shape.K, out)
+        fwd(x, shape.K, out)
     end.record(stream)
     torch.cuda.synchronize(dev)
     ranks.barrier()
@@ -430,7 +444,7 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
     pass_steps = max(1, min(steps, 50))
     layer.set_timing(True)
     for _ in range(pass_steps):
-        layer.forward(x, shape.K, out)
+        fwd(x, shape.K, out)
     all_ktimes = layer.kernel_times()
     layer.set_timing(False)
     r = {"ms_total": ms_total, "ms_step": ms_total / steps, "clocks": clk,
@@ -445,14 +459,26 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
         x_h = host["x"].pin_memory()
         out_h = torch.empty_like(x_h).pin_memory()
         e2e_steps = max(1, min(steps, 100))
+        if fp8:
+            # pinned x in, moe_forward_fp8, the output back: all on the stream, the read synchronised
+            xd = torch.empty_like(x)
+
+            def host_step():
+                xd.copy_(x_h, non_blocking=True)
+                layer.forward_fp8(xd, shape.K, out)
+                out_h.copy_(out, non_blocking=True)
+                torch.cuda.current_stream(dev).synchronize()
+        else:
+            def host_step():
+                layer.forward_host(x_h, shape.K, out_h)
         for _ in range(3):
-            layer.forward_host(x_h, shape.K, out_h)
+            host_step()
         ranks.barrier()
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(e2e_steps):
-            layer.forward_host(x_h, shape.K, out_h)
+            host_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ranks.barrier()
@@ -464,21 +490,26 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
     return r
 
 
-def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffic=None):
+def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffic=None, fp8: bool = False):
     """Roofline of the dominant kernel (the shared + routed gate/up GEMM with SwiGLU): tensor-bound
     when the routed experts' FLOPs per weight byte exceed the ridge (sustained bf16 FLOP/s over copy
-    bandwidth), else HBM-bound over the weights of the touched experts (the weight-streaming regime)."""
+    bandwidth), else HBM-bound over the weights of the touched experts (the weight-streaming regime).
+    fp8: the FP8 layer, against twice the measured bf16 peak (the nominal FP8 / bf16 ratio of the
+    tensor cores) and over 1-byte weights (plus one scale byte per 128 x 128 block)."""
     peak_flops, peak_name = choose_peak(peaks, r["ms_total"] * 1e-3, r["clocks"])
+    if fp8:
+        peak_flops, peak_name = 2.0 * peak_flops, f"2 x {peak_name} (fp8 = 2 x bf16, nominal ratio)"
     k_flop = 4.0 * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is)
-    wb = touched_weight_bytes(shape, r["counts"])
+    wb = touched_weight_bytes(shape, r["counts"], fp8)
     k_avg_ms = r["dominant_ms"]
     hbm = float(peaks["hbm_gbs"])
     if k_flop / wb["gate_up"] > float(peaks["bf16_tflops_sustained"]) * 1e12 / (hbm * 1e9):
         achieved = k_flop / (k_avg_ms * 1e-3) / 1e12
+        mult = 2.0 if fp8 else 1.0
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak_flops, "unit": "TFLOP/s",
                 "peak_source": f"{peak_src} {peak_name}",
-                "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
-                "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"])}
+                "frac_of_burst": achieved / (mult * float(peaks["bf16_tflops"])),
+                "frac_of_sustained": achieved / (mult * float(peaks["bf16_tflops_sustained"]))}
     else:
         achieved = wb["gate_up"] / (k_avg_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
@@ -490,10 +521,10 @@ def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffi
     return roof, peak_flops, peak_name
 
 
-def hbm_fractions(shape: W.LayerShape, r: dict, peaks: dict) -> dict:
+def hbm_fractions(shape: W.LayerShape, r: dict, peaks: dict, fp8: bool = False) -> dict:
     """Each expert GEMM's and the whole layer's rate over the touched experts' weight bytes, as a
     fraction of the measured copy bandwidth (the roofline of the weight-streaming shapes)."""
-    wb = touched_weight_bytes(shape, r["counts"])
+    wb = touched_weight_bytes(shape, r["counts"], fp8)
     hbm = float(peaks["hbm_gbs"])
     out = {"touched_experts": wb["touched_experts"], "weight_bytes": wb["layer"]}
     for k in ("gate_up", "down"):
@@ -538,20 +569,26 @@ def run_ours(args):
     warmup = max(3, args.warmup)
 
     shape = W.CONFIGS[args.config]
+    fp8 = args.fp8
     host = host_inputs(shape)
     d_in = to_device(host, dev)
-    r = measure_layer(B, shape, host, d_in, dev, local, ranks, args.steps, warmup, with_e2e=True)
+    r = measure_layer(B, shape, host, d_in, dev, local, ranks, args.steps, warmup, with_e2e=True, fp8=fp8)
     del d_in
     torch.cuda.empty_cache()
 
     peaks, peak_src = measured_peaks()
-    roofline, peak_flops, peak_name = roofline_of(shape, r, peaks, peak_src, profiled_traffic(shape))
+    roofline, peak_flops, peak_name = roofline_of(shape, r, peaks, peak_src,
+                                                  None if fp8 else profiled_traffic(shape), fp8)
     layer_tflops = world * layer_flop(shape) / (r["ms_step"] * 1e-3) / 1e12
+    config = workload_config(shape, f"replicas{world}" if world > 1 else "single")
+    if fp8:
+        config["expert_gemms"] = ("fp8: E4M3 operands, 1x128 activation and 128x128 weight scales (UE8M0), "
+                                  "fp32 accumulation; router in bf16/fp32")
     line = {
         "metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": warmup, "ms_per_step": r["ms_step"], "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(shape, f"replicas{world}" if world > 1 else "single"),
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3" if fp8 else "bf16", "data": "synthetic",
+        "config": config,
         "tflops": layer_tflops,
         "tflops_frac_of_peak": layer_tflops / (world * peak_flops),
         "tflops_peak": f"{peak_src} {peak_name}",
@@ -562,15 +599,15 @@ def run_ours(args):
         "clocks": r["clocks"],
     }
     if roofline["bound"] == "hbm":
-        line["hbm"] = hbm_fractions(shape, r, peaks)
+        line["hbm"] = hbm_fractions(shape, r, peaks, fp8)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(shape, host)
+        line["cpu_baseline"] = cpu_baseline(shape, host, fp8=fp8)
 
     # the other single-GPU workloads, measured after the headline one: ms per step, tokens/s and the
     # roofline that bounds each (tensor for the 2B layer, HBM over the touched experts' weights for
     # the 16B decode and V3 layers)
-    if not args.no_per_config:
+    if not args.no_per_config and not fp8:
         per = {}
         for name in PER_CONFIG:
             if name == args.config:
