@@ -115,20 +115,32 @@ struct DecodeArgs {
   uint64_t timeout_ns;
 };
 
-// Equal contiguous ranges of a space's `total` k-blocks over `workers` CTAs:
-// range c is [bound(c), bound(c + 1)).
+// Contiguous ranges of a space's `total` k-blocks over `workers` CTAs: range
+// c is [bound(c), bound(c + 1)).  Plain: equal ranges.  With lead tiles
+// (lead > 0): the first `lead` CTAs each also run one whole tile of lead_kbt
+// k-blocks of another space, and the ranges of this space are shifted so
+// that every CTA's total comes out equal:
+//   bound(c) = max(0, floor(c (total + lead lead_kbt) / workers) - min(c, lead) lead_kbt),
+// which is non-decreasing and reaches total at c = workers.
 struct DecSpace {
   long long total;
   int workers, kbt;  // kbt: k-blocks of every tile of the space
+  int lead, lead_kbt;
   __device__ __forceinline__ long long bound(int c) const {
-    return static_cast<long long>(c) * total / workers;
+    const long long all = total + static_cast<long long>(lead) * lead_kbt;
+    const long long b = static_cast<long long>(c) * all / workers - static_cast<long long>(min(c, lead)) * lead_kbt;
+    return b < 0 ? 0 : b;
   }
-  // the CTA whose range holds k-block x (empty ranges hold none)
+  // the CTA whose range holds k-block x: the largest c with bound(c) <= x
+  // (empty ranges hold none)
   __device__ __forceinline__ int cta_of(long long x) const {
-    int c = static_cast<int>(x * workers / total);
-    while (c + 1 < workers && bound(c + 1) <= x) ++c;
-    while (c > 0 && bound(c) > x) --c;
-    return c;
+    int lo = 0, hi = workers;  // bound(lo) <= x < bound(hi), bound(workers) = total
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (bound(mid) <= x) lo = mid;
+      else hi = mid;
+    }
+    return lo;
   }
 };
 
@@ -136,6 +148,8 @@ __device__ __forceinline__ DecSpace dec_space(long long tiles, int kbt, int ctas
   DecSpace s;
   s.total = tiles * kbt;
   s.kbt = kbt > 0 ? kbt : 1;
+  s.lead = 0;
+  s.lead_kbt = 0;
   const long long w = s.total / kDecMinIters;
   s.workers = static_cast<int>(w < 1 ? 1 : w > ctas ? ctas : w);
   if (s.total == 0) s.workers = 1;
@@ -256,7 +270,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int ctas = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
   const long long sh_tiles =
       a.sh_rows > 0 ? static_cast<long long>((a.sh_rows + kDecTB - 1) / kDecTB) * a.sh_n_wb : 0;
-  const DecSpace sp0 = dec_space(sh_tiles, a.sh_J * a.sh_kb_per_j, ctas);
+  // The shared experts' tiles need neither the router nor the permutation
+  // (they run before the grid dependency wait).  When they fit one per CTA
+  // the first sh_tiles CTAs each run one whole (no tile is cut, so no partial
+  // sums are summed later), and the routed ranges are shifted to even out
+  // every CTA's k-blocks; otherwise the shared space is cut like the routed
+  // one.  (Cutting every shared tile between ~7 CTAs left the CTAs that sum
+  // the parts up to 50 us behind the rest on the 16B decode layer.)
+  const int sh_kbt = a.sh_J * a.sh_kb_per_j;
+  const bool sh_whole = sh_tiles > 0 && sh_tiles <= ctas;
+  const DecSpace sp0 = dec_space(sh_whole ? 0 : sh_tiles, sh_kbt, ctas);
 
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
@@ -287,8 +310,34 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // after the grid dependency wait and publishes them on `tables`
   auto routed_space = [&]() {
     const long long tiles = G ? static_cast<long long>(s_tbs[G]) * a.n_wb : 0;
-    return dec_space(tiles, a.num_kb, ctas);
+    DecSpace sp = dec_space(tiles, a.num_kb, ctas);
+    // shifted ranges only when every CTA's range keeps at least kDecMinIters
+    // k-blocks (a split tile's parts must come from consecutive CTAs, none
+    // empty); a small batch keeps the plain ranges and the lead CTAs' extra tile
+    const long long all = tiles * a.num_kb + sh_tiles * sh_kbt;
+    if (sh_whole && all / ctas >= sh_kbt + kDecMinIters) {
+      sp.workers = ctas;
+      sp.lead = static_cast<int>(sh_tiles);
+      sp.lead_kbt = sh_kbt;
+    }
+    return sp;
   };
+  // the shared segments of CTA c: one whole tile, or its cut range
+  auto shared_walk = [&]() {
+    DecWalk w = dec_walk(sp0, c);
+    if (sh_whole) {
+      w.kbt = sh_kbt;
+      w.x = c < sh_tiles ? static_cast<long long>(c) * sh_kbt : 0;
+      w.end = c < sh_tiles ? w.x + sh_kbt : 0;
+    }
+    return w;
+  };
+  // a whole shared tile is never cut: the space's k-block count of a tile
+  const DecSpace sp0w = [&]() {
+    DecSpace t = sp0;
+    if (sh_whole) t.kbt = sh_kbt;
+    return t;
+  }();
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
@@ -337,7 +386,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (GU) tma_prefetch_desc(&tmW1);
         tma_prefetch_desc(&tmX);
       }
-      DecWalk w = dec_walk(sp0, c);
+      DecWalk w = shared_walk();
       long long tile;
       int k0, k1;
       while (!stop && w.next(tile, k0, k1)) load_segment(true, dec_shared_tile(tile, a.sh_rows), k0, k1);
@@ -430,7 +479,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     };
     {
-      DecWalk w = dec_walk(sp0, c);
+      DecWalk w = shared_walk();
       long long tile;
       int k0, k1;
       while (!stop && w.next(tile, k0, k1)) mma_segment(k0, k1);
@@ -552,10 +601,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     };
     {
-      DecWalk w = dec_walk(sp0, c);
+      DecWalk w = shared_walk();
       long long tile;
       int k0, k1;
-      while (!stop && w.next(tile, k0, k1)) epilogue(0, sp0, tile, k0, k1, true, dec_shared_tile(tile, a.sh_rows));
+      while (!stop && w.next(tile, k0, k1)) epilogue(0, sp0w, tile, k0, k1, true, dec_shared_tile(tile, a.sh_rows));
     }
     bool okt = stop ? false : mbar_wait(tables, 0, a.timeout_ns, abort_flag);
     okt = __all_sync(0xffffffffu, okt);

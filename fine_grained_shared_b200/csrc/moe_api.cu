@@ -208,6 +208,12 @@ moe_status check_config(const moe_config* c) {
   if (c->flags & ~known) return MOE_ERR_INVALID_ARG;
   if ((c->flags & MOE_FLAG_FP8) && (c->d_model % 128 || c->d_ff % 128 || (c->n_shared > 0 && c->d_ff_shared % 128)))
     return MOE_ERR_ALIGNMENT;
+  if (c->route_nodes != 0 || c->route_max_nodes != 0) {
+    if (c->route_nodes < 1 || c->route_nodes > kMaxRouteNodes || c->n_routed % c->route_nodes ||
+        c->route_max_nodes < 1 || c->route_max_nodes > c->route_nodes ||
+        c->max_k > c->route_max_nodes * (c->n_routed / c->route_nodes))
+      return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 
@@ -306,8 +312,12 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 template <int K>
 cudaError_t launch_router_k(bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, bool pdl, const CUtensorMap& tx,
                             const CUtensorMap& te, const RouterArgs& ra) {
-  return sigmoid ? launch_pdl(router_topk_kernel<K, true>, grid, dim3(kRouterThreads), smem, s, 1, pdl, tx, te, ra)
-                 : launch_pdl(router_topk_kernel<K, false>, grid, dim3(kRouterThreads), smem, s, 1, pdl, tx, te, ra);
+  const dim3 b(kRouterThreads);
+  if (ra.nodes > 0)
+    return sigmoid ? launch_pdl(router_topk_kernel<K, true, true>, grid, b, smem, s, 1, pdl, tx, te, ra)
+                   : launch_pdl(router_topk_kernel<K, false, true>, grid, b, smem, s, 1, pdl, tx, te, ra);
+  return sigmoid ? launch_pdl(router_topk_kernel<K, true, false>, grid, b, smem, s, 1, pdl, tx, te, ra)
+                 : launch_pdl(router_topk_kernel<K, false, false>, grid, b, smem, s, 1, pdl, tx, te, ra);
 }
 
 cudaError_t launch_router(int K, bool sigmoid, dim3 grid, size_t smem, cudaStream_t s, bool pdl,
@@ -326,11 +336,13 @@ cudaError_t launch_router(int K, bool sigmoid, dim3 grid, size_t smem, cudaStrea
 
 template <int K>
 cudaError_t set_router_attrs_k(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(router_topk_kernel<K, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(router_topk_kernel<K, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(smem));
+  const int sm = static_cast<int>(smem);
+  const auto attr = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(router_topk_kernel<K, true, false>, attr, sm)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(router_topk_kernel<K, false, false>, attr, sm)) != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(router_topk_kernel<K, true, true>, attr, sm)) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(router_topk_kernel<K, false, true>, attr, sm);
 }
 
 cudaError_t set_kernel_attrs() {
@@ -485,6 +497,11 @@ moe_status enqueue_router(moe_ctx* h, const void* x, int64_t T, const moe_router
   ra.done_counter = h->at<uint32_t>(L.done);
   ra.err = h->at<uint32_t>(L.err);
   ra.timeout_ns = kTimeoutNs;
+  if (c.route_nodes > 0) {
+    ra.nodes = c.route_nodes;
+    ra.per_node = (int)(N / c.route_nodes);
+    ra.max_nodes = c.route_max_nodes;
+  }
   KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
   if (T <= kSmallRouterMaxT) {
     // a few tokens: one CTA per token on the CUDA cores

@@ -46,10 +46,10 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode_fn = nullptr;
 
 template <int K>
 cudaError_t set_attrs_k(size_t smem) {
-  cudaError_t e = cudaFuncSetAttribute(fgs::router_topk_kernel<K, true>,
+  cudaError_t e = cudaFuncSetAttribute(fgs::router_topk_kernel<K, true, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(fgs::router_topk_kernel<K, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(fgs::router_topk_kernel<K, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(smem));
 }
 
@@ -96,9 +96,9 @@ template <int K>
 void launch_k(bool sigmoid, int grid, size_t smem, cudaStream_t s, const CUtensorMap& tx, const CUtensorMap& te,
               const fgs::RouterArgs& ra) {
   if (sigmoid)
-    fgs::router_topk_kernel<K, true><<<grid, fgs::kRouterThreads, smem, s>>>(tx, te, ra);
+    fgs::router_topk_kernel<K, true, false><<<grid, fgs::kRouterThreads, smem, s>>>(tx, te, ra);
   else
-    fgs::router_topk_kernel<K, false><<<grid, fgs::kRouterThreads, smem, s>>>(tx, te, ra);
+    fgs::router_topk_kernel<K, false, false><<<grid, fgs::kRouterThreads, smem, s>>>(tx, te, ra);
 }
 
 }  // namespace

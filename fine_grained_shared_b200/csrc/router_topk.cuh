@@ -51,7 +51,32 @@ struct RouterArgs {
   uint32_t* done_counter;    // CTAs finished; reset to 0 by the last CTA
   uint32_t* err;
   uint64_t timeout_ns;
+  // node-limited routing (0 nodes: off): the mN experts sit on `nodes` nodes
+  // in contiguous ranges of per_node; each token's K experts come from at
+  // most max_nodes nodes, those holding its largest keys
+  int nodes, per_node, max_nodes;
 };
+
+constexpr int kMaxRouteNodes = 16;
+
+// The nodes a token may use: max_nodes rounds, each taking the unchosen node
+// with the largest key maximum (ties to the lower node), as a bit mask.
+__device__ __forceinline__ uint32_t choose_nodes(const float (&nmax)[kMaxRouteNodes], int nodes, int max_nodes) {
+  uint32_t chosen = 0u;
+  for (int m = 0; m < max_nodes; ++m) {
+    float bv = -INFINITY;
+    int bg = kMaxRouteNodes;
+#pragma unroll
+    for (int g = 0; g < kMaxRouteNodes; ++g) {
+      if (g < nodes && !((chosen >> g) & 1u) && (nmax[g] > bv || (nmax[g] == bv && g < bg))) {
+        bv = nmax[g];
+        bg = g;
+      }
+    }
+    chosen |= 1u << bg;
+  }
+  return chosen;
+}
 
 __host__ __device__ constexpr size_t router_smem_bytes(int Npad) {
   return 1024 + static_cast<size_t>(router_stages(Npad)) * (16384 + static_cast<size_t>(Npad) * 128) +
@@ -63,7 +88,11 @@ __device__ __forceinline__ void record_error(uint32_t* err, volatile int* abort,
   atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
 }
 
-template <int K, bool SIGMOID>
+// NL: node-limited routing -- a first pass over the token's logits in TMEM
+// takes each node's largest key and picks the allowed nodes (choose_nodes);
+// the top-K pass then skips the experts of the other nodes.  The softmax
+// statistics still cover every expert.
+template <int K, bool SIGMOID, bool NL>
 __global__ void __launch_bounds__(kRouterThreads, 1)
     router_topk_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_e,
                        RouterArgs a) {
@@ -195,6 +224,32 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
       }
       float mx = -INFINITY, sum = 0.f;
       const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t allowed = 0xffffffffu;  // bit g: node g may hold a selected expert
+      if (NL) {
+        float nmax[kMaxRouteNodes];
+#pragma unroll
+        for (int g = 0; g < kMaxRouteNodes; ++g) nmax[g] = -INFINITY;
+        for (int c0 = 0; c0 < a.Npad; c0 += 16) {
+          uint32_t rr[16];
+          tmem_ld16(tbase + c0, rr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = c0 + j;
+            if (col < a.N) {
+              // the key exactly as the top-K pass below computes it
+              const float z = __uint_as_float(rr[j]);
+              float key = SIGMOID ? 1.f / (1.f + __expf(-z)) + bias[col] : z + bias[col];
+              if (isnan(key)) key = -INFINITY;
+              const int node = col / a.per_node;
+#pragma unroll
+              for (int g = 0; g < kMaxRouteNodes; ++g)
+                if (g == node) nmax[g] = fmaxf(nmax[g], key);
+            }
+          }
+        }
+        allowed = choose_nodes(nmax, a.nodes, a.max_nodes);
+      }
       for (int c0 = 0; c0 < a.Npad; c0 += 16) {
         uint32_t rr[16];
         tmem_ld16(tbase + c0, rr);
@@ -223,6 +278,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
             // number; the index order then still fills the K slots with
             // distinct experts in [0, N)
             if (isnan(key)) key = -INFINITY;
+            if (NL && !((allowed >> (col / a.per_node)) & 1u)) continue;  // a node not chosen
             // insert (key, col) into the list ordered by (key descending,
             // index ascending); an element pushed down keeps competing by the
             // same order, so ties always go to the lower expert index
@@ -445,6 +501,21 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     }
+    // node-limited routing: each node's largest key, then the allowed nodes
+    uint32_t allowed = 0xffffffffu;
+    if (a.nodes > 0) {
+      float nmax[kMaxRouteNodes];
+#pragma unroll
+      for (int g = 0; g < kMaxRouteNodes; ++g) {
+        float m = -INFINITY;
+        if (g < a.nodes)
+          for (int i = g * a.per_node + lane; i < (g + 1) * a.per_node; i += 32) m = fmaxf(m, key[i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        nmax[g] = m;
+      }
+      allowed = choose_nodes(nmax, a.nodes, a.max_nodes);
+    }
     uint32_t taken = 0;  // bit j: this lane's expert lane + 32 * j is already selected
     int sel[8];
     float sel_s[8];
@@ -454,6 +525,7 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
       int bi = 0x7fffffff;
       for (int j = 0, i = lane; i < a.N; ++j, i += 32) {
         if (taken & (1u << j)) continue;
+        if (a.nodes > 0 && !((allowed >> (i / a.per_node)) & 1u)) continue;
         const float v = key[i];
         if (v > bk || (v == bk && i < bi)) {
           bk = v;

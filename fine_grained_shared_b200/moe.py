@@ -37,7 +37,8 @@ KERNEL_NAMES = ("router", "permute", "gate_up", "down", "combine")
 class moe_config(ctypes.Structure):
     _fields_ = [("d_model", c_int32), ("n_routed", c_int32), ("d_ff", c_int32),
                 ("n_shared", c_int32), ("d_ff_shared", c_int32), ("max_tokens", c_int32),
-                ("max_k", c_int32), ("gate", c_int32), ("flags", c_uint32)]
+                ("max_k", c_int32), ("gate", c_int32), ("flags", c_uint32),
+                ("route_nodes", c_int32), ("route_max_nodes", c_int32)]
 
 
 class moe_router(ctypes.Structure):
@@ -205,10 +206,12 @@ class MoELayer:
     """
 
     def __init__(self, *, d_model, n_routed, d_ff, n_shared, d_ff_shared, max_tokens, max_k,
-                 gate="softmax", flags=0, device=0):
+                 gate="softmax", flags=0, device=0, node_limit=None):
+        nodes, max_nodes = node_limit if node_limit is not None else (0, 0)
         self.cfg = moe_config(d_model, n_routed, d_ff, n_shared, d_ff_shared if n_shared else 0,
                               max_tokens, max_k,
-                              MOE_GATE_SIGMOID_BIASED if gate == "sigmoid" else MOE_GATE_SOFTMAX, flags)
+                              MOE_GATE_SIGMOID_BIASED if gate == "sigmoid" else MOE_GATE_SOFTMAX, flags,
+                              nodes, max_nodes)
         st, self.h = moe_create(self.cfg, device)
         if st != MOE_OK:
             raise MoEError(st, "moe_create")

@@ -85,6 +85,19 @@ typedef struct moe_config {
   int32_t max_k;       /* largest mK passed to moe_forward */
   int32_t gate;        /* moe_gate_kind */
   uint32_t flags;      /* MOE_FLAG_* */
+  /* Node-limited routing (DeepSeek-V3 technical report summary, section 2:
+   * each token is sent to at most M nodes, chosen among those holding its
+   * highest-affinity experts).  route_nodes = the number of nodes the mN
+   * experts sit on, in equal contiguous ranges (expert i on node
+   * i / (mN / route_nodes)); route_max_nodes = M.  A node ranks by the largest
+   * selection key among its experts (ties to the lower node); the token's K
+   * experts are the top K of the chosen nodes' experts.  Gates as without the
+   * limit (softmax over all mN experts, or the selected sigmoids renormalised).
+   * Both 0: no limit.  Otherwise 1 <= route_nodes <= 16 dividing mN,
+   * 1 <= route_max_nodes <= route_nodes, max_k <= route_max_nodes * mN /
+   * route_nodes (else MOE_ERR_INVALID_ARG). */
+  int32_t route_nodes;
+  int32_t route_max_nodes;
 } moe_config;
 
 /* Router.  weight: bf16 [mN, d], row i is e_i.

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_entry_point():
 
 def _cfg(**kw):
     base = dict(d_model=256, n_routed=16, d_ff=128, n_shared=1, d_ff_shared=128, max_tokens=512, max_k=4,
-                gate=B.MOE_GATE_SOFTMAX, flags=0)
+                gate=B.MOE_GATE_SOFTMAX, flags=0, route_nodes=0, route_max_nodes=0)
     base.update(kw)
     return B.moe_config(**base)
 
@@ -52,6 +52,14 @@ def _cfg(**kw):
     ({"gate": 7}, B.MOE_ERR_INVALID_ARG),
     ({"flags": 0x40}, B.MOE_ERR_INVALID_ARG),
     ({"n_shared": 0, "d_ff_shared": 0}, B.MOE_OK),
+    # node-limited routing: nodes divide mN, 1 <= M <= nodes <= 16, K fits in M nodes' experts
+    ({"route_nodes": 4, "route_max_nodes": 2}, B.MOE_OK),
+    ({"route_nodes": 3, "route_max_nodes": 2}, B.MOE_ERR_INVALID_ARG),
+    ({"route_nodes": 4, "route_max_nodes": 5}, B.MOE_ERR_INVALID_ARG),
+    ({"route_nodes": 4, "route_max_nodes": 0}, B.MOE_ERR_INVALID_ARG),
+    ({"route_nodes": 16, "route_max_nodes": 1, "max_k": 2}, B.MOE_ERR_INVALID_ARG),
+    ({"route_nodes": 32, "route_max_nodes": 1, "n_routed": 64}, B.MOE_ERR_INVALID_ARG),
+    ({"route_nodes": 0, "route_max_nodes": 2}, B.MOE_ERR_INVALID_ARG),
     # the FP8 workspace wants 128-column groups
     ({"flags": 0x8}, B.MOE_OK),
     ({"flags": 0x8, "d_ff": 208}, B.MOE_ERR_ALIGNMENT),

@@ -208,6 +208,63 @@ def test_non_finite_tokens_still_route_to_valid_experts(T):
     H.compare_output(_gpu_rows(out, ok), h, "finite tokens beside non-finite ones")
 
 
+def _node_limited_gaps(key, K, nodes, M):
+    """Per token: the gap between the M-th and (M+1)-th node scores (a node's largest key) and
+    between the K-th and (K+1)-th keys among the chosen nodes' experts (+inf where there is none);
+    a gap under the near-tie threshold may flip in float32."""
+    T, N = key.shape
+    per = N // nodes
+    ns = np.sort(key.reshape(T, nodes, per).max(axis=2), axis=1)[:, ::-1]
+    node_gap = ns[:, M - 1] - ns[:, M] if M < nodes else np.full(T, np.inf)
+    chosen = np.argsort(-key.reshape(T, nodes, per).max(axis=2), axis=1, kind="stable")[:, :M]
+    allowed = np.zeros((T, nodes), dtype=bool)
+    np.put_along_axis(allowed, chosen, True, axis=1)
+    masked = np.where(np.repeat(allowed, per, axis=1), key, -np.inf)
+    srt = -np.sort(-masked, axis=1)
+    k_gap = srt[:, K - 1] - srt[:, K] if K < M * per else np.full(T, np.inf)
+    return np.minimum(node_gap, k_gap)
+
+
+@pytest.mark.parametrize("case", ["tc_softmax", "small_sigmoid", "v3_like"])
+def test_node_limited_routing_matches_the_oracle(case):
+    """Node-limited routing (DeepSeek-V3 report summary, section 2): each token's K experts come
+    from at most M nodes, those holding its largest keys; bit-exact against the oracle's
+    select_top_k_node_limited except at near-ties, and the layer's output as the oracle's."""
+    spec = {"tc_softmax": (LS("nl_soft", T=300, d=256, N=64, I=64, K=6, Ks=1, Is=64, sigma=0.05, seed=71), 8, 3),
+            "small_sigmoid": (LS("nl_sig", T=100, d=256, N=64, I=64, K=6, Ks=1, Is=64, gate="sigmoid",
+                                 sigma=0.03, bias="uniform", seed=72), 4, 2),
+            "v3_like": (LS("nl_v3", T=1000, d=512, N=256, I=64, K=8, Ks=1, Is=64, gate="sigmoid", sigma=0.006,
+                           bias="uniform", seed=73), 8, 4)}[case]
+    shape, nodes, M = spec
+    host, dev = H.device_inputs(shape)
+    layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks, d_ff_shared=shape.Is,
+                       max_tokens=shape.T, max_k=shape.K, gate=shape.gate, node_limit=(nodes, M))
+    layer.set_weights(dev["router"], (dev["w_gate"], dev["w_up"], dev["w_down"]),
+                      (dev["ws_gate"], dev["ws_up"], dev["ws_down"]), logit_bias=dev["logit_bias"],
+                      select_bias=dev["select_bias"])
+    out = H.run(layer, dev["x"], shape.K)
+    idx, gate, counts, offsets, src = (t.cpu().numpy() for t in layer.routing(shape.T, shape.K))
+    ref = O.route(host["x"], host["router"], shape.K, shape.gate, host["logit_bias"], host["select_bias"],
+                  node_limit=(nodes, M))
+    ok = _node_limited_gaps(ref.key, shape.K, nodes, M) >= H.GAP_EXEMPT
+    assert ok.sum() > 0.9 * shape.T
+    np.testing.assert_array_equal(idx[ok], ref.idx[ok])
+    np.testing.assert_allclose(gate[ok], ref.gate[ok], rtol=0, atol=H.GATE_TOL)
+    per = shape.N // nodes
+    assert all(len(set(r)) == shape.K and len({e // per for e in r}) <= M for r in idx.tolist())
+    perm = O.expert_permutation(idx.astype(np.int64), shape.N)
+    np.testing.assert_array_equal(counts, perm.counts)
+    np.testing.assert_array_equal(src, perm.src)
+    rows = np.nonzero(ok)[0]
+    h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
+                         H.oracle_shared(shape, host), gate_kind=shape.gate, logit_bias=host["logit_bias"],
+                         select_bias=host["select_bias"], routing=ref, rows=rows)
+    H.compare_output(_gpu_rows(out, rows), h, f"{case} output")
+    # without the limit the same inputs route differently on some tokens (the limit is live)
+    free = O.route(host["x"], host["router"], shape.K, shape.gate, host["logit_bias"], host["select_bias"])
+    assert (free.idx != ref.idx).any()
+
+
 def test_zero_router_sends_every_token_to_the_first_experts():
     shape = LS("zero_router", T=700, d=128, N=16, I=64, K=4, Ks=1, Is=64, sigma=0.05, seed=22)
     host, dev = _custom_layer(shape, router=torch.zeros((16, 128), dtype=torch.bfloat16))
