@@ -41,10 +41,18 @@ UNIT = "tokens/s"
 L2_BYTES = 126 * 2**20
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT = "gate_up"
-# committed ncu summaries of the dominant kernel, per workload: DRAM bytes per token (prefill) or per launch
-PROFILE_SUMMARIES = {"16b_prefill": os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt"),
-                     "16b_decode": os.path.join(ROOT, "profiles", "gemms_16b_decode.txt")}
-KERNEL_SOURCES = ["fine_grained_shared_b200/csrc/gateup_gemm.cuh", "fine_grained_shared_b200/csrc/sm100.cuh"]
+# committed ncu summaries of the dominant kernel (the gate/up GEMM of the path the workload runs), per
+# (workload, fp8): the summary file and the sources whose hash it records; DRAM bytes per token
+# (prefill) or per launch
+_CSRC = "fine_grained_shared_b200/csrc/"
+KERNEL_SOURCES = [_CSRC + "gateup_gemm.cuh", _CSRC + "sm100.cuh"]
+PROFILE_SUMMARIES = {
+    ("16b_prefill", False): (os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt"), KERNEL_SOURCES),
+    ("16b_decode", False): (os.path.join(ROOT, "profiles", "decode_gemms_16b_decode.txt"),
+                            [_CSRC + "decode_gemm.cuh", _CSRC + "sm100.cuh"]),
+    ("16b_prefill", True): (os.path.join(ROOT, "profiles", "fp8_gemms_16b_prefill.txt"),
+                            [_CSRC + "fp8_gemm.cuh", _CSRC + "fp8_util.cuh", _CSRC + "sm100.cuh"]),
+}
 FP8_PROFILES = {"16b_prefill": os.path.join(ROOT, "profiles", "fp8_quant_rows_16b_prefill.txt")}
 FP8_SOURCES = ["fine_grained_shared_b200/csrc/fp8_quant.cu"]
 
@@ -107,10 +115,11 @@ def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(shape: W.LayerShape, path=None, sources=KERNEL_SOURCES):
+def profiled_traffic(shape: W.LayerShape, path=None, sources=KERNEL_SOURCES, fp8: bool = False):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary of this workload, if it was taken on the current kernel source; else None."""
-    path = path or PROFILE_SUMMARIES.get(shape.name)
+    if path is None:
+        path, sources = PROFILE_SUMMARIES.get((shape.name, fp8), (None, sources))
     if path is None or not os.path.exists(path):
         return None
     vals = {}
@@ -515,8 +524,8 @@ def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffi
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "peak_source": f"{peak_src} hbm_gbs"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof.update({"traffic": traffic, "kernel": "gateup_gemm_kernel (shared and routed experts: gate/up GEMM + "
-                                               "SwiGLU)",
+    kname = ("fp8_gemm_kernel<true>" if fp8 else "decode_gemm_kernel<true>" if shape.T <= 64 else "gateup_gemm_kernel")
+    roof.update({"traffic": traffic, "kernel": f"{kname} (shared and routed experts: gate/up GEMM + SwiGLU)",
                  "flop_per_launch": k_flop, "weight_bytes_per_launch": wb["gate_up"], "avg_launch_ms": k_avg_ms})
     return roof, peak_flops, peak_name
 
@@ -577,8 +586,7 @@ def run_ours(args):
     torch.cuda.empty_cache()
 
     peaks, peak_src = measured_peaks()
-    roofline, peak_flops, peak_name = roofline_of(shape, r, peaks, peak_src,
-                                                  None if fp8 else profiled_traffic(shape), fp8)
+    roofline, peak_flops, peak_name = roofline_of(shape, r, peaks, peak_src, profiled_traffic(shape, fp8=fp8), fp8)
     layer_tflops = world * layer_flop(shape) / (r["ms_step"] * 1e-3) / 1e12
     config = workload_config(shape, f"replicas{world}" if world > 1 else "single")
     if fp8:

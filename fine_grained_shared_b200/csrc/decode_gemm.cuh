@@ -194,31 +194,57 @@ __device__ __forceinline__ DecTile dec_shared_tile(long long t, int sh_rows) {
   return d;
 }
 
-// Walks one CTA's range of a space as segments (tile, k-blocks [k0, k1)).
+// Walks one CTA's range of a space as segments (tile, k-blocks [k0, k1)):
+// first the range's cut parts -- its head (the end of a tile an earlier CTA
+// began) and its tail (the start of a tile a later CTA finishes) -- then the
+// whole tiles between them.  Whichever CTA counts a cut tile's last part sums
+// the parts; doing the cut parts first makes that happen early, while the
+// whole tiles' MMAs still run, instead of at the end of the kernel.
 struct DecWalk {
-  long long x, end;
-  int kbt;
+  long long lo[3], hi[3], x;
+  int n, i, kbt;
   __device__ __forceinline__ bool next(long long& tile, int& k0, int& k1) {
-    if (x >= end) return false;
-    tile = x / kbt;
-    k0 = static_cast<int>(x - tile * kbt);
-    const long long rem = end - x;
-    k1 = static_cast<int>(k0 + rem < kbt ? k0 + rem : kbt);
-    x = tile * kbt + k1;
-    return true;
+    while (i < n) {
+      if (x < hi[i]) {
+        tile = x / kbt;
+        k0 = static_cast<int>(x - tile * kbt);
+        const long long rem = hi[i] - x;
+        k1 = static_cast<int>(k0 + rem < kbt ? k0 + rem : kbt);
+        x = tile * kbt + k1;
+        return true;
+      }
+      if (++i < n) x = lo[i];
+    }
+    return false;
   }
 };
 
-__device__ __forceinline__ DecWalk dec_walk(const DecSpace& s, int c) {
+// The walk of [x0, x1) in tiles of kbt k-blocks.
+__device__ __forceinline__ DecWalk dec_walk_range(long long x0, long long x1, int kbt) {
   DecWalk w;
-  w.kbt = s.kbt;
-  if (c >= s.workers || s.total == 0) {
-    w.x = w.end = 0;
-  } else {
-    w.x = s.bound(c);
-    w.end = s.bound(c + 1);
+  w.kbt = kbt;
+  w.n = 0;
+  w.i = 0;
+  if (x0 < x1) {
+    const long long b0 = (x0 + kbt - 1) / kbt * kbt;  // first tile boundary at or after x0
+    const long long b1 = x1 / kbt * kbt;              // last tile boundary at or before x1
+    if (b0 > b1) {  // inside one tile
+      w.lo[0] = x0;
+      w.hi[0] = x1;
+      w.n = 1;
+    } else {
+      if (x0 < b0) { w.lo[w.n] = x0; w.hi[w.n] = b0; ++w.n; }  // head
+      if (b1 < x1) { w.lo[w.n] = b1; w.hi[w.n] = x1; ++w.n; }  // tail
+      if (b0 < b1) { w.lo[w.n] = b0; w.hi[w.n] = b1; ++w.n; }  // whole tiles
+    }
   }
+  w.x = w.n ? w.lo[0] : 0;
   return w;
+}
+
+__device__ __forceinline__ DecWalk dec_walk(const DecSpace& s, int c) {
+  if (c >= s.workers || s.total == 0) return dec_walk_range(0, 0, s.kbt);
+  return dec_walk_range(s.bound(c), s.bound(c + 1), s.kbt);
 }
 
 __device__ __forceinline__ void dec_record_error(uint32_t* err, volatile int* abort, uint32_t site) {
@@ -324,13 +350,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   };
   // the shared segments of CTA c: one whole tile, or its cut range
   auto shared_walk = [&]() {
-    DecWalk w = dec_walk(sp0, c);
     if (sh_whole) {
-      w.kbt = sh_kbt;
-      w.x = c < sh_tiles ? static_cast<long long>(c) * sh_kbt : 0;
-      w.end = c < sh_tiles ? w.x + sh_kbt : 0;
+      const long long x0 = c < sh_tiles ? static_cast<long long>(c) * sh_kbt : 0;
+      return dec_walk_range(x0, c < sh_tiles ? x0 + sh_kbt : 0, sh_kbt);
     }
-    return w;
+    return dec_walk(sp0, c);
   };
   // a whole shared tile is never cut: the space's k-block count of a tile
   const DecSpace sp0w = [&]() {

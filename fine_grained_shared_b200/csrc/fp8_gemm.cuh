@@ -333,6 +333,35 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       const int kgs = c.shared ? a.sh_kg_per_j : a.num_kg;
       const int n0 = c.n_tile * (GU ? kF8BN / 2 : kF8BN);
       for (int j = 0; j < J && !stop; ++j) {
+        // the B rows' block scales of every K group of this tile (and shared expert j), loaded once:
+        // lane l holds groups l and l + 32 (at most 64 groups: d, I, I_s <= 8192); a stage takes
+        // its byte by a shuffle instead of a global load on the producer's critical path
+        uint32_t sc0[2] = {127u, 127u}, sc1[2] = {127u, 127u};
+        {
+          const uint8_t* s0 = c.shared ? a.sh_w_scale0 : a.w_scale0;
+          const int rows128 = c.shared ? a.sh_w_rows128 : a.w_rows128;
+          const int groups = c.shared ? a.sh_kg_per_j : a.num_kg;
+          size_t base0, base1;
+          if (GU) {
+            // the shared experts' rows are K_s blocks of I_s side by side: block n0 / 128 of the whole
+            const size_t blk = c.shared ? static_cast<size_t>(n0 >> 7) : static_cast<size_t>(c.g) * rows128 + (n0 >> 7);
+            base0 = base1 = blk * groups;
+          } else {
+            const size_t mat = static_cast<size_t>(c.shared ? j : c.g) * rows128;
+            const int r0 = n0 >> 7;
+            base0 = (mat + r0) * groups;
+            base1 = r0 + 1 < rows128 ? (mat + r0 + 1) * groups : base0;  // rows past d are zero: any scale
+          }
+          const uint8_t* s1 = GU ? (c.shared ? a.sh_w_scale1 : a.w_scale1) : s0;
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int kgl = lane + 32 * h2;
+            if (kgl < kgs) {
+              sc0[h2] = __ldg(s0 + base0 + kgl);
+              sc1[h2] = __ldg(s1 + base1 + kgl);
+            }
+          }
+        }
         for (int kg = 0; kg < kgs; ++kg) {
           bool ok = true;
           if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag);
@@ -363,31 +392,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
                           &full[s]);
           }
           // the B rows' scales: one byte per 128 x 128 weight block, spread over its atom
-          uint32_t b0, b1;
-          {
-            const int kgw = kg;  // the weight's K group
-            if (GU) {
-              const uint8_t* s0 = c.shared ? a.sh_w_scale0 : a.w_scale0;
-              const uint8_t* s1 = c.shared ? a.sh_w_scale1 : a.w_scale1;
-              const int rows128 = c.shared ? a.sh_w_rows128 : a.w_rows128;
-              const int groups = c.shared ? a.sh_kg_per_j : a.num_kg;
-              // the shared experts' rows are K_s blocks of I_s side by side: block n0 / 128 of the whole
-              const size_t blk = c.shared ? static_cast<size_t>(n0 >> 7)
-                                          : static_cast<size_t>(c.g) * rows128 + (n0 >> 7);
-              b0 = __ldg(s0 + blk * groups + kgw);
-              b1 = __ldg(s1 + blk * groups + kgw);
-            } else {
-              const uint8_t* s0 = c.shared ? a.sh_w_scale0 : a.w_scale0;
-              const int rows128 = c.shared ? a.sh_w_rows128 : a.w_rows128;
-              const int groups = c.shared ? a.sh_kg_per_j : a.num_kg;
-              const int mat = c.shared ? j : c.g;
-              const int r0 = n0 >> 7;
-              const size_t base = static_cast<size_t>(mat) * rows128;
-              b0 = __ldg(s0 + (base + r0) * groups + kgw);
-              // rows past d (a ragged last tile) are zero in the weights: any scale does
-              b1 = r0 + 1 < rows128 ? __ldg(s0 + (base + r0 + 1) * groups + kgw) : 127u;
-            }
-          }
+          const uint32_t b0 = __shfl_sync(0xffffffffu, kg < 32 ? sc0[0] : sc0[1], kg & 31);
+          const uint32_t b1 = __shfl_sync(0xffffffffu, kg < 32 ? sc1[0] : sc1[1], kg & 31);
           const uint32_t w0 = 0x01010101u * b0, w1 = 0x01010101u * b1;
           reinterpret_cast<uint4*>(sfb)[lane] = make_uint4(w0, w0, w0, w0);
           reinterpret_cast<uint4*>(sfb + kSfAtomBytes)[lane] = make_uint4(w1, w1, w1, w1);
@@ -479,24 +485,24 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       const size_t row = static_cast<size_t>(c.row0) + r;
       if (GU) {
         // gate columns [64 h, 64 h + 64), up columns [128 + 64 h, ...): H columns n0 + 64 h ..
-        float hv[64];
-        {
-          uint32_t gr[16], ur[16];
+        // the raw accumulator into registers first and the accumulator freed, so that the next
+        // tile's MMAs run while this tile's SwiGLU and quantization are computed
+        uint32_t gr[64], ur[64];
 #pragma unroll
-          for (int cc = 0; cc < 64; cc += 16) {
-            tmem_ld16(tb + 64 * h + cc, gr);
-            tmem_ld16(tb + 128 + 64 * h + cc, ur);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float g = __uint_as_float(gr[j]), u = __uint_as_float(ur[j]);
-              hv[cc + j] = g / (1.f + __expf(-g)) * u;
-            }
-          }
+        for (int cc = 0; cc < 64; cc += 16) {
+          tmem_ld16(tb + 64 * h + cc, *reinterpret_cast<uint32_t(*)[16]>(gr + cc));
+          tmem_ld16(tb + 128 + 64 * h + cc, *reinterpret_cast<uint32_t(*)[16]>(ur + cc));
         }
+        tmem_ld_wait();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);  // the accumulator is in registers
+        float hv[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          const float g = __uint_as_float(gr[j]), u = __uint_as_float(ur[j]);
+          hv[j] = g / (1.f + __expf(-g)) * u;
+        }
         // the row's 1 x 128 group is this tile's 128 H columns: the two halves' maxima
         float m = 0.f;
 #pragma unroll
@@ -534,24 +540,22 @@ __global__ void __launch_bounds__(kF8Threads, 1)
       } else {
         // columns [128 h, 128 h + 128) of the tile: output columns n0 + 128 h ..
         const int n0 = c.n_tile * kF8BN + 128 * h;
-        const float sc = c.shared ? 1.f : a.row_scale[row];
         const int n_limit = c.shared ? a.sh_n_limit : a.n_limit;
         const int ld = c.shared ? a.sh_ld_out : a.ld_out;
-        uint32_t pk[64];
-        {
-          uint32_t v[16];
+        // the raw accumulator into registers and the accumulator freed before the gate's load
+        uint32_t v[128];
 #pragma unroll
-          for (int cc = 0; cc < 128; cc += 16) {
-            tmem_ld16(tb + 128 * h + cc, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              pk[cc / 2 + j] = pack_bf16x2(sc * __uint_as_float(v[2 * j]), sc * __uint_as_float(v[2 * j + 1]));
-          }
-        }
+        for (int cc = 0; cc < 128; cc += 16)
+          tmem_ld16(tb + 128 * h + cc, *reinterpret_cast<uint32_t(*)[16]>(v + cc));
+        tmem_ld_wait();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(acc_empty);
+        const float sc = c.shared ? 1.f : a.row_scale[row];
+        uint32_t pk[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          pk[j] = pack_bf16x2(sc * __uint_as_float(v[2 * j]), sc * __uint_as_float(v[2 * j + 1]));
         if (n0 < n_limit) {
           __nv_bfloat16* orow = (c.shared ? a.sh_y : a.y) + row * ld + n0;
 #pragma unroll

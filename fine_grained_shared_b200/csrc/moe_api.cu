@@ -208,6 +208,8 @@ moe_status check_config(const moe_config* c) {
   if (c->flags & ~known) return MOE_ERR_INVALID_ARG;
   if ((c->flags & MOE_FLAG_FP8) && (c->d_model % 128 || c->d_ff % 128 || (c->n_shared > 0 && c->d_ff_shared % 128)))
     return MOE_ERR_ALIGNMENT;
+  if ((c->flags & MOE_FLAG_FP8) && (c->d_model > 8192 || c->d_ff > 8192 || c->d_ff_shared > 8192))
+    return MOE_ERR_SHAPE;  // at most 64 scale groups along a GEMM's K
   if (c->route_nodes != 0 || c->route_max_nodes != 0) {
     if (c->route_nodes < 1 || c->route_nodes > kMaxRouteNodes || c->n_routed % c->route_nodes ||
         c->route_max_nodes < 1 || c->route_max_nodes > c->route_nodes ||

@@ -66,7 +66,8 @@ typedef enum moe_gate_kind {
 #define MOE_FLAG_NO_ROUTED 0x4u   /* drop the routed experts (routing still runs) */
 /* The handle also holds the workspace of moe_forward_fp8 (FP8 copies of the
  * permuted activations and of H, with their scales).  Requires d_model, d_ff
- * and d_ff_shared to be multiples of 128 (else MOE_ERR_ALIGNMENT). */
+ * and d_ff_shared to be multiples of 128 (else MOE_ERR_ALIGNMENT) and at most
+ * 8192 (else MOE_ERR_SHAPE). */
 #define MOE_FLAG_FP8 0x8u
 /* Test only: the first grouped-GEMM CTA waits on a barrier that nothing
  * arrives on, with a 20 ms limit; the call then reports MOE_ERR_TIMEOUT. */

@@ -65,6 +65,7 @@ def _cfg(**kw):
     ({"flags": 0x8, "d_ff": 208}, B.MOE_ERR_ALIGNMENT),
     ({"flags": 0x8, "d_ff_shared": 144}, B.MOE_ERR_ALIGNMENT),
     ({"flags": 0x8, "d_model": 272}, B.MOE_ERR_ALIGNMENT),
+    ({"flags": 0x8, "d_model": 8320}, B.MOE_ERR_SHAPE),
 ])
 def test_config_validation(kw, status):
     st, nbytes = B.moe_workspace_bytes(_cfg(**kw))
