@@ -33,8 +33,10 @@
 //   warp 0      TMA producer: per 64-column k-block the weight boxes
 //               [128 rows, 64] and the token box [32 rows, 64] (128-byte
 //               swizzle) into a ring of kStages stages
-//   warp 1      allocates 128 TMEM columns (two accumulator buffers of 64
-//               columns); one lane issues the MMAs
+//   warp 1      allocates all 512 TMEM columns: eight accumulator buffers
+//               of 64 columns, so that the MMAs run up to seven segments
+//               ahead of an epilogue that is summing a split tile; one lane
+//               issues the MMAs
 //   warps 2-5   epilogue: thread r holds weight row r of the accumulator,
 //               i.e. one output column for the tile's (up to) 32 tokens
 // The gate/up kernel runs the shared experts' space before waiting on the
@@ -51,7 +53,8 @@ constexpr int kDecWB = 128;   // weight rows per tile (MMA M)
 constexpr int kDecBK = 64;    // k-block: one 128-byte swizzle row of bf16
 constexpr uint32_t kDecBoxW = kDecWB * kDecBK * 2;  // 16 KB
 constexpr uint32_t kDecBoxX = kDecTB * kDecBK * 2;  // 4 KB
-constexpr uint32_t kDecTmemCols = 128;              // 2 buffers x 64 columns
+constexpr int kDecAccBufs = 8;                      // accumulator buffers of 64 columns
+constexpr uint32_t kDecTmemCols = 64 * kDecAccBufs;  // all 512 columns: one CTA per SM
 constexpr int kDecMinIters = 4;                     // fewest k-blocks in a CTA's range
 // TMA box heights the host must encode
 constexpr uint32_t kDecBoxRowsW = kDecWB;
@@ -87,7 +90,7 @@ __host__ __device__ constexpr size_t dec_partials_bytes(int ctas) {
 template <bool GU>
 __host__ __device__ constexpr size_t dec_smem_bytes() {
   return 1024 + static_cast<size_t>(DecCfg<GU>::kStages) * dec_stage_bytes<GU>() +
-         8 * (2 * DecCfg<GU>::kStages + 4 + 2) + 16 + 4 * (3 * 264 + 4);
+         8 * (2 * DecCfg<GU>::kStages + 2 * kDecAccBufs + 2) + 16 + 4 * (3 * 264 + 4);
 }
 static_assert(dec_smem_bytes<true>() <= 232448 && dec_smem_bytes<false>() <= 232448, "shared memory");
 
@@ -281,9 +284,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kStage);
   uint64_t* empty = full + S;
-  uint64_t* acc_full = empty + S;      // [2]
-  uint64_t* acc_empty = acc_full + 2;  // [2]
-  uint64_t* tables = acc_empty + 2;    // the routed tables are in shared memory
+  uint64_t* acc_full = empty + S;                // [kDecAccBufs]
+  uint64_t* acc_empty = acc_full + kDecAccBufs;  // [kDecAccBufs]
+  uint64_t* tables = acc_empty + kDecAccBufs;    // the routed tables are in shared memory
   uint64_t* teardown = tables + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -312,7 +315,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kDecAccBufs; ++i) {
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_empty[i], 4);  // one arrive per epilogue warp
     }
@@ -497,7 +500,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         }
       }
       umma_commit(&acc_full[buf]);
-      if (++buf == 2) {
+      if (++buf == kDecAccBufs) {
         buf = 0;
         buf_ph ^= 1u;
       }
@@ -546,7 +549,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the accumulator is in registers: free it
-      if (++buf == 2) {
+      if (++buf == kDecAccBufs) {
         buf = 0;
         buf_ph ^= 1u;
       }
