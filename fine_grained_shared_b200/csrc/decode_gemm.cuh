@@ -32,7 +32,10 @@
 // One persistent CTA per SM, 192 threads:
 //   warp 0      TMA producer: per 64-column k-block the weight boxes
 //               [128 rows, 64] and the token box [32 rows, 64] (128-byte
-//               swizzle) into a ring of kStages stages
+//               swizzle) into a ring of kStages stages.  Weights are read
+//               once, so their loads carry an L2 evict-first policy: the
+//               weight stream then does not push the tokens, the partial
+//               sums and the kernel's own code out of L2.
 //   warp 1      allocates all 512 TMEM columns: eight accumulator buffers
 //               of 64 columns, so that the MMAs run up to seven segments
 //               ahead of an epilogue that is summing a split tile; one lane
@@ -62,15 +65,20 @@ constexpr uint32_t kDecBoxRowsX = kDecTB;
 
 template <bool GU>
 struct DecCfg;
+// Ring depth: about 145 KB per SM in flight covers an SM's share of HBM
+// bandwidth (1/148 of it) over the loaded latency.  Deeper rings bring no more
+// bandwidth but lengthen the queue every other access of the SM waits in:
+// with 216 KB (6 gate/up stages) a cold instruction fetch or a store from the
+// epilogue took several microseconds, and both kernels ran 4% slower.
 template <>
 struct DecCfg<true> {  // gate/up: W_gate + W_up + tokens per stage
   static constexpr int kAcc = 2;
-  static constexpr int kStages = 6;
+  static constexpr int kStages = 4;
 };
 template <>
 struct DecCfg<false> {  // down: W_down + rows of H per stage
   static constexpr int kAcc = 1;
-  static constexpr int kStages = 10;
+  static constexpr int kStages = 7;
 };
 template <bool GU>
 __host__ __device__ constexpr uint32_t dec_stage_bytes() {
@@ -93,6 +101,13 @@ __host__ __device__ constexpr size_t dec_smem_bytes() {
          8 * (2 * DecCfg<GU>::kStages + 2 * kDecAccBufs + 2) + 16 + 4 * (3 * 264 + 4);
 }
 static_assert(dec_smem_bytes<true>() <= 232448 && dec_smem_bytes<false>() <= 232448, "shared memory");
+// Each CTA takes all 512 TMEM columns, so no two decode CTAs (a gate/up CTA
+// and a down CTA launched early behind it included) may share an SM: one
+// would wait in tcgen05.alloc until the other ends.  Shared memory keeps
+// them apart (233472 bytes per SM).
+static_assert(dec_smem_bytes<true>() + dec_smem_bytes<false>() > 233472 &&
+                  2 * dec_smem_bytes<true>() > 233472 && 2 * dec_smem_bytes<false>() > 233472,
+              "two decode CTAs would fit on one SM");
 
 struct DecodeArgs {
   // routed experts: the expert-ordered rows of X_perm (gate/up) or H (down)
@@ -197,12 +212,12 @@ __device__ __forceinline__ DecTile dec_shared_tile(long long t, int sh_rows) {
   return d;
 }
 
-// Walks one CTA's range of a space as segments (tile, k-blocks [k0, k1)):
-// first the range's cut parts -- its head (the end of a tile an earlier CTA
-// began) and its tail (the start of a tile a later CTA finishes) -- then the
-// whole tiles between them.  Whichever CTA counts a cut tile's last part sums
-// the parts; doing the cut parts first makes that happen early, while the
-// whole tiles' MMAs still run, instead of at the end of the kernel.
+// Walks one CTA's range of a space as segments (tile, k-blocks [k0, k1)) in
+// k order: its head (the end of a tile an earlier CTA began), the whole tiles,
+// then its tail (the start of a tile a later CTA finishes).  Whichever CTA
+// counts a cut tile's last part sums the parts.  (Taking the tail before the
+// whole tiles, so that its sum happens earlier, measured 3-5% slower on the
+// gate/up GEMM of the 16B decode layer.)
 struct DecWalk {
   long long lo[3], hi[3], x;
   int n, i, kbt;
@@ -237,8 +252,8 @@ __device__ __forceinline__ DecWalk dec_walk_range(long long x0, long long x1, in
       w.n = 1;
     } else {
       if (x0 < b0) { w.lo[w.n] = x0; w.hi[w.n] = b0; ++w.n; }  // head
-      if (b1 < x1) { w.lo[w.n] = b1; w.hi[w.n] = x1; ++w.n; }  // tail
       if (b0 < b1) { w.lo[w.n] = b0; w.hi[w.n] = b1; ++w.n; }  // whole tiles
+      if (b1 < x1) { w.lo[w.n] = b1; w.hi[w.n] = x1; ++w.n; }  // tail
     }
   }
   w.x = w.n ? w.lo[0] : 0;
@@ -369,6 +384,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
     int s = 0, issued = 0;
+    const uint64_t pol_w = l2_policy_evict_first();
     uint32_t ph = 0;
     bool stop = false;
     auto load_segment = [&](bool shared, const DecTile& t, int k0, int k1) {
@@ -383,16 +399,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int wrow = t.wb * kDecWB;
         if (GU) {
           const int kc = kb * kDecBK;
-          tma_load_3d(st, shared ? &tmWs0 : &tmW0, &full[s], kc, wrow, t.g);
-          tma_load_3d(st + kDecBoxW, shared ? &tmWs1 : &tmW1, &full[s], kc, wrow, t.g);
+          tma_load_3d_hint(st, shared ? &tmWs0 : &tmW0, &full[s], kc, wrow, t.g, pol_w);
+          tma_load_3d_hint(st + kDecBoxW, shared ? &tmWs1 : &tmW1, &full[s], kc, wrow, t.g, pol_w);
           tma_load_2d(st + 2 * kDecBoxW, shared ? &tmXs : &tmX, &full[s], kc, t.row0);
         } else if (shared) {
           const int j = kb / a.sh_kb_per_j, kc = (kb - j * a.sh_kb_per_j) * kDecBK;
-          tma_load_3d(st, &tmWs0, &full[s], kc, wrow, j);
+          tma_load_3d_hint(st, &tmWs0, &full[s], kc, wrow, j, pol_w);
           tma_load_2d(st + kDecBoxW, &tmXs, &full[s], j * a.sh_k_per_j + kc, t.row0);
         } else {
           const int kc = kb * kDecBK;
-          tma_load_3d(st, &tmW0, &full[s], kc, wrow, t.g);
+          tma_load_3d_hint(st, &tmW0, &full[s], kc, wrow, t.g, pol_w);
           tma_load_2d(st + kDecBoxW, &tmX, &full[s], kc, t.row0);
         }
         ++issued;
@@ -612,19 +628,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (col >= n_limit) return;
       __nv_bfloat16* obase = shared ? a.sh_out : a.out;
       const int ld = shared ? a.sh_ld_out : a.ld_out;
+      // kept short: this code first runs while the weight stream fills the
+      // memory system, and every instruction line it misses waits in that queue
+      __nv_bfloat16* op = obase + static_cast<size_t>(t.row0) * ld + col;
+      const float* rs = shared ? nullptr : a.row_scale + t.row0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         if (j < t.nvalid) {
-          const size_t row = static_cast<size_t>(t.row0) + j;
           float o;
           if (GU) {
             const float g = v[0][j], u = v[1][j];
-            o = g / (1.f + __expf(-g)) * u;
+            o = __fdividef(g, 1.f + __expf(-g)) * u;  // SiLU(g) u
           } else {
-            o = shared ? v[0][j] : a.row_scale[row] * v[0][j];
+            o = shared ? v[0][j] : rs[j] * v[0][j];
           }
-          obase[row * ld + col] = __float2bfloat16_rn(o);
+          *op = __float2bfloat16_rn(o);
         }
+        op += ld;
       }
     };
     {
