@@ -41,6 +41,8 @@ UNIT = "tokens/s"
 L2_BYTES = 126 * 2**20
 PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT = "gate_up"
+# batches of at most this many tokens run both expert GEMMs in one launch (the decode FFN), timed as gate_up
+DECODE_MAX_T = 64
 # committed ncu summaries of the dominant kernel (the gate/up GEMM of the path the workload runs), per
 # (workload, fp8): the summary file and the sources whose hash it records; DRAM bytes per token
 # (prefill) or per launch
@@ -48,8 +50,8 @@ _CSRC = "fine_grained_shared_b200/csrc/"
 KERNEL_SOURCES = [_CSRC + "gateup_gemm.cuh", _CSRC + "sm100.cuh"]
 PROFILE_SUMMARIES = {
     ("16b_prefill", False): (os.path.join(ROOT, "profiles", "gate_up_16b_prefill.txt"), KERNEL_SOURCES),
-    ("16b_decode", False): (os.path.join(ROOT, "profiles", "decode_gemms_16b_decode.txt"),
-                            [_CSRC + "decode_gemm.cuh", _CSRC + "sm100.cuh"]),
+    ("16b_decode", False): (os.path.join(ROOT, "profiles", "decode_ffn_16b_decode.txt"),
+                            [_CSRC + "decode_ffn.cuh", _CSRC + "sm100.cuh"]),
     ("16b_prefill", True): (os.path.join(ROOT, "profiles", "fp8_gemms_16b_prefill.txt"),
                             [_CSRC + "fp8_gemm.cuh", _CSRC + "fp8_util.cuh", _CSRC + "sm100.cuh"]),
 }
@@ -499,20 +501,28 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
     return r
 
 
+def fused_decode(shape: W.LayerShape, fp8: bool = False) -> bool:
+    """Whether the bf16 layer runs both expert GEMMs in one launch (the decode FFN)."""
+    return not fp8 and shape.T <= DECODE_MAX_T
+
+
 def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffic=None, fp8: bool = False):
-    """Roofline of the dominant kernel (the shared + routed gate/up GEMM with SwiGLU): tensor-bound
-    when the routed experts' FLOPs per weight byte exceed the ridge (sustained bf16 FLOP/s over copy
-    bandwidth), else HBM-bound over the weights of the touched experts (the weight-streaming regime).
-    fp8: the FP8 layer, against twice the measured bf16 peak (the nominal FP8 / bf16 ratio of the
-    tensor cores) and over 1-byte weights (plus one scale byte per 128 x 128 block)."""
+    """Roofline of the dominant kernel (the shared + routed gate/up GEMM with SwiGLU; for a decode
+    batch the one launch of both expert GEMMs): tensor-bound when the routed experts' FLOPs per
+    weight byte exceed the ridge (sustained bf16 FLOP/s over copy bandwidth), else HBM-bound over the
+    weights of the touched experts (the weight-streaming regime).  fp8: the FP8 layer, against twice
+    the measured bf16 peak (the nominal FP8 / bf16 ratio of the tensor cores) and over 1-byte weights
+    (plus one scale byte per 128 x 128 block)."""
     peak_flops, peak_name = choose_peak(peaks, r["ms_total"] * 1e-3, r["clocks"])
     if fp8:
         peak_flops, peak_name = 2.0 * peak_flops, f"2 x {peak_name} (fp8 = 2 x bf16, nominal ratio)"
-    k_flop = 4.0 * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is)
+    fused = fused_decode(shape, fp8)
+    k_flop = (6.0 if fused else 4.0) * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is)
     wb = touched_weight_bytes(shape, r["counts"], fp8)
+    k_bytes = wb["layer"] if fused else wb["gate_up"]
     k_avg_ms = r["dominant_ms"]
     hbm = float(peaks["hbm_gbs"])
-    if k_flop / wb["gate_up"] > float(peaks["bf16_tflops_sustained"]) * 1e12 / (hbm * 1e9):
+    if k_flop / k_bytes > float(peaks["bf16_tflops_sustained"]) * 1e12 / (hbm * 1e9):
         achieved = k_flop / (k_avg_ms * 1e-3) / 1e12
         mult = 2.0 if fp8 else 1.0
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak_flops, "unit": "TFLOP/s",
@@ -520,13 +530,18 @@ def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffi
                 "frac_of_burst": achieved / (mult * float(peaks["bf16_tflops"])),
                 "frac_of_sustained": achieved / (mult * float(peaks["bf16_tflops_sustained"]))}
     else:
-        achieved = wb["gate_up"] / (k_avg_ms * 1e-3) / 1e9
+        achieved = k_bytes / (k_avg_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "peak_source": f"{peak_src} hbm_gbs"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    kname = ("fp8_gemm_kernel<true>" if fp8 else "decode_gemm_kernel<true>" if shape.T <= 64 else "gateup_gemm_kernel")
-    roof.update({"traffic": traffic, "kernel": f"{kname} (shared and routed experts: gate/up GEMM + SwiGLU)",
-                 "flop_per_launch": k_flop, "weight_bytes_per_launch": wb["gate_up"], "avg_launch_ms": k_avg_ms})
+    if fused:
+        kname = ("decode_ffn_kernel (shared and routed experts: gate/up GEMM + SwiGLU and down GEMM + gate "
+                 "scale, one launch)")
+    else:
+        kname = ("fp8_gemm_kernel<true>" if fp8 else "gateup_gemm_kernel") + \
+            " (shared and routed experts: gate/up GEMM + SwiGLU)"
+    roof.update({"traffic": traffic, "kernel": kname, "flop_per_launch": k_flop, "weight_bytes_per_launch": k_bytes,
+                 "avg_launch_ms": k_avg_ms})
     return roof, peak_flops, peak_name
 
 
@@ -536,10 +551,15 @@ def hbm_fractions(shape: W.LayerShape, r: dict, peaks: dict, fp8: bool = False) 
     wb = touched_weight_bytes(shape, r["counts"], fp8)
     hbm = float(peaks["hbm_gbs"])
     out = {"touched_experts": wb["touched_experts"], "weight_bytes": wb["layer"]}
-    for k in ("gate_up", "down"):
-        ms = r["kernel_ms"].get(k, 0.0)
-        out[f"{k}_gbs"] = wb[k] / (ms * 1e-3) / 1e9 if ms > 0 else None
-        out[f"{k}_frac"] = out[f"{k}_gbs"] / hbm if ms > 0 else None
+    if fused_decode(shape, fp8):
+        ms = r["kernel_ms"].get("gate_up", 0.0)  # both GEMMs in one launch
+        out["ffn_gbs"] = wb["layer"] / (ms * 1e-3) / 1e9 if ms > 0 else None
+        out["ffn_frac"] = out["ffn_gbs"] / hbm if ms > 0 else None
+    else:
+        for k in ("gate_up", "down"):
+            ms = r["kernel_ms"].get(k, 0.0)
+            out[f"{k}_gbs"] = wb[k] / (ms * 1e-3) / 1e9 if ms > 0 else None
+            out[f"{k}_frac"] = out[f"{k}_gbs"] / hbm if ms > 0 else None
     out["layer_gbs"] = wb["layer"] / (r["ms_step"] * 1e-3) / 1e9
     out["layer_frac"] = out["layer_gbs"] / hbm
     return out

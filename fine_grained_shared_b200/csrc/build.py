@@ -14,7 +14,7 @@ PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libfgs_moe.so")
 SOURCES = ["moe_api.cu", "route_noalloc.cu", "fp8_quant.cu"]
-HEADERS = ["sm100.cuh", "router_topk.cuh", "permute.cuh", "gateup_gemm.cuh", "down_gemm.cuh", "decode_gemm.cuh",
+HEADERS = ["sm100.cuh", "router_topk.cuh", "permute.cuh", "gateup_gemm.cuh", "down_gemm.cuh", "decode_ffn.cuh",
            "fp8_util.cuh", "fp8_gemm.cuh"]
 
 

@@ -27,7 +27,7 @@
 #include <vector>
 
 #include "../../include/fgs_moe.h"
-#include "decode_gemm.cuh"
+#include "decode_ffn.cuh"
 #include "down_gemm.cuh"
 #include "fp8_gemm.cuh"
 #include "gateup_gemm.cuh"
@@ -37,11 +37,11 @@
 using namespace fgs;
 
 static_assert(kGemmBM == kExpertRowAlign, "GEMM pair tiles must not straddle two experts");
-static_assert(kDecBoxRowsW == kGuBoxRowsB && kDecBoxRowsW == kBoxRowsB,
-              "the decode GEMMs share the weight maps of the prefill GEMMs");
+static_assert(kFfnBoxRowsW == kGuBoxRowsB && kFfnBoxRowsW == kBoxRowsB,
+              "the decode FFN shares the weight maps of the prefill GEMMs");
 
 // Batches of at most this many tokens run the expert FFNs on the
-// weight-streaming decode GEMMs (decode_gemm.cuh); larger ones on the
+// weight-streaming decode kernel (decode_ffn.cuh); larger ones on the
 // 128-row-tile GEMMs.
 #ifndef FGS_DECODE_MAX_T
 #define FGS_DECODE_MAX_T 64
@@ -55,7 +55,6 @@ constexpr int kMaxK = 8;
 constexpr int64_t kMaxTokens = int64_t(1) << 20;
 constexpr uint64_t kTimeoutNs = 2000ull * 1000 * 1000;  // 2 s: no legitimate wait comes close
 constexpr int64_t kDecodeMaxT = FGS_DECODE_MAX_T;
-constexpr int kDecMaxCtas = 148;  // the decode GEMMs' grid: one CTA per SM, at most this many
 // the host-buffer forward pipelines batches of at least 2 x kHostChunkRows tokens in up to kHostChunks chunks
 constexpr int kHostChunks = 5;
 constexpr int64_t kHostChunkRows = 2048;
@@ -113,18 +112,17 @@ inline int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) 
 struct Layout {
   // byte offsets into the workspace
   size_t err, done, tile_ctr, tok_done, small_logits, idx, gate, slot, src, bc, counts, offsets, row_start, mtile,
-      mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, dec_part_gu, dec_part_dn, dec_ctr_gu, dec_ctr_dn,
-      dec_ctr_bytes, xq_perm, xs_perm, xq, xs, hq, hs_perm, hsq, hss, total;
+      mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, ffn_ctr, xq_perm, xs_perm, xq, xs, hq, hs_perm, hsq,
+      hss, total;
   int64_t P, Pa, Tpad, nblk;
 };
 
-// Tiles a decode GEMM launch can have: 32-token blocks of the shared experts'
-// rows, and of each routed expert's rows (at most one partial block per
-// expert that received a token), times the weight blocks.
-int64_t decode_max_tiles(int64_t T, int64_t K, int64_t N, int64_t routed_wb, int64_t shared_wb) {
-  const int64_t tb = (T + kDecTB - 1) / kDecTB;
-  const int64_t routed_tb = std::min<int64_t>(N, T * K) + (T * K + kDecTB - 1) / kDecTB;
-  return tb * shared_wb + routed_tb * routed_wb;
+// Token blocks a decode batch can have: 32-token blocks of the shared
+// experts' rows, and of each routed expert's rows (at most one partial block
+// per expert that received a token).  Each has a readiness counter in the
+// decode FFN, so a batch runs there only if they fit.
+int64_t decode_token_blocks(int64_t T, int64_t K, int64_t N) {
+  return (T + kFfnTB - 1) / kFfnTB + std::min<int64_t>(N, T * K) + (T * K + kFfnTB - 1) / kFfnTB;
 }
 
 Layout make_layout(const moe_config& c) {
@@ -163,17 +161,8 @@ Layout make_layout(const moe_config& c) {
   L.ys = take(c.n_shared > 0 ? L.Tpad * int64_t(c.d_model) * 2 : 0);
   L.xdev = take(Tm * c.d_model * 2);
   L.outdev = take(Tm * c.d_model * 2);
-  // the decode GEMMs' stream-K partial sums and per-quarter tile counters
-  const int64_t Td = std::min<int64_t>(Tm, kDecodeMaxT);
-  const int64_t sh_cols = int64_t(c.n_shared) * c.d_ff_shared;
-  const int64_t gu_tiles = decode_max_tiles(Td, Km, N, (c.d_ff + kDecWB - 1) / kDecWB, (sh_cols + kDecWB - 1) / kDecWB);
-  const int64_t dn_tiles =
-      decode_max_tiles(Td, Km, N, (c.d_model + kDecWB - 1) / kDecWB, (c.d_model + kDecWB - 1) / kDecWB);
-  L.dec_part_gu = take(dec_partials_bytes<true>(kDecMaxCtas));
-  L.dec_part_dn = take(dec_partials_bytes<false>(kDecMaxCtas));
-  L.dec_ctr_gu = take(size_t(gu_tiles) * 4 * 4 + size_t(dn_tiles) * 4 * 4);
-  L.dec_ctr_dn = L.dec_ctr_gu + size_t(gu_tiles) * 4 * 4;
-  L.dec_ctr_bytes = size_t(gu_tiles + dn_tiles) * 4 * 4;
+  // the decode FFN's tile counter and readiness counters
+  L.ffn_ctr = take(ffn_counter_bytes());
   // the FP8 path: E4M3 codes of the permuted rows, of x, of H and Hs, each with its scale atoms
   // (512 bytes per 128 rows and 128 columns)
   L.Pa = (L.P + 127) / 128 * 128;
@@ -362,11 +351,8 @@ cudaError_t set_kernel_attrs() {
   if ((e = cudaFuncSetAttribute(gateup_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
   const int gs = static_cast<int>(gemm_smem_bytes());
   if ((e = cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
-  if ((e = cudaFuncSetAttribute(decode_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(dec_smem_bytes<true>()))))
-    return e;
-  if ((e = cudaFuncSetAttribute(decode_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(dec_smem_bytes<false>()))))
+  if ((e = cudaFuncSetAttribute(decode_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(ffn_smem_bytes()))))
     return e;
   const int fs = static_cast<int>(fp8_gemm_smem_bytes());
   if ((e = cudaFuncSetAttribute(fp8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, fs))) return e;
@@ -404,13 +390,6 @@ cudaError_t launch_down(int pairs, cudaStream_t s, bool pdl, const CUtensorMap& 
                     ga);
 }
 
-template <bool GU>
-cudaError_t launch_decode(int ctas, cudaStream_t s, bool pdl, const CUtensorMap& W0, const CUtensorMap& W1,
-                          const CUtensorMap& X, const CUtensorMap& Ws0, const CUtensorMap& Ws1, const CUtensorMap& Xs,
-                          const DecodeArgs& da) {
-  return launch_pdl(decode_gemm_kernel<GU>, dim3(ctas), dim3(kDecThreads), dec_smem_bytes<GU>(), s, 1, pdl, W0, W1, X,
-                    Ws0, Ws1, Xs, da);
-}
 
 cudaError_t launch_gateup(int ctas, cudaStream_t s, bool pdl, const CUtensorMap& A, const CUtensorMap& G,
                           const CUtensorMap& U, const CUtensorMap& As, const CUtensorMap& Gs, const CUtensorMap& Us,
@@ -461,11 +440,15 @@ class KernelTimer {
   cudaEvent_t stop_ = nullptr;
 };
 
+PermuteArgs permute_args(moe_ctx* h, const void* x, int64_t T, int32_t K, const RouterArgs& ra, bool gather);
+
 // The router step shared by the bf16 and FP8 forwards: affinities, top-K, the
 // per-block expert histogram and the scan (router_topk.cuh).  Records the
-// call's stream, T and K for moe_get_routing / moe_status_query.
+// call's stream, T and K for moe_get_routing / moe_status_query.  fused > 0:
+// route_permute_decode_kernel, which also forms the permutation (fused == 2:
+// with the row copies); the caller launches no permutation then.
 moe_status enqueue_router(moe_ctx* h, const void* x, int64_t T, const moe_router* router, int32_t K,
-                          cudaStream_t s0, bool pdl, RouterArgs& ra) {
+                          cudaStream_t s0, bool pdl, RouterArgs& ra, int fused = 0) {
   const moe_config& c = h->cfg;
   const Layout& L = h->L;
   const int64_t d = c.d_model, N = c.n_routed;
@@ -505,6 +488,17 @@ moe_status enqueue_router(moe_ctx* h, const void* x, int64_t T, const moe_router
     ra.max_nodes = c.route_max_nodes;
   }
   KernelTimer kt(h, MOE_KERNEL_ROUTER, s0);
+  if (fused > 0) {
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    const __nv_bfloat16* eb = static_cast<const __nv_bfloat16*>(router->weight);
+    const PermuteArgs pa = permute_args(h, x, T, K, ra, fused == 2);
+    const RouteTables rt{ra.counts, ra.offsets, ra.row_start, ra.mtile_start, ra.mtile128_start, ra.block_counts};
+    const dim3 grid((unsigned)(T * kRouteCluster)), block(kRouteThreads);
+    const cudaError_t e =
+        sigmoid ? launch_pdl(route_permute_decode_kernel<true>, grid, block, 0, s0, 1, pdl, xb, eb, ra, pa, rt)
+                : launch_pdl(route_permute_decode_kernel<false>, grid, block, 0, s0, 1, pdl, xb, eb, ra, pa, rt);
+    return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   if (T <= kSmallRouterMaxT) {
     // a few tokens: one CTA per token on the CUDA cores
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
@@ -644,16 +638,16 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
     return MOE_ERR_NOMEM;
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
-  ok = ok && cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) == cudaSuccess;
+  ok = ok && cudaMemset(h->ws + h->L.ffn_ctr, 0, ffn_counter_bytes()) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
-  ok = ok && encode_bf16(&h->tm_xperm32, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kDecBoxRowsX, 2);
-  ok = ok && encode_bf16(&h->tm_h32, h->ws + h->L.h, 1, h->L.P, c.d_ff, kDecBoxRowsX, 2);
+  ok = ok && encode_bf16(&h->tm_xperm32, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kFfnBoxRowsX, 2);
+  ok = ok && encode_bf16(&h->tm_h32, h->ws + h->L.h, 1, h->L.P, c.d_ff, kFfnBoxRowsX, 2);
   if (c.n_shared > 0) {
     ok = ok && encode_bf16(&h->tm_hs, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kBoxRowsA, 2);
     ok = ok &&
-         encode_bf16(&h->tm_hs32, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kDecBoxRowsX, 2);
+         encode_bf16(&h->tm_hs32, h->ws + h->L.hs, 1, h->L.Tpad, int64_t(c.n_shared) * c.d_ff_shared, kFfnBoxRowsX, 2);
   }
   if (c.flags & MOE_FLAG_FP8) {
     const int64_t SI = int64_t(c.n_shared) * c.d_ff_shared;
@@ -709,9 +703,10 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
 
   // descriptors that follow the caller's pointers
-  const bool decode = T <= kDecodeMaxT;
+  // a decode batch: the weight-streaming FFN, if its token blocks fit the readiness counters
+  const bool decode = T <= kDecodeMaxT && decode_token_blocks(T, K, N) <= kFfnMaxBlocks;
   bool ok = true;
-  if (decode) ok = ok && refresh(h->tm_x32, x, T, 1, T, d, kDecBoxRowsX, 2);
+  if (decode) ok = ok && refresh(h->tm_x32, x, T, 1, T, d, kFfnBoxRowsX, 2);
   ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, kGuBoxRowsB, 3);
   ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, kGuBoxRowsB, 3);
   ok = ok && refresh(h->tm_wd, experts->w_down, 0, N, d, I, kBoxRowsB, 3);
@@ -726,88 +721,68 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   const int nblk = ceil_div(T, 128);
 
   // ---- router and permutation ----
+  // a decode batch with a small router matrix: both in one launch
+  const bool fused_route = decode && route_decode_fits(T, N, d, K);
   RouterArgs ra;
   {
-    const moe_status st = enqueue_router(h, x, T, router, K, s0, pdl, ra);
+    const moe_status st = enqueue_router(h, x, T, router, K, s0, pdl, ra, fused_route ? (do_routed ? 2 : 1) : 0);
     if (st != MOE_OK) return st;
   }
   PermuteArgs pa = permute_args(h, x, T, K, ra, do_routed);
-  {
+  if (!fused_route) {
     KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
     const dim3 grid(nblk, do_routed ? pa.split : 1);
     if (launch_pdl(permute_gather_kernel, grid, dim3(kPermThreads), 0, s0, 1, pdl, pa) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
 
-  // ---- the expert GEMMs of a small batch: weight-streaming, stream-K ----
+  // ---- the expert FFNs of a small batch: one weight-streaming launch (decode_ffn.cuh) ----
   if (decode && (do_routed || do_shared)) {
-    const int ctas = std::min(h->num_sms, kDecMaxCtas);
-    DecodeArgs g{};
+    FfnArgs f{};
+    f.T = (int)T;
     if (do_routed) {
-      g.num_groups = (int)N;
-      g.counts = ra.counts;
-      g.row_start = ra.row_start;
-      g.n_wb = ceil_div(I, kDecWB);
-      g.num_kb = ceil_div(d, kDecBK);
-      g.out = h->at<__nv_bfloat16>(L.h);
-      g.ld_out = (int)I;
-      g.n_limit = (int)I;
+      f.G = (int)N;
+      f.n_wb_gu = ceil_div(I, kFfnWB);
+      f.n_wb_dn = ceil_div(d, kFfnWB);
+      f.kb_gu = ceil_div(d, kFfnBK);
+      f.kb_dn = ceil_div(I, kFfnBK);
+      f.counts = ra.counts;
+      f.row_start = ra.row_start;
+      f.row_scale = pa.gate_perm;
+      f.h = h->at<__nv_bfloat16>(L.h);
+      f.y = h->at<__nv_bfloat16>(L.y);
     }
     if (do_shared) {
-      g.sh_rows = (int)T;
-      g.sh_n_wb = ceil_div(Ks * Is, kDecWB);
-      g.sh_J = 1;
-      g.sh_kb_per_j = ceil_div(d, kDecBK);
-      g.sh_out = h->at<__nv_bfloat16>(L.hs);
-      g.sh_ld_out = (int)(Ks * Is);
-      g.sh_n_limit = (int)(Ks * Is);
+      f.sh_blocks = ceil_div(T, kFfnTB);
+      f.sh_n_wb_gu = ceil_div(Ks * Is, kFfnWB);
+      f.sh_n_wb_dn = ceil_div(d, kFfnWB);
+      f.sh_J = (int)Ks;
+      f.sh_kb_per_j = ceil_div(Is, kFfnBK);
+      f.sh_k_per_j = (int)Is;
+      f.hs = h->at<__nv_bfloat16>(L.hs);
+      f.ys = h->at<__nv_bfloat16>(L.ys);
     }
-    g.partials = h->at<float>(L.dec_part_gu);
-    g.tile_ctr = h->at<uint32_t>(L.dec_ctr_gu);
-    g.err = h->at<uint32_t>(L.err);
-    g.timeout_ns = kTimeoutNs;
+    f.kb_gu = ceil_div(d, kFfnBK);  // the shared gate/up tiles' k loop too
+    f.I = (int)I;
+    f.sh_cols = (int)(Ks * Is);
+    f.d = (int)d;
+    f.ctr = h->at<uint32_t>(L.ffn_ctr);
+    f.err = h->at<uint32_t>(L.err);
+    f.timeout_ns = kTimeoutNs;
     // an absent part's maps are never read; the present part's stand in
-    const CUtensorMap& W0 = do_routed ? h->tm_wg.map : h->tm_swg.map;
-    const CUtensorMap& W1 = do_routed ? h->tm_wu.map : h->tm_swu.map;
-    const CUtensorMap& Ws0 = do_shared ? h->tm_swg.map : h->tm_wg.map;
-    const CUtensorMap& Ws1 = do_shared ? h->tm_swu.map : h->tm_wu.map;
-    {
-      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
-      if (launch_decode<true>(ctas, s0, pdl, W0, W1, h->tm_xperm32, Ws0, Ws1, h->tm_x32.map, g) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    DecodeArgs g2{};
-    if (do_routed) {
-      g2.num_groups = (int)N;
-      g2.counts = ra.counts;
-      g2.row_start = ra.row_start;
-      g2.n_wb = ceil_div(d, kDecWB);
-      g2.num_kb = ceil_div(I, kDecBK);
-      g2.row_scale = pa.gate_perm;
-      g2.out = h->at<__nv_bfloat16>(L.y);
-      g2.ld_out = (int)d;
-      g2.n_limit = (int)d;
-    }
-    if (do_shared) {
-      g2.sh_rows = (int)T;
-      g2.sh_n_wb = ceil_div(d, kDecWB);
-      g2.sh_J = (int)Ks;
-      g2.sh_kb_per_j = ceil_div(Is, kDecBK);
-      g2.sh_k_per_j = (int)Is;
-      g2.sh_out = h->at<__nv_bfloat16>(L.ys);
-      g2.sh_ld_out = (int)d;
-      g2.sh_n_limit = (int)d;
-    }
-    g2.partials = h->at<float>(L.dec_part_dn);
-    g2.tile_ctr = h->at<uint32_t>(L.dec_ctr_dn);
-    g2.err = h->at<uint32_t>(L.err);
-    g2.timeout_ns = kTimeoutNs;
-    const CUtensorMap& D0 = do_routed ? h->tm_wd.map : h->tm_swd.map;
-    const CUtensorMap& Ds0 = do_shared ? h->tm_swd.map : h->tm_wd.map;
-    const CUtensorMap& HX = do_routed ? h->tm_h32 : h->tm_hs32;
-    const CUtensorMap& HXs = do_shared ? h->tm_hs32 : h->tm_h32;
-    KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
-    if (launch_decode<false>(ctas, s0, pdl, D0, D0, HX, Ds0, Ds0, HXs, g2) != cudaSuccess) return MOE_ERR_CUDA;
+    const CUtensorMap& Wg = do_routed ? h->tm_wg.map : h->tm_swg.map;
+    const CUtensorMap& Wu = do_routed ? h->tm_wu.map : h->tm_swu.map;
+    const CUtensorMap& Wd = do_routed ? h->tm_wd.map : h->tm_swd.map;
+    const CUtensorMap& Xr = do_routed ? h->tm_xperm32 : h->tm_x32.map;
+    const CUtensorMap& Hr = do_routed ? h->tm_h32 : h->tm_hs32;
+    const CUtensorMap& Wsg = do_shared ? h->tm_swg.map : h->tm_wg.map;
+    const CUtensorMap& Wsu = do_shared ? h->tm_swu.map : h->tm_wu.map;
+    const CUtensorMap& Wsd = do_shared ? h->tm_swd.map : h->tm_wd.map;
+    const CUtensorMap& Hsm = do_shared ? h->tm_hs32 : h->tm_h32;
+    KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+    if (launch_pdl(decode_ffn_kernel, dim3(h->num_sms), dim3(kFfnThreads), ffn_smem_bytes(), s0, 1, pdl, Wg, Wu, Xr,
+                   Wsg, Wsu, h->tm_x32.map, Wd, Hr, Wsd, Hsm, f) != cudaSuccess)
+      return MOE_ERR_CUDA;
   }
 
   // ---- the expert GEMMs: shared experts' tiles first, then the routed experts' ----
@@ -1189,9 +1164,9 @@ moe_status moe_status_query(moe_handle h) {
   uint32_t err = 0;
   if (cudaMemcpy(&err, h->ws + h->L.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
   if (err) {
-    // a kernel that gave up may have left stream-K tile counters part-counted
+    // a kernel that gave up may have left the decode FFN's counters part-counted
     if (cudaMemset(h->ws + h->L.err, 0, 4) != cudaSuccess ||
-        cudaMemset(h->ws + h->L.dec_ctr_gu, 0, h->L.dec_ctr_bytes) != cudaSuccess)
+        cudaMemset(h->ws + h->L.ffn_ctr, 0, ffn_counter_bytes()) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_ERR_TIMEOUT;

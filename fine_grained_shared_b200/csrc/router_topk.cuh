@@ -414,6 +414,94 @@ constexpr int kSmallRouterGroup = 8;   // experts per CTA: one per warp
 static_assert(kSmallRouterThreads / 32 == kSmallRouterGroup, "one warp per expert of the group");
 constexpr int kSmallRouterPass = 8;    // 16-byte vectors per lane per pass (2048 columns)
 
+// Token t's selection by one warp from its N logits zrow (step 2 of the layer):
+// the keys (softmax: logit + logit bias; sigmoid: s + selection bias, NaN
+// ranked below every number), the softmax statistics over all N, the allowed
+// nodes under node-limited routing, then K rounds of a warp argmax ordered by
+// (key descending, index ascending); writes idx[t, :] and gate[t, :].  key and
+// sval are shared-memory rows of at least N floats; ZGLOBAL: zrow is in global
+// memory, written by other CTAs (read through L2).  lbias / sbias: the logit
+// and selection biases (either may be null).
+template <bool SIGMOID, bool ZGLOBAL>
+__device__ __forceinline__ void select_token_warp(int t, int K, const RouterArgs& a, const float* zrow, float* key,
+                                                  float* sval, const float* lbias, const float* sbias) {
+  const int lane = threadIdx.x & 31;
+  for (int i = lane; i < a.N; i += 32) {
+    const float z = ZGLOBAL ? __ldcg(zrow + i) : zrow[i];
+    if (SIGMOID) {
+      const float sv = 1.f / (1.f + __expf(-z));
+      sval[i] = sv;
+      const float k = sv + (sbias ? sbias[i] : 0.f);
+      key[i] = isnan(k) ? -INFINITY : k;  // NaN ranks below every number
+    } else {
+      const float k = z + (lbias ? lbias[i] : 0.f);  // softmax is monotone in z
+      key[i] = isnan(k) ? -INFINITY : k;
+    }
+  }
+  __syncwarp();
+  // softmax statistics over all N logits (softmax mode)
+  float mx = -INFINITY, sum = 0.f;
+  if (!SIGMOID) {
+    for (int i = lane; i < a.N; i += 32) mx = fmaxf(mx, key[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int i = lane; i < a.N; i += 32) sum += __expf(key[i] - mx);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  // node-limited routing: each node's largest key, then the allowed nodes
+  uint32_t allowed = 0xffffffffu;
+  if (a.nodes > 0) {
+    float nmax[kMaxRouteNodes];
+#pragma unroll
+    for (int g = 0; g < kMaxRouteNodes; ++g) {
+      float m = -INFINITY;
+      if (g < a.nodes)
+        for (int i = g * a.per_node + lane; i < (g + 1) * a.per_node; i += 32) m = fmaxf(m, key[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      nmax[g] = m;
+    }
+    allowed = choose_nodes(nmax, a.nodes, a.max_nodes);
+  }
+  uint32_t taken = 0;  // bit j: this lane's expert lane + 32 * j is already selected
+  int sel[8];
+  float sel_s[8];
+  float tot = 0.f;
+  for (int k = 0; k < K; ++k) {
+    float bk = -INFINITY;
+    int bi = 0x7fffffff;
+    for (int j = 0, i = lane; i < a.N; ++j, i += 32) {
+      if (taken & (1u << j)) continue;
+      if (a.nodes > 0 && !((allowed >> (i / a.per_node)) & 1u)) continue;
+      const float v = key[i];
+      if (v > bk || (v == bk && i < bi)) {
+        bk = v;
+        bi = i;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ov > bk || (ov == bk && oi < bi)) {
+        bk = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    sel[k] = bi;
+    sel_s[k] = SIGMOID ? sval[bi] : __expf(bk - mx) / sum;
+    tot += sel_s[k];
+  }
+  if (lane == 0) {
+    for (int k = 0; k < K; ++k) {
+      a.idx[static_cast<size_t>(t) * K + k] = sel[k];
+      a.gate[static_cast<size_t>(t) * K + k] = SIGMOID ? sel_s[k] / tot : sel_s[k];
+    }
+  }
+}
+
 struct SmallRouterArgs {
   float* logits;          // [T, N] fp32 scratch
   uint32_t* token_done;   // [T] CTAs finished per token, zero between calls
@@ -476,83 +564,9 @@ __global__ void __launch_bounds__(kSmallRouterThreads)
   if (!is_last) return;
   __threadfence();
   if (tid == 0) sa.token_done[t] = 0u;  // every CTA of this token has counted itself
-  if (warp == 0) {
-    const float* lrow = sa.logits + static_cast<size_t>(t) * a.N;
-    for (int i = lane; i < a.N; i += 32) {
-      const float z = __ldcg(lrow + i);
-      if (SIGMOID) {
-        const float sv = 1.f / (1.f + __expf(-z));
-        sval[i] = sv;
-        const float k = sv + (a.select_bias ? a.select_bias[i] : 0.f);
-        key[i] = isnan(k) ? -INFINITY : k;  // NaN ranks below every number
-      } else {
-        const float k = z + (a.logit_bias ? a.logit_bias[i] : 0.f);  // softmax is monotone in z
-        key[i] = isnan(k) ? -INFINITY : k;
-      }
-    }
-    __syncwarp();
-    // softmax statistics over all N logits (softmax mode)
-    float mx = -INFINITY, sum = 0.f;
-    if (!SIGMOID) {
-      for (int i = lane; i < a.N; i += 32) mx = fmaxf(mx, key[i]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      for (int i = lane; i < a.N; i += 32) sum += __expf(key[i] - mx);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    }
-    // node-limited routing: each node's largest key, then the allowed nodes
-    uint32_t allowed = 0xffffffffu;
-    if (a.nodes > 0) {
-      float nmax[kMaxRouteNodes];
-#pragma unroll
-      for (int g = 0; g < kMaxRouteNodes; ++g) {
-        float m = -INFINITY;
-        if (g < a.nodes)
-          for (int i = g * a.per_node + lane; i < (g + 1) * a.per_node; i += 32) m = fmaxf(m, key[i]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        nmax[g] = m;
-      }
-      allowed = choose_nodes(nmax, a.nodes, a.max_nodes);
-    }
-    uint32_t taken = 0;  // bit j: this lane's expert lane + 32 * j is already selected
-    int sel[8];
-    float sel_s[8];
-    float tot = 0.f;
-    for (int k = 0; k < K; ++k) {
-      float bk = -INFINITY;
-      int bi = 0x7fffffff;
-      for (int j = 0, i = lane; i < a.N; ++j, i += 32) {
-        if (taken & (1u << j)) continue;
-        if (a.nodes > 0 && !((allowed >> (i / a.per_node)) & 1u)) continue;
-        const float v = key[i];
-        if (v > bk || (v == bk && i < bi)) {
-          bk = v;
-          bi = i;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bk, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bk || (ov == bk && oi < bi)) {
-          bk = ov;
-          bi = oi;
-        }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      sel[k] = bi;
-      sel_s[k] = SIGMOID ? sval[bi] : __expf(bk - mx) / sum;
-      tot += sel_s[k];
-    }
-    if (lane == 0) {
-      for (int k = 0; k < K; ++k) {
-        a.idx[static_cast<size_t>(t) * K + k] = sel[k];
-        a.gate[static_cast<size_t>(t) * K + k] = SIGMOID ? sel_s[k] / tot : sel_s[k];
-      }
-    }
-  }
+  if (warp == 0)
+    select_token_warp<SIGMOID, true>(t, K, a, sa.logits + static_cast<size_t>(t) * a.N, key, sval, a.logit_bias,
+                                     a.select_bias);
   __threadfence();
   __syncthreads();
   if (tid == 0) is_last = (atomicAdd(a.done_counter, 1u) == static_cast<uint32_t>(gridDim.x - 1));

@@ -115,14 +115,20 @@ def test_roofline_of_the_dominant_kernel_from_its_own_numbers():
     assert roof["bound"] == "tensor" and roof["flop_per_launch"] == flop
     assert roof["achieved"] == pytest.approx(flop / 1.2252e-3 / 1e12)
     assert roof["frac"] == pytest.approx(roof["achieved"] / 1667.0) and peak == 1667.0
+    # a decode batch: both expert GEMMs are one launch (timed as gate_up), over all three projections
     decode = W.CONFIGS["16b_decode"]
     counts = [6] * 30 + [0] * 34                  # 30 of the 64 experts touched
-    r = dict(r, ms_total=20.0, ms_step=0.18, dominant_ms=0.11, counts=counts,
-             kernel_ms={"gate_up": 0.11, "down": 0.055})
+    r = dict(r, ms_total=20.0, ms_step=0.13, dominant_ms=0.11, counts=counts,
+             kernel_ms={"gate_up": 0.11, "down": 0.0})
     roof, _, _ = bench.roofline_of(decode, r, peaks, "measured")
-    wbytes = 2 * 2 * 2048 * (30 * 1408 + 2 * 1408)
+    wbytes = 3 * 2 * 2048 * (30 * 1408 + 2 * 1408)
     assert roof["bound"] == "hbm" and roof["weight_bytes_per_launch"] == wbytes
+    assert roof["flop_per_launch"] == 6.0 * 32 * 2048 * (6 * 1408 + 2 * 1408)
     assert roof["achieved"] == pytest.approx(wbytes / 0.11e-3 / 1e9)
+    assert "decode_ffn_kernel" in roof["kernel"]
     f = bench.hbm_fractions(decode, r, peaks)
-    assert f["down_gbs"] == pytest.approx(wbytes / 2 / 0.055e-3 / 1e9)
-    assert f["layer_frac"] == pytest.approx(1.5 * wbytes / 0.18e-3 / 1e9 / 6500.0)
+    assert f["ffn_gbs"] == pytest.approx(wbytes / 0.11e-3 / 1e9) and "down_gbs" not in f
+    assert f["layer_frac"] == pytest.approx(wbytes / 0.13e-3 / 1e9 / 6500.0)
+    # the FP8 layer keeps separate GEMM launches at every batch size
+    f8 = bench.hbm_fractions(decode, dict(r, kernel_ms={"gate_up": 0.05, "down": 0.03}), peaks, fp8=True)
+    assert f8["down_gbs"] is not None and "ffn_gbs" not in f8

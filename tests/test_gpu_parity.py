@@ -225,7 +225,7 @@ def _node_limited_gaps(key, K, nodes, M):
     return np.minimum(node_gap, k_gap)
 
 
-@pytest.mark.parametrize("case", ["tc_softmax", "small_sigmoid", "v3_like"])
+@pytest.mark.parametrize("case", ["tc_softmax", "small_sigmoid", "v3_like", "decode_softmax"])
 def test_node_limited_routing_matches_the_oracle(case):
     """Node-limited routing (DeepSeek-V3 report summary, section 2): each token's K experts come
     from at most M nodes, those holding its largest keys; bit-exact against the oracle's
@@ -234,7 +234,9 @@ def test_node_limited_routing_matches_the_oracle(case):
             "small_sigmoid": (LS("nl_sig", T=100, d=256, N=64, I=64, K=6, Ks=1, Is=64, gate="sigmoid",
                                  sigma=0.03, bias="uniform", seed=72), 4, 2),
             "v3_like": (LS("nl_v3", T=1000, d=512, N=256, I=64, K=8, Ks=1, Is=64, gate="sigmoid", sigma=0.006,
-                           bias="uniform", seed=73), 8, 4)}[case]
+                           bias="uniform", seed=73), 8, 4),
+            # a decode batch: one router CTA per token, the tables built by the permutation
+            "decode_softmax": (LS("nl_dec", T=48, d=512, N=64, I=64, K=6, Ks=1, Is=64, sigma=0.05, seed=74), 8, 3)}[case]
     shape, nodes, M = spec
     host, dev = H.device_inputs(shape)
     layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks, d_ff_shared=shape.Is,
@@ -501,9 +503,13 @@ def test_timing_records_only_the_kernels_asked_for():
     layer.set_timing(True)
     H.run(layer, dev["x"], shape.K)
     assert all(n == 1 for _, n in layer.kernel_times().values())
-    small = dev["x"][:40].contiguous()          # a decode-sized batch (the decode GEMMs) launches the same five
+    # a decode-sized batch: routing and permutation in one launch (timed as the router), both expert
+    # GEMMs in another (timed as gate_up)
+    small = dev["x"][:40].contiguous()
     H.run(layer, small, shape.K)
-    assert all(n == 1 for _, n in layer.kernel_times().values())
+    t = layer.kernel_times()
+    assert t["permute"][1] == 0 and t["down"][1] == 0
+    assert all(n == 1 for k, (_, n) in t.items() if k not in ("permute", "down"))
     layer.set_timing(False)
     H.run(layer, dev["x"], shape.K)
     assert all(n == 0 for _, n in layer.kernel_times().values())
