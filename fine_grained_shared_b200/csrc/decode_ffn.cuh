@@ -532,12 +532,18 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, kFfnTmemCols);
   }
+  // the last CTA to finish leaves the counters at zero for the next launch (all of its threads clear them)
+  __shared__ uint32_t s_last;
   if (tid == 0) {
-    // the last CTA to finish leaves the counters at zero for the next launch
     __threadfence();
-    if (atomicAdd(ctas_done, 1u) == gridDim.x - 1) {
-      __threadfence();
-      for (int i = 0; i < kFfnMaxBlocks; ++i) ready[i] = 0u;
+    s_last = atomicAdd(ctas_done, 1u) == gridDim.x - 1 ? 1u : 0u;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    for (int i = tid; i < kFfnMaxBlocks; i += kFfnThreads) ready[i] = 0u;
+    __syncthreads();
+    if (tid == 0) {
       *next_tile = 0u;
       __threadfence();
       *ctas_done = 0u;

@@ -266,9 +266,17 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteTh
     if (tid < N && ok(tid)) {
       const float ki = key[tid];
       int rank = 0;
-      for (int j = 0; j < N; ++j) {
-        const float kj = key[j];
-        rank += (ok(j) && (kj > ki || (kj == ki && j < tid))) ? 1 : 0;
+      if (a.nodes <= 0) {
+#pragma unroll 8
+        for (int j = 0; j < N; ++j) {
+          const float kj = key[j];
+          rank += (kj > ki || (kj == ki && j < tid)) ? 1 : 0;
+        }
+      } else {
+        for (int j = 0; j < N; ++j) {
+          const float kj = key[j];
+          rank += (ok(j) && (kj > ki || (kj == ki && j < tid))) ? 1 : 0;
+        }
       }
       if (rank < K) sel[rank] = tid;
     }
@@ -375,21 +383,33 @@ __global__ void __cluster_dims__(kRouteCluster, 1, 1) __launch_bounds__(kRouteTh
   }
   if (!p.gather) return;
   __syncthreads();
-  // one warp per (token, slot) pair over the cluster's 64 warps (a 32-token
-  // batch with K = 6 gives each warp three 4 KB rows; a warp per token row
-  // would leave half of the CTAs idle)
+  // one warp per (token, slot) pair over the cluster's 64 warps, up to three
+  // pairs at a time with all of their loads out before any store (a 32-token
+  // batch with K = 6 gives each warp three 4 KB rows; one row per round trip
+  // took 4.6 us, a warp per token row left half of the CTAs idle)
   const int nvec = d >> 3;
-  for (int q = r * (kRouteThreads / 32) + warp; q < T * K; q += kRouteCluster * (kRouteThreads / 32)) {
-    const uint4* srow = reinterpret_cast<const uint4*>(x + static_cast<size_t>(q / K) * d);
-    uint4* drow = reinterpret_cast<uint4*>(p.x_perm + static_cast<size_t>(dst[q]) * d);
-    for (int c = lane; c < nvec; c += 32 * 8) {
-      uint4 v[8];
+  constexpr int kW = kRouteCluster * (kRouteThreads / 32);
+  for (int q0 = r * (kRouteThreads / 32) + warp; q0 < T * K; q0 += 3 * kW) {
+    for (int c = lane; c < nvec; c += 32 * 4) {
+      uint4 v[3][4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (c + 32 * u < nvec) v[u] = __ldg(srow + c + 32 * u);
+      for (int pr = 0; pr < 3; ++pr) {
+        const int q = q0 + pr * kW;
+        const uint4* srow = reinterpret_cast<const uint4*>(x + static_cast<size_t>(q < T * K ? q / K : 0) * d);
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (c + 32 * u < nvec) drow[c + 32 * u] = v[u];
+        for (int u = 0; u < 4; ++u)
+          if (q < T * K && c + 32 * u < nvec) v[pr][u] = __ldg(srow + c + 32 * u);
+      }
+#pragma unroll
+      for (int pr = 0; pr < 3; ++pr) {
+        const int q = q0 + pr * kW;
+        if (q < T * K) {
+          uint4* drow = reinterpret_cast<uint4*>(p.x_perm + static_cast<size_t>(dst[q]) * d);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (c + 32 * u < nvec) drow[c + 32 * u] = v[pr][u];
+        }
+      }
     }
   }
 }
