@@ -28,6 +28,7 @@
 
 #include "../../include/fgs_moe.h"
 #include "decode_ffn.cuh"
+#include "decode_ffn8.cuh"
 #include "down_gemm.cuh"
 #include "fp8_gemm.cuh"
 #include "gateup_gemm.cuh"
@@ -242,9 +243,11 @@ struct moe_ctx {
   int last_K = 0;
   // TMA descriptors: workspace ones are fixed, the others follow the caller's pointers
   CUtensorMap tm_xperm, tm_h, tm_hs;
-  CUtensorMap tm_xperm32, tm_h32, tm_hs32;  // 32-row token boxes of the decode GEMMs
+  CUtensorMap tm_xperm32, tm_h32, tm_hs32;  // 32-row token boxes of the decode FFN
   CUtensorMap tm_xq_perm, tm_xq, tm_hq, tm_hsq;  // FP8 codes of the activations (128-row boxes)
+  CUtensorMap tm_xq_perm32, tm_xq32, tm_hq32, tm_hsq32;  // the same with 32-row boxes (FP8 decode FFN)
   MapCache tm8_wg, tm8_wu, tm8_wd, tm8_swg, tm8_swu, tm8_swd;  // FP8 weight codes
+  MapCache tm8_wd128, tm8_swd128;  // W_down codes with 128-row boxes (FP8 decode FFN)
   MapCache tm_x, tm_x32, tm_router, tm_wg, tm_wu, tm_wd, tm_swg, tm_swu, tm_swd;
   // host-buffer forward: copy streams and per-chunk events, created on first use
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
@@ -356,7 +359,9 @@ cudaError_t set_kernel_attrs() {
     return e;
   const int fs = static_cast<int>(fp8_gemm_smem_bytes());
   if ((e = cudaFuncSetAttribute(fp8_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, fs))) return e;
-  return cudaFuncSetAttribute(fp8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, fs);
+  if ((e = cudaFuncSetAttribute(fp8_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, fs))) return e;
+  return cudaFuncSetAttribute(decode_ffn8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(ffn8_smem_bytes()));
 }
 
 bool refresh_u8(MapCache& c, const void* p, uint64_t d2, uint64_t rows, uint64_t cols, uint32_t box_rows, int rank) {
@@ -655,6 +660,10 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
     ok = ok && encode_u8(&h->tm_xq, h->ws + h->L.xq, 1, h->L.Tpad, c.d_model, 128, 2);
     ok = ok && encode_u8(&h->tm_hq, h->ws + h->L.hq, 1, h->L.Pa, c.d_ff, 128, 2);
     if (SI > 0) ok = ok && encode_u8(&h->tm_hsq, h->ws + h->L.hsq, 1, h->L.Tpad, SI, 128, 2);
+    ok = ok && encode_u8(&h->tm_xq_perm32, h->ws + h->L.xq_perm, 1, h->L.Pa, c.d_model, kFfnBoxRowsX, 2);
+    ok = ok && encode_u8(&h->tm_xq32, h->ws + h->L.xq, 1, h->L.Tpad, c.d_model, kFfnBoxRowsX, 2);
+    ok = ok && encode_u8(&h->tm_hq32, h->ws + h->L.hq, 1, h->L.Pa, c.d_ff, kFfnBoxRowsX, 2);
+    if (SI > 0) ok = ok && encode_u8(&h->tm_hsq32, h->ws + h->L.hsq, 1, h->L.Tpad, SI, kFfnBoxRowsX, 2);
   }
   ok = ok && cudaDeviceSynchronize() == cudaSuccess;
   if (!ok) {
@@ -936,7 +945,76 @@ moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_rou
       return MOE_ERR_CUDA;
   }
 
-  if (do_routed || do_shared) {
+  // a decode batch: both expert GEMMs in one weight-streaming launch (decode_ffn8.cuh)
+  const bool decode = T <= kDecodeMaxT && decode_token_blocks(T, K, N) <= kFfnMaxBlocks;
+  if (decode && (do_routed || do_shared)) {
+    const int64_t SI = Ks * Is;
+    ok = refresh_u8(h->tm8_wd128, experts->w_down, N, d, I, kFfnBoxRowsW, 3);
+    if (shared) ok = ok && refresh_u8(h->tm8_swd128, shared->w_down, Ks, d, Is, kFfnBoxRowsW, 3);
+    if (!ok) return MOE_ERR_CUDA;
+    Ffn8Args f8{};
+    FfnArgs& f = f8.f;
+    f.T = (int)T;
+    f.kb_gu = (int)(d / kF8BK);
+    if (do_routed) {
+      f.G = (int)N;
+      f.n_wb_gu = (int)(I / kFfnWB);
+      f.n_wb_dn = (int)(d / kFfnWB);
+      f.kb_dn = (int)(I / kF8BK);
+      f.counts = ra.counts;
+      f.row_start = ra.row_start;
+      f.row_scale = h->at<float>(L.gate_perm);
+      f.y = h->at<__nv_bfloat16>(L.y);
+    }
+    if (do_shared) {
+      f.sh_blocks = ceil_div(T, kFfnTB);
+      f.sh_n_wb_gu = (int)(SI / kFfnWB);
+      f.sh_n_wb_dn = (int)(d / kFfnWB);
+      f.sh_J = (int)Ks;
+      f.sh_kb_per_j = (int)(Is / kF8BK);
+      f.sh_k_per_j = (int)Is;
+      f.ys = h->at<__nv_bfloat16>(L.ys);
+    }
+    f.I = (int)I;
+    f.sh_cols = (int)SI;
+    f.d = (int)d;
+    f.ctr = h->at<uint32_t>(L.ffn_ctr);
+    f.err = h->at<uint32_t>(L.err);
+    f.timeout_ns = kTimeoutNs;
+    f8.x_atoms = h->at<uint8_t>(L.xs_perm);
+    f8.xs_atoms = h->at<uint8_t>(L.xs);
+    f8.hq = h->at<uint8_t>(L.hq);
+    f8.h_atoms = h->at<uint8_t>(L.hs_perm);
+    f8.hsq = h->at<uint8_t>(L.hsq);
+    f8.hs_atoms = h->at<uint8_t>(L.hss);
+    f8.s_gate = experts->s_gate;
+    f8.s_up = experts->s_up;
+    f8.s_down = experts->s_down;
+    if (shared) {
+      f8.sh_s_gate = shared->s_gate;
+      f8.sh_s_up = shared->s_up;
+      f8.sh_s_down = shared->s_down;
+    }
+    // an absent part's maps are never read; the present part's stand in
+    const CUtensorMap& Wg = do_routed ? h->tm8_wg.map : h->tm8_swg.map;
+    const CUtensorMap& Wu = do_routed ? h->tm8_wu.map : h->tm8_swu.map;
+    const CUtensorMap& Wd = do_routed ? h->tm8_wd128.map : h->tm8_swd128.map;
+    const CUtensorMap& Xr = do_routed ? h->tm_xq_perm32 : h->tm_xq32;
+    const CUtensorMap& Hr = do_routed ? h->tm_hq32 : h->tm_hsq32;
+    const CUtensorMap& Wsg = do_shared ? h->tm8_swg.map : h->tm8_wg.map;
+    const CUtensorMap& Wsu = do_shared ? h->tm8_swu.map : h->tm8_wu.map;
+    const CUtensorMap& Wsd = do_shared ? h->tm8_swd128.map : h->tm8_wd128.map;
+    const CUtensorMap& Xs = do_shared ? h->tm_xq32 : h->tm_xq_perm32;
+    const CUtensorMap& Hs = do_shared ? h->tm_hsq32 : h->tm_hq32;
+    {
+      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+      if (launch_pdl(decode_ffn8_kernel, dim3(h->num_sms), dim3(kFfnThreads), ffn8_smem_bytes(), s0, 1, pdl, Wg,
+                     Wu, Xr, Wsg, Wsu, Xs, Wd, Hr, Wsd, Hs, f8) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+  }
+
+  if (!decode && (do_routed || do_shared)) {
     const int64_t SI = Ks * Is;
     // an absent part's maps are never read; the present part's stand in
     const CUtensorMap& A = do_routed ? h->tm_xq_perm : h->tm_xq;

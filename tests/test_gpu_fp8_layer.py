@@ -33,6 +33,11 @@ SHAPES = {
     "no_shared": LS("fp8_no_shared", T=200, d=128, N=12, I=384, K=3, Ks=0, Is=0, sigma=0.05, bias="normal",
                     seed=63),
     "decode": LS("fp8_decode", T=20, d=512, N=24, I=256, K=6, Ks=2, Is=128, sigma=0.03, bias="zipf", seed=64),
+    # decode batches run the FP8 decode FFN: two token blocks of routed rows without shared experts, and
+    # two shared token blocks
+    "decode_t64_sigmoid": LS("fp8_decode_t64", T=64, d=384, N=20, I=256, K=4, Ks=0, Is=0, gate="sigmoid",
+                             sigma=0.03, bias="uniform", seed=65),
+    "decode_t40": LS("fp8_decode_t40", T=40, d=256, N=12, I=384, K=2, Ks=2, Is=128, sigma=0.05, seed=66),
 }
 
 FLAGS_ROUTED = B.MOE_FLAG_NO_RESIDUAL | B.MOE_FLAG_NO_SHARED
@@ -94,6 +99,27 @@ def test_fp8_layer_16b_prefill_every_tile():
     print(f"16b_prefill fp8: compared rows {rows.size}, "
           + ", ".join(f"{k}: max err {v[0]:.2e} rms err {v[2]:.2e} rms {v[1]:.2e}"
                       for k, v in res.items() if k != "exempt"))
+
+
+def test_fp8_layer_16b_decode_every_token():
+    """The 16B decode layer (T = 32, the FP8 decode FFN) on every token."""
+    shape = W.CONFIGS["16b_decode"]
+    host, dev = H.device_inputs(shape)
+    ref = H.oracle_routing(shape, host)
+    rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
+    res = _check(shape, host, dev, rows, ref)
+    print(f"16b_decode fp8: compared rows {rows.size}, "
+          + ", ".join(f"{k}: max err {v[0]:.2e} rms err {v[2]:.2e} rms {v[1]:.2e}"
+                      for k, v in res.items() if k != "exempt"))
+
+
+def test_fp8_decode_ffn_is_deterministic():
+    shape = SHAPES["decode"]
+    host, dev = H.device_inputs(shape)
+    layer = _layer(shape, dev)
+    outs = [layer.forward_fp8(dev["x"], shape.K).clone() for _ in range(3)]
+    assert all(torch.equal(outs[0].view(torch.int16), o.view(torch.int16)) for o in outs[1:])
+    assert layer.status() == B.MOE_OK
 
 
 def test_fp8_layer_is_deterministic_and_close_to_the_bf16_layer():
