@@ -514,8 +514,8 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
 
 
 def fused_decode(shape: W.LayerShape, fp8: bool = False) -> bool:
-    """Whether the bf16 layer runs both expert GEMMs in one launch (the decode FFN)."""
-    return not fp8 and shape.T <= DECODE_MAX_T
+    """Whether the layer (bf16 or FP8) runs both expert GEMMs in one launch (the decode FFN)."""
+    return shape.T <= DECODE_MAX_T
 
 
 def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffic=None, fp8: bool = False):
@@ -547,8 +547,8 @@ def roofline_of(shape: W.LayerShape, r: dict, peaks: dict, peak_src: str, traffi
                 "peak_source": f"{peak_src} hbm_gbs"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     if fused:
-        kname = ("decode_ffn_kernel (shared and routed experts: gate/up GEMM + SwiGLU and down GEMM + gate "
-                 "scale, one launch)")
+        kname = (("decode_ffn8_kernel" if fp8 else "decode_ffn_kernel") +
+                 " (shared and routed experts: gate/up GEMM + SwiGLU and down GEMM + gate scale, one launch)")
     else:
         kname = ("fp8_gemm_kernel<true>" if fp8 else "gateup_gemm_kernel") + \
             " (shared and routed experts: gate/up GEMM + SwiGLU)"

@@ -258,37 +258,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           f.nkb = a.kb_dn;
         }
       }
-      if (lane == 0) {
-        if (!mbar_wait(&item_empty[it], it_ph ^ 1u, a.timeout_ns, abort_flag)) {
-          ffn_record_error(a.err, abort_flag, 1);
-          stop = true;
-        } else {
-          items[it] = f;
-          mbar_arrive(&item_full[it]);
-          if (++it == kFfnItems) {
-            it = 0;
-            it_ph ^= 1u;
-          }
-        }
-        if (f.kind < 0) stop = true;
-        if (!stop && (f.kind == 2 || f.kind == 3)) {
-          // the down tile's rows of H and their scales: wait for every gate/up tile of its token block
-          const uint32_t target = 4u * static_cast<uint32_t>(f.kind == 2 ? a.sh_n_wb_gu : a.n_wb_gu);
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_u32(ready + f.ready) < target) {
-            if (*abort_flag || globaltimer_ns() - t0 > a.timeout_ns) {
-              ffn_record_error(a.err, abort_flag, 2);
-              stop = true;
-              break;
-            }
-            __nanosleep(64);
-          }
-          fence_proxy_async_global();
-        }
-      }
-      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
-      if (stop) break;
-      __syncwarp();  // lane 0's acquire of the readiness counter orders the other lanes' loads of H's scales too
+      // the tile's scales go out before the item is published and the readiness wait, in one round trip
       // the tile's weight block scales, loaded once: lane l holds groups l and l + 32 (at most 64)
       uint32_t sc0[2] = {127u, 127u}, sc1[2] = {127u, 127u};
       {
@@ -323,6 +293,49 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
                              sf_atom_offset((f.row0 & 127) + lane);
       uint32_t cells[16];
       int cells_k0 = -16;
+      auto load_cells = [&](int k0) {  // the cells of groups k0 .. k0 + 15, one round trip
+        cells_k0 = k0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          cells[i] = k0 + i < f.nkb
+                         ? __ldcg(reinterpret_cast<const unsigned int*>(cell0 + static_cast<size_t>(k0 + i) *
+                                                                                    kSfAtomBytes))
+                         : 0u;
+      };
+      // the activation rows' scales are complete (the grid dependency wait); H's only after its readiness
+      if (f.kind >= 0 && f.kind < 2) load_cells(0);
+      if (lane == 0) {
+        if (!mbar_wait(&item_empty[it], it_ph ^ 1u, a.timeout_ns, abort_flag)) {
+          ffn_record_error(a.err, abort_flag, 1);
+          stop = true;
+        } else {
+          items[it] = f;
+          mbar_arrive(&item_full[it]);
+          if (++it == kFfnItems) {
+            it = 0;
+            it_ph ^= 1u;
+          }
+        }
+        if (f.kind < 0) stop = true;
+        if (!stop && (f.kind == 2 || f.kind == 3)) {
+          // the down tile's rows of H and their scales: wait for every gate/up tile of its token block
+          const uint32_t target = 4u * static_cast<uint32_t>(f.kind == 2 ? a.sh_n_wb_gu : a.n_wb_gu);
+          const uint64_t t0 = globaltimer_ns();
+          while (ld_acquire_u32(ready + f.ready) < target) {
+            if (*abort_flag || globaltimer_ns() - t0 > a.timeout_ns) {
+              ffn_record_error(a.err, abort_flag, 2);
+              stop = true;
+              break;
+            }
+            __nanosleep(64);
+          }
+          fence_proxy_async_global();
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+      if (stop) break;
+      __syncwarp();  // lane 0's acquire of the readiness counter orders the other lanes' loads of H's scales too
+      if (f.kind >= 2) load_cells(0);
       // stream the tile's groups: one per gate/up stage, two per down stage
       const int per = f.kind >= 2 ? 2 : 1;
       const int wrow = f.wb * kFfnWB;
@@ -365,15 +378,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         // the tokens' scales: lane n's cell at row n, column 0 of the tokens' atom
         for (int h = 0; h < n; ++h) {
           const int k = kb + h;
-          if (k >= cells_k0 + 16) {  // the next 16 groups' cells, one round trip
-            cells_k0 = k & ~15;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              cells[i] = cells_k0 + i < f.nkb
-                             ? __ldcg(reinterpret_cast<const unsigned int*>(cell0 + static_cast<size_t>(cells_k0 + i) *
-                                                                                        kSfAtomBytes))
-                             : 0u;
-          }
+          if (k >= cells_k0 + 16) load_cells(k & ~15);  // the next 16 groups' cells
           const uint32_t cell = cells[k - cells_k0];
           const uint32_t b0 = __shfl_sync(0xffffffffu, k < 32 ? sc0[0] : sc0[1], k & 31);
           const uint32_t w0 = 0x01010101u * b0;

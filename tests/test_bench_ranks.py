@@ -129,6 +129,13 @@ def test_roofline_of_the_dominant_kernel_from_its_own_numbers():
     f = bench.hbm_fractions(decode, r, peaks)
     assert f["ffn_gbs"] == pytest.approx(wbytes / 0.11e-3 / 1e9) and "down_gbs" not in f
     assert f["layer_frac"] == pytest.approx(wbytes / 0.13e-3 / 1e9 / 6500.0)
-    # the FP8 layer keeps separate GEMM launches at every batch size
-    f8 = bench.hbm_fractions(decode, dict(r, kernel_ms={"gate_up": 0.05, "down": 0.03}), peaks, fp8=True)
-    assert f8["down_gbs"] is not None and "ffn_gbs" not in f8
+    # the FP8 layer's decode batches too run both GEMMs in one launch, over 1-byte weights and their scales
+    f8 = bench.hbm_fractions(decode, dict(r, kernel_ms={"gate_up": 0.07, "down": 0.0}), peaks, fp8=True)
+    b8 = 3 * (1.0 + 1.0 / (128 * 128)) * 2048 * (30 * 1408 + 2 * 1408)
+    assert f8["ffn_gbs"] == pytest.approx(b8 / 0.07e-3 / 1e9) and "down_gbs" not in f8
+    roof8, _, _ = bench.roofline_of(decode, dict(r, dominant_ms=0.07), peaks, "measured", fp8=True)
+    assert roof8["bound"] == "hbm" and "decode_ffn8_kernel" in roof8["kernel"]
+    # a prefill batch keeps separate GEMM launches
+    f16 = bench.hbm_fractions(W.CONFIGS["v3"], dict(r, kernel_ms={"gate_up": 3.6, "down": 2.0},
+                                                      counts=[128] * 256), peaks)
+    assert f16["down_gbs"] is not None and "ffn_gbs" not in f16
