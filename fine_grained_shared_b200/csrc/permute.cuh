@@ -447,30 +447,31 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a, int cols_pe
   int slots[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) slots[k] = k < K ? a.slot_of[static_cast<size_t>(t) * a.K + k] : 0;
+  // every operand in its own register (an array filled at a running index lived in local memory)
+  auto add8 = [](float (&acc)[8], const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[2 * j] += bf16lo(w[j]);
+      acc[2 * j + 1] += bf16hi(w[j]);
+    }
+  };
   for (int col = c0 + lane * 8; col < c1; col += 256) {
-    uint4 v[10];
-    int nv = 0;
-    if (a.add_residual) v[nv++] = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + col));
-    if (a.ys) v[nv++] = __ldcg(reinterpret_cast<const uint4*>(a.ys + static_cast<size_t>(t) * a.d + col));
-    const int base = nv;
+    const size_t xo = static_cast<size_t>(t) * a.d + col;
+    uint4 vx = make_uint4(0u, 0u, 0u, 0u), vs = vx, vy[8];
+    if (a.add_residual) vx = __ldg(reinterpret_cast<const uint4*>(a.x + xo));
+    if (a.ys) vs = __ldcg(reinterpret_cast<const uint4*>(a.ys + xo));
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      if (k < K) v[base + k] = __ldcg(reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(slots[k]) * a.d + col));
-    nv = base + K;
+      vy[k] = k < K ? __ldcg(reinterpret_cast<const uint4*>(a.y + static_cast<size_t>(slots[k]) * a.d + col)) : vx;
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    if (a.add_residual) add8(acc, vx);
+    if (a.ys) add8(acc, vs);
 #pragma unroll
-    for (int i = 0; i < 10; ++i) {
-      if (i < nv) {
-        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[2 * j] += bf16lo(w[j]);
-          acc[2 * j + 1] += bf16hi(w[j]);
-        }
-      }
-    }
+    for (int k = 0; k < 8; ++k)
+      if (k < K) add8(acc, vy[k]);
     uint4 o;
     o.x = pack_bf16x2(acc[0], acc[1]);
     o.y = pack_bf16x2(acc[2], acc[3]);
