@@ -530,10 +530,11 @@ PermuteArgs permute_args(moe_ctx* h, const void* x, int64_t T, int32_t K, const 
   pa.K = K;
   pa.N = h->cfg.n_routed;
   pa.d = h->cfg.d_model;
-  const int split = (2 * h->num_sms + nblk - 1) / nblk;
-  // CTAs per 128-token block for the row copies: about two per SM in all, at most 8, or 32 for
-  // batches of up to 4 blocks (a 32-token decode batch copies one token row per CTA: 16B decode
-  // permutation 10.2 -> 8.6 us; more than 8 measured slower on the V3 layer, T = 4096)
+  const int split = (4 * h->num_sms + nblk - 1) / nblk;
+  // CTAs per 128-token block for the row copies: about four per SM in all (16B prefill, T = 16384:
+  // 0.110 -> 0.100 ms against two), at most 8, or 32 for batches of up to 4 blocks (a 32-token decode
+  // batch copies one token row per CTA: 16B decode permutation 10.2 -> 8.6 us; more than 8 measured
+  // slower on the V3 layer, T = 4096)
   const int max_split = nblk <= 4 ? 32 : 8;
   pa.split = split < 1 ? 1 : split > max_split ? max_split : split;
   pa.idx = ra.idx;
