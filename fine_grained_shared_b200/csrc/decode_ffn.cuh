@@ -78,7 +78,7 @@ struct FfnItem {
 
 __host__ __device__ constexpr size_t ffn_smem_bytes() {
   return 1024 + static_cast<size_t>(kFfnStages) * kFfnStage +
-         8 * (2 * kFfnStages + 2 * kFfnAccBufs + 2 * kFfnItems + 1) + 16 + sizeof(FfnItem) * kFfnItems +
+         8 * (2 * kFfnStages + 2 * kFfnAccBufs + 2 * kFfnItems + 2) + 16 + sizeof(FfnItem) * kFfnItems +
          4 * (3 * (kFfnMaxExperts + 8));
 }
 static_assert(ffn_smem_bytes() <= 232448, "shared memory");
@@ -105,11 +105,26 @@ struct FfnArgs {
   uint32_t* ctr;               // ffn_counter_bytes(), zero between launches
   uint32_t* err;
   uint64_t timeout_ns;
+  int debug_wait;              // test only: CTA 0's MMA lane waits 20 ms on a barrier nothing arrives on
 };
 
 __device__ __forceinline__ void ffn_record_error(uint32_t* err, volatile int* abort, uint32_t site) {
   *abort = 1;
   atomicOr(err, kErrTimeout | (1u << (kErrSiteShift + site)));
+}
+
+// Waits (bounded) until the readiness counter reaches target; gives up early once any CTA of the launch
+// has recorded an error (the tiles it waits for may belong to a CTA that stopped).
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p);
+__device__ __forceinline__ bool ffn_wait_ready(const uint32_t* ctr, uint32_t target, const uint32_t* err,
+                                               volatile int* abort, uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_u32(ctr) < target) {
+    if (*abort || *reinterpret_cast<const volatile uint32_t*>(err) != 0u || globaltimer_ns() - t0 > timeout_ns)
+      return false;
+    __nanosleep(64);
+  }
+  return true;
 }
 
 __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
@@ -156,7 +171,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   uint64_t* item_full = acc_empty + kFfnAccBufs;  // [kFfnItems]
   uint64_t* item_empty = item_full + kFfnItems;   // [kFfnItems]
   uint64_t* teardown = item_empty + kFfnItems;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* never = teardown + 1;  // test only: a barrier nothing arrives on
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   FfnItem* items = reinterpret_cast<FfnItem*>(tmem_slot + 4);
   int32_t* s_tbs = reinterpret_cast<int32_t*>(items + kFfnItems);  // [G + 1] prefix of 32-token blocks
@@ -178,6 +194,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       mbar_init(&item_empty[i], 5);  // the MMA lane and the four epilogue warps
     }
     mbar_init(teardown, 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -326,14 +343,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         if (!stop && f.kind >= 2) {
           // the down tile's rows of H: wait for every gate/up tile of its token block
           const uint32_t target = 4u * static_cast<uint32_t>(f.kind == 2 ? a.sh_n_wb_gu : a.n_wb_gu);
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_u32(ready + f.ready) < target) {
-            if (*abort_flag || globaltimer_ns() - t0 > a.timeout_ns) {
-              ffn_record_error(a.err, abort_flag, 2);
-              stop = true;
-              break;
-            }
-            __nanosleep(64);
+          if (!ffn_wait_ready(ready + f.ready, target, a.err, abort_flag, a.timeout_ns)) {
+            ffn_record_error(a.err, abort_flag, 2);
+            stop = true;
           }
           fence_proxy_async_global();
         }
@@ -393,7 +405,12 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     const uint32_t idesc = idesc_bf16_f32(kFfnWB, kFfnTB);
     int s = 0, buf = 0, it = 0;
     uint32_t ph = 0, buf_ph = 0, it_ph = 0;
-    while (true) {
+    bool stop = false;
+    if (a.debug_wait && blockIdx.x == 0 && !mbar_wait(never, 0, 20ull * 1000 * 1000, abort_flag)) {
+      ffn_record_error(a.err, abort_flag, 10);
+      stop = true;
+    }
+    while (!stop) {
       if (!mbar_wait(&item_full[it], it_ph, a.timeout_ns, abort_flag)) {
         ffn_record_error(a.err, abort_flag, 4);
         break;

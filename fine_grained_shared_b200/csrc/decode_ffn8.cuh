@@ -56,7 +56,7 @@ constexpr uint32_t kF8dTmemCols = 512;
 
 __host__ __device__ constexpr size_t ffn8_smem_bytes() {
   return 1024 + static_cast<size_t>(kF8dStages) * kF8dStage +
-         8 * (2 * kF8dStages + 2 * kF8dAccBufs + 2 * kFfnItems + 1) + 16 + sizeof(FfnItem) * kFfnItems +
+         8 * (2 * kF8dStages + 2 * kF8dAccBufs + 2 * kFfnItems + 2) + 16 + sizeof(FfnItem) * kFfnItems +
          4 * (3 * (kFfnMaxExperts + 8)) + 8 * 64 + 16;
 }
 static_assert(ffn8_smem_bytes() <= 232448, "shared memory");
@@ -102,7 +102,8 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   uint64_t* item_full = acc_empty + kF8dAccBufs;  // [kFfnItems]
   uint64_t* item_empty = item_full + kFfnItems;   // [kFfnItems]
   uint64_t* teardown = item_empty + kFfnItems;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* never = teardown + 1;  // test only: a barrier nothing arrives on
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   FfnItem* items = reinterpret_cast<FfnItem*>(tmem_slot + 4);
   int32_t* s_tbs = reinterpret_cast<int32_t*>(items + kFfnItems);
@@ -127,6 +128,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
       mbar_init(&item_empty[i], 5);
     }
     mbar_init(teardown, 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     for (int i = 0; i < 64; ++i) s_amax[i] = 0ull;
     s_arrive[0] = s_arrive[1] = 0u;
@@ -320,14 +322,9 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
         if (!stop && (f.kind == 2 || f.kind == 3)) {
           // the down tile's rows of H and their scales: wait for every gate/up tile of its token block
           const uint32_t target = 4u * static_cast<uint32_t>(f.kind == 2 ? a.sh_n_wb_gu : a.n_wb_gu);
-          const uint64_t t0 = globaltimer_ns();
-          while (ld_acquire_u32(ready + f.ready) < target) {
-            if (*abort_flag || globaltimer_ns() - t0 > a.timeout_ns) {
-              ffn_record_error(a.err, abort_flag, 2);
-              stop = true;
-              break;
-            }
-            __nanosleep(64);
+          if (!ffn_wait_ready(ready + f.ready, target, a.err, abort_flag, a.timeout_ns)) {
+            ffn_record_error(a.err, abort_flag, 2);
+            stop = true;
           }
           fence_proxy_async_global();
         }
@@ -416,7 +413,12 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     const uint32_t idesc = idesc_mxf8_e4m3(kFfnWB, kFfnTB);
     int s = 0, buf = 0, it = 0;
     uint32_t ph = 0, buf_ph = 0, it_ph = 0;
-    while (true) {
+    bool stop = false;
+    if (a.debug_wait && blockIdx.x == 0 && !mbar_wait(never, 0, 20ull * 1000 * 1000, abort_flag)) {
+      ffn_record_error(a.err, abort_flag, 10);
+      stop = true;
+    }
+    while (!stop) {
       if (!mbar_wait(&item_full[it], it_ph, a.timeout_ns, abort_flag)) {
         ffn_record_error(a.err, abort_flag, 4);
         break;

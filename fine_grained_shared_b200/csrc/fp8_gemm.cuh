@@ -66,7 +66,7 @@ constexpr uint32_t kF8BoxRowsW = 128;                  // W_gate / W_up boxes; W
 constexpr uint32_t kF8BoxRowsWd = 256;
 
 __host__ __device__ constexpr size_t fp8_gemm_smem_bytes() {
-  return 1024 + static_cast<size_t>(kF8Stages) * kF8Stage + 8 * (2 * kF8Stages + 2 + 1) + 16 +
+  return 1024 + static_cast<size_t>(kF8Stages) * kF8Stage + 8 * (2 * kF8Stages + 2 + 2) + 16 +
          4 * (2 * 264) + 4 * 2 * 2 * 128 + 4 * 2 * 4 * 2;
 }
 static_assert(fp8_gemm_smem_bytes() <= 232448, "shared memory");
@@ -208,6 +208,7 @@ struct Fp8GemmArgs {
   int sh_ld_out, sh_n_limit;
   uint32_t* err;
   uint64_t timeout_ns;
+  int debug_wait;              // test only: CTA 0 waits 20 ms on a barrier nothing arrives on
 };
 
 struct F8Tile {
@@ -272,7 +273,8 @@ __global__ void __launch_bounds__(kF8Threads, 1)
   uint64_t* acc_full = empty + kF8Stages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* teardown = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(teardown + 1);
+  uint64_t* never = teardown + 1;  // test only: a barrier nothing arrives on
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_mts = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [264]
   int32_t* s_rows = s_mts + 264;
@@ -291,6 +293,7 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 8);  // one arrive per epilogue warp
     mbar_init(teardown, 1);
+    mbar_init(never, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -422,6 +425,10 @@ __global__ void __launch_bounds__(kF8Threads, 1)
     int s = 0, slot = 0;
     uint32_t ph = 0, acc_ph = 0;
     bool stop = false;
+    if (a.debug_wait && blockIdx.x == 0 && !mbar_wait(never, 0, 20ull * 1000 * 1000, abort_flag)) {
+      f8_record_error(a.err, abort_flag, 10);
+      stop = true;
+    }
     for (int tile = blockIdx.x; tile < total_tiles && !stop; tile += gridDim.x) {
       const int kgs = tile < sh_tiles ? a.sh_J * a.sh_kg_per_j : a.num_kg;
       if (!mbar_wait(acc_empty, acc_ph ^ 1u, a.timeout_ns, abort_flag)) {

@@ -779,6 +779,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
     f.ctr = h->at<uint32_t>(L.ffn_ctr);
     f.err = h->at<uint32_t>(L.err);
     f.timeout_ns = kTimeoutNs;
+    f.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
     // an absent part's maps are never read; the present part's stand in
     const CUtensorMap& Wg = do_routed ? h->tm_wg.map : h->tm_swg.map;
     const CUtensorMap& Wu = do_routed ? h->tm_wu.map : h->tm_swu.map;
@@ -982,6 +983,7 @@ moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_rou
     f.ctr = h->at<uint32_t>(L.ffn_ctr);
     f.err = h->at<uint32_t>(L.err);
     f.timeout_ns = kTimeoutNs;
+    f.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
     f8.x_atoms = h->at<uint8_t>(L.xs_perm);
     f8.xs_atoms = h->at<uint8_t>(L.xs);
     f8.hq = h->at<uint8_t>(L.hq);
@@ -1060,6 +1062,7 @@ moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_rou
     }
     g.err = h->at<uint32_t>(L.err);
     g.timeout_ns = kTimeoutNs;
+    g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
     const int sh_tiles = do_shared ? ceil_div(T, kF8BM) * g.sh_n_tiles : 0;
     const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
     {

@@ -122,6 +122,26 @@ def test_fp8_decode_ffn_is_deterministic():
     assert layer.status() == B.MOE_OK
 
 
+@pytest.mark.parametrize("name", ["small", "decode_t40"])
+def test_fp8_device_wait_timeout_is_reported_and_the_context_stays_usable(name):
+    """A bounded wait that runs out in the FP8 gate/up GEMM (prefill) or the FP8 decode FFN: the call
+    reports MOE_ERR_TIMEOUT and a later forward gives the same bits as one taken before it."""
+    shape = SHAPES[name]
+    host, dev = H.device_inputs(shape)
+    good = _layer(shape, dev)
+    before = good.forward_fp8(dev["x"], shape.K).clone()
+    assert good.status() == B.MOE_OK
+    bad = _layer(shape, dev, B.MOE_FLAG_DEBUG_WAIT_TIMEOUT)
+    for _ in range(2):
+        bad.forward_fp8(dev["x"], shape.K)
+        assert bad.status() == B.MOE_ERR_TIMEOUT
+        assert bad.status() == B.MOE_OK
+    bad.close()
+    after = good.forward_fp8(dev["x"], shape.K)
+    assert good.status() == B.MOE_OK
+    assert torch.equal(before.view(torch.int16), after.view(torch.int16))
+
+
 def test_fp8_layer_is_deterministic_and_close_to_the_bf16_layer():
     shape = SHAPES["small"]
     host, dev = H.device_inputs(shape)

@@ -389,20 +389,28 @@ def test_bad_arguments_are_rejected_before_launch():
     H.run(layer, x, shape.K)
 
 
-def test_device_wait_timeout_is_reported_and_the_context_stays_usable():
+@pytest.mark.parametrize("tokens", [None, 32], ids=["grouped_gemms", "decode_ffn"])
+def test_device_wait_timeout_is_reported_and_the_context_stays_usable(tokens):
+    """A bounded wait that runs out (a barrier nothing arrives on) in the grouped GEMMs of a prefill batch,
+    or in the decode FFN of a batch of 32 tokens: the call reports MOE_ERR_TIMEOUT, every other CTA stops
+    within its own limit, and the next forward on the same handle and on a new one is correct."""
     shape = W.CONFIGS["tiny"]
     host, dev = H.device_inputs(shape)
+    x = dev["x"] if tokens is None else dev["x"][:tokens]
     bad = H.make_layer(shape, dev, flags=B.MOE_FLAG_DEBUG_WAIT_TIMEOUT)
-    bad.forward(dev["x"], shape.K)
-    assert bad.status() == B.MOE_ERR_TIMEOUT
-    assert bad.status() == B.MOE_OK          # the error word is cleared once reported
+    for _ in range(2):                       # the handle's counters are left usable after the error
+        bad.forward(x, shape.K)
+        assert bad.status() == B.MOE_ERR_TIMEOUT
+        assert bad.status() == B.MOE_OK      # the error word is cleared once reported
     bad.close()
     good = H.make_layer(shape, dev)
-    out = H.run(good, dev["x"], shape.K)
     ref = H.oracle_routing(shape, host)
     h, _ = O.moe_forward(host["x"], host["router"], shape.K, H.oracle_experts(shape, host),
                          H.oracle_shared(shape, host), routing=ref)
     rows = np.nonzero(ref.gap >= H.GAP_EXEMPT)[0]
+    if tokens is not None:
+        rows = rows[rows < tokens]
+    out = H.run(good, x, shape.K)
     H.compare_output(_gpu_rows(out, rows), h[rows], "after a timeout")
 
 
