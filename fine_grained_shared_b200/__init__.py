@@ -11,5 +11,6 @@ from .moe import (  # noqa: F401
     MOE_FLAG_NO_ROUTED, MOE_FLAG_NO_SHARED, MOE_GATE_SIGMOID_BIASED, MOE_GATE_SOFTMAX, MOE_OK,
     MoEError, MoELayer, lib, moe_config, moe_create, moe_destroy, moe_experts, moe_forward,
     moe_forward_host, moe_get_routing, moe_router, moe_shared, moe_status_query, moe_workspace_bytes, moe_set_timing, moe_kernel_times, moe_update_bias, KERNEL_NAMES,
-    status_string,
+    status_string, ExpertParallelLayer, connect_emulated, connect_ipc, forward_emulated, nccl_barrier,
+    moe_ep_plan,
 )

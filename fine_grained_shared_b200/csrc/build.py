@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 LIB = os.path.join(PKG, "libfgs_moe.so")
 SOURCES = ["moe_api.cu", "route_noalloc.cu", "fp8_quant.cu"]
 HEADERS = ["sm100.cuh", "router_topk.cuh", "permute.cuh", "gateup_gemm.cuh", "down_gemm.cuh", "decode_ffn.cuh",
-           "fp8_util.cuh", "fp8_gemm.cuh", "decode_ffn8.cuh"]
+           "fp8_util.cuh", "fp8_gemm.cuh", "decode_ffn8.cuh", "ep_plan.h", "ep.cuh"]
 
 
 def nvcc_path() -> str:

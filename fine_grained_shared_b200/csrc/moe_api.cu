@@ -30,6 +30,7 @@
 #include "decode_ffn.cuh"
 #include "decode_ffn8.cuh"
 #include "down_gemm.cuh"
+#include "ep.cuh"
 #include "fp8_gemm.cuh"
 #include "gateup_gemm.cuh"
 #include "permute.cuh"
@@ -114,7 +115,7 @@ struct Layout {
   // byte offsets into the workspace
   size_t err, done, tile_ctr, tok_done, small_logits, idx, gate, slot, src, bc, counts, offsets, row_start, mtile,
       mtile128, gate_perm, x_perm, h, y, hs, ys, xdev, outdev, ffn_ctr, xq_perm, xs_perm, xq, xs, hq, hs_perm, hsq,
-      hss, total;
+      hss, ep_base, ep_counts, ep_row_start, ep_mtile, ep_mtile128, total;
   int64_t P, Pa, Tpad, nblk;
 };
 
@@ -130,8 +131,10 @@ Layout make_layout(const moe_config& c) {
   Layout L{};
   const int64_t Tm = c.max_tokens, Km = c.max_k, N = c.n_routed;
   L.nblk = ceil_div(Tm, 128);
-  // sum over experts of ceil(count / 256) * 256 <= T*K + 255*N
-  L.P = Tm * Km + N * (kExpertRowAlign - 1);
+  // sum over experts of ceil(count / 256) * 256 <= T*K + 255*N; an expert-parallel rank holds N / G
+  // experts and may receive every rank's T*K rows
+  const int64_t G = c.ep_ranks > 1 ? c.ep_ranks : 1;
+  L.P = G * Tm * Km + (N / G) * (kExpertRowAlign - 1);
   L.Tpad = int64_t(ceil_div(Tm, kGemmBM)) * kGemmBM;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -151,6 +154,12 @@ Layout make_layout(const moe_config& c) {
   L.bc = take(L.nblk * N * 4);
   L.counts = take(N * 4);
   L.offsets = take((N + 1) * 4);
+  // expert parallelism: this rank's destination rows per expert, its own experts' tables
+  L.ep_base = take(N * 4);
+  L.ep_counts = take((N + 1) * 4);
+  L.ep_row_start = take((N + 1) * 4);
+  L.ep_mtile = take((N + 1) * 4);
+  L.ep_mtile128 = take((N + 1) * 4);
   L.row_start = take((N + 1) * 4);
   L.mtile = take((N + 1) * 4);
   L.mtile128 = take((N + 1) * 4);
@@ -200,6 +209,13 @@ moe_status check_config(const moe_config* c) {
     return MOE_ERR_ALIGNMENT;
   if ((c->flags & MOE_FLAG_FP8) && (c->d_model > 8192 || c->d_ff > 8192 || c->d_ff_shared > 8192))
     return MOE_ERR_SHAPE;  // at most 64 scale groups along a GEMM's K
+  if (c->ep_ranks > 1) {
+    if (c->ep_ranks > kEpMaxRanks || c->n_routed % c->ep_ranks || c->ep_rank < 0 || c->ep_rank >= c->ep_ranks)
+      return MOE_ERR_INVALID_ARG;
+    if (c->flags & MOE_FLAG_FP8) return MOE_ERR_UNSUPPORTED;
+  } else if (c->ep_ranks < 0 || c->ep_rank != 0) {
+    return MOE_ERR_INVALID_ARG;
+  }
   if (c->route_nodes != 0 || c->route_max_nodes != 0) {
     if (c->route_nodes < 1 || c->route_nodes > kMaxRouteNodes || c->n_routed % c->route_nodes ||
         c->route_max_nodes < 1 || c->route_max_nodes > c->route_nodes ||
@@ -257,6 +273,15 @@ struct moe_ctx {
   uint32_t timing_mask = 0;  // bit k: time kernel k
   std::vector<cudaEvent_t> ev_pool[MOE_KERNEL_COUNT];
   size_t ev_used[MOE_KERNEL_COUNT] = {};
+  // expert parallelism: the ranks' workspaces, which of them this handle opened, the
+  // forward's tokens and its step (1 routed, 2 dispatched, 3 experts done, 4 combined)
+  EpPeers peers{};
+  bool peers_set = false;
+  bool ipc_opened[kEpMaxRanks] = {};
+  const void* ep_x = nullptr;
+  int64_t ep_T = 0;
+  int ep_K = 0;
+  int ep_stage = 0;
 
   template <typename T>
   T* at(size_t off) const {
@@ -570,6 +595,92 @@ moe_status launch_combine(moe_ctx* h, const CombineArgs& ca, int64_t T, int64_t 
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// The routed experts' tables of the grouped GEMMs (device pointers; G = 0: no routed tiles).
+struct ExpertTables {
+  int G;                     // routed experts (groups of the row buffer)
+  const int32_t* mtile128;   // [G + 1] prefix of ceil(rows / 128): the gate/up GEMM's m-tiles
+  const int32_t* mtile;      // [G + 1] prefix of ceil(rows / 256): the down GEMM's pair tiles
+  const int32_t* row_start;  // [G + 1] first row of each expert in X_perm, H and Y
+  const float* row_scale;    // the gate of each row
+};
+
+// The expert GEMMs of a batch above the decode size, on the weight maps of the
+// handle: gate/up + SwiGLU, then down + gate scale, each one persistent launch
+// with the shared experts' tiles (the T rows of x) first and then the routed
+// experts' (tables on the device).
+moe_status enqueue_expert_gemms(moe_ctx* h, int64_t T, bool do_shared, const ExpertTables& et, int* tile_ctr,
+                                cudaStream_t s0, bool pdl) {
+  const moe_config& c = h->cfg;
+  const Layout& L = h->L;
+  const int64_t d = c.d_model, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const bool do_routed = et.G > 0;
+  const int num_kb = ceil_div(d, kGuBK);
+  GateUpArgs g{};
+  if (do_routed) {
+    g.num_groups = et.G;
+    g.mtile_start = et.mtile128;
+    g.row_start = et.row_start;
+    g.n_tiles = ceil_div(I, kGuBN / 2);
+    g.n_limit = (int)I;
+    g.out = h->at<__nv_bfloat16>(L.h);
+    g.ld_out = (int)I;
+  }
+  if (do_shared) {
+    g.sh_rows = (int)T;
+    g.sh_n_tiles = ceil_div(Ks * Is, kGuBN / 2);
+    g.sh_n_limit = (int)(Ks * Is);
+    g.sh_out = h->at<__nv_bfloat16>(L.hs);
+    g.sh_ld_out = (int)(Ks * Is);
+  }
+  g.num_kb = num_kb;
+  g.tile_ctr = tile_ctr;
+  g.die_split = h->num_sms / 2;
+  g.err = h->at<uint32_t>(L.err);
+  g.timeout_ns = kTimeoutNs;
+  g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
+  // with routed tiles the count is known only on the device: one CTA per SM
+  const int sh_tiles = do_shared ? ceil_div(T, kGuBM) * g.sh_n_tiles : 0;
+  const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
+  // an absent part's maps are never read; the present part's stand in
+  const CUtensorMap& sA = do_shared ? h->tm_x.map : h->tm_xperm;
+  const CUtensorMap& sG = do_shared ? h->tm_swg.map : h->tm_wg.map;
+  const CUtensorMap& sU = do_shared ? h->tm_swu.map : h->tm_wu.map;
+  {
+    KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+    if (launch_gateup(ctas, s0, pdl, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+
+  GemmArgs g2{};
+  if (do_routed) {
+    g2.num_groups = et.G;
+    g2.mtile_start = et.mtile;
+    g2.row_start = et.row_start;
+    g2.num_kb = ceil_div(I, kGemmBK);
+    g2.row_scale = et.row_scale;
+    g2.out = h->at<__nv_bfloat16>(L.y);
+  }
+  if (do_shared) {
+    g2.sh_rows = (int)T;
+    g2.sh_num_kb = ceil_div(Is, kGemmBK);
+    g2.sh_J = (int)Ks;
+    g2.sh_k_per_j = (int)Is;
+    g2.sh_out = h->at<__nv_bfloat16>(L.ys);
+  }
+  g2.n_tiles = ceil_div(d, kGemmBN);
+  g2.n_limit = (int)d;
+  g2.ld_out = (int)d;
+  g2.err = h->at<uint32_t>(L.err);
+  g2.timeout_ns = kTimeoutNs;
+  const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
+  const int pairs = do_routed || sh_tiles2 > h->max_pairs ? h->max_pairs : sh_tiles2;
+  const CUtensorMap& sA2 = do_shared ? h->tm_hs : h->tm_h;
+  const CUtensorMap& sB2 = do_shared ? h->tm_swd.map : h->tm_wd.map;
+  KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
+  if (launch_down(pairs, s0, pdl, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -681,6 +792,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
                        void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   const moe_config& c = h->cfg;
+  if (c.ep_ranks > 1) return MOE_ERR_UNSUPPORTED;
   if (T < 0 || T > c.max_tokens) return MOE_ERR_SHAPE;
   if (K < 1 || K > c.max_k || K > c.n_routed) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;  // nothing to enqueue (an empty tensor may carry a null pointer)
@@ -798,70 +910,10 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
 
   // ---- the expert GEMMs: shared experts' tiles first, then the routed experts' ----
   if (!decode && (do_routed || do_shared)) {
-    const int num_kb = ceil_div(d, kGuBK);
-    GateUpArgs g{};
-    if (do_routed) {
-      g.num_groups = (int)N;
-      g.mtile_start = ra.mtile128_start;
-      g.row_start = ra.row_start;
-      g.n_tiles = ceil_div(I, kGuBN / 2);
-      g.n_limit = (int)I;
-      g.out = h->at<__nv_bfloat16>(L.h);
-      g.ld_out = (int)I;
-    }
-    if (do_shared) {
-      g.sh_rows = (int)T;
-      g.sh_n_tiles = ceil_div(Ks * Is, kGuBN / 2);
-      g.sh_n_limit = (int)(Ks * Is);
-      g.sh_out = h->at<__nv_bfloat16>(L.hs);
-      g.sh_ld_out = (int)(Ks * Is);
-    }
-    g.num_kb = num_kb;
-    g.tile_ctr = pa.tile_ctr;
-    g.die_split = h->num_sms / 2;
-    g.err = h->at<uint32_t>(L.err);
-    g.timeout_ns = kTimeoutNs;
-    g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
-    // with routed tiles the count is known only on the device: one CTA per SM
-    const int sh_tiles = do_shared ? ceil_div(T, kGuBM) * g.sh_n_tiles : 0;
-    const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
-    // an absent part's maps are never read; the present part's stand in
-    const CUtensorMap& sA = do_shared ? h->tm_x.map : h->tm_xperm;
-    const CUtensorMap& sG = do_shared ? h->tm_swg.map : h->tm_wg.map;
-    const CUtensorMap& sU = do_shared ? h->tm_swu.map : h->tm_wu.map;
-    {
-      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
-      if (launch_gateup(ctas, s0, pdl, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-
-    GemmArgs g2{};
-    if (do_routed) {
-      g2.num_groups = (int)N;
-      g2.mtile_start = ra.mtile_start;
-      g2.row_start = ra.row_start;
-      g2.num_kb = ceil_div(I, kGemmBK);
-      g2.row_scale = pa.gate_perm;
-      g2.out = h->at<__nv_bfloat16>(L.y);
-    }
-    if (do_shared) {
-      g2.sh_rows = (int)T;
-      g2.sh_num_kb = ceil_div(Is, kGemmBK);
-      g2.sh_J = (int)Ks;
-      g2.sh_k_per_j = (int)Is;
-      g2.sh_out = h->at<__nv_bfloat16>(L.ys);
-    }
-    g2.n_tiles = ceil_div(d, kGemmBN);
-    g2.n_limit = (int)d;
-    g2.ld_out = (int)d;
-    g2.err = h->at<uint32_t>(L.err);
-    g2.timeout_ns = kTimeoutNs;
-    const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
-    const int pairs = do_routed || sh_tiles2 > h->max_pairs ? h->max_pairs : sh_tiles2;
-    const CUtensorMap& sA2 = do_shared ? h->tm_hs : h->tm_h;
-    const CUtensorMap& sB2 = do_shared ? h->tm_swd.map : h->tm_wd.map;
-    KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
-    if (launch_down(pairs, s0, pdl, h->tm_h, h->tm_wd.map, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
+    ExpertTables et{};
+    if (do_routed) et = ExpertTables{(int)N, ra.mtile128_start, ra.mtile_start, ra.row_start, pa.gate_perm};
+    const moe_status st = enqueue_expert_gemms(h, T, do_shared, et, pa.tile_ctr, s0, pdl);
+    if (st != MOE_OK) return st;
   }
 
   // ---- the final sum ----
@@ -1133,6 +1185,7 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
                             const moe_experts* experts, const moe_shared* shared, int32_t K, void* out_host,
                             void* stream) {
   if (!h || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (h->cfg.ep_ranks > 1) return MOE_ERR_UNSUPPORTED;
   if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_SHAPE;
   if (T == 0) return MOE_OK;
   DeviceGuard guard(h->device);
@@ -1208,6 +1261,259 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
       return finish(MOE_ERR_CUDA);
   }
   return finish(MOE_OK);
+}
+
+// ---------------------------------------------------------------------------
+// Expert parallelism: the four steps of a forward and the peers' workspaces
+// ---------------------------------------------------------------------------
+
+static_assert(sizeof(cudaIpcMemHandle_t) == 64, "the header promises 64-byte IPC handles");
+static_assert(kEpRowAlign == kExpertRowAlign, "the owner's row buffer has the single-GPU layout");
+
+moe_status moe_ep_workspace(moe_handle h, void** workspace) {
+  if (!h || !workspace || h->cfg.ep_ranks < 2) return MOE_ERR_INVALID_ARG;
+  *workspace = h->ws;
+  return MOE_OK;
+}
+
+moe_status moe_ep_set_peers(moe_handle h, void* const* workspaces) {
+  if (!h || !workspaces || h->cfg.ep_ranks < 2) return MOE_ERR_INVALID_ARG;
+  const int G = h->cfg.ep_ranks;
+  if (workspaces[h->cfg.ep_rank] != h->ws) return MOE_ERR_INVALID_ARG;
+  for (int r = 0; r < G; ++r)
+    if (!workspaces[r] || (reinterpret_cast<uintptr_t>(workspaces[r]) & 255u)) return MOE_ERR_INVALID_ARG;
+  for (int r = 0; r < G; ++r) h->peers.ws[r] = static_cast<uint8_t*>(workspaces[r]);
+  h->peers_set = true;
+  return MOE_OK;
+}
+
+moe_status moe_ep_ipc_handle(moe_handle h, void* handle) {
+  if (!h || !handle || h->cfg.ep_ranks < 2) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  cudaIpcMemHandle_t m;
+  if (cudaIpcGetMemHandle(&m, h->ws) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  std::memcpy(handle, &m, sizeof(m));
+  return MOE_OK;
+}
+
+namespace {
+void close_ipc_peers(moe_ctx* h) {
+  for (int r = 0; r < kEpMaxRanks; ++r) {
+    if (h->ipc_opened[r]) cudaIpcCloseMemHandle(h->peers.ws[r]);
+    h->ipc_opened[r] = false;
+  }
+  h->peers_set = false;
+}
+}  // namespace
+
+moe_status moe_ep_open_peers(moe_handle h, const void* handles) {
+  if (!h || !handles || h->cfg.ep_ranks < 2) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  close_ipc_peers(h);
+  const int G = h->cfg.ep_ranks, me = h->cfg.ep_rank;
+  for (int r = 0; r < G; ++r) {
+    if (r == me) {
+      h->peers.ws[r] = h->ws;
+      continue;
+    }
+    cudaIpcMemHandle_t m;
+    std::memcpy(&m, static_cast<const uint8_t*>(handles) + 64 * r, sizeof(m));
+    void* p = nullptr;
+    if (cudaIpcOpenMemHandle(&p, m, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+      cudaGetLastError();
+      close_ipc_peers(h);
+      return MOE_ERR_CUDA;
+    }
+    h->peers.ws[r] = static_cast<uint8_t*>(p);
+    h->ipc_opened[r] = true;
+  }
+  h->peers_set = true;
+  return MOE_OK;
+}
+
+moe_status moe_ep_route(moe_handle h, const void* x, int64_t T, const moe_router* router, int32_t K,
+                        void* stream) {
+  if (!h || h->cfg.ep_ranks < 2) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_SHAPE;
+  if (K < 1 || K > c.max_k || K > c.n_routed) return MOE_ERR_INVALID_ARG;
+  if (!router || !router->weight || (T > 0 && !x)) return MOE_ERR_INVALID_ARG;
+  const bool sigmoid = c.gate == MOE_GATE_SIGMOID_BIASED;
+  if (sigmoid ? router->logit_bias != nullptr : router->select_bias != nullptr) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x, router->weight, static_cast<const void*>(router->logit_bias),
+                        static_cast<const void*>(router->select_bias)})
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  h->ep_stage = 0;
+  h->ep_x = x;
+  h->ep_T = T;
+  h->ep_K = K;
+  if (T == 0) {
+    // no tokens: counts of zero for the other ranks' plans
+    h->last_stream = s0;
+    h->last_T = 0;
+    h->last_K = K;
+    if (cudaMemsetAsync(h->ws + h->L.counts, 0, size_t(c.n_routed) * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
+  } else {
+    RouterArgs ra;
+    const moe_status st = enqueue_router(h, x, T, router, K, s0, false, ra, 0);
+    if (st != MOE_OK) return st;
+  }
+  h->ep_stage = 1;
+  return MOE_OK;
+}
+
+moe_status moe_ep_dispatch(moe_handle h, void* stream) {
+  if (!h || h->cfg.ep_ranks < 2 || !h->peers_set || h->ep_stage != 1) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  const Layout& L = h->L;
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const int G = c.ep_ranks, N = c.n_routed;
+  const int64_t T = h->ep_T;
+  KernelTimer kt(h, MOE_KERNEL_PERMUTE, s0);
+  EpPlanArgs pa{};
+  pa.G = G;
+  pa.N = N;
+  pa.rank = c.ep_rank;
+  pa.counts_off = L.counts;
+  pa.peers = h->peers;
+  pa.base = h->at<int32_t>(L.ep_base);
+  pa.counts_loc = h->at<int32_t>(L.ep_counts);
+  pa.row_start = h->at<int32_t>(L.ep_row_start);
+  pa.mtile_start = h->at<int32_t>(L.ep_mtile);
+  pa.mtile128_start = h->at<int32_t>(L.ep_mtile128);
+  ep_plan_kernel<<<1, kEpPlanThreads, ep_plan_smem_bytes(G, N), s0>>>(pa);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (T > 0) {
+    const int nblk = ceil_div(T, 128);
+    const int split = std::max(1, std::min(nblk <= 4 ? 32 : 8, (4 * h->num_sms + nblk - 1) / nblk));
+    EpDispatchArgs da{};
+    da.T = (int)T;
+    da.K = h->ep_K;
+    da.N = N;
+    da.d = c.d_model;
+    da.split = split;
+    da.per_rank = N / G;
+    da.idx = h->at<int32_t>(L.idx);
+    da.gate = h->at<float>(L.gate);
+    da.block_base = h->at<int32_t>(L.bc);
+    da.offsets = h->at<int32_t>(L.offsets);
+    da.base = pa.base;
+    da.src = h->at<int32_t>(L.src);
+    da.slot_of = h->at<int32_t>(L.slot);
+    da.x = static_cast<const __nv_bfloat16*>(h->ep_x);
+    da.xperm_off = L.x_perm;
+    da.gate_off = L.gate_perm;
+    da.peers = h->peers;
+    da.tile_ctr = h->at<int>(L.tile_ctr);
+    ep_dispatch_kernel<<<dim3(nblk, split), kPermThreads, 0, s0>>>(da);
+  } else if (cudaMemsetAsync(h->ws + L.tile_ctr, 0, 8, s0) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  h->ep_stage = 2;
+  return MOE_OK;
+}
+
+moe_status moe_ep_experts(moe_handle h, const moe_experts* experts, const moe_shared* shared, void* stream) {
+  if (!h || h->cfg.ep_ranks < 2 || !h->peers_set || h->ep_stage != 2) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (!experts || !experts->w_gate || !experts->w_up || !experts->w_down) return MOE_ERR_INVALID_ARG;
+  if ((c.n_shared > 0) != (shared != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (shared && (!shared->w_gate || !shared->w_up || !shared->w_down)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {experts->w_gate, experts->w_up, experts->w_down, shared ? shared->w_gate : nullptr,
+                        shared ? shared->w_up : nullptr, shared ? shared->w_down : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  const int64_t d = c.d_model, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const int per = c.n_routed / c.ep_ranks;
+  const int64_t T = h->ep_T;
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const Layout& L = h->L;
+  const bool do_shared = Ks > 0 && !(c.flags & MOE_FLAG_NO_SHARED) && T > 0;
+  const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
+  bool ok = refresh(h->tm_wg, experts->w_gate, 0, per, I, d, kGuBoxRowsB, 3);
+  ok = ok && refresh(h->tm_wu, experts->w_up, 0, per, I, d, kGuBoxRowsB, 3);
+  ok = ok && refresh(h->tm_wd, experts->w_down, 0, per, d, I, kBoxRowsB, 3);
+  if (shared) {
+    ok = ok && refresh(h->tm_swg, shared->w_gate, 0, 1, Ks * Is, d, kGuBoxRowsB, 3);
+    ok = ok && refresh(h->tm_swu, shared->w_up, 0, 1, Ks * Is, d, kGuBoxRowsB, 3);
+    ok = ok && refresh(h->tm_swd, shared->w_down, 0, Ks, d, Is, kBoxRowsB, 3);
+  }
+  if (!ok) return MOE_ERR_CUDA;
+  if (do_routed || do_shared) {
+    ExpertTables et{};
+    if (do_routed)
+      et = ExpertTables{per, h->at<int32_t>(L.ep_mtile128), h->at<int32_t>(L.ep_mtile),
+                        h->at<int32_t>(L.ep_row_start), h->at<float>(L.gate_perm)};
+    const moe_status st = enqueue_expert_gemms(h, T, do_shared, et, h->at<int>(L.tile_ctr), s0, false);
+    if (st != MOE_OK) return st;
+  }
+  h->ep_stage = 3;
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine(moe_handle h, void* out, void* stream) {
+  if (!h || h->cfg.ep_ranks < 2 || !h->peers_set || h->ep_stage != 3) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  const int64_t T = h->ep_T, d = c.d_model;
+  if (T > 0 && !out) return MOE_ERR_INVALID_ARG;
+  if (out && !aligned16(out)) return MOE_ERR_ALIGNMENT;
+  if (overlaps(out, size_t(T) * d * 2, h->ep_x, size_t(T) * d * 2)) return MOE_ERR_INVALID_ARG;
+  h->ep_stage = 4;
+  if (T == 0) return MOE_OK;
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const Layout& L = h->L;
+  const bool do_shared = c.n_shared > 0 && !(c.flags & MOE_FLAG_NO_SHARED);
+  EpCombineArgs ca{};
+  ca.T = (int)T;
+  ca.K = h->ep_K;
+  ca.d = (int)d;
+  ca.per_rank = c.n_routed / c.ep_ranks;
+  ca.x = static_cast<const __nv_bfloat16*>(h->ep_x);
+  ca.ys = do_shared ? h->at<__nv_bfloat16>(L.ys) : nullptr;
+  ca.idx = h->at<int32_t>(L.idx);
+  ca.slot_of = h->at<int32_t>(L.slot);
+  ca.y_off = L.y;
+  ca.peers = h->peers;
+  ca.out = static_cast<__nv_bfloat16*>(out);
+  ca.add_residual = (c.flags & MOE_FLAG_NO_RESIDUAL) ? 0 : 1;
+  ca.add_routed = (c.flags & MOE_FLAG_NO_ROUTED) ? 0 : 1;
+  // the split of combine_kernel: whole rows per warp once the batch fills the SMs, shorter chunks below
+  const int64_t resident = int64_t(h->num_sms) * 64;
+  int cols = (int)d;
+  if (T < resident) {
+    const int chunks = ceil_div(2 * resident, T);
+    cols = ceil_div(ceil_div(d, chunks), 256) * 256;
+  }
+  const int64_t warps = T * ceil_div(d, cols);
+  KernelTimer kt(h, MOE_KERNEL_COMBINE, s0);
+  ep_combine_kernel<<<ceil_div(warps * 32, 256), 256, 0, s0>>>(ca, cols);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t G, int32_t n_routed, int32_t rank, int32_t* base,
+                       int32_t* counts_local, int32_t* row_start, int32_t* mtile_start, int32_t* mtile128_start) {
+  if (!counts_all || !base || !counts_local || !row_start || !mtile_start || !mtile128_start)
+    return MOE_ERR_INVALID_ARG;
+  if (G < 2 || G > kEpMaxRanks || n_routed < 1 || n_routed > kMaxRouted || n_routed % G || rank < 0 || rank >= G)
+    return MOE_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < int64_t(G) * n_routed; ++i)
+    if (counts_all[i] < 0) return MOE_ERR_INVALID_ARG;
+  const int32_t* rows[kEpMaxRanks];
+  for (int r = 0; r < G; ++r) rows[r] = counts_all + int64_t(r) * n_routed;
+  for (int e = 0; e < n_routed; ++e) base[e] = ep_dest_base(rows, G, n_routed, rank, e);
+  const int per = n_routed / G;
+  for (int l = 0; l <= per; ++l)
+    ep_owner_entry(rows, G, n_routed, rank, l, counts_local + l, row_start + l, mtile_start + l, mtile128_start + l);
+  return MOE_OK;
 }
 
 moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts, int32_t* offsets,
@@ -1293,6 +1599,7 @@ moe_status moe_destroy(moe_handle h) {
     for (auto& pool : h->ev_pool)
       for (cudaEvent_t e : pool) cudaEventDestroy(e);
     release_host_pipeline(h);
+    close_ipc_peers(h);
     if (h->ws) cudaFree(h->ws);
   }
   delete h;

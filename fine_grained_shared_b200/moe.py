@@ -38,7 +38,8 @@ class moe_config(ctypes.Structure):
     _fields_ = [("d_model", c_int32), ("n_routed", c_int32), ("d_ff", c_int32),
                 ("n_shared", c_int32), ("d_ff_shared", c_int32), ("max_tokens", c_int32),
                 ("max_k", c_int32), ("gate", c_int32), ("flags", c_uint32),
-                ("route_nodes", c_int32), ("route_max_nodes", c_int32)]
+                ("route_nodes", c_int32), ("route_max_nodes", c_int32), ("ep_ranks", c_int32),
+                ("ep_rank", c_int32)]
 
 
 class moe_router(ctypes.Structure):
@@ -94,12 +95,23 @@ def lib() -> ctypes.CDLL:
     L.moe_update_bias.argtypes = [moe_handle, c_void_p, ctypes.c_float, c_void_p]
     L.moe_quantize_fp8_rows.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
     L.moe_quantize_fp8_blocks.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
+    L.moe_ep_workspace.argtypes = [moe_handle, POINTER(c_void_p)]
+    L.moe_ep_set_peers.argtypes = [moe_handle, POINTER(c_void_p)]
+    L.moe_ep_ipc_handle.argtypes = [moe_handle, c_void_p]
+    L.moe_ep_open_peers.argtypes = [moe_handle, c_void_p]
+    L.moe_ep_route.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), c_int32, c_void_p]
+    L.moe_ep_dispatch.argtypes = [moe_handle, c_void_p]
+    L.moe_ep_experts.argtypes = [moe_handle, POINTER(moe_experts), POINTER(moe_shared), c_void_p]
+    L.moe_ep_combine.argtypes = [moe_handle, c_void_p, c_void_p]
+    L.moe_ep_plan.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.moe_status_string.argtypes = [c_int]
     L.moe_status_string.restype = c_char_p
     for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_forward_fp8",
                  "moe_get_routing",
                  "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc",
-                 "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks"):
+                 "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_ep_workspace",
+                 "moe_ep_set_peers", "moe_ep_ipc_handle", "moe_ep_open_peers", "moe_ep_route", "moe_ep_dispatch",
+                 "moe_ep_experts", "moe_ep_combine", "moe_ep_plan"):
         getattr(L, name).restype = c_int
     _lib = L
     return L
@@ -185,6 +197,60 @@ def moe_quantize_fp8_blocks(w, batch, rows, cols, q, scale, stream):
     return lib().moe_quantize_fp8_blocks(w, int(batch), int(rows), int(cols), q, scale, stream)
 
 
+def moe_ep_workspace(h):
+    p = c_void_p()
+    st = lib().moe_ep_workspace(h, ctypes.byref(p))
+    return st, p.value
+
+
+def moe_ep_set_peers(h, workspaces):
+    arr = (c_void_p * len(workspaces))(*workspaces)
+    return lib().moe_ep_set_peers(h, arr)
+
+
+def moe_ep_ipc_handle(h):
+    buf = ctypes.create_string_buffer(64)
+    st = lib().moe_ep_ipc_handle(h, buf)
+    return st, buf.raw
+
+
+def moe_ep_open_peers(h, handles):
+    """handles: one 64-byte IPC handle per rank, in rank order."""
+    blob = ctypes.create_string_buffer(b"".join(handles), 64 * len(handles))
+    return lib().moe_ep_open_peers(h, blob)
+
+
+def moe_ep_route(h, x, T, router, K, stream):
+    return lib().moe_ep_route(h, x, int(T), ctypes.byref(router), int(K), stream)
+
+
+def moe_ep_dispatch(h, stream):
+    return lib().moe_ep_dispatch(h, stream)
+
+
+def moe_ep_experts(h, experts, shared, stream):
+    return lib().moe_ep_experts(h, ctypes.byref(experts), ctypes.byref(shared) if shared is not None else None,
+                                stream)
+
+
+def moe_ep_combine(h, out, stream):
+    return lib().moe_ep_combine(h, out, stream)
+
+
+def moe_ep_plan(counts_all, G, n_routed, rank):
+    """Host computation of the dispatch plan (no GPU): counts_all int32 [G, mN] (a C-contiguous
+    numpy array) -> (status, base [mN], counts_local, row_start, mtile_start, mtile128_start
+    [mN / G + 1] each)."""
+    import numpy as np
+    counts_all = np.ascontiguousarray(counts_all, dtype=np.int32)
+    per = max(1, n_routed // max(G, 1))
+    base = np.zeros(max(n_routed, 1), np.int32)
+    tabs = [np.zeros(per + 1, np.int32) for _ in range(4)]
+    st = lib().moe_ep_plan(counts_all.ctypes.data_as(c_void_p), int(G), int(n_routed), int(rank),
+                           base.ctypes.data_as(c_void_p), *(t.ctypes.data_as(c_void_p) for t in tabs))
+    return (st, base, *tabs)
+
+
 # --- torch convenience wrapper (pointers and sizes only) --------------------
 
 def _ptr(t):
@@ -206,12 +272,12 @@ class MoELayer:
     """
 
     def __init__(self, *, d_model, n_routed, d_ff, n_shared, d_ff_shared, max_tokens, max_k,
-                 gate="softmax", flags=0, device=0, node_limit=None):
+                 gate="softmax", flags=0, device=0, node_limit=None, ep_ranks=0, ep_rank=0):
         nodes, max_nodes = node_limit if node_limit is not None else (0, 0)
         self.cfg = moe_config(d_model, n_routed, d_ff, n_shared, d_ff_shared if n_shared else 0,
                               max_tokens, max_k,
                               MOE_GATE_SIGMOID_BIASED if gate == "sigmoid" else MOE_GATE_SOFTMAX, flags,
-                              nodes, max_nodes)
+                              nodes, max_nodes, ep_ranks, ep_rank)
         st, self.h = moe_create(self.cfg, device)
         if st != MOE_OK:
             raise MoEError(st, "moe_create")
@@ -318,6 +384,110 @@ class MoELayer:
         if st != MOE_OK:
             raise MoEError(st, "moe_kernel_times")
         return t
+
+
+class ExpertParallelLayer(MoELayer):
+    """Rank ``ep_rank`` of a layer whose mN routed experts are split over ``ep_ranks`` ranks: it
+    holds experts [ep_rank * mN / G, (ep_rank + 1) * mN / G) (``set_weights`` takes those, stacked)
+    and all shared experts, and runs the layer for its own tokens.
+
+    A forward is four calls with a barrier across the ranks between them, ordered on the stream
+    (see the header): ``forward`` takes that barrier as a callable (``nccl_barrier``);
+    ``forward_emulated`` runs the ranks of one process in lockstep on one stream, whose order is
+    the barrier.  Peers: ``connect_emulated`` (handles of one process) or ``connect_ipc`` (one
+    process per rank)."""
+
+    def __init__(self, *, ep_ranks, ep_rank, **kw):
+        super().__init__(ep_ranks=ep_ranks, ep_rank=ep_rank, **kw)
+        self.ep_ranks, self.ep_rank = ep_ranks, ep_rank
+
+    def _check(self, st, what):
+        if st != MOE_OK:
+            raise MoEError(st, what)
+
+    def workspace(self):
+        st, p = moe_ep_workspace(self.h)
+        self._check(st, "moe_ep_workspace")
+        return p
+
+    def set_peers(self, workspaces):
+        self._check(moe_ep_set_peers(self.h, workspaces), "moe_ep_set_peers")
+
+    def ipc_handle(self):
+        st, hnd = moe_ep_ipc_handle(self.h)
+        self._check(st, "moe_ep_ipc_handle")
+        return hnd
+
+    def open_peers(self, handles):
+        self._check(moe_ep_open_peers(self.h, handles), "moe_ep_open_peers")
+
+    def route(self, x, K, stream=None):
+        self._x = x
+        self._check(moe_ep_route(self.h, _ptr(x) if x.numel() else None, x.shape[0], self.router, K,
+                                 _stream_ptr(stream)), "moe_ep_route")
+
+    def dispatch(self, stream=None):
+        self._check(moe_ep_dispatch(self.h, _stream_ptr(stream)), "moe_ep_dispatch")
+
+    def experts_step(self, stream=None):
+        self._check(moe_ep_experts(self.h, self.experts, self.shared, _stream_ptr(stream)), "moe_ep_experts")
+
+    def combine(self, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty_like(self._x)
+        self._check(moe_ep_combine(self.h, _ptr(out) if out.numel() else None, _stream_ptr(stream)),
+                    "moe_ep_combine")
+        return out
+
+    def forward(self, x, K, barrier, out=None, stream=None):
+        """This rank's part of one forward; ``barrier()`` must order every rank's work on the stream."""
+        self.route(x, K, stream)
+        barrier()
+        self.dispatch(stream)
+        barrier()
+        self.experts_step(stream)
+        barrier()
+        return self.combine(out, stream)
+
+
+def connect_emulated(layers):
+    """Expert-parallel layers of one process (one GPU, or GPUs with peer access): each learns the
+    others' workspaces."""
+    ws = [layer.workspace() for layer in layers]
+    for layer in layers:
+        layer.set_peers(ws)
+
+
+def connect_ipc(layer, group=None):
+    """One process per rank: exchange the workspaces' IPC handles over torch.distributed and open them."""
+    import torch.distributed as dist
+    handles = [None] * layer.ep_ranks
+    dist.all_gather_object(handles, layer.ipc_handle(), group=group)
+    layer.open_peers(handles)
+
+
+def nccl_barrier(device, group=None):
+    """A barrier across the ranks ordered on the current stream: a one-element all-reduce."""
+    import torch
+    import torch.distributed as dist
+    flag = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def barrier():
+        dist.all_reduce(flag, group=group)
+    return barrier
+
+
+def forward_emulated(layers, xs, K, outs=None, stream=None):
+    """The G ranks' forwards in lockstep on one stream (each step of every rank before the next
+    step of any): the stream order takes the place of the barriers."""
+    for layer, x in zip(layers, xs):
+        layer.route(x, K, stream)
+    for layer in layers:
+        layer.dispatch(stream)
+    for layer in layers:
+        layer.experts_step(stream)
+    return [layer.combine(None if outs is None else outs[r], stream) for r, layer in enumerate(layers)]
 
 
 def quantize_fp8_rows(x, stream=None):

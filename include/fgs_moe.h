@@ -99,6 +99,14 @@ typedef struct moe_config {
    * route_nodes (else MOE_ERR_INVALID_ARG). */
   int32_t route_nodes;
   int32_t route_max_nodes;
+  /* Expert parallelism (see moe_ep_route below).  ep_ranks = G ranks that
+   * split the mN routed experts in equal contiguous ranges (expert i on rank
+   * i / (mN / G)); this handle is rank ep_rank and holds mN / G of them.
+   * 0 or 1: a single-GPU handle (moe_forward).  Otherwise 2 <= G <= 32
+   * dividing mN, 0 <= ep_rank < G, and no MOE_FLAG_FP8 (else
+   * MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED). */
+  int32_t ep_ranks;
+  int32_t ep_rank;
 } moe_config;
 
 /* Router.  weight: bf16 [mN, d], row i is e_i.
@@ -317,6 +325,92 @@ moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, uint
                                  void* stream);
 moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, int32_t cols, uint8_t* q,
                                    uint8_t* scale, void* stream);
+
+/* Expert parallelism (DeepSeek-V3 technical report summary, section 3.1
+ * "Compute Clusters": the routed experts of a layer spread over many GPUs;
+ * section 3.2.1 "DualPipe and Computation-Communication Overlap": an
+ * all-to-all dispatch sends each token to the GPUs of its experts and an
+ * all-to-all combine brings the results back; section 2: node-limited routing
+ * bounds how many of them a token reaches -- moe_config.route_nodes /
+ * route_max_nodes, with route_nodes = G to limit the ranks).
+ *
+ * G handles, one per rank (usually one per GPU of one NVLink domain), each
+ * created with ep_ranks = G and its own ep_rank, all with the same other
+ * fields.  Each rank passes its own tokens; the layer's result for a token is
+ * the single-GPU layer's.  A forward is four calls, each asynchronous on
+ * `stream`, separated on every rank by a barrier across the ranks that is
+ * ordered on the same stream (for example a one-element all-reduce):
+ *
+ *   moe_ep_route     router and top-K of this rank's T tokens (T may be 0);
+ *                    the per-expert counts that the other ranks read
+ *   -- barrier --
+ *   moe_ep_dispatch  from every rank's counts: where each row goes; stores
+ *                    each (token, slot) row of x and its gate into the row
+ *                    buffer of the rank that holds the slot's expert
+ *   -- barrier --
+ *   moe_ep_experts   the grouped GEMMs of this rank's experts on the rows it
+ *                    received (all ranks' rows of expert e in ascending rank,
+ *                    then ascending token), and of the shared experts on its
+ *                    own T tokens
+ *   -- barrier --
+ *   moe_ep_combine   out = x + shared + the K g-scaled rows, read from the
+ *                    ranks that computed them, summed in ascending k
+ *
+ * Before the next moe_ep_route every rank must have passed the third barrier
+ * (the calls above on one stream, in this order, ensure it).  x stays
+ * borrowed from moe_ep_route to moe_ep_combine.  The row buffers hold
+ * G * max_tokens * max_k rows (plus padding), so every rank may send all of
+ * its rows to one rank.  Batches of any size run the grouped GEMMs (the decode
+ * FFN of moe_forward is not used).
+ *
+ * The ranks address each other's workspaces directly: moe_ep_set_peers takes
+ * every rank's workspace pointer as this device addresses it (handles on one
+ * GPU, or GPUs of one process with peer access enabled); moe_ep_ipc_handle /
+ * moe_ep_open_peers exchange and open CUDA IPC handles between processes.
+ * The calls below return MOE_ERR_INVALID_ARG on a single-GPU handle, before
+ * the peers are set, or out of order (dispatch before route, ...); other
+ * errors as for moe_forward.  moe_forward and moe_forward_fp8 return
+ * MOE_ERR_UNSUPPORTED on an expert-parallel handle. */
+
+/* This handle's workspace (device pointer), for moe_ep_set_peers of the other
+ * handles when all are in one process. */
+moe_status moe_ep_workspace(moe_handle h, void** workspace);
+/* workspaces[r], r < G: rank r's workspace as this handle's device addresses
+ * it; workspaces[ep_rank] must be this handle's own.  The pointers stay
+ * borrowed for the life of the handle. */
+moe_status moe_ep_set_peers(moe_handle h, void* const* workspaces);
+/* The CUDA IPC handle (64 bytes, written to `handle`) of this handle's
+ * workspace, for the other processes' moe_ep_open_peers. */
+moe_status moe_ep_ipc_handle(moe_handle h, void* handle);
+/* handles: G x 64 bytes, rank r's IPC handle at byte 64 r (this rank's own
+ * entry is ignored).  Opens the others' workspaces (closed by moe_destroy)
+ * and sets them as the peers. */
+moe_status moe_ep_open_peers(moe_handle h, const void* handles);
+
+/* router as for moe_forward; x bf16 [T, d], 0 <= T <= max_tokens. */
+moe_status moe_ep_route(moe_handle h, const void* x, int64_t T, const moe_router* router, int32_t K, void* stream);
+moe_status moe_ep_dispatch(moe_handle h, void* stream);
+/* experts: this rank's mN / G routed experts, stacked as for moe_forward
+ * (w_gate, w_up bf16 [mN / G, I, d]; w_down bf16 [mN / G, d, I]); local
+ * expert l is global expert ep_rank * mN / G + l.  shared as for moe_forward
+ * (every rank holds all K_s shared experts). */
+moe_status moe_ep_experts(moe_handle h, const moe_experts* experts, const moe_shared* shared, void* stream);
+/* out: bf16 [T, d] of the T tokens of the last moe_ep_route. */
+moe_status moe_ep_combine(moe_handle h, void* out, void* stream);
+
+/* The dispatch plan on the host, from every rank's counts (counts_all int32
+ * [G, mN], row r = rank r's rows per global expert): base int32 [mN] = the
+ * first row, in the buffer of expert e's rank, of rank `rank`'s rows of e; and
+ * rank `rank`'s own tables over its mN / G experts, each int32 [mN / G + 1]:
+ * counts_local (rows received per expert; the last entry 0), row_start
+ * (padded to multiples of 256 rows), mtile_start (prefix sum of
+ * ceil(rows / 256)), mtile128_start (prefix sum of ceil(rows / 128)); the
+ * last entry of each prefix is the total.  moe_ep_dispatch computes the same
+ * on the device.  Plain host arithmetic: needs no GPU.  Errors: a null
+ * pointer, G outside [2, 32], mN outside [1, 256] or not a multiple of G,
+ * rank outside [0, G), a negative count -> MOE_ERR_INVALID_ARG. */
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t G, int32_t n_routed, int32_t rank, int32_t* base,
+                       int32_t* counts_local, int32_t* row_start, int32_t* mtile_start, int32_t* mtile128_start);
 
 /* A static string naming the status. */
 const char* moe_status_string(moe_status s);
