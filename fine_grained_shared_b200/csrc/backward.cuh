@@ -1,0 +1,407 @@
+// backward.cuh -- the streaming and CUDA-core steps of the layer's backward
+// pass for the input and the router (DeepSeek-V3 technical report summary,
+// section 3.2.1 "DualPipe and Computation-Communication Overlap": the MoE
+// layer's backward for input and backward for weights are separate pieces of
+// a training step; the formulas are the chain rule through the forward).
+//
+// With dh the gradient of the layer output, for a routed row (token t, slot k,
+// expert e, gate g) and m = SiLU(a) * b, a = W_gate x, b = W_up x:
+//   dm_raw = W_down^T dh               (grouped GEMM, down_gemm.cuh)
+//   dg     = dm_raw . m                (partial sums in the recompute's epilogue)
+//   da, db = g dm_raw b SiLU'(a), g dm_raw SiLU(a)   (gateup_gemm_kernel<true>)
+//   dx_row = W_gate^T da + W_up^T db   (grouped GEMM, down_gemm.cuh)
+//   dx[t]  = dh[t] + shared rows' dx + sum_k dx_row(t, k) + (dz E)[t]
+// and through the gates to the router logits z (softmax: dz = s (ds - s.ds),
+// ds_i = the dg of the slot that chose i; sigmoid, g = s / S over the chosen:
+// ds_k = (dg_k - g . dg) / S, dz = ds s (1 - s) on the chosen experts):
+//   dE = dz^T x, d(logit bias) = sum_t dz.
+// This file holds the steps that are not tensor-core GEMMs: the weight
+// transposes that give the GEMMs K-major operands, the gather of dh into the
+// expert-ordered rows, the gate gradient's reduction, the router backward on
+// the CUDA cores (mN <= 256 dot products per token) and the final sum.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "sm100.cuh"
+
+namespace fgs {
+
+// ---------------------------------------------------------------------------
+// Batched transpose: dst[b][c][col0 + r] = src[b][r][c], r < R, c < C
+// (R, C, dst_ld and col0 multiples of 16).  64 x 64 tiles through shared memory.
+// ---------------------------------------------------------------------------
+struct TransposeArgs {
+  const __nv_bfloat16* src;
+  __nv_bfloat16* dst;
+  int R, C, dst_ld, col0;
+  long long src_bs, dst_bs;  // batch strides in elements
+};
+
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeArgs a) {
+  __shared__ uint16_t tile[64][66];
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64, b = blockIdx.z;
+  const uint16_t* src = reinterpret_cast<const uint16_t*>(a.src) + b * a.src_bs;
+  uint16_t* dst = reinterpret_cast<uint16_t*>(a.dst) + b * a.dst_bs;
+  const int tr = threadIdx.x >> 2, tc = (threadIdx.x & 3) * 16;
+  if (r0 + tr < a.R && c0 + tc < a.C) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(r0 + tr) * a.C + c0 + tc);
+    const uint4 v0 = p[0], v1 = p[1];
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      tile[tr][tc + 2 * j] = static_cast<uint16_t>(w[j] & 0xFFFFu);
+      tile[tr][tc + 2 * j + 1] = static_cast<uint16_t>(w[j] >> 16);
+    }
+  }
+  __syncthreads();
+  // thread (oc, orr): output row c0 + oc, its 16 values r0 + orr .. + 15
+  const int oc = threadIdx.x >> 2, orr = (threadIdx.x & 3) * 16;
+  if (c0 + oc < a.C && r0 + orr < a.R) {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      w[j] = static_cast<uint32_t>(tile[orr + 2 * j][oc]) | (static_cast<uint32_t>(tile[orr + 2 * j + 1][oc]) << 16);
+    uint4* q = reinterpret_cast<uint4*>(dst + static_cast<size_t>(c0 + oc) * a.dst_ld + a.col0 + r0 + orr);
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dh into the expert-ordered rows: dh_perm[slot[t, k]] = dh[t]; a warp per (t, k)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bwd_gather_kernel(const __nv_bfloat16* __restrict__ dh, const int32_t* slot_of,
+                                                        int TK, int K, int d, __nv_bfloat16* dh_perm) {
+  const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (w >= TK) return;
+  const int t = w / K;
+  const uint4* s = reinterpret_cast<const uint4*>(dh + static_cast<size_t>(t) * d);
+  uint4* o = reinterpret_cast<uint4*>(dh_perm + static_cast<size_t>(slot_of[w]) * d);
+  for (int c = lane; c < (d >> 3); c += 32) o[c] = __ldg(s + c);
+}
+
+// ---------------------------------------------------------------------------
+// dgate[t, k] = sum over the 128-column tiles n (ascending) of dg_part[slot[t, k], n]
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) dg_reduce_kernel(const float* dg_part, const int32_t* slot_of, int TK,
+                                                       int n_tiles, float* dgate) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= TK) return;
+  const float* p = dg_part + static_cast<size_t>(slot_of[i]) * n_tiles;
+  float s = 0.f;
+  for (int n = 0; n < n_tiles; ++n) s += p[n];
+  dgate[i] = s;
+}
+
+// ---------------------------------------------------------------------------
+// Router backward on 32-token blocks: recompute z = x E^T (+ c) in fp32, the
+// affinities s, dz from the gates' gradient, and dx_router = dz E.
+// ---------------------------------------------------------------------------
+constexpr int kRbTokens = 32;
+constexpr int kRbCols = 64;  // columns of x and E per staged chunk
+
+struct RouterBwdArgs {
+  int T, N, d, K, sigmoid;
+  const __nv_bfloat16* x;    // [T, d]
+  const __nv_bfloat16* e;    // [N, d]
+  const float* logit_bias;   // [N] or nullptr (softmax)
+  const int32_t* idx;        // [T, K]
+  const float* dgate;        // [T, K]
+  float* dz;                 // [T, N] out
+  float* dx_router;          // [T, d] out
+};
+
+__host__ __device__ constexpr size_t router_bwd_smem_bytes(int N) {
+  // E chunk [N][65], x chunk [32][65], z / dz [32][N + 1]
+  return (static_cast<size_t>(N) * (kRbCols + 1) + kRbTokens * (kRbCols + 1) + kRbTokens * (N + 1)) * 4;
+}
+
+__global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdArgs a) {
+  extern __shared__ float rb_smem[];
+  const int N = a.N, d = a.d;
+  float* es = rb_smem;                          // [N][65]
+  float* xs = es + N * (kRbCols + 1);           // [32][65]
+  float* zs = xs + kRbTokens * (kRbCols + 1);   // [32][N + 1]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t0 = blockIdx.x * kRbTokens;
+  const int nt = min(kRbTokens, a.T - t0);
+  // ---- z: thread (tg, ig) accumulates tokens 4 tg .. + 3 and experts ig + 32 j ----
+  const int tg = tid & 7, ig = tid >> 3;
+  float acc[4][8];
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
+  for (int c0 = 0; c0 < d; c0 += kRbCols) {
+    __syncthreads();
+    for (int i = tid; i < N * (kRbCols / 8); i += 256) {  // 8 columns per 16-byte load
+      const int r = i / (kRbCols / 8), cc = (i - r * (kRbCols / 8)) * 8;
+      const uint4 v = c0 + cc < d ? __ldg(reinterpret_cast<const uint4*>(a.e + static_cast<size_t>(r) * d + c0 + cc))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        es[r * (kRbCols + 1) + cc + 2 * j] = bf16lo(w[j]);
+        es[r * (kRbCols + 1) + cc + 2 * j + 1] = bf16hi(w[j]);
+      }
+    }
+    for (int i = tid; i < kRbTokens * (kRbCols / 8); i += 256) {
+      const int r = i / (kRbCols / 8), cc = (i - r * (kRbCols / 8)) * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < nt && c0 + cc < d) v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + r) * d + c0 + cc));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xs[r * (kRbCols + 1) + cc + 2 * j] = bf16lo(w[j]);
+        xs[r * (kRbCols + 1) + cc + 2 * j + 1] = bf16hi(w[j]);
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int c = 0; c < kRbCols; ++c) {
+      float xv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) xv[m] = xs[(4 * tg + m) * (kRbCols + 1) + c];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = ig + 32 * j;
+        if (i < N) {
+          const float ev = es[i * (kRbCols + 1) + c];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) acc[m][j] = fmaf(xv[m], ev, acc[m][j]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = ig + 32 * j;
+      if (i < N) zs[(4 * tg + m) * (N + 1) + i] = acc[m][j] + (a.logit_bias ? a.logit_bias[i] : 0.f);
+    }
+  __syncthreads();
+  // ---- s and dz: a warp per token ----
+  for (int tl = warp; tl < nt; tl += 8) {
+    float* z = zs + tl * (N + 1);
+    const int t = t0 + tl;
+    if (!a.sigmoid) {
+      float mx = -INFINITY;
+      for (int i = lane; i < N; i += 32) mx = fmaxf(mx, z[i]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.f;
+      for (int i = lane; i < N; i += 32) {
+        const float ex = __expf(z[i] - mx);
+        z[i] = ex;
+        sum += ex;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      const float inv = 1.f / sum;
+      __syncwarp();
+      // s . ds = sum over the chosen slots of s_i dg_k
+      float sds = 0.f;
+      for (int k = 0; k < a.K; ++k) {
+        const int i = a.idx[static_cast<size_t>(t) * a.K + k];
+        sds += z[i] * inv * a.dgate[static_cast<size_t>(t) * a.K + k];
+      }
+      __syncwarp();
+      for (int i = lane; i < N; i += 32) {
+        float ds = 0.f;
+        for (int k = 0; k < a.K; ++k)
+          if (a.idx[static_cast<size_t>(t) * a.K + k] == i) ds = a.dgate[static_cast<size_t>(t) * a.K + k];
+        const float s = z[i] * inv;
+        z[i] = s * (ds - sds);
+      }
+    } else {
+      // g_k = s_k / S over the chosen; ds_k = (dg_k - g . dg) / S; dz = ds s (1 - s) there, 0 elsewhere
+      float S = 0.f, gdg = 0.f;
+      for (int k = 0; k < a.K; ++k) S += 1.f / (1.f + __expf(-z[a.idx[static_cast<size_t>(t) * a.K + k]]));
+      for (int k = 0; k < a.K; ++k) {
+        const float s = 1.f / (1.f + __expf(-z[a.idx[static_cast<size_t>(t) * a.K + k]]));
+        gdg += s / S * a.dgate[static_cast<size_t>(t) * a.K + k];
+      }
+      __syncwarp();
+      for (int i = lane; i < N; i += 32) {
+        float dzi = 0.f;
+        for (int k = 0; k < a.K; ++k)
+          if (a.idx[static_cast<size_t>(t) * a.K + k] == i) {
+            const float s = 1.f / (1.f + __expf(-z[i]));
+            dzi = (a.dgate[static_cast<size_t>(t) * a.K + k] - gdg) / S * s * (1.f - s);
+          }
+        z[i] = dzi;
+      }
+    }
+    __syncwarp();
+    for (int i = lane; i < N; i += 32) a.dz[static_cast<size_t>(t) * N + i] = z[i];
+  }
+  __syncthreads();
+  // ---- dx_router = dz E: thread (row tl = tid / 8, 8 columns (tid % 8) * 8) per 64-column chunk ----
+  const int tl = tid >> 3, cg = (tid & 7) * 8;
+  for (int c0 = 0; c0 < d; c0 += kRbCols) {
+    __syncthreads();
+    for (int i = tid; i < N * (kRbCols / 8); i += 256) {
+      const int r = i / (kRbCols / 8), cc = (i - r * (kRbCols / 8)) * 8;
+      const uint4 v = c0 + cc < d ? __ldg(reinterpret_cast<const uint4*>(a.e + static_cast<size_t>(r) * d + c0 + cc))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        es[r * (kRbCols + 1) + cc + 2 * j] = bf16lo(w[j]);
+        es[r * (kRbCols + 1) + cc + 2 * j + 1] = bf16hi(w[j]);
+      }
+    }
+    __syncthreads();
+    float o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = 0.f;
+    const float* z = zs + tl * (N + 1);
+    for (int i = 0; i < N; ++i) {
+      const float dzi = z[i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = fmaf(dzi, es[i * (kRbCols + 1) + cg + j], o[j]);
+    }
+    if (tl < nt && c0 + cg < d) {
+      float4* q = reinterpret_cast<float4*>(a.dx_router + static_cast<size_t>(t0 + tl) * d + c0 + cg);
+      q[0] = make_float4(o[0], o[1], o[2], o[3]);
+      q[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dE = dz^T x (and d(logit bias) = sum_t dz) in fixed order: CTA (column
+// block of 128, 16 experts, token segment) sums its segment's tokens in
+// ascending order into part[seg]; router_de_reduce_kernel adds the segments
+// in ascending order.
+// ---------------------------------------------------------------------------
+constexpr int kDeCols = 128;
+constexpr int kDeExperts = 16;
+
+struct RouterDeArgs {
+  int T, N, d, seg_tokens;
+  const float* dz;           // [T, N]
+  const __nv_bfloat16* x;    // [T, d]
+  float* part;               // [segments][N][d]
+  float* part_bias;          // [segments][N] or nullptr
+};
+
+__global__ void __launch_bounds__(256) router_de_kernel(RouterDeArgs a) {
+  __shared__ float dzs[kRbTokens][kDeExperts];
+  __shared__ float xs[kRbTokens][kDeCols];
+  const int c0 = blockIdx.x * kDeCols, i0 = blockIdx.y * kDeExperts, seg = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int il = tid >> 4, cl = (tid & 15) * 8;  // expert i0 + il, columns c0 + cl .. + 7
+  const int tb = seg * a.seg_tokens, te = min(a.T, tb + a.seg_tokens);
+  float o[8], ob = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) o[j] = 0.f;
+  for (int t0 = tb; t0 < te; t0 += kRbTokens) {
+    __syncthreads();
+    for (int i = tid; i < kRbTokens * kDeExperts; i += 256) {
+      const int r = i / kDeExperts, e = i - r * kDeExperts;
+      dzs[r][e] = (t0 + r < te && i0 + e < a.N) ? a.dz[static_cast<size_t>(t0 + r) * a.N + i0 + e] : 0.f;
+    }
+    for (int i = tid; i < kRbTokens * (kDeCols / 8); i += 256) {
+      const int r = i / (kDeCols / 8), cc = (i - r * (kDeCols / 8)) * 8;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (t0 + r < te && c0 + cc < a.d) v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + r) * a.d + c0 + cc));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        xs[r][cc + 2 * j] = bf16lo(w[j]);
+        xs[r][cc + 2 * j + 1] = bf16hi(w[j]);
+      }
+    }
+    __syncthreads();
+    for (int r = 0; r < kRbTokens; ++r) {
+      const float dzi = dzs[r][il];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = fmaf(dzi, xs[r][cl + j], o[j]);
+      ob += dzi;
+    }
+  }
+  const int i = i0 + il;
+  if (i < a.N && c0 + cl < a.d) {
+    float4* q = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(seg) * a.N + i) * a.d + c0 + cl);
+    q[0] = make_float4(o[0], o[1], o[2], o[3]);
+    q[1] = make_float4(o[4], o[5], o[6], o[7]);
+  }
+  if (a.part_bias && blockIdx.x == 0 && cl == 0 && i < a.N) a.part_bias[static_cast<size_t>(seg) * a.N + i] = ob;
+}
+
+__global__ void __launch_bounds__(256) router_de_reduce_kernel(const float* part, int segments, size_t n,
+                                                              float* out) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float s = 0.f;
+  for (int g = 0; g < segments; ++g) s += part[static_cast<size_t>(g) * n + i];
+  out[i] = s;
+}
+
+// ---------------------------------------------------------------------------
+// dx[t] = dh[t] + dxs[t] + dx_router[t] + sum_k dx_perm[slot[t, k]] (k ascending), fp32, one rounding;
+// a warp per (token, chunk of cols_per_warp columns)
+// ---------------------------------------------------------------------------
+struct BwdCombineArgs {
+  int T, K, d;
+  const __nv_bfloat16* dh;       // or nullptr (no residual)
+  const __nv_bfloat16* dxs;      // shared experts' rows, or nullptr
+  const float* dx_router;        // or nullptr
+  const __nv_bfloat16* dx_perm;  // routed rows, or nullptr
+  const int32_t* slot_of;
+  __nv_bfloat16* dx;
+};
+
+__global__ void __launch_bounds__(256) bwd_combine_kernel(BwdCombineArgs a, int cols_per_warp) {
+  const int chunks = (a.d + cols_per_warp - 1) / cols_per_warp;
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= a.T * chunks) return;
+  const int t = gw / chunks;
+  const int c0 = (gw - t * chunks) * cols_per_warp, c1 = min(a.d, c0 + cols_per_warp);
+  const int K = a.dx_perm ? a.K : 0;
+  int slots[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) slots[k] = k < K ? a.slot_of[static_cast<size_t>(t) * a.K + k] : 0;
+  auto add8 = [](float (&acc)[8], const uint4& v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      acc[2 * j] += bf16lo(w[j]);
+      acc[2 * j + 1] += bf16hi(w[j]);
+    }
+  };
+  for (int col = c0 + lane * 8; col < c1; col += 256) {
+    const size_t xo = static_cast<size_t>(t) * a.d + col;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    if (a.dh) add8(acc, __ldg(reinterpret_cast<const uint4*>(a.dh + xo)));
+    if (a.dxs) add8(acc, __ldcg(reinterpret_cast<const uint4*>(a.dxs + xo)));
+    if (a.dx_router) {
+      const float4 r0 = __ldcg(reinterpret_cast<const float4*>(a.dx_router + xo));
+      const float4 r1 = __ldcg(reinterpret_cast<const float4*>(a.dx_router + xo) + 1);
+      acc[0] += r0.x; acc[1] += r0.y; acc[2] += r0.z; acc[3] += r0.w;
+      acc[4] += r1.x; acc[5] += r1.y; acc[6] += r1.z; acc[7] += r1.w;
+    }
+    uint4 vy[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      vy[k] = k < K ? __ldcg(reinterpret_cast<const uint4*>(a.dx_perm + static_cast<size_t>(slots[k]) * a.d + col))
+                    : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < K) add8(acc, vy[k]);
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(a.dx + xo) = o;
+  }
+}
+
+}  // namespace fgs

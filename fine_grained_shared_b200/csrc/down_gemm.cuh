@@ -67,7 +67,7 @@ struct GemmArgs {
   const int32_t* mtile_start;  // [num_groups + 1] prefix sum of ceil(count / 256)
   const int32_t* row_start;    // [num_groups + 1]
   int num_kb;                  // 64-wide k-blocks over I
-  const float* row_scale;      // g of each row of Y
+  const float* row_scale;      // g of each row of Y, or nullptr: 1
   __nv_bfloat16* out;          // Y
   // shared experts (dense rows of Hs; their tiles come first)
   int sh_rows;                 // tokens; 0: no shared tiles
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
       {
         const int n0 = c.n_tile * kGemmBN;
-        const float sc = c.shared ? 1.f : a.row_scale[row];
+        const float sc = c.shared || !a.row_scale ? 1.f : a.row_scale[row];
         __nv_bfloat16* orow = (c.shared ? a.sh_out : a.out) + row * a.ld_out;
 #pragma unroll 1
         for (int cc = 0; cc < kGemmBN; cc += 16) {

@@ -73,6 +73,15 @@ struct GateUpArgs {
   uint32_t* err;
   uint64_t timeout_ns;
   int debug_wait;              // CTA 0 waits on a barrier nothing arrives on
+  // the backward's recompute (gateup_gemm_kernel<true>): the incoming gradient of each H element and
+  // what the epilogue writes instead of H
+  const __nv_bfloat16* dm;     // routed: dL/dm per row of X_perm before the gate scale, [rows, n_limit]
+  int ld_dm;
+  const __nv_bfloat16* sh_dm;  // shared: dL/dm per token, [T, sh_n_limit]
+  int sh_ld_dm;
+  const float* row_gate;       // routed: the gate of each row
+  float* dg_part;              // routed: [rows, n_tiles] per 128-column tile, sum of dm * m over its columns
+  int sh_I;                    // shared: columns of one shared expert (I_s)
 };
 
 constexpr int kGuQueue = 4;  // tile-id queue entries
@@ -125,6 +134,16 @@ __device__ __forceinline__ GuTile gu_decode(int tile, int sh_tiles, int sh_n_til
 // with a 128-row box.  tmAs: x with a 128-row box; tmGs, tmUs: the shared
 // experts' W_gate, W_up as [1][K_s * I_s][d].  Maps of an absent part are
 // never read.
+//
+// BWD = false: the forward, H = SiLU(a) * b from the accumulators a = A W_gate^T
+// and b = A W_up^T.  BWD = true: the backward's recompute of a and b, whose
+// epilogue takes the gradient dm of m = SiLU(a) * b (routed rows: before the
+// gate scale g) and writes, per element, da = g dm b SiLU'(a) and
+// db = g dm SiLU(a), SiLU'(a) = sigma(a) (1 + a (1 - sigma(a))): routed rows
+// [da | db] as [rows, 2 I]; shared rows expert by expert, [da_j | db_j] for
+// j < K_s; and, per routed row and 128-column tile, the partial sum of dm * m
+// that makes the gate's gradient dg = dh . y (y = W_down m).
+template <bool BWD>
 __global__ void __launch_bounds__(kGuThreads, 1)
     gateup_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
                        const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmAs,
@@ -372,6 +391,57 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       const int n0 = c.n_tile * (kGuBN / 2);
       const int n_limit = c.shared ? a.sh_n_limit : a.n_limit;
       __nv_bfloat16* orow = c.shared ? a.sh_out + row * a.sh_ld_out : a.out + row * a.ld_out;
+      if constexpr (BWD) {
+        const float gsc = c.shared ? 1.f : a.row_gate[row];
+        const __nv_bfloat16* dmrow = c.shared ? a.sh_dm + row * a.sh_ld_dm : a.dm + row * a.ld_dm;
+        float dg = 0.f;
+#pragma unroll 1
+        for (int cc = 0; cc < kGuBN / 2; cc += 16) {
+          uint32_t gr[16], ur[16];
+          tmem_ld16(tb + cc, gr);
+          tmem_ld16(tb + kGuBN / 2 + cc, ur);
+          tmem_ld_wait();
+          const int col = n0 + cc;
+          if (col < n_limit) {
+            const uint4* src = reinterpret_cast<const uint4*>(dmrow + col);
+            const uint4 d0 = src[0], d1 = src[1];
+            const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+            uint32_t pa[8], pb[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float da2[2], db2[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const float av = __uint_as_float(gr[2 * j + h]), bv = __uint_as_float(ur[2 * j + h]);
+                const float dmr = h ? bf16hi(dw[j]) : bf16lo(dw[j]);
+                const float sg = 1.f / (1.f + __expf(-av));
+                const float silu = av * sg;
+                dg = fmaf(dmr, silu * bv, dg);
+                const float dmv = gsc * dmr;
+                db2[h] = dmv * silu;
+                da2[h] = dmv * bv * sg * (1.f + av * (1.f - sg));
+              }
+              pa[j] = pack_bf16x2(da2[0], da2[1]);
+              pb[j] = pack_bf16x2(db2[0], db2[1]);
+            }
+            __nv_bfloat16* pda;
+            __nv_bfloat16* pdb;
+            if (c.shared) {  // shared expert j's [da_j | db_j]
+              const int j = col / a.sh_I, i = col - j * a.sh_I;
+              pda = orow + static_cast<size_t>(j) * 2 * a.sh_I + i;
+              pdb = pda + a.sh_I;
+            } else {
+              pda = orow + col;
+              pdb = orow + a.n_limit + col;
+            }
+            reinterpret_cast<uint4*>(pda)[0] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+            reinterpret_cast<uint4*>(pda)[1] = make_uint4(pa[4], pa[5], pa[6], pa[7]);
+            reinterpret_cast<uint4*>(pdb)[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+            reinterpret_cast<uint4*>(pdb)[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
+          }
+        }
+        if (!c.shared) a.dg_part[row * a.n_tiles + c.n_tile] = dg;
+      } else {
 #pragma unroll 1
       for (int cc = 0; cc < kGuBN / 2; cc += 16) {
         uint32_t gr[16], ur[16];
@@ -393,6 +463,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
+      }
       }
       tc_fence_before_sync();
       mbar_arrive(&acc_empty[acc]);

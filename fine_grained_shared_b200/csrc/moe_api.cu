@@ -27,6 +27,7 @@
 #include <vector>
 
 #include "../../include/fgs_moe.h"
+#include "backward.cuh"
 #include "decode_ffn.cuh"
 #include "decode_ffn8.cuh"
 #include "down_gemm.cuh"
@@ -191,6 +192,40 @@ Layout make_layout(const moe_config& c) {
   return L;
 }
 
+// The backward's buffers: K-major copies of the expert weights for its two data-gradient GEMMs, the
+// recompute's [da | db] rows, the gate gradient's partial sums, the router's dz and dz E, and the
+// per-segment partial sums of dE.
+constexpr int kDeMaxSegments = 8;
+struct BwdLayout {
+  size_t wdT, wguT, swdT, swguT, dab, dabs, dg_part, dz, dxr, de_part, de_bias_part, dgate, total;
+};
+
+BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
+  BwdLayout B{};
+  const int64_t N = c.n_routed, I = c.d_ff, d = c.d_model, Ks = c.n_shared, Is = c.d_ff_shared;
+  const int64_t Tm = c.max_tokens, Km = c.max_k;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  B.wdT = take(size_t(N) * I * d * 2);
+  B.wguT = take(size_t(N) * d * 2 * I * 2);
+  B.swdT = take(size_t(Ks) * Is * d * 2);
+  B.swguT = take(size_t(Ks) * d * 2 * Is * 2);
+  B.dab = take(size_t(L.P) * 2 * I * 2);
+  B.dabs = take(size_t(L.Tpad) * Ks * 2 * Is * 2);
+  B.dg_part = take(size_t(L.P) * ceil_div(I, kGuBN / 2) * 4);
+  B.dz = take(size_t(Tm) * N * 4);
+  B.dxr = take(size_t(Tm) * d * 4);
+  B.de_part = take(size_t(kDeMaxSegments) * N * d * 4);
+  B.de_bias_part = take(size_t(kDeMaxSegments) * N * 4);
+  B.dgate = take(size_t(Tm) * Km * 4);
+  B.total = o;
+  return B;
+}
+
 moe_status check_config(const moe_config* c) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (c->gate != MOE_GATE_SOFTMAX && c->gate != MOE_GATE_SIGMOID_BIASED) return MOE_ERR_INVALID_ARG;
@@ -282,6 +317,12 @@ struct moe_ctx {
   int64_t ep_T = 0;
   int ep_K = 0;
   int ep_stage = 0;
+  // the last forward: 1 moe_forward (the backward may follow), 0 anything else
+  int last_forward = 0;
+  // the backward's own buffers (allocated by its first call) and their descriptors
+  uint8_t* bws = nullptr;
+  CUtensorMap tm_b_dhperm, tm_b_wdT, tm_b_swdT, tm_b_dab, tm_b_wguT, tm_b_dabs, tm_b_swguT;
+  MapCache tm_b_dh;
 
   template <typename T>
   T* at(size_t off) const {
@@ -376,9 +417,13 @@ cudaError_t set_kernel_attrs() {
   if ((e = set_router_attrs_k<7>(rs)) != cudaSuccess) return e;
   if ((e = set_router_attrs_k<8>(rs)) != cudaSuccess) return e;
   const int us = static_cast<int>(gateup_smem_bytes());
-  if ((e = cudaFuncSetAttribute(gateup_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
+  if ((e = cudaFuncSetAttribute(gateup_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
+  if ((e = cudaFuncSetAttribute(gateup_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
   const int gs = static_cast<int>(gemm_smem_bytes());
   if ((e = cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
+  if ((e = cudaFuncSetAttribute(router_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(router_bwd_smem_bytes(kMaxRouted)))))
+    return e;
   if ((e = cudaFuncSetAttribute(decode_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(ffn_smem_bytes()))))
     return e;
@@ -423,9 +468,11 @@ cudaError_t launch_down(int pairs, cudaStream_t s, bool pdl, const CUtensorMap& 
 
 cudaError_t launch_gateup(int ctas, cudaStream_t s, bool pdl, const CUtensorMap& A, const CUtensorMap& G,
                           const CUtensorMap& U, const CUtensorMap& As, const CUtensorMap& Gs, const CUtensorMap& Us,
-                          const GateUpArgs& ga) {
-  return launch_pdl(gateup_gemm_kernel, dim3(ctas), dim3(kGuThreads), gateup_smem_bytes(), s, 1, pdl, A, G, U, As, Gs,
-                    Us, ga);
+                          const GateUpArgs& ga, bool backward = false) {
+  return backward ? launch_pdl(gateup_gemm_kernel<true>, dim3(ctas), dim3(kGuThreads), gateup_smem_bytes(), s, 1, pdl,
+                               A, G, U, As, Gs, Us, ga)
+                  : launch_pdl(gateup_gemm_kernel<false>, dim3(ctas), dim3(kGuThreads), gateup_smem_bytes(), s, 1, pdl,
+                               A, G, U, As, Gs, Us, ga);
 }
 
 // Destroys the host-buffer forward's copy streams and events (those that exist).
@@ -917,6 +964,7 @@ moe_status moe_forward(moe_handle h, const void* x, int64_t T, const moe_router*
   }
 
   // ---- the final sum ----
+  h->last_forward = 1;
   CombineArgs ca{};
   ca.T = (int)T;
   ca.K = K;
@@ -937,6 +985,7 @@ moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_rou
   if (!h) return MOE_ERR_INVALID_ARG;
   const moe_config& c = h->cfg;
   if (!(c.flags & MOE_FLAG_FP8)) return MOE_ERR_UNSUPPORTED;
+  h->last_forward = 0;  // the workspace will hold FP8 rows: no backward follows
   if (T < 0 || T > c.max_tokens) return MOE_ERR_SHAPE;
   if (K < 1 || K > c.max_k || K > c.n_routed) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
@@ -1181,9 +1230,24 @@ moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_rou
   return launch_combine(h, ca, T, d, s0, pdl);
 }
 
+namespace {
+moe_status forward_host_chunks(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
+                               const moe_experts* experts, const moe_shared* shared, int32_t K, void* out_host,
+                               void* stream);
+}  // namespace
+
 moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
                             const moe_experts* experts, const moe_shared* shared, int32_t K, void* out_host,
                             void* stream) {
+  const moe_status st = forward_host_chunks(h, x_host, T, router, experts, shared, K, out_host, stream);
+  if (h) h->last_forward = 0;  // the workspace holds the device copies' (or the last chunk's) routing
+  return st;
+}
+
+namespace {
+moe_status forward_host_chunks(moe_handle h, const void* x_host, int64_t T, const moe_router* router,
+                               const moe_experts* experts, const moe_shared* shared, int32_t K, void* out_host,
+                               void* stream) {
   if (!h || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
   if (h->cfg.ep_ranks > 1) return MOE_ERR_UNSUPPORTED;
   if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_SHAPE;
@@ -1262,6 +1326,7 @@ moe_status moe_forward_host(moe_handle h, const void* x_host, int64_t T, const m
   }
   return finish(MOE_OK);
 }
+}  // namespace
 
 // ---------------------------------------------------------------------------
 // Expert parallelism: the four steps of a forward and the peers' workspaces
@@ -1516,6 +1581,297 @@ moe_status moe_ep_plan(const int32_t* counts_all, int32_t G, int32_t n_routed, i
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// The backward pass for the input and the router (backward.cuh states the formulas)
+// ---------------------------------------------------------------------------
+
+namespace {
+cudaError_t launch_transpose(const void* src, void* dst, int batch, int R, int C, int dst_ld, int col0,
+                             cudaStream_t s) {
+  TransposeArgs t{};
+  t.src = static_cast<const __nv_bfloat16*>(src);
+  t.dst = static_cast<__nv_bfloat16*>(dst);
+  t.R = R;
+  t.C = C;
+  t.dst_ld = dst_ld;
+  t.col0 = col0;
+  t.src_bs = static_cast<long long>(R) * C;
+  t.dst_bs = static_cast<long long>(C) * dst_ld;
+  transpose_bf16_kernel<<<dim3(ceil_div(C, 64), ceil_div(R, 64), batch), 256, 0, s>>>(t);
+  return cudaGetLastError();
+}
+
+// the backward's buffers and their fixed descriptors, on first use
+moe_status ensure_backward_buffers(moe_ctx* h) {
+  if (h->bws) return MOE_OK;
+  const moe_config& c = h->cfg;
+  const Layout& L = h->L;
+  const BwdLayout B = make_bwd_layout(c, L);
+  if (cudaMalloc(&h->bws, B.total) != cudaSuccess) {
+    cudaGetLastError();
+    h->bws = nullptr;
+    return MOE_ERR_NOMEM;
+  }
+  const int64_t N = c.n_routed, I = c.d_ff, d = c.d_model, Ks = c.n_shared, Is = c.d_ff_shared;
+  bool ok = encode_bf16(&h->tm_b_dhperm, h->ws + L.y, 1, L.P, d, kBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_b_wdT, h->bws + B.wdT, N, I, d, kBoxRowsB, 3);
+  ok = ok && encode_bf16(&h->tm_b_dab, h->bws + B.dab, 1, L.P, 2 * I, kBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_b_wguT, h->bws + B.wguT, N, d, 2 * I, kBoxRowsB, 3);
+  if (Ks > 0) {
+    ok = ok && encode_bf16(&h->tm_b_swdT, h->bws + B.swdT, 1, Ks * Is, d, kBoxRowsB, 3);
+    ok = ok && encode_bf16(&h->tm_b_dabs, h->bws + B.dabs, 1, L.Tpad, Ks * 2 * Is, kBoxRowsA, 2);
+    ok = ok && encode_bf16(&h->tm_b_swguT, h->bws + B.swguT, Ks, d, 2 * Is, kBoxRowsB, 3);
+  } else {
+    h->tm_b_swdT = h->tm_b_wdT;
+    h->tm_b_dabs = h->tm_b_dab;
+    h->tm_b_swguT = h->tm_b_wguT;
+  }
+  if (!ok) {
+    cudaFree(h->bws);
+    h->bws = nullptr;
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router* router, const moe_experts* experts,
+                        const moe_shared* shared, int32_t K, const void* dh, void* dx, float* d_router,
+                        float* d_logit_bias, float* dgate, void* stream) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (c.ep_ranks > 1) return MOE_ERR_UNSUPPORTED;
+  if (T < 0 || T > c.max_tokens) return MOE_ERR_SHAPE;
+  if (K < 1 || K > c.max_k || K > c.n_routed) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (h->last_forward != 1 || T != h->last_T || K != h->last_K) return MOE_ERR_INVALID_ARG;
+  if (!x || !dh || !dx || !router || !router->weight || !experts || !experts->w_gate || !experts->w_up ||
+      !experts->w_down)
+    return MOE_ERR_INVALID_ARG;
+  if ((c.n_shared > 0) != (shared != nullptr)) return MOE_ERR_INVALID_ARG;
+  if (shared && (!shared->w_gate || !shared->w_up || !shared->w_down)) return MOE_ERR_INVALID_ARG;
+  const bool sigmoid = c.gate == MOE_GATE_SIGMOID_BIASED;
+  if (sigmoid ? router->logit_bias != nullptr : router->select_bias != nullptr) return MOE_ERR_INVALID_ARG;
+  if (d_logit_bias && !router->logit_bias) return MOE_ERR_INVALID_ARG;  // no logit bias, no gradient of it
+  const void* ptrs[] = {x, dh, dx, router->weight, experts->w_gate, experts->w_up, experts->w_down,
+                        shared ? shared->w_gate : nullptr, shared ? shared->w_up : nullptr,
+                        shared ? shared->w_down : nullptr, d_router, d_logit_bias, dgate};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  const int64_t d = c.d_model, N = c.n_routed, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const size_t rows_bytes = size_t(T) * d * 2;
+  if (overlaps(dx, rows_bytes, x, rows_bytes) || overlaps(dx, rows_bytes, dh, rows_bytes)) return MOE_ERR_INVALID_ARG;
+
+  DeviceGuard guard(h->device);
+  moe_status st = ensure_backward_buffers(h);
+  if (st != MOE_OK) return st;
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const Layout& L = h->L;
+  const BwdLayout B = make_bwd_layout(c, L);
+  const bool do_shared = Ks > 0 && !(c.flags & MOE_FLAG_NO_SHARED);
+  const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
+  const bool residual = !(c.flags & MOE_FLAG_NO_RESIDUAL);
+  auto bw = [&](size_t off) { return h->bws + off; };
+  h->last_stream = s0;
+
+  // descriptors of the caller's pointers
+  bool ok = refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2);
+  ok = ok && refresh(h->tm_b_dh, dh, T, 1, T, d, kBoxRowsA, 2);
+  ok = ok && refresh(h->tm_wg, experts->w_gate, 0, N, I, d, kGuBoxRowsB, 3);
+  ok = ok && refresh(h->tm_wu, experts->w_up, 0, N, I, d, kGuBoxRowsB, 3);
+  if (shared) {
+    ok = ok && refresh(h->tm_swg, shared->w_gate, 0, 1, Ks * Is, d, kGuBoxRowsB, 3);
+    ok = ok && refresh(h->tm_swu, shared->w_up, 0, 1, Ks * Is, d, kGuBoxRowsB, 3);
+  }
+  if (!ok) return MOE_ERR_CUDA;
+
+  // ---- K-major copies of the weights the data-gradient GEMMs contract over their other dimension ----
+  cudaError_t e = cudaSuccess;
+  if (do_routed) {
+    e = launch_transpose(experts->w_down, bw(B.wdT), (int)N, (int)d, (int)I, (int)d, 0, s0);  // [N][I][d]
+    if (e == cudaSuccess) e = launch_transpose(experts->w_gate, bw(B.wguT), (int)N, (int)I, (int)d, (int)(2 * I), 0, s0);
+    if (e == cudaSuccess)
+      e = launch_transpose(experts->w_up, bw(B.wguT), (int)N, (int)I, (int)d, (int)(2 * I), (int)I, s0);
+  }
+  if (do_shared && e == cudaSuccess) {
+    e = launch_transpose(shared->w_down, bw(B.swdT), (int)Ks, (int)d, (int)Is, (int)d, 0, s0);  // [Ks Is][d]
+    if (e == cudaSuccess)
+      e = launch_transpose(shared->w_gate, bw(B.swguT), (int)Ks, (int)Is, (int)d, (int)(2 * Is), 0, s0);
+    if (e == cudaSuccess)
+      e = launch_transpose(shared->w_up, bw(B.swguT), (int)Ks, (int)Is, (int)d, (int)(2 * Is), (int)Is, s0);
+  }
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+  const int32_t* slot_of = h->at<int32_t>(L.slot);
+  const int TK = (int)(T * K);
+  // ---- dm: routed rows (dh gathered into the expert order, times W_down) and shared rows ----
+  if (do_routed) {
+    bwd_gather_kernel<<<ceil_div(int64_t(TK) * 32, 256), 256, 0, s0>>>(static_cast<const __nv_bfloat16*>(dh), slot_of,
+                                                                       TK, K, (int)d, h->at<__nv_bfloat16>(L.y));
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    GemmArgs g{};
+    g.num_groups = (int)N;
+    g.mtile_start = h->at<int32_t>(L.mtile);
+    g.row_start = h->at<int32_t>(L.row_start);
+    g.num_kb = ceil_div(d, kGemmBK);
+    g.row_scale = nullptr;
+    g.out = h->at<__nv_bfloat16>(L.h);
+    g.n_tiles = ceil_div(I, kGemmBN);
+    g.n_limit = (int)I;
+    g.ld_out = (int)I;
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
+    if (launch_down(h->max_pairs, s0, false, h->tm_b_dhperm, h->tm_b_wdT, h->tm_b_dhperm, h->tm_b_wdT, g) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (do_shared) {
+    GemmArgs g{};
+    g.sh_rows = (int)T;
+    g.sh_num_kb = ceil_div(d, kGemmBK);
+    g.sh_J = 1;
+    g.sh_k_per_j = (int)d;
+    g.sh_out = h->at<__nv_bfloat16>(L.hs);
+    g.n_tiles = ceil_div(Ks * Is, kGemmBN);
+    g.n_limit = (int)(Ks * Is);
+    g.ld_out = (int)(Ks * Is);
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
+    const int tiles = ceil_div(T, kGemmBM) * g.n_tiles;
+    if (launch_down(std::min(h->max_pairs, tiles), s0, false, h->tm_b_dh.map, h->tm_b_swdT, h->tm_b_dh.map, h->tm_b_swdT, g) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  // ---- the recompute of a, b with the SwiGLU backward in its epilogue ----
+  if (do_routed || do_shared) {
+    if (cudaMemsetAsync(h->ws + L.tile_ctr, 0, 8, s0) != cudaSuccess) return MOE_ERR_CUDA;
+    GateUpArgs g{};
+    if (do_routed) {
+      g.num_groups = (int)N;
+      g.mtile_start = h->at<int32_t>(L.mtile128);
+      g.row_start = h->at<int32_t>(L.row_start);
+      g.n_tiles = ceil_div(I, kGuBN / 2);
+      g.n_limit = (int)I;
+      g.out = reinterpret_cast<__nv_bfloat16*>(bw(B.dab));
+      g.ld_out = (int)(2 * I);
+      g.dm = h->at<__nv_bfloat16>(L.h);
+      g.ld_dm = (int)I;
+      g.row_gate = h->at<float>(L.gate_perm);
+      g.dg_part = reinterpret_cast<float*>(bw(B.dg_part));
+    }
+    if (do_shared) {
+      g.sh_rows = (int)T;
+      g.sh_n_tiles = ceil_div(Ks * Is, kGuBN / 2);
+      g.sh_n_limit = (int)(Ks * Is);
+      g.sh_out = reinterpret_cast<__nv_bfloat16*>(bw(B.dabs));
+      g.sh_ld_out = (int)(Ks * 2 * Is);
+      g.sh_dm = h->at<__nv_bfloat16>(L.hs);
+      g.sh_ld_dm = (int)(Ks * Is);
+      g.sh_I = (int)Is;
+    }
+    g.num_kb = ceil_div(d, kGuBK);
+    g.tile_ctr = h->at<int>(L.tile_ctr);
+    g.die_split = h->num_sms / 2;
+    g.err = h->at<uint32_t>(L.err);
+    g.timeout_ns = kTimeoutNs;
+    const int sh_tiles = do_shared ? ceil_div(T, kGuBM) * g.sh_n_tiles : 0;
+    const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
+    const CUtensorMap& sA = do_shared ? h->tm_x.map : h->tm_xperm;
+    const CUtensorMap& sG = do_shared ? h->tm_swg.map : h->tm_wg.map;
+    const CUtensorMap& sU = do_shared ? h->tm_swu.map : h->tm_wu.map;
+    if (launch_gateup(ctas, s0, false, h->tm_xperm, h->tm_wg.map, h->tm_wu.map, sA, sG, sU, g, true) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    // ---- dx rows: [da | db] times [W_gate ; W_up] (routed rows into Y's buffer, shared into Ys') ----
+    GemmArgs g2{};
+    if (do_routed) {
+      g2.num_groups = (int)N;
+      g2.mtile_start = h->at<int32_t>(L.mtile);
+      g2.row_start = h->at<int32_t>(L.row_start);
+      g2.num_kb = ceil_div(2 * I, kGemmBK);
+      g2.row_scale = nullptr;
+      g2.out = h->at<__nv_bfloat16>(L.y);
+    }
+    if (do_shared) {
+      g2.sh_rows = (int)T;
+      g2.sh_num_kb = ceil_div(2 * Is, kGemmBK);
+      g2.sh_J = (int)Ks;
+      g2.sh_k_per_j = (int)(2 * Is);
+      g2.sh_out = h->at<__nv_bfloat16>(L.ys);
+    }
+    g2.n_tiles = ceil_div(d, kGemmBN);
+    g2.n_limit = (int)d;
+    g2.ld_out = (int)d;
+    g2.err = h->at<uint32_t>(L.err);
+    g2.timeout_ns = kTimeoutNs;
+    const int sh_tiles2 = do_shared ? ceil_div(T, kGemmBM) * g2.n_tiles : 0;
+    const int pairs = do_routed || sh_tiles2 > h->max_pairs ? h->max_pairs : sh_tiles2;
+    const CUtensorMap& sA2 = do_shared ? h->tm_b_dabs : h->tm_b_dab;
+    const CUtensorMap& sB2 = do_shared ? h->tm_b_swguT : h->tm_b_wguT;
+    if (launch_down(pairs, s0, false, h->tm_b_dab, h->tm_b_wguT, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // ---- the gates' gradient, and through them the router's ----
+  float* dg = dgate ? dgate : reinterpret_cast<float*>(bw(B.dgate));
+  float* dxr = nullptr;
+  if (do_routed) {
+    dg_reduce_kernel<<<ceil_div(TK, 256), 256, 0, s0>>>(reinterpret_cast<const float*>(bw(B.dg_part)), slot_of, TK,
+                                                         ceil_div(I, kGuBN / 2), dg);
+    RouterBwdArgs rb{};
+    rb.T = (int)T;
+    rb.N = (int)N;
+    rb.d = (int)d;
+    rb.K = K;
+    rb.sigmoid = sigmoid ? 1 : 0;
+    rb.x = static_cast<const __nv_bfloat16*>(x);
+    rb.e = static_cast<const __nv_bfloat16*>(router->weight);
+    rb.logit_bias = router->logit_bias;
+    rb.idx = h->at<int32_t>(L.idx);
+    rb.dgate = dg;
+    rb.dz = reinterpret_cast<float*>(bw(B.dz));
+    rb.dx_router = dxr = reinterpret_cast<float*>(bw(B.dxr));
+    router_bwd_kernel<<<ceil_div(T, kRbTokens), 256, router_bwd_smem_bytes((int)N), s0>>>(rb);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (d_router || d_logit_bias) {
+      const int segs = (int)std::max<int64_t>(1, std::min<int64_t>(kDeMaxSegments, T / 256));
+      RouterDeArgs de{};
+      de.T = (int)T;
+      de.N = (int)N;
+      de.d = (int)d;
+      de.seg_tokens = ceil_div(ceil_div(T, segs), kRbTokens) * kRbTokens;
+      de.dz = rb.dz;
+      de.x = rb.x;
+      de.part = reinterpret_cast<float*>(bw(B.de_part));
+      de.part_bias = d_logit_bias ? reinterpret_cast<float*>(bw(B.de_bias_part)) : nullptr;
+      router_de_kernel<<<dim3(ceil_div(d, kDeCols), ceil_div(N, kDeExperts), segs), 256, 0, s0>>>(de);
+      if (d_router)
+        router_de_reduce_kernel<<<ceil_div(N * d, 256), 256, 0, s0>>>(de.part, segs, size_t(N) * d, d_router);
+      if (d_logit_bias)
+        router_de_reduce_kernel<<<ceil_div(N, 256), 256, 0, s0>>>(de.part_bias, segs, size_t(N), d_logit_bias);
+    }
+  } else {
+    // the routed term left out: the gates and the router have no gradient
+    if (dgate && cudaMemsetAsync(dgate, 0, size_t(TK) * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (d_router && cudaMemsetAsync(d_router, 0, size_t(N) * d * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
+    if (d_logit_bias && cudaMemsetAsync(d_logit_bias, 0, size_t(N) * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // ---- dx = dh + shared rows + router term + the K routed rows (k ascending) ----
+  BwdCombineArgs bc{};
+  bc.T = (int)T;
+  bc.K = K;
+  bc.d = (int)d;
+  bc.dh = residual ? static_cast<const __nv_bfloat16*>(dh) : nullptr;
+  bc.dxs = do_shared ? h->at<__nv_bfloat16>(L.ys) : nullptr;
+  bc.dx_router = dxr;
+  bc.dx_perm = do_routed ? h->at<__nv_bfloat16>(L.y) : nullptr;
+  bc.slot_of = slot_of;
+  bc.dx = static_cast<__nv_bfloat16*>(dx);
+  const int64_t resident = int64_t(h->num_sms) * 64;
+  int cols = (int)d;
+  if (T < resident) cols = ceil_div(ceil_div(d, ceil_div(2 * resident, T)), 256) * 256;
+  const int64_t warps = T * ceil_div(d, cols);
+  bwd_combine_kernel<<<ceil_div(warps * 32, 256), 256, 0, s0>>>(bc, cols);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 moe_status moe_get_routing(moe_handle h, int32_t* idx, float* gate, int32_t* counts, int32_t* offsets,
                            int32_t* src, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
@@ -1600,6 +1956,7 @@ moe_status moe_destroy(moe_handle h) {
       for (cudaEvent_t e : pool) cudaEventDestroy(e);
     release_host_pipeline(h);
     close_ipc_peers(h);
+    if (h->bws) cudaFree(h->bws);
     if (h->ws) cudaFree(h->ws);
   }
   delete h;

@@ -95,6 +95,9 @@ def lib() -> ctypes.CDLL:
     L.moe_update_bias.argtypes = [moe_handle, c_void_p, ctypes.c_float, c_void_p]
     L.moe_quantize_fp8_rows.argtypes = [c_void_p, c_int64, c_int32, c_void_p, c_void_p, c_void_p]
     L.moe_quantize_fp8_blocks.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
+    L.moe_backward.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), POINTER(moe_experts),
+                               POINTER(moe_shared), c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p]
     L.moe_ep_workspace.argtypes = [moe_handle, POINTER(c_void_p)]
     L.moe_ep_set_peers.argtypes = [moe_handle, POINTER(c_void_p)]
     L.moe_ep_ipc_handle.argtypes = [moe_handle, c_void_p]
@@ -109,7 +112,8 @@ def lib() -> ctypes.CDLL:
     for name in ("moe_workspace_bytes", "moe_create", "moe_forward", "moe_forward_host", "moe_forward_fp8",
                  "moe_get_routing",
                  "moe_status_query", "moe_destroy", "moe_set_timing", "moe_kernel_times", "moe_route_noalloc",
-                 "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_ep_workspace",
+                 "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_backward",
+                 "moe_ep_workspace",
                  "moe_ep_set_peers", "moe_ep_ipc_handle", "moe_ep_open_peers", "moe_ep_route", "moe_ep_dispatch",
                  "moe_ep_experts", "moe_ep_combine", "moe_ep_plan"):
         getattr(L, name).restype = c_int
@@ -195,6 +199,13 @@ def moe_quantize_fp8_rows(x, rows, cols, q, scale, stream):
 def moe_quantize_fp8_blocks(w, batch, rows, cols, q, scale, stream):
     """E4M3 codes and UE8M0 scales of 128 x 128 blocks of `batch` matrices; see the header."""
     return lib().moe_quantize_fp8_blocks(w, int(batch), int(rows), int(cols), q, scale, stream)
+
+
+def moe_backward(h, x, T, router, experts, shared, K, dh, dx, d_router, d_logit_bias, dgate, stream):
+    """The backward for the input and the router of the last moe_forward; see the header."""
+    return lib().moe_backward(h, x, int(T), ctypes.byref(router), ctypes.byref(experts),
+                              ctypes.byref(shared) if shared is not None else None, int(K), dh, dx, d_router,
+                              d_logit_bias, dgate, stream)
 
 
 def moe_ep_workspace(h):
@@ -310,6 +321,27 @@ class MoELayer:
         if check and st != MOE_OK:
             raise MoEError(st, "moe_forward")
         return out if check else (st, out)
+
+    def backward(self, x, K, dh, dx=None, router_grad=False, stream=None):
+        """Gradients of the last ``forward(x, K)`` for the upstream gradient dh (bf16 [T, d]):
+        returns (dx bf16 [T, d], dgate float32 [T, K], d_router float32 [mN, d] or None,
+        d_logit_bias float32 [mN] or None).  ``router_grad`` asks for d_router (and d_logit_bias
+        when the layer has a logit bias)."""
+        import torch
+        T = x.shape[0]
+        dev = x.device
+        if dx is None:
+            dx = torch.empty_like(x)
+        dgate = torch.empty((T, K), dtype=torch.float32, device=dev)
+        d_router = torch.empty((self.cfg.n_routed, self.cfg.d_model), dtype=torch.float32, device=dev) \
+            if router_grad else None
+        d_bias = torch.empty(self.cfg.n_routed, dtype=torch.float32, device=dev) \
+            if router_grad and self.router.logit_bias else None
+        st = moe_backward(self.h, _ptr(x), T, self.router, self.experts, self.shared, K, _ptr(dh), _ptr(dx),
+                          _ptr(d_router), _ptr(d_bias), _ptr(dgate), _stream_ptr(stream))
+        if st != MOE_OK:
+            raise MoEError(st, "moe_backward")
+        return dx, dgate, d_router, d_bias
 
     def set_weights_fp8(self, experts_fp8, shared_fp8=None):
         """FP8 expert weights for forward_fp8: (codes, scales) pairs as quantize_fp8_blocks returns

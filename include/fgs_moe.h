@@ -326,6 +326,43 @@ moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, uint
 moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, int32_t cols, uint8_t* q,
                                    uint8_t* scale, void* stream);
 
+/* The backward pass for the input and the router (DeepSeek-V3 technical
+ * report summary, section 3.2.1 "DualPipe and Computation-Communication
+ * Overlap": a training step runs the MoE layer's backward for input and its
+ * backward for weights as separate pieces; the pages print no formula, so
+ * these are the chain rule through the forward above, with the top-K choice
+ * held fixed: the gradient reaches the router through the chosen experts'
+ * gate values only, and the sigmoid variant's selection bias gets none).
+ *
+ * For the last moe_forward on this handle -- called with the same x, T,
+ * router, experts, shared and K, with no other forward (moe_forward_fp8,
+ * moe_forward_host) on the handle since: its routing and expert-ordered rows
+ * are read from the workspace -- and the gradient dh = dL/dh of its output:
+ *   dx        bf16 [T, d] out: dL/du, the residual's dh + the shared experts'
+ *             and the routed experts' input gradients + the router's (dz E)
+ *   d_router  float32 [mN, d] out or NULL: dL/dE = dz^T u
+ *   d_logit_bias float32 [mN] out or NULL: dL/dc = sum_t dz_t (only with a
+ *             logit bias: else MOE_ERR_INVALID_ARG)
+ *   dgate     float32 [T, K] out or NULL: dL/dg_{t,k} = dh_t . FFN_{Sel_t,k}(u_t)
+ * where dz is dL/dz of the affinity logits (softmax: dz = s (ds - s . ds),
+ * ds_i the dgate of the slot that chose expert i, 0 for the others; sigmoid:
+ * ds_k = (dgate_k - g . dgate) / sum of the chosen s, dz = ds s (1 - s) on the
+ * chosen experts, 0 elsewhere).  The debug flags leave the same terms out as
+ * in the forward.  The expert and shared weights' own gradients are not
+ * computed.
+ *
+ * Asynchronous on `stream`.  The first call allocates the backward's buffers
+ * (a K-major copy of the expert weights, rewritten by every call, and
+ * activations of the forward's row count).  Errors: the last forward was not a
+ * moe_forward with this T and K, or another argument error of moe_forward
+ * -> MOE_ERR_INVALID_ARG / SHAPE / ALIGNMENT; dx overlapping x or dh ->
+ * MOE_ERR_INVALID_ARG; an expert-parallel handle -> MOE_ERR_UNSUPPORTED; no
+ * memory for the buffers -> MOE_ERR_NOMEM.  Overwrites the forward's
+ * intermediate rows (H, Y, Hs, Ys) in the workspace. */
+moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router* router, const moe_experts* experts,
+                        const moe_shared* shared, int32_t K, const void* dh, void* dx, float* d_router,
+                        float* d_logit_bias, float* dgate, void* stream);
+
 /* Expert parallelism (DeepSeek-V3 technical report summary, section 3.1
  * "Compute Clusters": the routed experts of a layer spread over many GPUs;
  * section 3.2.1 "DualPipe and Computation-Communication Overlap": an

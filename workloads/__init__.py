@@ -49,6 +49,7 @@ TID_X, TID_ROUTER, TID_BIAS = 0, 1, 2
 TID_W_GATE, TID_W_UP, TID_W_DOWN = 3, 4, 5
 TID_WS_GATE, TID_WS_UP, TID_WS_DOWN = 6, 7, 8
 TID_SAMPLE = 9
+TID_DH = 10
 
 
 @dataclass(frozen=True)
@@ -128,6 +129,11 @@ def normal_bf16(seed: int, tensor_id: int, sub: int, shape, sigma: float) -> tor
 def tokens(shape: LayerShape) -> torch.Tensor:
     """u: bf16 [T, d], entries ~ N(0, 1)."""
     return normal_bf16(shape.seed, TID_X, 0, (shape.T, shape.d), 1.0)
+
+
+def output_gradient(shape: LayerShape, scale: float = 1.0) -> torch.Tensor:
+    """dh: bf16 [T, d], the upstream gradient of the layer's output for the backward, ~ N(0, scale)."""
+    return normal_bf16(shape.seed, TID_DH, 0, (shape.T, shape.d), scale)
 
 
 def router_weight(shape: LayerShape) -> torch.Tensor:
