@@ -69,6 +69,95 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
+// Activations transposed for the weight gradients (whose GEMMs contract over
+// rows): dst[c][r] = scale(r) * src[r][c] for the rows that hold a (token,
+// slot) pair and 0 for the others, every r < R (C a multiple of 16).  Valid
+// rows: G > 0: r - row_start[e] < counts[e] for the expert e whose segment
+// holds r; G = 0: r < row_limit.  scale: nullptr (1) or [R], read only on
+// valid rows.
+// ---------------------------------------------------------------------------
+struct RowTransposeArgs {
+  const __nv_bfloat16* src;
+  __nv_bfloat16* dst;
+  int R, C;
+  long long dst_ld;
+  const float* scale;
+  const int32_t* row_start;  // [G + 1]
+  const int32_t* counts;     // [G]
+  int G, row_limit;
+  int src_rows;              // rows of src that may be read (the others are not valid)
+};
+
+__global__ void __launch_bounds__(256) transpose_rows_kernel(RowTransposeArgs a) {
+  __shared__ uint16_t tile[64][66];
+  __shared__ float rowf[64];  // per row: its scale, or 0 for a row without a pair
+  __shared__ int rowok[64];
+  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  if (tid < 64) {
+    const int r = r0 + tid;
+    bool ok = r < a.R && r < a.src_rows;
+    if (ok && a.G > 0) {
+      int lo = 0, hi = a.G;  // the last expert whose segment starts at or before r
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (a.row_start[mid] <= r) lo = mid;
+        else hi = mid;
+      }
+      ok = r - a.row_start[lo] < a.counts[lo];
+    } else if (ok) {
+      ok = r < a.row_limit;
+    }
+    rowok[tid] = ok ? 1 : 0;
+    rowf[tid] = ok ? (a.scale ? a.scale[r] : 1.f) : 0.f;
+  }
+  const int tr = tid >> 2, tc = (tid & 3) * 16;
+  if (r0 + tr < a.src_rows && c0 + tc < a.C) {
+    const uint4* p = reinterpret_cast<const uint4*>(a.src + static_cast<size_t>(r0 + tr) * a.C + c0 + tc);
+    const uint4 v0 = p[0], v1 = p[1];
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      tile[tr][tc + 2 * j] = static_cast<uint16_t>(w[j] & 0xFFFFu);
+      tile[tr][tc + 2 * j + 1] = static_cast<uint16_t>(w[j] >> 16);
+    }
+  }
+  __syncthreads();
+  const int oc = tid >> 2, orr = (tid & 3) * 16;
+  if (c0 + oc >= a.C || r0 + orr >= a.R) return;
+  uint16_t v[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int rl = orr + j;
+    uint16_t o = 0;
+    if (rowok[rl]) {
+      const float f = rowf[rl] * __uint_as_float(static_cast<uint32_t>(tile[rl][oc]) << 16);
+      o = static_cast<uint16_t>(pack_bf16x2(f, 0.f) & 0xFFFFu);
+    }
+    v[j] = o;
+  }
+  uint16_t* q = reinterpret_cast<uint16_t*>(a.dst) + static_cast<size_t>(c0 + oc) * a.dst_ld + r0 + orr;
+  if (r0 + orr + 16 <= a.R && ((reinterpret_cast<uintptr_t>(q) & 15u) == 0)) {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) w[j] = static_cast<uint32_t>(v[2 * j]) | (static_cast<uint32_t>(v[2 * j + 1]) << 16);
+    reinterpret_cast<uint4*>(q)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(q)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else {
+    for (int j = 0; j < 16 && r0 + orr + j < a.R; ++j) q[j] = v[j];
+  }
+}
+
+// the shared experts' K ranges for the weight-gradient GEMMs: every expert j < n over rows [0, T)
+__global__ void fill_dense_groups_kernel(int32_t* k_start, int32_t* k_count, int n, int T) {
+  const int i = threadIdx.x;
+  if (i < n) {
+    k_start[i] = 0;
+    k_count[i] = T;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // dh into the expert-ordered rows: dh_perm[slot[t, k]] = dh[t]; a warp per (t, k)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_gather_kernel(const __nv_bfloat16* __restrict__ dh, const int32_t* slot_of,

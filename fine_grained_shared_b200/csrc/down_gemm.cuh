@@ -82,6 +82,21 @@ struct GemmArgs {
   uint32_t* err;
   uint64_t timeout_ns;
   int debug_wait;              // CTA 0 waits on a barrier nothing arrives on
+  // weight-gradient mode (kg_groups > 0; the parts above unused): group g multiplies rows
+  // [g * kg_a_row_step, + kg_M) of A by the rows of B (third coordinate g * kg_bz_step), both
+  // K-major, over the K range [kg_k_start[g], + kg_k_count[g]) (zero beyond the count: the
+  // operands hold zeros there); fp32 output [kg_M rows][n_limit] per group, rows >= kg_split of a
+  // group into kg_out2
+  int kg_groups;
+  const int32_t* kg_k_start;   // [groups], multiples of 8
+  const int32_t* kg_k_count;   // [groups]
+  int kg_m_tiles;              // 256-row tiles of a group's kg_M rows
+  int kg_M;
+  int kg_a_row_step;
+  int kg_bz_step;
+  int kg_split;
+  float* kg_out;               // [groups][kg_split][n_limit]
+  float* kg_out2;              // [groups][kg_M - kg_split][n_limit]
 };
 
 __host__ __device__ constexpr size_t gemm_smem_bytes() {
@@ -160,6 +175,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
 
   const int G = a.num_groups;
+  const int KG = a.kg_groups;
+  const int kg_per_group = a.kg_m_tiles * a.n_tiles;
   const int sh_tiles = a.sh_rows > 0 ? (a.sh_rows + kGemmBM - 1) / kGemmBM * a.n_tiles : 0;
   if (tid == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
@@ -181,15 +198,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   pdl_wait();  // H, Hs and the router's tables are complete from here
   pdl_launch_dependents();
-  for (int i = tid; i <= G; i += kGemmThreads) {
-    s_mts[i] = G ? a.mtile_start[i] : 0;
-    s_rows[i] = G ? a.row_start[i] : 0;
+  if (KG) {  // weight-gradient mode: s_mts = the groups' K counts, s_rows = their K starts
+    for (int i = tid; i < KG; i += kGemmThreads) {
+      s_mts[i] = a.kg_k_count[i];
+      s_rows[i] = a.kg_k_start[i];
+    }
+  } else {
+    for (int i = tid; i <= G; i += kGemmThreads) {
+      s_mts[i] = G ? a.mtile_start[i] : 0;
+      s_rows[i] = G ? a.row_start[i] : 0;
+    }
   }
   tc_fence_before_sync();
   cluster_sync();  // both CTAs' barriers exist before any copy or arrive targets them
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const int total_tiles = sh_tiles + s_mts[G] * a.n_tiles;
+  const int total_tiles = KG ? KG * kg_per_group : sh_tiles + s_mts[G] * a.n_tiles;
   const uint32_t full_lead = mapa_shared(smem_u32(full), 0);         // the even CTA's full[0]
   const uint32_t acc_empty_lead = mapa_shared(smem_u32(acc_empty), 0);
   bool aborted = false;
@@ -207,6 +231,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int s = 0, issued = 0;
     uint32_t ph = 0;
     for (int tile = pair; tile < total_tiles && !aborted; tile += num_pairs) {
+      if (KG) {
+        const int g = tile / kg_per_group, local = tile - g * kg_per_group;
+        const int mt = local / a.n_tiles, nt = local - mt * a.n_tiles;
+        const int arow = g * a.kg_a_row_step + mt * kGemmBM + static_cast<int>(rank) * kCtaRows;
+        const int brow = nt * kGemmBN + static_cast<int>(rank) * (kGemmBN / 2);
+        const int bz = a.kg_bz_step ? g : 0;
+        const int nkb = (s_mts[g] + kGemmBK - 1) / kGemmBK;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, a.timeout_ns, abort_flag)) {
+            pair_record_error(a.err, abort_flag, rank, 3);
+            aborted = true;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kStageA + kStageB));
+          const int kc = s_rows[g] + kb * kGemmBK;
+          const uint32_t fb = full_lead + 8u * static_cast<uint32_t>(s);
+          tma_load_2d_pair(sA + s * kStageA, &tmA, fb, kc, arow);
+          tma_load_3d_pair(sB + s * kStageB, &tmB, fb, kc, brow, bz);
+          ++issued;
+          if (++s == kGemmStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        continue;
+      }
       const TileCoord c = decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
       const int row0 = c.row0 + static_cast<int>(rank) * kCtaRows;
       // each CTA stages its half of the tile's 256 output columns of W_down
@@ -260,7 +310,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     for (int tile = pair; tile < total_tiles && !aborted; tile += num_pairs) {
-      const int kblocks = tile < sh_tiles ? a.sh_J * a.sh_num_kb : a.num_kb;
+      const int kblocks = KG ? (s_mts[tile / kg_per_group] + kGemmBK - 1) / kGemmBK
+                             : tile < sh_tiles ? a.sh_J * a.sh_num_kb : a.num_kb;
       if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1u, a.timeout_ns, abort_flag)) {
         pair_record_error(a.err, abort_flag, rank, 5);
         aborted = true;
@@ -302,7 +353,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int tile = pair; tile < total_tiles; tile += num_pairs) {
-      const TileCoord c = decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
+      const TileCoord c = KG ? TileCoord{} : decode_tile(tile, sh_tiles, s_mts, s_rows, G, a.n_tiles);
       bool ok = mbar_wait(&acc_full[acc], acc_ph, a.timeout_ns, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
@@ -314,7 +365,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t tb = tmem + static_cast<uint32_t>(acc * kGemmBN) + (static_cast<uint32_t>(q * 32) << 16);
       const size_t row = static_cast<size_t>(c.row0) + rank * kCtaRows + r;
 
-      {
+      if (KG) {
+        // fp32 weight gradient rows; a group without rows is all zeros (no MMA wrote the accumulator)
+        const int g = tile / kg_per_group, local = tile - g * kg_per_group;
+        const int mt = local / a.n_tiles, nt = local - mt * a.n_tiles;
+        const int m = mt * kGemmBM + static_cast<int>(rank) * kCtaRows + r;
+        const bool empty_group = s_mts[g] == 0;
+        float* orow = nullptr;
+        if (m < a.kg_M)
+          orow = m < a.kg_split
+                     ? a.kg_out + (static_cast<size_t>(g) * a.kg_split + m) * a.n_limit
+                     : a.kg_out2 + (static_cast<size_t>(g) * (a.kg_M - a.kg_split) + (m - a.kg_split)) * a.n_limit;
+#pragma unroll 1
+        for (int cc = 0; cc < kGemmBN; cc += 16) {
+          uint32_t vr[16];
+          tmem_ld16(tb + cc, vr);
+          tmem_ld_wait();
+          const int col = nt * kGemmBN + cc;
+          if (orow && col < a.n_limit) {
+            float4* dst = reinterpret_cast<float4*>(orow + col);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = empty_group ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                   : make_float4(__uint_as_float(vr[4 * j]), __uint_as_float(vr[4 * j + 1]),
+                                                 __uint_as_float(vr[4 * j + 2]), __uint_as_float(vr[4 * j + 3]));
+          }
+        }
+      } else {
         const int n0 = c.n_tile * kGemmBN;
         const float sc = c.shared || !a.row_scale ? 1.f : a.row_scale[row];
         __nv_bfloat16* orow = (c.shared ? a.sh_out : a.out) + row * a.ld_out;

@@ -82,13 +82,22 @@ struct GateUpArgs {
   const float* row_gate;       // routed: the gate of each row
   float* dg_part;              // routed: [rows, n_tiles] per 128-column tile, sum of dm * m over its columns
   int sh_I;                    // shared: columns of one shared expert (I_s)
+  // for the weight gradients (nullptr: not written): m, da and db transposed -- column c of a
+  // row r at [c][r] -- with zeros in the rows that hold no (token, slot) pair
+  const int32_t* counts;       // routed: [G] rows of each expert (the rest of its segment is padding)
+  __nv_bfloat16* mT;           // routed: [I][ldT]
+  __nv_bfloat16* dabT;         // routed: [2 I][ldT], da rows then db rows
+  long long ldT;
+  __nv_bfloat16* sh_mT;        // shared: [K_s I_s][sh_ldT]
+  __nv_bfloat16* sh_dabT;      // shared: [K_s 2 I_s][sh_ldT], expert j's da rows then its db rows
+  long long sh_ldT;
 };
 
 constexpr int kGuQueue = 4;  // tile-id queue entries
 
 __host__ __device__ constexpr size_t gateup_smem_bytes() {
   return 1024 + static_cast<size_t>(kGuStages) * (kGuStageA + kGuStageB) +
-         8 * (2 * kGuStages + 4 + 2 + 2 * kGuQueue) + 16 + 4 * (2 * 264 + kGuQueue);
+         8 * (2 * kGuStages + 4 + 2 + 2 * kGuQueue) + 16 + 4 * (3 * 264 + kGuQueue);
 }
 
 __device__ __forceinline__ void gu_record_error(uint32_t* err, volatile int* abort, uint32_t site) {
@@ -166,6 +175,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
   int32_t* s_mts = reinterpret_cast<int32_t*>(tmem_slot + 4);  // [264]
   int32_t* s_rows = s_mts + 264;                                // [264]
   volatile int32_t* s_tq = s_rows + 264;                        // [kGuQueue]
+  int32_t* s_cnt = const_cast<int32_t*>(s_tq) + kGuQueue;       // [264] the backward's row counts
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -267,6 +277,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
     for (int i = lane; i <= G; i += 32) {
       s_mts[i] = G ? a.mtile_start[i] : 0;
       s_rows[i] = G ? a.row_start[i] : 0;
+      if (BWD) s_cnt[i] = (i < G && a.counts) ? a.counts[i] : 0;
     }
     __syncwarp();
     if (lane == 0) {
@@ -394,6 +405,12 @@ __global__ void __launch_bounds__(kGuThreads, 1)
       if constexpr (BWD) {
         const float gsc = c.shared ? 1.f : a.row_gate[row];
         const __nv_bfloat16* dmrow = c.shared ? a.sh_dm + row * a.sh_ld_dm : a.dm + row * a.ld_dm;
+        // a row that holds no (token, slot) pair (expert padding, or past the tokens) stores zeros
+        // in the transposed outputs, whose sums over rows would otherwise take it in
+        const bool valid = c.shared ? static_cast<int>(row) < a.sh_rows
+                                    : static_cast<int>(row) - s_rows[c.g] < s_cnt[c.g];
+        __nv_bfloat16* mT = c.shared ? a.sh_mT : a.mT;
+        const long long ldT = c.shared ? a.sh_ldT : a.ldT;
         float dg = 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < kGuBN / 2; cc += 16) {
@@ -406,23 +423,48 @@ __global__ void __launch_bounds__(kGuThreads, 1)
             const uint4* src = reinterpret_cast<const uint4*>(dmrow + col);
             const uint4 d0 = src[0], d1 = src[1];
             const uint32_t dw[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-            uint32_t pa[8], pb[8];
+            uint32_t pa[8], pb[8], pm[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              float da2[2], db2[2];
+              float da2[2], db2[2], m2[2];
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const float av = __uint_as_float(gr[2 * j + h]), bv = __uint_as_float(ur[2 * j + h]);
                 const float dmr = h ? bf16hi(dw[j]) : bf16lo(dw[j]);
                 const float sg = 1.f / (1.f + __expf(-av));
                 const float silu = av * sg;
-                dg = fmaf(dmr, silu * bv, dg);
+                m2[h] = silu * bv;
+                dg = fmaf(dmr, m2[h], dg);
                 const float dmv = gsc * dmr;
                 db2[h] = dmv * silu;
                 da2[h] = dmv * bv * sg * (1.f + av * (1.f - sg));
               }
               pa[j] = pack_bf16x2(da2[0], da2[1]);
               pb[j] = pack_bf16x2(db2[0], db2[1]);
+              pm[j] = valid ? pack_bf16x2(m2[0], m2[1]) : 0u;
+            }
+            if (mT) {
+              // column-major stores: the warp's 32 rows of one column are 64 contiguous bytes
+              __nv_bfloat16* dT = c.shared ? a.sh_dabT : a.dabT;
+              size_t ra, rb;  // rows of da and db of column col in dT
+              if (c.shared) {
+                const int j = col / a.sh_I, i = col - j * a.sh_I;
+                ra = static_cast<size_t>(j) * 2 * a.sh_I + i;
+                rb = ra + a.sh_I;
+              } else {
+                ra = static_cast<size_t>(col);
+                rb = ra + a.n_limit;
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const uint32_t sel = (j & 1) ? 16u : 0u;
+                const uint16_t mv = static_cast<uint16_t>(pm[j >> 1] >> sel);
+                const uint16_t av = valid ? static_cast<uint16_t>(pa[j >> 1] >> sel) : uint16_t(0);
+                const uint16_t bv = valid ? static_cast<uint16_t>(pb[j >> 1] >> sel) : uint16_t(0);
+                reinterpret_cast<uint16_t*>(mT)[static_cast<size_t>(col + j) * ldT + row] = mv;
+                reinterpret_cast<uint16_t*>(dT)[(ra + j) * ldT + row] = av;
+                reinterpret_cast<uint16_t*>(dT)[(rb + j) * ldT + row] = bv;
+              }
             }
             __nv_bfloat16* pda;
             __nv_bfloat16* pdb;

@@ -197,7 +197,10 @@ Layout make_layout(const moe_config& c) {
 // per-segment partial sums of dE.
 constexpr int kDeMaxSegments = 8;
 struct BwdLayout {
-  size_t wdT, wguT, swdT, swguT, dab, dabs, dg_part, dz, dxr, de_part, de_bias_part, dgate, total;
+  size_t wdT, wguT, swdT, swguT, dab, dabs, dg_part, dz, dxr, de_part, de_bias_part, dgate;
+  // the weight gradients' operands: activations transposed (rows of the forward as columns)
+  size_t dyT, xpermT, mT, dabT, dhT, xT, msT, dabsT, sh_kstart, sh_kcount, total;
+  int64_t Pt;  // row count of the transposed routed activations (the forward's rows, padded to 64)
 };
 
 BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
@@ -222,6 +225,17 @@ BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
   B.de_part = take(size_t(kDeMaxSegments) * N * d * 4);
   B.de_bias_part = take(size_t(kDeMaxSegments) * N * 4);
   B.dgate = take(size_t(Tm) * Km * 4);
+  B.Pt = (L.P + 63) / 64 * 64;
+  B.dyT = take(size_t(d) * B.Pt * 2);
+  B.xpermT = take(size_t(d) * B.Pt * 2);
+  B.mT = take(size_t(I) * B.Pt * 2);
+  B.dabT = take(size_t(2 * I) * B.Pt * 2);
+  B.dhT = take(size_t(d) * L.Tpad * 2);
+  B.xT = take(size_t(d) * L.Tpad * 2);
+  B.msT = take(size_t(Ks) * Is * L.Tpad * 2);
+  B.dabsT = take(size_t(Ks) * 2 * Is * L.Tpad * 2);
+  B.sh_kstart = take(64 * 4);
+  B.sh_kcount = take(64 * 4);
   B.total = o;
   return B;
 }
@@ -322,6 +336,7 @@ struct moe_ctx {
   // the backward's own buffers (allocated by its first call) and their descriptors
   uint8_t* bws = nullptr;
   CUtensorMap tm_b_dhperm, tm_b_wdT, tm_b_swdT, tm_b_dab, tm_b_wguT, tm_b_dabs, tm_b_swguT;
+  CUtensorMap tm_b_dyT, tm_b_xpermT, tm_b_mT, tm_b_dabT, tm_b_dhT, tm_b_xT, tm_b_msT, tm_b_dabsT;
   MapCache tm_b_dh;
 
   template <typename T>
@@ -1614,6 +1629,13 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
   }
   const int64_t N = c.n_routed, I = c.d_ff, d = c.d_model, Ks = c.n_shared, Is = c.d_ff_shared;
   bool ok = encode_bf16(&h->tm_b_dhperm, h->ws + L.y, 1, L.P, d, kBoxRowsA, 2);
+  // the weight gradients: A operands 2-D [rows][K = forward rows], B operands 3-D [groups][rows][K]
+  ok = ok && encode_bf16(&h->tm_b_dyT, h->bws + B.dyT, 1, d, B.Pt, kBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_b_dabT, h->bws + B.dabT, 1, 2 * I, B.Pt, kBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_b_mT, h->bws + B.mT, 1, I, B.Pt, kBoxRowsB, 3);
+  ok = ok && encode_bf16(&h->tm_b_xpermT, h->bws + B.xpermT, 1, d, B.Pt, kBoxRowsB, 3);
+  ok = ok && encode_bf16(&h->tm_b_dhT, h->bws + B.dhT, 1, d, L.Tpad, kBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_b_xT, h->bws + B.xT, 1, d, L.Tpad, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_wdT, h->bws + B.wdT, N, I, d, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_dab, h->bws + B.dab, 1, L.P, 2 * I, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_wguT, h->bws + B.wguT, N, d, 2 * I, kBoxRowsB, 3);
@@ -1621,7 +1643,11 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
     ok = ok && encode_bf16(&h->tm_b_swdT, h->bws + B.swdT, 1, Ks * Is, d, kBoxRowsB, 3);
     ok = ok && encode_bf16(&h->tm_b_dabs, h->bws + B.dabs, 1, L.Tpad, Ks * 2 * Is, kBoxRowsA, 2);
     ok = ok && encode_bf16(&h->tm_b_swguT, h->bws + B.swguT, Ks, d, 2 * Is, kBoxRowsB, 3);
+    ok = ok && encode_bf16(&h->tm_b_msT, h->bws + B.msT, Ks, Is, L.Tpad, kBoxRowsB, 3);
+    ok = ok && encode_bf16(&h->tm_b_dabsT, h->bws + B.dabsT, 1, Ks * 2 * Is, L.Tpad, kBoxRowsA, 2);
   } else {
+    h->tm_b_msT = h->tm_b_mT;
+    h->tm_b_dabsT = h->tm_b_dabT;
     h->tm_b_swdT = h->tm_b_wdT;
     h->tm_b_dabs = h->tm_b_dab;
     h->tm_b_swguT = h->tm_b_wguT;
@@ -1637,7 +1663,7 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
 
 moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router* router, const moe_experts* experts,
                         const moe_shared* shared, int32_t K, const void* dh, void* dx, float* d_router,
-                        float* d_logit_bias, float* dgate, void* stream) {
+                        float* d_logit_bias, float* dgate, const moe_weight_grads* wgrad, void* stream) {
   if (!h) return MOE_ERR_INVALID_ARG;
   const moe_config& c = h->cfg;
   if (c.ep_ranks > 1) return MOE_ERR_UNSUPPORTED;
@@ -1653,9 +1679,15 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   const bool sigmoid = c.gate == MOE_GATE_SIGMOID_BIASED;
   if (sigmoid ? router->logit_bias != nullptr : router->select_bias != nullptr) return MOE_ERR_INVALID_ARG;
   if (d_logit_bias && !router->logit_bias) return MOE_ERR_INVALID_ARG;  // no logit bias, no gradient of it
+  if (wgrad && (!wgrad->w_gate || !wgrad->w_up || !wgrad->w_down ||
+                (c.n_shared > 0 && (!wgrad->ws_gate || !wgrad->ws_up || !wgrad->ws_down))))
+    return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {x, dh, dx, router->weight, experts->w_gate, experts->w_up, experts->w_down,
                         shared ? shared->w_gate : nullptr, shared ? shared->w_up : nullptr,
-                        shared ? shared->w_down : nullptr, d_router, d_logit_bias, dgate};
+                        shared ? shared->w_down : nullptr, d_router, d_logit_bias, dgate,
+                        wgrad ? wgrad->w_gate : nullptr, wgrad ? wgrad->w_up : nullptr,
+                        wgrad ? wgrad->w_down : nullptr, wgrad ? wgrad->ws_gate : nullptr,
+                        wgrad ? wgrad->ws_up : nullptr, wgrad ? wgrad->ws_down : nullptr};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
   const int64_t d = c.d_model, N = c.n_routed, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
@@ -1709,6 +1741,27 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     bwd_gather_kernel<<<ceil_div(int64_t(TK) * 32, 256), 256, 0, s0>>>(static_cast<const __nv_bfloat16*>(dh), slot_of,
                                                                        TK, K, (int)d, h->at<__nv_bfloat16>(L.y));
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (wgrad) {
+      // dy = g dh and X_perm per row, transposed, zero on the rows without a pair
+      RowTransposeArgs rt{};
+      rt.R = (int)L.P;
+      rt.src_rows = (int)L.P;
+      rt.C = (int)d;
+      rt.dst_ld = B.Pt;
+      rt.row_start = h->at<int32_t>(L.row_start);
+      rt.counts = h->at<int32_t>(L.counts);
+      rt.G = (int)N;
+      const dim3 grid(ceil_div(d, 64), ceil_div(L.P, 64));
+      rt.src = h->at<__nv_bfloat16>(L.y);
+      rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dyT));
+      rt.scale = h->at<float>(L.gate_perm);
+      transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
+      rt.src = h->at<__nv_bfloat16>(L.x_perm);
+      rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xpermT));
+      rt.scale = nullptr;
+      transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
+      if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    }
     GemmArgs g{};
     g.num_groups = (int)N;
     g.mtile_start = h->at<int32_t>(L.mtile);
@@ -1724,6 +1777,26 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     if (launch_down(h->max_pairs, s0, false, h->tm_b_dhperm, h->tm_b_wdT, h->tm_b_dhperm, h->tm_b_wdT, g) !=
         cudaSuccess)
       return MOE_ERR_CUDA;
+  }
+  if (do_shared && wgrad) {
+    // dh and x transposed, zero past the T tokens
+    RowTransposeArgs rt{};
+    rt.R = (int)L.Tpad;  // rows T .. Tpad are written as zeros, never read from the sources
+    rt.src_rows = (int)T;
+    rt.C = (int)d;
+    rt.dst_ld = L.Tpad;
+    rt.G = 0;
+    rt.row_limit = (int)T;
+    const dim3 grid(ceil_div(d, 64), ceil_div(L.Tpad, 64));
+    rt.src = static_cast<const __nv_bfloat16*>(dh);
+    rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dhT));
+    transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
+    rt.src = static_cast<const __nv_bfloat16*>(x);
+    rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
+    transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
+    fill_dense_groups_kernel<<<1, 64, 0, s0>>>(reinterpret_cast<int32_t*>(bw(B.sh_kstart)),
+                                               reinterpret_cast<int32_t*>(bw(B.sh_kcount)), (int)Ks, (int)T);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (do_shared) {
     GemmArgs g{};
@@ -1758,6 +1831,12 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       g.ld_dm = (int)I;
       g.row_gate = h->at<float>(L.gate_perm);
       g.dg_part = reinterpret_cast<float*>(bw(B.dg_part));
+      if (wgrad) {
+        g.counts = h->at<int32_t>(L.counts);
+        g.mT = reinterpret_cast<__nv_bfloat16*>(bw(B.mT));
+        g.dabT = reinterpret_cast<__nv_bfloat16*>(bw(B.dabT));
+        g.ldT = B.Pt;
+      }
     }
     if (do_shared) {
       g.sh_rows = (int)T;
@@ -1768,6 +1847,11 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       g.sh_dm = h->at<__nv_bfloat16>(L.hs);
       g.sh_ld_dm = (int)(Ks * Is);
       g.sh_I = (int)Is;
+      if (wgrad) {
+        g.sh_mT = reinterpret_cast<__nv_bfloat16*>(bw(B.msT));
+        g.sh_dabT = reinterpret_cast<__nv_bfloat16*>(bw(B.dabsT));
+        g.sh_ldT = L.Tpad;
+      }
     }
     g.num_kb = ceil_div(d, kGuBK);
     g.tile_ctr = h->at<int>(L.tile_ctr);
@@ -1808,6 +1892,60 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     const CUtensorMap& sA2 = do_shared ? h->tm_b_dabs : h->tm_b_dab;
     const CUtensorMap& sB2 = do_shared ? h->tm_b_swguT : h->tm_b_wguT;
     if (launch_down(pairs, s0, false, h->tm_b_dab, h->tm_b_wguT, sA2, sB2, g2) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  // ---- the expert weights' gradients: per expert, sums over its rows (GEMMs with K = the rows) ----
+  if (wgrad) {
+    auto kg_gemm = [&](const CUtensorMap& A, const CUtensorMap& Bm, int groups, const int32_t* kstart,
+                       const int32_t* kcount, int M, int a_step, int bz_step, int split, int Ncols, float* out,
+                       float* out2) {
+      GemmArgs k{};
+      k.kg_groups = groups;
+      k.kg_k_start = kstart;
+      k.kg_k_count = kcount;
+      k.kg_M = M;
+      k.kg_m_tiles = ceil_div(M, kGemmBM);
+      k.kg_a_row_step = a_step;
+      k.kg_bz_step = bz_step;
+      k.kg_split = split;
+      k.kg_out = out;
+      k.kg_out2 = out2;
+      k.n_tiles = ceil_div(Ncols, kGemmBN);
+      k.n_limit = Ncols;
+      k.err = h->at<uint32_t>(L.err);
+      k.timeout_ns = kTimeoutNs;
+      const int tiles = groups * k.kg_m_tiles * k.n_tiles;
+      return launch_down(std::min(h->max_pairs, tiles), s0, false, A, Bm, A, Bm, k);
+    };
+    cudaError_t ke = cudaSuccess;
+    if (do_routed) {
+      const int32_t* ks = h->at<int32_t>(L.row_start);
+      const int32_t* kc = h->at<int32_t>(L.counts);
+      ke = kg_gemm(h->tm_b_dyT, h->tm_b_mT, (int)N, ks, kc, (int)d, 0, 0, (int)d, (int)I, wgrad->w_down, nullptr);
+      if (ke == cudaSuccess)
+        ke = kg_gemm(h->tm_b_dabT, h->tm_b_xpermT, (int)N, ks, kc, (int)(2 * I), 0, 0, (int)I, (int)d, wgrad->w_gate,
+                     wgrad->w_up);
+    } else {
+      const size_t wb = size_t(N) * I * d * 4;
+      if (cudaMemsetAsync(wgrad->w_gate, 0, wb, s0) != cudaSuccess ||
+          cudaMemsetAsync(wgrad->w_up, 0, wb, s0) != cudaSuccess ||
+          cudaMemsetAsync(wgrad->w_down, 0, wb, s0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    if (Ks > 0 && do_shared && ke == cudaSuccess) {
+      const int32_t* ks = reinterpret_cast<const int32_t*>(bw(B.sh_kstart));
+      const int32_t* kc = reinterpret_cast<const int32_t*>(bw(B.sh_kcount));
+      ke = kg_gemm(h->tm_b_dhT, h->tm_b_msT, (int)Ks, ks, kc, (int)d, 0, 1, (int)d, (int)Is, wgrad->ws_down, nullptr);
+      if (ke == cudaSuccess)
+        ke = kg_gemm(h->tm_b_dabsT, h->tm_b_xT, (int)Ks, ks, kc, (int)(2 * Is), (int)(2 * Is), 0, (int)Is, (int)d,
+                     wgrad->ws_gate, wgrad->ws_up);
+    } else if (Ks > 0 && ke == cudaSuccess) {
+      const size_t wb = size_t(Ks) * Is * d * 4;
+      if (cudaMemsetAsync(wgrad->ws_gate, 0, wb, s0) != cudaSuccess ||
+          cudaMemsetAsync(wgrad->ws_up, 0, wb, s0) != cudaSuccess ||
+          cudaMemsetAsync(wgrad->ws_down, 0, wb, s0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    }
+    if (ke != cudaSuccess) return MOE_ERR_CUDA;
   }
   // ---- the gates' gradient, and through them the router's ----
   float* dg = dgate ? dgate : reinterpret_cast<float*>(bw(B.dgate));

@@ -54,6 +54,11 @@ class moe_shared(ctypes.Structure):
     _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p)]
 
 
+class moe_weight_grads(ctypes.Structure):
+    _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p),
+                ("ws_gate", c_void_p), ("ws_up", c_void_p), ("ws_down", c_void_p)]
+
+
 class moe_experts_fp8(ctypes.Structure):
     _fields_ = [("w_gate", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p),
                 ("s_gate", c_void_p), ("s_up", c_void_p), ("s_down", c_void_p)]
@@ -97,7 +102,7 @@ def lib() -> ctypes.CDLL:
     L.moe_quantize_fp8_blocks.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p]
     L.moe_backward.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), POINTER(moe_experts),
                                POINTER(moe_shared), c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
-                               c_void_p]
+                               POINTER(moe_weight_grads), c_void_p]
     L.moe_ep_workspace.argtypes = [moe_handle, POINTER(c_void_p)]
     L.moe_ep_set_peers.argtypes = [moe_handle, POINTER(c_void_p)]
     L.moe_ep_ipc_handle.argtypes = [moe_handle, c_void_p]
@@ -201,11 +206,11 @@ def moe_quantize_fp8_blocks(w, batch, rows, cols, q, scale, stream):
     return lib().moe_quantize_fp8_blocks(w, int(batch), int(rows), int(cols), q, scale, stream)
 
 
-def moe_backward(h, x, T, router, experts, shared, K, dh, dx, d_router, d_logit_bias, dgate, stream):
-    """The backward for the input and the router of the last moe_forward; see the header."""
+def moe_backward(h, x, T, router, experts, shared, K, dh, dx, d_router, d_logit_bias, dgate, wgrad, stream):
+    """The backward of the last moe_forward (input, router and, with wgrad, expert weights); see the header."""
     return lib().moe_backward(h, x, int(T), ctypes.byref(router), ctypes.byref(experts),
                               ctypes.byref(shared) if shared is not None else None, int(K), dh, dx, d_router,
-                              d_logit_bias, dgate, stream)
+                              d_logit_bias, dgate, ctypes.byref(wgrad) if wgrad is not None else None, stream)
 
 
 def moe_ep_workspace(h):
@@ -322,11 +327,13 @@ class MoELayer:
             raise MoEError(st, "moe_forward")
         return out if check else (st, out)
 
-    def backward(self, x, K, dh, dx=None, router_grad=False, stream=None):
+    def backward(self, x, K, dh, dx=None, router_grad=False, weight_grads=False, stream=None):
         """Gradients of the last ``forward(x, K)`` for the upstream gradient dh (bf16 [T, d]):
         returns (dx bf16 [T, d], dgate float32 [T, K], d_router float32 [mN, d] or None,
-        d_logit_bias float32 [mN] or None).  ``router_grad`` asks for d_router (and d_logit_bias
-        when the layer has a logit bias)."""
+        d_logit_bias float32 [mN] or None), and with ``weight_grads`` a fifth item: a dict of
+        float32 gradients "w_gate", "w_up", "w_down" (and "ws_*" with shared experts) in the
+        weights' layouts.  ``router_grad`` asks for d_router (and d_logit_bias when the layer has
+        a logit bias)."""
         import torch
         T = x.shape[0]
         dev = x.device
@@ -337,11 +344,23 @@ class MoELayer:
             if router_grad else None
         d_bias = torch.empty(self.cfg.n_routed, dtype=torch.float32, device=dev) \
             if router_grad and self.router.logit_bias else None
+        wg, wgrad = None, None
+        if weight_grads:
+            c = self.cfg
+            N, I, d, Ks, Is = c.n_routed, c.d_ff, c.d_model, c.n_shared, c.d_ff_shared
+            f32 = dict(dtype=torch.float32, device=dev)
+            wg = {"w_gate": torch.empty((N, I, d), **f32), "w_up": torch.empty((N, I, d), **f32),
+                  "w_down": torch.empty((N, d, I), **f32)}
+            if Ks:
+                wg.update(ws_gate=torch.empty((Ks, Is, d), **f32), ws_up=torch.empty((Ks, Is, d), **f32),
+                          ws_down=torch.empty((Ks, d, Is), **f32))
+            wgrad = moe_weight_grads(*(wg[k].data_ptr() if k in wg else None
+                                       for k in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")))
         st = moe_backward(self.h, _ptr(x), T, self.router, self.experts, self.shared, K, _ptr(dh), _ptr(dx),
-                          _ptr(d_router), _ptr(d_bias), _ptr(dgate), _stream_ptr(stream))
+                          _ptr(d_router), _ptr(d_bias), _ptr(dgate), wgrad, _stream_ptr(stream))
         if st != MOE_OK:
             raise MoEError(st, "moe_backward")
-        return dx, dgate, d_router, d_bias
+        return (dx, dgate, d_router, d_bias) + ((wg,) if weight_grads else ())
 
     def set_weights_fp8(self, experts_fp8, shared_fp8=None):
         """FP8 expert weights for forward_fp8: (codes, scales) pairs as quantize_fp8_blocks returns

@@ -344,12 +344,17 @@ moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, i
  *   d_logit_bias float32 [mN] out or NULL: dL/dc = sum_t dz_t (only with a
  *             logit bias: else MOE_ERR_INVALID_ARG)
  *   dgate     float32 [T, K] out or NULL: dL/dg_{t,k} = dh_t . FFN_{Sel_t,k}(u_t)
+ *   wgrad     NULL, or the expert weights' gradients (every pointer set; the
+ *             shared ones when K_s > 0), float32 in the weights' layouts:
+ *             dW_down,e = sum over e's rows of (g dh) m^T, dW_gate,e = sum of
+ *             da u^T, dW_up,e = sum of db u^T (m = SiLU(a) b, da, db as below);
+ *             the shared experts' the same with g = 1 over every token
  * where dz is dL/dz of the affinity logits (softmax: dz = s (ds - s . ds),
  * ds_i the dgate of the slot that chose expert i, 0 for the others; sigmoid:
  * ds_k = (dgate_k - g . dgate) / sum of the chosen s, dz = ds s (1 - s) on the
- * chosen experts, 0 elsewhere).  The debug flags leave the same terms out as
- * in the forward.  The expert and shared weights' own gradients are not
- * computed.
+ * chosen experts, 0 elsewhere); for a routed row, da = g dm b SiLU'(a) and
+ * db = g dm SiLU(a) with dm = W_down^T dh.  The debug flags leave the same
+ * terms out as in the forward (a left-out part's weight gradients are zero).
  *
  * Asynchronous on `stream`.  The first call allocates the backward's buffers
  * (a K-major copy of the expert weights, rewritten by every call, and
@@ -359,9 +364,18 @@ moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, i
  * MOE_ERR_INVALID_ARG; an expert-parallel handle -> MOE_ERR_UNSUPPORTED; no
  * memory for the buffers -> MOE_ERR_NOMEM.  Overwrites the forward's
  * intermediate rows (H, Y, Hs, Ys) in the workspace. */
+typedef struct moe_weight_grads {
+  float* w_gate;  /* [mN, I, d] */
+  float* w_up;    /* [mN, I, d] */
+  float* w_down;  /* [mN, d, I] */
+  float* ws_gate; /* [K_s, I_s, d] */
+  float* ws_up;   /* [K_s, I_s, d] */
+  float* ws_down; /* [K_s, d, I_s] */
+} moe_weight_grads;
+
 moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router* router, const moe_experts* experts,
                         const moe_shared* shared, int32_t K, const void* dh, void* dx, float* d_router,
-                        float* d_logit_bias, float* dgate, void* stream);
+                        float* d_logit_bias, float* dgate, const moe_weight_grads* wgrad, void* stream);
 
 /* Expert parallelism (DeepSeek-V3 technical report summary, section 3.1
  * "Compute Clusters": the routed experts of a layer spread over many GPUs;

@@ -13,6 +13,14 @@ Comparison rules (the tolerances are written in the asserts below):
   (2^-9 relative each, through sums of I and d terms) and each of the K rows
   before the k-ordered sum, as in the forward.
 * d_router = dz^T u and d_logit_bias = sum_t dz: the term rule.
+* the expert weights' gradients, per tensor: RMS(gpu - oracle) <= 1e-2 *
+  RMS(oracle) and max |gpu - oracle| <= 2e-2 * max |oracle|.  Each element is a
+  sum over an expert's rows of products of bf16-rounded operands (g dh, m, da,
+  db; u is exact), so its error is up to about 2^-8 of the sum of the terms'
+  magnitudes; the largest elements (sums of mostly same-signed terms, up to
+  ~30x the tensor's RMS) keep that relative error, which a bound relative to
+  the RMS would not admit.  Against an oracle that rounds the same operands to
+  bf16 the GPU agrees to ~1e-5 of the RMS.
 Tokens at a near-tie of the selection (the forward tests' exemption) would
 route differently on the two sides and change dE; the seeded shapes have none,
 which the tests assert.  Inside a token's K experts two nearly equal keys may
@@ -59,6 +67,16 @@ def _compare(got, want, what, tol):
     return err / rms, rms_err / rms
 
 
+def _compare_wgrad(got, want, what):
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    top = float(np.max(np.abs(want)))
+    err = float(np.max(np.abs(got - want)))
+    rms_err = float(np.sqrt(np.mean((got - want) ** 2)))
+    assert np.isfinite(got).all(), f"{what}: non-finite"
+    assert err <= 2e-2 * top, f"{what}: max|diff| {err:.3e} > 2e-2 * max|oracle| {top:.3e}"
+    assert rms_err <= 1e-2 * rms, f"{what}: rms diff {rms_err:.3e} > 1e-2 * rms {rms:.3e}"
+
+
 def _oracle_dgate(shape, host, dh, idx, rows=None):
     """dL/dg = dh . FFN_e(u) per (token, slot) for the experts idx [n, K], from the oracle's FFN."""
     u = O.f64(host["x"]) if rows is None else O.f64(host["x"])[rows]
@@ -77,10 +95,10 @@ def _same_expert_sets(gpu_idx, ref_idx):
     np.testing.assert_array_equal(np.sort(gpu_idx, axis=1), np.sort(ref_idx, axis=1))
 
 
-def _run(shape, dev, flags, dh, router_grad=True):
+def _run(shape, dev, flags, dh, router_grad=True, weight_grads=False):
     layer = H.make_layer(shape, dev, flags=flags)
     H.run(layer, dev["x"], shape.K)
-    res = layer.backward(dev["x"], shape.K, dh, router_grad=router_grad)
+    res = layer.backward(dev["x"], shape.K, dh, router_grad=router_grad, weight_grads=weight_grads)
     assert layer.status() == B.MOE_OK, B.status_string(layer.status())
     idx = layer.routing(shape.T, shape.K)[0].cpu().numpy()
     layer.close()
@@ -98,8 +116,14 @@ def test_backward_matches_the_oracle(name):
     grads = OB.moe_backward(host["x"], host["router"], shape.K, (host["w_gate"], host["w_up"], host["w_down"]),
                             H.oracle_shared(shape, host), dh=dh_host, gate_kind=shape.gate,
                             logit_bias=host["logit_bias"], select_bias=host["select_bias"])
-    dx, dgate, d_router, d_bias, idx = _run(shape, dev, 0, dh)
+    dx, dgate, d_router, d_bias, wg, idx = _run(shape, dev, 0, dh, weight_grads=True)
     _same_expert_sets(idx, route.idx)
+    for key, want in (("w_gate", grads.d_w_gate), ("w_up", grads.d_w_up), ("w_down", grads.d_w_down),
+                      ("ws_gate", grads.d_ws_gate), ("ws_up", grads.d_ws_up), ("ws_down", grads.d_ws_down)):
+        if want is None:
+            assert key not in wg
+            continue
+        _compare_wgrad(wg[key].cpu().numpy().astype(np.float64), want, f"{name} d{key}")
     _compare(_rows(dgate), _oracle_dgate(shape, host, dh_host, idx), f"{name} dgate", 2e-2)
     _compare(_rows(dx), grads.du, f"{name} dx", 2e-2)
     _compare(d_router.cpu().numpy().astype(np.float64), grads.d_router, f"{name} d_router", 5e-2)
