@@ -184,242 +184,134 @@ __global__ void __launch_bounds__(256) dg_reduce_kernel(const float* dg_part, co
 }
 
 // ---------------------------------------------------------------------------
-// Router backward on 32-token blocks: recompute z = x E^T (+ c) in fp32, the
-// affinities s, dz from the gates' gradient, and dx_router = dz E.
+// The router's backward between its three GEMMs (z = x E^T, dz E and dz^T x,
+// on the tensor cores): per token, the affinities from the recomputed logits
+// z (+ c) and dz from the gates' gradient; a warp per token.  Writes dz in
+// fp32 [T, N] (for d(logit bias)) and in bf16 [T, Npad] (the GEMMs' operand,
+// zero in the padding columns).
 // ---------------------------------------------------------------------------
-constexpr int kRbTokens = 32;
-constexpr int kRbCols = 64;  // columns of x and E per staged chunk
-
-struct RouterBwdArgs {
-  int T, N, d, K, sigmoid;
-  const __nv_bfloat16* x;    // [T, d]
-  const __nv_bfloat16* e;    // [N, d]
+struct RouterDzArgs {
+  int T, N, Npad, K, sigmoid;
+  const float* z;            // [T, Npad] logits x E^T (without the logit bias)
   const float* logit_bias;   // [N] or nullptr (softmax)
   const int32_t* idx;        // [T, K]
   const float* dgate;        // [T, K]
   float* dz;                 // [T, N] out
-  float* dx_router;          // [T, d] out
+  __nv_bfloat16* dzb;        // [T, Npad] out
 };
 
-__host__ __device__ constexpr size_t router_bwd_smem_bytes(int N) {
-  // E chunk [N][65], x chunk [32][65], z / dz [32][N + 1]
-  return (static_cast<size_t>(N) * (kRbCols + 1) + kRbTokens * (kRbCols + 1) + kRbTokens * (N + 1)) * 4;
-}
-
-__global__ void __launch_bounds__(256) router_bwd_kernel(RouterBwdArgs a) {
-  extern __shared__ float rb_smem[];
-  const int N = a.N, d = a.d;
-  float* es = rb_smem;                          // [N][65]
-  float* xs = es + N * (kRbCols + 1);           // [32][65]
-  float* zs = xs + kRbTokens * (kRbCols + 1);   // [32][N + 1]
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int t0 = blockIdx.x * kRbTokens;
-  const int nt = min(kRbTokens, a.T - t0);
-  // ---- z: thread (tg, ig) accumulates tokens 4 tg .. + 3 and experts ig + 32 j ----
-  const int tg = tid & 7, ig = tid >> 3;
-  float acc[4][8];
+__global__ void __launch_bounds__(256) router_dz_kernel(RouterDzArgs a) {
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (t >= a.T) return;
+  const int N = a.N, K = a.K;
+  const float* zr = a.z + static_cast<size_t>(t) * a.Npad;
+  float zv[8];  // experts lane + 32 j
 #pragma unroll
-  for (int m = 0; m < 4; ++m)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[m][j] = 0.f;
-  for (int c0 = 0; c0 < d; c0 += kRbCols) {
-    __syncthreads();
-    for (int i = tid; i < N * (kRbCols / 8); i += 256) {  // 8 columns per 16-byte load
-      const int r = i / (kRbCols / 8), cc = (i - r * (kRbCols / 8)) * 8;
-      const uint4 v = c0 + cc < d ? __ldg(reinterpret_cast<const uint4*>(a.e + static_cast<size_t>(r) * d + c0 + cc))
-                                  : make_uint4(0u, 0u, 0u, 0u);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        es[r * (kRbCols + 1) + cc + 2 * j] = bf16lo(w[j]);
-        es[r * (kRbCols + 1) + cc + 2 * j + 1] = bf16hi(w[j]);
-      }
-    }
-    for (int i = tid; i < kRbTokens * (kRbCols / 8); i += 256) {
-      const int r = i / (kRbCols / 8), cc = (i - r * (kRbCols / 8)) * 8;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < nt && c0 + cc < d) v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + r) * d + c0 + cc));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        xs[r * (kRbCols + 1) + cc + 2 * j] = bf16lo(w[j]);
-        xs[r * (kRbCols + 1) + cc + 2 * j + 1] = bf16hi(w[j]);
-      }
-    }
-    __syncthreads();
-#pragma unroll 4
-    for (int c = 0; c < kRbCols; ++c) {
-      float xv[4];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) xv[m] = xs[(4 * tg + m) * (kRbCols + 1) + c];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = ig + 32 * j;
-        if (i < N) {
-          const float ev = es[i * (kRbCols + 1) + c];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) acc[m][j] = fmaf(xv[m], ev, acc[m][j]);
-        }
-      }
-    }
+  for (int j = 0; j < 8; ++j) {
+    const int i = lane + 32 * j;
+    zv[j] = i < N ? zr[i] + (a.logit_bias ? a.logit_bias[i] : 0.f) : -INFINITY;
   }
-  __syncthreads();
+  int ki[8];
+  float kg[8];
 #pragma unroll
-  for (int m = 0; m < 4; ++m)
+  for (int k = 0; k < 8; ++k) {
+    ki[k] = k < K ? a.idx[static_cast<size_t>(t) * K + k] : -1;
+    kg[k] = k < K ? a.dgate[static_cast<size_t>(t) * K + k] : 0.f;
+  }
+  float dzv[8];
+  if (!a.sigmoid) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx = fmaxf(mx, zv[j]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sv[8], sum = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int i = ig + 32 * j;
-      if (i < N) zs[(4 * tg + m) * (N + 1) + i] = acc[m][j] + (a.logit_bias ? a.logit_bias[i] : 0.f);
+      sv[j] = lane + 32 * j < N ? __expf(zv[j] - mx) : 0.f;
+      sum += sv[j];
     }
-  __syncthreads();
-  // ---- s and dz: a warp per token ----
-  for (int tl = warp; tl < nt; tl += 8) {
-    float* z = zs + tl * (N + 1);
-    const int t = t0 + tl;
-    if (!a.sigmoid) {
-      float mx = -INFINITY;
-      for (int i = lane; i < N; i += 32) mx = fmaxf(mx, z[i]);
 #pragma unroll
-      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.f;
-      for (int i = lane; i < N; i += 32) {
-        const float ex = __expf(z[i] - mx);
-        z[i] = ex;
-        sum += ex;
-      }
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.f / sum;
+    // s . ds = sum over the chosen slots of s_i dg_k (each chosen expert once)
+    float sds = 0.f;
 #pragma unroll
-      for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      const float inv = 1.f / sum;
-      __syncwarp();
-      // s . ds = sum over the chosen slots of s_i dg_k
-      float sds = 0.f;
-      for (int k = 0; k < a.K; ++k) {
-        const int i = a.idx[static_cast<size_t>(t) * a.K + k];
-        sds += z[i] * inv * a.dgate[static_cast<size_t>(t) * a.K + k];
-      }
-      __syncwarp();
-      for (int i = lane; i < N; i += 32) {
-        float ds = 0.f;
-        for (int k = 0; k < a.K; ++k)
-          if (a.idx[static_cast<size_t>(t) * a.K + k] == i) ds = a.dgate[static_cast<size_t>(t) * a.K + k];
-        const float s = z[i] * inv;
-        z[i] = s * (ds - sds);
-      }
-    } else {
-      // g_k = s_k / S over the chosen; ds_k = (dg_k - g . dg) / S; dz = ds s (1 - s) there, 0 elsewhere
-      float S = 0.f, gdg = 0.f;
-      for (int k = 0; k < a.K; ++k) S += 1.f / (1.f + __expf(-z[a.idx[static_cast<size_t>(t) * a.K + k]]));
-      for (int k = 0; k < a.K; ++k) {
-        const float s = 1.f / (1.f + __expf(-z[a.idx[static_cast<size_t>(t) * a.K + k]]));
-        gdg += s / S * a.dgate[static_cast<size_t>(t) * a.K + k];
-      }
-      __syncwarp();
-      for (int i = lane; i < N; i += 32) {
-        float dzi = 0.f;
-        for (int k = 0; k < a.K; ++k)
-          if (a.idx[static_cast<size_t>(t) * a.K + k] == i) {
-            const float s = 1.f / (1.f + __expf(-z[i]));
-            dzi = (a.dgate[static_cast<size_t>(t) * a.K + k] - gdg) / S * s * (1.f - s);
-          }
-        z[i] = dzi;
-      }
+    for (int j = 0; j < 8; ++j) {
+      const int i = lane + 32 * j;
+      sv[j] *= inv;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (ki[k] == i) sds += sv[j] * kg[k];
     }
-    __syncwarp();
-    for (int i = lane; i < N; i += 32) a.dz[static_cast<size_t>(t) * N + i] = z[i];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sds += __shfl_xor_sync(0xffffffffu, sds, o);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = lane + 32 * j;
+      float ds = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (ki[k] == i) ds = kg[k];
+      dzv[j] = sv[j] * (ds - sds);
+    }
+  } else {
+    // g_k = s_k / S over the chosen; ds_k = (dg_k - g . dg) / S; dz = ds s (1 - s) there, 0 elsewhere
+    float S = 0.f, sdg = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = lane + 32 * j;
+      const float s = 1.f / (1.f + __expf(-zv[j]));
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (ki[k] == i) {
+          S += s;
+          sdg += s * kg[k];
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      S += __shfl_xor_sync(0xffffffffu, S, o);
+      sdg += __shfl_xor_sync(0xffffffffu, sdg, o);
+    }
+    const float gdg = sdg / S;  // sum over the chosen of g_l dg_l
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = lane + 32 * j;
+      const float s = 1.f / (1.f + __expf(-zv[j]));
+      float v = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (ki[k] == i) v = (kg[k] - gdg) / S * s * (1.f - s);
+      dzv[j] = v;
+    }
   }
-  __syncthreads();
-  // ---- dx_router = dz E: thread (row tl = tid / 8, 8 columns (tid % 8) * 8) per 64-column chunk ----
-  const int tl = tid >> 3, cg = (tid & 7) * 8;
-  for (int c0 = 0; c0 < d; c0 += kRbCols) {
-    __syncthreads();
-    for (int i = tid; i < N * (kRbCols / 8); i += 256) {
-      const int r = i / (kRbCols / 8), cc = (i - r * (kRbCols / 8)) * 8;
-      const uint4 v = c0 + cc < d ? __ldg(reinterpret_cast<const uint4*>(a.e + static_cast<size_t>(r) * d + c0 + cc))
-                                  : make_uint4(0u, 0u, 0u, 0u);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  float* dzr = a.dz + static_cast<size_t>(t) * N;
+  __nv_bfloat16* dbr = a.dzb + static_cast<size_t>(t) * a.Npad;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        es[r * (kRbCols + 1) + cc + 2 * j] = bf16lo(w[j]);
-        es[r * (kRbCols + 1) + cc + 2 * j + 1] = bf16hi(w[j]);
-      }
-    }
-    __syncthreads();
-    float o[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) o[j] = 0.f;
-    const float* z = zs + tl * (N + 1);
-    for (int i = 0; i < N; ++i) {
-      const float dzi = z[i];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = fmaf(dzi, es[i * (kRbCols + 1) + cg + j], o[j]);
-    }
-    if (tl < nt && c0 + cg < d) {
-      float4* q = reinterpret_cast<float4*>(a.dx_router + static_cast<size_t>(t0 + tl) * d + c0 + cg);
-      q[0] = make_float4(o[0], o[1], o[2], o[3]);
-      q[1] = make_float4(o[4], o[5], o[6], o[7]);
-    }
+  for (int j = 0; j < 8; ++j) {
+    const int i = lane + 32 * j;
+    if (i < N) dzr[i] = dzv[j];
+    if (i < a.Npad) dbr[i] = __float2bfloat16_rn(i < N ? dzv[j] : 0.f);
   }
 }
 
-// ---------------------------------------------------------------------------
-// dE = dz^T x (and d(logit bias) = sum_t dz) in fixed order: CTA (column
-// block of 128, 16 experts, token segment) sums its segment's tokens in
-// ascending order into part[seg]; router_de_reduce_kernel adds the segments
-// in ascending order.
-// ---------------------------------------------------------------------------
-constexpr int kDeCols = 128;
-constexpr int kDeExperts = 16;
+// d(logit bias)_i = sum over t (ascending) of dz[t, i]; a thread per expert
+__global__ void __launch_bounds__(256) column_sum_kernel(const float* dz, int T, int N, float* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  float s = 0.f;
+  for (int t = 0; t < T; ++t) s += dz[static_cast<size_t>(t) * N + i];
+  out[i] = s;
+}
 
-struct RouterDeArgs {
-  int T, N, d, seg_tokens;
-  const float* dz;           // [T, N]
-  const __nv_bfloat16* x;    // [T, d]
-  float* part;               // [segments][N][d]
-  float* part_bias;          // [segments][N] or nullptr
-};
-
-__global__ void __launch_bounds__(256) router_de_kernel(RouterDeArgs a) {
-  __shared__ float dzs[kRbTokens][kDeExperts];
-  __shared__ float xs[kRbTokens][kDeCols];
-  const int c0 = blockIdx.x * kDeCols, i0 = blockIdx.y * kDeExperts, seg = blockIdx.z;
-  const int tid = threadIdx.x;
-  const int il = tid >> 4, cl = (tid & 15) * 8;  // expert i0 + il, columns c0 + cl .. + 7
-  const int tb = seg * a.seg_tokens, te = min(a.T, tb + a.seg_tokens);
-  float o[8], ob = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) o[j] = 0.f;
-  for (int t0 = tb; t0 < te; t0 += kRbTokens) {
-    __syncthreads();
-    for (int i = tid; i < kRbTokens * kDeExperts; i += 256) {
-      const int r = i / kDeExperts, e = i - r * kDeExperts;
-      dzs[r][e] = (t0 + r < te && i0 + e < a.N) ? a.dz[static_cast<size_t>(t0 + r) * a.N + i0 + e] : 0.f;
-    }
-    for (int i = tid; i < kRbTokens * (kDeCols / 8); i += 256) {
-      const int r = i / (kDeCols / 8), cc = (i - r * (kDeCols / 8)) * 8;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (t0 + r < te && c0 + cc < a.d) v = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + r) * a.d + c0 + cc));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        xs[r][cc + 2 * j] = bf16lo(w[j]);
-        xs[r][cc + 2 * j + 1] = bf16hi(w[j]);
-      }
-    }
-    __syncthreads();
-    for (int r = 0; r < kRbTokens; ++r) {
-      const float dzi = dzs[r][il];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = fmaf(dzi, xs[r][cl + j], o[j]);
-      ob += dzi;
-    }
+// the K ranges of a GEMM split into `n` segments of `seg` rows (the last one shorter) over [0, total)
+__global__ void fill_segments_kernel(int32_t* k_start, int32_t* k_count, int n, int seg, int total) {
+  const int i = threadIdx.x;
+  if (i < n) {
+    k_start[i] = i * seg;
+    k_count[i] = min(seg, total - i * seg);
   }
-  const int i = i0 + il;
-  if (i < a.N && c0 + cl < a.d) {
-    float4* q = reinterpret_cast<float4*>(a.part + (static_cast<size_t>(seg) * a.N + i) * a.d + c0 + cl);
-    q[0] = make_float4(o[0], o[1], o[2], o[3]);
-    q[1] = make_float4(o[4], o[5], o[6], o[7]);
-  }
-  if (a.part_bias && blockIdx.x == 0 && cl == 0 && i < a.N) a.part_bias[static_cast<size_t>(seg) * a.N + i] = ob;
 }
 
 __global__ void __launch_bounds__(256) router_de_reduce_kernel(const float* part, int segments, size_t n,

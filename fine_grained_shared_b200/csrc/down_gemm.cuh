@@ -95,8 +95,9 @@ struct GemmArgs {
   int kg_a_row_step;
   int kg_bz_step;
   int kg_split;
-  float* kg_out;               // [groups][kg_split][n_limit]
-  float* kg_out2;              // [groups][kg_M - kg_split][n_limit]
+  int kg_ld;                   // output row stride (>= n_limit, a multiple of 16)
+  float* kg_out;               // [groups][kg_split][kg_ld]
+  float* kg_out2;              // [groups][kg_M - kg_split][kg_ld]
 };
 
 __host__ __device__ constexpr size_t gemm_smem_bytes() {
@@ -374,8 +375,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         float* orow = nullptr;
         if (m < a.kg_M)
           orow = m < a.kg_split
-                     ? a.kg_out + (static_cast<size_t>(g) * a.kg_split + m) * a.n_limit
-                     : a.kg_out2 + (static_cast<size_t>(g) * (a.kg_M - a.kg_split) + (m - a.kg_split)) * a.n_limit;
+                     ? a.kg_out + (static_cast<size_t>(g) * a.kg_split + m) * a.kg_ld
+                     : a.kg_out2 + (static_cast<size_t>(g) * (a.kg_M - a.kg_split) + (m - a.kg_split)) * a.kg_ld;
 #pragma unroll 1
         for (int cc = 0; cc < kGemmBN; cc += 16) {
           uint32_t vr[16];

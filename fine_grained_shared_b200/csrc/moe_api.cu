@@ -195,9 +195,12 @@ Layout make_layout(const moe_config& c) {
 // The backward's buffers: K-major copies of the expert weights for its two data-gradient GEMMs, the
 // recompute's [da | db] rows, the gate gradient's partial sums, the router's dz and dz E, and the
 // per-segment partial sums of dE.
-constexpr int kDeMaxSegments = 8;
+constexpr int kDeMaxSegments = 16;
 struct BwdLayout {
-  size_t wdT, wguT, swdT, swguT, dab, dabs, dg_part, dz, dxr, de_part, de_bias_part, dgate;
+  size_t wdT, wguT, swdT, swguT, dab, dabs, dg_part, dz, dxr, de_part, dgate;
+  // the router's GEMM operands: logits, dz in bf16 (and transposed), E transposed, K-range tables
+  size_t zf, dzb, dzT, ET, rt_kstart, rt_kcount;
+  int64_t Npad;
   // the weight gradients' operands: activations transposed (rows of the forward as columns)
   size_t dyT, xpermT, mT, dabT, dhT, xT, msT, dabsT, sh_kstart, sh_kcount, total;
   int64_t Pt;  // row count of the transposed routed activations (the forward's rows, padded to 64)
@@ -223,8 +226,14 @@ BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
   B.dz = take(size_t(Tm) * N * 4);
   B.dxr = take(size_t(Tm) * d * 4);
   B.de_part = take(size_t(kDeMaxSegments) * N * d * 4);
-  B.de_bias_part = take(size_t(kDeMaxSegments) * N * 4);
   B.dgate = take(size_t(Tm) * Km * 4);
+  B.Npad = (N + 15) / 16 * 16;
+  B.zf = take(size_t(Tm) * B.Npad * 4);
+  B.dzb = take(size_t(Tm) * B.Npad * 2);
+  B.dzT = take(size_t(B.Npad) * L.Tpad * 2);
+  B.ET = take(size_t(d) * B.Npad * 2);
+  B.rt_kstart = take(kDeMaxSegments * 4);
+  B.rt_kcount = take(kDeMaxSegments * 4);
   B.Pt = (L.P + 63) / 64 * 64;
   B.dyT = take(size_t(d) * B.Pt * 2);
   B.xpermT = take(size_t(d) * B.Pt * 2);
@@ -337,7 +346,8 @@ struct moe_ctx {
   uint8_t* bws = nullptr;
   CUtensorMap tm_b_dhperm, tm_b_wdT, tm_b_swdT, tm_b_dab, tm_b_wguT, tm_b_dabs, tm_b_swguT;
   CUtensorMap tm_b_dyT, tm_b_xpermT, tm_b_mT, tm_b_dabT, tm_b_dhT, tm_b_xT, tm_b_msT, tm_b_dabsT;
-  MapCache tm_b_dh;
+  CUtensorMap tm_b_dzb, tm_b_ET, tm_b_dzT;
+  MapCache tm_b_dh, tm_b_E;
 
   template <typename T>
   T* at(size_t off) const {
@@ -436,9 +446,6 @@ cudaError_t set_kernel_attrs() {
   if ((e = cudaFuncSetAttribute(gateup_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, us))) return e;
   const int gs = static_cast<int>(gemm_smem_bytes());
   if ((e = cudaFuncSetAttribute(down_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gs))) return e;
-  if ((e = cudaFuncSetAttribute(router_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(router_bwd_smem_bytes(kMaxRouted)))))
-    return e;
   if ((e = cudaFuncSetAttribute(decode_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(ffn_smem_bytes()))))
     return e;
@@ -1636,6 +1643,9 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
   ok = ok && encode_bf16(&h->tm_b_xpermT, h->bws + B.xpermT, 1, d, B.Pt, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_dhT, h->bws + B.dhT, 1, d, L.Tpad, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_xT, h->bws + B.xT, 1, d, L.Tpad, kBoxRowsB, 3);
+  ok = ok && encode_bf16(&h->tm_b_dzb, h->bws + B.dzb, 1, c.max_tokens, B.Npad, kBoxRowsA, 2);
+  ok = ok && encode_bf16(&h->tm_b_ET, h->bws + B.ET, 1, d, B.Npad, kBoxRowsB, 3);
+  ok = ok && encode_bf16(&h->tm_b_dzT, h->bws + B.dzT, 1, B.Npad, L.Tpad, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_wdT, h->bws + B.wdT, N, I, d, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_dab, h->bws + B.dab, 1, L.P, 2 * I, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_wguT, h->bws + B.wguT, N, d, 2 * I, kBoxRowsB, 3);
@@ -1705,6 +1715,29 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   const bool residual = !(c.flags & MOE_FLAG_NO_RESIDUAL);
   auto bw = [&](size_t off) { return h->bws + off; };
   h->last_stream = s0;
+  // a GEMM in the per-group mode of down_gemm_kernel (fp32 out, rows >= split into out2)
+  auto kg_gemm = [&](const CUtensorMap& A, const CUtensorMap& Bm, int groups, const int32_t* kstart,
+                     const int32_t* kcount, int M, int a_step, int bz_step, int split, int Ncols, int ld, float* out,
+                     float* out2) {
+    GemmArgs k{};
+    k.kg_groups = groups;
+    k.kg_k_start = kstart;
+    k.kg_k_count = kcount;
+    k.kg_M = M;
+    k.kg_m_tiles = ceil_div(M, kGemmBM);
+    k.kg_a_row_step = a_step;
+    k.kg_bz_step = bz_step;
+    k.kg_split = split;
+    k.kg_ld = ld;
+    k.kg_out = out;
+    k.kg_out2 = out2;
+    k.n_tiles = ceil_div(Ncols, kGemmBN);
+    k.n_limit = Ncols;
+    k.err = h->at<uint32_t>(L.err);
+    k.timeout_ns = kTimeoutNs;
+    const int tiles = groups * k.kg_m_tiles * k.n_tiles;
+    return launch_down(std::min(h->max_pairs, tiles), s0, false, A, Bm, A, Bm, k);
+  };
 
   // descriptors of the caller's pointers
   bool ok = refresh(h->tm_x, x, T, 1, T, d, kGuBoxRowsA, 2);
@@ -1895,35 +1928,15 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   }
   // ---- the expert weights' gradients: per expert, sums over its rows (GEMMs with K = the rows) ----
   if (wgrad) {
-    auto kg_gemm = [&](const CUtensorMap& A, const CUtensorMap& Bm, int groups, const int32_t* kstart,
-                       const int32_t* kcount, int M, int a_step, int bz_step, int split, int Ncols, float* out,
-                       float* out2) {
-      GemmArgs k{};
-      k.kg_groups = groups;
-      k.kg_k_start = kstart;
-      k.kg_k_count = kcount;
-      k.kg_M = M;
-      k.kg_m_tiles = ceil_div(M, kGemmBM);
-      k.kg_a_row_step = a_step;
-      k.kg_bz_step = bz_step;
-      k.kg_split = split;
-      k.kg_out = out;
-      k.kg_out2 = out2;
-      k.n_tiles = ceil_div(Ncols, kGemmBN);
-      k.n_limit = Ncols;
-      k.err = h->at<uint32_t>(L.err);
-      k.timeout_ns = kTimeoutNs;
-      const int tiles = groups * k.kg_m_tiles * k.n_tiles;
-      return launch_down(std::min(h->max_pairs, tiles), s0, false, A, Bm, A, Bm, k);
-    };
     cudaError_t ke = cudaSuccess;
     if (do_routed) {
       const int32_t* ks = h->at<int32_t>(L.row_start);
       const int32_t* kc = h->at<int32_t>(L.counts);
-      ke = kg_gemm(h->tm_b_dyT, h->tm_b_mT, (int)N, ks, kc, (int)d, 0, 0, (int)d, (int)I, wgrad->w_down, nullptr);
+      ke = kg_gemm(h->tm_b_dyT, h->tm_b_mT, (int)N, ks, kc, (int)d, 0, 0, (int)d, (int)I, (int)I, wgrad->w_down,
+                   nullptr);
       if (ke == cudaSuccess)
-        ke = kg_gemm(h->tm_b_dabT, h->tm_b_xpermT, (int)N, ks, kc, (int)(2 * I), 0, 0, (int)I, (int)d, wgrad->w_gate,
-                     wgrad->w_up);
+        ke = kg_gemm(h->tm_b_dabT, h->tm_b_xpermT, (int)N, ks, kc, (int)(2 * I), 0, 0, (int)I, (int)d, (int)d,
+                     wgrad->w_gate, wgrad->w_up);
     } else {
       const size_t wb = size_t(N) * I * d * 4;
       if (cudaMemsetAsync(wgrad->w_gate, 0, wb, s0) != cudaSuccess ||
@@ -1934,10 +1947,11 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     if (Ks > 0 && do_shared && ke == cudaSuccess) {
       const int32_t* ks = reinterpret_cast<const int32_t*>(bw(B.sh_kstart));
       const int32_t* kc = reinterpret_cast<const int32_t*>(bw(B.sh_kcount));
-      ke = kg_gemm(h->tm_b_dhT, h->tm_b_msT, (int)Ks, ks, kc, (int)d, 0, 1, (int)d, (int)Is, wgrad->ws_down, nullptr);
+      ke = kg_gemm(h->tm_b_dhT, h->tm_b_msT, (int)Ks, ks, kc, (int)d, 0, 1, (int)d, (int)Is, (int)Is,
+                   wgrad->ws_down, nullptr);
       if (ke == cudaSuccess)
         ke = kg_gemm(h->tm_b_dabsT, h->tm_b_xT, (int)Ks, ks, kc, (int)(2 * Is), (int)(2 * Is), 0, (int)Is, (int)d,
-                     wgrad->ws_gate, wgrad->ws_up);
+                     (int)d, wgrad->ws_gate, wgrad->ws_up);
     } else if (Ks > 0 && ke == cudaSuccess) {
       const size_t wb = size_t(Ks) * Is * d * 4;
       if (cudaMemsetAsync(wgrad->ws_gate, 0, wb, s0) != cudaSuccess ||
@@ -1953,38 +1967,77 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   if (do_routed) {
     dg_reduce_kernel<<<ceil_div(TK, 256), 256, 0, s0>>>(reinterpret_cast<const float*>(bw(B.dg_part)), slot_of, TK,
                                                          ceil_div(I, kGuBN / 2), dg);
-    RouterBwdArgs rb{};
-    rb.T = (int)T;
-    rb.N = (int)N;
-    rb.d = (int)d;
-    rb.K = K;
-    rb.sigmoid = sigmoid ? 1 : 0;
-    rb.x = static_cast<const __nv_bfloat16*>(x);
-    rb.e = static_cast<const __nv_bfloat16*>(router->weight);
-    rb.logit_bias = router->logit_bias;
-    rb.idx = h->at<int32_t>(L.idx);
-    rb.dgate = dg;
-    rb.dz = reinterpret_cast<float*>(bw(B.dz));
-    rb.dx_router = dxr = reinterpret_cast<float*>(bw(B.dxr));
-    router_bwd_kernel<<<ceil_div(T, kRbTokens), 256, router_bwd_smem_bytes((int)N), s0>>>(rb);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-    if (d_router || d_logit_bias) {
-      const int segs = (int)std::max<int64_t>(1, std::min<int64_t>(kDeMaxSegments, T / 256));
-      RouterDeArgs de{};
-      de.T = (int)T;
-      de.N = (int)N;
-      de.d = (int)d;
-      de.seg_tokens = ceil_div(ceil_div(T, segs), kRbTokens) * kRbTokens;
-      de.dz = rb.dz;
-      de.x = rb.x;
-      de.part = reinterpret_cast<float*>(bw(B.de_part));
-      de.part_bias = d_logit_bias ? reinterpret_cast<float*>(bw(B.de_bias_part)) : nullptr;
-      router_de_kernel<<<dim3(ceil_div(d, kDeCols), ceil_div(N, kDeExperts), segs), 256, 0, s0>>>(de);
-      if (d_router)
-        router_de_reduce_kernel<<<ceil_div(N * d, 256), 256, 0, s0>>>(de.part, segs, size_t(N) * d, d_router);
-      if (d_logit_bias)
-        router_de_reduce_kernel<<<ceil_div(N, 256), 256, 0, s0>>>(de.part_bias, segs, size_t(N), d_logit_bias);
+    // the router's three contractions on the tensor cores (the GEMM's per-group mode, one group
+    // or a K split into segments): z = x E^T, dx_router = dz E, dE = dz^T x
+    if (!refresh(h->tm_b_E, router->weight, 0, 1, N, d, kBoxRowsB, 3)) return MOE_ERR_CUDA;
+    int32_t* ks = reinterpret_cast<int32_t*>(bw(B.rt_kstart));
+    int32_t* kc = reinterpret_cast<int32_t*>(bw(B.rt_kcount));
+    const int Np = (int)B.Npad;
+    fill_segments_kernel<<<1, 32, 0, s0>>>(ks, kc, 1, (int)d, (int)d);
+    if (kg_gemm(h->tm_x.map, h->tm_b_E.map, 1, ks, kc, (int)T, 0, 0, (int)T, (int)N, Np,
+                reinterpret_cast<float*>(bw(B.zf)), nullptr) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    RouterDzArgs rz{};
+    rz.T = (int)T;
+    rz.N = (int)N;
+    rz.Npad = Np;
+    rz.K = K;
+    rz.sigmoid = sigmoid ? 1 : 0;
+    rz.z = reinterpret_cast<const float*>(bw(B.zf));
+    rz.logit_bias = router->logit_bias;
+    rz.idx = h->at<int32_t>(L.idx);
+    rz.dgate = dg;
+    rz.dz = reinterpret_cast<float*>(bw(B.dz));
+    rz.dzb = reinterpret_cast<__nv_bfloat16*>(bw(B.dzb));
+    router_dz_kernel<<<ceil_div(T * 32, 256), 256, 0, s0>>>(rz);
+    // E^T [d][Npad] (zero columns past mN)
+    RowTransposeArgs rt{};
+    rt.src = static_cast<const __nv_bfloat16*>(router->weight);
+    rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.ET));
+    rt.R = Np;
+    rt.src_rows = (int)N;
+    rt.C = (int)d;
+    rt.dst_ld = Np;
+    rt.G = 0;
+    rt.row_limit = (int)N;
+    transpose_rows_kernel<<<dim3(ceil_div(d, 64), ceil_div(Np, 64)), 256, 0, s0>>>(rt);
+    fill_segments_kernel<<<1, 32, 0, s0>>>(ks + 1, kc + 1, 1, (int)N, (int)N);
+    dxr = reinterpret_cast<float*>(bw(B.dxr));
+    if (kg_gemm(h->tm_b_dzb, h->tm_b_ET, 1, ks + 1, kc + 1, (int)T, 0, 0, (int)T, (int)d, (int)d, dxr, nullptr) !=
+        cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (d_router) {
+      // dz^T [Npad][Tpad] and (unless the shared weights' gradients made it) x^T, then dE over
+      // token segments summed in segment order
+      RowTransposeArgs t2{};
+      t2.src = rz.dzb;
+      t2.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dzT));
+      t2.R = (int)L.Tpad;
+      t2.src_rows = (int)T;
+      t2.C = Np;
+      t2.dst_ld = L.Tpad;
+      t2.G = 0;
+      t2.row_limit = (int)T;
+      transpose_rows_kernel<<<dim3(ceil_div(Np, 64), ceil_div(L.Tpad, 64)), 256, 0, s0>>>(t2);
+      if (!(do_shared && wgrad)) {
+        RowTransposeArgs t3 = t2;
+        t3.src = static_cast<const __nv_bfloat16*>(x);
+        t3.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
+        t3.C = (int)d;
+        transpose_rows_kernel<<<dim3(ceil_div(d, 64), ceil_div(L.Tpad, 64)), 256, 0, s0>>>(t3);
+      }
+      const int want = (int)std::max<int64_t>(1, std::min<int64_t>(kDeMaxSegments, T / 512));
+      const int seg = ceil_div(ceil_div(T, want), 64) * 64;
+      const int segs = ceil_div(T, seg);
+      fill_segments_kernel<<<1, 32, 0, s0>>>(ks, kc, segs, seg, (int)T);
+      float* part = reinterpret_cast<float*>(bw(B.de_part));
+      if (kg_gemm(h->tm_b_dzT, h->tm_b_xT, segs, ks, kc, (int)N, 0, 0, (int)N, (int)d, (int)d, part, nullptr) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+      router_de_reduce_kernel<<<ceil_div(N * d, 256), 256, 0, s0>>>(part, segs, size_t(N) * d, d_router);
     }
+    if (d_logit_bias) column_sum_kernel<<<ceil_div(N, 256), 256, 0, s0>>>(rz.dz, (int)T, (int)N, d_logit_bias);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   } else {
     // the routed term left out: the gates and the router have no gradient
     if (dgate && cudaMemsetAsync(dgate, 0, size_t(TK) * 4, s0) != cudaSuccess) return MOE_ERR_CUDA;
