@@ -74,6 +74,8 @@ def parse_args():
                    help="the layer with FP8 expert GEMMs (moe_forward_fp8) on the --config workload alone")
     p.add_argument("--fp8-quant", action="store_true",
                    help="time the FP8 1x128 quantization of one forward's permuted activations instead")
+    p.add_argument("--training-step", action="store_true",
+                   help="time only the layer's training step (forward + backward) on the --config workload")
     return p.parse_args()
 
 
@@ -513,6 +515,71 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
     return r
 
 
+def measure_training_step(B, shape: W.LayerShape, d_in: dict, dev, local: int, ranks, warmup: int,
+                          fwd_ms: float, peaks: dict, peak_src: str) -> dict:
+    """The layer's training step on the headline workload: moe_forward, then moe_backward for a seeded
+    upstream gradient dh, with every gradient asked for (dx, the gates', the router's and the expert
+    and shared weights' in fp32).  Timed like the forward (CUDA events on the launching stream over
+    at least ~0.5 s, barrier + synchronize on both sides, max over ranks).  Algorithmic FLOPs: the
+    forward's, plus twice them for the backward (each GEMM of the forward has one for its input and
+    one for its weights); the backward also recomputes the gate/up GEMM (executed FLOPs, reported
+    beside them)."""
+    world = ranks.world
+    layer = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks,
+                       d_ff_shared=shape.Is, max_tokens=shape.T, max_k=shape.K, gate=shape.gate, device=local)
+    shared = (d_in["ws_gate"], d_in["ws_up"], d_in["ws_down"]) if shape.Ks else None
+    layer.set_weights(d_in["router"], (d_in["w_gate"], d_in["w_up"], d_in["w_down"]), shared,
+                      logit_bias=d_in["logit_bias"], select_bias=d_in["select_bias"])
+    x = d_in["x"]
+    out, dx = torch.empty_like(x), torch.empty_like(x)
+    dh = W.output_gradient(shape).to(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(x, shape.K, out)
+        layer.backward(x, shape.K, dh, dx=dx, router_grad=True, weight_grads=True)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    est = time.perf_counter()
+    step()
+    torch.cuda.synchronize(dev)
+    steps = max(10, int(0.5 / max(time.perf_counter() - est, 1e-6)))
+    st = layer.status()
+    if st != B.MOE_OK:
+        raise B.MoEError(st, "training step warm-up")
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ranks.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    ranks.barrier()
+    clk = clocks.stop()
+    st = layer.status()
+    if st != B.MOE_OK:
+        raise B.MoEError(st, "training step timed region")
+    ms = ranks.max(start.elapsed_time(end)) / steps
+    layer.close()
+    fwd_flop = layer_flop(shape)
+    alg_flop = 3 * fwd_flop
+    executed = alg_flop + 4 * shape.T * shape.d * (shape.K * shape.I + shape.Ks * shape.Is) + shape.router_flop
+    peak, peak_name = choose_peak(peaks, ms * steps * 1e-3, clk)
+    tflops = world * alg_flop / (ms * 1e-3) / 1e12
+    return {"workload": workload_config(shape, f"replicas{world}" if world > 1 else "single")["workload"],
+            "what": "moe_forward + moe_backward (dx, dgate, d_router, d_logit_bias when present, expert and "
+                    "shared weight gradients in fp32)",
+            "steps": steps, "ms_per_step": ms, "ms_backward": ms - fwd_ms,
+            "tokens_per_s": aggregate_rate(shape.T, world, ms),
+            "tflops": tflops, "tflops_frac_of_peak": tflops / (world * peak), "tflops_peak": f"{peak_src} {peak_name}",
+            "algorithmic_tflop_per_step": alg_flop / 1e12, "executed_tflop_per_step": executed / 1e12,
+            "clocks": clk}
+
+
 def fused_decode(shape: W.LayerShape, fp8: bool = False) -> bool:
     """Whether the layer (bf16 or FP8) runs both expert GEMMs in one launch (the decode FFN)."""
     return shape.T <= DECODE_MAX_T
@@ -599,6 +666,32 @@ def estimate_step_s(B, shape: W.LayerShape, d_in: dict, dev, local: int) -> floa
     return dt
 
 
+def run_training_step(args):
+    """One JSON line for the layer's training step alone (moe_forward + moe_backward) on --config."""
+    from fine_grained_shared_b200 import moe as B
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    shape = W.CONFIGS[args.config]
+    host = host_inputs(shape)
+    d_in = to_device(host, dev)
+    peaks, peak_src = measured_peaks()
+    fwd = measure_layer(B, shape, host, d_in, dev, local, ranks, max(3, args.steps), max(3, args.warmup),
+                        with_e2e=False)
+    t = measure_training_step(B, shape, d_in, dev, local, ranks, max(3, args.warmup), fwd["ms_step"], peaks, peak_src)
+    line = {"metric": "MoE layer training step (forward + backward) tokens/s", "value": t["tokens_per_s"],
+            "unit": UNIT, "n_gpus": ranks.world, "steps": t["steps"], "warmup": max(3, args.warmup),
+            "ms_per_step": t["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(shape, f"replicas{ranks.world}" if ranks.world > 1 else "single"),
+            "forward_ms_per_step": fwd["ms_step"], "training_step": t}
+    if ranks.rank == 0:
+        print(json.dumps(line), flush=True)
+    ranks.close()
+
+
 def run_ours(args):
     from fine_grained_shared_b200 import moe as B
 
@@ -643,6 +736,14 @@ def run_ours(args):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(shape, host, fp8=fp8)
+
+    # the layer's training step (forward + backward) on the same workload, after the headline
+    if not args.no_per_config and not fp8 and not fused_decode(shape):
+        d_in = to_device(host, dev)
+        line["training_step"] = measure_training_step(B, shape, d_in, dev, local, ranks, warmup, r["ms_step"],
+                                                      peaks, peak_src)
+        del d_in
+        torch.cuda.empty_cache()
 
     # the other single-GPU workloads, measured after the headline one: ms per step, tokens/s and the
     # roofline that bounds each (tensor for the 2B layer, HBM over the touched experts' weights for
@@ -814,6 +915,8 @@ def main():
         run_reference_fp8(args) if args.fp8_quant else run_reference(args)
     elif args.fp8_quant:
         run_fp8_quant(args)
+    elif args.training_step:
+        run_training_step(args)
     else:
         run_ours(args)
 

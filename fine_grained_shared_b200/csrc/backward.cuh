@@ -28,8 +28,58 @@
 namespace fgs {
 
 // ---------------------------------------------------------------------------
-// Batched transpose: dst[b][c][col0 + r] = src[b][r][c], r < R, c < C
-// (R, C, dst_ld and col0 multiples of 16).  64 x 64 tiles through shared memory.
+// Transposes through shared memory, tiles of 64 x 64: each thread loads 32
+// contiguous bytes of one source row and stores 32 contiguous bytes (16
+// source rows) of one destination row.
+// ---------------------------------------------------------------------------
+constexpr int kTrRows = 64, kTrCols = 64;
+
+// tile[r][c] <- src rows r0 .. + 63 (rows >= nrows zero), columns c0 .. + 63 (C a multiple of 16)
+__device__ __forceinline__ void tr_load_tile(uint16_t (*tile)[kTrCols + 2], const uint16_t* src, long long ld, int C,
+                                             int r0, int nrows, int c0) {
+  const int tr = threadIdx.x >> 2, tc = (threadIdx.x & 3) * 16;
+  uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+  if (r0 + tr < nrows && c0 + tc < C) {
+    const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(r0 + tr) * ld + c0 + tc);
+    v0 = p[0];
+    v1 = p[1];
+  }
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    tile[tr][tc + 2 * j] = static_cast<uint16_t>(w[j] & 0xFFFFu);
+    tile[tr][tc + 2 * j + 1] = static_cast<uint16_t>(w[j] >> 16);
+  }
+}
+
+// dst row (c0 + oc), values of source rows r0 + orr .. + 15: thread (oc = tid / 4, orr = (tid % 4) * 16);
+// rowf / rowok (or nullptr): each row's scale and whether it holds a pair (zero if not)
+__device__ __forceinline__ void tr_store_row(const uint16_t (*tile)[kTrCols + 2], uint16_t* q, int nvalid,
+                                             const float* rowf, const int* rowok, int orr, int oc) {
+  uint32_t w[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t lo = tile[orr + 2 * j][oc], hi = tile[orr + 2 * j + 1][oc];
+    if (rowf) {
+      lo = rowok[orr + 2 * j] ? (pack_bf16x2(rowf[orr + 2 * j] * __uint_as_float(lo << 16), 0.f) & 0xFFFFu) : 0u;
+      hi = rowok[orr + 2 * j + 1] ? (pack_bf16x2(rowf[orr + 2 * j + 1] * __uint_as_float(hi << 16), 0.f) & 0xFFFFu)
+                                  : 0u;
+    }
+    w[j] = lo | (hi << 16);
+  }
+  if (nvalid >= 16 && (reinterpret_cast<uintptr_t>(q) & 15u) == 0) {
+    reinterpret_cast<uint4*>(q)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(q)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < nvalid) q[j] = static_cast<uint16_t>(w[j >> 1] >> ((j & 1) * 16));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Batched transpose: dst[b][c][col0 + r] = src[b][r][c], r < R, c < C (R, C,
+// dst_ld and col0 multiples of 16).
 // ---------------------------------------------------------------------------
 struct TransposeArgs {
   const __nv_bfloat16* src;
@@ -39,33 +89,16 @@ struct TransposeArgs {
 };
 
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeArgs a) {
-  __shared__ uint16_t tile[64][66];
-  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64, b = blockIdx.z;
+  __shared__ uint16_t tile[kTrRows][kTrCols + 2];
+  const int c0 = blockIdx.x * kTrCols, r0 = blockIdx.y * kTrRows, b = blockIdx.z;
   const uint16_t* src = reinterpret_cast<const uint16_t*>(a.src) + b * a.src_bs;
   uint16_t* dst = reinterpret_cast<uint16_t*>(a.dst) + b * a.dst_bs;
-  const int tr = threadIdx.x >> 2, tc = (threadIdx.x & 3) * 16;
-  if (r0 + tr < a.R && c0 + tc < a.C) {
-    const uint4* p = reinterpret_cast<const uint4*>(src + static_cast<size_t>(r0 + tr) * a.C + c0 + tc);
-    const uint4 v0 = p[0], v1 = p[1];
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      tile[tr][tc + 2 * j] = static_cast<uint16_t>(w[j] & 0xFFFFu);
-      tile[tr][tc + 2 * j + 1] = static_cast<uint16_t>(w[j] >> 16);
-    }
-  }
+  tr_load_tile(tile, src, a.C, a.C, r0, a.R, c0);
   __syncthreads();
-  // thread (oc, orr): output row c0 + oc, its 16 values r0 + orr .. + 15
   const int oc = threadIdx.x >> 2, orr = (threadIdx.x & 3) * 16;
-  if (c0 + oc < a.C && r0 + orr < a.R) {
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      w[j] = static_cast<uint32_t>(tile[orr + 2 * j][oc]) | (static_cast<uint32_t>(tile[orr + 2 * j + 1][oc]) << 16);
-    uint4* q = reinterpret_cast<uint4*>(dst + static_cast<size_t>(c0 + oc) * a.dst_ld + a.col0 + r0 + orr);
-    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  }
+  if (c0 + oc >= a.C || r0 + orr >= a.R) return;
+  tr_store_row(tile, dst + static_cast<size_t>(c0 + oc) * a.dst_ld + a.col0 + r0 + orr, a.R - r0 - orr, nullptr,
+               nullptr, orr, oc);
 }
 
 // ---------------------------------------------------------------------------
@@ -73,8 +106,8 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeArgs a) {
 // rows): dst[c][r] = scale(r) * src[r][c] for the rows that hold a (token,
 // slot) pair and 0 for the others, every r < R (C a multiple of 16).  Valid
 // rows: G > 0: r - row_start[e] < counts[e] for the expert e whose segment
-// holds r; G = 0: r < row_limit.  scale: nullptr (1) or [R], read only on
-// valid rows.
+// holds r (G <= 256; the tables are read into shared memory first); G = 0:
+// r < row_limit.  scale: nullptr (1) or [R], read only on valid rows.
 // ---------------------------------------------------------------------------
 struct RowTransposeArgs {
   const __nv_bfloat16* src;
@@ -89,63 +122,40 @@ struct RowTransposeArgs {
 };
 
 __global__ void __launch_bounds__(256) transpose_rows_kernel(RowTransposeArgs a) {
-  __shared__ uint16_t tile[64][66];
-  __shared__ float rowf[64];  // per row: its scale, or 0 for a row without a pair
-  __shared__ int rowok[64];
-  const int c0 = blockIdx.x * 64, r0 = blockIdx.y * 64;
+  __shared__ uint16_t tile[kTrRows][kTrCols + 2];
+  __shared__ float rowf[kTrRows];  // per row: its scale
+  __shared__ int rowok[kTrRows];   // per row: holds a pair
+  __shared__ int32_t s_rs[256], s_cnt[256];
+  const int c0 = blockIdx.x * kTrCols, r0 = blockIdx.y * kTrRows;
   const int tid = threadIdx.x;
-  if (tid < 64) {
+  for (int i = tid; i < a.G; i += 256) {
+    s_rs[i] = a.row_start[i];
+    s_cnt[i] = a.counts[i];
+  }
+  tr_load_tile(tile, reinterpret_cast<const uint16_t*>(a.src), a.C, a.C, r0, min(a.R, a.src_rows), c0);
+  __syncthreads();
+  if (tid < kTrRows) {
     const int r = r0 + tid;
     bool ok = r < a.R && r < a.src_rows;
     if (ok && a.G > 0) {
       int lo = 0, hi = a.G;  // the last expert whose segment starts at or before r
       while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (a.row_start[mid] <= r) lo = mid;
+        if (s_rs[mid] <= r) lo = mid;
         else hi = mid;
       }
-      ok = r - a.row_start[lo] < a.counts[lo];
+      ok = r - s_rs[lo] < s_cnt[lo];
     } else if (ok) {
       ok = r < a.row_limit;
     }
     rowok[tid] = ok ? 1 : 0;
     rowf[tid] = ok ? (a.scale ? a.scale[r] : 1.f) : 0.f;
   }
-  const int tr = tid >> 2, tc = (tid & 3) * 16;
-  if (r0 + tr < a.src_rows && c0 + tc < a.C) {
-    const uint4* p = reinterpret_cast<const uint4*>(a.src + static_cast<size_t>(r0 + tr) * a.C + c0 + tc);
-    const uint4 v0 = p[0], v1 = p[1];
-    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      tile[tr][tc + 2 * j] = static_cast<uint16_t>(w[j] & 0xFFFFu);
-      tile[tr][tc + 2 * j + 1] = static_cast<uint16_t>(w[j] >> 16);
-    }
-  }
   __syncthreads();
   const int oc = tid >> 2, orr = (tid & 3) * 16;
   if (c0 + oc >= a.C || r0 + orr >= a.R) return;
-  uint16_t v[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int rl = orr + j;
-    uint16_t o = 0;
-    if (rowok[rl]) {
-      const float f = rowf[rl] * __uint_as_float(static_cast<uint32_t>(tile[rl][oc]) << 16);
-      o = static_cast<uint16_t>(pack_bf16x2(f, 0.f) & 0xFFFFu);
-    }
-    v[j] = o;
-  }
-  uint16_t* q = reinterpret_cast<uint16_t*>(a.dst) + static_cast<size_t>(c0 + oc) * a.dst_ld + r0 + orr;
-  if (r0 + orr + 16 <= a.R && ((reinterpret_cast<uintptr_t>(q) & 15u) == 0)) {
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) w[j] = static_cast<uint32_t>(v[2 * j]) | (static_cast<uint32_t>(v[2 * j + 1]) << 16);
-    reinterpret_cast<uint4*>(q)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    reinterpret_cast<uint4*>(q)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-  } else {
-    for (int j = 0; j < 16 && r0 + orr + j < a.R; ++j) q[j] = v[j];
-  }
+  tr_store_row(tile, reinterpret_cast<uint16_t*>(a.dst) + static_cast<size_t>(c0 + oc) * a.dst_ld + r0 + orr,
+               a.R - r0 - orr, rowf, rowok, orr, oc);
 }
 
 // the shared experts' K ranges for the weight-gradient GEMMs: every expert j < n over rows [0, T)

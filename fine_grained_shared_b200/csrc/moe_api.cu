@@ -1619,7 +1619,7 @@ cudaError_t launch_transpose(const void* src, void* dst, int batch, int R, int C
   t.col0 = col0;
   t.src_bs = static_cast<long long>(R) * C;
   t.dst_bs = static_cast<long long>(C) * dst_ld;
-  transpose_bf16_kernel<<<dim3(ceil_div(C, 64), ceil_div(R, 64), batch), 256, 0, s>>>(t);
+  transpose_bf16_kernel<<<dim3(ceil_div(C, kTrCols), ceil_div(R, kTrRows), batch), 256, 0, s>>>(t);
   return cudaGetLastError();
 }
 
@@ -1784,7 +1784,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       rt.row_start = h->at<int32_t>(L.row_start);
       rt.counts = h->at<int32_t>(L.counts);
       rt.G = (int)N;
-      const dim3 grid(ceil_div(d, 64), ceil_div(L.P, 64));
+      const dim3 grid(ceil_div(d, kTrCols), ceil_div(L.P, kTrRows));
       rt.src = h->at<__nv_bfloat16>(L.y);
       rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dyT));
       rt.scale = h->at<float>(L.gate_perm);
@@ -1820,7 +1820,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     rt.dst_ld = L.Tpad;
     rt.G = 0;
     rt.row_limit = (int)T;
-    const dim3 grid(ceil_div(d, 64), ceil_div(L.Tpad, 64));
+    const dim3 grid(ceil_div(d, kTrCols), ceil_div(L.Tpad, kTrRows));
     rt.src = static_cast<const __nv_bfloat16*>(dh);
     rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dhT));
     transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
@@ -2000,7 +2000,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     rt.dst_ld = Np;
     rt.G = 0;
     rt.row_limit = (int)N;
-    transpose_rows_kernel<<<dim3(ceil_div(d, 64), ceil_div(Np, 64)), 256, 0, s0>>>(rt);
+    transpose_rows_kernel<<<dim3(ceil_div(d, kTrCols), ceil_div(Np, kTrRows)), 256, 0, s0>>>(rt);
     fill_segments_kernel<<<1, 32, 0, s0>>>(ks + 1, kc + 1, 1, (int)N, (int)N);
     dxr = reinterpret_cast<float*>(bw(B.dxr));
     if (kg_gemm(h->tm_b_dzb, h->tm_b_ET, 1, ks + 1, kc + 1, (int)T, 0, 0, (int)T, (int)d, (int)d, dxr, nullptr) !=
@@ -2018,13 +2018,13 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       t2.dst_ld = L.Tpad;
       t2.G = 0;
       t2.row_limit = (int)T;
-      transpose_rows_kernel<<<dim3(ceil_div(Np, 64), ceil_div(L.Tpad, 64)), 256, 0, s0>>>(t2);
+      transpose_rows_kernel<<<dim3(ceil_div(Np, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t2);
       if (!(do_shared && wgrad)) {
         RowTransposeArgs t3 = t2;
         t3.src = static_cast<const __nv_bfloat16*>(x);
         t3.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
         t3.C = (int)d;
-        transpose_rows_kernel<<<dim3(ceil_div(d, 64), ceil_div(L.Tpad, 64)), 256, 0, s0>>>(t3);
+        transpose_rows_kernel<<<dim3(ceil_div(d, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t3);
       }
       const int want = (int)std::max<int64_t>(1, std::min<int64_t>(kDeMaxSegments, T / 512));
       const int seg = ceil_div(ceil_div(T, want), 64) * 64;
