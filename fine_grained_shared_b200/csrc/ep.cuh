@@ -9,7 +9,10 @@
 //                       rows (ep_plan.h) and its own experts' GEMM tables
 //   ep_dispatch_kernel  the permutation of permute.cuh with each (token, slot)
 //                       row, and its gate, stored into the buffer of the rank
-//                       that holds the slot's expert
+//                       that holds the slot's expert; in the FP8 layer the row
+//                       is quantized once (1 x 128 groups, as permute_quant_kernel)
+//                       and its E4M3 codes and scale cells are what is sent
+//                       (the DeepSeek-V3 report's FP8 dispatch, section 3.3)
 //   ep_combine_kernel   out[t] = x[t] + ys[t] + sum_k y_owner(k)[slot_of[t, k]],
 //                       the g-scaled rows loaded from their owners, k ascending
 //
@@ -21,6 +24,7 @@
 #pragma once
 
 #include "ep_plan.h"
+#include "fp8_gemm.cuh"
 #include "permute.cuh"
 
 namespace fgs {
@@ -83,6 +87,11 @@ struct EpDispatchArgs {
   size_t xperm_off, gate_off;  // byte offsets of the row buffer and its gates in every workspace
   EpPeers peers;
   int* tile_ctr;              // [2] this rank's gate/up tile counter, zeroed for its GEMMs
+  // FP8 layer: byte offsets of the codes [P, d] and scale atoms of the row buffer in every
+  // workspace, and this rank's own dense codes of x with their atoms (the shared experts' A) or null
+  size_t xq_off, xs_off;
+  uint8_t* xq;
+  uint8_t* xs;
 };
 
 // grid (nblk, split), as permute_gather_kernel: CTA (b, s) ranks block b's
@@ -90,6 +99,7 @@ struct EpDispatchArgs {
 // rank that holds one of the token's experts (one 16-byte store stream per
 // (token, slot) pair; a rank that holds several of a token's experts receives
 // the row once per expert, the layout its grouped GEMMs read).
+template <bool FP8>
 __global__ void __launch_bounds__(kPermThreads) ep_dispatch_kernel(EpDispatchArgs a) {
   __shared__ uint32_t masks[256 * 4];
   __shared__ int32_t sbase[256], roff[256], ebase[256];
@@ -136,8 +146,43 @@ __global__ void __launch_bounds__(kPermThreads) ep_dispatch_kernel(EpDispatchArg
     }
   }
   __syncthreads();
-  // one warp per token row, read once and stored to each of its K destinations
   const int warp = tid >> 5, lane = tid & 31, nwarps = kPermThreads / 32;
+  if constexpr (FP8) {
+    // quantize each token row once: a warp per row, 256 columns (two 128-column groups) per pass,
+    // lanes 0-15 the first group and 16-31 the second; codes and scale cells to every destination
+    const int groups = a.d / kF8BK;
+    for (int tl = sp + a.split * warp; tl < ntok; tl += a.split * nwarps) {
+      const size_t t = static_cast<size_t>(t0 + tl);
+      const __nv_bfloat16* srow = a.x + t * a.d;
+      for (int c0 = 0; c0 < a.d; c0 += 2 * kF8BK) {
+        const int col = c0 + lane * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (col < a.d) v = __ldg(reinterpret_cast<const uint4*>(srow + col));
+        float m = amax8(v);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const int e = scale_exponent(m);
+        if (col < a.d) {
+          const uint2 codes = encode8(v, pow2_neg(e));
+          const int g = col / kF8BK;
+          const uint32_t sbyte = static_cast<uint32_t>(e + 127);
+          for (int k = 0; k < K; ++k) {
+            uint8_t* ws = a.peers.ws[dstq[tl * K + k]];
+            const size_t R = static_cast<size_t>(dst[tl * K + k]);
+            *reinterpret_cast<uint2*>(ws + a.xq_off + R * a.d + col) = codes;
+            if ((lane & 15) == 0) put_scale(ws + a.xs_off, R, g, groups, sbyte);
+          }
+          if (a.xq) {
+            *reinterpret_cast<uint2*>(a.xq + t * a.d + col) = codes;
+            if ((lane & 15) == 0) put_scale(a.xs, t, g, groups, sbyte);
+          }
+        }
+      }
+    }
+    __threadfence_system();
+    return;
+  }
+  // one warp per token row, read once and stored to each of its K destinations
   const int nvec = a.d >> 3;
   for (int tl = sp + a.split * warp; tl < ntok; tl += a.split * nwarps) {
     const uint4* srow = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + tl) * a.d);

@@ -270,7 +270,6 @@ moe_status check_config(const moe_config* c) {
   if (c->ep_ranks > 1) {
     if (c->ep_ranks > kEpMaxRanks || c->n_routed % c->ep_ranks || c->ep_rank < 0 || c->ep_rank >= c->ep_ranks)
       return MOE_ERR_INVALID_ARG;
-    if (c->flags & MOE_FLAG_FP8) return MOE_ERR_UNSUPPORTED;
   } else if (c->ep_ranks < 0 || c->ep_rank != 0) {
     return MOE_ERR_INVALID_ARG;
   }
@@ -750,6 +749,114 @@ moe_status enqueue_expert_gemms(moe_ctx* h, int64_t T, bool do_shared, const Exp
   return MOE_OK;
 }
 
+// The FP8 layer's expert GEMMs (fp8_gemm.cuh): gate/up with SwiGLU and H's quantization, then down with the
+// gate scale; the shared experts' tiles over the T rows of x's codes first, then the routed experts' (G groups,
+// tables on the device; G = 0: none).  The FP8 weight maps of the handle must hold the caller's pointers.
+moe_status enqueue_fp8_expert_gemms(moe_ctx* h, int64_t T, bool do_shared, int G, const int32_t* mtile128,
+                                    const int32_t* row_start, const moe_experts_fp8* experts,
+                                    const moe_experts_fp8* shared, cudaStream_t s0, bool pdl) {
+  const moe_config& c = h->cfg;
+  const Layout& L = h->L;
+  const int64_t d = c.d_model, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const bool do_routed = G > 0;
+  const int64_t SI = Ks * Is;
+  // an absent part's maps are never read; the present part's stand in
+  const CUtensorMap& A = do_routed ? h->tm_xq_perm : h->tm_xq;
+  const CUtensorMap& As = do_shared ? h->tm_xq : h->tm_xq_perm;
+  const CUtensorMap& Wg = do_routed ? h->tm8_wg.map : h->tm8_swg.map;
+  const CUtensorMap& Wu = do_routed ? h->tm8_wu.map : h->tm8_swu.map;
+  const CUtensorMap& Wgs = do_shared ? h->tm8_swg.map : h->tm8_wg.map;
+  const CUtensorMap& Wus = do_shared ? h->tm8_swu.map : h->tm8_wu.map;
+  Fp8GemmArgs g{};
+  if (do_routed) {
+    g.num_groups = G;
+    g.mtile_start = mtile128;
+    g.row_start = row_start;
+    g.n_tiles = ceil_div(I, kF8BN / 2);
+    g.num_kg = (int)(d / kF8BK);
+    g.a_atoms = h->at<uint8_t>(L.xs_perm);
+    g.a_groups = (int)(d / kF8BK);
+    g.w_scale0 = experts->s_gate;
+    g.w_scale1 = experts->s_up;
+    g.w_rows128 = (int)(I / 128);
+    g.hq = h->at<uint8_t>(L.hq);
+    g.hs_atoms = h->at<uint8_t>(L.hs_perm);
+    g.h_groups = (int)(I / kF8BK);
+    g.ld_out = (int)I;
+    g.n_limit = (int)I;
+  }
+  if (do_shared) {
+    g.sh_rows = (int)T;
+    g.sh_n_tiles = ceil_div(SI, kF8BN / 2);
+    g.sh_J = 1;
+    g.sh_kg_per_j = (int)(d / kF8BK);
+    g.sh_a_atoms = h->at<uint8_t>(L.xs);
+    g.sh_a_groups = (int)(d / kF8BK);
+    g.sh_w_scale0 = shared->s_gate;
+    g.sh_w_scale1 = shared->s_up;
+    g.sh_w_rows128 = (int)(Is / 128);
+    g.sh_hq = h->at<uint8_t>(L.hsq);
+    g.sh_hs_atoms = h->at<uint8_t>(L.hss);
+    g.sh_h_groups = (int)(SI / kF8BK);
+    g.sh_ld_out = (int)SI;
+    g.sh_n_limit = (int)SI;
+  }
+  g.err = h->at<uint32_t>(L.err);
+  g.timeout_ns = kTimeoutNs;
+  g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
+  const int sh_tiles = do_shared ? ceil_div(T, kF8BM) * g.sh_n_tiles : 0;
+  const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
+  {
+    KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
+    if (launch_pdl(fp8_gemm_kernel<true>, dim3(ctas), dim3(kF8Threads), fp8_gemm_smem_bytes(), s0, 1, pdl, A, Wg,
+                   Wu, As, Wgs, Wus, g) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  const CUtensorMap& HA = do_routed ? h->tm_hq : h->tm_hsq;
+  const CUtensorMap& HAs = do_shared ? h->tm_hsq : h->tm_hq;
+  const CUtensorMap& Wd = do_routed ? h->tm8_wd.map : h->tm8_swd.map;
+  const CUtensorMap& Wds = do_shared ? h->tm8_swd.map : h->tm8_wd.map;
+  Fp8GemmArgs g2{};
+  if (do_routed) {
+    g2.num_groups = G;
+    g2.mtile_start = mtile128;
+    g2.row_start = row_start;
+    g2.n_tiles = ceil_div(d, kF8BN);
+    g2.num_kg = (int)(I / kF8BK);
+    g2.a_atoms = h->at<uint8_t>(L.hs_perm);
+    g2.a_groups = (int)(I / kF8BK);
+    g2.w_scale0 = experts->s_down;
+    g2.w_rows128 = (int)(d / 128);
+    g2.row_scale = h->at<float>(L.gate_perm);
+    g2.y = h->at<__nv_bfloat16>(L.y);
+    g2.ld_out = (int)d;
+    g2.n_limit = (int)d;
+  }
+  if (do_shared) {
+    g2.sh_rows = (int)T;
+    g2.sh_n_tiles = ceil_div(d, kF8BN);
+    g2.sh_J = (int)Ks;
+    g2.sh_kg_per_j = (int)(Is / kF8BK);
+    g2.sh_k_per_j = (int)Is;
+    g2.sh_a_atoms = h->at<uint8_t>(L.hss);
+    g2.sh_a_groups = (int)(SI / kF8BK);
+    g2.sh_w_scale0 = shared->s_down;
+    g2.sh_w_rows128 = (int)(d / 128);
+    g2.sh_y = h->at<__nv_bfloat16>(L.ys);
+    g2.sh_ld_out = (int)d;
+    g2.sh_n_limit = (int)d;
+  }
+  g2.err = h->at<uint32_t>(L.err);
+  g2.timeout_ns = kTimeoutNs;
+  const int sh_tiles2 = do_shared ? ceil_div(T, kF8BM) * g2.sh_n_tiles : 0;
+  const int ctas2 = do_routed || sh_tiles2 > h->num_sms ? h->num_sms : sh_tiles2;
+  KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
+  if (launch_pdl(fp8_gemm_kernel<false>, dim3(ctas2), dim3(kF8Threads), fp8_gemm_smem_bytes(), s0, 1, pdl, HA, Wd,
+                 Wd, HAs, Wds, Wds, g2) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1141,101 +1248,9 @@ moe_status moe_forward_fp8(moe_handle h, const void* x, int64_t T, const moe_rou
   }
 
   if (!decode && (do_routed || do_shared)) {
-    const int64_t SI = Ks * Is;
-    // an absent part's maps are never read; the present part's stand in
-    const CUtensorMap& A = do_routed ? h->tm_xq_perm : h->tm_xq;
-    const CUtensorMap& As = do_shared ? h->tm_xq : h->tm_xq_perm;
-    const CUtensorMap& Wg = do_routed ? h->tm8_wg.map : h->tm8_swg.map;
-    const CUtensorMap& Wu = do_routed ? h->tm8_wu.map : h->tm8_swu.map;
-    const CUtensorMap& Wgs = do_shared ? h->tm8_swg.map : h->tm8_wg.map;
-    const CUtensorMap& Wus = do_shared ? h->tm8_swu.map : h->tm8_wu.map;
-    Fp8GemmArgs g{};
-    if (do_routed) {
-      g.num_groups = (int)N;
-      g.mtile_start = ra.mtile128_start;
-      g.row_start = ra.row_start;
-      g.n_tiles = ceil_div(I, kF8BN / 2);
-      g.num_kg = (int)(d / kF8BK);
-      g.a_atoms = h->at<uint8_t>(L.xs_perm);
-      g.a_groups = (int)(d / kF8BK);
-      g.w_scale0 = experts->s_gate;
-      g.w_scale1 = experts->s_up;
-      g.w_rows128 = (int)(I / 128);
-      g.hq = h->at<uint8_t>(L.hq);
-      g.hs_atoms = h->at<uint8_t>(L.hs_perm);
-      g.h_groups = (int)(I / kF8BK);
-      g.ld_out = (int)I;
-      g.n_limit = (int)I;
-    }
-    if (do_shared) {
-      g.sh_rows = (int)T;
-      g.sh_n_tiles = ceil_div(SI, kF8BN / 2);
-      g.sh_J = 1;
-      g.sh_kg_per_j = (int)(d / kF8BK);
-      g.sh_a_atoms = h->at<uint8_t>(L.xs);
-      g.sh_a_groups = (int)(d / kF8BK);
-      g.sh_w_scale0 = shared->s_gate;
-      g.sh_w_scale1 = shared->s_up;
-      g.sh_w_rows128 = (int)(Is / 128);
-      g.sh_hq = h->at<uint8_t>(L.hsq);
-      g.sh_hs_atoms = h->at<uint8_t>(L.hss);
-      g.sh_h_groups = (int)(SI / kF8BK);
-      g.sh_ld_out = (int)SI;
-      g.sh_n_limit = (int)SI;
-    }
-    g.err = h->at<uint32_t>(L.err);
-    g.timeout_ns = kTimeoutNs;
-    g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
-    const int sh_tiles = do_shared ? ceil_div(T, kF8BM) * g.sh_n_tiles : 0;
-    const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
-    {
-      KernelTimer kt(h, MOE_KERNEL_GATE_UP, s0);
-      if (launch_pdl(fp8_gemm_kernel<true>, dim3(ctas), dim3(kF8Threads), fp8_gemm_smem_bytes(), s0, 1, pdl, A, Wg,
-                     Wu, As, Wgs, Wus, g) != cudaSuccess)
-        return MOE_ERR_CUDA;
-    }
-    const CUtensorMap& HA = do_routed ? h->tm_hq : h->tm_hsq;
-    const CUtensorMap& HAs = do_shared ? h->tm_hsq : h->tm_hq;
-    const CUtensorMap& Wd = do_routed ? h->tm8_wd.map : h->tm8_swd.map;
-    const CUtensorMap& Wds = do_shared ? h->tm8_swd.map : h->tm8_wd.map;
-    Fp8GemmArgs g2{};
-    if (do_routed) {
-      g2.num_groups = (int)N;
-      g2.mtile_start = ra.mtile128_start;
-      g2.row_start = ra.row_start;
-      g2.n_tiles = ceil_div(d, kF8BN);
-      g2.num_kg = (int)(I / kF8BK);
-      g2.a_atoms = h->at<uint8_t>(L.hs_perm);
-      g2.a_groups = (int)(I / kF8BK);
-      g2.w_scale0 = experts->s_down;
-      g2.w_rows128 = (int)(d / 128);
-      g2.row_scale = h->at<float>(L.gate_perm);
-      g2.y = h->at<__nv_bfloat16>(L.y);
-      g2.ld_out = (int)d;
-      g2.n_limit = (int)d;
-    }
-    if (do_shared) {
-      g2.sh_rows = (int)T;
-      g2.sh_n_tiles = ceil_div(d, kF8BN);
-      g2.sh_J = (int)Ks;
-      g2.sh_kg_per_j = (int)(Is / kF8BK);
-      g2.sh_k_per_j = (int)Is;
-      g2.sh_a_atoms = h->at<uint8_t>(L.hss);
-      g2.sh_a_groups = (int)(SI / kF8BK);
-      g2.sh_w_scale0 = shared->s_down;
-      g2.sh_w_rows128 = (int)(d / 128);
-      g2.sh_y = h->at<__nv_bfloat16>(L.ys);
-      g2.sh_ld_out = (int)d;
-      g2.sh_n_limit = (int)d;
-    }
-    g2.err = h->at<uint32_t>(L.err);
-    g2.timeout_ns = kTimeoutNs;
-    const int sh_tiles2 = do_shared ? ceil_div(T, kF8BM) * g2.sh_n_tiles : 0;
-    const int ctas2 = do_routed || sh_tiles2 > h->num_sms ? h->num_sms : sh_tiles2;
-    KernelTimer kt(h, MOE_KERNEL_DOWN, s0);
-    if (launch_pdl(fp8_gemm_kernel<false>, dim3(ctas2), dim3(kF8Threads), fp8_gemm_smem_bytes(), s0, 1, pdl, HA, Wd,
-                   Wd, HAs, Wds, Wds, g2) != cudaSuccess)
-      return MOE_ERR_CUDA;
+    const moe_status st = enqueue_fp8_expert_gemms(h, T, do_shared, do_routed ? (int)N : 0, ra.mtile128_start,
+                                                   ra.row_start, experts, shared, s0, pdl);
+    if (st != MOE_OK) return st;
   }
 
   CombineArgs ca{};
@@ -1498,7 +1513,17 @@ moe_status moe_ep_dispatch(moe_handle h, void* stream) {
     da.gate_off = L.gate_perm;
     da.peers = h->peers;
     da.tile_ctr = h->at<int>(L.tile_ctr);
-    ep_dispatch_kernel<<<dim3(nblk, split), kPermThreads, 0, s0>>>(da);
+    if (c.flags & MOE_FLAG_FP8) {
+      // the FP8 layer sends each row's E4M3 codes and scale cells; the dense codes of x stay here
+      const bool dense = c.n_shared > 0 && !(c.flags & MOE_FLAG_NO_SHARED);
+      da.xq_off = L.xq_perm;
+      da.xs_off = L.xs_perm;
+      da.xq = dense ? h->at<uint8_t>(L.xq) : nullptr;
+      da.xs = dense ? h->at<uint8_t>(L.xs) : nullptr;
+      ep_dispatch_kernel<true><<<dim3(nblk, split), kPermThreads, 0, s0>>>(da);
+    } else {
+      ep_dispatch_kernel<false><<<dim3(nblk, split), kPermThreads, 0, s0>>>(da);
+    }
   } else if (cudaMemsetAsync(h->ws + L.tile_ctr, 0, 8, s0) != cudaSuccess) {
     return MOE_ERR_CUDA;
   }
@@ -1510,6 +1535,7 @@ moe_status moe_ep_dispatch(moe_handle h, void* stream) {
 moe_status moe_ep_experts(moe_handle h, const moe_experts* experts, const moe_shared* shared, void* stream) {
   if (!h || h->cfg.ep_ranks < 2 || !h->peers_set || h->ep_stage != 2) return MOE_ERR_INVALID_ARG;
   const moe_config& c = h->cfg;
+  if (c.flags & MOE_FLAG_FP8) return MOE_ERR_UNSUPPORTED;  // the rows were sent as FP8 codes
   if (!experts || !experts->w_gate || !experts->w_up || !experts->w_down) return MOE_ERR_INVALID_ARG;
   if ((c.n_shared > 0) != (shared != nullptr)) return MOE_ERR_INVALID_ARG;
   if (shared && (!shared->w_gate || !shared->w_up || !shared->w_down)) return MOE_ERR_INVALID_ARG;
@@ -1540,6 +1566,46 @@ moe_status moe_ep_experts(moe_handle h, const moe_experts* experts, const moe_sh
       et = ExpertTables{per, h->at<int32_t>(L.ep_mtile128), h->at<int32_t>(L.ep_mtile),
                         h->at<int32_t>(L.ep_row_start), h->at<float>(L.gate_perm)};
     const moe_status st = enqueue_expert_gemms(h, T, do_shared, et, h->at<int>(L.tile_ctr), s0, false);
+    if (st != MOE_OK) return st;
+  }
+  h->ep_stage = 3;
+  return MOE_OK;
+}
+
+moe_status moe_ep_experts_fp8(moe_handle h, const moe_experts_fp8* experts, const moe_experts_fp8* shared,
+                              void* stream) {
+  if (!h || h->cfg.ep_ranks < 2 || !h->peers_set || h->ep_stage != 2) return MOE_ERR_INVALID_ARG;
+  const moe_config& c = h->cfg;
+  if (!(c.flags & MOE_FLAG_FP8)) return MOE_ERR_UNSUPPORTED;
+  auto complete = [](const moe_experts_fp8* e) {
+    return e->w_gate && e->w_up && e->w_down && e->s_gate && e->s_up && e->s_down;
+  };
+  if (!experts || !complete(experts)) return MOE_ERR_INVALID_ARG;
+  if ((c.n_shared > 0) != (shared != nullptr) || (shared && !complete(shared))) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {experts->w_gate, experts->w_up, experts->w_down, shared ? shared->w_gate : nullptr,
+                        shared ? shared->w_up : nullptr, shared ? shared->w_down : nullptr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_ALIGNMENT;
+  const int64_t d = c.d_model, I = c.d_ff, Ks = c.n_shared, Is = c.d_ff_shared;
+  const int per = c.n_routed / c.ep_ranks;
+  const int64_t T = h->ep_T;
+  DeviceGuard guard(h->device);
+  cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+  const Layout& L = h->L;
+  const bool do_shared = Ks > 0 && !(c.flags & MOE_FLAG_NO_SHARED) && T > 0;
+  const bool do_routed = !(c.flags & MOE_FLAG_NO_ROUTED);
+  bool ok = refresh_u8(h->tm8_wg, experts->w_gate, per, I, d, kF8BoxRowsW, 3) &&
+            refresh_u8(h->tm8_wu, experts->w_up, per, I, d, kF8BoxRowsW, 3) &&
+            refresh_u8(h->tm8_wd, experts->w_down, per, d, I, kF8BoxRowsWd, 3);
+  if (shared)
+    ok = ok && refresh_u8(h->tm8_swg, shared->w_gate, 1, Ks * Is, d, kF8BoxRowsW, 3) &&
+         refresh_u8(h->tm8_swu, shared->w_up, 1, Ks * Is, d, kF8BoxRowsW, 3) &&
+         refresh_u8(h->tm8_swd, shared->w_down, Ks, d, Is, kF8BoxRowsWd, 3);
+  if (!ok) return MOE_ERR_CUDA;
+  if (do_routed || do_shared) {
+    const moe_status st = enqueue_fp8_expert_gemms(h, T, do_shared, do_routed ? per : 0,
+                                                   h->at<int32_t>(L.ep_mtile128), h->at<int32_t>(L.ep_row_start),
+                                                   experts, shared, s0, false);
     if (st != MOE_OK) return st;
   }
   h->ep_stage = 3;

@@ -110,6 +110,7 @@ def lib() -> ctypes.CDLL:
     L.moe_ep_route.argtypes = [moe_handle, c_void_p, c_int64, POINTER(moe_router), c_int32, c_void_p]
     L.moe_ep_dispatch.argtypes = [moe_handle, c_void_p]
     L.moe_ep_experts.argtypes = [moe_handle, POINTER(moe_experts), POINTER(moe_shared), c_void_p]
+    L.moe_ep_experts_fp8.argtypes = [moe_handle, POINTER(moe_experts_fp8), POINTER(moe_experts_fp8), c_void_p]
     L.moe_ep_combine.argtypes = [moe_handle, c_void_p, c_void_p]
     L.moe_ep_plan.argtypes = [c_void_p, c_int32, c_int32, c_int32, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]
     L.moe_status_string.argtypes = [c_int]
@@ -120,7 +121,7 @@ def lib() -> ctypes.CDLL:
                  "moe_update_bias", "moe_quantize_fp8_rows", "moe_quantize_fp8_blocks", "moe_backward",
                  "moe_ep_workspace",
                  "moe_ep_set_peers", "moe_ep_ipc_handle", "moe_ep_open_peers", "moe_ep_route", "moe_ep_dispatch",
-                 "moe_ep_experts", "moe_ep_combine", "moe_ep_plan"):
+                 "moe_ep_experts", "moe_ep_experts_fp8", "moe_ep_combine", "moe_ep_plan"):
         getattr(L, name).restype = c_int
     _lib = L
     return L
@@ -247,6 +248,11 @@ def moe_ep_dispatch(h, stream):
 def moe_ep_experts(h, experts, shared, stream):
     return lib().moe_ep_experts(h, ctypes.byref(experts), ctypes.byref(shared) if shared is not None else None,
                                 stream)
+
+
+def moe_ep_experts_fp8(h, experts, shared, stream):
+    return lib().moe_ep_experts_fp8(h, ctypes.byref(experts), ctypes.byref(shared) if shared is not None else None,
+                                    stream)
 
 
 def moe_ep_combine(h, out, stream):
@@ -481,7 +487,11 @@ class ExpertParallelLayer(MoELayer):
         self._check(moe_ep_dispatch(self.h, _stream_ptr(stream)), "moe_ep_dispatch")
 
     def experts_step(self, stream=None):
-        self._check(moe_ep_experts(self.h, self.experts, self.shared, _stream_ptr(stream)), "moe_ep_experts")
+        if self.cfg.flags & MOE_FLAG_FP8:   # the dispatch sent FP8 rows: the FP8 expert GEMMs
+            self._check(moe_ep_experts_fp8(self.h, self.experts_fp8, self.shared_fp8, _stream_ptr(stream)),
+                        "moe_ep_experts_fp8")
+        else:
+            self._check(moe_ep_experts(self.h, self.experts, self.shared, _stream_ptr(stream)), "moe_ep_experts")
 
     def combine(self, out=None, stream=None):
         import torch

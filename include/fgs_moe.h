@@ -103,8 +103,8 @@ typedef struct moe_config {
    * split the mN routed experts in equal contiguous ranges (expert i on rank
    * i / (mN / G)); this handle is rank ep_rank and holds mN / G of them.
    * 0 or 1: a single-GPU handle (moe_forward).  Otherwise 2 <= G <= 32
-   * dividing mN, 0 <= ep_rank < G, and no MOE_FLAG_FP8 (else
-   * MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED). */
+   * dividing mN and 0 <= ep_rank < G (else MOE_ERR_INVALID_ARG); with
+   * MOE_FLAG_FP8 the dispatch sends FP8 rows (moe_ep_experts_fp8). */
   int32_t ep_ranks;
   int32_t ep_rank;
 } moe_config;
@@ -446,6 +446,15 @@ moe_status moe_ep_dispatch(moe_handle h, void* stream);
  * expert l is global expert ep_rank * mN / G + l.  shared as for moe_forward
  * (every rank holds all K_s shared experts). */
 moe_status moe_ep_experts(moe_handle h, const moe_experts* experts, const moe_shared* shared, void* stream);
+/* The FP8 layer's step 3 (handles created with MOE_FLAG_FP8, whose dispatch
+ * quantized each row once, 1 x 128 groups as moe_forward_fp8 does, and sent
+ * its E4M3 codes and scale bytes instead of the bf16 row: the FP8 dispatch of
+ * the DeepSeek-V3 report, section 3.3): this rank's mN / G experts and the
+ * shared experts in the moe_experts_fp8 format of moe_forward_fp8.
+ * moe_ep_experts returns MOE_ERR_UNSUPPORTED on such a handle, and this call
+ * on a bf16 one. */
+moe_status moe_ep_experts_fp8(moe_handle h, const moe_experts_fp8* experts, const moe_experts_fp8* shared,
+                              void* stream);
 /* out: bf16 [T, d] of the T tokens of the last moe_ep_route. */
 moe_status moe_ep_combine(moe_handle h, void* out, void* stream);
 

@@ -122,7 +122,8 @@ def test_config_checks_of_an_expert_parallel_handle():
     assert create(ep_rank=2) == B.MOE_ERR_INVALID_ARG
     assert create(ep_ranks=0, ep_rank=1) == B.MOE_ERR_INVALID_ARG
     assert create(ep_ranks=64, n_routed=64) == B.MOE_ERR_INVALID_ARG
-    assert create(flags=B.MOE_FLAG_FP8, d_model=128, d_ff=128) == B.MOE_ERR_UNSUPPORTED
+    assert create(flags=B.MOE_FLAG_FP8, d_model=128, d_ff=128) == B.MOE_OK         # FP8 dispatch
+    assert create(flags=B.MOE_FLAG_FP8, d_model=64, d_ff=128) == B.MOE_ERR_ALIGNMENT   # the FP8 rule holds
     # the row buffers of a rank hold every rank's rows: 4 x 4096 x 2 rows (+ 255 per local expert)
     # against 4096 x 2 (+ 255 per expert)
     one = B.moe_workspace_bytes(B.moe_config(64, 8, 64, 0, 0, 4096, 2, 0, 0, 0, 0, 0, 0))[1]

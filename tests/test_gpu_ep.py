@@ -119,6 +119,52 @@ def test_expert_parallel_v3_on_eight_ranks_node_limited():
     _run_case(shape, 8, [512] * 8, (8, 4), 0, repeats=1, oracle_rows_per_rank=2)
 
 
+@pytest.mark.parametrize("G,Ts", [(2, [300, 333]), (4, [257, 0, 129, 200])])
+def test_expert_parallel_fp8_layer_equals_the_single_gpu_fp8_layer(G, Ts):
+    """The FP8 layer split over G ranks: the dispatch sends each row's E4M3 codes and scale bytes
+    (quantized once, 1 x 128 groups, as moe_forward_fp8 does), the owners run the FP8 expert GEMMs;
+    every rank's output bit-identical to moe_forward_fp8 on its tokens."""
+    shape = LS("ep_fp8", T=sum(Ts), d=256, N=16, I=256, K=4, Ks=1, Is=128, sigma=0.05, seed=86)
+    host, dev = H.device_inputs(shape)
+    cut = _split(shape, Ts)
+    xs = [dev["x"][cut[r]:cut[r + 1]] for r in range(G)]
+    qw = tuple(B.quantize_fp8_blocks(dev[k]) for k in ("w_gate", "w_up", "w_down"))
+    qs = tuple(B.quantize_fp8_blocks(dev[k]) for k in ("ws_gate", "ws_up", "ws_down"))
+    per = shape.N // G
+    layers = []
+    for r in range(G):
+        layer = B.ExpertParallelLayer(ep_ranks=G, ep_rank=r, d_model=shape.d, n_routed=shape.N, d_ff=shape.I,
+                                      n_shared=shape.Ks, d_ff_shared=shape.Is, max_tokens=max(Ts), max_k=shape.K,
+                                      flags=B.MOE_FLAG_FP8)
+        layer.set_weights(dev["router"], (dev["w_gate"], dev["w_up"], dev["w_down"]),
+                          (dev["ws_gate"], dev["ws_up"], dev["ws_down"]))
+        sl = slice(r * per, (r + 1) * per)
+        layer.set_weights_fp8(tuple((c[sl], sc[sl]) for c, sc in qw), qs)
+        layers.append(layer)
+    B.connect_emulated(layers)
+    outs = B.forward_emulated(layers, xs, shape.K)
+    single = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks, d_ff_shared=shape.Is,
+                        max_tokens=max(Ts), max_k=shape.K, flags=B.MOE_FLAG_FP8)
+    single.set_weights(dev["router"], (dev["w_gate"], dev["w_up"], dev["w_down"]),
+                       (dev["ws_gate"], dev["ws_up"], dev["ws_down"]))
+    single.set_weights_fp8(qw, qs)
+    for r in range(G):
+        assert layers[r].status() == B.MOE_OK
+        if Ts[r] == 0:
+            continue
+        want = single.forward_fp8(xs[r], shape.K)
+        assert single.status() == B.MOE_OK
+        assert torch.equal(outs[r].view(torch.int16), want.view(torch.int16)), f"rank {r}"
+    # on an FP8 handle the bf16 experts step is refused (the rows arrived as FP8 codes)
+    layers[0].route(xs[0], shape.K)
+    layers[0].dispatch()
+    assert B.moe_ep_experts(layers[0].h, layers[0].experts, layers[0].shared, None) == B.MOE_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    for layer in layers:
+        layer.close()
+    single.close()
+
+
 def test_expert_parallel_calls_check_their_order_and_peers():
     shape = LS("ep_args", T=256, d=128, N=8, I=64, K=2, Ks=1, Is=64, sigma=0.05, seed=84)
     host, dev = H.device_inputs(shape)
