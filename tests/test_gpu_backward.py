@@ -77,11 +77,11 @@ def _compare_wgrad(got, want, what):
     assert rms_err <= 1e-2 * rms, f"{what}: rms diff {rms_err:.3e} > 1e-2 * rms {rms:.3e}"
 
 
-def _oracle_dgate(shape, host, dh, idx, rows=None):
+def _oracle_dgate(shape, host, dh, idx, rows=None, experts=None):
     """dL/dg = dh . FFN_e(u) per (token, slot) for the experts idx [n, K], from the oracle's FFN."""
     u = O.f64(host["x"]) if rows is None else O.f64(host["x"])[rows]
     dh = O.f64(dh) if rows is None else O.f64(dh)[rows]
-    experts = H.oracle_experts(shape, host)
+    experts = experts if experts is not None else H.oracle_experts(shape, host)
     fn = experts if callable(experts) else (lambda e: (experts[0][e], experts[1][e], experts[2][e]))
     dg = np.zeros(idx.shape)
     for ex in np.unique(idx):
@@ -177,10 +177,13 @@ def test_backward_checks_its_forward():
     assert layer.status() == B.MOE_OK
 
 
-def test_backward_16b_prefill_every_tile():
-    """The 16B prefill layer's backward on a token set with a row in every GEMM tile: dx and dgate of
-    those tokens (tokens are independent in both, so the oracle runs on them alone)."""
-    shape = W.CONFIGS["16b_prefill"]
+@pytest.mark.parametrize("name", ["16b_prefill", "2b", "v3"])
+def test_backward_full_size_every_tile(name):
+    """A full-size layer's backward on a token set with a row in every GEMM tile: dx and dgate of
+    those tokens (tokens are independent in both, so the oracle runs on them alone).  The 2B layer
+    has an odd number of routed experts (63) and a logit bias; V3 the sigmoid gate with a selection
+    bias over 256 experts."""
+    shape = W.CONFIGS[name]
     host, dev = H.device_inputs(shape)
     dh_host = W.output_gradient(shape)
     dh = dh_host.to("cuda")
@@ -192,17 +195,19 @@ def test_backward_16b_prefill_every_tile():
     dx, dgate, _, _ = layer.backward(dev["x"], shape.K, dh)
     assert layer.status() == B.MOE_OK
     gpu_idx = layer.routing(shape.T, shape.K)[0].cpu().numpy()
-    ok = ref.gap[rows] >= H.GAP_EXEMPT
-    rows = rows[ok]
+    layer.close()
+    rows = rows[ref.gap[rows] >= H.GAP_EXEMPT]
     sub = O.route(host["x"][rows], host["router"], shape.K, shape.gate, host["logit_bias"], host["select_bias"])
+    _same_expert_sets(gpu_idx[rows], sub.idx)
     u = O.f64(host["x"])[rows]
     dhr = O.f64(dh_host)[rows]
-    experts = H.oracle_experts(shape, host)
+    experts = H.oracle_experts(shape, host, prefetch=np.unique(sub.idx))
     fn = experts if callable(experts) else (lambda e: (experts[0][e], experts[1][e], experts[2][e]))
     du = dhr.copy()
-    sg, su, sd = (O.f64(w) for w in H.oracle_shared(shape, host))
-    for j in range(shape.Ks):
-        du += OB.swiglu_ffn_backward(u, sg[j], su[j], sd[j], dhr)[0]
+    if shape.Ks:
+        sg, su, sd = (O.f64(w) for w in H.oracle_shared(shape, host))
+        for j in range(shape.Ks):
+            du += OB.swiglu_ffn_backward(u, sg[j], su[j], sd[j], dhr)[0]
     dg = np.zeros(sub.idx.shape)
     for ex in np.unique(sub.idx):
         r, k = np.nonzero(sub.idx == ex)
@@ -211,8 +216,7 @@ def test_backward_16b_prefill_every_tile():
         np.add.at(du, r, OB.swiglu_ffn_backward(u[r], wg, wu, wd, sub.gate[r, k][:, None] * dhr[r])[0])
     dz = OB.gate_logit_backward(sub.s, sub.idx, sub.gate, dg, shape.gate)
     du += dz @ O.f64(host["router"])
-    _same_expert_sets(gpu_idx[rows], sub.idx)
-    dg_gpu_order = _oracle_dgate(shape, host, dh_host, gpu_idx[rows], rows)
-    e1 = _compare(_rows(dgate)[rows], dg_gpu_order, "16b_prefill dgate", 2e-2)
-    e2 = _compare(_rows(dx)[rows], du, "16b_prefill dx", 2e-2)
-    print(f"16b_prefill backward: {rows.size} rows; dgate max/rms err {e1}, dx {e2}")
+    dg_gpu_order = _oracle_dgate(shape, host, dh_host, gpu_idx[rows], rows, experts)
+    e1 = _compare(_rows(dgate)[rows], dg_gpu_order, f"{name} dgate", 2e-2)
+    e2 = _compare(_rows(dx)[rows], du, f"{name} dx", 2e-2)
+    print(f"{name} backward: {rows.size} rows; dgate max/rms err {e1}, dx {e2}")
