@@ -76,6 +76,9 @@ def parse_args():
                    help="time the FP8 1x128 quantization of one forward's permuted activations instead")
     p.add_argument("--training-step", action="store_true",
                    help="time only the layer's training step (forward + backward) on the --config workload")
+    p.add_argument("--ep-emulate", type=int, default=0, metavar="G",
+                   help="the expert-parallel layer with G ranks emulated on this GPU (each rank T / G tokens "
+                        "and mN / G experts), against the single-GPU layer on the same tokens")
     return p.parse_args()
 
 
@@ -666,6 +669,76 @@ def estimate_step_s(B, shape: W.LayerShape, d_in: dict, dev, local: int) -> floa
     return dt
 
 
+def run_ep_emulated(args):
+    """One JSON line: the expert-parallel forward with G ranks emulated on one GPU (G handles whose
+    kernels address each other's workspaces, the steps of all ranks in order on one stream, so the
+    time is the sum of the ranks' kernels and no NVLink transfer is measured), beside the single-GPU
+    layer on the same T tokens.  The V3 workload routes each token to at most 4 ranks when G = 8."""
+    from fine_grained_shared_b200 import moe as B
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    shape = W.CONFIGS[args.config]
+    G = args.ep_emulate
+    if G < 2 or shape.N % G or shape.T % G:
+        raise SystemExit(f"--ep-emulate {G}: needs G >= 2 dividing mN = {shape.N} and T = {shape.T}")
+    node_limit = (8, 4) if (shape.name == "v3" and G == 8) else None
+    host, d_in = device_layer_inputs(shape, dev)
+    Tr, per = shape.T // G, shape.N // G
+    xs = [d_in["x"][r * Tr:(r + 1) * Tr] for r in range(G)]
+    shared = (d_in["ws_gate"], d_in["ws_up"], d_in["ws_down"]) if shape.Ks else None
+    layers = []
+    for r in range(G):
+        layer = B.ExpertParallelLayer(ep_ranks=G, ep_rank=r, d_model=shape.d, n_routed=shape.N, d_ff=shape.I,
+                                      n_shared=shape.Ks, d_ff_shared=shape.Is, max_tokens=Tr, max_k=shape.K,
+                                      gate=shape.gate, node_limit=node_limit)
+        sl = slice(r * per, (r + 1) * per)
+        layer.set_weights(d_in["router"], (d_in["w_gate"][sl], d_in["w_up"][sl], d_in["w_down"][sl]), shared,
+                          logit_bias=d_in["logit_bias"], select_bias=d_in["select_bias"])
+        layers.append(layer)
+    B.connect_emulated(layers)
+    single = B.MoELayer(d_model=shape.d, n_routed=shape.N, d_ff=shape.I, n_shared=shape.Ks, d_ff_shared=shape.Is,
+                        max_tokens=shape.T, max_k=shape.K, gate=shape.gate, node_limit=node_limit)
+    single.set_weights(d_in["router"], (d_in["w_gate"], d_in["w_up"], d_in["w_down"]), shared,
+                       logit_bias=d_in["logit_bias"], select_bias=d_in["select_bias"])
+    outs = [torch.empty_like(x) for x in xs]
+    out1 = torch.empty_like(d_in["x"])
+    warmup, steps = max(3, args.warmup), max(3, args.steps)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / steps
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    ms_ep = timed(lambda: B.forward_emulated(layers, xs, shape.K, outs))
+    ms_1 = timed(lambda: single.forward(d_in["x"], shape.K, out1))
+    clk = clocks.stop()
+    for layer in layers:
+        st = layer.status()
+        if st != B.MOE_OK:
+            raise B.MoEError(st, "expert-parallel forward")
+    same = all(torch.equal(outs[r].view(torch.int16), out1[r * Tr:(r + 1) * Tr].view(torch.int16))
+               for r in range(G)) if Tr > 256 or shape.T <= 256 else None
+    line = {"metric": "MoE layer fwd tokens/s, expert-parallel ranks emulated on one GPU", "value": shape.T / (ms_ep * 1e-3),
+            "unit": UNIT, "n_gpus": 1, "ep_ranks_emulated": G, "steps": steps, "warmup": warmup,
+            "ms_per_step": ms_ep, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": workload_config(shape, f"ep{G}-emulated"),
+            "single_gpu_ms_per_step": ms_1, "node_limit": node_limit,
+            "bit_identical_to_single_gpu": same, "clocks": clk}
+    print(json.dumps(line), flush=True)
+    for layer in layers:
+        layer.close()
+    single.close()
+
+
 def run_training_step(args):
     """One JSON line for the layer's training step alone (moe_forward + moe_backward) on --config."""
     from fine_grained_shared_b200 import moe as B
@@ -917,6 +990,8 @@ def main():
         run_fp8_quant(args)
     elif args.training_step:
         run_training_step(args)
+    elif args.ep_emulate:
+        run_ep_emulated(args)
     else:
         run_ours(args)
 

@@ -1957,6 +1957,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     g.die_split = h->num_sms / 2;
     g.err = h->at<uint32_t>(L.err);
     g.timeout_ns = kTimeoutNs;
+    g.debug_wait = (c.flags & MOE_FLAG_DEBUG_WAIT_TIMEOUT) ? 1 : 0;
     const int sh_tiles = do_shared ? ceil_div(T, kGuBM) * g.sh_n_tiles : 0;
     const int ctas = do_routed || sh_tiles > h->num_sms ? h->num_sms : sh_tiles;
     const CUtensorMap& sA = do_shared ? h->tm_x.map : h->tm_xperm;

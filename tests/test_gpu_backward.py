@@ -158,6 +158,28 @@ def test_backward_is_deterministic():
                            b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32))
 
 
+def test_backward_wait_timeout_is_reported():
+    """The test-only flag makes CTA 0 of the backward's recompute wait 20 ms on a barrier nothing
+    arrives on: the backward reports MOE_ERR_TIMEOUT, and a new handle's backward is correct."""
+    shape = SHAPES["softmax_logit_bias"]
+    host, dev = H.device_inputs(shape)
+    dh = W.output_gradient(shape).to("cuda")
+    bad = H.make_layer(shape, dev, flags=B.MOE_FLAG_DEBUG_WAIT_TIMEOUT)
+    bad.forward(dev["x"], shape.K)
+    assert bad.status() == B.MOE_ERR_TIMEOUT        # the forward's GEMM took the flag too
+    bad.backward(dev["x"], shape.K, dh)
+    assert bad.status() == B.MOE_ERR_TIMEOUT
+    assert bad.status() == B.MOE_OK
+    bad.close()
+    good = H.make_layer(shape, dev)
+    H.run(good, dev["x"], shape.K)
+    dx = good.backward(dev["x"], shape.K, dh)[0]
+    assert good.status() == B.MOE_OK
+    want = H.make_layer(shape, dev)
+    H.run(want, dev["x"], shape.K)
+    assert torch.equal(dx.view(torch.int16), want.backward(dev["x"], shape.K, dh)[0].view(torch.int16))
+
+
 def test_backward_checks_its_forward():
     shape = SHAPES["softmax_logit_bias"]
     host, dev = H.device_inputs(shape)
