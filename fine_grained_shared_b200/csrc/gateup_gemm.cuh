@@ -444,7 +444,9 @@ __global__ void __launch_bounds__(kGuThreads, 1)
               pm[j] = valid ? pack_bf16x2(m2[0], m2[1]) : 0u;
             }
             if (mT) {
-              // column-major stores: the warp's 32 rows of one column are 64 contiguous bytes
+              // column-major stores of two rows at a time: lanes 2i and 2i + 1 (rows r and r + 1)
+              // swap half their columns, so that the even lane holds both rows of columns 0-7 and the
+              // odd lane both rows of columns 8-15; each 4-byte store covers two rows of one column
               __nv_bfloat16* dT = c.shared ? a.sh_dabT : a.dabT;
               size_t ra, rb;  // rows of da and db of column col in dT
               if (c.shared) {
@@ -455,15 +457,35 @@ __global__ void __launch_bounds__(kGuThreads, 1)
                 ra = static_cast<size_t>(col);
                 rb = ra + a.n_limit;
               }
+              const bool odd = (lane & 1) != 0;
+              const size_t r2 = row & ~static_cast<size_t>(1);  // the pair's first row
+              const int cbase = odd ? 8 : 0;                       // the columns this lane stores
+              uint32_t own[3][4], other[3][4];
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const uint32_t sel = (j & 1) ? 16u : 0u;
-                const uint16_t mv = static_cast<uint16_t>(pm[j >> 1] >> sel);
-                const uint16_t av = valid ? static_cast<uint16_t>(pa[j >> 1] >> sel) : uint16_t(0);
-                const uint16_t bv = valid ? static_cast<uint16_t>(pb[j >> 1] >> sel) : uint16_t(0);
-                reinterpret_cast<uint16_t*>(mT)[static_cast<size_t>(col + j) * ldT + row] = mv;
-                reinterpret_cast<uint16_t*>(dT)[(ra + j) * ldT + row] = av;
-                reinterpret_cast<uint16_t*>(dT)[(rb + j) * ldT + row] = bv;
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t am = valid ? pa[j] : 0u, an = valid ? pa[4 + j] : 0u;
+                const uint32_t bm = valid ? pb[j] : 0u, bn = valid ? pb[4 + j] : 0u;
+                own[0][j] = odd ? pm[4 + j] : pm[j];
+                own[1][j] = odd ? an : am;
+                own[2][j] = odd ? bn : bm;
+                // the partner needs the other half: an odd lane sends columns 0-7, an even one 8-15
+                other[0][j] = __shfl_xor_sync(0xffffffffu, odd ? pm[j] : pm[4 + j], 1);
+                other[1][j] = __shfl_xor_sync(0xffffffffu, odd ? am : an, 1);
+                other[2][j] = __shfl_xor_sync(0xffffffffu, odd ? bm : bn, 1);
+              }
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const uint32_t sh = (q & 1) ? 16u : 0u;
+                uint32_t w[3];
+#pragma unroll
+                for (int v = 0; v < 3; ++v) {
+                  const uint32_t mine = (own[v][q >> 1] >> sh) & 0xFFFFu, theirs = (other[v][q >> 1] >> sh) & 0xFFFFu;
+                  w[v] = odd ? (theirs | (mine << 16)) : (mine | (theirs << 16));  // row r2 low, r2 + 1 high
+                }
+                const size_t cc2 = static_cast<size_t>(cbase + q);
+                *reinterpret_cast<uint32_t*>(mT + (col + cc2) * ldT + r2) = w[0];
+                *reinterpret_cast<uint32_t*>(dT + (ra + cc2) * ldT + r2) = w[1];
+                *reinterpret_cast<uint32_t*>(dT + (rb + cc2) * ldT + r2) = w[2];
               }
             }
             __nv_bfloat16* pda;
