@@ -16,6 +16,8 @@ import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import oracle as O
 from fine_grained_shared_b200 import moe as B
@@ -97,6 +99,27 @@ def test_plan_matches_the_counting_sort_of_the_concatenated_batch(G, N, K, Ts):
         assert np.unique(taken).size == taken.size
         want = np.concatenate([np.arange(rs[l], rs[l] + cnt[l]) for l in range(per)])
         np.testing.assert_array_equal(np.sort(taken), want)
+
+
+@settings(max_examples=60, deadline=None)
+@given(st.integers(min_value=0, max_value=3), st.integers(min_value=1, max_value=8), st.data())
+def test_plan_on_random_splits(log_g, per_rank, data):
+    """Any G in {2, 4, 8} (and 1 expert per rank and up), K up to 8, ragged batches including empty
+    ranks: the plan still places every rank's rows at the concatenated batch's counting-sort rows."""
+    G = 2 ** max(1, log_g)
+    N = G * per_rank
+    K = data.draw(st.integers(min_value=1, max_value=min(8, N)))
+    Ts = data.draw(st.lists(st.integers(min_value=0, max_value=300), min_size=G, max_size=G))
+    rng = np.random.default_rng(data.draw(st.integers(min_value=0, max_value=2**31)))
+    idx_list = [_routing(rng, T, K, N) for T in Ts]
+    counts_all = np.stack([_counts(i, N) for i in idx_list])
+    dest, tables = _expected(idx_list, N, G)
+    for r in range(G):
+        st_, base, cnt, rs, mt, m1 = B.moe_ep_plan(counts_all, G, N, r)
+        assert st_ == B.MOE_OK
+        np.testing.assert_array_equal(_planned_rows(base, idx_list[r], N), dest[r][1])
+        for got, want in zip((cnt, rs, mt, m1), tables[r]):
+            np.testing.assert_array_equal(got, want)
 
 
 def test_plan_rejects_bad_arguments():
