@@ -1,5 +1,5 @@
 // backward.cuh -- the streaming and CUDA-core steps of the layer's backward
-// pass for the input and the router (DeepSeek-V3 technical report summary,
+// pass: input, router and expert-weight gradients (DeepSeek-V3 technical report summary,
 // section 3.2.1 "DualPipe and Computation-Communication Overlap": the MoE
 // layer's backward for input and backward for weights are separate pieces of
 // a training step; the formulas are the chain rule through the forward).

@@ -326,7 +326,8 @@ moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, uint
 moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, int32_t cols, uint8_t* q,
                                    uint8_t* scale, void* stream);
 
-/* The backward pass for the input and the router (DeepSeek-V3 technical
+/* The backward pass: gradients for the input, the router and the expert
+ * weights (DeepSeek-V3 technical
  * report summary, section 3.2.1 "DualPipe and Computation-Communication
  * Overlap": a training step runs the MoE layer's backward for input and its
  * backward for weights as separate pieces; the pages print no formula, so
@@ -356,7 +357,8 @@ moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, i
  * db = g dm SiLU(a) with dm = W_down^T dh.  The debug flags leave the same
  * terms out as in the forward (a left-out part's weight gradients are zero).
  *
- * Asynchronous on `stream`.  The first call allocates the backward's buffers
+ * Asynchronous on `stream`, which must be the forward's stream or ordered after
+ * it.  The first call allocates the backward's buffers
  * (a K-major copy of the expert weights, rewritten by every call, and
  * activations of the forward's row count).  Errors: the last forward was not a
  * moe_forward with this T and K, or another argument error of moe_forward
