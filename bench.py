@@ -519,11 +519,11 @@ def measure_layer(B, shape: W.LayerShape, host: dict, d_in: dict, dev, local: in
 
 
 def measure_training_step(B, shape: W.LayerShape, d_in: dict, dev, local: int, ranks, warmup: int,
-                          fwd_ms: float, peaks: dict, peak_src: str) -> dict:
+                          fwd_ms: float, peaks: dict, peak_src: str, steps: int = 0) -> dict:
     """The layer's training step on the headline workload: moe_forward, then moe_backward for a seeded
     upstream gradient dh, with every gradient asked for (dx, the gates', the router's and the expert
     and shared weights' in fp32).  Timed like the forward (CUDA events on the launching stream over
-    at least ~0.5 s, barrier + synchronize on both sides, max over ranks).  Algorithmic FLOPs: the
+    at least ~0.5 s unless `steps` fixes the count, barrier + synchronize on both sides, max over ranks).  Algorithmic FLOPs: the
     forward's, plus twice them for the backward (each GEMM of the forward has one for its input and
     one for its weights); the backward also recomputes the gate/up GEMM (executed FLOPs, reported
     beside them)."""
@@ -547,7 +547,8 @@ def measure_training_step(B, shape: W.LayerShape, d_in: dict, dev, local: int, r
     est = time.perf_counter()
     step()
     torch.cuda.synchronize(dev)
-    steps = max(10, int(0.5 / max(time.perf_counter() - est, 1e-6)))
+    if steps <= 0:
+        steps = max(10, int(0.5 / max(time.perf_counter() - est, 1e-6)))
     st = layer.status()
     if st != B.MOE_OK:
         raise B.MoEError(st, "training step warm-up")
@@ -753,7 +754,8 @@ def run_training_step(args):
     peaks, peak_src = measured_peaks()
     fwd = measure_layer(B, shape, host, d_in, dev, local, ranks, max(3, args.steps), max(3, args.warmup),
                         with_e2e=False)
-    t = measure_training_step(B, shape, d_in, dev, local, ranks, max(3, args.warmup), fwd["ms_step"], peaks, peak_src)
+    t = measure_training_step(B, shape, d_in, dev, local, ranks, max(3, args.warmup), fwd["ms_step"], peaks, peak_src,
+                              steps=args.steps)
     line = {"metric": "MoE layer training step (forward + backward) tokens/s", "value": t["tokens_per_s"],
             "unit": UNIT, "n_gpus": ranks.world, "steps": t["steps"], "warmup": max(3, args.warmup),
             "ms_per_step": t["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -168,16 +168,31 @@ __global__ void fill_dense_groups_kernel(int32_t* k_start, int32_t* k_count, int
 }
 
 // ---------------------------------------------------------------------------
-// dh into the expert-ordered rows: dh_perm[slot[t, k]] = dh[t]; a warp per (t, k)
+// dh into the expert-ordered rows: dh_perm[slot[t, k]] = dh[t], and (dy not null)
+// dy[slot[t, k]] = g[t, k] dh[t], the weight gradient's operand; a warp per (t, k)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) bwd_gather_kernel(const __nv_bfloat16* __restrict__ dh, const int32_t* slot_of,
-                                                        int TK, int K, int d, __nv_bfloat16* dh_perm) {
+                                                        int TK, int K, int d, __nv_bfloat16* dh_perm,
+                                                        const float* gate, __nv_bfloat16* dy) {
   const int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (w >= TK) return;
   const int t = w / K;
+  const size_t row = static_cast<size_t>(slot_of[w]);
   const uint4* s = reinterpret_cast<const uint4*>(dh + static_cast<size_t>(t) * d);
-  uint4* o = reinterpret_cast<uint4*>(dh_perm + static_cast<size_t>(slot_of[w]) * d);
-  for (int c = lane; c < (d >> 3); c += 32) o[c] = __ldg(s + c);
+  uint4* o = reinterpret_cast<uint4*>(dh_perm + row * d);
+  uint4* oy = dy ? reinterpret_cast<uint4*>(dy + row * d) : nullptr;
+  const float g = dy ? gate[w] : 0.f;
+  for (int c = lane; c < (d >> 3); c += 32) {
+    const uint4 v = __ldg(s + c);
+    o[c] = v;
+    if (oy) {
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+      uint32_t q[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) q[j] = pack_bf16x2(g * bf16lo(wv[j]), g * bf16hi(wv[j]));
+      oy[c] = make_uint4(q[0], q[1], q[2], q[3]);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -61,6 +61,21 @@ constexpr uint32_t kBoxRowsB = kGemmBN / 2;
 static_assert(kStageA == kBoxRowsA * kGemmBK * 2 && kStageB == kBoxRowsB * kGemmBK * 2, "stage = one TMA box");
 
 
+// Shared-memory matrix descriptor of an MN-major operand in the 128-byte swizzle: the tile is stored as
+// chunks of 64 MN elements (128 bytes) x its K rows, chunk after chunk `lbo` bytes apart, each chunk's
+// rows 128 bytes apart with the 16-byte units of row r XOR-ed with r % 8 (the layout a TMA box of
+// 64 MN elements x K rows writes); groups of 8 K rows are 1024 bytes apart.  A step of 16 K rows
+// moves the start address by 2048 bytes.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>(1024u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(2u) << 61;
+  return d;
+}
+
 struct GemmArgs {
   // routed experts (grouped rows of H; tiles after the shared ones)
   int num_groups;              // experts; 0: no routed tiles
@@ -96,6 +111,11 @@ struct GemmArgs {
   int kg_bz_step;
   int kg_split;
   int kg_ld;                   // output row stride (>= n_limit, a multiple of 16)
+  // 1: both operands MN-major -- row-major [K rows][MN columns] buffers read through 2-D maps with
+  // 64 x 64 boxes, two per operand and stage; group g's A columns start at g * kg_a_row_step and its B
+  // columns at g * kg_b_col_step (with kg_bz_step set); 0: K-major operands as described above
+  int kg_mn;
+  int kg_b_col_step;
   float* kg_out;               // [groups][kg_split][kg_ld]
   float* kg_out2;              // [groups][kg_M - kg_split][kg_ld]
 };
@@ -236,7 +256,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int g = tile / kg_per_group, local = tile - g * kg_per_group;
         const int mt = local / a.n_tiles, nt = local - mt * a.n_tiles;
         const int arow = g * a.kg_a_row_step + mt * kGemmBM + static_cast<int>(rank) * kCtaRows;
-        const int brow = nt * kGemmBN + static_cast<int>(rank) * (kGemmBN / 2);
+        const int brow = (a.kg_mn && a.kg_bz_step ? g * a.kg_b_col_step : 0) + nt * kGemmBN +
+                         static_cast<int>(rank) * (kGemmBN / 2);
         const int bz = a.kg_bz_step ? g : 0;
         const int nkb = (s_mts[g] + kGemmBK - 1) / kGemmBK;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -248,8 +269,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kStageA + kStageB));
           const int kc = s_rows[g] + kb * kGemmBK;
           const uint32_t fb = full_lead + 8u * static_cast<uint32_t>(s);
-          tma_load_2d_pair(sA + s * kStageA, &tmA, fb, kc, arow);
-          tma_load_3d_pair(sB + s * kStageB, &tmB, fb, kc, brow, bz);
+          if (a.kg_mn) {  // MN-major: x = the MN column, y = the K row; two 64-column boxes per operand
+            tma_load_2d_pair(sA + s * kStageA, &tmA, fb, arow, kc);
+            tma_load_2d_pair(sA + s * kStageA + kStageA / 2, &tmA, fb, arow + 64, kc);
+            tma_load_2d_pair(sB + s * kStageB, &tmB, fb, brow, kc);
+            tma_load_2d_pair(sB + s * kStageB + kStageB / 2, &tmB, fb, brow + 64, kc);
+          } else {
+            tma_load_2d_pair(sA + s * kStageA, &tmA, fb, kc, arow);
+            tma_load_3d_pair(sB + s * kStageB, &tmB, fb, kc, brow, bz);
+          }
           ++issued;
           if (++s == kGemmStages) {
             s = 0;
@@ -301,7 +329,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------- MMA issuer (even CTA) --------------------------
-    const uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN);
+    // MN-major operands (weight-gradient mode): bits 15 and 16 of the instruction descriptor
+    const uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN) | (KG && a.kg_mn ? (1u << 15) | (1u << 16) : 0u);
+    const bool mn = KG && a.kg_mn;
     int s = 0, acc = 0;
     uint32_t ph = 0, acc_ph = 0;
     if (a.debug_wait && blockIdx.x == 0) {
@@ -327,11 +357,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after_sync();
-        const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + s * kStageA));
-        const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + s * kStageB));
+        // K-major: 16 K columns are 32 bytes along a row (+2 in 16-byte units); MN-major: 16 K rows of
+        // 128 bytes (+128), the two 64-element MN chunks of a stage 8 KB apart
+        const uint64_t ad = mn ? sw128_mnmajor_desc(smem_u32(sA + s * kStageA), kStageA / 2)
+                               : sw128_kmajor_desc(smem_u32(sA + s * kStageA));
+        const uint64_t bd = mn ? sw128_mnmajor_desc(smem_u32(sB + s * kStageB), kStageB / 2)
+                               : sw128_kmajor_desc(smem_u32(sB + s * kStageB));
+        const uint64_t kstep = mn ? 128u : 2u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss_pair(d_tmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_bf16_ss_pair(d_tmem, ad + kstep * kk, bd + kstep * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
         umma_commit_pair_multicast(&empty[s], 0x3);
         if (++s == kGemmStages) {
           s = 0;

@@ -82,15 +82,11 @@ struct GateUpArgs {
   const float* row_gate;       // routed: the gate of each row
   float* dg_part;              // routed: [rows, n_tiles] per 128-column tile, sum of dm * m over its columns
   int sh_I;                    // shared: columns of one shared expert (I_s)
-  // for the weight gradients (nullptr: not written): m, da and db transposed -- column c of a
-  // row r at [c][r] -- with zeros in the rows that hold no (token, slot) pair
+  // for the weight gradients (nullptr: not written): m row by row, and zeros in every output row
+  // (m, da, db) that holds no (token, slot) pair, since the weight-gradient GEMMs sum over rows
   const int32_t* counts;       // routed: [G] rows of each expert (the rest of its segment is padding)
-  __nv_bfloat16* mT;           // routed: [I][ldT]
-  __nv_bfloat16* dabT;         // routed: [2 I][ldT], da rows then db rows
-  long long ldT;
-  __nv_bfloat16* sh_mT;        // shared: [K_s I_s][sh_ldT]
-  __nv_bfloat16* sh_dabT;      // shared: [K_s 2 I_s][sh_ldT], expert j's da rows then its db rows
-  long long sh_ldT;
+  __nv_bfloat16* m_out;        // routed: [rows, n_limit]
+  __nv_bfloat16* sh_m_out;     // shared: [T_pad, sh_n_limit]
 };
 
 constexpr int kGuQueue = 4;  // tile-id queue entries
@@ -409,8 +405,8 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         // in the transposed outputs, whose sums over rows would otherwise take it in
         const bool valid = c.shared ? static_cast<int>(row) < a.sh_rows
                                     : static_cast<int>(row) - s_rows[c.g] < s_cnt[c.g];
-        __nv_bfloat16* mT = c.shared ? a.sh_mT : a.mT;
-        const long long ldT = c.shared ? a.sh_ldT : a.ldT;
+        __nv_bfloat16* mrow = c.shared ? (a.sh_m_out ? a.sh_m_out + row * a.sh_n_limit : nullptr)
+                                       : (a.m_out ? a.m_out + row * a.n_limit : nullptr);
         float dg = 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < kGuBN / 2; cc += 16) {
@@ -443,49 +439,14 @@ __global__ void __launch_bounds__(kGuThreads, 1)
               pb[j] = pack_bf16x2(db2[0], db2[1]);
               pm[j] = valid ? pack_bf16x2(m2[0], m2[1]) : 0u;
             }
-            if (mT) {
-              // column-major stores of two rows at a time: lanes 2i and 2i + 1 (rows r and r + 1)
-              // swap half their columns, so that the even lane holds both rows of columns 0-7 and the
-              // odd lane both rows of columns 8-15; each 4-byte store covers two rows of one column
-              __nv_bfloat16* dT = c.shared ? a.sh_dabT : a.dabT;
-              size_t ra, rb;  // rows of da and db of column col in dT
-              if (c.shared) {
-                const int j = col / a.sh_I, i = col - j * a.sh_I;
-                ra = static_cast<size_t>(j) * 2 * a.sh_I + i;
-                rb = ra + a.sh_I;
-              } else {
-                ra = static_cast<size_t>(col);
-                rb = ra + a.n_limit;
-              }
-              const bool odd = (lane & 1) != 0;
-              const size_t r2 = row & ~static_cast<size_t>(1);  // the pair's first row
-              const int cbase = odd ? 8 : 0;                       // the columns this lane stores
-              uint32_t own[3][4], other[3][4];
+            if (mrow) {
+              uint4* q = reinterpret_cast<uint4*>(mrow + col);
+              q[0] = make_uint4(pm[0], pm[1], pm[2], pm[3]);
+              q[1] = make_uint4(pm[4], pm[5], pm[6], pm[7]);
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const uint32_t am = valid ? pa[j] : 0u, an = valid ? pa[4 + j] : 0u;
-                const uint32_t bm = valid ? pb[j] : 0u, bn = valid ? pb[4 + j] : 0u;
-                own[0][j] = odd ? pm[4 + j] : pm[j];
-                own[1][j] = odd ? an : am;
-                own[2][j] = odd ? bn : bm;
-                // the partner needs the other half: an odd lane sends columns 0-7, an even one 8-15
-                other[0][j] = __shfl_xor_sync(0xffffffffu, odd ? pm[j] : pm[4 + j], 1);
-                other[1][j] = __shfl_xor_sync(0xffffffffu, odd ? am : an, 1);
-                other[2][j] = __shfl_xor_sync(0xffffffffu, odd ? bm : bn, 1);
-              }
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const uint32_t sh = (q & 1) ? 16u : 0u;
-                uint32_t w[3];
-#pragma unroll
-                for (int v = 0; v < 3; ++v) {
-                  const uint32_t mine = (own[v][q >> 1] >> sh) & 0xFFFFu, theirs = (other[v][q >> 1] >> sh) & 0xFFFFu;
-                  w[v] = odd ? (theirs | (mine << 16)) : (mine | (theirs << 16));  // row r2 low, r2 + 1 high
-                }
-                const size_t cc2 = static_cast<size_t>(cbase + q);
-                *reinterpret_cast<uint32_t*>(mT + (col + cc2) * ldT + r2) = w[0];
-                *reinterpret_cast<uint32_t*>(dT + (ra + cc2) * ldT + r2) = w[1];
-                *reinterpret_cast<uint32_t*>(dT + (rb + cc2) * ldT + r2) = w[2];
+              for (int j = 0; j < 8; ++j) {
+                pa[j] = valid ? pa[j] : 0u;
+                pb[j] = valid ? pb[j] : 0u;
               }
             }
             __nv_bfloat16* pda;

@@ -201,9 +201,9 @@ struct BwdLayout {
   // the router's GEMM operands: logits, dz in bf16 (and transposed), E transposed, K-range tables
   size_t zf, dzb, dzT, ET, rt_kstart, rt_kcount;
   int64_t Npad;
-  // the weight gradients' operands: activations transposed (rows of the forward as columns)
-  size_t dyT, xpermT, mT, dabT, dhT, xT, msT, dabsT, sh_kstart, sh_kcount, total;
-  int64_t Pt;  // row count of the transposed routed activations (the forward's rows, padded to 64)
+  // the weight gradients' operands (row-major, read MN-major by the GEMMs): g dh and m per routed row,
+  // m per token of the shared experts; x transposed for the router's dE
+  size_t dy, mrows, msrows, xT, sh_kstart, sh_kcount, total;
 };
 
 BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
@@ -234,15 +234,10 @@ BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
   B.ET = take(size_t(d) * B.Npad * 2);
   B.rt_kstart = take(kDeMaxSegments * 4);
   B.rt_kcount = take(kDeMaxSegments * 4);
-  B.Pt = (L.P + 63) / 64 * 64;
-  B.dyT = take(size_t(d) * B.Pt * 2);
-  B.xpermT = take(size_t(d) * B.Pt * 2);
-  B.mT = take(size_t(I) * B.Pt * 2);
-  B.dabT = take(size_t(2 * I) * B.Pt * 2);
-  B.dhT = take(size_t(d) * L.Tpad * 2);
+  B.dy = take(size_t(L.P) * d * 2);
+  B.mrows = take(size_t(L.P) * I * 2);
+  B.msrows = take(size_t(L.Tpad) * Ks * Is * 2);
   B.xT = take(size_t(d) * L.Tpad * 2);
-  B.msT = take(size_t(Ks) * Is * L.Tpad * 2);
-  B.dabsT = take(size_t(Ks) * 2 * Is * L.Tpad * 2);
   B.sh_kstart = take(64 * 4);
   B.sh_kcount = take(64 * 4);
   B.total = o;
@@ -344,9 +339,9 @@ struct moe_ctx {
   // the backward's own buffers (allocated by its first call) and their descriptors
   uint8_t* bws = nullptr;
   CUtensorMap tm_b_dhperm, tm_b_wdT, tm_b_swdT, tm_b_dab, tm_b_wguT, tm_b_dabs, tm_b_swguT;
-  CUtensorMap tm_b_dyT, tm_b_xpermT, tm_b_mT, tm_b_dabT, tm_b_dhT, tm_b_xT, tm_b_msT, tm_b_dabsT;
+  CUtensorMap tm_w_dy, tm_w_m, tm_w_dab, tm_w_xperm, tm_w_ms, tm_w_dabs, tm_b_xT;  // 64 x 64 MN-major boxes
   CUtensorMap tm_b_dzb, tm_b_ET, tm_b_dzT;
-  MapCache tm_b_dh, tm_b_E;
+  MapCache tm_b_dh, tm_b_E, tm_w_dh, tm_w_x;
 
   template <typename T>
   T* at(size_t off) const {
@@ -932,6 +927,9 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
   ok = ok && cudaMemset(h->ws + h->L.ffn_ctr, 0, ffn_counter_bytes()) == cudaSuccess;
+  // X_perm's padding rows are never written by a forward: zero them once, so that they are finite
+  // (zero, or an earlier forward's token row) when the backward's weight gradients sum over them
+  ok = ok && cudaMemset(h->ws + h->L.x_perm, 0, size_t(h->L.P) * cfg->d_model * 2) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
@@ -1702,12 +1700,11 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
   }
   const int64_t N = c.n_routed, I = c.d_ff, d = c.d_model, Ks = c.n_shared, Is = c.d_ff_shared;
   bool ok = encode_bf16(&h->tm_b_dhperm, h->ws + L.y, 1, L.P, d, kBoxRowsA, 2);
-  // the weight gradients: A operands 2-D [rows][K = forward rows], B operands 3-D [groups][rows][K]
-  ok = ok && encode_bf16(&h->tm_b_dyT, h->bws + B.dyT, 1, d, B.Pt, kBoxRowsA, 2);
-  ok = ok && encode_bf16(&h->tm_b_dabT, h->bws + B.dabT, 1, 2 * I, B.Pt, kBoxRowsA, 2);
-  ok = ok && encode_bf16(&h->tm_b_mT, h->bws + B.mT, 1, I, B.Pt, kBoxRowsB, 3);
-  ok = ok && encode_bf16(&h->tm_b_xpermT, h->bws + B.xpermT, 1, d, B.Pt, kBoxRowsB, 3);
-  ok = ok && encode_bf16(&h->tm_b_dhT, h->bws + B.dhT, 1, d, L.Tpad, kBoxRowsA, 2);
+  // the weight gradients' operands: row-major [K = forward rows][MN], 64 K rows x 64 MN elements per box
+  ok = ok && encode_bf16(&h->tm_w_dy, h->bws + B.dy, 1, L.P, d, 64, 2);
+  ok = ok && encode_bf16(&h->tm_w_m, h->bws + B.mrows, 1, L.P, I, 64, 2);
+  ok = ok && encode_bf16(&h->tm_w_dab, h->bws + B.dab, 1, L.P, 2 * I, 64, 2);
+  ok = ok && encode_bf16(&h->tm_w_xperm, h->ws + L.x_perm, 1, L.P, d, 64, 2);
   ok = ok && encode_bf16(&h->tm_b_xT, h->bws + B.xT, 1, d, L.Tpad, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_dzb, h->bws + B.dzb, 1, c.max_tokens, B.Npad, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_ET, h->bws + B.ET, 1, d, B.Npad, kBoxRowsB, 3);
@@ -1719,11 +1716,11 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
     ok = ok && encode_bf16(&h->tm_b_swdT, h->bws + B.swdT, 1, Ks * Is, d, kBoxRowsB, 3);
     ok = ok && encode_bf16(&h->tm_b_dabs, h->bws + B.dabs, 1, L.Tpad, Ks * 2 * Is, kBoxRowsA, 2);
     ok = ok && encode_bf16(&h->tm_b_swguT, h->bws + B.swguT, Ks, d, 2 * Is, kBoxRowsB, 3);
-    ok = ok && encode_bf16(&h->tm_b_msT, h->bws + B.msT, Ks, Is, L.Tpad, kBoxRowsB, 3);
-    ok = ok && encode_bf16(&h->tm_b_dabsT, h->bws + B.dabsT, 1, Ks * 2 * Is, L.Tpad, kBoxRowsA, 2);
+    ok = ok && encode_bf16(&h->tm_w_ms, h->bws + B.msrows, 1, L.Tpad, Ks * Is, 64, 2);
+    ok = ok && encode_bf16(&h->tm_w_dabs, h->bws + B.dabs, 1, L.Tpad, Ks * 2 * Is, 64, 2);
   } else {
-    h->tm_b_msT = h->tm_b_mT;
-    h->tm_b_dabsT = h->tm_b_dabT;
+    h->tm_w_ms = h->tm_w_m;
+    h->tm_w_dabs = h->tm_w_dab;
     h->tm_b_swdT = h->tm_b_wdT;
     h->tm_b_dabs = h->tm_b_dab;
     h->tm_b_swguT = h->tm_b_wguT;
@@ -1784,7 +1781,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   // a GEMM in the per-group mode of down_gemm_kernel (fp32 out, rows >= split into out2)
   auto kg_gemm = [&](const CUtensorMap& A, const CUtensorMap& Bm, int groups, const int32_t* kstart,
                      const int32_t* kcount, int M, int a_step, int bz_step, int split, int Ncols, int ld, float* out,
-                     float* out2) {
+                     float* out2, int mn = 0, int b_col_step = 0) {
     GemmArgs k{};
     k.kg_groups = groups;
     k.kg_k_start = kstart;
@@ -1795,6 +1792,8 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     k.kg_bz_step = bz_step;
     k.kg_split = split;
     k.kg_ld = ld;
+    k.kg_mn = mn;
+    k.kg_b_col_step = b_col_step;
     k.kg_out = out;
     k.kg_out2 = out2;
     k.n_tiles = ceil_div(Ncols, kGemmBN);
@@ -1837,30 +1836,14 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   const int TK = (int)(T * K);
   // ---- dm: routed rows (dh gathered into the expert order, times W_down) and shared rows ----
   if (do_routed) {
+    // dy = g dh per routed row for the weight gradients: zero first, so that the padding rows the
+    // GEMMs' K ranges reach read as zeros
+    __nv_bfloat16* dy = wgrad ? reinterpret_cast<__nv_bfloat16*>(bw(B.dy)) : nullptr;
+    if (dy && cudaMemsetAsync(dy, 0, size_t(L.P) * d * 2, s0) != cudaSuccess) return MOE_ERR_CUDA;
     bwd_gather_kernel<<<ceil_div(int64_t(TK) * 32, 256), 256, 0, s0>>>(static_cast<const __nv_bfloat16*>(dh), slot_of,
-                                                                       TK, K, (int)d, h->at<__nv_bfloat16>(L.y));
+                                                                       TK, K, (int)d, h->at<__nv_bfloat16>(L.y),
+                                                                       h->at<float>(L.gate), dy);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-    if (wgrad) {
-      // dy = g dh and X_perm per row, transposed, zero on the rows without a pair
-      RowTransposeArgs rt{};
-      rt.R = (int)L.P;
-      rt.src_rows = (int)L.P;
-      rt.C = (int)d;
-      rt.dst_ld = B.Pt;
-      rt.row_start = h->at<int32_t>(L.row_start);
-      rt.counts = h->at<int32_t>(L.counts);
-      rt.G = (int)N;
-      const dim3 grid(ceil_div(d, kTrCols), ceil_div(L.P, kTrRows));
-      rt.src = h->at<__nv_bfloat16>(L.y);
-      rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dyT));
-      rt.scale = h->at<float>(L.gate_perm);
-      transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
-      rt.src = h->at<__nv_bfloat16>(L.x_perm);
-      rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xpermT));
-      rt.scale = nullptr;
-      transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
-      if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-    }
     GemmArgs g{};
     g.num_groups = (int)N;
     g.mtile_start = h->at<int32_t>(L.mtile);
@@ -1878,21 +1861,10 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       return MOE_ERR_CUDA;
   }
   if (do_shared && wgrad) {
-    // dh and x transposed, zero past the T tokens
-    RowTransposeArgs rt{};
-    rt.R = (int)L.Tpad;  // rows T .. Tpad are written as zeros, never read from the sources
-    rt.src_rows = (int)T;
-    rt.C = (int)d;
-    rt.dst_ld = L.Tpad;
-    rt.G = 0;
-    rt.row_limit = (int)T;
-    const dim3 grid(ceil_div(d, kTrCols), ceil_div(L.Tpad, kTrRows));
-    rt.src = static_cast<const __nv_bfloat16*>(dh);
-    rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dhT));
-    transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
-    rt.src = static_cast<const __nv_bfloat16*>(x);
-    rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
-    transpose_rows_kernel<<<grid, 256, 0, s0>>>(rt);
+    // the shared experts' weight gradients sum over the T tokens (dh and x read MN-major in place: the
+    // maps end at T, so the rows past it read as zeros)
+    if (!refresh(h->tm_w_dh, dh, T, 1, T, d, 64, 2) || !refresh(h->tm_w_x, x, T, 1, T, d, 64, 2))
+      return MOE_ERR_CUDA;
     fill_dense_groups_kernel<<<1, 64, 0, s0>>>(reinterpret_cast<int32_t*>(bw(B.sh_kstart)),
                                                reinterpret_cast<int32_t*>(bw(B.sh_kcount)), (int)Ks, (int)T);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -1932,9 +1904,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       g.dg_part = reinterpret_cast<float*>(bw(B.dg_part));
       if (wgrad) {
         g.counts = h->at<int32_t>(L.counts);
-        g.mT = reinterpret_cast<__nv_bfloat16*>(bw(B.mT));
-        g.dabT = reinterpret_cast<__nv_bfloat16*>(bw(B.dabT));
-        g.ldT = B.Pt;
+        g.m_out = reinterpret_cast<__nv_bfloat16*>(bw(B.mrows));
       }
     }
     if (do_shared) {
@@ -1946,11 +1916,7 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       g.sh_dm = h->at<__nv_bfloat16>(L.hs);
       g.sh_ld_dm = (int)(Ks * Is);
       g.sh_I = (int)Is;
-      if (wgrad) {
-        g.sh_mT = reinterpret_cast<__nv_bfloat16*>(bw(B.msT));
-        g.sh_dabT = reinterpret_cast<__nv_bfloat16*>(bw(B.dabsT));
-        g.sh_ldT = L.Tpad;
-      }
+      if (wgrad) g.sh_m_out = reinterpret_cast<__nv_bfloat16*>(bw(B.msrows));
     }
     g.num_kb = ceil_div(d, kGuBK);
     g.tile_ctr = h->at<int>(L.tile_ctr);
@@ -1999,11 +1965,12 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     if (do_routed) {
       const int32_t* ks = h->at<int32_t>(L.row_start);
       const int32_t* kc = h->at<int32_t>(L.counts);
-      ke = kg_gemm(h->tm_b_dyT, h->tm_b_mT, (int)N, ks, kc, (int)d, 0, 0, (int)d, (int)I, (int)I, wgrad->w_down,
-                   nullptr);
+      // MN-major operands straight from the row-major buffers: dW_down = dy^T m, dW_gate|up = [da|db]^T x
+      ke = kg_gemm(h->tm_w_dy, h->tm_w_m, (int)N, ks, kc, (int)d, 0, 0, (int)d, (int)I, (int)I, wgrad->w_down,
+                   nullptr, 1);
       if (ke == cudaSuccess)
-        ke = kg_gemm(h->tm_b_dabT, h->tm_b_xpermT, (int)N, ks, kc, (int)(2 * I), 0, 0, (int)I, (int)d, (int)d,
-                     wgrad->w_gate, wgrad->w_up);
+        ke = kg_gemm(h->tm_w_dab, h->tm_w_xperm, (int)N, ks, kc, (int)(2 * I), 0, 0, (int)I, (int)d, (int)d,
+                     wgrad->w_gate, wgrad->w_up, 1);
     } else {
       const size_t wb = size_t(N) * I * d * 4;
       if (cudaMemsetAsync(wgrad->w_gate, 0, wb, s0) != cudaSuccess ||
@@ -2014,11 +1981,11 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     if (Ks > 0 && do_shared && ke == cudaSuccess) {
       const int32_t* ks = reinterpret_cast<const int32_t*>(bw(B.sh_kstart));
       const int32_t* kc = reinterpret_cast<const int32_t*>(bw(B.sh_kcount));
-      ke = kg_gemm(h->tm_b_dhT, h->tm_b_msT, (int)Ks, ks, kc, (int)d, 0, 1, (int)d, (int)Is, (int)Is,
-                   wgrad->ws_down, nullptr);
+      ke = kg_gemm(h->tm_w_dh.map, h->tm_w_ms, (int)Ks, ks, kc, (int)d, 0, 1, (int)d, (int)Is, (int)Is,
+                   wgrad->ws_down, nullptr, 1, (int)Is);
       if (ke == cudaSuccess)
-        ke = kg_gemm(h->tm_b_dabsT, h->tm_b_xT, (int)Ks, ks, kc, (int)(2 * Is), (int)(2 * Is), 0, (int)Is, (int)d,
-                     (int)d, wgrad->ws_gate, wgrad->ws_up);
+        ke = kg_gemm(h->tm_w_dabs, h->tm_w_x.map, (int)Ks, ks, kc, (int)(2 * Is), (int)(2 * Is), 0, (int)Is, (int)d,
+                     (int)d, wgrad->ws_gate, wgrad->ws_up, 1);
     } else if (Ks > 0 && ke == cudaSuccess) {
       const size_t wb = size_t(Ks) * Is * d * 4;
       if (cudaMemsetAsync(wgrad->ws_gate, 0, wb, s0) != cudaSuccess ||
@@ -2086,13 +2053,11 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       t2.G = 0;
       t2.row_limit = (int)T;
       transpose_rows_kernel<<<dim3(ceil_div(Np, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t2);
-      if (!(do_shared && wgrad)) {
-        RowTransposeArgs t3 = t2;
-        t3.src = static_cast<const __nv_bfloat16*>(x);
-        t3.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
-        t3.C = (int)d;
-        transpose_rows_kernel<<<dim3(ceil_div(d, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t3);
-      }
+      RowTransposeArgs t3 = t2;
+      t3.src = static_cast<const __nv_bfloat16*>(x);
+      t3.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
+      t3.C = (int)d;
+      transpose_rows_kernel<<<dim3(ceil_div(d, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t3);
       const int want = (int)std::max<int64_t>(1, std::min<int64_t>(kDeMaxSegments, T / 512));
       const int seg = ceil_div(ceil_div(T, want), 64) * 64;
       const int segs = ceil_div(T, seg);
