@@ -16,9 +16,10 @@
 // ds_k = (dg_k - g . dg) / S, dz = ds s (1 - s) on the chosen experts):
 //   dE = dz^T x, d(logit bias) = sum_t dz.
 // This file holds the steps that are not tensor-core GEMMs: the weight
-// transposes that give the GEMMs K-major operands, the gather of dh into the
-// expert-ordered rows, the gate gradient's reduction, the router backward on
-// the CUDA cores (mN <= 256 dot products per token) and the final sum.
+// transposes that give the data-gradient GEMMs K-major operands, the gather of
+// dh into the expert-ordered rows (and g dh for the weight gradients), the gate
+// gradient's reduction, the router's dz step (the softmax or sigmoid Jacobian
+// per token; its three contractions run on the tensor cores) and the final sum.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -52,19 +53,13 @@ __device__ __forceinline__ void tr_load_tile(uint16_t (*tile)[kTrCols + 2], cons
   }
 }
 
-// dst row (c0 + oc), values of source rows r0 + orr .. + 15: thread (oc = tid / 4, orr = (tid % 4) * 16);
-// rowf / rowok (or nullptr): each row's scale and whether it holds a pair (zero if not)
-__device__ __forceinline__ void tr_store_row(const uint16_t (*tile)[kTrCols + 2], uint16_t* q, int nvalid,
-                                             const float* rowf, const int* rowok, int orr, int oc) {
+// dst row (c0 + oc), values of source rows r0 + orr .. + 15: thread (oc = tid / 4, orr = (tid % 4) * 16)
+__device__ __forceinline__ void tr_store_row(const uint16_t (*tile)[kTrCols + 2], uint16_t* q, int nvalid, int orr,
+                                             int oc) {
   uint32_t w[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    uint32_t lo = tile[orr + 2 * j][oc], hi = tile[orr + 2 * j + 1][oc];
-    if (rowf) {
-      lo = rowok[orr + 2 * j] ? (pack_bf16x2(rowf[orr + 2 * j] * __uint_as_float(lo << 16), 0.f) & 0xFFFFu) : 0u;
-      hi = rowok[orr + 2 * j + 1] ? (pack_bf16x2(rowf[orr + 2 * j + 1] * __uint_as_float(hi << 16), 0.f) & 0xFFFFu)
-                                  : 0u;
-    }
+    const uint32_t lo = tile[orr + 2 * j][oc], hi = tile[orr + 2 * j + 1][oc];
     w[j] = lo | (hi << 16);
   }
   if (nvalid >= 16 && (reinterpret_cast<uintptr_t>(q) & 15u) == 0) {
@@ -97,65 +92,7 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeArgs a) {
   __syncthreads();
   const int oc = threadIdx.x >> 2, orr = (threadIdx.x & 3) * 16;
   if (c0 + oc >= a.C || r0 + orr >= a.R) return;
-  tr_store_row(tile, dst + static_cast<size_t>(c0 + oc) * a.dst_ld + a.col0 + r0 + orr, a.R - r0 - orr, nullptr,
-               nullptr, orr, oc);
-}
-
-// ---------------------------------------------------------------------------
-// Activations transposed for the weight gradients (whose GEMMs contract over
-// rows): dst[c][r] = scale(r) * src[r][c] for the rows that hold a (token,
-// slot) pair and 0 for the others, every r < R (C a multiple of 16).  Valid
-// rows: G > 0: r - row_start[e] < counts[e] for the expert e whose segment
-// holds r (G <= 256; the tables are read into shared memory first); G = 0:
-// r < row_limit.  scale: nullptr (1) or [R], read only on valid rows.
-// ---------------------------------------------------------------------------
-struct RowTransposeArgs {
-  const __nv_bfloat16* src;
-  __nv_bfloat16* dst;
-  int R, C;
-  long long dst_ld;
-  const float* scale;
-  const int32_t* row_start;  // [G + 1]
-  const int32_t* counts;     // [G]
-  int G, row_limit;
-  int src_rows;              // rows of src that may be read (the others are not valid)
-};
-
-__global__ void __launch_bounds__(256) transpose_rows_kernel(RowTransposeArgs a) {
-  __shared__ uint16_t tile[kTrRows][kTrCols + 2];
-  __shared__ float rowf[kTrRows];  // per row: its scale
-  __shared__ int rowok[kTrRows];   // per row: holds a pair
-  __shared__ int32_t s_rs[256], s_cnt[256];
-  const int c0 = blockIdx.x * kTrCols, r0 = blockIdx.y * kTrRows;
-  const int tid = threadIdx.x;
-  for (int i = tid; i < a.G; i += 256) {
-    s_rs[i] = a.row_start[i];
-    s_cnt[i] = a.counts[i];
-  }
-  tr_load_tile(tile, reinterpret_cast<const uint16_t*>(a.src), a.C, a.C, r0, min(a.R, a.src_rows), c0);
-  __syncthreads();
-  if (tid < kTrRows) {
-    const int r = r0 + tid;
-    bool ok = r < a.R && r < a.src_rows;
-    if (ok && a.G > 0) {
-      int lo = 0, hi = a.G;  // the last expert whose segment starts at or before r
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (s_rs[mid] <= r) lo = mid;
-        else hi = mid;
-      }
-      ok = r - s_rs[lo] < s_cnt[lo];
-    } else if (ok) {
-      ok = r < a.row_limit;
-    }
-    rowok[tid] = ok ? 1 : 0;
-    rowf[tid] = ok ? (a.scale ? a.scale[r] : 1.f) : 0.f;
-  }
-  __syncthreads();
-  const int oc = tid >> 2, orr = (tid & 3) * 16;
-  if (c0 + oc >= a.C || r0 + orr >= a.R) return;
-  tr_store_row(tile, reinterpret_cast<uint16_t*>(a.dst) + static_cast<size_t>(c0 + oc) * a.dst_ld + r0 + orr,
-               a.R - r0 - orr, rowf, rowok, orr, oc);
+  tr_store_row(tile, dst + static_cast<size_t>(c0 + oc) * a.dst_ld + a.col0 + r0 + orr, a.R - r0 - orr, orr, oc);
 }
 
 // the shared experts' K ranges for the weight-gradient GEMMs: every expert j < n over rows [0, T)

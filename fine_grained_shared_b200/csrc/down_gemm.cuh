@@ -111,9 +111,10 @@ struct GemmArgs {
   int kg_bz_step;
   int kg_split;
   int kg_ld;                   // output row stride (>= n_limit, a multiple of 16)
-  // 1: both operands MN-major -- row-major [K rows][MN columns] buffers read through 2-D maps with
-  // 64 x 64 boxes, two per operand and stage; group g's A columns start at g * kg_a_row_step and its B
-  // columns at g * kg_b_col_step (with kg_bz_step set); 0: K-major operands as described above
+  // bit 0: A MN-major, bit 1: B MN-major -- a row-major [K rows][MN columns] buffer read through a
+  // 2-D map with 64 x 64 boxes, two per operand and stage; group g's A columns start at
+  // g * kg_a_row_step and its B columns at g * kg_b_col_step (with kg_bz_step set); a clear bit: that
+  // operand K-major as described above
   int kg_mn;
   int kg_b_col_step;
   float* kg_out;               // [groups][kg_split][kg_ld]
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int g = tile / kg_per_group, local = tile - g * kg_per_group;
         const int mt = local / a.n_tiles, nt = local - mt * a.n_tiles;
         const int arow = g * a.kg_a_row_step + mt * kGemmBM + static_cast<int>(rank) * kCtaRows;
-        const int brow = (a.kg_mn && a.kg_bz_step ? g * a.kg_b_col_step : 0) + nt * kGemmBN +
+        const int brow = ((a.kg_mn & 2) && a.kg_bz_step ? g * a.kg_b_col_step : 0) + nt * kGemmBN +
                          static_cast<int>(rank) * (kGemmBN / 2);
         const int bz = a.kg_bz_step ? g : 0;
         const int nkb = (s_mts[g] + kGemmBK - 1) / kGemmBK;
@@ -269,13 +270,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kStageA + kStageB));
           const int kc = s_rows[g] + kb * kGemmBK;
           const uint32_t fb = full_lead + 8u * static_cast<uint32_t>(s);
-          if (a.kg_mn) {  // MN-major: x = the MN column, y = the K row; two 64-column boxes per operand
+          // MN-major: x = the MN column, y = the K row, two 64-column boxes per operand
+          if (a.kg_mn & 1) {
             tma_load_2d_pair(sA + s * kStageA, &tmA, fb, arow, kc);
             tma_load_2d_pair(sA + s * kStageA + kStageA / 2, &tmA, fb, arow + 64, kc);
+          } else {
+            tma_load_2d_pair(sA + s * kStageA, &tmA, fb, kc, arow);
+          }
+          if (a.kg_mn & 2) {
             tma_load_2d_pair(sB + s * kStageB, &tmB, fb, brow, kc);
             tma_load_2d_pair(sB + s * kStageB + kStageB / 2, &tmB, fb, brow + 64, kc);
           } else {
-            tma_load_2d_pair(sA + s * kStageA, &tmA, fb, kc, arow);
             tma_load_3d_pair(sB + s * kStageB, &tmB, fb, kc, brow, bz);
           }
           ++issued;
@@ -329,9 +334,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------- MMA issuer (even CTA) --------------------------
-    // MN-major operands (weight-gradient mode): bits 15 and 16 of the instruction descriptor
-    const uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN) | (KG && a.kg_mn ? (1u << 15) | (1u << 16) : 0u);
-    const bool mn = KG && a.kg_mn;
+    // MN-major operands (per-group mode): bits 15 (A) and 16 (B) of the instruction descriptor
+    const bool mn_a = KG && (a.kg_mn & 1), mn_b = KG && (a.kg_mn & 2);
+    const uint32_t idesc = idesc_bf16_f32(kGemmBM, kGemmBN) | (mn_a ? 1u << 15 : 0u) | (mn_b ? 1u << 16 : 0u);
     int s = 0, acc = 0;
     uint32_t ph = 0, acc_ph = 0;
     if (a.debug_wait && blockIdx.x == 0) {
@@ -359,14 +364,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after_sync();
         // K-major: 16 K columns are 32 bytes along a row (+2 in 16-byte units); MN-major: 16 K rows of
         // 128 bytes (+128), the two 64-element MN chunks of a stage 8 KB apart
-        const uint64_t ad = mn ? sw128_mnmajor_desc(smem_u32(sA + s * kStageA), kStageA / 2)
-                               : sw128_kmajor_desc(smem_u32(sA + s * kStageA));
-        const uint64_t bd = mn ? sw128_mnmajor_desc(smem_u32(sB + s * kStageB), kStageB / 2)
-                               : sw128_kmajor_desc(smem_u32(sB + s * kStageB));
-        const uint64_t kstep = mn ? 128u : 2u;
+        const uint64_t ad = mn_a ? sw128_mnmajor_desc(smem_u32(sA + s * kStageA), kStageA / 2)
+                                 : sw128_kmajor_desc(smem_u32(sA + s * kStageA));
+        const uint64_t bd = mn_b ? sw128_mnmajor_desc(smem_u32(sB + s * kStageB), kStageB / 2)
+                                 : sw128_kmajor_desc(smem_u32(sB + s * kStageB));
+        const uint64_t astep = mn_a ? 128u : 2u, bstep = mn_b ? 128u : 2u;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16_ss_pair(d_tmem, ad + kstep * kk, bd + kstep * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+          umma_bf16_ss_pair(d_tmem, ad + astep * kk, bd + bstep * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
         umma_commit_pair_multicast(&empty[s], 0x3);
         if (++s == kGemmStages) {
           s = 0;

@@ -198,12 +198,12 @@ Layout make_layout(const moe_config& c) {
 constexpr int kDeMaxSegments = 16;
 struct BwdLayout {
   size_t wdT, wguT, swdT, swguT, dab, dabs, dg_part, dz, dxr, de_part, dgate;
-  // the router's GEMM operands: logits, dz in bf16 (and transposed), E transposed, K-range tables
-  size_t zf, dzb, dzT, ET, rt_kstart, rt_kcount;
+  // the router's GEMM operands: logits, dz in bf16, K-range tables
+  size_t zf, dzb, rt_kstart, rt_kcount;
   int64_t Npad;
   // the weight gradients' operands (row-major, read MN-major by the GEMMs): g dh and m per routed row,
-  // m per token of the shared experts; x transposed for the router's dE
-  size_t dy, mrows, msrows, xT, sh_kstart, sh_kcount, total;
+  // m per token of the shared experts
+  size_t dy, mrows, msrows, sh_kstart, sh_kcount, total;
 };
 
 BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
@@ -230,14 +230,11 @@ BwdLayout make_bwd_layout(const moe_config& c, const Layout& L) {
   B.Npad = (N + 15) / 16 * 16;
   B.zf = take(size_t(Tm) * B.Npad * 4);
   B.dzb = take(size_t(Tm) * B.Npad * 2);
-  B.dzT = take(size_t(B.Npad) * L.Tpad * 2);
-  B.ET = take(size_t(d) * B.Npad * 2);
   B.rt_kstart = take(kDeMaxSegments * 4);
   B.rt_kcount = take(kDeMaxSegments * 4);
   B.dy = take(size_t(L.P) * d * 2);
   B.mrows = take(size_t(L.P) * I * 2);
   B.msrows = take(size_t(L.Tpad) * Ks * Is * 2);
-  B.xT = take(size_t(d) * L.Tpad * 2);
   B.sh_kstart = take(64 * 4);
   B.sh_kcount = take(64 * 4);
   B.total = o;
@@ -339,9 +336,9 @@ struct moe_ctx {
   // the backward's own buffers (allocated by its first call) and their descriptors
   uint8_t* bws = nullptr;
   CUtensorMap tm_b_dhperm, tm_b_wdT, tm_b_swdT, tm_b_dab, tm_b_wguT, tm_b_dabs, tm_b_swguT;
-  CUtensorMap tm_w_dy, tm_w_m, tm_w_dab, tm_w_xperm, tm_w_ms, tm_w_dabs, tm_b_xT;  // 64 x 64 MN-major boxes
-  CUtensorMap tm_b_dzb, tm_b_ET, tm_b_dzT;
-  MapCache tm_b_dh, tm_b_E, tm_w_dh, tm_w_x;
+  CUtensorMap tm_w_dy, tm_w_m, tm_w_dab, tm_w_xperm, tm_w_ms, tm_w_dabs;  // 64 x 64 MN-major boxes
+  CUtensorMap tm_b_dzb;
+  MapCache tm_b_dh, tm_b_E, tm_w_dh, tm_w_x, tm_w_E, tm_w_dzb;
 
   template <typename T>
   T* at(size_t off) const {
@@ -1705,10 +1702,7 @@ moe_status ensure_backward_buffers(moe_ctx* h) {
   ok = ok && encode_bf16(&h->tm_w_m, h->bws + B.mrows, 1, L.P, I, 64, 2);
   ok = ok && encode_bf16(&h->tm_w_dab, h->bws + B.dab, 1, L.P, 2 * I, 64, 2);
   ok = ok && encode_bf16(&h->tm_w_xperm, h->ws + L.x_perm, 1, L.P, d, 64, 2);
-  ok = ok && encode_bf16(&h->tm_b_xT, h->bws + B.xT, 1, d, L.Tpad, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_dzb, h->bws + B.dzb, 1, c.max_tokens, B.Npad, kBoxRowsA, 2);
-  ok = ok && encode_bf16(&h->tm_b_ET, h->bws + B.ET, 1, d, B.Npad, kBoxRowsB, 3);
-  ok = ok && encode_bf16(&h->tm_b_dzT, h->bws + B.dzT, 1, B.Npad, L.Tpad, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_wdT, h->bws + B.wdT, N, I, d, kBoxRowsB, 3);
   ok = ok && encode_bf16(&h->tm_b_dab, h->bws + B.dab, 1, L.P, 2 * I, kBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_b_wguT, h->bws + B.wguT, N, d, 2 * I, kBoxRowsB, 3);
@@ -1778,7 +1772,8 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   const bool residual = !(c.flags & MOE_FLAG_NO_RESIDUAL);
   auto bw = [&](size_t off) { return h->bws + off; };
   h->last_stream = s0;
-  // a GEMM in the per-group mode of down_gemm_kernel (fp32 out, rows >= split into out2)
+  // a GEMM in the per-group mode of down_gemm_kernel (fp32 out, rows >= split into out2; mn: bit 0 A and
+  // bit 1 B MN-major, read through 64 x 64 boxes)
   auto kg_gemm = [&](const CUtensorMap& A, const CUtensorMap& Bm, int groups, const int32_t* kstart,
                      const int32_t* kcount, int M, int a_step, int bz_step, int split, int Ncols, int ld, float* out,
                      float* out2, int mn = 0, int b_col_step = 0) {
@@ -1967,10 +1962,10 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       const int32_t* kc = h->at<int32_t>(L.counts);
       // MN-major operands straight from the row-major buffers: dW_down = dy^T m, dW_gate|up = [da|db]^T x
       ke = kg_gemm(h->tm_w_dy, h->tm_w_m, (int)N, ks, kc, (int)d, 0, 0, (int)d, (int)I, (int)I, wgrad->w_down,
-                   nullptr, 1);
+                   nullptr, 3);
       if (ke == cudaSuccess)
         ke = kg_gemm(h->tm_w_dab, h->tm_w_xperm, (int)N, ks, kc, (int)(2 * I), 0, 0, (int)I, (int)d, (int)d,
-                     wgrad->w_gate, wgrad->w_up, 1);
+                     wgrad->w_gate, wgrad->w_up, 3);
     } else {
       const size_t wb = size_t(N) * I * d * 4;
       if (cudaMemsetAsync(wgrad->w_gate, 0, wb, s0) != cudaSuccess ||
@@ -1982,10 +1977,10 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
       const int32_t* ks = reinterpret_cast<const int32_t*>(bw(B.sh_kstart));
       const int32_t* kc = reinterpret_cast<const int32_t*>(bw(B.sh_kcount));
       ke = kg_gemm(h->tm_w_dh.map, h->tm_w_ms, (int)Ks, ks, kc, (int)d, 0, 1, (int)d, (int)Is, (int)Is,
-                   wgrad->ws_down, nullptr, 1, (int)Is);
+                   wgrad->ws_down, nullptr, 3, (int)Is);
       if (ke == cudaSuccess)
         ke = kg_gemm(h->tm_w_dabs, h->tm_w_x.map, (int)Ks, ks, kc, (int)(2 * Is), (int)(2 * Is), 0, (int)Is, (int)d,
-                     (int)d, wgrad->ws_gate, wgrad->ws_up, 1);
+                     (int)d, wgrad->ws_gate, wgrad->ws_up, 3);
     } else if (Ks > 0 && ke == cudaSuccess) {
       const size_t wb = size_t(Ks) * Is * d * 4;
       if (cudaMemsetAsync(wgrad->ws_gate, 0, wb, s0) != cudaSuccess ||
@@ -2024,47 +2019,25 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
     rz.dz = reinterpret_cast<float*>(bw(B.dz));
     rz.dzb = reinterpret_cast<__nv_bfloat16*>(bw(B.dzb));
     router_dz_kernel<<<ceil_div(T * 32, 256), 256, 0, s0>>>(rz);
-    // E^T [d][Npad] (zero columns past mN)
-    RowTransposeArgs rt{};
-    rt.src = static_cast<const __nv_bfloat16*>(router->weight);
-    rt.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.ET));
-    rt.R = Np;
-    rt.src_rows = (int)N;
-    rt.C = (int)d;
-    rt.dst_ld = Np;
-    rt.G = 0;
-    rt.row_limit = (int)N;
-    transpose_rows_kernel<<<dim3(ceil_div(d, kTrCols), ceil_div(Np, kTrRows)), 256, 0, s0>>>(rt);
+    // dx_router = dz E: dz K-major, E [mN][d] read MN-major in place (its rows past mN read as zeros)
+    if (!refresh(h->tm_w_E, router->weight, N, 1, N, d, 64, 2)) return MOE_ERR_CUDA;
     fill_segments_kernel<<<1, 32, 0, s0>>>(ks + 1, kc + 1, 1, (int)N, (int)N);
     dxr = reinterpret_cast<float*>(bw(B.dxr));
-    if (kg_gemm(h->tm_b_dzb, h->tm_b_ET, 1, ks + 1, kc + 1, (int)T, 0, 0, (int)T, (int)d, (int)d, dxr, nullptr) !=
-        cudaSuccess)
+    if (kg_gemm(h->tm_b_dzb, h->tm_w_E.map, 1, ks + 1, kc + 1, (int)T, 0, 0, (int)T, (int)d, (int)d, dxr, nullptr,
+                2) != cudaSuccess)
       return MOE_ERR_CUDA;
     if (d_router) {
-      // dz^T [Npad][Tpad] and (unless the shared weights' gradients made it) x^T, then dE over
-      // token segments summed in segment order
-      RowTransposeArgs t2{};
-      t2.src = rz.dzb;
-      t2.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.dzT));
-      t2.R = (int)L.Tpad;
-      t2.src_rows = (int)T;
-      t2.C = Np;
-      t2.dst_ld = L.Tpad;
-      t2.G = 0;
-      t2.row_limit = (int)T;
-      transpose_rows_kernel<<<dim3(ceil_div(Np, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t2);
-      RowTransposeArgs t3 = t2;
-      t3.src = static_cast<const __nv_bfloat16*>(x);
-      t3.dst = reinterpret_cast<__nv_bfloat16*>(bw(B.xT));
-      t3.C = (int)d;
-      transpose_rows_kernel<<<dim3(ceil_div(d, kTrCols), ceil_div(L.Tpad, kTrRows)), 256, 0, s0>>>(t3);
+      // dE = dz^T x over token segments summed in segment order, both operands MN-major in place (the
+      // maps end at T, so the rows past it read as zeros)
+      if (!refresh(h->tm_w_dzb, bw(B.dzb), T, 1, T, Np, 64, 2) || !refresh(h->tm_w_x, x, T, 1, T, d, 64, 2))
+        return MOE_ERR_CUDA;
       const int want = (int)std::max<int64_t>(1, std::min<int64_t>(kDeMaxSegments, T / 512));
       const int seg = ceil_div(ceil_div(T, want), 64) * 64;
       const int segs = ceil_div(T, seg);
       fill_segments_kernel<<<1, 32, 0, s0>>>(ks, kc, segs, seg, (int)T);
       float* part = reinterpret_cast<float*>(bw(B.de_part));
-      if (kg_gemm(h->tm_b_dzT, h->tm_b_xT, segs, ks, kc, (int)N, 0, 0, (int)N, (int)d, (int)d, part, nullptr) !=
-          cudaSuccess)
+      if (kg_gemm(h->tm_w_dzb.map, h->tm_w_x.map, segs, ks, kc, (int)N, 0, 0, (int)N, (int)d, (int)d, part,
+                  nullptr, 3) != cudaSuccess)
         return MOE_ERR_CUDA;
       router_de_reduce_kernel<<<ceil_div(N * d, 256), 256, 0, s0>>>(part, segs, size_t(N) * d, d_router);
     }
