@@ -402,7 +402,7 @@ __global__ void __launch_bounds__(kGuThreads, 1)
         const float gsc = c.shared ? 1.f : a.row_gate[row];
         const __nv_bfloat16* dmrow = c.shared ? a.sh_dm + row * a.sh_ld_dm : a.dm + row * a.ld_dm;
         // a row that holds no (token, slot) pair (expert padding, or past the tokens) stores zeros
-        // in the transposed outputs, whose sums over rows would otherwise take it in
+        // in m, da and db, since the weight gradients' sums over rows would otherwise take it in
         const bool valid = c.shared ? static_cast<int>(row) < a.sh_rows
                                     : static_cast<int>(row) - s_rows[c.g] < s_cnt[c.g];
         __nv_bfloat16* mrow = c.shared ? (a.sh_m_out ? a.sh_m_out + row * a.sh_n_limit : nullptr)

@@ -360,7 +360,7 @@ moe_status moe_quantize_fp8_blocks(const void* w, int32_t batch, int32_t rows, i
  * Asynchronous on `stream`, which must be the forward's stream or ordered after
  * it.  The first call allocates the backward's buffers
  * (a K-major copy of the expert weights, rewritten by every call, and
- * activations of the forward's row count).  Errors: the last forward was not a
+ * row-major activations of the forward's row count).  Errors: the last forward was not a
  * moe_forward with this T and K, or another argument error of moe_forward
  * -> MOE_ERR_INVALID_ARG / SHAPE / ALIGNMENT; dx overlapping x or dh ->
  * MOE_ERR_INVALID_ARG; an expert-parallel handle -> MOE_ERR_UNSUPPORTED; no
