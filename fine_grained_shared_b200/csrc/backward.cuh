@@ -95,6 +95,31 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(TransposeArgs a) {
   tr_store_row(tile, dst + static_cast<size_t>(c0 + oc) * a.dst_ld + a.col0 + r0 + orr, a.R - r0 - orr, orr, oc);
 }
 
+// ---------------------------------------------------------------------------
+// Zero, in each expert's segment, the rows past its count up to the next
+// multiple of 64 rows, in a [rows, d] and (if given) b [rows, d]: the
+// weight-gradient GEMMs sum over whole 64-row blocks of an expert's rows, and a
+// padding row may still hold an earlier call's values, which a zero operand
+// on the other side would not cancel if they are not finite.  One CTA per
+// expert; d a multiple of 8.  The rows stay inside the segment, which is
+// padded to a multiple of 256 rows.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) zero_tail_rows_kernel(const int32_t* row_start, const int32_t* counts, int d,
+                                                             __nv_bfloat16* a, __nv_bfloat16* b) {
+  const int e = blockIdx.x;
+  const int cnt = counts[e];
+  const int n = ((cnt + 63) & ~63) - cnt;  // rows to clear, 0 .. 63
+  const size_t r0 = static_cast<size_t>(row_start[e]) + static_cast<size_t>(cnt);
+  const int per_row = d >> 3;              // 16-byte units per row
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = threadIdx.x; i < n * per_row; i += blockDim.x) {
+    const int r = i / per_row, c = i - r * per_row;
+    const size_t off = (r0 + static_cast<size_t>(r)) * static_cast<size_t>(d) + static_cast<size_t>(c) * 8;
+    *reinterpret_cast<uint4*>(a + off) = z;
+    if (b) *reinterpret_cast<uint4*>(b + off) = z;
+  }
+}
+
 // the shared experts' K ranges for the weight-gradient GEMMs: every expert j < n over rows [0, T)
 __global__ void fill_dense_groups_kernel(int32_t* k_start, int32_t* k_count, int n, int T) {
   const int i = threadIdx.x;

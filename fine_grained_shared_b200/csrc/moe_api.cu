@@ -924,9 +924,6 @@ moe_status moe_create(const moe_config* cfg, int device, moe_handle* out) {
   }
   bool ok = cudaMemset(h->ws, 0, align256(4096)) == cudaSuccess;
   ok = ok && cudaMemset(h->ws + h->L.ffn_ctr, 0, ffn_counter_bytes()) == cudaSuccess;
-  // X_perm's padding rows are never written by a forward: zero them once, so that they are finite
-  // (zero, or an earlier forward's token row) when the backward's weight gradients sum over them
-  ok = ok && cudaMemset(h->ws + h->L.x_perm, 0, size_t(h->L.P) * cfg->d_model * 2) == cudaSuccess;
   const moe_config& c = *cfg;
   ok = ok && encode_bf16(&h->tm_xperm, h->ws + h->L.x_perm, 1, h->L.P, c.d_model, kGuBoxRowsA, 2);
   ok = ok && encode_bf16(&h->tm_h, h->ws + h->L.h, 1, h->L.P, c.d_ff, kBoxRowsA, 2);
@@ -1831,13 +1828,16 @@ moe_status moe_backward(moe_handle h, const void* x, int64_t T, const moe_router
   const int TK = (int)(T * K);
   // ---- dm: routed rows (dh gathered into the expert order, times W_down) and shared rows ----
   if (do_routed) {
-    // dy = g dh per routed row for the weight gradients: zero first, so that the padding rows the
-    // GEMMs' K ranges reach read as zeros
+    // dy = g dh per routed row for the weight gradients
     __nv_bfloat16* dy = wgrad ? reinterpret_cast<__nv_bfloat16*>(bw(B.dy)) : nullptr;
-    if (dy && cudaMemsetAsync(dy, 0, size_t(L.P) * d * 2, s0) != cudaSuccess) return MOE_ERR_CUDA;
     bwd_gather_kernel<<<ceil_div(int64_t(TK) * 32, 256), 256, 0, s0>>>(static_cast<const __nv_bfloat16*>(dh), slot_of,
                                                                        TK, K, (int)d, h->at<__nv_bfloat16>(L.y),
                                                                        h->at<float>(L.gate), dy);
+    // the padding rows the weight-gradient GEMMs' K blocks reach, in X_perm and dy, as zeros (they may
+    // hold an earlier call's rows)
+    if (dy)
+      zero_tail_rows_kernel<<<(int)N, 256, 0, s0>>>(h->at<int32_t>(L.row_start), h->at<int32_t>(L.counts), (int)d,
+                                                     h->at<__nv_bfloat16>(L.x_perm), dy);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     GemmArgs g{};
     g.num_groups = (int)N;

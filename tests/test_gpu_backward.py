@@ -144,6 +144,35 @@ def test_backward_matches_the_oracle(name):
         _compare(_rows(dx_r), du_nr - shared_du, f"{name} routed and router terms of dx", 5e-2)
 
 
+def test_weight_gradients_ignore_an_earlier_forwards_rows():
+    """A forward of all-NaN tokens (every key ranks last, so every token takes experts 0..K-1) and its
+    backward leave NaN in X_perm's and g dh's rows of those experts' segments.  A later clean forward
+    routes about T*K/mN rows to each expert, so those rows are now the padding past each expert's count
+    inside the weight-gradient GEMMs' last 64-row K block; the clean backward's weight gradients must
+    still be finite and match the oracle."""
+    shape = SHAPES["softmax_logit_bias"]
+    host, dev = H.device_inputs(shape)
+    dh_host = W.output_gradient(shape)
+    dh = dh_host.to("cuda")
+    layer = H.make_layer(shape, dev)
+    bad = torch.full_like(dev["x"], float("nan"))
+    layer.forward(bad, shape.K)
+    layer.backward(bad, shape.K, dh, weight_grads=True)
+    assert layer.status() == B.MOE_OK
+    H.run(layer, dev["x"], shape.K)
+    wg = layer.backward(dev["x"], shape.K, dh, weight_grads=True)[4]
+    assert layer.status() == B.MOE_OK
+    counts = np.bincount(layer.routing(shape.T, shape.K)[0].cpu().numpy().ravel(), minlength=shape.N)
+    assert (counts[:shape.K] % 64 != 0).all()        # each stale segment has padding rows in a K block
+    layer.close()
+    grads = OB.moe_backward(host["x"], host["router"], shape.K, (host["w_gate"], host["w_up"], host["w_down"]),
+                            H.oracle_shared(shape, host), dh=dh_host, gate_kind=shape.gate,
+                            logit_bias=host["logit_bias"], select_bias=host["select_bias"])
+    for key, want in (("w_gate", grads.d_w_gate), ("w_up", grads.d_w_up), ("w_down", grads.d_w_down),
+                      ("ws_gate", grads.d_ws_gate), ("ws_up", grads.d_ws_up), ("ws_down", grads.d_ws_down)):
+        _compare_wgrad(wg[key].cpu().numpy().astype(np.float64), want, f"after a NaN forward: d{key}")
+
+
 def test_backward_is_deterministic():
     shape = SHAPES["sigmoid"]
     host, dev = H.device_inputs(shape)
