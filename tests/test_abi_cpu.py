@@ -106,6 +106,19 @@ def test_null_handles():
     assert lib.moe_forward_host(None, None, 1, ctypes.byref(r), ctypes.byref(e), None, 1, None, None) == \
         B.MOE_ERR_INVALID_ARG
     assert lib.moe_kernel_times(None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_fp8(None, None, 1, ctypes.byref(r), None, None, 1, None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_backward(None, None, 1, ctypes.byref(r), ctypes.byref(e), None, 1, None, None, None, None, None,
+                            None, None) == B.MOE_ERR_INVALID_ARG
+    # the expert-parallel calls
+    assert lib.moe_ep_workspace(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_set_peers(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_ipc_handle(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_open_peers(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_route(None, None, 1, ctypes.byref(r), 1, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_dispatch(None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_experts(None, ctypes.byref(e), None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_experts_fp8(None, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_combine(None, None, None) == B.MOE_ERR_INVALID_ARG
 
 
 def test_fp8_quantize_arguments_are_checked_before_any_cuda_call():
