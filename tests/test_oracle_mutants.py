@@ -304,6 +304,29 @@ def _logit_backward_wrong_sign(s, idx, gate, dg, gate_kind):
     return -_origb["gate_logit_backward"](s, idx, gate, dg, gate_kind)
 
 
+def _ffn_backward_down_grad_without_silu(u, w_gate, w_up, w_down, dy):
+    du, dwg, dwu, _ = _origb["swiglu_ffn_backward"](u, w_gate, w_up, w_down, dy)
+    a, b = u @ M.f64(w_gate).T, u @ M.f64(w_up).T
+    return du, dwg, dwu, dy.T @ (a * b)
+
+
+def _ffn_backward_drops_gate_path(u, w_gate, w_up, w_down, dy):
+    du, dwg, dwu, dwd = _origb["swiglu_ffn_backward"](u, w_gate, w_up, w_down, dy)
+    wg, wu, wd = M.f64(w_gate), M.f64(w_up), M.f64(w_down)
+    a, b = u @ wg.T, u @ wu.T
+    da = (dy @ wd) * b * _origb["silu_grad"](a)
+    return du - da @ wg, dwg, dwu, dwd
+
+
+def _ffn_backward_weight_grads_transposed_inputs(u, w_gate, w_up, w_down, dy):
+    """dW_gate from the rows of dy instead of u (the two operands of the outer product mixed up)."""
+    du, dwg, dwu, dwd = _origb["swiglu_ffn_backward"](u, w_gate, w_up, w_down, dy)
+    wg, wu, wd = M.f64(w_gate), M.f64(w_up), M.f64(w_down)
+    a, b = u @ wg.T, u @ wu.T
+    da = (dy @ wd) * b * _origb["silu_grad"](a)
+    return du, da.T @ dy, dwu, dwd
+
+
 MUTANTS_BWD = {
     "silu_grad_sigma_only": ("silu_grad", _silu_grad_sigma_only),
     "ffn_backward_drops_up_path": ("swiglu_ffn_backward", _ffn_backward_drops_up_path),
@@ -311,6 +334,9 @@ MUTANTS_BWD = {
     "softmax_backward_not_centred": ("gate_logit_backward", _softmax_backward_not_centred),
     "sigmoid_backward_not_normalised": ("gate_logit_backward", _sigmoid_backward_not_normalised),
     "logit_backward_wrong_sign": ("gate_logit_backward", _logit_backward_wrong_sign),
+    "down_grad_without_silu": ("swiglu_ffn_backward", _ffn_backward_down_grad_without_silu),
+    "ffn_backward_drops_gate_path": ("swiglu_ffn_backward", _ffn_backward_drops_gate_path),
+    "gate_weight_grad_from_dy": ("swiglu_ffn_backward", _ffn_backward_weight_grads_transposed_inputs),
 }
 
 PINS_BWD = [
